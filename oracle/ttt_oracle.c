@@ -1,0 +1,318 @@
+/*
+ * Float64 CPU oracle for the TTT layer inner-loop forward.
+ *
+ * TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.  Only the test suite, the
+ * smoke check and the benchmark's CPU-baseline leg may load this library.  It
+ * shares no code, header or constant with the CUDA path.
+ *
+ * What it computes (paper: "Learning to (Learn at Test Time): RNNs with
+ * Expressive Hidden States"; the passages are those of the paper digest on
+ * equinox-blog, "论文速览 | TTT"):
+ *
+ *   - Naive TTT, update then output (section 3.1):
+ *         W_t = W_{t-1} - eta * grad l(W_{t-1}; x_t),   z_t = f(x_t; W_t)
+ *   - Multi-view reconstruction loss and output rule (section 3.3):
+ *         l(W; x_t) = || f(theta_K x_t; W) - theta_V x_t ||^2,
+ *         z_t = f(theta_Q x_t; W_t)
+ *     The projections are outside this path: the oracle receives k_t, v_t,
+ *     q_t directly.
+ *   - Mini-batch gradient descent (section 3.5): inside a mini-batch of b
+ *     tokens every gradient is taken at the state W_{t'} of the batch start,
+ *     and the updates are applied cumulatively token by token:
+ *         G_t = grad l(W_{t'}; x_t),   W_t = W_{t-1} - eta_t G_t.
+ *     This is written out literally (the "primal" form); the dual form of
+ *     sections 3.6-3.7 is an algebraic rewrite of the same result and is the
+ *     GPU's route, not the oracle's.
+ *   - Inner models (section 4.4): linear f(x) = x W; LN+residual
+ *     f(x) = x + LN(x W + c); two-layer MLP f(x) = GELU(x W1 + c1) W2 + c2
+ *     with hidden size 4d.
+ *   - Learnable per-token learning rate (section 4.6): eta_t is an input, one
+ *     value per token, scaling that token's own gradient.
+ *   - Decode / generate uses the primal form one token at a time (section
+ *     6.11): the b = 1 update followed by the output.
+ *
+ * Readings of points the pages leave open (each one is listed in the design
+ * notes of the repository):
+ *   - Row-vector convention f(x) = x W (W is d_in x d_out).
+ *   - Half-loss gradient: grad of 1/2 ||f - v||^2.  The pages' dual form
+ *     carries a factor 2 that is folded into eta.
+ *   - Biases c, c1, c2 are parameters of f and are part of the state:
+ *     updated by the same gradient step and returned.
+ *   - LN uses the biased variance over the d features and eps = ln_eps;
+ *     gamma and beta are fixed during the inner loop.
+ *   - GELU is the exact erf form x * Phi(x).
+ *   - A short last mini-batch (T not a multiple of b) follows the same rules.
+ *
+ * Layouts (all row-major, float64):
+ *   Q, K, V, Z : [B, H, T, d]          eta : [B, H, T]
+ *   W0         : unit (n, h) reads W0 + n * W0_bstride + h * d * d   (d x d)
+ *   c0, gamma, beta : [H, d] (c0 with the same batch-stride rule, may be NULL)
+ *   W_out      : [B, H, d, d]          c_out : [B, H, d] (may be NULL)
+ *   MLP: W1 [.., d, 4d], c1 [.., 4d], W2 [.., 4d, d], c2 [.., d]
+ *
+ * Parallel over (sequence, head) units with OpenMP; each unit is computed
+ * serially in the order written above.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double gelu(double x) { return 0.5 * x * (1.0 + erf(x / sqrt(2.0))); }
+
+/* d/dx [x Phi(x)] = Phi(x) + x phi(x) */
+static double gelu_grad(double x) {
+    const double Phi = 0.5 * (1.0 + erf(x / sqrt(2.0)));
+    const double phi = exp(-0.5 * x * x) / sqrt(2.0 * M_PI);
+    return Phi + x * phi;
+}
+
+/* y[j] = sum_i x[i] W[i][j]  (x: n_in, W: n_in x n_out) */
+static void vec_mat(int n_in, int n_out, const double *x, const double *W, double *y) {
+    for (int j = 0; j < n_out; ++j) y[j] = 0.0;
+    for (int i = 0; i < n_in; ++i) {
+        const double xi = x[i];
+        const double *Wi = W + (size_t)i * n_out;
+        for (int j = 0; j < n_out; ++j) y[j] += xi * Wi[j];
+    }
+}
+
+/* LayerNorm over n features, biased variance.  Writes xhat and returns r = 1/sqrt(var+eps). */
+static double layer_norm(int n, const double *y, double eps, double *xhat) {
+    double mu = 0.0;
+    for (int j = 0; j < n; ++j) mu += y[j];
+    mu /= n;
+    double var = 0.0;
+    for (int j = 0; j < n; ++j) var += (y[j] - mu) * (y[j] - mu);
+    var /= n;
+    const double r = 1.0 / sqrt(var + eps);
+    for (int j = 0; j < n; ++j) xhat[j] = (y[j] - mu) * r;
+    return r;
+}
+
+/* f(x; W, c) for the linear / LN+residual inner model. */
+static void linear_model_forward(int d, const double *x, const double *W, const double *c, int use_ln,
+                                 const double *gamma, const double *beta, double eps, double *out,
+                                 double *tmp_y, double *tmp_xh) {
+    vec_mat(d, d, x, W, tmp_y);
+    if (!use_ln) {
+        for (int j = 0; j < d; ++j) out[j] = tmp_y[j];
+        return;
+    }
+    for (int j = 0; j < d; ++j) tmp_y[j] += c[j];
+    layer_norm(d, tmp_y, eps, tmp_xh);
+    for (int j = 0; j < d; ++j) out[j] = x[j] + gamma[j] * tmp_xh[j] + beta[j];
+}
+
+/*
+ * Gradient of 1/2 || f(k; W, c) - v ||^2 with respect to the pre-activation
+ * y = k W (+ c).  grad_W = k^T delta, grad_c = delta.
+ */
+static void linear_model_delta(int d, const double *k, const double *v, const double *W, const double *c,
+                               int use_ln, const double *gamma, const double *beta, double eps,
+                               double *delta, double *y, double *xh) {
+    vec_mat(d, d, k, W, y);
+    if (!use_ln) {
+        for (int j = 0; j < d; ++j) delta[j] = y[j] - v[j];
+        return;
+    }
+    for (int j = 0; j < d; ++j) y[j] += c[j];
+    const double r = layer_norm(d, y, eps, xh);
+    /* e = f(k) - v ; g = dL/dxhat = gamma * e */
+    double mean_g = 0.0, mean_gx = 0.0;
+    for (int j = 0; j < d; ++j) {
+        const double e = k[j] + gamma[j] * xh[j] + beta[j] - v[j];
+        const double g = gamma[j] * e;
+        delta[j] = g; /* keep g for now */
+        mean_g += g;
+        mean_gx += g * xh[j];
+    }
+    mean_g /= d;
+    mean_gx /= d;
+    /* backward through xhat = (y - mu) r */
+    for (int j = 0; j < d; ++j) delta[j] = r * (delta[j] - mean_g - xh[j] * mean_gx);
+}
+
+static void linear_unit(int T, int d, int b, const double *Q, const double *K, const double *V,
+                        const double *eta, const double *W0, const double *c0, int use_ln, const double *gamma,
+                        const double *beta, double eps, double *Z, double *W_out, double *c_out) {
+    const size_t dd = (size_t)d * d;
+    double *Ws = malloc(dd * sizeof(double));   /* state at the mini-batch start */
+    double *Wc = malloc(dd * sizeof(double));   /* running state W_t */
+    double *cs = calloc(d, sizeof(double));
+    double *cc = calloc(d, sizeof(double));
+    double *delta = malloc(d * sizeof(double));
+    double *y = malloc(d * sizeof(double));
+    double *xh = malloc(d * sizeof(double));
+    memcpy(Wc, W0, dd * sizeof(double));
+    if (c0) memcpy(cc, c0, d * sizeof(double));
+
+    for (int t0 = 0; t0 < T; t0 += b) {
+        const int t1 = (t0 + b < T) ? t0 + b : T;
+        memcpy(Ws, Wc, dd * sizeof(double));
+        memcpy(cs, cc, d * sizeof(double));
+        for (int t = t0; t < t1; ++t) {
+            const double *k = K + (size_t)t * d, *v = V + (size_t)t * d, *q = Q + (size_t)t * d;
+            /* gradient at the batch-start state */
+            linear_model_delta(d, k, v, Ws, cs, use_ln, gamma, beta, eps, delta, y, xh);
+            /* cumulative update W_t = W_{t-1} - eta_t G_t */
+            const double et = eta[t];
+            for (int i = 0; i < d; ++i) {
+                const double a = et * k[i];
+                double *Wi = Wc + (size_t)i * d;
+                for (int j = 0; j < d; ++j) Wi[j] -= a * delta[j];
+            }
+            if (use_ln)
+                for (int j = 0; j < d; ++j) cc[j] -= et * delta[j];
+            /* output with the updated state */
+            linear_model_forward(d, q, Wc, cc, use_ln, gamma, beta, eps, Z + (size_t)t * d, y, xh);
+        }
+    }
+    memcpy(W_out, Wc, dd * sizeof(double));
+    if (c_out) memcpy(c_out, cc, d * sizeof(double));
+    free(Ws); free(Wc); free(cs); free(cc); free(delta); free(y); free(xh);
+}
+
+int ttt_oracle_linear_forward(int B, int H, int T, int d, int b, const double *Q, const double *K,
+                              const double *V, const double *eta, const double *W0, long long W0_bstride,
+                              const double *c0, long long c0_bstride, int use_ln, const double *gamma,
+                              const double *beta, double eps, double *Z, double *W_out, double *c_out,
+                              int nthreads) {
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0) return 1;
+    if (!W0 || !W_out || (T > 0 && (!Q || !K || !V || !eta || !Z))) return 1;
+    if (use_ln && (!gamma || !beta)) return 1;
+    const long long units = (long long)B * H;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long long u = 0; u < units; ++u) {
+        const int n = (int)(u / H), h = (int)(u % H);
+        const size_t tok = (size_t)u * T * d;
+        linear_unit(T, d, b, Q + tok, K + tok, V + tok, eta + (size_t)u * T,
+                    W0 + (size_t)n * W0_bstride + (size_t)h * d * d,
+                    c0 ? c0 + (size_t)n * c0_bstride + (size_t)h * d : NULL, use_ln,
+                    use_ln ? gamma + (size_t)h * d : NULL, use_ln ? beta + (size_t)h * d : NULL, eps,
+                    Z + tok, W_out + (size_t)u * d * d, c_out ? c_out + (size_t)u * d : NULL);
+    }
+    (void)nthreads;
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Two-layer MLP inner model f(x) = GELU(x W1 + c1) W2 + c2, hidden size m.
+ * ------------------------------------------------------------------------- */
+static void mlp_unit(int T, int d, int m, int b, const double *Q, const double *K, const double *V,
+                     const double *eta, const double *W1_0, const double *c1_0, const double *W2_0,
+                     const double *c2_0, double *Z, double *W1_out, double *c1_out, double *W2_out,
+                     double *c2_out) {
+    const size_t n1 = (size_t)d * m, n2 = (size_t)m * d;
+    double *W1s = malloc(n1 * sizeof(double)), *W1c = malloc(n1 * sizeof(double));
+    double *W2s = malloc(n2 * sizeof(double)), *W2c = malloc(n2 * sizeof(double));
+    double *c1s = malloc(m * sizeof(double)), *c1c = malloc(m * sizeof(double));
+    double *c2s = malloc(d * sizeof(double)), *c2c = malloc(d * sizeof(double));
+    double *a = malloc(m * sizeof(double)), *hh = malloc(m * sizeof(double));
+    double *d1 = malloc(m * sizeof(double)), *e = malloc(d * sizeof(double));
+    memcpy(W1c, W1_0, n1 * sizeof(double));
+    memcpy(W2c, W2_0, n2 * sizeof(double));
+    if (c1_0) memcpy(c1c, c1_0, m * sizeof(double)); else memset(c1c, 0, m * sizeof(double));
+    if (c2_0) memcpy(c2c, c2_0, d * sizeof(double)); else memset(c2c, 0, d * sizeof(double));
+
+    for (int t0 = 0; t0 < T; t0 += b) {
+        const int t1 = (t0 + b < T) ? t0 + b : T;
+        memcpy(W1s, W1c, n1 * sizeof(double));
+        memcpy(W2s, W2c, n2 * sizeof(double));
+        memcpy(c1s, c1c, m * sizeof(double));
+        memcpy(c2s, c2c, d * sizeof(double));
+        for (int t = t0; t < t1; ++t) {
+            const double *k = K + (size_t)t * d, *v = V + (size_t)t * d, *q = Q + (size_t)t * d;
+            /* forward at the batch-start parameters */
+            vec_mat(d, m, k, W1s, a);
+            for (int p = 0; p < m; ++p) { a[p] += c1s[p]; hh[p] = gelu(a[p]); }
+            vec_mat(m, d, hh, W2s, e);
+            for (int j = 0; j < d; ++j) e[j] += c2s[j] - v[j];
+            /* backward: d1 = (e W2^T) * GELU'(a) */
+            for (int p = 0; p < m; ++p) {
+                double s = 0.0;
+                const double *W2p = W2s + (size_t)p * d;
+                for (int j = 0; j < d; ++j) s += W2p[j] * e[j];
+                d1[p] = s * gelu_grad(a[p]);
+            }
+            /* cumulative update with this token's gradient */
+            const double et = eta[t];
+            for (int i = 0; i < d; ++i) {
+                const double ak = et * k[i];
+                double *row = W1c + (size_t)i * m;
+                for (int p = 0; p < m; ++p) row[p] -= ak * d1[p];
+            }
+            for (int p = 0; p < m; ++p) c1c[p] -= et * d1[p];
+            for (int p = 0; p < m; ++p) {
+                const double ah = et * hh[p];
+                double *row = W2c + (size_t)p * d;
+                for (int j = 0; j < d; ++j) row[j] -= ah * e[j];
+            }
+            for (int j = 0; j < d; ++j) c2c[j] -= et * e[j];
+            /* output with the updated parameters */
+            vec_mat(d, m, q, W1c, a);
+            for (int p = 0; p < m; ++p) hh[p] = gelu(a[p] + c1c[p]);
+            double *z = Z + (size_t)t * d;
+            vec_mat(m, d, hh, W2c, z);
+            for (int j = 0; j < d; ++j) z[j] += c2c[j];
+        }
+    }
+    memcpy(W1_out, W1c, n1 * sizeof(double));
+    memcpy(W2_out, W2c, n2 * sizeof(double));
+    if (c1_out) memcpy(c1_out, c1c, m * sizeof(double));
+    if (c2_out) memcpy(c2_out, c2c, d * sizeof(double));
+    free(W1s); free(W1c); free(W2s); free(W2c); free(c1s); free(c1c); free(c2s); free(c2c);
+    free(a); free(hh); free(d1); free(e);
+}
+
+int ttt_oracle_mlp_forward(int B, int H, int T, int d, int m, int b, const double *Q, const double *K,
+                           const double *V, const double *eta, const double *W1, const double *c1,
+                           const double *W2, const double *c2, long long p_bstride_scale, double *Z,
+                           double *W1_out, double *c1_out, double *W2_out, double *c2_out, int nthreads) {
+    /* p_bstride_scale = 0: parameters are [H, ...] shared over the batch;
+       1: parameters are [B, H, ...] (one set per sequence). */
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || m <= 0 || b <= 0) return 1;
+    if (!W1 || !W2 || !W1_out || !W2_out || (T > 0 && (!Q || !K || !V || !eta || !Z))) return 1;
+    const long long units = (long long)B * H;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long long u = 0; u < units; ++u) {
+        const long long pu = p_bstride_scale ? u : (u % H);
+        const size_t tok = (size_t)u * T * d;
+        mlp_unit(T, d, m, b, Q + tok, K + tok, V + tok, eta + (size_t)u * T, W1 + (size_t)pu * d * m,
+                 c1 ? c1 + (size_t)pu * m : NULL, W2 + (size_t)pu * m * d, c2 ? c2 + (size_t)pu * d : NULL,
+                 Z + tok, W1_out + (size_t)u * d * m, c1_out ? c1_out + (size_t)u * m : NULL,
+                 W2_out + (size_t)u * m * d, c2_out ? c2_out + (size_t)u * d : NULL);
+    }
+    (void)nthreads;
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Decode: one token per unit, b = 1 primal step, in place on W [B,H,d,d].
+ *   W <- W - eta k^T (k W - v),   z = q W  (after the update)
+ * ------------------------------------------------------------------------- */
+int ttt_oracle_linear_decode_step(int B, int H, int d, double *W, const double *q, const double *k,
+                                  const double *v, const double *eta, double *z) {
+    if (B < 0 || H < 0 || d <= 0 || !W || !q || !k || !v || !eta || !z) return 1;
+    const long long units = (long long)B * H;
+    for (long long u = 0; u < units; ++u) {
+        double *Wu = W + (size_t)u * d * d;
+        const double *qu = q + (size_t)u * d, *ku = k + (size_t)u * d, *vu = v + (size_t)u * d;
+        double *e = malloc(d * sizeof(double));
+        vec_mat(d, d, ku, Wu, e);
+        for (int j = 0; j < d; ++j) e[j] -= vu[j];
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) Wu[(size_t)i * d + j] -= eta[u] * ku[i] * e[j];
+        vec_mat(d, d, qu, Wu, z + (size_t)u * d);
+        free(e);
+    }
+    return 0;
+}

@@ -1,0 +1,60 @@
+"""Plant mistakes in a copy of the oracle (on the CPU) and check that the pins
+catch every one of them.
+
+Each mutation is a one-line change of ``oracle/ttt_oracle.c`` compiled into a
+temporary library; the pin suite (``test_oracle_pins.py``) is then run against
+it in a subprocess and must fail.  This is evidence that the pins are strong
+enough to detect the plausible mistakes a primal TTT implementation can make.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "ttt_oracle.c")
+
+MUTATIONS = {
+    "update_sign": ("Wi[j] -= a * delta[j];", "Wi[j] += a * delta[j];"),
+    "output_from_batch_start": ("linear_model_forward(d, q, Wc, cc,", "linear_model_forward(d, q, Ws, cs,"),
+    "gradient_at_running_state": ("linear_model_delta(d, k, v, Ws, cs,", "linear_model_delta(d, k, v, Wc, cc,"),
+    "ln_unbiased_variance": ("    var /= n;\n", "    var /= (n - 1);\n"),
+    "ln_dropped_backward_term": ("r * (delta[j] - mean_g - xh[j] * mean_gx)", "r * (delta[j] - mean_g)"),
+    "gelu_grad_missing_term": ("return Phi + x * phi;", "return Phi;"),
+    "eta_ignored": ("const double et = eta[t];", "const double et = 0.1;"),
+    "transposed_state": ("y[j] += xi * Wi[j];", "y[j] += xi * W[(size_t)j * n_out + i];"),
+    "mlp_bias2_not_updated": ("c2c[j] -= et * e[j];", "(void)0;"),
+    "mlp_w2_update_uses_prev_h": ("const double ah = et * hh[p];", "const double ah = et * a[p];"),
+    "decode_output_before_update": (
+        "        vec_mat(d, d, qu, Wu, z + (size_t)u * d);\n        free(e);",
+        "        free(e);"),
+}
+
+
+def _build_mutant(name, old, new, tmp):
+    src = open(SRC).read()
+    assert src.count(old) >= 1, name
+    mut = src.replace(old, new, 1)
+    if name == "decode_output_before_update":
+        mut = mut.replace("        vec_mat(d, d, ku, Wu, e);\n",
+                          "        vec_mat(d, d, qu, Wu, z + (size_t)u * d);\n        vec_mat(d, d, ku, Wu, e);\n", 1)
+    c = os.path.join(tmp, f"{name}.c")
+    so = os.path.join(tmp, f"{name}.so")
+    open(c, "w").write(mut)
+    subprocess.run(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-D_GNU_SOURCE", "-o", so, c,
+                    "-lm"], check=True)
+    return so
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name):
+    old, new = MUTATIONS[name]
+    with tempfile.TemporaryDirectory() as tmp:
+        so = _build_mutant(name, old, new, tmp)
+        env = dict(os.environ, TTT_ORACLE_LIB_OVERRIDE=so)
+        r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                           env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+        assert r.returncode != 0, f"mutation {name} survived the pins:\n{r.stdout[-2000:]}"
