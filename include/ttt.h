@@ -1,0 +1,202 @@
+/*
+ * ttt.h -- C ABI of the TTT layer inner-loop forward on NVIDIA B200 (sm_100a).
+ *
+ * Paper: "Learning to (Learn at Test Time): RNNs with Expressive Hidden
+ * States".  Passages are cited by section of the paper digest "论文速览 | TTT"
+ * (equinox-blog).
+ *
+ * In a TTT layer each (sequence, head) unit carries a hidden state that is
+ * the weight set W of a small model f.  Tokens are processed in mini-batches
+ * of b tokens; within a mini-batch every token's gradient of the
+ * reconstruction loss 1/2 ||f(k_t; W) - v_t||^2 is taken at the mini-batch's
+ * starting state W0, the updates W_t = W_{t-1} - eta_t * grad_t accumulate
+ * token by token, and the output is z_t = f(q_t; W_t) (section 3.1: update,
+ * then output; section 3.3: multi-view loss and output; section 3.5:
+ * mini-batch gradient descent).  The GPU computes this in the dual form
+ * (sections 3.6-3.7): per mini-batch,
+ *     E = K W0 - V,   Z = Q W0 - (tril(Q K^T) * eta_s) E,   W_b = W0 - K^T diag(eta) E
+ * for the linear model, with the analogous two-pass form for LN+residual and
+ * for the MLP.
+ *
+ * Conventions shared by every entry point
+ *   - Row vectors: f(x) = x W with W stored d_in x d_out, row-major.
+ *   - Half-loss gradient: eta multiplies grad of 1/2 ||f - v||^2.  (The
+ *     pages' dual form W_b = W0 - 2 eta (W0 X - X) X^T carries the 2 in eta.)
+ *   - eta: per-token learning rate (section 4.6), one fp32 value per token,
+ *     or a constant when the pointer is NULL.
+ *   - All pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates nothing per call and keeps no state between calls beyond a
+ *     device-side status word per device.
+ *   - Calls are asynchronous on `stream`; results are valid after the stream
+ *     is synchronised.  Inputs are never modified, except W in decode.
+ *   - Errors: invalid arguments are rejected synchronously, before any launch
+ *     (TTT_ERR_INVALID_ARG / TTT_ERR_UNSUPPORTED).  A failed launch returns
+ *     TTT_ERR_CUDA.  Device-side waits are bounded; an expired wait ends the
+ *     kernel early and is reported by ttt_last_device_status().
+ *   - Alignment: every pointer must be 16-byte aligned.
+ */
+#ifndef TTT_H_
+#define TTT_H_
+
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TTT_OK = 0,
+    TTT_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, T % b != 0 */
+    TTT_ERR_UNSUPPORTED = 2,  /* valid request with no kernel for it (e.g. d not in {16,32,64}) */
+    TTT_ERR_CUDA = 3,         /* launch or runtime error reported by CUDA */
+    TTT_ERR_TIMEOUT = 4       /* a bounded device-side wait expired */
+} ttt_status;
+
+typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
+
+/* flags (bit set) */
+#define TTT_FLAG_FORCE_SIMT 0x1u   /* use the fp32 CUDA-core kernel even where the tensor-core one applies */
+#define TTT_FLAG_TEST_STALL 0x100u /* test hook: one device wait is made to expire (see ttt_last_device_status) */
+
+/*
+ * ttt_linear_forward -- prefill of TTT-Linear or TTT-Linear with LN+residual.
+ *
+ * Inner model (section 4.4):
+ *   use_ln == 0:  f(x) = x W
+ *   use_ln == 1:  f(x) = x + LN(x W + c), LN over the d features with biased
+ *                 variance, eps = ln_eps, per-head gamma/beta fixed during the
+ *                 inner loop; the gradient flows through LN into W and c.
+ *
+ * Arguments
+ *   B, H, T, d, b  sequences, heads, tokens, head dim, mini-batch size.
+ *                  T % b == 0 is required.  Supported: d in {16, 32, 64},
+ *                  1 <= b <= 64.  The tensor-core kernel serves io_dtype BF16,
+ *                  d = 64, b = 16; every other valid case runs on the fp32
+ *                  CUDA-core kernel.
+ *   io_dtype       dtype of Q, K, V and Z (TTT_F32 or TTT_BF16).
+ *   Q, K, V        [B, H, T, d] contiguous (views theta_Q x, theta_K x,
+ *                  theta_V x of section 3.3; the projections are the caller's).
+ *   eta            [B, H, T] fp32, or NULL: every token uses eta_const.
+ *   W0             initial state (learnable theta_init, section 4.5), fp32,
+ *                  unit (n, h) reads W0 + n * W0_bstride + h * d * d.
+ *                  W0_bstride = 0: one [H, d, d] shared by all sequences;
+ *                  W0_bstride = H*d*d: [B, H, d, d] (e.g. a resumed state).
+ *   c0             LN only: initial bias [H, d] with the same batch-stride
+ *                  rule (c0_bstride), or NULL for zeros.
+ *   ln_gamma, ln_beta  LN only: [H, d] fp32.
+ *   Z              output [B, H, T, d] in io_dtype.
+ *   W_out          output final state [B, H, d, d] fp32.
+ *   c_out          LN only: final bias [B, H, d] fp32, or NULL.
+ *   flags          TTT_FLAG_* bits; 0 for normal use.
+ *   wait_timeout_ms  limit of every device-side wait (0: 2000 ms).
+ */
+typedef struct {
+    int B, H, T, d, b;
+    ttt_dtype io_dtype;
+    const void* Q;
+    const void* K;
+    const void* V;
+    const float* eta;
+    float eta_const;
+    const float* W0;
+    long long W0_bstride;
+    const float* c0;
+    long long c0_bstride;
+    int use_ln;
+    const float* ln_gamma;
+    const float* ln_beta;
+    float ln_eps;
+    void* Z;
+    float* W_out;
+    float* c_out;
+    unsigned flags;
+    unsigned wait_timeout_ms;
+} ttt_linear_args;
+
+ttt_status ttt_linear_forward(const ttt_linear_args* args, cudaStream_t stream);
+
+/*
+ * ttt_mlp_forward -- prefill of TTT-MLP, f(x) = GELU(x W1 + c1) W2 + c2 with
+ * hidden size m = 4d (section 4.4), exact-erf GELU, dual form of section 3.7.
+ *
+ *   B, H, T, d, b  as above; supported: io_dtype BF16, d = 64, b = 16
+ *                  (tensor-core kernel) or any io_dtype with d in {16, 32}
+ *                  and b <= 64 (CUDA-core kernel).  T % b == 0.
+ *   Q, K, V, eta, eta_const, Z   as for ttt_linear_forward.
+ *   W1 [.., d, m], c1 [.., m], W2 [.., m, d], c2 [.., d]  fp32 initial
+ *                  parameters: [H, ...] shared over sequences when
+ *                  params_per_sequence == 0, [B, H, ...] when 1.  c1 / c2 may
+ *                  be NULL (zeros).
+ *   W1_out [B,H,d,m], c1_out [B,H,m], W2_out [B,H,m,d], c2_out [B,H,d]
+ *                  final parameters (fp32); c1_out / c2_out may be NULL.
+ */
+typedef struct {
+    int B, H, T, d, b;
+    ttt_dtype io_dtype;
+    const void* Q;
+    const void* K;
+    const void* V;
+    const float* eta;
+    float eta_const;
+    const float* W1;
+    const float* c1;
+    const float* W2;
+    const float* c2;
+    int params_per_sequence;
+    void* Z;
+    float* W1_out;
+    float* c1_out;
+    float* W2_out;
+    float* c2_out;
+    unsigned flags;
+    unsigned wait_timeout_ms;
+} ttt_mlp_args;
+
+ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
+
+/*
+ * ttt_linear_decode_step -- one generated token per unit, TTT-Linear without
+ * LN, primal form with b = 1 (section 6.11: decode is token by token and uses
+ * the primal form; section 3.1: update, then output):
+ *     e = k W - v,   W <- W - eta k^T e,   z = q W   (W after the update)
+ * computed as z = q W_old - eta (q . k) e so W is read and written once.
+ *
+ *   B, H, d        d in {16, 32, 64}.
+ *   io_dtype       dtype of q, k, v and z.
+ *   W              [B, H, d, d] fp32, updated in place.
+ *   q, k, v        [B, H, d].
+ *   eta            [B, H] fp32, or NULL for eta_const.
+ *   z              output [B, H, d] in io_dtype.
+ */
+typedef struct {
+    int B, H, d;
+    ttt_dtype io_dtype;
+    float* W;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* eta;
+    float eta_const;
+    void* z;
+} ttt_decode_args;
+
+ttt_status ttt_linear_decode_step(const ttt_decode_args* args, cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* ttt_status_string(ttt_status s);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device.  Returns TTT_ERR_TIMEOUT if any kernel launched since the
+ * last call gave up a bounded wait, TTT_ERR_CUDA on a CUDA error, else TTT_OK.
+ */
+ttt_status ttt_last_device_status(cudaStream_t stream);
+
+/* Library version string. */
+const char* ttt_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TTT_H_ */

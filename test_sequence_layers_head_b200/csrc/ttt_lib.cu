@@ -1,0 +1,315 @@
+// libttt: C ABI of the TTT inner-loop forward on B200 (sm_100a).
+//
+// Host side: argument validation (synchronous, before any launch), kernel
+// selection, TMA descriptor creation and launch.  The declarations and the
+// contract of every entry point are in include/ttt.h.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/ttt.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "linear_tc.cuh"
+#include "simt.cuh"
+#include "tmap.h"
+
+namespace ttt {
+
+// Per-device status word (bit kStatusTimeout: a bounded wait expired).
+__device__ int g_status_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+int* g_status_ptr[kMaxDevices] = {};
+std::mutex g_mu;
+
+// Device address of the status word on the current device (looked up once
+// per device with that device current).
+int* status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<int*>(p);
+    }
+    return g_status_ptr[dev];
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+
+ttt_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        fprintf(stderr, "libttt: launch failed: %s\n", cudaGetErrorString(e));
+        return TTT_ERR_CUDA;
+    }
+    return TTT_OK;
+}
+
+// Raise the dynamic shared memory limit of a kernel once per device.
+template <typename K>
+bool set_smem(K kernel, size_t bytes) {
+    if (bytes <= 48 * 1024) return true;
+    if (bytes > 227 * 1024) return false;
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
+}
+
+unsigned long long wait_ns(unsigned ms) { return 1000000ull * (ms ? ms : kDefaultWaitMs); }
+
+// ---------------------------------------------------------------------------
+// TTT-Linear
+// ---------------------------------------------------------------------------
+template <int D, bool LN, typename IO>
+ttt_status launch_simt_linear(const ttt_linear_args* a, cudaStream_t st) {
+    SimtLinearParams p;
+    p.H = a->H;
+    p.T = a->T;
+    p.b = a->b;
+    p.Q = a->Q;
+    p.K = a->K;
+    p.V = a->V;
+    p.eta = a->eta;
+    p.eta_const = a->eta_const;
+    p.W0 = a->W0;
+    p.W0_bstride = a->W0_bstride;
+    p.c0 = a->c0;
+    p.c0_bstride = a->c0_bstride;
+    p.gamma = a->ln_gamma;
+    p.beta = a->ln_beta;
+    p.eps = a->ln_eps;
+    p.Z = a->Z;
+    p.W_out = a->W_out;
+    p.c_out = a->c_out;
+    const size_t smem = simt_linear_smem(D, a->b);
+    auto k = simt_linear_kernel<D, LN, IO>;
+    if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
+    k<<<a->B * a->H, kSimtThreads, smem, st>>>(p);
+    return launch_status();
+}
+
+template <int D, bool LN>
+ttt_status simt_linear_dtype(const ttt_linear_args* a, cudaStream_t st) {
+    return a->io_dtype == TTT_F32 ? launch_simt_linear<D, LN, float>(a, st)
+                                  : launch_simt_linear<D, LN, __nv_bfloat16>(a, st);
+}
+
+template <bool LN>
+ttt_status simt_linear(const ttt_linear_args* a, cudaStream_t st) {
+    switch (a->d) {
+        case 16: return simt_linear_dtype<16, LN>(a, st);
+        case 32: return simt_linear_dtype<32, LN>(a, st);
+        case 64: return simt_linear_dtype<64, LN>(a, st);
+        default: return TTT_ERR_UNSUPPORTED;
+    }
+}
+
+template <bool LN>
+ttt_status tc_linear(const ttt_linear_args* a, cudaStream_t st) {
+    using namespace ltc;
+    const long long U = (long long)a->B * a->H;
+    const long long rows = U * a->T;
+    CUtensorMap mQ, mK, mV, mZ;
+    const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!encode_2d(&mQ, a->Q, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&mK, a->K, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&mV, a->V, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&mZ, a->Z, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return TTT_ERR_CUDA;
+    Params p;
+    p.U = (int)U;
+    p.H = a->H;
+    p.T = a->T;
+    p.nsteps = a->T / kTok;
+    p.eta = a->eta;
+    p.eta_const = a->eta_const;
+    p.W0 = a->W0;
+    p.W0_bstride = a->W0_bstride;
+    p.c0 = a->c0;
+    p.c0_bstride = a->c0_bstride;
+    p.gamma = a->ln_gamma;
+    p.beta = a->ln_beta;
+    p.eps = a->ln_eps;
+    p.W_out = a->W_out;
+    p.c_out = a->c_out;
+    p.status = status_ptr();
+    p.wait_ns = wait_ns(a->wait_timeout_ms);
+    p.flags = a->flags;
+    if (!p.status) return TTT_ERR_CUDA;
+    auto k = linear_tc_kernel<LN>;
+    if (!set_smem(k, kSmemBytes)) return TTT_ERR_CUDA;
+    const int grid = (int)((U + 1) / 2);
+    k<<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, mZ, p);
+    return launch_status();
+}
+
+ttt_status validate_common(int B, int H, int T, int d, int b, ttt_dtype io) {
+    if (B < 0 || H < 0 || T < 0 || b < 1) return TTT_ERR_INVALID_ARG;
+    if (io != TTT_F32 && io != TTT_BF16) return TTT_ERR_INVALID_ARG;
+    if (d <= 0) return TTT_ERR_INVALID_ARG;
+    if (T % b != 0) return TTT_ERR_INVALID_ARG;
+    if (d != 16 && d != 32 && d != 64) return TTT_ERR_UNSUPPORTED;
+    if (b > 64) return TTT_ERR_UNSUPPORTED;
+    const long long rows = (long long)B * H * T;
+    if ((long long)B * H > (1ll << 30) || rows >= (1ll << 31)) return TTT_ERR_UNSUPPORTED;
+    return TTT_OK;
+}
+
+}  // namespace
+}  // namespace ttt
+
+using namespace ttt;
+
+extern "C" ttt_status ttt_linear_forward(const ttt_linear_args* a, cudaStream_t stream) {
+    if (!a) return TTT_ERR_INVALID_ARG;
+    ttt_status v = validate_common(a->B, a->H, a->T, a->d, a->b, a->io_dtype);
+    if (v != TTT_OK) return v;
+    const long long units = (long long)a->B * a->H;
+    if (units == 0) return TTT_OK;
+    if (a->T > 0 && (!ok_ptr(a->Q) || !ok_ptr(a->K) || !ok_ptr(a->V) || !ok_ptr(a->Z)))
+        return TTT_ERR_INVALID_ARG;
+    if (!ok_ptr(a->W0) || !ok_ptr(a->W_out) || !ok_opt(a->eta)) return TTT_ERR_INVALID_ARG;
+    if (a->W0_bstride < 0 || a->c0_bstride < 0) return TTT_ERR_INVALID_ARG;
+    if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
+    if (a->use_ln) {
+        if (!ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !ok_opt(a->c0) || !ok_opt(a->c_out))
+            return TTT_ERR_INVALID_ARG;
+        if (!(a->ln_eps > 0.f)) return TTT_ERR_INVALID_ARG;
+    }
+    if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL)) return TTT_ERR_INVALID_ARG;
+    const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
+                    !(a->flags & TTT_FLAG_FORCE_SIMT);
+    if (tc) return a->use_ln ? tc_linear<true>(a, stream) : tc_linear<false>(a, stream);
+    if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
+    return a->use_ln ? simt_linear<true>(a, stream) : simt_linear<false>(a, stream);
+}
+
+// ---------------------------------------------------------------------------
+// TTT-MLP
+// ---------------------------------------------------------------------------
+namespace ttt {
+namespace {
+
+template <int D, typename IO>
+ttt_status launch_simt_mlp(const ttt_mlp_args* a, cudaStream_t st) {
+    SimtMlpParams p;
+    p.H = a->H;
+    p.T = a->T;
+    p.b = a->b;
+    p.Q = a->Q;
+    p.K = a->K;
+    p.V = a->V;
+    p.eta = a->eta;
+    p.eta_const = a->eta_const;
+    p.W1 = a->W1;
+    p.c1 = a->c1;
+    p.W2 = a->W2;
+    p.c2 = a->c2;
+    p.per_seq = a->params_per_sequence;
+    p.Z = a->Z;
+    p.W1_out = a->W1_out;
+    p.c1_out = a->c1_out;
+    p.W2_out = a->W2_out;
+    p.c2_out = a->c2_out;
+    const size_t smem = simt_mlp_smem(D, a->b);
+    auto k = simt_mlp_kernel<D, IO>;
+    if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
+    k<<<a->B * a->H, kSimtThreads, smem, st>>>(p);
+    return launch_status();
+}
+
+template <int D>
+ttt_status simt_mlp_dtype(const ttt_mlp_args* a, cudaStream_t st) {
+    return a->io_dtype == TTT_F32 ? launch_simt_mlp<D, float>(a, st) : launch_simt_mlp<D, __nv_bfloat16>(a, st);
+}
+
+}  // namespace
+}  // namespace ttt
+
+extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream) {
+    if (!a) return TTT_ERR_INVALID_ARG;
+    ttt_status v = validate_common(a->B, a->H, a->T, a->d, a->b, a->io_dtype);
+    if (v != TTT_OK) return v;
+    const long long units = (long long)a->B * a->H;
+    if (units == 0) return TTT_OK;
+    if (a->T > 0 && (!ok_ptr(a->Q) || !ok_ptr(a->K) || !ok_ptr(a->V) || !ok_ptr(a->Z)))
+        return TTT_ERR_INVALID_ARG;
+    if (!ok_ptr(a->W1) || !ok_ptr(a->W2) || !ok_opt(a->c1) || !ok_opt(a->c2) || !ok_opt(a->eta))
+        return TTT_ERR_INVALID_ARG;
+    if (!ok_ptr(a->W1_out) || !ok_ptr(a->W2_out) || !ok_opt(a->c1_out) || !ok_opt(a->c2_out))
+        return TTT_ERR_INVALID_ARG;
+    if (a->params_per_sequence != 0 && a->params_per_sequence != 1) return TTT_ERR_INVALID_ARG;
+    if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL)) return TTT_ERR_INVALID_ARG;
+    if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
+    switch (a->d) {
+        case 16: return simt_mlp_dtype<16>(a, stream);
+        case 32: return simt_mlp_dtype<32>(a, stream);
+        case 64: return simt_mlp_dtype<64>(a, stream);
+        default: return TTT_ERR_UNSUPPORTED;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Decode
+// ---------------------------------------------------------------------------
+namespace ttt {
+namespace {
+template <int D>
+ttt_status launch_decode(const ttt_decode_args* a, cudaStream_t st) {
+    DecodeParams p{a->W, a->q, a->k, a->v, a->eta, a->eta_const, a->z};
+    const int units = a->B * a->H;
+    if (a->io_dtype == TTT_F32)
+        decode_kernel<D, float><<<units, (D / 4) * (D / 4), 0, st>>>(p);
+    else
+        decode_kernel<D, __nv_bfloat16><<<units, (D / 4) * (D / 4), 0, st>>>(p);
+    return launch_status();
+}
+}  // namespace
+}  // namespace ttt
+
+extern "C" ttt_status ttt_linear_decode_step(const ttt_decode_args* a, cudaStream_t stream) {
+    if (!a) return TTT_ERR_INVALID_ARG;
+    if (a->B < 0 || a->H < 0 || a->d <= 0) return TTT_ERR_INVALID_ARG;
+    if (a->io_dtype != TTT_F32 && a->io_dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
+    if (a->d != 16 && a->d != 32 && a->d != 64) return TTT_ERR_UNSUPPORTED;
+    if ((long long)a->B * a->H > (1ll << 30)) return TTT_ERR_UNSUPPORTED;
+    if ((long long)a->B * a->H == 0) return TTT_OK;
+    if (!ok_ptr(a->W) || !ok_ptr(a->q) || !ok_ptr(a->k) || !ok_ptr(a->v) || !ok_ptr(a->z) || !ok_opt(a->eta))
+        return TTT_ERR_INVALID_ARG;
+    switch (a->d) {
+        case 16: return launch_decode<16>(a, stream);
+        case 32: return launch_decode<32>(a, stream);
+        default: return launch_decode<64>(a, stream);
+    }
+}
+
+extern "C" const char* ttt_status_string(ttt_status s) {
+    switch (s) {
+        case TTT_OK: return "TTT_OK";
+        case TTT_ERR_INVALID_ARG: return "TTT_ERR_INVALID_ARG";
+        case TTT_ERR_UNSUPPORTED: return "TTT_ERR_UNSUPPORTED";
+        case TTT_ERR_CUDA: return "TTT_ERR_CUDA";
+        case TTT_ERR_TIMEOUT: return "TTT_ERR_TIMEOUT";
+    }
+    return "TTT_ERR_UNKNOWN";
+}
+
+extern "C" ttt_status ttt_last_device_status(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return TTT_ERR_CUDA;
+    int* p = status_ptr();
+    if (!p) return TTT_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return TTT_ERR_CUDA;
+    if (h != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TTT_ERR_CUDA;
+    }
+    return (h & kStatusTimeout) ? TTT_ERR_TIMEOUT : TTT_OK;
+}
+
+extern "C" const char* ttt_version(void) { return "ttt-b200 0.1.0 (sm_100a)"; }

@@ -1,0 +1,184 @@
+"""ctypes binding of libttt (include/ttt.h).
+
+Argument marshalling only: torch tensors provide device memory and the
+current CUDA stream; every step of the computation runs in the library's
+CUDA kernels.  Functions take CUDA tensors and return CUDA tensors; outputs
+may be passed in (preallocated) or are allocated with torch.
+
+Raises :class:`TTTError` when the library returns a non-OK status and
+:class:`RuntimeError` when the library is missing (there is no fallback).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libttt.so")
+
+TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED, TTT_ERR_CUDA, TTT_ERR_TIMEOUT = range(5)
+TTT_F32, TTT_BF16 = 0, 1
+FLAG_FORCE_SIMT = 0x1
+FLAG_TEST_STALL = 0x100
+
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_ll = ctypes.c_longlong
+_u = ctypes.c_uint
+
+
+class LinearArgs(ctypes.Structure):
+    _fields_ = [("B", _i), ("H", _i), ("T", _i), ("d", _i), ("b", _i), ("io_dtype", _i),
+                ("Q", _vp), ("K", _vp), ("V", _vp), ("eta", _vp), ("eta_const", _f),
+                ("W0", _vp), ("W0_bstride", _ll), ("c0", _vp), ("c0_bstride", _ll),
+                ("use_ln", _i), ("ln_gamma", _vp), ("ln_beta", _vp), ("ln_eps", _f),
+                ("Z", _vp), ("W_out", _vp), ("c_out", _vp), ("flags", _u), ("wait_timeout_ms", _u)]
+
+
+class MlpArgs(ctypes.Structure):
+    _fields_ = [("B", _i), ("H", _i), ("T", _i), ("d", _i), ("b", _i), ("io_dtype", _i),
+                ("Q", _vp), ("K", _vp), ("V", _vp), ("eta", _vp), ("eta_const", _f),
+                ("W1", _vp), ("c1", _vp), ("W2", _vp), ("c2", _vp), ("params_per_sequence", _i),
+                ("Z", _vp), ("W1_out", _vp), ("c1_out", _vp), ("W2_out", _vp), ("c2_out", _vp),
+                ("flags", _u), ("wait_timeout_ms", _u)]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("B", _i), ("H", _i), ("d", _i), ("io_dtype", _i), ("W", _vp), ("q", _vp), ("k", _vp),
+                ("v", _vp), ("eta", _vp), ("eta_const", _f), ("z", _vp)]
+
+
+class TTTError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)}")
+        self.code = code
+
+
+_lib = None
+
+# Every symbol include/ttt.h declares.
+EXPORTS = ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_status_string",
+           "ttt_last_device_status", "ttt_version")
+
+
+def library() -> ctypes.CDLL:
+    """Load libttt.so (built in-tree by ``build.py``); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libttt.so not found at {LIB_PATH}; build it with "
+                               "`python -m test_sequence_layers_head_b200.build` (no CPU fallback exists)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.ttt_linear_forward.argtypes = [ctypes.POINTER(LinearArgs), _vp]
+        L.ttt_linear_forward.restype = _i
+        L.ttt_mlp_forward.argtypes = [ctypes.POINTER(MlpArgs), _vp]
+        L.ttt_mlp_forward.restype = _i
+        L.ttt_linear_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
+        L.ttt_linear_decode_step.restype = _i
+        L.ttt_status_string.argtypes = [_i]
+        L.ttt_status_string.restype = ctypes.c_char_p
+        L.ttt_last_device_status.argtypes = [_vp]
+        L.ttt_last_device_status.restype = _i
+        L.ttt_version.argtypes = []
+        L.ttt_version.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return library().ttt_status_string(code).decode()
+
+
+def version() -> str:
+    return library().ttt_version().decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libttt takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libttt takes contiguous tensors only")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _io_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return TTT_BF16
+    if t.dtype == torch.float32:
+        return TTT_F32
+    raise ValueError(f"unsupported io dtype {t.dtype}")
+
+
+def _check(code: int, what: str):
+    if code != TTT_OK:
+        raise TTTError(code, what)
+
+
+def linear_forward(Q, K, V, eta, W0, b, *, eta_const=0.0, use_ln=False, c0=None, gamma=None, beta=None,
+                   eps=1e-6, Z=None, W_out=None, c_out=None, flags=0, wait_timeout_ms=0, stream=None):
+    """TTT-Linear (optionally LN+residual) prefill; see ``ttt_linear_forward``.
+
+    Q, K, V: [B,H,T,d] bf16 or fp32; eta: [B,H,T] fp32 or None (eta_const);
+    W0: [H,d,d] (shared) or [B,H,d,d] fp32.  Returns (Z, W_out, c_out).
+    """
+    B, H, T, d = Q.shape
+    dev = Q.device
+    if Z is None:
+        Z = torch.empty_like(Q)
+    if W_out is None:
+        W_out = torch.empty((B, H, d, d), device=dev, dtype=torch.float32)
+    if use_ln and c_out is None:
+        c_out = torch.empty((B, H, d), device=dev, dtype=torch.float32)
+    W0_bstride = 0 if W0.dim() == 3 else H * d * d
+    c0_bstride = H * d if (c0 is not None and c0.dim() == 3) else 0
+    a = LinearArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
+                   _ptr(W0), W0_bstride, _ptr(c0), c0_bstride, int(bool(use_ln)), _ptr(gamma), _ptr(beta),
+                   float(eps), _ptr(Z), _ptr(W_out), _ptr(c_out), int(flags), int(wait_timeout_ms))
+    _check(library().ttt_linear_forward(ctypes.byref(a), _stream(stream)), "ttt_linear_forward")
+    return Z, W_out, c_out
+
+
+def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, *, eta_const=0.0, Z=None, W1_out=None, c1_out=None,
+                W2_out=None, c2_out=None, flags=0, wait_timeout_ms=0, stream=None):
+    """TTT-MLP prefill; see ``ttt_mlp_forward``.  Returns (Z, W1, c1, W2, c2)."""
+    B, H, T, d = Q.shape
+    m = W1.shape[-1]
+    dev = Q.device
+    f32 = torch.float32
+    Z = torch.empty_like(Q) if Z is None else Z
+    W1_out = torch.empty((B, H, d, m), device=dev, dtype=f32) if W1_out is None else W1_out
+    c1_out = torch.empty((B, H, m), device=dev, dtype=f32) if c1_out is None else c1_out
+    W2_out = torch.empty((B, H, m, d), device=dev, dtype=f32) if W2_out is None else W2_out
+    c2_out = torch.empty((B, H, d), device=dev, dtype=f32) if c2_out is None else c2_out
+    per_seq = 1 if W1.dim() == 4 else 0
+    a = MlpArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
+                _ptr(W1), _ptr(c1), _ptr(W2), _ptr(c2), per_seq, _ptr(Z), _ptr(W1_out), _ptr(c1_out),
+                _ptr(W2_out), _ptr(c2_out), int(flags), int(wait_timeout_ms))
+    _check(library().ttt_mlp_forward(ctypes.byref(a), _stream(stream)), "ttt_mlp_forward")
+    return Z, W1_out, c1_out, W2_out, c2_out
+
+
+def linear_decode_step(W, q, k, v, eta, *, eta_const=0.0, z=None, stream=None):
+    """One decode token per unit; W [B,H,d,d] fp32 is updated in place.  Returns z."""
+    B, H, d = q.shape
+    z = torch.empty_like(q) if z is None else z
+    a = DecodeArgs(B, H, d, _io_dtype(q), _ptr(W), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), float(eta_const),
+                   _ptr(z))
+    _check(library().ttt_linear_decode_step(ctypes.byref(a), _stream(stream)), "ttt_linear_decode_step")
+    return z
+
+
+def last_device_status(stream=None) -> int:
+    """Synchronise and return (and clear) the device status (TTT_OK / TTT_ERR_TIMEOUT / ...)."""
+    return library().ttt_last_device_status(_stream(stream))

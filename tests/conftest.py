@@ -18,3 +18,12 @@ def oracle_mod():
     from oracle import oracle
     oracle.lib()
     return oracle
+
+
+@pytest.fixture(scope="session")
+def ttt_lib():
+    """The CUDA library, built in-tree if it is missing or stale."""
+    from test_sequence_layers_head_b200 import build, ttt
+    build.build()
+    ttt.library()
+    return ttt

@@ -1,0 +1,110 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/ttt.h declares, and rejects invalid arguments
+synchronously, before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "ttt.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(ttt_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_entry_points():
+    syms = declared_symbols()
+    for s in ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step"):
+        assert s in syms
+
+
+def test_library_exports_every_declared_symbol(ttt_lib):
+    L = ttt_lib.library()
+    for s in declared_symbols():
+        assert hasattr(L, s), s
+    assert set(declared_symbols()) <= set(ttt_lib.EXPORTS) | set(declared_symbols())
+
+
+def test_status_strings(ttt_lib):
+    assert ttt_lib.status_string(0) == "TTT_OK"
+    assert ttt_lib.status_string(4) == "TTT_ERR_TIMEOUT"
+    assert ttt_lib.version().startswith("ttt-b200")
+
+
+def _linear_args(ttt, **kw):
+    a = ttt.LinearArgs()
+    a.B, a.H, a.T, a.d, a.b, a.io_dtype = 1, 1, 32, 64, 16, ttt.TTT_BF16
+    fake = 1 << 20  # aligned fake device address; never dereferenced (validation fails first)
+    a.Q = a.K = a.V = a.Z = a.W0 = a.W_out = fake
+    a.ln_eps = 1e-6
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("T", 30, 1),          # T % b != 0
+    ("b", 0, 1),
+    ("B", -1, 1),
+    ("d", 48, 2),          # unsupported head dim
+    ("d", 0, 1),
+    ("b", 128, 1),         # T = 32 is not a multiple of 128
+    ("io_dtype", 7, 1),
+    ("Q", None, 1),        # null pointer
+    ("K", (1 << 20) + 4, 1),  # misaligned
+    ("W_out", None, 1),
+    ("eta", (1 << 20) + 8, 1),
+    ("use_ln", 2, 1),
+    ("flags", 0x8000, 1),
+    ("W0_bstride", -1, 1),
+])
+def test_linear_forward_rejects_invalid_arguments(ttt_lib, field, value, code):
+    a = _linear_args(ttt_lib, **{field: value})
+    assert ttt_lib.library().ttt_linear_forward(ctypes.byref(a), None) == code
+
+
+def test_linear_forward_large_b_unsupported(ttt_lib):
+    a = _linear_args(ttt_lib, b=128, T=256)
+    assert ttt_lib.library().ttt_linear_forward(ctypes.byref(a), None) == 2
+
+
+def test_linear_forward_ln_requires_gamma_beta(ttt_lib):
+    a = _linear_args(ttt_lib, use_ln=1)
+    assert ttt_lib.library().ttt_linear_forward(ctypes.byref(a), None) == 1
+
+
+def test_empty_batch_is_a_no_op(ttt_lib):
+    a = _linear_args(ttt_lib, B=0)
+    assert ttt_lib.library().ttt_linear_forward(ctypes.byref(a), None) == 0
+
+
+def test_null_args_struct(ttt_lib):
+    L = ttt_lib.library()
+    assert L.ttt_linear_forward(None, None) == 1
+    assert L.ttt_mlp_forward(None, None) == 1
+    assert L.ttt_linear_decode_step(None, None) == 1
+
+
+def test_mlp_and_decode_validation(ttt_lib):
+    L = ttt_lib.library()
+    m = ttt_lib.MlpArgs()
+    m.B, m.H, m.T, m.d, m.b, m.io_dtype = 1, 1, 32, 64, 16, ttt_lib.TTT_BF16
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1   # null pointers
+    m.T = 33
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
+    dargs = ttt_lib.DecodeArgs()
+    dargs.B, dargs.H, dargs.d, dargs.io_dtype = 2, 2, 64, ttt_lib.TTT_BF16
+    assert L.ttt_linear_decode_step(ctypes.byref(dargs), None) == 1
+    dargs.d = 24
+    assert L.ttt_linear_decode_step(ctypes.byref(dargs), None) == 2
+
+
+def test_binding_refuses_cpu_tensors(ttt_lib):
+    import torch
+    x = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ttt_lib.linear_forward(x, x, x, None, torch.zeros(1, 64, 64), 16)

@@ -1,0 +1,291 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Small cases span several mini-batches, odd unit counts (the tensor-core
+kernel pairs units per CTA) and every inner model; the full-size workloads
+are checked on sampled units that the oracle recomputes one by one.
+Tolerances are the problem statement's: max relative error <= 1e-4 for fp32
+workloads, normwise <= 2e-2 on Z and on the final state for bf16 inputs with
+fp32 state.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from test_sequence_layers_head_b200 import workloads as WL
+from tests.gpu_util import assert_close, normwise, poison_like, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+def run_linear(ttt, inp, use_ln=False, flags=0, eta_none=False):
+    r, w = inp.raw, inp.w
+    Q, K, V = to_dev(r["Q"]), to_dev(r["K"]), to_dev(r["V"])
+    eta = None if eta_none else to_dev(r["eta"])
+    W0 = to_dev(r["W0"])
+    kw = {}
+    if use_ln:
+        kw = dict(c0=to_dev(r["c0"]), gamma=to_dev(r["gamma"]), beta=to_dev(r["beta"]), eps=w.ln_eps)
+    B, H, T, d = Q.shape
+    Z = poison_like(Q)
+    Wout = torch.full((B, H, d, d), float("nan"), device="cuda")
+    cout = torch.full((B, H, d), float("nan"), device="cuda") if use_ln else None
+    ttt.linear_forward(Q, K, V, eta, W0, w.b, eta_const=w.eta_const, use_ln=use_ln, Z=Z, W_out=Wout,
+                       c_out=cout, flags=flags, **kw)
+    torch.cuda.synchronize()
+    assert ttt.last_device_status() == ttt.TTT_OK
+    return to_host(Z), to_host(Wout), (to_host(cout) if use_ln else None)
+
+
+def oracle_linear(inp, use_ln=False):
+    e, w = inp.exact, inp.w
+    kw = dict(c0=e["c0"], gamma=e["gamma"], beta=e["beta"], eps=w.ln_eps) if use_ln else {}
+    return O.linear_forward(e["Q"], e["K"], e["V"], e["eta"], e["W0"], w.b, use_ln=use_ln, **kw)
+
+
+def check_linear(ttt, inp, use_ln=False, flags=0):
+    Zg, Wg, cg = run_linear(ttt, inp, use_ln, flags)
+    Zo, Wo, co = oracle_linear(inp, use_ln)
+    ez = assert_close("Z", Zg, Zo, inp.w.io_dtype)
+    ew = assert_close("W_out", Wg, Wo, inp.w.io_dtype)
+    if use_ln:
+        assert_close("c_out", cg, co, inp.w.io_dtype)
+    return ez, ew
+
+
+# ---------------------------------------------------------------------------
+# TTT-Linear, tensor-core kernel (bf16, d = 64, b = 16)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,H,T", [(1, 1, 16), (1, 2, 48), (1, 3, 160), (2, 5, 64), (3, 3, 256)])
+@pytest.mark.parametrize("use_ln", [False, True])
+def test_linear_tc_small(ttt_lib, B, H, T, use_ln):
+    inp = WL.random_case("ln" if use_ln else "linear", B, H, T, 64, 16, seed=B * 100 + H * 10 + T)
+    ez, ew = check_linear(ttt_lib, inp, use_ln)
+    # the bf16-operand error is well below the tolerance at these sizes
+    assert ez < 1e-2 and ew < 1e-2, (ez, ew)
+
+
+@pytest.mark.parametrize("use_ln", [False, True])
+def test_linear_tc_matches_simt(ttt_lib, use_ln):
+    """The tensor-core and the fp32 CUDA-core kernels agree on the same inputs."""
+    inp = WL.random_case("ln" if use_ln else "linear", 2, 3, 128, 64, 16, seed=5)
+    Zt, Wt, _ = run_linear(ttt_lib, inp, use_ln)
+    Zs, Ws, _ = run_linear(ttt_lib, inp, use_ln, flags=ttt_lib.FLAG_FORCE_SIMT)
+    assert normwise(Zt, Zs) < 1e-2 and normwise(Wt, Ws) < 1e-2
+
+
+def test_linear_tc_constant_eta_and_per_sequence_W0(ttt_lib):
+    w = WL.Workload("c", "linear", 2, 2, 96, 64, 16, WL.BF16, "const", 0.02, 11)
+    inp = WL.make_inputs(w, threads=1)
+    # per-sequence initial state [B,H,d,d]
+    rng = np.random.default_rng(3)
+    W0 = rng.standard_normal((2, 2, 64, 64)) / 8.0
+    raw, ex = WL.store(W0, WL.F32)
+    inp.raw["W0"], inp.exact["W0"] = raw, ex
+    Zg, Wg, _ = run_linear(ttt_lib, inp, eta_none=True)
+    e = inp.exact
+    Zo, Wo, _ = O.linear_forward(e["Q"], e["K"], e["V"], np.full((2, 2, 96), np.float32(0.02)), e["W0"], 16)
+    assert_close("Z", Zg, Zo, WL.BF16)
+    assert_close("W_out", Wg, Wo, WL.BF16)
+
+
+def test_linear_tc_theorem1(ttt_lib):
+    """W0 = 0, eta = 1, b = T = 16: causal linear attention (section 4.1)."""
+    w = WL.Workload("t1", "linear", 1, 2, 16, 64, 16, WL.BF16, "const", 1.0, 13)
+    inp = WL.make_inputs(w, threads=1)
+    inp.raw["W0"] = np.zeros((2, 64, 64), np.float32)
+    inp.exact["W0"] = np.zeros((2, 64, 64))
+    Zg, _, _ = run_linear(ttt_lib, inp, eta_none=True)
+    q, k, v = (inp.exact[n][0] for n in "QKV")
+    ref = np.einsum("hts,hsd->htd", np.tril(np.einsum("htd,hsd->hts", q, k)), v)
+    assert normwise(Zg[0], ref) < 1e-2
+
+
+def test_linear_tc_eta_zero(ttt_lib):
+    w = WL.Workload("z", "linear", 1, 3, 64, 64, 16, WL.BF16, "const", 0.0, 17)
+    inp = WL.make_inputs(w, threads=1)
+    Zg, Wg, _ = run_linear(ttt_lib, inp, eta_none=True)
+    assert np.array_equal(Wg, np.broadcast_to(inp.exact["W0"][None], Wg.shape))
+    Zo = np.einsum("bhtd,hde->bhte", inp.exact["Q"], inp.exact["W0"])
+    assert normwise(Zg, Zo) < 1e-2
+
+
+@pytest.mark.parametrize("use_ln", [False, True])
+def test_linear_tc_chunked_calls(ttt_lib, use_ln):
+    """forward(T1) then forward(T2) from its final state equals forward(T1+T2)."""
+    inp = WL.random_case("ln" if use_ln else "linear", 1, 3, 96, 64, 16, seed=23)
+    r = inp.raw
+    dev = {k: to_dev(v) for k, v in r.items()}
+    kw = dict(gamma=dev["gamma"], beta=dev["beta"]) if use_ln else {}
+    Zf, Wf, cf = ttt_lib.linear_forward(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], 16, use_ln=use_ln,
+                                        c0=dev.get("c0"), **kw)
+    T1 = 48
+    sl = lambda t, a, b: t[:, :, a:b].contiguous()
+    Za, Wa, ca = ttt_lib.linear_forward(sl(dev["Q"], 0, T1), sl(dev["K"], 0, T1), sl(dev["V"], 0, T1),
+                                        sl(dev["eta"], 0, T1), dev["W0"], 16, use_ln=use_ln, c0=dev.get("c0"),
+                                        **kw)
+    Zb, Wb, cb = ttt_lib.linear_forward(sl(dev["Q"], T1, 96), sl(dev["K"], T1, 96), sl(dev["V"], T1, 96),
+                                        sl(dev["eta"], T1, 96), Wa, 16, use_ln=use_ln, c0=ca, **kw)
+    torch.cuda.synchronize()
+    # identical arithmetic on both routes except the bf16 rounding of the
+    # resumed state, which is the same fp32 value: results match exactly
+    assert torch.equal(torch.cat([Za, Zb], 2), Zf)
+    assert torch.equal(Wb, Wf)
+
+
+# ---------------------------------------------------------------------------
+# TTT-Linear, fp32 CUDA-core kernel
+# ---------------------------------------------------------------------------
+
+def test_linear_d16_f32_workload(ttt_lib):
+    """The fp32 workload (d = 16, T = 256, eta = 0.1): max relative error <= 1e-4."""
+    w = WL.WORKLOADS["linear_d16_T256_f32"]
+    inp = WL.make_inputs(w, threads=1)
+    Zg, Wg, _ = run_linear(ttt_lib, inp, eta_none=True)
+    e = inp.exact
+    Zo, Wo, _ = O.linear_forward(e["Q"], e["K"], e["V"], np.full(e["eta"].shape, np.float32(0.1)), e["W0"], 16)
+    assert_close("Z", Zg, Zo, WL.F32)
+    assert_close("W_out", Wg, Wo, WL.F32)
+
+
+@pytest.mark.parametrize("d,b,T,io", [(16, 1, 37, WL.F32), (32, 8, 64, WL.F32), (64, 64, 128, WL.F32),
+                                      (32, 16, 96, WL.BF16), (16, 4, 0, WL.F32)])
+@pytest.mark.parametrize("use_ln", [False, True])
+def test_linear_simt_shapes(ttt_lib, d, b, T, io, use_ln):
+    if T % b:
+        pytest.skip("T must be a multiple of b")
+    inp = WL.random_case("ln" if use_ln else "linear", 2, 2, T, d, b, io_dtype=io, seed=d + b + T)
+    check_linear(ttt_lib, inp, use_ln)
+
+
+# ---------------------------------------------------------------------------
+# TTT-MLP
+# ---------------------------------------------------------------------------
+
+def run_mlp(ttt, inp, flags=0):
+    r, w = inp.raw, inp.w
+    args = [to_dev(r[n]) for n in ("Q", "K", "V", "eta", "W1", "c1", "W2", "c2")]
+    out = ttt.mlp_forward(*args, w.b, eta_const=w.eta_const, flags=flags)
+    torch.cuda.synchronize()
+    return [to_host(x) for x in out]
+
+
+def check_mlp(ttt, inp, flags=0):
+    got = run_mlp(ttt, inp, flags)
+    e = inp.exact
+    ref = O.mlp_forward(e["Q"], e["K"], e["V"], e["eta"], e["W1"], e["c1"], e["W2"], e["c2"], inp.w.b)
+    errs = [assert_close(n, g, o, inp.w.io_dtype) for n, g, o in zip(("Z", "W1", "c1", "W2", "c2"), got, ref)]
+    return errs
+
+
+@pytest.mark.parametrize("d,b,T,io", [(16, 16, 64, WL.F32), (32, 8, 48, WL.F32), (16, 4, 32, WL.BF16)])
+def test_mlp_simt_shapes(ttt_lib, d, b, T, io):
+    inp = WL.random_case("mlp", 2, 2, T, d, b, io_dtype=io, eta_mode="const", eta_const=0.05, seed=d * b)
+    check_mlp(ttt_lib, inp)
+
+
+@pytest.mark.parametrize("B,H,T", [(1, 1, 16), (1, 2, 64), (2, 3, 128)])
+def test_mlp_d64_bf16(ttt_lib, B, H, T):
+    inp = WL.random_case("mlp", B, H, T, 64, 16, io_dtype=WL.BF16, eta_mode="const", eta_const=1 / 64,
+                         seed=B + H + T)
+    check_mlp(ttt_lib, inp)
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d,io", [(64, WL.BF16), (32, WL.F32), (16, WL.BF16)])
+def test_decode_steps(ttt_lib, d, io):
+    w = WL.Workload("dec", "linear", 3, 5, 1, d, 1, io, "sigmoid", 0.0, 31)
+    rng = np.random.default_rng(d)
+    W = rng.standard_normal((3, 5, d, d)) / np.sqrt(d)
+    Wd = torch.tensor(W, dtype=torch.float32, device="cuda")
+    Wo = Wd.double().cpu().numpy()
+    for step in range(6):
+        raw, ex = WL.make_decode_tokens(w, step)
+        q, k, v, eta = (to_dev(raw[n]) for n in ("q", "k", "v", "eta"))
+        z = ttt_lib.linear_decode_step(Wd, q, k, v, eta)
+        Wo, zo = O.linear_decode_step(Wo, ex["q"], ex["k"], ex["v"], ex["eta"])
+        torch.cuda.synchronize()
+        if io == WL.F32:
+            assert_close("z", to_host(z), zo, io)
+        else:
+            assert normwise(to_host(z), zo) < 1e-2
+        assert normwise(to_host(Wd), Wo) < 1e-5
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, sampled units
+# ---------------------------------------------------------------------------
+
+def sampled_parity(ttt, w, units, flags=0):
+    inp = WL.make_inputs(w, want_exact=False)
+    r = inp.raw
+    dev = {k: to_dev(v) for k, v in r.items()}
+    B, H = w.B, w.H
+    if w.kind == "mlp":
+        out = ttt.mlp_forward(dev["Q"], dev["K"], dev["V"], None, dev["W1"], dev["c1"], dev["W2"], dev["c2"], w.b,
+                              eta_const=w.eta_const, flags=flags)
+    else:
+        ln = w.kind == "ln"
+        kw = dict(c0=dev["c0"], gamma=dev["gamma"], beta=dev["beta"], eps=w.ln_eps) if ln else {}
+        out = ttt.linear_forward(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], w.b, use_ln=ln, flags=flags,
+                                 **kw)
+    torch.cuda.synchronize()
+    assert ttt.last_device_status() == ttt.TTT_OK
+    del dev
+    errs = []
+    for u in units:
+        n, h = divmod(u, H)
+        one = WL.make_unit_inputs(w, u)
+        e = one.exact
+        if w.kind == "mlp":
+            ref = O.mlp_forward(e["Q"], e["K"], e["V"], np.full(e["eta"].shape, w.eta_const), e["W1"], e["c1"],
+                                e["W2"], e["c2"], w.b)
+            names = ("Z", "W1", "c1", "W2", "c2")
+        else:
+            ln = w.kind == "ln"
+            kw = dict(c0=e["c0"], gamma=e["gamma"], beta=e["beta"], eps=w.ln_eps) if ln else {}
+            ref = O.linear_forward(e["Q"], e["K"], e["V"], e["eta"], e["W0"], w.b, use_ln=ln, **kw)
+            names = ("Z", "W_out", "c_out")[: 3 if ln else 2]
+        for nm, g, o in zip(names, out, ref):
+            errs.append(assert_close(f"{nm}[unit {u}]", to_host(g[n, h]), o[0, 0], w.io_dtype))
+    return max(errs)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,units", [
+    ("linear_B8_H12_T2048", [0, 1, 47, 95]),
+    ("ln_B4_H32_T8192", [0, 77, 127]),
+    ("mlp_B2_H32_T8192", [0, 63]),
+    ("linear_B16_H32_T32768_decode1024", [0, 257, 511]),
+])
+def test_full_size_sampled(ttt_lib, name, units):
+    sampled_parity(ttt_lib, WL.WORKLOADS[name], units)
+
+
+@pytest.mark.slow
+def test_long_decode_after_prefill(ttt_lib):
+    """Decode phase of the long-context workload (all 16 x 32 units, 1024
+    steps) starting from a prefill's final state; every step's z and the
+    final state are compared with the oracle.  The prefill is shortened to
+    T = 256 here so that the oracle stays cheap; the full-length prefill is
+    covered by test_full_size_sampled."""
+    w = WL.scaled(WL.WORKLOADS["linear_B16_H32_T32768_decode1024"], T=256)
+    inp = WL.make_inputs(w)
+    dev = {k: to_dev(v) for k, v in inp.raw.items()}
+    _, Wd, _ = ttt_lib.linear_forward(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], 16)
+    e = inp.exact
+    _, Wo, _ = O.linear_forward(e["Q"], e["K"], e["V"], e["eta"], e["W0"], 16)
+    Wo = to_host(Wd)   # continue the oracle from the GPU prefill state to isolate the decode error
+    worst = 0.0
+    for step in range(w.decode_steps):
+        raw, ex = WL.make_decode_tokens(w, step)
+        z = ttt_lib.linear_decode_step(Wd, *(to_dev(raw[n]) for n in ("q", "k", "v", "eta")))
+        Wo, zo = O.linear_decode_step(Wo, ex["q"], ex["k"], ex["v"], ex["eta"])
+        worst = max(worst, normwise(to_host(z), zo))
+    torch.cuda.synchronize()
+    assert worst < 2e-2
+    assert normwise(to_host(Wd), Wo) < 2e-2
