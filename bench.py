@@ -1,0 +1,477 @@
+"""Benchmark of the TTT inner-loop forward on B200.
+
+Default workload: the long-context TTT-Linear prefill (B=16 sequences,
+H=32 heads, d=64, T=32768 tokens, mini-batch b=16, bf16 Q/K/V/Z, fp32
+state), the largest single-GPU configuration.  One step = one call of
+ttt_linear_forward over the whole batch (every row of the hot path:
+TMA loads, the key-side residual, the causal outputs, the in-place state
+update and the final-state store).
+
+Prints ONE JSON line:
+  value       prefill tokens/s per layer (B*T / time, all heads), summed over
+              ranks (weak scaling: every rank runs its own B=16 batch)
+  roofline    the prefill kernel against HBM bandwidth (algorithmic bytes:
+              Q, K, V, Z bf16 + eta fp32 per token-head, W0 per head, W_out per
+              unit), achieved from CUDA events around each launch
+  cpu_baseline  the float64 oracle on a bounded sample, host cores
+  e2e         the same metric through the public API with pinned host
+              buffers (H2D of Q/K/V/eta, D2H of Z and the final state inside
+              the timed region)
+  decode      the 1024-step decode phase of the same workload (CUDA graph)
+  rows        the other workloads measured the same way (informational)
+
+--impl reference times the float64 oracle (the reference arm) on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from test_sequence_layers_head_b200 import workloads as WL  # noqa: E402
+
+METRIC = "TTT layer tokens/sec (prefill, per B200) and % of dual-form roofline"
+UNIT = "tokens/s"
+DEFAULT_WORKLOAD = "linear_B16_H32_T32768_decode1024"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work (per launch)
+# ---------------------------------------------------------------------------
+
+def algorithmic_bytes(w: WL.Workload) -> int:
+    """Bytes a launch must move: Q, K, V read and Z written (io dtype), eta
+    read (fp32, when per-token), the initial state read once per head and the
+    final state written once per unit."""
+    io = 2 if w.io_dtype == WL.BF16 else 4
+    th = w.units * w.T
+    per_tok = 4 * w.d * io + (4 if w.eta_mode == "sigmoid" else 0)
+    if w.kind == "mlp":
+        state = 2 * w.d * w.hidden + w.hidden + w.d
+    else:
+        state = w.d * w.d + (w.d if w.kind == "ln" else 0)
+    return th * per_tok + 4 * state * (w.H + w.units)
+
+
+def algorithmic_flops(w: WL.Workload) -> int:
+    """Dual-form flops per token-head: linear 6 d^2 + 4 b d (key residual,
+    outputs, state update, causal term); LN adds the causal +1 term; MLP is
+    the two-layer version with hidden m = 4d."""
+    d, b, m = w.d, w.b, w.hidden
+    if w.kind == "mlp":
+        per = 2 * d * m * 2 + 2 * m * d * 2 + 2 * m * d + 2 * d * m + 2 * b * d + 2 * b * m + 2 * b * m + 2 * b * d
+    else:
+        per = 6 * d * d + 4 * b * d
+    return w.units * w.T * per
+
+
+def tokens(w: WL.Workload) -> int:
+    return w.B * w.T
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", FALLBACK_HBM_GBS), d.get("bf16_tflops", FALLBACK_BF16_TFLOPS), "measured"
+    return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        loaded = [r[0] for r in rows if r[2] > 200.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def shard_units(total_sequences: int, world: int, rank: int):
+    """Sequences owned by `rank` when `total_sequences` are split evenly
+    (used when a fixed global batch is spread over ranks)."""
+    per = (total_sequences + world - 1) // world
+    lo = min(rank * per, total_sequences)
+    return lo, min(lo + per, total_sequences)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def to_dev(raw, torch):
+    if raw.dtype == np.uint16:
+        return torch.from_numpy(np.ascontiguousarray(raw).view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(np.ascontiguousarray(raw)).cuda()
+
+
+def call_forward(ttt, w, dev, out):
+    if w.kind == "mlp":
+        return ttt.mlp_forward(dev["Q"], dev["K"], dev["V"], dev.get("eta"), dev["W1"], dev["c1"], dev["W2"],
+                               dev["c2"], w.b, eta_const=w.eta_const, Z=out["Z"], W1_out=out["W1"],
+                               c1_out=out["c1"], W2_out=out["W2"], c2_out=out["c2"])
+    ln = w.kind == "ln"
+    kw = dict(c0=dev["c0"], gamma=dev["gamma"], beta=dev["beta"], eps=w.ln_eps) if ln else {}
+    return ttt.linear_forward(dev["Q"], dev["K"], dev["V"], dev.get("eta"), dev["W0"], w.b, eta_const=w.eta_const,
+                              use_ln=ln, Z=out["Z"], W_out=out["W"], c_out=out.get("c"), **kw)
+
+
+def alloc_outputs(w, torch):
+    B, H, T, d = w.B, w.H, w.T, w.d
+    io = torch.bfloat16 if w.io_dtype == WL.BF16 else torch.float32
+    out = {"Z": torch.empty((B, H, T, d), dtype=io, device="cuda")}
+    if w.kind == "mlp":
+        m = w.hidden
+        out.update(W1=torch.empty((B, H, d, m), device="cuda"), c1=torch.empty((B, H, m), device="cuda"),
+                   W2=torch.empty((B, H, m, d), device="cuda"), c2=torch.empty((B, H, d), device="cuda"))
+    else:
+        out["W"] = torch.empty((B, H, d, d), device="cuda")
+        if w.kind == "ln":
+            out["c"] = torch.empty((B, H, d), device="cuda")
+    return out
+
+
+def device_inputs(w, torch, threads):
+    inp = WL.make_inputs(w, want_exact=False, threads=threads)
+    dev = {k: to_dev(v, torch) for k, v in inp.raw.items()}
+    if w.eta_mode == "const":
+        dev.pop("eta")
+    return inp, dev
+
+
+def time_launches(torch, fn, steps, warmup, flush=None):
+    """Per-launch CUDA-event durations (ms) plus the whole timed span (ms)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        if flush is not None:
+            flush()
+        evs[i][0].record(st)
+        fn()
+        evs[i][1].record(st)
+    torch.cuda.synchronize()
+    per = [a.elapsed_time(b) for a, b in evs]
+    return per
+
+
+def measure_decode(ttt, w, torch, steps=3):
+    """Decode phase: w.decode_steps single-token steps for all units, captured
+    in one CUDA graph; returns per-step time and roofline numbers."""
+    B, H, d = w.B, w.H, w.d
+    g = np.random.default_rng(0)
+    W = torch.tensor((g.standard_normal((B, H, d, d)) / np.sqrt(d)).astype(np.float32), device="cuda")
+    n = w.decode_steps
+    toks = [WL.make_decode_tokens(w, s)[0] for s in range(n)]
+    q = torch.stack([to_dev(t["q"], torch) for t in toks])
+    k = torch.stack([to_dev(t["k"], torch) for t in toks])
+    v = torch.stack([to_dev(t["v"], torch) for t in toks])
+    eta = torch.stack([to_dev(t["eta"], torch) for t in toks])
+    z = torch.empty_like(q)
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        for s in range(3):   # warm-up outside the graph
+            ttt.linear_decode_step(W, q[s], k[s], v[s], eta[s], z=z[s], stream=st)
+    torch.cuda.current_stream().wait_stream(st)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cs = torch.cuda.current_stream()
+        for s in range(n):
+            ttt.linear_decode_step(W, q[s], k[s], v[s], eta[s], z=z[s], stream=cs)
+    graph.replay()
+    torch.cuda.synchronize()
+    per = time_launches(torch, graph.replay, steps, 1)
+    ms = statistics.median(per)
+    io = 2
+    bytes_step = w.units * (2 * d * d * 4 + 4 * d * io + 4)
+    del graph
+    return {"steps_per_graph": n, "us_per_step": 1000.0 * ms / n, "tokens_per_s": w.B * n / (ms / 1000.0),
+            "bytes_per_step": bytes_step, "achieved_gbs": bytes_step * n / (ms / 1000.0) / 1e9,
+            "note": "W (8.4 MB) stays L2-resident across steps; GB/s is against HBM peak for reference",
+            "gpu_launches_per_graph": n}
+
+
+def measure_e2e(ttt, w, inp, torch, steps):
+    """The public API on pinned host buffers: H2D inputs, forward, D2H of Z
+    and the final state, all inside the timed region, every step."""
+    host = {}
+    for k_, v_ in inp.raw.items():
+        a = np.ascontiguousarray(v_)
+        th = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        if a.dtype == np.uint16:
+            th = th.view(torch.bfloat16)
+        host[k_] = th.pin_memory()
+    if w.eta_mode == "const":
+        host.pop("eta")
+    dev = {k_: torch.empty_like(v_, device="cuda") for k_, v_ in host.items()}
+    out = alloc_outputs(w, torch)
+    out_host = {k_: torch.empty_like(v_, device="cpu").pin_memory() for k_, v_ in out.items()}
+    h2d = sum(v_.numel() * v_.element_size() for v_ in host.values())
+    d2h = sum(v_.numel() * v_.element_size() for v_ in out.values())
+
+    def step():
+        for k_ in host:
+            dev[k_].copy_(host[k_], non_blocking=True)
+        call_forward(ttt, w, dev, out)
+        for k_ in out:
+            out_host[k_].copy_(out[k_], non_blocking=True)
+
+    per = time_launches(torch, step, steps, 1)
+    ms = statistics.mean(per)
+    del dev, out, host, out_host
+    return {"value": tokens(w) / (ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms}
+
+
+def cpu_baseline(w, sample_sequences=4):
+    """The float64 oracle on a bounded sample: `sample_sequences` sequences
+    (all heads, full length) of the workload, on every host core."""
+    from oracle import oracle as O
+    ws = WL.scaled(w, B=sample_sequences)
+    inp = WL.make_inputs(ws, threads=O.default_threads())
+    e = inp.exact
+    cores = O.default_threads()
+    t0 = time.perf_counter()
+    if w.kind == "mlp":
+        O.mlp_forward(e["Q"], e["K"], e["V"], np.full(e["eta"].shape, w.eta_const), e["W1"], e["c1"], e["W2"],
+                      e["c2"], w.b, threads=cores)
+    else:
+        ln = w.kind == "ln"
+        kw = dict(c0=e["c0"], gamma=e["gamma"], beta=e["beta"], eps=w.ln_eps) if ln else {}
+        eta = e["eta"] if w.eta_mode == "sigmoid" else np.full(e["eta"].shape, w.eta_const)
+        O.linear_forward(e["Q"], e["K"], e["V"], eta, e["W0"], w.b, use_ln=ln, threads=cores, **kw)
+    dt = time.perf_counter() - t0
+    return {"value": sample_sequences * w.T / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{sample_sequences} of {w.B} sequences x {w.H} heads x T={w.T} (float64 primal, OpenMP)",
+            "seconds": dt}
+
+
+def run_ours(args):
+    import torch
+    from test_sequence_layers_head_b200 import ttt
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist = None
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    w = WL.WORKLOADS[args.workload]
+    if args.T:
+        w = WL.scaled(w, T=args.T)
+    threads = max(1, len(os.sched_getaffinity(0)) // max(1, ws))
+    inp, dev = device_inputs(w, torch, threads)
+    out = alloc_outputs(w, torch)
+    fn = lambda: call_forward(ttt, w, dev, out)   # noqa: E731
+    fn()
+    torch.cuda.synchronize()
+    assert ttt.last_device_status() == ttt.TTT_OK
+    hbm, tflops, peak_src = measured_peaks()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    with ClockSampler(local) as clk:
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        st = torch.cuda.current_stream()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        t0.record(st)
+        for i in range(args.steps):
+            evs[i][0].record(st)
+            fn()
+            evs[i][1].record(st)
+        t1.record(st)
+        torch.cuda.synchronize()
+        barrier()
+    clocks = clk.summary()
+    total_ms = t0.elapsed_time(t1)
+    launch_ms = [a.elapsed_time(b) for a, b in evs]
+    if dist is not None:
+        tt = torch.tensor([total_ms, statistics.mean(launch_ms)], device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms, mean_launch = tt.tolist()
+    else:
+        mean_launch = statistics.mean(launch_ms)
+    status = ttt.last_device_status()
+    ms_step = total_ms / args.steps
+    value = ws * tokens(w) / (ms_step / 1000.0)
+
+    abytes = algorithmic_bytes(w)
+    aflops = algorithmic_flops(w)
+    if w.kind == "mlp":
+        achieved = aflops / (mean_launch / 1000.0) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tflops, "unit": "TFLOP/s",
+                "frac": achieved / tflops, "peak_source": peak_src}
+    else:
+        achieved = abytes / (mean_launch / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_source": peak_src}
+    roof.update({"kernel": "linear_tc_kernel" if w.kind != "mlp" else "mlp kernel",
+                 "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": aflops,
+                 "mean_launch_ms": mean_launch, "traffic": args.traffic})
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.io_dtype == WL.BF16 else "f32",
+            "data": "synthetic (seeded PCG64 Gaussian inputs with the workload's distributions)",
+            "config": {"workload": w.name, "kind": w.kind, "B_per_gpu": w.B, "H": w.H, "T": w.T, "d": w.d,
+                       "b": w.b, "global_batch": w.B * ws, "parallelism": f"replicas x{ws} (units sharded, no collective)",
+                       "l2": f"inputs larger than L2 ({abytes / 1e9:.2f} GB per step)"},
+            "roofline": roof, "clocks": clocks, "gpu_launches": args.steps, "device_status": status}
+    if rank == 0 and not args.no_extras:
+        line["e2e"] = measure_e2e(ttt, w, inp, torch, steps=args.e2e_steps)
+        if w.decode_steps:
+            line["decode"] = measure_decode(ttt, w, torch)
+        if not args.no_rows:
+            line["rows"] = measure_rows(ttt, torch, threads)
+        line["cpu_baseline"] = cpu_baseline(w)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure_rows(ttt, torch, threads):
+    """The other workloads, each timed over a few launches with an L2 flush
+    between launches (informational; parity lives in the tests)."""
+    res = {}
+    flush_buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")
+    hbm, tflops, _ = measured_peaks()
+    for name in ("linear_B8_H12_T2048", "ln_B4_H32_T8192", "mlp_B2_H32_T8192", "linear_d16_T256_f32"):
+        w = WL.WORKLOADS[name]
+        _, dev = device_inputs(w, torch, threads)
+        out = alloc_outputs(w, torch)
+        per = time_launches(torch, lambda: call_forward(ttt, w, dev, out), 5, 2, flush=lambda: flush_buf.zero_())
+        ms = statistics.median(per)
+        r = {"ms": ms, "tokens_per_s": tokens(w) / (ms / 1000.0),
+             "hbm_frac": algorithmic_bytes(w) / (ms / 1000.0) / 1e9 / hbm,
+             "tensor_frac": algorithmic_flops(w) / (ms / 1000.0) / 1e12 / tflops}
+        res[name] = r
+        del dev, out
+    return res
+
+
+def run_reference(args):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return
+    w = WL.WORKLOADS[args.workload]
+    if args.T:
+        w = WL.scaled(w, T=args.T)
+    for _ in range(args.warmup):
+        cpu_baseline(w, sample_sequences=1)
+    vals = [cpu_baseline(w, sample_sequences=1) for _ in range(args.steps)]
+    value = statistics.mean(v["value"] for v in vals)
+    secs = sum(v["seconds"] for v in vals)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "kind": w.kind, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "b": w.b},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"], "kind": "oracle",
+                             "sample": f"each step: 1 of {w.B} sequences x {w.H} heads x T={w.T}"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WL.WORKLOAD_ORDER)
+    ap.add_argument("--T", type=int, default=0, help="override T (profiling a smaller case)")
+    ap.add_argument("--no-extras", action="store_true", help="only the timed prefill (profiling)")
+    ap.add_argument("--no-rows", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch from an ncu capture of the current kernel build")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
