@@ -78,6 +78,20 @@ def algorithmic_flops(w: WL.Workload) -> int:
     return w.units * w.T * per
 
 
+def recorded_traffic(kernel: str, src: str):
+    """DRAM bytes per launch recorded from an ncu capture in profiles/traffic.json,
+    or None when the kernel source changed since the capture."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))[kernel]
+        sha = hashlib.sha256(open(os.path.join(ROOT, "test_sequence_layers_head_b200", "csrc", src), "rb").read())
+        if sha.hexdigest()[:16] == rec["src_sha256_16"]:
+            return rec["bytes_per_launch"]
+    except (OSError, KeyError, ValueError):
+        pass
+    return None
+
+
 def tokens(w: WL.Workload) -> int:
     return w.B * w.T
 
@@ -160,6 +174,15 @@ def shard_units(total_sequences: int, world: int, rank: int):
     per = (total_sequences + world - 1) // world
     lo = min(rank * per, total_sequences)
     return lo, min(lo + per, total_sequences)
+
+
+def max_over_ranks(values, dist, device="cpu"):
+    """Element-wise maximum of per-rank timings (the slowest rank decides)."""
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
 
 
 # ---------------------------------------------------------------------------
@@ -366,12 +389,7 @@ def run_ours(args):
     clocks = clk.summary()
     total_ms = t0.elapsed_time(t1)
     launch_ms = [a.elapsed_time(b) for a, b in evs]
-    if dist is not None:
-        tt = torch.tensor([total_ms, statistics.mean(launch_ms)], device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms, mean_launch = tt.tolist()
-    else:
-        mean_launch = statistics.mean(launch_ms)
+    total_ms, mean_launch = max_over_ranks([total_ms, statistics.mean(launch_ms)], dist, "cuda")
     status = ttt.last_device_status()
     ms_step = total_ms / args.steps
     value = ws * tokens(w) / (ms_step / 1000.0)
@@ -388,7 +406,10 @@ def run_ours(args):
                 "peak_source": peak_src}
     roof.update({"kernel": "linear_tc_kernel" if w.kind != "mlp" else "mlp kernel",
                  "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": aflops,
-                 "mean_launch_ms": mean_launch, "traffic": args.traffic})
+                 "mean_launch_ms": mean_launch,
+                 "traffic": args.traffic if args.traffic is not None else (
+                     recorded_traffic("linear_tc_kernel", "linear_tc.cuh")
+                     if (w.kind == "linear" and w.name == DEFAULT_WORKLOAD and not args.T) else None)})
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.io_dtype == WL.BF16 else "f32",
