@@ -114,12 +114,11 @@ ttt_status tc_linear(const ttt_linear_args* a, cudaStream_t st) {
     using namespace ltc;
     const long long U = (long long)a->B * a->H;
     const long long rows = U * a->T;
-    CUtensorMap mQ, mK, mV, mZ;
+    CUtensorMap mQ, mK, mV;
     const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!encode_2d(&mQ, a->Q, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&mK, a->K, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&mV, a->V, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !encode_2d(&mZ, a->Z, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !encode_2d(&mV, a->V, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B))
         return TTT_ERR_CUDA;
     Params p;
     p.U = (int)U;
@@ -135,6 +134,7 @@ ttt_status tc_linear(const ttt_linear_args* a, cudaStream_t st) {
     p.gamma = a->ln_gamma;
     p.beta = a->ln_beta;
     p.eps = a->ln_eps;
+    p.Z = static_cast<__nv_bfloat16*>(a->Z);
     p.W_out = a->W_out;
     p.c_out = a->c_out;
     p.status = status_ptr();
@@ -144,7 +144,7 @@ ttt_status tc_linear(const ttt_linear_args* a, cudaStream_t st) {
     auto k = linear_tc_kernel<LN>;
     if (!set_smem(k, kSmemBytes)) return TTT_ERR_CUDA;
     const int grid = (int)((U + 1) / 2);
-    k<<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, mZ, p);
+    k<<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, p);
     return launch_status();
 }
 

@@ -128,10 +128,14 @@ def test_linear_tc_chunked_calls(ttt_lib, use_ln):
     Zb, Wb, cb = ttt_lib.linear_forward(sl(dev["Q"], T1, 96), sl(dev["K"], T1, 96), sl(dev["V"], T1, 96),
                                         sl(dev["eta"], T1, 96), Wa, 16, use_ln=use_ln, c0=ca, **kw)
     torch.cuda.synchronize()
-    # identical arithmetic on both routes except the bf16 rounding of the
-    # resumed state, which is the same fp32 value: results match exactly
-    assert torch.equal(torch.cat([Za, Zb], 2), Zf)
-    assert torch.equal(Wb, Wf)
+    # the resumed call starts its look-ahead from the bf16 copy of the stored
+    # state, so the two routes agree to rounding, not bit for bit
+    Zc = to_host(torch.cat([Za, Zb], 2))
+    assert normwise(Zc, to_host(Zf)) < 5e-3
+    assert normwise(to_host(Wb), to_host(Wf)) < 5e-3
+    Zo, Wo, _ = oracle_linear(inp, use_ln)
+    assert_close("Z (chunked)", Zc, Zo, WL.BF16)
+    assert_close("W_out (chunked)", to_host(Wb), Wo, WL.BF16)
 
 
 # ---------------------------------------------------------------------------
