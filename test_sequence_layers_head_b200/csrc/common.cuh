@@ -9,7 +9,7 @@
 namespace ttt {
 
 // Bits of the per-device status word written by kernels.
-enum : int { kStatusTimeout = 1 };
+enum : int { kStatusTimeout = 1, kStatusBadSmem = 2 };
 
 // Default limit of one device-side wait.
 constexpr unsigned kDefaultWaitMs = 2000;

@@ -37,10 +37,12 @@
 // tcgen05's M range for the 16 x 16 products Q K^T, K_i K_{i-1}^T and
 // Q_i K_{i-1}^T; two helper warps compute them with mma.sync.
 //
-// Warp roles (256 threads): warp 0 TMA producer, warp 1 MMA issuer, warps 2-3
-// helpers (one per unit), warps 4-7 epilogue (warp 4+q reads TMEM lanes
-// 32q..32q+31: warps 4-5 unit 0, warps 6-7 unit 1; thread = one output
-// feature j of one unit).
+// Warp roles (256 threads): warps 0-3 epilogue (warp q reads TMEM lanes
+// 32q..32q+31: warps 0-1 unit 0, warps 2-3 unit 1; thread = one output
+// feature j of one unit), warp 4 TMA producer, warp 5 MMA issuer, warps 6-7
+// helpers (one per unit).  The epilogue warps hold the lowest warp ids, so
+// on each SM sub-partition the scheduler favours them over the helper and
+// waiting warps that share it.
 //
 // Every wait is bounded; on expiry the kernel records kStatusTimeout, stops
 // issuing new asynchronous work, drains what it issued and returns.
@@ -74,9 +76,9 @@ constexpr int kStageBytes = 17408;                   // 17 KB, multiple of 1024
 constexpr int kOffStages = 0;
 constexpr int kOffRed = kStages * kStageBytes;       // LN: 3 buffers x [4 warps][16] float2
 constexpr int kOffBar = kOffRed + 3 * 4 * 16 * 8;
-constexpr int kNumBars = 3 * kStages + 4;
+constexpr int kNumBars = 3 * kStages + 5;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmemBytes = kOffMisc + 64 + 1024;     // + alignment slack
+constexpr int kSmemBytes = kOffMisc + 64;
 
 // TMEM columns
 constexpr uint32_t kTmemCols = 256;
@@ -151,19 +153,6 @@ __device__ __forceinline__ void load_b_frags(uint32_t tile, int lane, uint32_t (
         ldsm_x4(tile + row * 128 + ((ch ^ (row & 7)) << 4), f[ks]);
     }
 }
-// acc[nt][4] (16 x 16) = A (16 x 64) . B^T (64 x 16)
-__device__ __forceinline__ void mm16(const uint32_t (*a)[4], const uint32_t (*b)[4], float (*acc)[4]) {
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[nt][c] = 0.f;
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-        mma_16816(acc[0], a[ks], b[ks][0], b[ks][1]);
-        mma_16816(acc[1], a[ks], b[ks][2], b[ks][3]);
-    }
-}
-
 // Butterfly reduce-scatter of two 16-vectors over the 32 lanes of a warp:
 // afterwards a[0], b[0] of lanes 2t and 2t+1 hold the warp sums of token t.
 __device__ __forceinline__ void warp_reduce2(float* a, float* b, int lane) {
@@ -228,8 +217,15 @@ template <bool LN>
 __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
     linear_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, Params p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // No static shared memory: the dynamic buffer starts at the beginning of
+    // the CTA's shared window (1024-byte aligned, as the 128B-swizzled tiles
+    // need).  Addressing it directly keeps every access in the shared state
+    // space (no generic-address loads).
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicOr(p.status, kStatusBadSmem);
+        return;
+    }
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint64_t* full = bars;                    // [kStages] TMA landed
     uint64_t* empty = bars + kStages;         // [kStages] stage free: MMA commit + 4 epilogue warps
@@ -238,6 +234,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
     uint64_t* grp_done = op_ready + 1;        // one MMA group complete
     uint64_t* drain = op_ready + 2;           // final MMA drain
     uint64_t* stall = op_ready + 3;           // never arrived on (test hook)
+    uint64_t* w_done = op_ready + 4;          // the group's state update (MMA_W) complete
     uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffMisc);
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -258,10 +255,11 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
         mbar_init(grp_done, 1);
         mbar_init(drain, 1);
         mbar_init(stall, 1);
+        mbar_init(w_done, 1);
         *s_abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == 5) {
         tmem_alloc(s_tmem, kTmemCols);
         tmem_relinquish();
     }
@@ -275,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
         atomicOr(p.status, kStatusTimeout);
     };
 
-    if (warp == 0) {
+    if (warp == 4) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             int issued_last = -1;
@@ -312,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 if (!wait_bounded(&full[i % kStages], (i / kStages) & 1, lim, nullptr)) fail();
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 5) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const uint32_t idP = make_idesc_bf16(128, 64, 0, 0);
@@ -327,22 +325,25 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 const int s = g % kStages;
                 const uint32_t par = (g / kStages) & 1;
                 const uint32_t st = smem_u32(smem + kOffStages + s * kStageBytes);
+                const uint32_t sp = smem_u32(smem + kOffStages + ((g + kStages - 1) % kStages) * kStageBytes);
+                uint64_t bdP[4];
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) bdP[ks] = make_sdesc(st + kOffK0 + 32 * ks, 16, 1024, kSwizzle128B);
+                const uint64_t bdC = make_sdesc(st + kOffBC, 128, 256, kSwizzleNone);
+                // B = [K0 | K1] of the previous batch, MN-major: two 64-wide atoms 4 KB apart
+                const uint64_t bdW = make_sdesc(sp + kOffK0, 4096, 1024, kSwizzle128B);
                 if (g < nsteps && !wait_bounded(&full[s], par, lim, s_abort)) { fail(); break; }
                 if (g >= 1 && g < nsteps && !wait_bounded(&aux[s], par, lim, s_abort)) { fail(); break; }
                 if (!wait_bounded(op_ready, g & 1, lim, s_abort)) { fail(); break; }
                 tc_fence_after();
+                // the state update first, with its own commit, so that the
+                // epilogue converts W_g while MMA_P / MMA_C run
+                if (g >= 1) umma_ts(tbase + kColW, tbase + kColA, bdW, idW, 1);
+                umma_commit(w_done);
                 if (g < nsteps) {
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_ts(tbase + kColP, tbase + kColAW + 8 * ks,
-                                make_sdesc(st + kOffK0 + 32 * ks, 16, 1024, kSwizzle128B), idP, ks > 0);
-                    if (g >= 1)
-                        umma_ts(tbase + kColP, tbase + kColA, make_sdesc(st + kOffBC, 128, 256, kSwizzleNone), idP, 1);
-                }
-                if (g >= 1) {
-                    const uint32_t sp = smem_u32(smem + kOffStages + ((g - 1) % kStages) * kStageBytes);
-                    // B = [K0 | K1] of the previous batch, MN-major: two 64-wide atoms 4 KB apart
-                    umma_ts(tbase + kColW, tbase + kColA, make_sdesc(sp + kOffK0, 4096, 1024, kSwizzle128B), idW, 1);
+                    for (int ks = 0; ks < 4; ++ks) umma_ts(tbase + kColP, tbase + kColAW + 8 * ks, bdP[ks], idP, ks > 0);
+                    if (g >= 1) umma_ts(tbase + kColP, tbase + kColA, bdC, idP, 1);
                 }
                 umma_commit(grp_done);
                 if (g >= 1) umma_commit(&empty[(g - 1) % kStages]);
@@ -351,9 +352,9 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             umma_commit(drain);
             if (!wait_bounded(drain, 0, lim, nullptr)) fail();
         }
-    } else if (warp == 2 || warp == 3) {
+    } else if (warp >= 6) {
         // ------------------------------------- helpers: 16 x 16 products, one unit each
-        const int u = warp - 2;
+        const int u = warp - 6;
         const int r0 = lane >> 2, c0 = 2 * (lane & 3);
         for (int i = 0; i < nsteps; ++i) {
             const int s = i % kStages;
@@ -363,12 +364,32 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             }
             uint8_t* st = smem + kOffStages + s * kStageBytes;
             const uint32_t kt = smem_u32(st + (u ? kOffK1 : kOffK0)), qt = smem_u32(st + (u ? kOffQ1 : kOffQ0));
-            uint32_t fq[4][4], fk[4][4];
-            float acc[2][4];
+            // fragments: Q_i and K_i as A (rows = tokens), K_i and K_{i-1} as B
+            uint32_t fq[4][4], fka[4][4], fkb[4][4], fp[4][4];
             load_a_frags(qt, lane, fq);
-            load_b_frags(kt, lane, fk);
-            mm16(fq, fk, acc);   // S = Q_i K_i^T
+            load_b_frags(kt, lane, fkb);
+            const bool prev = i >= 1;
+            if (prev) {
+                const uint8_t* pst = smem + kOffStages + ((i - 1) % kStages) * kStageBytes;
+                load_a_frags(kt, lane, fka);
+                load_b_frags(smem_u32(pst + (u ? kOffK1 : kOffK0)), lane, fp);
+            }
+            // S = Q_i K_i^T, CQ = Q_i K_{i-1}^T, CK = K_i K_{i-1}^T, k-steps
+            // interleaved across the six independent accumulators
+            float aS[2][4] = {}, aQ[2][4] = {}, aK[2][4] = {};
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                mma_16816(aS[0], fq[ks], fkb[ks][0], fkb[ks][1]);
+                mma_16816(aS[1], fq[ks], fkb[ks][2], fkb[ks][3]);
+                if (prev) {
+                    mma_16816(aQ[0], fq[ks], fp[ks][0], fp[ks][1]);
+                    mma_16816(aQ[1], fq[ks], fp[ks][2], fp[ks][3]);
+                    mma_16816(aK[0], fka[ks], fp[ks][0], fp[ks][1]);
+                    mma_16816(aK[1], fka[ks], fp[ks][2], fp[ks][3]);
+                }
+            }
             float* S = reinterpret_cast<float*>(st + (u ? kOffS1 : kOffS0));
+            uint8_t* bc = st + kOffBC;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -376,42 +397,22 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                     const int t = r0 + 8 * hh, ss = 8 * nt + c0;
                     const float add = LN ? 1.f : 0.f;
                     *reinterpret_cast<float2*>(S + t * 16 + ss) =
-                        make_float2(acc[nt][2 * hh] + add, acc[nt][2 * hh + 1] + add);
-                }
-            if (i >= 1) {
-                // B_C rows (n = 32u + t): K_i K_{i-1}^T; rows 32u + 16 + t: Q_i K_{i-1}^T
-                const uint8_t* pst = smem + kOffStages + ((i - 1) % kStages) * kStageBytes;
-                uint32_t fp[4][4];
-                load_b_frags(smem_u32(pst + (u ? kOffK1 : kOffK0)), lane, fp);
-                uint8_t* bc = st + kOffBC;
-                mm16(fq, fp, acc);
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int t = r0 + 8 * hh, ss = 8 * nt + c0;
-                        *reinterpret_cast<uint32_t*>(bc + nosw_off(32 * u + 16 + t, ss)) =
-                            pack_bf16x2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
-                    }
-                uint32_t fk2[4][4];
-                load_a_frags(kt, lane, fk2);
-                mm16(fk2, fp, acc);
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const int t = r0 + 8 * hh, ss = 8 * nt + c0;
+                        make_float2(aS[nt][2 * hh] + add, aS[nt][2 * hh + 1] + add);
+                    if (prev) {
+                        // B_C rows (n = 32u + t): K_i K_{i-1}^T; rows 32u + 16 + t: Q_i K_{i-1}^T
                         *reinterpret_cast<uint32_t*>(bc + nosw_off(32 * u + t, ss)) =
-                            pack_bf16x2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+                            pack_bf16x2(aK[nt][2 * hh], aK[nt][2 * hh + 1]);
+                        *reinterpret_cast<uint32_t*>(bc + nosw_off(32 * u + 16 + t, ss)) =
+                            pack_bf16x2(aQ[nt][2 * hh], aQ[nt][2 * hh + 1]);
                     }
-            }
+                }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&aux[s]);
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp - 4, u = q >> 1;
+        const int q = warp, u = q >> 1;
         const int j = 32 * (q & 1) + lane;
         const int unit = u ? unit1 : unit0;
         const bool store_unit = (u == 0) || has1;
@@ -459,27 +460,55 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             const int s = i % kStages;
             const uint32_t par = (i / kStages) & 1;
             const uint8_t* st = smem + kOffStages + s * kStageBytes;
-            if (!dead && (!wait_bounded(grp_done, i & 1, lim, s_abort) || !wait_bounded(&full[s], par, lim, s_abort) ||
-                          !wait_bounded(&aux[s], par, lim, s_abort))) {
+            // 1. inputs of the batch (independent of the tensor cores): eta_t, eta_t v_t
+            if (!dead && (!wait_bounded(&full[s], par, lim, s_abort) || !wait_bounded(&aux[s], par, lim, s_abort))) {
+                dead = true;
+                fail();
+            }
+            const uint8_t* vtile = st + (u ? kOffV1 : kOffV0);
+            const float* etas = reinterpret_cast<const float*>(st + (u ? kOffEta1 : kOffEta0));
+            float et[16], ev[16];
+            if (p.eta) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float4 e4 = reinterpret_cast<const float4*>(etas)[c];
+                    et[4 * c] = e4.x;
+                    et[4 * c + 1] = e4.y;
+                    et[4 * c + 2] = e4.z;
+                    et[4 * c + 3] = e4.w;
+                }
+            } else {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) et[t] = p.eta_const;
+            }
+#pragma unroll
+            for (int t = 0; t < 16; ++t) ev[t] = et[t] * ld_bf16(vtile, sw128_off(t, j));
+            // 2. W_i (after this group's MMA_W) -> bf16, held in registers
+            if (!dead && !wait_bounded(w_done, i & 1, lim, s_abort)) {
+                dead = true;
+                fail();
+            }
+            tc_fence_after();
+            tmem_ld_32x32b_x32(tl + kColW + 64 * u, w);
+            tmem_ld_32x32b_x32(tl + kColW + 64 * u + 32, w + 32);
+            tmem_wait_ld();
+            uint32_t pk[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+            // 3. P of this batch -> A row j; publish A and bf16 W^T for the next group
+            if (!dead && !wait_bounded(grp_done, i & 1, lim, s_abort)) {
                 dead = true;
                 fail();
             }
             tc_fence_after();
             uint32_t pr[32];
             tmem_ld_32x32b_x32(tl + kColP + 32 * u, pr);
-            tmem_ld_32x32b_x32(tl + kColW + 64 * u, w);
-            tmem_ld_32x32b_x32(tl + kColW + 64 * u + 32, w + 32);
             tmem_wait_ld();
-            const uint8_t* vtile = st + (u ? kOffV1 : kOffV0);
-            const float* etas = reinterpret_cast<const float*>(st + (u ? kOffEta1 : kOffEta0));
             float av[16];   // A row j: -eta_t * delta_t
             const float c_old = cj;
             if (!LN) {
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float et = p.eta ? etas[t] : p.eta_const;
-                    av[t] = -et * (__uint_as_float(pr[t]) - ld_bf16(vtile, sw128_off(t, j)));
-                }
+                for (int t = 0; t < 16; ++t) av[t] = fmaf(-et[t], __uint_as_float(pr[t]), ev[t]);
             } else {
                 const uint8_t* ktile = st + (u ? kOffK1 : kOffK0);
                 float y[16], y2[16], x[16];
@@ -497,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                     const float r = rsqrtf(fmaxf(y2[t] * (1.f / kD) - mu * mu, 0.f) + p.eps);
                     x[t] = (x[t] - mu) * r;   // xhat
                     y[t] = r;
+                    // e = k + gamma xhat + beta - v ; ev holds eta v
                     const float e = ld_bf16(ktile, sw128_off(t, j)) + gam * x[t] + bet - ld_bf16(vtile, sw128_off(t, j));
                     g[t] = gam * e;
                     gx[t] = g[t] * x[t];
@@ -506,19 +536,18 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 float csum = 0.f;
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
-                    const float et = p.eta ? etas[t] : p.eta_const;
                     const float delta = y[t] * (av[t] - g[t] * (1.f / kD) - x[t] * gx[t] * (1.f / kD));
-                    av[t] = -et * delta;
+                    av[t] = -et[t] * delta;
                     csum += av[t];
                 }
                 cj += csum;
             }
-            {   // A row j (bf16) -> TMEM; bf16 W^T row j -> TMEM
+            {
                 uint32_t pa[8];
 #pragma unroll
                 for (int c = 0; c < 8; ++c) pa[c] = pack_bf16x2(av[2 * c], av[2 * c + 1]);
                 tmem_st_32x32b_x8(tl + kColA, pa);
-                write_aw();
+                tmem_st_32x32b_x32(tl + kColAW, pk);
                 tmem_wait_st();
             }
             tc_fence_before();
@@ -566,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             if (lane == 0) mbar_arrive(&empty[s]);
         }
         // final state: W after the last group's update
-        if (!dead && !wait_bounded(grp_done, nsteps & 1, lim, s_abort)) {
+        if (!dead && !wait_bounded(w_done, nsteps & 1, lim, s_abort)) {
             dead = true;
             fail();
         }
@@ -583,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == 5) {
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
     }

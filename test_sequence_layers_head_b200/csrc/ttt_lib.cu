@@ -309,6 +309,7 @@ extern "C" ttt_status ttt_last_device_status(cudaStream_t stream) {
         const int zero = 0;
         if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return TTT_ERR_CUDA;
     }
+    if (h & kStatusBadSmem) return TTT_ERR_CUDA;
     return (h & kStatusTimeout) ? TTT_ERR_TIMEOUT : TTT_OK;
 }
 
