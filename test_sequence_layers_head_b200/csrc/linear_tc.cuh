@@ -66,12 +66,11 @@ constexpr int kOffK1 = 2 * kTile;
 constexpr int kOffQ1 = 3 * kTile;
 constexpr int kOffV0 = 4 * kTile;
 constexpr int kOffV1 = 5 * kTile;
-constexpr int kOffS0 = 6 * kTile;                    // fp32 16 x 16 (S, or S + 1 for LN), 1 KB per unit
-constexpr int kOffS1 = kOffS0 + 1024;
-constexpr int kOffBC = kOffS1 + 1024;                // bf16 64 x 16 B operand of MMA_C (K-major, no swizzle)
+constexpr int kOffBS = 6 * kTile;                    // bf16 32 x 16 B operand of MMA_Z: tril(Q K^T) of both units
+constexpr int kOffBC = kOffBS + 1024;                // bf16 64 x 16 B operand of MMA_C (K-major, no swizzle)
 constexpr int kOffEta0 = kOffBC + 2048;              // 64 B per unit
 constexpr int kOffEta1 = kOffEta0 + 64;
-constexpr int kStageBytes = 17408;                   // 17 KB, multiple of 1024
+constexpr int kStageBytes = 16384;                   // 16 KB, multiple of 1024
 
 constexpr int kOffStages = 0;
 constexpr int kOffRed = kStages * kStageBytes;       // LN: 3 buffers x [4 warps][16] float2
@@ -80,12 +79,14 @@ constexpr int kNumBars = 3 * kStages + 5;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64;
 
-// TMEM columns
+// TMEM columns (unit 0 in lanes 0-63, unit 1 in lanes 64-127)
 constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColW = 0;      // fp32 W^T: unit 0 in columns [0,64), unit 1 in [64,128)
-constexpr uint32_t kColP = 128;    // fp32 P: unit 0 [128,160) = [E | Zq], unit 1 [160,192)
-constexpr uint32_t kColAW = 192;   // bf16 W^T (A operand of MMA_P), 32 columns
-constexpr uint32_t kColA = 224;    // bf16 A = -eta * Delta^T (A operand of MMA_C / MMA_W), 8 columns
+constexpr uint32_t kColW = 0;       // fp32 W^T, 64 columns (both units)
+constexpr uint32_t kColP = 64;      // fp32 P: unit 0 columns [64,96) = [E | Zq], unit 1 [96,128)
+constexpr uint32_t kColZc = 128;    // fp32 causal term of the previous batch: unit 0 [128,144), unit 1 [144,160)
+constexpr uint32_t kColAW = 160;    // bf16 W^T (A operand of MMA_P), 32 columns
+constexpr uint32_t kColA = 192;     // bf16 A = -eta * Delta^T (A operand of MMA_C, MMA_Z), 8 columns
+constexpr uint32_t kColAblk = 200;  // bf16 block-diagonal [A_0 0; 0 A_1] (A operand of MMA_W), 16 columns
 
 struct Params {
     int U, H, T;
@@ -312,9 +313,15 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
         }
     } else if (warp == 5) {
         // ---------------------------------------------------------- MMA issuer
+        // group g (0..nsteps) consumes A_{g-1} and bf16 W_{g-1}^T:
+        //   MMA_W  W^T += A_{g-1} K_{g-1}           (block-diagonal A, two MMAs)
+        //   MMA_Z  Zc   = A_{g-1} S_{g-1}^T         (causal term of batch g-1)
+        //   MMA_P  P    = W_{g-1}^T [K_g | Q_g]^T    (four k-steps)
+        //   MMA_C  P   += A_{g-1} [K_{g-1} K_g^T | K_{g-1} Q_g^T]
         if (lane == 0) {
             const uint32_t idP = make_idesc_bf16(128, 64, 0, 0);
-            const uint32_t idW = make_idesc_bf16(128, 128, 0, 1);
+            const uint32_t idW = make_idesc_bf16(128, 64, 0, 1);
+            const uint32_t idZ = make_idesc_bf16(128, 32, 0, 0);
             bool ok = true;
             if (p.flags & TTT_FLAG_TEST_STALL) {
                 // test hook: wait on a barrier nothing arrives on
@@ -330,16 +337,22 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) bdP[ks] = make_sdesc(st + kOffK0 + 32 * ks, 16, 1024, kSwizzle128B);
                 const uint64_t bdC = make_sdesc(st + kOffBC, 128, 256, kSwizzleNone);
-                // B = [K0 | K1] of the previous batch, MN-major: two 64-wide atoms 4 KB apart
-                const uint64_t bdW = make_sdesc(sp + kOffK0, 4096, 1024, kSwizzle128B);
+                // K tiles of the previous batch as MN-major B (one 64-wide atom each)
+                const uint64_t bdW0 = make_sdesc(sp + kOffK0, 1024, 1024, kSwizzle128B);
+                const uint64_t bdW1 = make_sdesc(sp + kOffK1, 1024, 1024, kSwizzle128B);
+                const uint64_t bdZ = make_sdesc(sp + kOffBS, 128, 256, kSwizzleNone);
                 if (g < nsteps && !wait_bounded(&full[s], par, lim, s_abort)) { fail(); break; }
                 if (g >= 1 && g < nsteps && !wait_bounded(&aux[s], par, lim, s_abort)) { fail(); break; }
                 if (!wait_bounded(op_ready, g & 1, lim, s_abort)) { fail(); break; }
                 tc_fence_after();
                 // the state update first, with its own commit, so that the
-                // epilogue converts W_g while MMA_P / MMA_C run
-                if (g >= 1) umma_ts(tbase + kColW, tbase + kColA, bdW, idW, 1);
+                // epilogue converts W_g while the rest of the group runs
+                if (g >= 1) {
+                    umma_ts(tbase + kColW, tbase + kColAblk, bdW0, idW, 1);
+                    umma_ts(tbase + kColW, tbase + kColAblk + 8, bdW1, idW, 1);
+                }
                 umma_commit(w_done);
+                if (g >= 1) umma_ts(tbase + kColZc, tbase + kColA, bdZ, idZ, 0);
                 if (g < nsteps) {
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) umma_ts(tbase + kColP, tbase + kColAW + 8 * ks, bdP[ks], idP, ks > 0);
@@ -388,16 +401,16 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                     mma_16816(aK[1], fka[ks], fp[ks][2], fp[ks][3]);
                 }
             }
-            float* S = reinterpret_cast<float*>(st + (u ? kOffS1 : kOffS0));
+            uint8_t* bs = st + kOffBS;
             uint8_t* bc = st + kOffBC;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int t = r0 + 8 * hh, ss = 8 * nt + c0;
-                    const float add = LN ? 1.f : 0.f;
-                    *reinterpret_cast<float2*>(S + t * 16 + ss) =
-                        make_float2(aS[nt][2 * hh] + add, aS[nt][2 * hh + 1] + add);
+                    // B_S rows (n = 16u + t): tril(Q_i K_i^T), strictly s <= t
+                    *reinterpret_cast<uint32_t*>(bs + nosw_off(16 * u + t, ss)) =
+                        pack_bf16x2(ss <= t ? aS[nt][2 * hh] : 0.f, ss + 1 <= t ? aS[nt][2 * hh + 1] : 0.f);
                     if (prev) {
                         // B_C rows (n = 32u + t): K_i K_{i-1}^T; rows 32u + 16 + t: Q_i K_{i-1}^T
                         *reinterpret_cast<uint32_t*>(bc + nosw_off(32 * u + t, ss)) =
@@ -433,22 +446,17 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             const float* W0u = p.W0 + (size_t)n * p.W0_bstride + (size_t)h * kD * kD;
 #pragma unroll
             for (int i = 0; i < 64; ++i) w[i] = __float_as_uint(W0u[i * kD + j]);
-            uint32_t z[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) z[i] = 0u;
-            // own columns hold W^T, the other unit's columns start at zero
-            tmem_st_32x32b_x32(tl + kColW + 64 * u, w);
-            tmem_st_32x32b_x32(tl + kColW + 64 * u + 32, w + 32);
-            tmem_st_32x32b_x32(tl + kColW + 64 * (1 - u), z);
-            tmem_st_32x32b_x32(tl + kColW + 64 * (1 - u) + 32, z);
-        }
-        auto write_aw = [&]() {   // bf16 W^T row j -> A operand of MMA_P
-            uint32_t pk[32];
+            tmem_st_32x32b_x32(tl + kColW, w);
+            tmem_st_32x32b_x32(tl + kColW + 32, w + 32);
+            uint32_t pk[32], zero[8];
 #pragma unroll
             for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+#pragma unroll
+            for (int c = 0; c < 8; ++c) zero[c] = 0u;
             tmem_st_32x32b_x32(tl + kColAW, pk);
-        };
-        write_aw();
+            // the other unit's half of the block-diagonal A stays zero
+            tmem_st_32x32b_x8(tl + kColAblk + 8 * (1 - u), zero);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -456,6 +464,34 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
 
         bool dead = false;   // set when a wait expired: run the loop without waiting
         __nv_bfloat16* Zu = p.Z + (size_t)unit * p.T * kD + j;
+        float zb[16];        // previous batch: Zq (+ LN: c and the causal "+1" term)
+        // Z of batch i-1 = zb + this group's causal term; the LN residual reads
+        // Q of batch i-1, so its stage is released one step later.
+        auto finish_z = [&](int i1, const float* zc, const uint8_t* pst) {
+            float z[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) z[t] = zb[t] + zc[t];
+            if (LN) {
+                float y[16], y2[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    y[t] = z[t];
+                    y2[t] = z[t] * z[t];
+                }
+                feature_sum2(y, y2, red2, q, lane);
+                const uint8_t* qtile = pst + (u ? kOffQ1 : kOffQ0);
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const float mu = y[t] * (1.f / kD);
+                    const float r = rsqrtf(fmaxf(y2[t] * (1.f / kD) - mu * mu, 0.f) + p.eps);
+                    z[t] = ld_bf16(qtile, sw128_off(t, j)) + gam * (z[t] - mu) * r + bet;
+                }
+            }
+            if (!dead && store_unit) {
+#pragma unroll
+                for (int t = 0; t < 16; ++t) Zu[(size_t)(i1 * kTok + t) * kD] = __float2bfloat16_rn(z[t]);
+            }
+        };
         for (int i = 0; i < nsteps; ++i) {
             const int s = i % kStages;
             const uint32_t par = (i / kStages) & 1;
@@ -481,16 +517,18 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
 #pragma unroll
                 for (int t = 0; t < 16; ++t) et[t] = p.eta_const;
             }
+            if (!LN) {
 #pragma unroll
-            for (int t = 0; t < 16; ++t) ev[t] = et[t] * ld_bf16(vtile, sw128_off(t, j));
+                for (int t = 0; t < 16; ++t) ev[t] = et[t] * ld_bf16(vtile, sw128_off(t, j));
+            }
             // 2. W_i (after this group's MMA_W) -> bf16, held in registers
             if (!dead && !wait_bounded(w_done, i & 1, lim, s_abort)) {
                 dead = true;
                 fail();
             }
             tc_fence_after();
-            tmem_ld_32x32b_x32(tl + kColW + 64 * u, w);
-            tmem_ld_32x32b_x32(tl + kColW + 64 * u + 32, w + 32);
+            tmem_ld_32x32b_x32(tl + kColW, w);
+            tmem_ld_32x32b_x32(tl + kColW + 32, w + 32);
             tmem_wait_ld();
             uint32_t pk[32];
 #pragma unroll
@@ -501,8 +539,9 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 fail();
             }
             tc_fence_after();
-            uint32_t pr[32];
+            uint32_t pr[32], zr[16];
             tmem_ld_32x32b_x32(tl + kColP + 32 * u, pr);
+            tmem_ld_32x32b_x16(tl + kColZc + 16 * u, zr);
             tmem_wait_ld();
             float av[16];   // A row j: -eta_t * delta_t
             const float c_old = cj;
@@ -526,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                     const float r = rsqrtf(fmaxf(y2[t] * (1.f / kD) - mu * mu, 0.f) + p.eps);
                     x[t] = (x[t] - mu) * r;   // xhat
                     y[t] = r;
-                    // e = k + gamma xhat + beta - v ; ev holds eta v
+                    // e = k + gamma xhat + beta - v
                     const float e = ld_bf16(ktile, sw128_off(t, j)) + gam * x[t] + bet - ld_bf16(vtile, sw128_off(t, j));
                     g[t] = gam * e;
                     gx[t] = g[t] * x[t];
@@ -547,6 +586,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
 #pragma unroll
                 for (int c = 0; c < 8; ++c) pa[c] = pack_bf16x2(av[2 * c], av[2 * c + 1]);
                 tmem_st_32x32b_x8(tl + kColA, pa);
+                tmem_st_32x32b_x8(tl + kColAblk + 8 * u, pa);
                 tmem_st_32x32b_x32(tl + kColAW, pk);
                 tmem_wait_st();
             }
@@ -554,55 +594,40 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             __syncwarp();
             if (lane == 0) mbar_arrive(op_ready);
 
-            // outputs: Zq + this batch's causal term (fp32), then the LN residual
-            const float* S = reinterpret_cast<const float*>(st + (u ? kOffS1 : kOffS0));
-            float z[16];
+            // outputs of the previous batch, then keep this batch's pre-residual
+            if (i >= 1) {
+                float zc[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) zc[t] = __uint_as_float(zr[t]);
+                const uint8_t* pst = smem + kOffStages + ((i - 1) % kStages) * kStageBytes;
+                finish_z(i - 1, zc, pst);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[(i - 1) % kStages]);
+            }
+            float pre = LN ? c_old : 0.f;
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
-                float acc = __uint_as_float(pr[16 + t]) + (LN ? c_old : 0.f);
-                const float4* Sr = reinterpret_cast<const float4*>(S + t * 16);
-#pragma unroll
-                for (int c4 = 0; c4 <= t / 4; ++c4) {
-                    const float4 sv = Sr[c4];
-                    const float sx[4] = {sv.x, sv.y, sv.z, sv.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (4 * c4 + e <= t) acc += av[4 * c4 + e] * sx[e];
-                }
-                z[t] = acc;
+                if (LN) pre += av[t];   // causal "+1" term: sum_{s<=t} A[s]
+                zb[t] = __uint_as_float(pr[16 + t]) + pre;
             }
-            if (LN) {
-                float y[16], y2[16];
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    y[t] = z[t];
-                    y2[t] = z[t] * z[t];
-                }
-                feature_sum2(y, y2, red2, q, lane);
-                const uint8_t* qtile = st + (u ? kOffQ1 : kOffQ0);
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const float mu = y[t] * (1.f / kD);
-                    const float r = rsqrtf(fmaxf(y2[t] * (1.f / kD) - mu * mu, 0.f) + p.eps);
-                    z[t] = ld_bf16(qtile, sw128_off(t, j)) + gam * (z[t] - mu) * r + bet;
-                }
-            }
-            if (!dead && store_unit) {
-#pragma unroll
-                for (int t = 0; t < 16; ++t) Zu[(size_t)(i * kTok + t) * kD] = __float2bfloat16_rn(z[t]);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
         }
-        // final state: W after the last group's update
-        if (!dead && !wait_bounded(w_done, nsteps & 1, lim, s_abort)) {
+        // final group: the last batch's causal term and the final state
+        if (!dead && !wait_bounded(grp_done, nsteps & 1, lim, s_abort)) {
             dead = true;
             fail();
         }
         tc_fence_after();
-        tmem_ld_32x32b_x32(tl + kColW + 64 * u, w);
-        tmem_ld_32x32b_x32(tl + kColW + 64 * u + 32, w + 32);
+        uint32_t zr[16];
+        tmem_ld_32x32b_x16(tl + kColZc + 16 * u, zr);
+        tmem_ld_32x32b_x32(tl + kColW, w);
+        tmem_ld_32x32b_x32(tl + kColW + 32, w + 32);
         tmem_wait_ld();
+        if (nsteps >= 1) {
+            float zc[16];
+#pragma unroll
+            for (int t = 0; t < 16; ++t) zc[t] = __uint_as_float(zr[t]);
+            finish_z(nsteps - 1, zc, smem + kOffStages + ((nsteps - 1) % kStages) * kStageBytes);
+        }
         if (store_unit && !dead) {
             float* Wo = p.W_out + (size_t)unit * kD * kD;
 #pragma unroll
