@@ -1,0 +1,631 @@
+// Tensor-core (tcgen05) persistent kernel of the TTT-MLP prefill:
+// f(x) = GELU(x W1 + c1) W2 + c2, d = 64, hidden m = 256, mini-batch b = 16,
+// bf16 Q/K/V/Z, fp32 state.
+//
+// Method (paper digest "论文速览 | TTT", section 3.7, half-loss convention).
+// Per (sequence, head) unit and mini-batch with batch-start parameters:
+//   A  = K W1 + c1,  Hk = GELU(A),  E = Hk W2 + c2 - V
+//   D1 = (E W2^T) * GELU'(A)
+//   Aq = Q W1 + c1 - (tril(Q K^T + 1) * eta_s) D1,  Hq = GELU(Aq)
+//   Z  = Hq W2 + c2 - (tril(Hq Hk^T + 1) * eta_s) E
+//   W1 -= K^T diag(eta) D1,  c1 -= eta^T D1,  W2 -= Hk^T diag(eta) E,  c2 -= eta^T E
+//
+// Mapping onto sm_100a (everything transposed so that the hidden dim m = 256
+// or the head dim d = 64 is the MMA's M):
+//   S1  [A^T | Aq0^T] (m x 32)  = W1^T . [K^T | Q^T]           2 tiles x 4 k-steps
+//   S2  E0^T (d x 16)           = W2^T . Hk^T                  16 k-steps (K = m)
+//   S3  G^T (m x 16)            = W2 . E^T                     2 tiles x 4 k-steps
+//   S4  W1^T += (-eta D1)^T K,  Aq^T += (-eta D1)^T tril(Q K^T)^T,
+//       W2   += (-eta Hk)^T E                                  6 MMAs
+//   S5  Z0^T (d x 16)           = W2^T . Hq^T + (-eta E)^T tril(Hq Hk^T)^T
+// The fp32 accumulators W1^T (m x d) and W2 (m x d) stay in tensor memory for
+// the whole sequence; bf16 W1^T is refreshed in tensor memory (A operand of
+// S1) and bf16 W2 in shared memory (A operand of S2/S5 as MN-major, of S3 as
+// K-major) once per mini-batch.  The "+1" bias terms of the causal matrices,
+// the biases and GELU are applied in fp32 registers by the epilogue; the
+// 16 x 16 products Q K^T and Hq Hk^T (below tcgen05's M range) are computed
+// by two helper warps with mma.sync.
+//
+// One unit per CTA.  Warps 0-3: epilogue (warp q reads TMEM lanes 32q..32q+31;
+// thread owns hidden rows h = 32q + lane and 128 + 32q + lane, and for the
+// d-sized stages feature j = 16q + lane, lane < 16); warp 4 TMA producer;
+// warp 5 MMA issuer; warps 6-7 helpers.  Every wait is bounded; on expiry
+// the kernel records kStatusTimeout, drains what it issued and returns.
+#pragma once
+#include "common.cuh"
+#include "linear_tc.cuh"
+#include "ptx.cuh"
+
+namespace ttt {
+namespace mtc {
+
+using ltc::ld_bf16;
+using ltc::ldsm_x4;
+using ltc::mma_16816;
+using ltc::nosw_off;
+using ltc::sw128_off;
+using ltc::tmem_st_32x32b_x32;
+using ltc::tmem_st_32x32b_x8;
+using ltc::umma_ts;
+
+constexpr int kD = 64, kM = 256, kTok = 16;
+constexpr int kStages = 4;
+constexpr int kThreads = 256;
+constexpr int kTile = kTok * kD * 2;   // 2048
+
+// stage layout
+constexpr int kOffK = 0;               // [K | Q]: B operand of S1 (N = 32)
+constexpr int kOffQ = kTile;
+constexpr int kOffV = 2 * kTile;
+constexpr int kOffS1 = 3 * kTile;      // bf16 16 x 16 tril(Q K^T), K-major no swizzle
+constexpr int kOffEta = kOffS1 + 512;
+constexpr int kStageBytes = 7168;
+
+constexpr int kOffStages = 0;
+constexpr int kOffW2 = 28672;          // bf16 W2 [h][j], 128B swizzle, 256 rows (32 KB)
+constexpr int kOffHk = kOffW2 + 32768; // bf16 Hk [t][h]: 4 K-major sub-tiles of 16 x 64 (8 KB)
+constexpr int kOffHq = kOffHk + 8192;  // bf16 Hq [t][h] (8 KB)
+constexpr int kOffE = kOffHq + 8192;   // bf16 E [t][j], 128B swizzle (2 KB)
+constexpr int kOffAE = kOffE + 2048;   // bf16 (-eta E)^T [j][t], K-major no swizzle (2 KB)
+constexpr int kOffS2 = kOffAE + 2048;  // bf16 tril(Hq Hk^T), K-major no swizzle (512 B)
+constexpr int kOffBar = kOffS2 + 512;
+constexpr int kNumBars = 3 * kStages + 14;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmemBytes = kOffMisc + 64;
+
+// TMEM columns (M = 128 tiles: lane = hidden row mod 128; M = 64 stages use
+// lanes 0-15 of each 32-lane quadrant)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t cW1 = 0;     // fp32 W1^T, tile t at 64 t
+constexpr uint32_t cW2 = 128;   // fp32 W2, tile t at 128 + 64 t
+constexpr uint32_t cA = 256;    // fp32 [A | Aq], tile t at 256 + 32 t
+constexpr uint32_t cG = 320;    // fp32 G^T, tile t at 320 + 16 t
+constexpr uint32_t cE = 352;    // fp32 E0^T (M = 64)
+constexpr uint32_t cZ = 368;    // fp32 Z0^T (M = 64)
+constexpr uint32_t cAW1 = 384;  // bf16 W1^T (A of S1), tile t at 384 + 32 t
+constexpr uint32_t cAD1 = 448;  // bf16 (-eta D1)^T, tile t at 448 + 8 t
+constexpr uint32_t cAHk = 464;  // bf16 (-eta Hk)^T, tile t at 464 + 8 t
+
+struct Params {
+    int H, T, nsteps, per_seq;
+    const float* eta;
+    float eta_const;
+    const float* W1;
+    const float* c1;
+    const float* W2;
+    const float* c2;
+    __nv_bfloat16* Z;
+    float* W1_out;
+    float* c1_out;
+    float* W2_out;
+    float* c2_out;
+    int* status;
+    unsigned long long wait_ns;
+    unsigned flags;
+};
+
+__device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b_x16(taddr, r); }
+
+// 16 x 16 tril(X Y^T) with X, Y stored as [t][k] K-major 128B-swizzled
+// sub-tiles of 64 columns (nsub of them); n-tile nt (8 columns) only.
+__device__ __forceinline__ void tril_product(uint32_t xbase, uint32_t ybase, int nsub, int nt, int lane,
+                                             uint8_t* dst) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int arow = (lane & 7) + 8 * ((lane >> 3) & 1);
+    const int brow = 8 * nt + (lane & 7);
+    for (int sub = 0; sub < nsub; ++sub) {
+        const uint32_t xs = xbase + 2048 * sub, ys = ybase + 2048 * sub;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a[4], b[4];
+            const int ach = 2 * ks + (lane >> 4);
+            ldsm_x4(xs + arow * 128 + ((ach ^ (arow & 7)) << 4), a);
+            // matrices: (rows 8nt.., chunk 2ks), (.., 2ks+1) twice (x4 keeps the code uniform)
+            const int bch = 2 * ks + ((lane >> 3) & 1);
+            ldsm_x4(ys + brow * 128 + ((bch ^ (brow & 7)) << 4), b);
+            mma_16816(acc, a, b[0], b[1]);
+        }
+    }
+    const int r0 = lane >> 2, c0 = 2 * (lane & 3);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int t = r0 + 8 * hh, s = 8 * nt + c0;
+        *reinterpret_cast<uint32_t*>(dst + nosw_off(t, s)) =
+            pack_bf16x2(s <= t ? acc[2 * hh] : 0.f, s + 1 <= t ? acc[2 * hh + 1] : 0.f);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    mlp_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, Params p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicOr(p.status, kStatusBadSmem);
+        return;
+    }
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* full = bars;                    // [kStages] TMA landed
+    uint64_t* empty = bars + kStages;         // [kStages] MMA (after S4) + 4 epilogue warps (after E2)
+    uint64_t* aux1 = bars + 2 * kStages;      // [kStages] tril(Q K^T) written (helper warp 6)
+    uint64_t* d_a = bars + 3 * kStages;       // S1 done
+    uint64_t* d_e = d_a + 1;                  // S2 done
+    uint64_t* d_g = d_a + 2;                  // S3 done
+    uint64_t* d_u = d_a + 3;                  // S4 done
+    uint64_t* d_z = d_a + 4;                  // S5 done
+    uint64_t* hk_rdy = d_a + 5;               // Hk^T, (-eta Hk)^T written (4 epilogue warps)
+    uint64_t* e_rdy = d_a + 6;                // E, (-eta E)^T written
+    uint64_t* d1_rdy = d_a + 7;               // (-eta D1)^T written
+    uint64_t* hq_rdy = d_a + 8;               // Hq^T written
+    uint64_t* aux2 = d_a + 9;                 // tril(Hq Hk^T) written (2 helper warps)
+    uint64_t* aw1_rdy = d_a + 10;             // bf16 W1^T refreshed
+    uint64_t* w2_rdy = d_a + 11;              // bf16 W2 refreshed
+    uint64_t* drain = d_a + 12;
+    uint64_t* stall = d_a + 13;
+    uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffMisc);
+    volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int unit = blockIdx.x;
+    const int nsteps = p.nsteps;
+    const uint64_t lim = p.wait_ns;
+
+    if (tid == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 5);
+            mbar_init(&aux1[s], 1);
+        }
+        for (uint64_t* b = d_a; b <= d_z; ++b) mbar_init(b, 1);
+        mbar_init(hk_rdy, 4);
+        mbar_init(e_rdy, 4);
+        mbar_init(d1_rdy, 4);
+        mbar_init(hq_rdy, 4);
+        mbar_init(aux2, 2);
+        mbar_init(aw1_rdy, 4);
+        mbar_init(w2_rdy, 4);
+        mbar_init(drain, 1);
+        mbar_init(stall, 1);
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(s_tmem, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *s_tmem;
+    auto fail = [&]() {
+        *s_abort = 1;
+        atomicOr(p.status, kStatusTimeout);
+    };
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int issued_last = -1;
+            prefetch_tmap(&tmQ);
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            const uint32_t bytes = 3 * kTile + (p.eta ? 64 : 0);
+            for (int i = 0; i < nsteps; ++i) {
+                const int s = i % kStages;
+                if (i >= kStages && !wait_bounded(&empty[s], ((i / kStages) - 1) & 1, lim, s_abort)) {
+                    fail();
+                    break;
+                }
+                if (*s_abort) break;
+                uint8_t* st = smem + kOffStages + s * kStageBytes;
+                mbar_arrive_expect_tx(&full[s], bytes);
+                const int y = unit * p.T + i * kTok;
+                tma_load_2d(st + kOffK, &tmK, 0, y, &full[s]);
+                tma_load_2d(st + kOffQ, &tmQ, 0, y, &full[s]);
+                tma_load_2d(st + kOffV, &tmV, 0, y, &full[s]);
+                if (p.eta) bulk_load(st + kOffEta, p.eta + (size_t)y, 64, &full[s]);
+                issued_last = i;
+            }
+            for (int i = issued_last - kStages + 1; i <= issued_last; ++i) {
+                if (i < 0) continue;
+                if (!wait_bounded(&full[i % kStages], (i / kStages) & 1, lim, nullptr)) fail();
+            }
+        }
+    } else if (warp == 5) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idS1 = make_idesc_bf16(128, 32, 0, 0);
+            const uint32_t idS2 = make_idesc_bf16(64, 16, 1, 0);   // A = W2 as MN-major
+            const uint32_t idS3 = make_idesc_bf16(128, 16, 0, 0);
+            const uint32_t idUpd = make_idesc_bf16(128, 64, 0, 1); // B MN-major (K or E tile)
+            const uint32_t idAq = make_idesc_bf16(128, 16, 0, 0);
+            const uint32_t idZc = make_idesc_bf16(64, 16, 0, 0);
+            const uint32_t w2 = smem_u32(smem + kOffW2), hk = smem_u32(smem + kOffHk), hq = smem_u32(smem + kOffHq);
+            const uint32_t et = smem_u32(smem + kOffE), ae = smem_u32(smem + kOffAE), s2 = smem_u32(smem + kOffS2);
+            bool ok = true;
+            if (p.flags & TTT_FLAG_TEST_STALL) {
+                if (!wait_bounded(stall, 0, lim, s_abort)) fail();
+                ok = false;
+            }
+            auto W = [&](uint64_t* b, uint32_t par) {
+                if (!wait_bounded(b, par, lim, s_abort)) {
+                    fail();
+                    ok = false;
+                }
+                return ok;
+            };
+            for (int i = 0; ok && i < nsteps; ++i) {
+                const int s = i % kStages;
+                const uint32_t par = (i / kStages) & 1, ip = i & 1;
+                const uint32_t st = smem_u32(smem + kOffStages + s * kStageBytes);
+                // S1
+                if (!W(&full[s], par) || !W(aw1_rdy, ip)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_ts(tbase + cA + 32 * tt, tbase + cAW1 + 32 * tt + 8 * ks,
+                                make_sdesc(st + kOffK + 32 * ks, 16, 1024, kSwizzle128B), idS1, ks > 0);
+                umma_commit(d_a);
+                // S2
+                if (!W(hk_rdy, ip) || !W(w2_rdy, ip)) break;
+                tc_fence_after();
+                for (int ks = 0; ks < 16; ++ks)
+                    umma_bf16(tbase + cE, make_sdesc(w2 + 2048 * ks, 1024, 1024, kSwizzle128B),
+                              make_sdesc(hk + 2048 * (ks >> 2) + 32 * (ks & 3), 16, 1024, kSwizzle128B), idS2, ks > 0);
+                umma_commit(d_e);
+                // S3
+                if (!W(e_rdy, ip)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        umma_bf16(tbase + cG + 16 * tt, make_sdesc(w2 + 16384 * tt + 32 * ks, 16, 1024, kSwizzle128B),
+                                  make_sdesc(et + 32 * ks, 16, 1024, kSwizzle128B), idS3, ks > 0);
+                umma_commit(d_g);
+                // S4
+                if (!W(d1_rdy, ip) || !W(&aux1[s], par)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    umma_ts(tbase + cW1 + 64 * tt, tbase + cAD1 + 8 * tt,
+                            make_sdesc(st + kOffK, 1024, 1024, kSwizzle128B), idUpd, 1);
+                    umma_ts(tbase + cA + 32 * tt + 16, tbase + cAD1 + 8 * tt,
+                            make_sdesc(st + kOffS1, 128, 256, kSwizzleNone), idAq, 1);
+                    umma_ts(tbase + cW2 + 64 * tt, tbase + cAHk + 8 * tt, make_sdesc(et, 1024, 1024, kSwizzle128B),
+                            idUpd, 1);
+                }
+                umma_commit(d_u);
+                umma_commit(&empty[s]);
+                // S5
+                if (!W(hq_rdy, ip) || !W(aux2, ip)) break;
+                tc_fence_after();
+                for (int ks = 0; ks < 16; ++ks)
+                    umma_bf16(tbase + cZ, make_sdesc(w2 + 2048 * ks, 1024, 1024, kSwizzle128B),
+                              make_sdesc(hq + 2048 * (ks >> 2) + 32 * (ks & 3), 16, 1024, kSwizzle128B), idS2, ks > 0);
+                umma_bf16(tbase + cZ, make_sdesc(ae, 128, 256, kSwizzleNone), make_sdesc(s2, 128, 256, kSwizzleNone),
+                          idZc, 1);
+                umma_commit(d_z);
+            }
+            umma_commit(drain);
+            if (!wait_bounded(drain, 0, lim, nullptr)) fail();
+        }
+    } else if (warp >= 6) {
+        // ------------------------------------------------------------ helpers
+        const int hw = warp - 6;
+        for (int i = 0; i < nsteps; ++i) {
+            const int s = i % kStages;
+            uint8_t* st = smem + kOffStages + s * kStageBytes;
+            if (hw == 0) {
+                // tril(Q K^T) of this batch (both n-tiles)
+                if (!wait_bounded(&full[s], (i / kStages) & 1, lim, s_abort)) {
+                    if (lane == 0) fail();
+                    break;
+                }
+                tril_product(smem_u32(st + kOffQ), smem_u32(st + kOffK), 1, 0, lane, st + kOffS1);
+                tril_product(smem_u32(st + kOffQ), smem_u32(st + kOffK), 1, 1, lane, st + kOffS1);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&aux1[s]);
+            }
+            // tril(Hq Hk^T): n-tile hw
+            if (!wait_bounded(hq_rdy, i & 1, lim, s_abort)) {
+                if (lane == 0) fail();
+                break;
+            }
+            tril_product(smem_u32(smem + kOffHq), smem_u32(smem + kOffHk), 4, hw, lane, smem + kOffS2);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(aux2);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int q = warp;
+        const int hr[2] = {32 * q + lane, 128 + 32 * q + lane};   // hidden rows of this thread
+        const bool jl = lane < 16;                                // owns a feature row in d-sized stages
+        const int j = 16 * q + (lane & 15);
+        const int pu = p.per_seq ? unit : unit % p.H;
+        const uint32_t tl = tbase + ((uint32_t)(32 * q) << 16);
+        uint8_t* w2s = smem + kOffW2;
+        uint8_t* hks = smem + kOffHk;
+        uint8_t* hqs = smem + kOffHq;
+        uint8_t* es = smem + kOffE;
+        uint8_t* aes = smem + kOffAE;
+        float c1[2], c2 = 0.f;
+        // initial state
+        {
+            const float* W1u = p.W1 + (size_t)pu * kD * kM;
+            const float* W2u = p.W2 + (size_t)pu * kM * kD;
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                const int h = hr[tt];
+                c1[tt] = p.c1 ? p.c1[(size_t)pu * kM + h] : 0.f;
+                uint32_t w[32], pk[16];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(W1u[(size_t)(32 * half + i) * kM + h]);
+                    tmem_st_32x32b_x32(tl + cW1 + 64 * tt + 32 * half, w);
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        pk[c] = pack_bf16x2(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+                    tmem_st_32x32b_x16(tl + cAW1 + 32 * tt + 16 * half, pk);
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(W2u[(size_t)h * kD + 32 * half + i]);
+                    tmem_st_32x32b_x32(tl + cW2 + 64 * tt + 32 * half, w);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(w[8 * c + 0]), __uint_as_float(w[8 * c + 1]));
+                        v.y = pack_bf16x2(__uint_as_float(w[8 * c + 2]), __uint_as_float(w[8 * c + 3]));
+                        v.z = pack_bf16x2(__uint_as_float(w[8 * c + 4]), __uint_as_float(w[8 * c + 5]));
+                        v.w = pack_bf16x2(__uint_as_float(w[8 * c + 6]), __uint_as_float(w[8 * c + 7]));
+                        const int ch = 4 * half + c;
+                        *reinterpret_cast<uint4*>(w2s + (h >> 3) * 1024 + (h & 7) * 128 + ((ch ^ (h & 7)) << 4)) = v;
+                    }
+                }
+            }
+            if (jl) c2 = p.c2 ? p.c2[(size_t)pu * kD + j] : 0.f;
+        }
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(aw1_rdy);
+            mbar_arrive(w2_rdy);
+        }
+        bool dead = false;
+        auto WT = [&](uint64_t* b, uint32_t par) {
+            if (!dead && !wait_bounded(b, par, lim, s_abort)) {
+                dead = true;
+                fail();
+            }
+        };
+        __nv_bfloat16* Zu = p.Z + (size_t)unit * p.T * kD + j;
+        for (int i = 0; i < nsteps; ++i) {
+            const int s = i % kStages;
+            const uint32_t par = (i / kStages) & 1, ip = i & 1;
+            const uint8_t* st = smem + kOffStages + s * kStageBytes;
+            WT(&full[s], par);
+            float et[16];
+            {
+                const float* etas = reinterpret_cast<const float*>(st + kOffEta);
+#pragma unroll
+                for (int t = 0; t < 16; ++t) et[t] = p.eta ? etas[t] : p.eta_const;
+            }
+            // E1: A -> Hk, GELU'(A); keep Aq0
+            WT(d_a, ip);
+            tc_fence_after();
+            float gp[2][16];
+            {
+                uint32_t ra[2][32];
+                tmem_ld_32x32b_x32(tl + cA, ra[0]);
+                tmem_ld_32x32b_x32(tl + cA + 32, ra[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    const int h = hr[tt];
+                    uint8_t* sub = hks + 2048 * (h >> 6);
+                    float ah[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        const float a = __uint_as_float(ra[tt][t]) + c1[tt];
+                        const float hk = gelu_f(a);
+                        gp[tt][t] = gelu_grad_f(a);
+                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(t, h & 63)) = __float2bfloat16_rn(hk);
+                        ah[t] = -et[t] * hk;
+                    }
+                    uint32_t pa[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) pa[c] = pack_bf16x2(ah[2 * c], ah[2 * c + 1]);
+                    tmem_st_32x32b_x8(tl + cAHk + 8 * tt, pa);
+                }
+            }
+            fence_proxy_async_smem();
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(hk_rdy);
+            // E2: E = E0 + c2 - V -> E tile, (-eta E)^T; c2 update
+            WT(d_e, ip);
+            tc_fence_after();
+            float zb[16];   // c2 before the update + sum_{s<=t} (-eta_s e_s): the Z bias and "+1" term
+            {
+                uint32_t re[16];
+                tmem_ld_x16(tl + cE, re);
+                tmem_wait_ld();
+                if (jl) {
+                    const uint8_t* vt = st + kOffV;
+                    float ae[16], pre = c2;
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        const float e = __uint_as_float(re[t]) + c2 - ld_bf16(vt, sw128_off(t, j));
+                        *reinterpret_cast<__nv_bfloat16*>(es + sw128_off(t, j)) = __float2bfloat16_rn(e);
+                        ae[t] = -et[t] * e;
+                        pre += ae[t];
+                        zb[t] = pre;
+                    }
+                    c2 = pre;
+                    uint4 v0, v1;
+                    v0.x = pack_bf16x2(ae[0], ae[1]);
+                    v0.y = pack_bf16x2(ae[2], ae[3]);
+                    v0.z = pack_bf16x2(ae[4], ae[5]);
+                    v0.w = pack_bf16x2(ae[6], ae[7]);
+                    v1.x = pack_bf16x2(ae[8], ae[9]);
+                    v1.y = pack_bf16x2(ae[10], ae[11]);
+                    v1.z = pack_bf16x2(ae[12], ae[13]);
+                    v1.w = pack_bf16x2(ae[14], ae[15]);
+                    *reinterpret_cast<uint4*>(aes + nosw_off(j, 0)) = v0;
+                    *reinterpret_cast<uint4*>(aes + nosw_off(j, 8)) = v1;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(e_rdy);
+                mbar_arrive(&empty[s]);
+            }
+            // E3: D1 = G * GELU'(A) -> (-eta D1)^T; c1 update
+            WT(d_g, ip);
+            tc_fence_after();
+            float aqb[2][16];   // c1 before the update + sum_{s<=t} (-eta_s d1_s)
+            {
+                uint32_t rg[2][16];
+                tmem_ld_x16(tl + cG, rg[0]);
+                tmem_ld_x16(tl + cG + 16, rg[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    float ad[16], pre = c1[tt];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        ad[t] = -et[t] * __uint_as_float(rg[tt][t]) * gp[tt][t];
+                        pre += ad[t];
+                        aqb[tt][t] = pre;
+                    }
+                    c1[tt] = pre;
+                    uint32_t pa[8];
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) pa[c] = pack_bf16x2(ad[2 * c], ad[2 * c + 1]);
+                    tmem_st_32x32b_x8(tl + cAD1 + 8 * tt, pa);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(d1_rdy);
+            // E4: Hq = GELU(Aq) -> Hq^T; refresh bf16 W1^T
+            WT(d_u, ip);
+            tc_fence_after();
+            {
+                uint32_t rq[2][16];
+                tmem_ld_x16(tl + cA + 16, rq[0]);
+                tmem_ld_x16(tl + cA + 32 + 16, rq[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    const int h = hr[tt];
+                    uint8_t* sub = hqs + 2048 * (h >> 6);
+#pragma unroll
+                    for (int t = 0; t < 16; ++t)
+                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(t, h & 63)) =
+                            __float2bfloat16_rn(gelu_f(__uint_as_float(rq[tt][t]) + aqb[tt][t]));
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(hq_rdy);
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t w[32], pk[16];
+                    tmem_ld_32x32b_x32(tl + cW1 + 64 * tt + 32 * half, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 16; ++c)
+                        pk[c] = pack_bf16x2(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
+                    tmem_st_32x32b_x16(tl + cAW1 + 32 * tt + 16 * half, pk);
+                }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(aw1_rdy);
+            // E5: Z = Z0 + zb -> global; refresh bf16 W2 (S5 has finished reading it)
+            WT(d_z, ip);
+            tc_fence_after();
+            {
+                uint32_t rz[16];
+                tmem_ld_x16(tl + cZ, rz);
+                tmem_wait_ld();
+                if (jl && !dead) {
+#pragma unroll
+                    for (int t = 0; t < 16; ++t)
+                        Zu[(size_t)(i * kTok + t) * kD] = __float2bfloat16_rn(__uint_as_float(rz[t]) + zb[t]);
+                }
+            }
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                const int h = hr[tt];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t w[32];
+                    tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * half, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(w[8 * c + 0]), __uint_as_float(w[8 * c + 1]));
+                        v.y = pack_bf16x2(__uint_as_float(w[8 * c + 2]), __uint_as_float(w[8 * c + 3]));
+                        v.z = pack_bf16x2(__uint_as_float(w[8 * c + 4]), __uint_as_float(w[8 * c + 5]));
+                        v.w = pack_bf16x2(__uint_as_float(w[8 * c + 6]), __uint_as_float(w[8 * c + 7]));
+                        const int ch = 4 * half + c;
+                        *reinterpret_cast<uint4*>(w2s + (h >> 3) * 1024 + (h & 7) * 128 + ((ch ^ (h & 7)) << 4)) = v;
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(w2_rdy);
+        }
+        // final state (after the last S4; W1^T / W2 accumulators in TMEM)
+        if (!dead) {
+            float* W1o = p.W1_out + (size_t)unit * kD * kM;
+            float* W2o = p.W2_out + (size_t)unit * kM * kD;
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                const int h = hr[tt];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t w[32];
+                    tmem_ld_32x32b_x32(tl + cW1 + 64 * tt + 32 * half, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) W1o[(size_t)(32 * half + i) * kM + h] = __uint_as_float(w[i]);
+                    tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * half, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) W2o[(size_t)h * kD + 32 * half + i] = __uint_as_float(w[i]);
+                }
+                if (p.c1_out) p.c1_out[(size_t)unit * kM + h] = c1[tt];
+            }
+            if (jl && p.c2_out) p.c2_out[(size_t)unit * kD + j] = c2;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tbase, kTmemCols);
+    }
+}
+
+}  // namespace mtc
+}  // namespace ttt

@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "linear_tc.cuh"
+#include "mlp_tc.cuh"
 #include "simt.cuh"
 #include "tmap.h"
 
@@ -231,6 +232,45 @@ ttt_status simt_mlp_dtype(const ttt_mlp_args* a, cudaStream_t st) {
 }  // namespace
 }  // namespace ttt
 
+namespace ttt {
+namespace {
+ttt_status tc_mlp(const ttt_mlp_args* a, cudaStream_t st) {
+    using namespace mtc;
+    const long long U = (long long)a->B * a->H;
+    const long long rows = U * a->T;
+    CUtensorMap mQ, mK, mV;
+    const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!encode_2d(&mQ, a->Q, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&mK, a->K, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !encode_2d(&mV, a->V, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B))
+        return TTT_ERR_CUDA;
+    Params p;
+    p.H = a->H;
+    p.T = a->T;
+    p.nsteps = a->T / kTok;
+    p.per_seq = a->params_per_sequence;
+    p.eta = a->eta;
+    p.eta_const = a->eta_const;
+    p.W1 = a->W1;
+    p.c1 = a->c1;
+    p.W2 = a->W2;
+    p.c2 = a->c2;
+    p.Z = static_cast<__nv_bfloat16*>(a->Z);
+    p.W1_out = a->W1_out;
+    p.c1_out = a->c1_out;
+    p.W2_out = a->W2_out;
+    p.c2_out = a->c2_out;
+    p.status = status_ptr();
+    p.wait_ns = wait_ns(a->wait_timeout_ms);
+    p.flags = a->flags;
+    if (!p.status) return TTT_ERR_CUDA;
+    if (!set_smem(mlp_tc_kernel, kSmemBytes)) return TTT_ERR_CUDA;
+    mlp_tc_kernel<<<(int)U, kThreads, kSmemBytes, st>>>(mQ, mK, mV, p);
+    return launch_status();
+}
+}  // namespace
+}  // namespace ttt
+
 extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream) {
     if (!a) return TTT_ERR_INVALID_ARG;
     ttt_status v = validate_common(a->B, a->H, a->T, a->d, a->b, a->io_dtype);
@@ -245,6 +285,9 @@ extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream
         return TTT_ERR_INVALID_ARG;
     if (a->params_per_sequence != 0 && a->params_per_sequence != 1) return TTT_ERR_INVALID_ARG;
     if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL)) return TTT_ERR_INVALID_ARG;
+    const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
+                    !(a->flags & TTT_FLAG_FORCE_SIMT);
+    if (tc) return tc_mlp(a, stream);
     if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
     switch (a->d) {
         case 16: return simt_mlp_dtype<16>(a, stream);

@@ -196,6 +196,25 @@ def test_mlp_d64_bf16(ttt_lib, B, H, T):
     check_mlp(ttt_lib, inp)
 
 
+def test_mlp_tc_matches_simt(ttt_lib):
+    """The tensor-core and the fp32 CUDA-core MLP kernels agree on the same inputs."""
+    inp = WL.random_case("mlp", 1, 3, 96, 64, 16, io_dtype=WL.BF16, eta_mode="const", eta_const=1 / 64, seed=41)
+    a = run_mlp(ttt_lib, inp)
+    b = run_mlp(ttt_lib, inp, flags=ttt_lib.FLAG_FORCE_SIMT)
+    for x, y in zip(a, b):
+        assert normwise(x, y) < 1e-2
+
+
+def test_mlp_tc_sigmoid_eta_and_biases(ttt_lib):
+    """Per-token eta and non-zero initial biases through the tensor-core MLP kernel."""
+    inp = WL.random_case("mlp", 2, 2, 64, 64, 16, io_dtype=WL.BF16, eta_mode="sigmoid", seed=43)
+    rng = np.random.default_rng(5)
+    for nm, shape in (("c1", (2, 256)), ("c2", (2, 64))):
+        raw, ex = WL.store(rng.standard_normal(shape) * 0.1, WL.F32)
+        inp.raw[nm], inp.exact[nm] = raw, ex
+    check_mlp(ttt_lib, inp)
+
+
 # ---------------------------------------------------------------------------
 # decode
 # ---------------------------------------------------------------------------
