@@ -26,6 +26,10 @@
 // 16 x 16 products Q K^T and Hq Hk^T (below tcgen05's M range) are computed
 // by two helper warps with mma.sync.
 //
+// The output path of a mini-batch (Hq, S5, Z) is software-pipelined behind
+// the next mini-batch's S1/E1: bf16 W2, Hk and Hq are double-buffered so S5
+// of batch i reads the state of batch i while S2 of batch i+1 reads the next.
+//
 // One unit per CTA.  Warps 0-3: epilogue (warp q reads TMEM lanes 32q..32q+31;
 // thread owns hidden rows h = 32q + lane and 128 + 32q + lane, and for the
 // d-sized stages feature j = 16q + lane, lane < 16); warp 4 TMA producer;
@@ -62,10 +66,10 @@ constexpr int kOffEta = kOffS1 + 512;
 constexpr int kStageBytes = 7168;
 
 constexpr int kOffStages = 0;
-constexpr int kOffW2 = 28672;          // bf16 W2 [h][j], 128B swizzle, 256 rows (32 KB)
-constexpr int kOffHk = kOffW2 + 32768; // bf16 Hk [t][h]: 4 K-major sub-tiles of 16 x 64 (8 KB)
-constexpr int kOffHq = kOffHk + 8192;  // bf16 Hq [t][h] (8 KB)
-constexpr int kOffE = kOffHq + 8192;   // bf16 E [t][j], 128B swizzle (2 KB)
+constexpr int kOffW2 = 28672;          // 2 x bf16 W2 [h][j], 128B swizzle, 256 rows (32 KB each)
+constexpr int kOffHk = kOffW2 + 65536; // 2 x bf16 Hk [t][h]: 4 K-major sub-tiles of 16 x 64 (8 KB each)
+constexpr int kOffHq = kOffHk + 16384; // 2 x bf16 Hq [t][h] (8 KB each)
+constexpr int kOffE = kOffHq + 16384;  // bf16 E [t][j], 128B swizzle (2 KB)
 constexpr int kOffAE = kOffE + 2048;   // bf16 (-eta E)^T [j][t], K-major no swizzle (2 KB)
 constexpr int kOffS2 = kOffAE + 2048;  // bf16 tril(Hq Hk^T), K-major no swizzle (512 B)
 constexpr int kOffBar = kOffS2 + 512;
@@ -253,10 +257,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 return ok;
             };
+            // S5 of batch i2: Z0^T = W2_i2^T Hq_i2^T + (-eta E_i2)^T tril(Hq Hk^T)^T
+            auto issue_s5 = [&](int i2) {
+                if (!W(hq_rdy, i2 & 1) || !W(aux2, i2 & 1)) return false;
+                tc_fence_after();
+                const uint32_t w2b = w2 + 32768 * (i2 & 1), hqb = hq + 8192 * (i2 & 1);
+                for (int ks = 0; ks < 16; ++ks)
+                    umma_bf16(tbase + cZ, make_sdesc(w2b + 2048 * ks, 1024, 1024, kSwizzle128B),
+                              make_sdesc(hqb + 2048 * (ks >> 2) + 32 * (ks & 3), 16, 1024, kSwizzle128B), idS2,
+                              ks > 0);
+                umma_bf16(tbase + cZ, make_sdesc(ae, 128, 256, kSwizzleNone), make_sdesc(s2, 128, 256, kSwizzleNone),
+                          idZc, 1);
+                umma_commit(d_z);
+                return true;
+            };
             for (int i = 0; ok && i < nsteps; ++i) {
                 const int s = i % kStages;
                 const uint32_t par = (i / kStages) & 1, ip = i & 1;
                 const uint32_t st = smem_u32(smem + kOffStages + s * kStageBytes);
+                const uint32_t w2b = w2 + 32768 * ip, hkb = hk + 8192 * ip;
                 // S1
                 if (!W(&full[s], par) || !W(aw1_rdy, ip)) break;
                 tc_fence_after();
@@ -267,12 +286,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                         umma_ts(tbase + cA + 32 * tt, tbase + cAW1 + 32 * tt + 8 * ks,
                                 make_sdesc(st + kOffK + 32 * ks, 16, 1024, kSwizzle128B), idS1, ks > 0);
                 umma_commit(d_a);
+                // the previous batch's output path runs while E1 of this batch does
+                if (i >= 1 && !issue_s5(i - 1)) break;
                 // S2
                 if (!W(hk_rdy, ip) || !W(w2_rdy, ip)) break;
                 tc_fence_after();
                 for (int ks = 0; ks < 16; ++ks)
-                    umma_bf16(tbase + cE, make_sdesc(w2 + 2048 * ks, 1024, 1024, kSwizzle128B),
-                              make_sdesc(hk + 2048 * (ks >> 2) + 32 * (ks & 3), 16, 1024, kSwizzle128B), idS2, ks > 0);
+                    umma_bf16(tbase + cE, make_sdesc(w2b + 2048 * ks, 1024, 1024, kSwizzle128B),
+                              make_sdesc(hkb + 2048 * (ks >> 2) + 32 * (ks & 3), 16, 1024, kSwizzle128B), idS2, ks > 0);
                 umma_commit(d_e);
                 // S3
                 if (!W(e_rdy, ip)) break;
@@ -281,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tbase + cG + 16 * tt, make_sdesc(w2 + 16384 * tt + 32 * ks, 16, 1024, kSwizzle128B),
+                        umma_bf16(tbase + cG + 16 * tt, make_sdesc(w2b + 16384 * tt + 32 * ks, 16, 1024, kSwizzle128B),
                                   make_sdesc(et + 32 * ks, 16, 1024, kSwizzle128B), idS3, ks > 0);
                 umma_commit(d_g);
                 // S4
@@ -298,16 +319,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 umma_commit(d_u);
                 umma_commit(&empty[s]);
-                // S5
-                if (!W(hq_rdy, ip) || !W(aux2, ip)) break;
-                tc_fence_after();
-                for (int ks = 0; ks < 16; ++ks)
-                    umma_bf16(tbase + cZ, make_sdesc(w2 + 2048 * ks, 1024, 1024, kSwizzle128B),
-                              make_sdesc(hq + 2048 * (ks >> 2) + 32 * (ks & 3), 16, 1024, kSwizzle128B), idS2, ks > 0);
-                umma_bf16(tbase + cZ, make_sdesc(ae, 128, 256, kSwizzleNone), make_sdesc(s2, 128, 256, kSwizzleNone),
-                          idZc, 1);
-                umma_commit(d_z);
             }
+            if (ok && nsteps >= 1) issue_s5(nsteps - 1);
             umma_commit(drain);
             if (!wait_bounded(drain, 0, lim, nullptr)) fail();
         }
@@ -334,7 +347,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) fail();
                 break;
             }
-            tril_product(smem_u32(smem + kOffHq), smem_u32(smem + kOffHk), 4, hw, lane, smem + kOffS2);
+            tril_product(smem_u32(smem + kOffHq + 8192 * (i & 1)), smem_u32(smem + kOffHk + 8192 * (i & 1)), 4, hw,
+                         lane, smem + kOffS2);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(aux2);
@@ -407,6 +421,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         __nv_bfloat16* Zu = p.Z + (size_t)unit * p.T * kD + j;
+        // bf16 W2 (state after batch i's update) -> buffer (i+1)&1, row h of each tile
+        auto refresh_w2 = [&](int buf) {
+            uint8_t* dst = w2s + 32768 * buf;
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                const int h = hr[tt];
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t w[32];
+                    tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * half, w);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint4 v;
+                        v.x = pack_bf16x2(__uint_as_float(w[8 * c + 0]), __uint_as_float(w[8 * c + 1]));
+                        v.y = pack_bf16x2(__uint_as_float(w[8 * c + 2]), __uint_as_float(w[8 * c + 3]));
+                        v.z = pack_bf16x2(__uint_as_float(w[8 * c + 4]), __uint_as_float(w[8 * c + 5]));
+                        v.w = pack_bf16x2(__uint_as_float(w[8 * c + 6]), __uint_as_float(w[8 * c + 7]));
+                        const int ch = 4 * half + c;
+                        *reinterpret_cast<uint4*>(dst + (h >> 3) * 1024 + (h & 7) * 128 + ((ch ^ (h & 7)) << 4)) = v;
+                    }
+                }
+            }
+        };
+        float zb[16];   // c2 before the update + sum_{s<=t} (-eta_s e_s): the Z bias and "+1" term
+        // E5 of batch i2: Z = Z0 + zb -> global
+        auto finish_z = [&](int i2) {
+            WT(d_z, i2 & 1);
+            tc_fence_after();
+            uint32_t rz[16];
+            tmem_ld_x16(tl + cZ, rz);
+            tmem_wait_ld();
+            if (jl && !dead) {
+#pragma unroll
+                for (int t = 0; t < 16; ++t)
+                    Zu[(size_t)(i2 * kTok + t) * kD] = __float2bfloat16_rn(__uint_as_float(rz[t]) + zb[t]);
+            }
+        };
         for (int i = 0; i < nsteps; ++i) {
             const int s = i % kStages;
             const uint32_t par = (i / kStages) & 1, ip = i & 1;
@@ -427,10 +479,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_32x32b_x32(tl + cA, ra[0]);
                 tmem_ld_32x32b_x32(tl + cA + 32, ra[1]);
                 tmem_wait_ld();
+                uint8_t* hkb = hks + 8192 * ip;
 #pragma unroll
                 for (int tt = 0; tt < 2; ++tt) {
                     const int h = hr[tt];
-                    uint8_t* sub = hks + 2048 * (h >> 6);
+                    uint8_t* sub = hkb + 2048 * (h >> 6);
                     float ah[16];
 #pragma unroll
                     for (int t = 0; t < 16; ++t) {
@@ -451,10 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(hk_rdy);
+            // the previous batch's outputs, while S2 of this batch runs
+            if (i >= 1) finish_z(i - 1);
             // E2: E = E0 + c2 - V -> E tile, (-eta E)^T; c2 update
             WT(d_e, ip);
             tc_fence_after();
-            float zb[16];   // c2 before the update + sum_{s<=t} (-eta_s e_s): the Z bias and "+1" term
             {
                 uint32_t re[16];
                 tmem_ld_x16(tl + cE, re);
@@ -520,27 +574,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(d1_rdy);
-            // E4: Hq = GELU(Aq) -> Hq^T; refresh bf16 W1^T
+            // E4: bf16 W1^T for the next S1 first, then Hq = GELU(Aq) -> Hq^T, then bf16 W2
             WT(d_u, ip);
             tc_fence_after();
-            {
-                uint32_t rq[2][16];
-                tmem_ld_x16(tl + cA + 16, rq[0]);
-                tmem_ld_x16(tl + cA + 32 + 16, rq[1]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
-                    const int h = hr[tt];
-                    uint8_t* sub = hqs + 2048 * (h >> 6);
-#pragma unroll
-                    for (int t = 0; t < 16; ++t)
-                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(t, h & 63)) =
-                            __float2bfloat16_rn(gelu_f(__uint_as_float(rq[tt][t]) + aqb[tt][t]));
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(hq_rdy);
+            uint32_t rq[2][16];
+            tmem_ld_x16(tl + cA + 16, rq[0]);
+            tmem_ld_x16(tl + cA + 32 + 16, rq[1]);
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
@@ -557,44 +596,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(aw1_rdy);
-            // E5: Z = Z0 + zb -> global; refresh bf16 W2 (S5 has finished reading it)
-            WT(d_z, ip);
-            tc_fence_after();
             {
-                uint32_t rz[16];
-                tmem_ld_x16(tl + cZ, rz);
-                tmem_wait_ld();
-                if (jl && !dead) {
+                uint8_t* hqb = hqs + 8192 * ip;
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    const int h = hr[tt];
+                    uint8_t* sub = hqb + 2048 * (h >> 6);
 #pragma unroll
                     for (int t = 0; t < 16; ++t)
-                        Zu[(size_t)(i * kTok + t) * kD] = __float2bfloat16_rn(__uint_as_float(rz[t]) + zb[t]);
-                }
-            }
-#pragma unroll
-            for (int tt = 0; tt < 2; ++tt) {
-                const int h = hr[tt];
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t w[32];
-                    tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * half, w);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(w[8 * c + 0]), __uint_as_float(w[8 * c + 1]));
-                        v.y = pack_bf16x2(__uint_as_float(w[8 * c + 2]), __uint_as_float(w[8 * c + 3]));
-                        v.z = pack_bf16x2(__uint_as_float(w[8 * c + 4]), __uint_as_float(w[8 * c + 5]));
-                        v.w = pack_bf16x2(__uint_as_float(w[8 * c + 6]), __uint_as_float(w[8 * c + 7]));
-                        const int ch = 4 * half + c;
-                        *reinterpret_cast<uint4*>(w2s + (h >> 3) * 1024 + (h & 7) * 128 + ((ch ^ (h & 7)) << 4)) = v;
-                    }
+                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(t, h & 63)) =
+                            __float2bfloat16_rn(gelu_f(__uint_as_float(rq[tt][t]) + aqb[tt][t]));
                 }
             }
             fence_proxy_async_smem();
-            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(hq_rdy);
+            refresh_w2((i + 1) & 1);
+            fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(w2_rdy);
         }
+        if (nsteps >= 1) finish_z(nsteps - 1);
         // final state (after the last S4; W1^T / W2 accumulators in TMEM)
         if (!dead) {
             float* W1o = p.W1_out + (size_t)unit * kD * kM;

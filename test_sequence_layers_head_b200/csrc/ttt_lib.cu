@@ -302,15 +302,25 @@ extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream
 // ---------------------------------------------------------------------------
 namespace ttt {
 namespace {
+template <int D, typename IO>
+ttt_status launch_decode_t(const ttt_decode_args* a, cudaStream_t st) {
+    DecodeParams p{a->W, a->q, a->k, a->v, a->eta, a->eta_const, a->z};
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(a->B * a->H));
+    cfg.blockDim = dim3(D * 4);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, decode_kernel<D, IO>, p) != cudaSuccess) return launch_status();
+    return launch_status();
+}
 template <int D>
 ttt_status launch_decode(const ttt_decode_args* a, cudaStream_t st) {
-    DecodeParams p{a->W, a->q, a->k, a->v, a->eta, a->eta_const, a->z};
-    const int units = a->B * a->H;
-    if (a->io_dtype == TTT_F32)
-        decode_kernel<D, float><<<units, (D / 4) * (D / 4), 0, st>>>(p);
-    else
-        decode_kernel<D, __nv_bfloat16><<<units, (D / 4) * (D / 4), 0, st>>>(p);
-    return launch_status();
+    return a->io_dtype == TTT_F32 ? launch_decode_t<D, float>(a, st) : launch_decode_t<D, __nv_bfloat16>(a, st);
 }
 }  // namespace
 }  // namespace ttt
