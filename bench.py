@@ -78,6 +78,17 @@ def algorithmic_flops(w: WL.Workload) -> int:
     return w.units * w.T * per
 
 
+def dominant_kernel(w):
+    """(kernel name, source file under csrc/) of the one kernel a step of workload w launches."""
+    if w.io_dtype != WL.BF16 or w.d != 64 or w.b != 16:
+        return ("simt_mlp_kernel" if w.kind == "mlp" else "simt_linear_kernel"), "simt.cuh"
+    if w.kind == "mlp":
+        return "mlp_tc_kernel", "mlp_tc.cuh"
+    if w.kind == "ln":
+        return "linear_tc_kernel<1>", "linear_tc.cuh"
+    return "linear_frag_kernel", "linear_frag.cuh"
+
+
 def recorded_traffic(kernel: str, src: str):
     """DRAM bytes per launch recorded from an ncu capture in profiles/traffic.json,
     or None when the kernel source changed since the capture."""
@@ -404,12 +415,12 @@ def run_ours(args):
         achieved = abytes / (mean_launch / 1000.0) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                 "peak_source": peak_src}
-    roof.update({"kernel": "linear_tc_kernel" if w.kind != "mlp" else "mlp kernel",
+    kname, ksrc = dominant_kernel(w)
+    roof.update({"kernel": kname,
                  "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": aflops,
                  "mean_launch_ms": mean_launch,
                  "traffic": args.traffic if args.traffic is not None else (
-                     recorded_traffic("linear_tc_kernel", "linear_tc.cuh")
-                     if (w.kind == "linear" and w.name == DEFAULT_WORKLOAD and not args.T) else None)})
+                     recorded_traffic(kname, ksrc) if (w.name == DEFAULT_WORKLOAD and not args.T) else None)})
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.io_dtype == WL.BF16 else "f32",
