@@ -85,8 +85,8 @@ def dominant_kernel(w):
     if w.kind == "mlp":
         return "mlp_tc_kernel", "mlp_tc.cuh"
     if w.kind == "ln":
-        return "linear_tc_kernel<1>", "linear_tc.cuh"
-    return "linear_frag_kernel", "linear_frag.cuh"
+        return "linear_frag_kernel<1>", "linear_frag.cuh"
+    return "linear_frag_kernel<0>", "linear_frag.cuh"
 
 
 def recorded_traffic(kernel: str, src: str):

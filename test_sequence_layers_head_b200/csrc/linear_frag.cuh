@@ -1,6 +1,7 @@
-// Tensor-core persistent kernel of the plain TTT-Linear prefill (f(x) = x W),
-// d = 64, mini-batch b = 16, bf16 Q/K/V/Z, fp32 state.  Mini-batches are
-// processed in pairs, so that every tensor-core round trip serves two of them.
+// Tensor-core persistent kernel of the TTT-Linear prefill, plain (f(x) = x W)
+// and LN+residual (f(x) = x + LN(x W + c)), d = 64, mini-batch b = 16, bf16
+// Q/K/V/Z, fp32 state.  Mini-batches are processed in pairs, so that every
+// tensor-core round trip serves two of them.
 //
 // Method (paper digest "论文速览 | TTT", section 3.6, half-loss convention):
 // per (sequence, head) unit and mini-batch i of 16 tokens with batch-start
@@ -14,6 +15,16 @@
 //     W_{2g+2}^T = W^T + A_a K_a + A_b K_b
 // (W_b = W_a + A_a K_a substituted into E_b and Zq_b: an identity, not an
 // approximation.)
+// LN+residual (section 4.4): the pre-activation x = k W + c replaces k W, E
+// is replaced by the LN backward Delta (gamma, beta frozen, biased variance),
+// the bias c is state (c += sum_s A[., s]) and enters every token product as
+// "+1": with c = c_a,
+//     X_b^T = W^T K_b^T + c + A_a (K_a K_b^T + 1)
+//     pre_a^T = W^T Q_a^T + c + A_a tril(Q_a K_a^T + 1)^T
+//     pre_b^T = W^T Q_b^T + c + A_a (K_a Q_b^T + 1) + A_b tril(Q_b K_b^T + 1)^T
+// and Z = Q + LN(pre).  The per-token reductions over the 64 features are
+// in-thread sums over 4 rows, three shuffle levels and one exchange between
+// the unit's two warps.
 //
 // Mapping onto sm_100a.  Two units share a CTA and are stacked in M = 128
 // (unit 0 in TMEM lanes 0-63, unit 1 in 64-127).  Per pair:
@@ -37,18 +48,18 @@
 // and returns.
 #pragma once
 #include "common.cuh"
-#include "linear_tc.cuh"
 #include "ptx.cuh"
+#include "tc_common.cuh"
 
 namespace ttt {
 namespace lfr {
 
-using ltc::ldsm_x4;
-using ltc::load_a_frags;
-using ltc::load_b_frags;
-using ltc::Params;
-using ltc::tmem_st_32x32b_x32;
-using ltc::umma_ts;
+using tcc::ldsm_x4;
+using tcc::load_a_frags;
+using tcc::load_b_frags;
+using Params = tcc::LinearParams;
+using tcc::tmem_st_32x32b_x32;
+using tcc::umma_ts;
 
 constexpr int kD = 64;
 constexpr int kTok = 16;
@@ -80,7 +91,8 @@ constexpr int kOffAblk = kOffH + kHring * kHslot;         // 84992 (1024-aligned
 constexpr int kAblkBytes = 16384;                         // bf16 [128 rows][64 k], K-major, no swizzle
 constexpr int kOffZs = kOffAblk + kAblkBytes;             // Z staging: [4 warps] 32 tokens x 32 j, 64B swizzle
 constexpr int kZsBytes = 2048;
-constexpr int kOffBar = kOffZs + 4 * kZsBytes;
+constexpr int kOffRed = kOffZs + 4 * kZsBytes;           // LN: 2 buffers x [4 warps][16 tokens] float2
+constexpr int kOffBar = kOffRed + 2 * 4 * 16 * 8;
 constexpr int kNumBars = 2 * kStages + 2 * kHring + 6;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64;
@@ -125,10 +137,11 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Helper: the 16 x 16 product X Y^T of two 16 x 64 tiles (fragments given),
-// masked to s <= t if `causal`, stored in bf16 at `dst` (layout of mat_off).
+// Helper: the 16 x 16 product X Y^T + add of two 16 x 64 tiles (fragments
+// given), masked to s <= t if `causal`, stored in bf16 at `dst` (layout of
+// mat_off).
 __device__ __forceinline__ void product_store(const uint32_t (*fa)[4], const uint32_t (*fb)[4], bool causal,
-                                              uint8_t* dst, int lane) {
+                                              float add, uint8_t* dst, int lane) {
     float acc[2][4] = {};
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
@@ -141,7 +154,7 @@ __device__ __forceinline__ void product_store(const uint32_t (*fa)[4], const uin
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             const int t = r0 + 8 * hh, s = 8 * nt + c0;
-            float lo = acc[nt][2 * hh], hi = acc[nt][2 * hh + 1];
+            float lo = acc[nt][2 * hh] + add, hi = acc[nt][2 * hh + 1] + add;
             if (causal) {
                 lo = s <= t ? lo : 0.f;
                 hi = s + 1 <= t ? hi : 0.f;
@@ -150,7 +163,40 @@ __device__ __forceinline__ void product_store(const uint32_t (*fa)[4], const uin
         }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+// LN: sums over the unit's 64 features of two per-token quantities.  The
+// thread's tokens are k = 2 nt + e1 -> t = 8 nt + 2 c + e1; sa, sb hold its
+// partial sums over its four rows.  Afterwards every thread holds the unit's
+// totals for its four tokens.
+__device__ __forceinline__ void tok_sum2(float* sa, float* sb, float2* red, int q, int lane) {
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            sa[k] += __shfl_xor_sync(0xffffffffu, sa[k], o);
+            sb[k] += __shfl_xor_sync(0xffffffffu, sb[k], o);
+        }
+    const int c = lane & 3;
+    if (lane < 4) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) red[q * 16 + 8 * (k >> 1) + 2 * c + (k & 1)] = make_float2(sa[k], sb[k]);
+    }
+    named_bar_sync(1 + (q >> 1), 64);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 o = red[(q ^ 1) * 16 + 8 * (k >> 1) + 2 * c + (k & 1)];
+        sa[k] += o.x;
+        sb[k] += o.y;
+    }
+}
+
+// bf16 element e (0..3, accumulator order) of an ldmatrix.trans fragment pair
+__device__ __forceinline__ float frag_val(const uint32_t* f, int nt, int e) {
+    const uint32_t x = f[2 * nt + (e >> 1)];
+    return (e & 1) ? bf16_hi(x) : bf16_lo(x);
+}
+
+template <bool LN>
+__global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
     linear_frag_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZ,
                        const __grid_constant__ CUtensorMap tmZ1, Params p) {
@@ -317,14 +363,16 @@ __global__ void __launch_bounds__(kThreads, 2)
             uint32_t fka[4][4], fx[4][4], fy[4][4];
             load_b_frags(st + off_k(u, 0), lane, fka);      // K_a as B
             load_a_frags(st + off_q(u, 0), lane, fx);       // Q_a as A
-            product_store(fx, fka, true, hs, lane);         // S_a
+            // LN: "+1" for the bias term of every token product
+            const float one = LN ? 1.f : 0.f;
+            product_store(fx, fka, true, one, hs, lane);         // S_a
             if (hasb) {
                 load_a_frags(st + off_q(u, 1), lane, fx);   // Q_b as A
-                product_store(fx, fka, false, hs + 3 * kMat, lane);   // M2 = Q_b K_a^T
+                product_store(fx, fka, false, one, hs + 3 * kMat, lane);   // M2 = Q_b K_a^T (+1)
                 load_b_frags(st + off_k(u, 1), lane, fy);   // K_b as B
-                product_store(fx, fy, true, hs + kMat, lane);         // S_b
+                product_store(fx, fy, true, one, hs + kMat, lane);         // S_b
                 load_a_frags(st + off_k(u, 1), lane, fx);   // K_b as A
-                product_store(fx, fka, false, hs + 2 * kMat, lane);   // M1 = K_b K_a^T
+                product_store(fx, fka, false, one, hs + 2 * kMat, lane);   // M1 = K_b K_a^T (+1)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&haux[g % kHring]);
@@ -339,6 +387,25 @@ __global__ void __launch_bounds__(kThreads, 2)
         const int n = unit / p.H, h = unit % p.H;
         const uint32_t tl = tbase + ((uint32_t)(32 * q) << 16);
         uint8_t* zs = smem + kOffZs + q * kZsBytes;   // this warp's Z staging tile
+        // LN: gamma, beta and the bias state c of this thread's rows jb + 16 mt + r + 8 h
+        float gam[2][2], bet[2][2], cst[2][2];
+        float2* red = reinterpret_cast<float2*>(smem + kOffRed);
+        int nred = 0;   // reductions so far (two alternating buffers)
+        if (LN) {
+#pragma unroll
+            for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int j = jb + 16 * mt + r + 8 * hh;
+                    gam[mt][hh] = p.gamma[(size_t)h * kD + j];
+                    bet[mt][hh] = p.beta[(size_t)h * kD + j];
+                    cst[mt][hh] = p.c0 ? p.c0[(size_t)n * p.c0_bstride + (size_t)h * kD + j] : 0.f;
+                }
+        }
+        auto rsum = [&](float* sa, float* sb) {
+            tok_sum2(sa, sb, red + (nred & 1) * 64, q, lane);
+            ++nred;
+        };
         // W_0^T row j = column j of W_0, in fp32 and bf16; the other unit's
         // half of this warp's rows in the block-diagonal A stays zero
         {
@@ -402,7 +469,8 @@ __global__ void __launch_bounds__(kThreads, 2)
             WT(&full[g % kStages], (g / kStages) & 1);
             WT(&haux[g % kHring], (g / kHring) & 1);
             float et[2][4];          // [hb]: eta of tokens 2c, 2c+1, 8+2c, 9+2c
-            float ev[2][2][2][4];    // [hb][mt][nt][e]: eta_t * V[t][j]
+            float ev[2][2][2][4];    // plain: [hb][mt][nt][e]: eta_t * V[t][j]
+            uint32_t vf[2][2][4], kf[2][2][4], qf[2][2][4];   // LN: [hb][mt] bf16 fragments of V, K, Q
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb) {
                 if (p.eta) {
@@ -422,14 +490,18 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
                 for (int mt = 0; mt < 2; ++mt) {
                     const int jblk = (jb >> 3) + 2 * mt + (mi & 1);
-                    uint32_t v[4];
-                    ldsm_x4_t(vt + t * 128 + ((jblk ^ (t & 7)) << 4), v);
+                    const uint32_t off = t * 128 + ((jblk ^ (t & 7)) << 4);
+                    if (LN) {
+                        ldsm_x4_t(vt + off, vf[hb][mt]);
+                        ldsm_x4_t(smem_u32(st + off_k(u, hb)) + off, kf[hb][mt]);
+                        ldsm_x4_t(smem_u32(st + off_q(u, hb)) + off, qf[hb][mt]);
+                    } else {
+                        uint32_t v[4];
+                        ldsm_x4_t(vt + off, v);
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        ev[hb][mt][nt][0] = et[hb][2 * nt] * bf16_lo(v[2 * nt]);
-                        ev[hb][mt][nt][1] = et[hb][2 * nt + 1] * bf16_hi(v[2 * nt]);
-                        ev[hb][mt][nt][2] = et[hb][2 * nt] * bf16_lo(v[2 * nt + 1]);
-                        ev[hb][mt][nt][3] = et[hb][2 * nt + 1] * bf16_hi(v[2 * nt + 1]);
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) ev[hb][mt][nt][e] = et[hb][2 * nt + (e & 1)] * frag_val(v, nt, e);
                     }
                 }
             }
@@ -453,7 +525,104 @@ __global__ void __launch_bounds__(kThreads, 2)
                     tmem_ld_16x256b_x2(tbase + ((uint32_t)(32 * q + 16 * mt) << 16) + kColP + 64 * hb + 32 * u, pe[hb][mt]);
             tmem_wait_ld();
             // 3. A_a = eta (V_a - E_a); E_b += A_a M1^T; A_b = eta (V_b - E_b)
+            //    (LN: A = -eta Delta of the LN backward at X_a, X_b)
             uint32_t aa[2][4], ab[2][4];
+            float c_old[2][2];
+            if (LN) {
+                // one mini-batch of the LN chain: x (pre-activation, accumulator
+                // layout) -> A (fp32 in x, packed bf16 fragments in fr)
+                auto ln_batch = [&](float (&x)[2][2][4], int hb, uint32_t (&fr)[2][4]) {
+                    float s1[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float v = x[mt][nt][e];
+                                s1[2 * nt + (e & 1)] += v;
+                                s2[2 * nt + (e & 1)] += v * v;
+                            }
+                    rsum(s1, s2);
+                    float rr[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float mu = s1[k] * (1.f / kD);
+                        rr[k] = rsqrtf(fmaxf(s2[k] * (1.f / kD) - mu * mu, 0.f) + p.eps);
+                        s1[k] = mu;
+                    }
+                    float gg[2][2][4], t1[4] = {0.f, 0.f, 0.f, 0.f}, t2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int k = 2 * nt + (e & 1), hh = e >> 1;
+                                const float xh = (x[mt][nt][e] - s1[k]) * rr[k];   // x-hat
+                                // e = k + gamma xhat + beta - v (residual of f), g = gamma e
+                                const float res = frag_val(kf[hb][mt], nt, e) + gam[mt][hh] * xh + bet[mt][hh] -
+                                                  frag_val(vf[hb][mt], nt, e);
+                                const float g = gam[mt][hh] * res;
+                                gg[mt][nt][e] = g;
+                                x[mt][nt][e] = xh;
+                                t1[k] += g;
+                                t2[k] += g * xh;
+                            }
+                    rsum(t1, t2);
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int k = 2 * nt + (e & 1);
+                                const float delta = rr[k] * (gg[mt][nt][e] - t1[k] * (1.f / kD) -
+                                                             x[mt][nt][e] * t2[k] * (1.f / kD));
+                                x[mt][nt][e] = -et[hb][k] * delta;
+                            }
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        fr[mt][0] = pack_bf16x2(x[mt][0][0], x[mt][0][1]);
+                        fr[mt][1] = pack_bf16x2(x[mt][0][2], x[mt][0][3]);
+                        fr[mt][2] = pack_bf16x2(x[mt][1][0], x[mt][1][1]);
+                        fr[mt][3] = pack_bf16x2(x[mt][1][2], x[mt][1][3]);
+                    }
+                };
+                float xa[2][2][4], xb[2][2][4];
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            xa[mt][nt][e] = __uint_as_float(pe[0][mt][4 * nt + e]) + cst[mt][e >> 1];
+                            xb[mt][nt][e] = __uint_as_float(pe[1][mt][4 * nt + e]) + cst[mt][e >> 1];
+                        }
+                ln_batch(xa, 0, aa);
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) mma16816(xb[mt][nt], aa[mt], m1[2 * nt], m1[2 * nt + 1]);
+                ln_batch(xb, 1, ab);
+                // bias state: c += sum over the pair's tokens of A (fp32); a missing
+                // second mini-batch contributes nothing
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float cs = 0.f;
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e1 = 0; e1 < 2; ++e1)
+                                cs += xa[mt][nt][2 * hh + e1] + (hasb ? xb[mt][nt][2 * hh + e1] : 0.f);
+                        cs += __shfl_xor_sync(0xffffffffu, cs, 1);
+                        cs += __shfl_xor_sync(0xffffffffu, cs, 2);
+                        c_old[mt][hh] = cst[mt][hh];
+                        cst[mt][hh] += cs;
+                    }
+            } else {
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
                 float a[2][4], b[2][4];
@@ -480,6 +649,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 ab[mt][2] = pack_bf16x2(b[1][0], b[1][1]);
                 ab[mt][3] = pack_bf16x2(b[1][2], b[1][3]);
             }
+            }
             // 4. A_a, A_b into the block-diagonal A operand of MMA_W (k = 32 u + 16 hb + s)
 #pragma unroll
             for (int mt = 0; mt < 2; ++mt) {
@@ -501,6 +671,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             // 5. outputs while MMA_W runs:
             //    Z_a^T = P_Zqa + A_a S_a^T,  Z_b^T = P_Zqb + A_a M2^T + A_b S_b^T
             uint32_t zp[2][2][2][2];   // [hb][mt][nt][rows r / r+8]: bf16 pairs of tokens (2c, 2c+1)
+            float zf[2][2][2][4];      // [hb][mt][nt][e]: pre-output (LN: then output) in fp32
             {
                 uint32_t pq[2][2][8];
 #pragma unroll
@@ -514,21 +685,61 @@ __global__ void __launch_bounds__(kThreads, 2)
                 for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
-                        float da[4], db[4];
+                        float* da = zf[0][mt][nt];
+                        float* db = zf[1][mt][nt];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) {
-                            da[e] = __uint_as_float(pq[0][mt][4 * nt + e]);
-                            db[e] = __uint_as_float(pq[1][mt][4 * nt + e]);
+                            da[e] = __uint_as_float(pq[0][mt][4 * nt + e]) + (LN ? c_old[mt][e >> 1] : 0.f);
+                            db[e] = __uint_as_float(pq[1][mt][4 * nt + e]) + (LN ? c_old[mt][e >> 1] : 0.f);
                         }
                         mma16816(da, aa[mt], msa[2 * nt], msa[2 * nt + 1]);
                         mma16816(db, aa[mt], m2[2 * nt], m2[2 * nt + 1]);
                         mma16816(db, ab[mt], msb[2 * nt], msb[2 * nt + 1]);
-                        zp[0][mt][nt][0] = pack_bf16x2(da[0], da[1]);
-                        zp[0][mt][nt][1] = pack_bf16x2(da[2], da[3]);
-                        zp[1][mt][nt][0] = pack_bf16x2(db[0], db[1]);
-                        zp[1][mt][nt][1] = pack_bf16x2(db[2], db[3]);
                     }
             }
+            if (LN) {
+                // Z = Q + gamma LN(pre) + beta, per mini-batch of the pair
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    float s1[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float v = zf[hb][mt][nt][e];
+                                s1[2 * nt + (e & 1)] += v;
+                                s2[2 * nt + (e & 1)] += v * v;
+                            }
+                    rsum(s1, s2);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float mu = s1[k] * (1.f / kD);
+                        s2[k] = rsqrtf(fmaxf(s2[k] * (1.f / kD) - mu * mu, 0.f) + p.eps);
+                        s1[k] = mu;
+                    }
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int k = 2 * nt + (e & 1), hh = e >> 1;
+                                zf[hb][mt][nt][e] = frag_val(qf[hb][mt], nt, e) +
+                                                    gam[mt][hh] * (zf[hb][mt][nt][e] - s1[k]) * s2[k] + bet[mt][hh];
+                            }
+                }
+            }
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        zp[hb][mt][nt][0] = pack_bf16x2(zf[hb][mt][nt][0], zf[hb][mt][nt][1]);
+                        zp[hb][mt][nt][1] = pack_bf16x2(zf[hb][mt][nt][2], zf[hb][mt][nt][3]);
+                    }
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&hfree[g % kHring]);
@@ -566,6 +777,14 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 32; ++k) Wo[(32 * half + k) * kD] = __uint_as_float(w[k]);
+            }
+            if (LN && p.c_out && c == 0) {
+                // the four lanes of a row group hold the same bias rows; lane c = 0 writes them
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        p.c_out[(size_t)unit * kD + jb + 16 * mt + r + 8 * hh] = cst[mt][hh];
             }
         }
     }

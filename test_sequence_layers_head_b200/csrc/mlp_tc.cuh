@@ -37,20 +37,20 @@
 // the kernel records kStatusTimeout, drains what it issued and returns.
 #pragma once
 #include "common.cuh"
-#include "linear_tc.cuh"
+#include "tc_common.cuh"
 #include "ptx.cuh"
 
 namespace ttt {
 namespace mtc {
 
-using ltc::ld_bf16;
-using ltc::ldsm_x4;
-using ltc::mma_16816;
-using ltc::nosw_off;
-using ltc::sw128_off;
-using ltc::tmem_st_32x32b_x32;
-using ltc::tmem_st_32x32b_x8;
-using ltc::umma_ts;
+using tcc::ld_bf16;
+using tcc::ldsm_x4;
+using tcc::mma_16816;
+using tcc::nosw_off;
+using tcc::sw128_off;
+using tcc::tmem_st_32x32b_x32;
+using tcc::tmem_st_32x32b_x8;
+using tcc::umma_ts;
 
 constexpr int kD = 64, kM = 256, kTok = 16;
 constexpr int kStages = 4;

@@ -11,7 +11,6 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "linear_frag.cuh"
-#include "linear_tc.cuh"
 #include "mlp_tc.cuh"
 #include "simt.cuh"
 #include "tmap.h"
@@ -113,7 +112,7 @@ ttt_status simt_linear(const ttt_linear_args* a, cudaStream_t st) {
 
 template <bool LN>
 ttt_status tc_linear(const ttt_linear_args* a, cudaStream_t st) {
-    using namespace ltc;
+    using namespace lfr;
     const long long U = (long long)a->B * a->H;
     const long long rows = U * a->T;
     CUtensorMap mQ, mK, mV;
@@ -122,7 +121,7 @@ ttt_status tc_linear(const ttt_linear_args* a, cudaStream_t st) {
         !encode_2d(&mK, a->K, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !encode_2d(&mV, a->V, bf, kD, rows, kD * 2, kD, kTok, CU_TENSOR_MAP_SWIZZLE_128B))
         return TTT_ERR_CUDA;
-    Params p;
+    tcc::LinearParams p;
     p.U = (int)U;
     p.H = a->H;
     p.T = a->T;
@@ -144,22 +143,16 @@ ttt_status tc_linear(const ttt_linear_args* a, cudaStream_t st) {
     p.flags = a->flags;
     if (!p.status) return TTT_ERR_CUDA;
     const int grid = (int)((U + 1) / 2);
-    if (LN) {
-        auto k = linear_tc_kernel<true>;
-        if (!set_smem(k, kSmemBytes)) return TTT_ERR_CUDA;
-        k<<<grid, kThreads, kSmemBytes, st>>>(mQ, mK, mV, p);
-    } else {
-        // plain model: pairs of mini-batches per tensor-core round trip; Z is
-        // written by TMA stores of 32-token (and, for an odd last mini-batch,
-        // 16-token) boxes of 32 features
-        CUtensorMap mZ, mZ1;
-        if (!encode_2d(&mZ, a->Z, bf, kD, rows, kD * 2, 32, 2 * kTok, CU_TENSOR_MAP_SWIZZLE_64B) ||
-            !encode_2d(&mZ1, a->Z, bf, kD, rows, kD * 2, 32, kTok, CU_TENSOR_MAP_SWIZZLE_64B))
-            return TTT_ERR_CUDA;
-        auto k = lfr::linear_frag_kernel;
-        if (!set_smem(k, lfr::kSmemBytes)) return TTT_ERR_CUDA;
-        k<<<grid, lfr::kThreads, lfr::kSmemBytes, st>>>(mQ, mK, mV, mZ, mZ1, p);
-    }
+    // pairs of mini-batches per tensor-core round trip; Z is written by TMA
+    // stores of 32-token (and, for an odd last mini-batch, 16-token) boxes of
+    // 32 features
+    CUtensorMap mZ, mZ1;
+    if (!encode_2d(&mZ, a->Z, bf, kD, rows, kD * 2, 32, 2 * kTok, CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !encode_2d(&mZ1, a->Z, bf, kD, rows, kD * 2, 32, kTok, CU_TENSOR_MAP_SWIZZLE_64B))
+        return TTT_ERR_CUDA;
+    auto k = lfr::linear_frag_kernel<LN>;
+    if (!set_smem(k, lfr::kSmemBytes)) return TTT_ERR_CUDA;
+    k<<<grid, lfr::kThreads, lfr::kSmemBytes, st>>>(mQ, mK, mV, mZ, mZ1, p);
     return launch_status();
 }
 
