@@ -439,6 +439,28 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             }
         };
         const int mi = lane >> 3;   // ldmatrix / stmatrix: matrix served by this lane's address
+        // Z of a pair (bf16 pairs of tokens 2c, 2c+1: [hb][mt][nt][rows r / r+8]) is
+        // staged and stored while the next pair's MMA_P runs
+        uint32_t zp[2][2][2][2];
+        auto store_z = [&](int g1) {
+            if (lane == 0) bulk_wait_read<0>();   // the previous store has read the staging tile
+            __syncwarp();
+            const int t8 = 8 * (mi >> 1) + (lane & 7);
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb)
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    const int t = 16 * hb + t8, chunk = 2 * mt + (mi & 1);
+                    stsm_x4_t(smem_u32(zs) + t * 64 + ((chunk ^ ((t >> 1) & 3)) << 4), zp[hb][mt][0][0],
+                              zp[hb][mt][0][1], zp[hb][mt][1][0], zp[hb][mt][1][1]);
+                }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && !dead && store_unit) {
+                tma_store_2d(2 * g1 + 1 < nsteps ? &tmZ : &tmZ1, zs, jb, unit * p.T + 2 * g1 * kTok);
+                bulk_commit();
+            }
+        };
         for (int g = 0; g < npairs; ++g) {
             const uint8_t* st = stage_ptr(g);
             const uint32_t hs = smem_u32(hslot_ptr(g) + u * 4 * kMat);
@@ -464,6 +486,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                     mbar_arrive(aw_ready);
                     mbar_arrive(&empty[(g - 1) % kStages]);   // MMA_W of pair g-1 was its last reader
                 }
+                store_z(g - 1);
             }
             // 1. inputs: eta, eta * V (accumulator layout), the token products
             WT(&full[g % kStages], (g / kStages) & 1);
@@ -670,7 +693,6 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             if (lane == 0) mbar_arrive(a_ready);
             // 5. outputs while MMA_W runs:
             //    Z_a^T = P_Zqa + A_a S_a^T,  Z_b^T = P_Zqb + A_a M2^T + A_b S_b^T
-            uint32_t zp[2][2][2][2];   // [hb][mt][nt][rows r / r+8]: bf16 pairs of tokens (2c, 2c+1)
             float zf[2][2][2][4];      // [hb][mt][nt][e]: pre-output (LN: then output) in fp32
             {
                 uint32_t pq[2][2][8];
@@ -741,29 +763,9 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                         zp[hb][mt][nt][1] = pack_bf16x2(zf[hb][mt][nt][2], zf[hb][mt][nt][3]);
                     }
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&hfree[g % kHring]);
-                bulk_wait_read<0>();   // the previous pair's store has read the staging tile
-            }
-            __syncwarp();
-            {
-                const int t8 = 8 * (mi >> 1) + (lane & 7);
-#pragma unroll
-                for (int hb = 0; hb < 2; ++hb)
-#pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
-                        const int t = 16 * hb + t8, chunk = 2 * mt + (mi & 1);
-                        stsm_x4_t(smem_u32(zs) + t * 64 + ((chunk ^ ((t >> 1) & 3)) << 4), zp[hb][mt][0][0],
-                                  zp[hb][mt][0][1], zp[hb][mt][1][0], zp[hb][mt][1][1]);
-                    }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0 && !dead && store_unit) {
-                tma_store_2d(hasb ? &tmZ : &tmZ1, zs, jb, unit * p.T + 2 * g * kTok);
-                bulk_commit();
-            }
+            if (lane == 0) mbar_arrive(&hfree[g % kHring]);
         }
+        store_z(npairs - 1);
         // final state (MMA_W of the last pair)
         WT(w_done, (npairs - 1) & 1);
         tc_fence_after();
