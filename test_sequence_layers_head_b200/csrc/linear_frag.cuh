@@ -64,6 +64,7 @@ using tcc::umma_ts;
 constexpr int kD = 64;
 constexpr int kTok = 16;
 constexpr int kThreads = 256;
+constexpr long long kOneUnitMaxUnits = 148;   // one unit per CTA up to this many units (the SM count)
 constexpr int kStages = 3;       // input pipeline depth, in pairs of mini-batches
 constexpr int kHring = 2;        // helper product slots, in pairs
 
@@ -165,8 +166,10 @@ __device__ __forceinline__ void product_store(const uint32_t (*fa)[4], const uin
 
 // LN: sums over the unit's 64 features of two per-token quantities.  The
 // thread's tokens are k = 2 nt + e1 -> t = 8 nt + 2 c + e1; sa, sb hold its
-// partial sums over its four rows.  Afterwards every thread holds the unit's
-// totals for its four tokens.
+// partial sums over its rows.  The unit's rows are spread over NW warps
+// (2: warps q, q ^ 1; 4: warps 0-3).  Afterwards every thread holds the
+// unit's totals for its four tokens.
+template <int NW>
 __device__ __forceinline__ void tok_sum2(float* sa, float* sb, float2* red, int q, int lane) {
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1)
@@ -180,12 +183,28 @@ __device__ __forceinline__ void tok_sum2(float* sa, float* sb, float2* red, int 
 #pragma unroll
         for (int k = 0; k < 4; ++k) red[q * 16 + 8 * (k >> 1) + 2 * c + (k & 1)] = make_float2(sa[k], sb[k]);
     }
-    named_bar_sync(1 + (q >> 1), 64);
+    if (NW == 2) {
+        named_bar_sync(1 + (q >> 1), 64);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float2 o = red[(q ^ 1) * 16 + 8 * (k >> 1) + 2 * c + (k & 1)];
-        sa[k] += o.x;
-        sb[k] += o.y;
+        for (int k = 0; k < 4; ++k) {
+            const float2 o = red[(q ^ 1) * 16 + 8 * (k >> 1) + 2 * c + (k & 1)];
+            sa[k] += o.x;
+            sb[k] += o.y;
+        }
+    } else {
+        named_bar_sync(1, 128);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float a = 0.f, b = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float2 o = red[w * 16 + 8 * (k >> 1) + 2 * c + (k & 1)];
+                a += o.x;
+                b += o.y;
+            }
+            sa[k] = a;
+            sb[k] = b;
+        }
     }
 }
 
@@ -195,7 +214,13 @@ __device__ __forceinline__ float frag_val(const uint32_t* f, int nt, int e) {
     return (e & 1) ? bf16_hi(x) : bf16_lo(x);
 }
 
-template <bool LN>
+// UPC = units per CTA.  2: two units stacked in M = 128, each epilogue warp
+// owns 32 state rows (two m16 tiles).  1: the CTA's unit is loaded into both
+// halves of M = 128 and each epilogue warp owns 16 of its rows, one m16 tile
+// on its own lane quadrant (rows 0-15, 32-47 from the first half, 16-31,
+// 48-63 from the second); the other lanes carry unused copies.  1 is for
+// workloads with fewer units than SMs: half the serial work per warp.
+template <bool LN, int UPC>
 __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
     linear_frag_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmZ,
@@ -221,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
     volatile int* s_abort = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int unit0 = 2 * blockIdx.x;
-    const bool has1 = unit0 + 1 < p.U;
+    const int unit0 = UPC * blockIdx.x;
+    const bool has1 = UPC == 2 && unit0 + 1 < p.U;
     const int unit1 = has1 ? unit0 + 1 : unit0;
     const int nsteps = p.nsteps;
     const int npairs = (nsteps + 1) / 2;
@@ -380,20 +405,23 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
     } else {
         // ------------------------------------------------------------ epilogue
         const int q = warp, u = q >> 1;
-        const int jb = 32 * (q & 1);          // first state row (feature) of this warp
+        const int jb = 32 * (q & 1) + (UPC == 1 ? 16 * u : 0);   // first state row (feature) of this warp
+        constexpr int NMT = UPC == 2 ? 2 : 1;                     // m16 tiles per warp
+        // TMEM lane of the first row of m-tile mt (rows and lanes coincide within a unit half)
+        auto lane0 = [&](int mt) { return 64 * u + jb + 16 * mt; };
         const int r = lane >> 2, c = lane & 3;
         const int unit = u ? unit1 : unit0;
-        const bool store_unit = (u == 0) || has1;
+        const bool store_unit = (u == 0) || has1 || UPC == 1;
         const int n = unit / p.H, h = unit % p.H;
         const uint32_t tl = tbase + ((uint32_t)(32 * q) << 16);
         uint8_t* zs = smem + kOffZs + q * kZsBytes;   // this warp's Z staging tile
         // LN: gamma, beta and the bias state c of this thread's rows jb + 16 mt + r + 8 h
-        float gam[2][2], bet[2][2], cst[2][2];
+        float gam[2][2] = {}, bet[2][2] = {}, cst[2][2] = {};
         float2* red = reinterpret_cast<float2*>(smem + kOffRed);
         int nred = 0;   // reductions so far (two alternating buffers)
         if (LN) {
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
+            for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const int j = jb + 16 * mt + r + 8 * hh;
@@ -403,13 +431,13 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 }
         }
         auto rsum = [&](float* sa, float* sb) {
-            tok_sum2(sa, sb, red + (nred & 1) * 64, q, lane);
+            tok_sum2<4 / NMT>(sa, sb, red + (nred & 1) * 64, q, lane);
             ++nred;
         };
         // W_0^T row j = column j of W_0, in fp32 and bf16; the other unit's
         // half of this warp's rows in the block-diagonal A stays zero
         {
-            const int j = jb + lane;
+            const int j = 32 * (q & 1) + lane;   // row held by this lane of the quadrant
             const float* W0u = p.W0 + (size_t)n * p.W0_bstride + (size_t)h * kD * kD;
             uint32_t w[64], pk[32];
 #pragma unroll
@@ -421,9 +449,16 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             tmem_st_32x32b_x32(tl + kColAW, pk);
             const int m = 64 * u + j;
             const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+            if (UPC == 2) {
 #pragma unroll
-            for (int k = 0; k < 32; k += 8)
-                *reinterpret_cast<uint4*>(smem + kOffAblk + ablk_off(m, 32 * (1 - u) + k)) = z4;
+                for (int k = 0; k < 32; k += 8)
+                    *reinterpret_cast<uint4*>(smem + kOffAblk + ablk_off(m, 32 * (1 - u) + k)) = z4;
+            } else {
+                // rows not owned by an epilogue warp keep an all-zero A
+#pragma unroll
+                for (int k = 0; k < 64; k += 8)
+                    *reinterpret_cast<uint4*>(smem + kOffAblk + ablk_off(m, k)) = z4;
+            }
         }
         fence_proxy_async_smem();
         tmem_wait_st();
@@ -449,10 +484,12 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb)
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
+                for (int mt = 0; mt < NMT; ++mt) {
                     const int t = 16 * hb + t8, chunk = 2 * mt + (mi & 1);
-                    stsm_x4_t(smem_u32(zs) + t * 64 + ((chunk ^ ((t >> 1) & 3)) << 4), zp[hb][mt][0][0],
-                              zp[hb][mt][0][1], zp[hb][mt][1][0], zp[hb][mt][1][1]);
+                    const uint32_t off = UPC == 2 ? t * 64 + ((chunk ^ ((t >> 1) & 3)) << 4)    // 64B swizzle
+                                                  : t * 32 + ((chunk ^ ((t >> 2) & 1)) << 4);   // 32B swizzle
+                    stsm_x4_t(smem_u32(zs) + off, zp[hb][mt][0][0], zp[hb][mt][0][1], zp[hb][mt][1][0],
+                              zp[hb][mt][1][1]);
                 }
             fence_proxy_async_smem();
             __syncwarp();
@@ -511,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 const uint32_t vt = smem_u32(st + off_v(u, hb));
                 const int t = 8 * (mi >> 1) + (lane & 7);
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt) {
+                for (int mt = 0; mt < NMT; ++mt) {
                     const int jblk = (jb >> 3) + 2 * mt + (mi & 1);
                     const uint32_t off = t * 128 + ((jblk ^ (t & 7)) << 4);
                     if (LN) {
@@ -544,8 +581,8 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb)
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
-                    tmem_ld_16x256b_x2(tbase + ((uint32_t)(32 * q + 16 * mt) << 16) + kColP + 64 * hb + 32 * u, pe[hb][mt]);
+                for (int mt = 0; mt < NMT; ++mt)
+                    tmem_ld_16x256b_x2(tbase + ((uint32_t)lane0(mt) << 16) + kColP + 64 * hb + 32 * u, pe[hb][mt]);
             tmem_wait_ld();
             // 3. A_a = eta (V_a - E_a); E_b += A_a M1^T; A_b = eta (V_b - E_b)
             //    (LN: A = -eta Delta of the LN backward at X_a, X_b)
@@ -557,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 auto ln_batch = [&](float (&x)[2][2][4], int hb, uint32_t (&fr)[2][4]) {
                     float s1[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
+                    for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -576,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                     }
                     float gg[2][2][4], t1[4] = {0.f, 0.f, 0.f, 0.f}, t2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
+                    for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -594,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                             }
                     rsum(t1, t2);
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
+                    for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -605,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                                 x[mt][nt][e] = -et[hb][k] * delta;
                             }
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt) {
+                    for (int mt = 0; mt < NMT; ++mt) {
                         fr[mt][0] = pack_bf16x2(x[mt][0][0], x[mt][0][1]);
                         fr[mt][1] = pack_bf16x2(x[mt][0][2], x[mt][0][3]);
                         fr[mt][2] = pack_bf16x2(x[mt][1][0], x[mt][1][1]);
@@ -614,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 };
                 float xa[2][2][4], xb[2][2][4];
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -624,14 +661,14 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                         }
                 ln_batch(xa, 0, aa);
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) mma16816(xb[mt][nt], aa[mt], m1[2 * nt], m1[2 * nt + 1]);
                 ln_batch(xb, 1, ab);
                 // bias state: c += sum over the pair's tokens of A (fp32); a missing
                 // second mini-batch contributes nothing
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         float cs = 0.f;
@@ -647,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                     }
             } else {
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
+            for (int mt = 0; mt < NMT; ++mt) {
                 float a[2][4], b[2][4];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
@@ -675,7 +712,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
             }
             // 4. A_a, A_b into the block-diagonal A operand of MMA_W (k = 32 u + 16 hb + s)
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
+            for (int mt = 0; mt < NMT; ++mt) {
                 const int m = 64 * u + jb + 16 * mt + r;
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {
@@ -699,12 +736,12 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb)
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
-                        tmem_ld_16x256b_x2(tbase + ((uint32_t)(32 * q + 16 * mt) << 16) + kColP + 64 * hb + 32 * u + 16,
+                    for (int mt = 0; mt < NMT; ++mt)
+                        tmem_ld_16x256b_x2(tbase + ((uint32_t)lane0(mt) << 16) + kColP + 64 * hb + 32 * u + 16,
                                            pq[hb][mt]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
                         float* da = zf[0][mt][nt];
@@ -725,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 for (int hb = 0; hb < 2; ++hb) {
                     float s1[4] = {0.f, 0.f, 0.f, 0.f}, s2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
+                    for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -742,7 +779,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                         s1[k] = mu;
                     }
 #pragma unroll
-                    for (int mt = 0; mt < 2; ++mt)
+                    for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -756,7 +793,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
 #pragma unroll
             for (int hb = 0; hb < 2; ++hb)
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
                         zp[hb][mt][nt][0] = pack_bf16x2(zf[hb][mt][nt][0], zf[hb][mt][nt][1]);
@@ -772,18 +809,22 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
         if (lane == 0) bulk_wait<0>();   // Z stores complete before the CTA exits
         if (store_unit && !dead) {
             uint32_t w[32];
-            float* Wo = p.W_out + (size_t)unit * kD * kD + jb + lane;
+            // lane l of the quadrant holds row 32 (q & 1) + l of its unit half
+            const bool own = UPC == 2 || (lane >> 4) == u;
+            float* Wo = p.W_out + (size_t)unit * kD * kD + 32 * (q & 1) + lane;
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 tmem_ld_32x32b_x32(tl + kColW + 32 * half, w);
                 tmem_wait_ld();
+                if (own) {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) Wo[(32 * half + k) * kD] = __uint_as_float(w[k]);
+                    for (int k = 0; k < 32; ++k) Wo[(32 * half + k) * kD] = __uint_as_float(w[k]);
+                }
             }
             if (LN && p.c_out && c == 0) {
                 // the four lanes of a row group hold the same bias rows; lane c = 0 writes them
 #pragma unroll
-                for (int mt = 0; mt < 2; ++mt)
+                for (int mt = 0; mt < NMT; ++mt)
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh)
                         p.c_out[(size_t)unit * kD + jb + 16 * mt + r + 8 * hh] = cst[mt][hh];

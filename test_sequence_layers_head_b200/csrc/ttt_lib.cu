@@ -145,14 +145,18 @@ ttt_status tc_linear(const ttt_linear_args* a, cudaStream_t st) {
     const int grid = (int)((U + 1) / 2);
     // pairs of mini-batches per tensor-core round trip; Z is written by TMA
     // stores of 32-token (and, for an odd last mini-batch, 16-token) boxes of
-    // 32 features
+    // the 32 (two units per CTA) or 16 (one unit per CTA) features of a warp
+    const bool one = (a->flags & TTT_FLAG_ONE_UNIT_PER_CTA) ||
+                     (!(a->flags & TTT_FLAG_TWO_UNITS_PER_CTA) && U <= kOneUnitMaxUnits);
+    const uint32_t zcols = one ? 16 : 32;
+    const auto zswz = one ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B;
     CUtensorMap mZ, mZ1;
-    if (!encode_2d(&mZ, a->Z, bf, kD, rows, kD * 2, 32, 2 * kTok, CU_TENSOR_MAP_SWIZZLE_64B) ||
-        !encode_2d(&mZ1, a->Z, bf, kD, rows, kD * 2, 32, kTok, CU_TENSOR_MAP_SWIZZLE_64B))
+    if (!encode_2d(&mZ, a->Z, bf, kD, rows, kD * 2, zcols, 2 * kTok, zswz) ||
+        !encode_2d(&mZ1, a->Z, bf, kD, rows, kD * 2, zcols, kTok, zswz))
         return TTT_ERR_CUDA;
-    auto k = lfr::linear_frag_kernel<LN>;
+    auto k = one ? lfr::linear_frag_kernel<LN, 1> : lfr::linear_frag_kernel<LN, 2>;
     if (!set_smem(k, lfr::kSmemBytes)) return TTT_ERR_CUDA;
-    k<<<grid, lfr::kThreads, lfr::kSmemBytes, st>>>(mQ, mK, mV, mZ, mZ1, p);
+    k<<<one ? (int)U : grid, lfr::kThreads, lfr::kSmemBytes, st>>>(mQ, mK, mV, mZ, mZ1, p);
     return launch_status();
 }
 
@@ -189,7 +193,11 @@ extern "C" ttt_status ttt_linear_forward(const ttt_linear_args* a, cudaStream_t 
             return TTT_ERR_INVALID_ARG;
         if (!(a->ln_eps > 0.f)) return TTT_ERR_INVALID_ARG;
     }
-    if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL)) return TTT_ERR_INVALID_ARG;
+    if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL | TTT_FLAG_ONE_UNIT_PER_CTA |
+                     TTT_FLAG_TWO_UNITS_PER_CTA))
+        return TTT_ERR_INVALID_ARG;
+    if ((a->flags & TTT_FLAG_ONE_UNIT_PER_CTA) && (a->flags & TTT_FLAG_TWO_UNITS_PER_CTA))
+        return TTT_ERR_INVALID_ARG;
     const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
                     !(a->flags & TTT_FLAG_FORCE_SIMT);
     if (tc) return a->use_ln ? tc_linear<true>(a, stream) : tc_linear<false>(a, stream);

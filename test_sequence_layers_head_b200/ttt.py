@@ -22,6 +22,8 @@ LIB_PATH = os.path.join(HERE, "libttt.so")
 TTT_OK, TTT_ERR_INVALID_ARG, TTT_ERR_UNSUPPORTED, TTT_ERR_CUDA, TTT_ERR_TIMEOUT = range(5)
 TTT_F32, TTT_BF16 = 0, 1
 FLAG_FORCE_SIMT = 0x1
+FLAG_ONE_UNIT_PER_CTA = 0x2
+FLAG_TWO_UNITS_PER_CTA = 0x4
 FLAG_TEST_STALL = 0x100
 
 _vp = ctypes.c_void_p

@@ -60,6 +60,7 @@ def _linear_args(ttt, **kw):
     ("eta", (1 << 20) + 8, 1),
     ("use_ln", 2, 1),
     ("flags", 0x8000, 1),
+    ("flags", 0x6, 1),     # one and two units per CTA at once
     ("W0_bstride", -1, 1),
 ])
 def test_linear_forward_rejects_invalid_arguments(ttt_lib, field, value, code):

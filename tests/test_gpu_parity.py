@@ -59,11 +59,29 @@ def check_linear(ttt, inp, use_ln=False, flags=0):
 
 @pytest.mark.parametrize("B,H,T", [(1, 1, 16), (1, 2, 48), (1, 3, 160), (2, 5, 64), (3, 3, 256)])
 @pytest.mark.parametrize("use_ln", [False, True])
-def test_linear_tc_small(ttt_lib, B, H, T, use_ln):
+@pytest.mark.parametrize("layout", ["one", "two"])
+def test_linear_tc_small(ttt_lib, B, H, T, use_ln, layout):
+    """Both CTA layouts of the tensor-core kernel (one or two units per CTA)."""
     inp = WL.random_case("ln" if use_ln else "linear", B, H, T, 64, 16, seed=B * 100 + H * 10 + T)
-    ez, ew = check_linear(ttt_lib, inp, use_ln)
+    flags = ttt_lib.FLAG_ONE_UNIT_PER_CTA if layout == "one" else ttt_lib.FLAG_TWO_UNITS_PER_CTA
+    ez, ew = check_linear(ttt_lib, inp, use_ln, flags)
     # the bf16-operand error is well below the tolerance at these sizes
     assert ez < 1e-2 and ew < 1e-2, (ez, ew)
+
+
+@pytest.mark.parametrize("use_ln", [False, True])
+def test_linear_tc_layouts_agree(ttt_lib, use_ln):
+    """One and two units per CTA run the same products in the same order (the
+    LN feature sums differ only in their summation order, which flips the
+    bf16 rounding of a few Z elements: Z is compared at 2e-3, a fraction of
+    one bf16 ulp (2^-8), the fp32 state at 1e-4)."""
+    inp = WL.random_case("ln" if use_ln else "linear", 2, 3, 224, 64, 16, seed=29)
+    Z1, W1, c1 = run_linear(ttt_lib, inp, use_ln, flags=ttt_lib.FLAG_ONE_UNIT_PER_CTA)
+    Z2, W2, c2 = run_linear(ttt_lib, inp, use_ln, flags=ttt_lib.FLAG_TWO_UNITS_PER_CTA)
+    if use_ln:
+        assert normwise(Z1, Z2) < 2e-3 and normwise(W1, W2) < 1e-4 and normwise(c1, c2) < 1e-4
+    else:
+        assert np.array_equal(Z1, Z2) and np.array_equal(W1, W2)
 
 
 @pytest.mark.parametrize("use_ln", [False, True])
