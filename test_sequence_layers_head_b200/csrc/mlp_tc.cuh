@@ -70,8 +70,9 @@ constexpr int kOffW2 = 28672;          // 2 x bf16 W2 [h][j], 128B swizzle, 256 
 constexpr int kOffHk = kOffW2 + 65536; // 2 x bf16 Hk [t][h]: 4 K-major sub-tiles of 16 x 64 (8 KB each)
 constexpr int kOffHq = kOffHk + 16384; // 2 x bf16 Hq [t][h] (8 KB each)
 constexpr int kOffE = kOffHq + 16384;  // bf16 E [t][j], 128B swizzle (2 KB)
-constexpr int kOffAE = kOffE + 2048;   // bf16 (-eta E)^T [j][t], K-major no swizzle (2 KB)
-constexpr int kOffS2 = kOffAE + 2048;  // bf16 tril(Hq Hk^T), K-major no swizzle (512 B)
+constexpr int kOffAE = kOffE + 2048;   // 2 x bf16 (-eta E)^T [j][t], K-major no swizzle (2 KB each): S5 of
+                                       // batch i reads it while E2 of batch i+1 writes the other one
+constexpr int kOffS2 = kOffAE + 4096;  // bf16 tril(Hq Hk^T + 1), K-major no swizzle (512 B)
 constexpr int kOffBar = kOffS2 + 512;
 constexpr int kNumBars = 3 * kStages + 14;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -110,10 +111,28 @@ struct Params {
 
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b_x16(taddr, r); }
 
+// ldmatrix / stmatrix x4 with transpose
+__device__ __forceinline__ void ldsm_x4_tr(uint32_t addr, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void stsm_x4_tr(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0), "r"(r1),
+                 "r"(r2), "r"(r3)
+                 : "memory");
+}
+// element e (accumulator order) of an ldmatrix.trans fragment set: n-tile nt,
+// rows r (e < 2) or r + 8, tokens 2c + (e & 1)
+__device__ __forceinline__ float frag_at(const uint32_t* f, int nt, int e) {
+    const uint32_t x = f[2 * nt + (e >> 1)];
+    return (e & 1) ? bf16_hi(x) : bf16_lo(x);
+}
+
 // 16 x 16 tril(X Y^T) with X, Y stored as [t][k] K-major 128B-swizzled
 // sub-tiles of 64 columns (nsub of them); n-tile nt (8 columns) only.
 __device__ __forceinline__ void tril_product(uint32_t xbase, uint32_t ybase, int nsub, int nt, int lane,
-                                             uint8_t* dst) {
+                                             uint8_t* dst, float add = 0.f) {
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     const int arow = (lane & 7) + 8 * ((lane >> 3) & 1);
     const int brow = 8 * nt + (lane & 7);
@@ -135,7 +154,7 @@ __device__ __forceinline__ void tril_product(uint32_t xbase, uint32_t ybase, int
     for (int hh = 0; hh < 2; ++hh) {
         const int t = r0 + 8 * hh, s = 8 * nt + c0;
         *reinterpret_cast<uint32_t*>(dst + nosw_off(t, s)) =
-            pack_bf16x2(s <= t ? acc[2 * hh] : 0.f, s + 1 <= t ? acc[2 * hh + 1] : 0.f);
+            pack_bf16x2(s <= t ? acc[2 * hh] + add : 0.f, s + 1 <= t ? acc[2 * hh + 1] + add : 0.f);
     }
 }
 
@@ -266,8 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma_bf16(tbase + cZ, make_sdesc(w2b + 2048 * ks, 1024, 1024, kSwizzle128B),
                               make_sdesc(hqb + 2048 * (ks >> 2) + 32 * (ks & 3), 16, 1024, kSwizzle128B), idS2,
                               ks > 0);
-                umma_bf16(tbase + cZ, make_sdesc(ae, 128, 256, kSwizzleNone), make_sdesc(s2, 128, 256, kSwizzleNone),
-                          idZc, 1);
+                umma_bf16(tbase + cZ, make_sdesc(ae + 2048 * (i2 & 1), 128, 256, kSwizzleNone),
+                          make_sdesc(s2, 128, 256, kSwizzleNone), idZc, 1);
                 umma_commit(d_z);
                 return true;
             };
@@ -275,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = i % kStages;
                 const uint32_t par = (i / kStages) & 1, ip = i & 1;
                 const uint32_t st = smem_u32(smem + kOffStages + s * kStageBytes);
-                const uint32_t w2b = w2 + 32768 * ip, hkb = hk + 8192 * ip;
+                const uint32_t w2b = w2 + 32768 * ip;
                 // S1
                 if (!W(&full[s], par) || !W(aw1_rdy, ip)) break;
                 tc_fence_after();
@@ -288,14 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(d_a);
                 // the previous batch's output path runs while E1 of this batch does
                 if (i >= 1 && !issue_s5(i - 1)) break;
-                // S2
-                if (!W(hk_rdy, ip) || !W(w2_rdy, ip)) break;
-                tc_fence_after();
-                for (int ks = 0; ks < 16; ++ks)
-                    umma_bf16(tbase + cE, make_sdesc(w2b + 2048 * ks, 1024, 1024, kSwizzle128B),
-                              make_sdesc(hkb + 2048 * (ks >> 2) + 32 * (ks & 3), 16, 1024, kSwizzle128B), idS2, ks > 0);
-                umma_commit(d_e);
-                // S3
+                // S3 (S2, E0 = W2^T Hk^T, runs on the epilogue warps' mma.sync)
                 if (!W(e_rdy, ip)) break;
                 tc_fence_after();
 #pragma unroll
@@ -347,8 +359,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (lane == 0) fail();
                 break;
             }
+            // tril(Hq Hk^T + 1): the "+1" carries the bias c2 updated token by token
             tril_product(smem_u32(smem + kOffHq + 8192 * (i & 1)), smem_u32(smem + kOffHk + 8192 * (i & 1)), 4, hw,
-                         lane, smem + kOffS2);
+                         lane, smem + kOffS2, 1.f);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(aux2);
@@ -366,7 +379,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* hqs = smem + kOffHq;
         uint8_t* es = smem + kOffE;
         uint8_t* aes = smem + kOffAE;
-        float c1[2], c2 = 0.f;
+        const int r = lane >> 2, c = lane & 3;   // accumulator layout: rows 16q + r (+8), tokens 2c (+1, +8, +9)
+        float c1[2], c2f[2] = {0.f, 0.f};      // c2 of rows 16q + r + 8h
         // initial state
         {
             const float* W1u = p.W1 + (size_t)pu * kD * kM;
@@ -403,7 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            if (jl) c2 = p.c2 ? p.c2[(size_t)pu * kD + j] : 0.f;
+            if (p.c2) {
+                c2f[0] = p.c2[(size_t)pu * kD + 16 * q + r];
+                c2f[1] = p.c2[(size_t)pu * kD + 16 * q + r + 8];
+            }
         }
         fence_proxy_async_smem();
         tmem_wait_st();
@@ -445,9 +462,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         };
-        float zb[16];   // c2 before the update + sum_{s<=t} (-eta_s e_s): the Z bias and "+1" term
-        // E5 of batch i2: Z = Z0 + zb -> global
-        auto finish_z = [&](int i2) {
+        float zc2 = 0.f;   // c2 of this thread's feature j before the batch's update (the Z bias;
+                           // the updates within the batch are the "+1" of tril(Hq Hk^T + 1) in S5)
+        // E5 of batch i2: Z = Z0 + c2 -> global
+        auto finish_z = [&](int i2, float zc) {
             WT(d_z, i2 & 1);
             tc_fence_after();
             uint32_t rz[16];
@@ -456,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (jl && !dead) {
 #pragma unroll
                 for (int t = 0; t < 16; ++t)
-                    Zu[(size_t)(i2 * kTok + t) * kD] = __float2bfloat16_rn(__uint_as_float(rz[t]) + zb[t]);
+                    Zu[(size_t)(i2 * kTok + t) * kD] = __float2bfloat16_rn(__uint_as_float(rz[t]) + zc);
             }
         };
         for (int i = 0; i < nsteps; ++i) {
@@ -503,40 +521,83 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(hk_rdy);
-            // the previous batch's outputs, while S2 of this batch runs
-            if (i >= 1) finish_z(i - 1);
-            // E2: E = E0 + c2 - V -> E tile, (-eta E)^T; c2 update
-            WT(d_e, ip);
-            tc_fence_after();
+            // S2 on the epilogue warps (mma.sync): E0^T = W2^T Hk^T over the 256 hidden
+            // rows, warp q rows j = 16q .. 16q + 15, accumulator layout.  Every warp's Hk
+            // rows must be in shared memory first.
+            named_bar_sync(1, 128);
+            float e0[2][4] = {};
             {
-                uint32_t re[16];
-                tmem_ld_x16(tl + cE, re);
-                tmem_wait_ld();
-                if (jl) {
-                    const uint8_t* vt = st + kOffV;
-                    float ae[16], pre = c2;
-#pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        const float e = __uint_as_float(re[t]) + c2 - ld_bf16(vt, sw128_off(t, j));
-                        *reinterpret_cast<__nv_bfloat16*>(es + sw128_off(t, j)) = __float2bfloat16_rn(e);
-                        ae[t] = -et[t] * e;
-                        pre += ae[t];
-                        zb[t] = pre;
-                    }
-                    c2 = pre;
-                    uint4 v0, v1;
-                    v0.x = pack_bf16x2(ae[0], ae[1]);
-                    v0.y = pack_bf16x2(ae[2], ae[3]);
-                    v0.z = pack_bf16x2(ae[4], ae[5]);
-                    v0.w = pack_bf16x2(ae[6], ae[7]);
-                    v1.x = pack_bf16x2(ae[8], ae[9]);
-                    v1.y = pack_bf16x2(ae[10], ae[11]);
-                    v1.z = pack_bf16x2(ae[12], ae[13]);
-                    v1.w = pack_bf16x2(ae[14], ae[15]);
-                    *reinterpret_cast<uint4*>(aes + nosw_off(j, 0)) = v0;
-                    *reinterpret_cast<uint4*>(aes + nosw_off(j, 8)) = v1;
+                const int mi = lane >> 3;
+                const uint32_t w2b = smem_u32(w2s + 32768 * ip), hkb = smem_u32(hks + 8192 * ip);
+                const int arow = 8 * (mi >> 1) + (lane & 7);                // h within the k-step
+                const int ach = 2 * q + (mi & 1);                           // 16-byte chunk of j
+                const int brow = 8 * (mi >> 1) + (lane & 7);                // token t
+#pragma unroll 4
+                for (int ks = 0; ks < 16; ++ks) {
+                    uint32_t a[4], b[4];
+                    const int h = 16 * ks + arow;
+                    ldsm_x4_tr(w2b + (h >> 3) * 1024 + (h & 7) * 128 + ((ach ^ (h & 7)) << 4), a);
+                    const int bch = 2 * (ks & 3) + (mi & 1);                // 16-byte chunk of h within its sub-tile
+                    ldsm_x4(hkb + 2048 * (ks >> 2) + brow * 128 + ((bch ^ (brow & 7)) << 4), b);
+                    mma_16816(e0[0], a, b[0], b[1]);
+                    mma_16816(e0[1], a, b[2], b[3]);
                 }
+            }
+            // E2: E = E0 + c2 - V -> E tile [t][j], (-eta E)^T [j][t]; c2 update
+            {
+                const int mi = lane >> 3;
+                const int t8 = 8 * (mi >> 1) + (lane & 7);
+                const uint32_t vt = smem_u32(st + kOffV);
+                uint32_t v[4];
+                ldsm_x4_tr(vt + t8 * 128 + (((2 * q + (mi & 1)) ^ (t8 & 7)) << 4), v);
+                // eta of tokens 2c, 2c+1, 8+2c, 9+2c (read again from the stage: indexing et[]
+                // by the lane would move it to local memory)
+                float etc[4];
+                if (p.eta) {
+                    const float* etas = reinterpret_cast<const float*>(st + kOffEta);
+                    const float2 e0v = *reinterpret_cast<const float2*>(etas + 2 * c);
+                    const float2 e1v = *reinterpret_cast<const float2*>(etas + 8 + 2 * c);
+                    etc[0] = e0v.x;
+                    etc[1] = e0v.y;
+                    etc[2] = e1v.x;
+                    etc[3] = e1v.y;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) etc[k] = p.eta_const;
+                }
+                float ev[2][4], ae[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        ev[nt][e] = e0[nt][e] + c2f[e >> 1] - frag_at(v, nt, e);
+                        ae[nt][e] = -etc[2 * nt + (e & 1)] * ev[nt][e];
+                    }
+                stsm_x4_tr(smem_u32(es) + t8 * 128 + (((2 * q + (mi & 1)) ^ (t8 & 7)) << 4),
+                           pack_bf16x2(ev[0][0], ev[0][1]), pack_bf16x2(ev[0][2], ev[0][3]),
+                           pack_bf16x2(ev[1][0], ev[1][1]), pack_bf16x2(ev[1][2], ev[1][3]));
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        *reinterpret_cast<uint32_t*>(aes + 2048 * ip + nosw_off(16 * q + r + 8 * hh, 8 * nt + 2 * c)) =
+                            pack_bf16x2(ae[nt][2 * hh], ae[nt][2 * hh + 1]);
+                // Z bias of this batch for finish_z's thread layout (feature 16q + (lane & 15))
+                const int l15 = lane & 15;
+                const float x0 = __shfl_sync(0xffffffffu, c2f[0], (l15 & 7) * 4);
+                const float x1 = __shfl_sync(0xffffffffu, c2f[1], (l15 & 7) * 4);
+                const float zc_now = l15 < 8 ? x0 : x1;
+                // c2 += sum over the batch's tokens of -eta e
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float cs = ae[0][2 * hh] + ae[0][2 * hh + 1] + ae[1][2 * hh] + ae[1][2 * hh + 1];
+                    cs += __shfl_xor_sync(0xffffffffu, cs, 1);
+                    cs += __shfl_xor_sync(0xffffffffu, cs, 2);
+                    c2f[hh] += cs;
+                }
+                // the previous batch's outputs go out first (its bias is zc2), then keep this one's
+                if (i >= 1) finish_z(i - 1, zc2);
+                zc2 = zc_now;
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -616,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(w2_rdy);
         }
-        if (nsteps >= 1) finish_z(nsteps - 1);
+        if (nsteps >= 1) finish_z(nsteps - 1, zc2);
         // final state (after the last S4; W1^T / W2 accumulators in TMEM)
         if (!dead) {
             float* W1o = p.W1_out + (size_t)unit * kD * kM;
@@ -638,7 +699,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (p.c1_out) p.c1_out[(size_t)unit * kM + h] = c1[tt];
             }
-            if (jl && p.c2_out) p.c2_out[(size_t)unit * kD + j] = c2;
+            if (p.c2_out && c == 0) {
+                p.c2_out[(size_t)unit * kD + 16 * q + r] = c2f[0];
+                p.c2_out[(size_t)unit * kD + 16 * q + r + 8] = c2f[1];
+            }
         }
     }
     tc_fence_before();
