@@ -506,8 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int t = 0; t < 16; ++t) {
                         const float a = __uint_as_float(ra[tt][t]) + c1[tt];
-                        const float hk = gelu_f(a);
-                        gp[tt][t] = gelu_grad_f(a);
+                        float hk;
+                        gelu_and_grad_fast(a, hk, gp[tt][t]);
                         *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(t, h & 63)) = __float2bfloat16_rn(hk);
                         ah[t] = -et[t] * hk;
                     }
@@ -666,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int t = 0; t < 16; ++t)
                         *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(t, h & 63)) =
-                            __float2bfloat16_rn(gelu_f(__uint_as_float(rq[tt][t]) + aqb[tt][t]));
+                            __float2bfloat16_rn(gelu_fast(__uint_as_float(rq[tt][t]) + aqb[tt][t]));
                 }
             }
             fence_proxy_async_smem();
