@@ -54,7 +54,7 @@ using tcc::umma_ts;
 
 constexpr int kD = 64, kM = 256, kTok = 16;
 constexpr int kStages = 4;
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // 8 epilogue warps (0-3, 8-11), producer 4, MMA 5, helpers 6-7
 constexpr int kTile = kTok * kD * 2;   // 2048
 
 // stage layout
@@ -73,7 +73,8 @@ constexpr int kOffE = kOffHq + 16384;  // bf16 E [t][j], 128B swizzle (2 KB)
 constexpr int kOffAE = kOffE + 2048;   // 2 x bf16 (-eta E)^T [j][t], K-major no swizzle (2 KB each): S5 of
                                        // batch i reads it while E2 of batch i+1 writes the other one
 constexpr int kOffS2 = kOffAE + 4096;  // bf16 tril(Hq Hk^T + 1), K-major no swizzle (512 B)
-constexpr int kOffBar = kOffS2 + 512;
+constexpr int kOffXch = kOffS2 + 512;  // two buffers x [2 halves][4 quadrants][4][32] float2 (partial sums)
+constexpr int kOffBar = kOffXch + 2 * 1024 * 8;
 constexpr int kNumBars = 3 * kStages + 14;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
 constexpr int kSmemBytes = kOffMisc + 64;
@@ -121,6 +122,26 @@ __device__ __forceinline__ void stsm_x4_tr(uint32_t addr, uint32_t r0, uint32_t 
     asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r0), "r"(r1),
                  "r"(r2), "r"(r3)
                  : "memory");
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_tr(uint32_t addr, uint32_t* r) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(addr));
+}
+__device__ __forceinline__ void stsm_x2_tr(uint32_t addr, uint32_t r0, uint32_t r1) {
+    asm volatile("stmatrix.sync.aligned.m8n8.x2.trans.shared.b16 [%0], {%1,%2};" ::"r"(addr), "r"(r0), "r"(r1)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
 }
 // element e (accumulator order) of an ldmatrix.trans fragment set: n-tile nt,
 // rows r (e < 2) or r + 8, tokens 2c + (e & 1)
@@ -195,17 +216,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 5);
+            mbar_init(&empty[s], 9);
             mbar_init(&aux1[s], 1);
         }
         for (uint64_t* b = d_a; b <= d_z; ++b) mbar_init(b, 1);
-        mbar_init(hk_rdy, 4);
-        mbar_init(e_rdy, 4);
-        mbar_init(d1_rdy, 4);
-        mbar_init(hq_rdy, 4);
+        mbar_init(hk_rdy, 8);
+        mbar_init(e_rdy, 8);
+        mbar_init(d1_rdy, 8);
+        mbar_init(hq_rdy, 8);
         mbar_init(aux2, 2);
-        mbar_init(aw1_rdy, 4);
-        mbar_init(w2_rdy, 4);
+        mbar_init(aw1_rdy, 8);
+        mbar_init(w2_rdy, 8);
         mbar_init(drain, 1);
         mbar_init(stall, 1);
         *s_abort = 0;
@@ -336,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(drain);
             if (!wait_bounded(drain, 0, lim, nullptr)) fail();
         }
-    } else if (warp >= 6) {
+    } else if (warp == 6 || warp == 7) {
         // ------------------------------------------------------------ helpers
         const int hw = warp - 6;
         for (int i = 0; i < nsteps; ++i) {
@@ -348,8 +369,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (lane == 0) fail();
                     break;
                 }
-                tril_product(smem_u32(st + kOffQ), smem_u32(st + kOffK), 1, 0, lane, st + kOffS1);
-                tril_product(smem_u32(st + kOffQ), smem_u32(st + kOffK), 1, 1, lane, st + kOffS1);
+                // tril(Q K^T + 1): the "+1" carries the bias c1 updated token by token into Aq
+                tril_product(smem_u32(st + kOffQ), smem_u32(st + kOffK), 1, 0, lane, st + kOffS1, 1.f);
+                tril_product(smem_u32(st + kOffQ), smem_u32(st + kOffK), 1, 1, lane, st + kOffS1, 1.f);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&aux1[s]);
@@ -368,20 +390,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------------------------------ epilogue
-        const int q = warp;
-        const int hr[2] = {32 * q + lane, 128 + 32 * q + lane};   // hidden rows of this thread
-        const bool jl = lane < 16;                                // owns a feature row in d-sized stages
-        const int j = 16 * q + (lane & 15);
+        // Warps 0-3 and 8-11.  Warp w reads TMEM lane quadrant qd = w & 3 (hidden
+        // rows h = 32 qd + lane of each 128-row tile) and takes the tokens of its
+        // half hf = w >> 3 (8 hf .. 8 hf + 7) in every elementwise stage, and
+        // the m16 x n8 tile (features 16 qd .., tokens of its half) in the
+        // d-sized stages.
+        const int qd = warp & 3, hf = warp >> 3;
+        const int hr[2] = {32 * qd + lane, 128 + 32 * qd + lane};   // hidden rows of this thread
+        const bool jl = lane < 16;                                  // M = 64 stages: feature row of this lane
+        const int j = 16 * qd + (lane & 15);
         const int pu = p.per_seq ? unit : unit % p.H;
-        const uint32_t tl = tbase + ((uint32_t)(32 * q) << 16);
+        const uint32_t tl = tbase + ((uint32_t)(32 * qd) << 16);
         uint8_t* w2s = smem + kOffW2;
         uint8_t* hks = smem + kOffHk;
         uint8_t* hqs = smem + kOffHq;
         uint8_t* es = smem + kOffE;
         uint8_t* aes = smem + kOffAE;
-        const int r = lane >> 2, c = lane & 3;   // accumulator layout: rows 16q + r (+8), tokens 2c (+1, +8, +9)
-        float c1[2], c2f[2] = {0.f, 0.f};      // c2 of rows 16q + r + 8h
-        // initial state
+        float2* xch = reinterpret_cast<float2*>(smem + kOffXch);   // partial sums of the two token halves
+        const int r = lane >> 2, c = lane & 3;   // accumulator layout: rows 16 qd + r (+8), tokens 8 hf + 2c (+1)
+        float c1[2], c2f[2] = {0.f, 0.f};        // c1 of rows hr; c2 of rows 16 qd + r + 8 hh
+        // initial state: this warp writes columns 32 hf .. 32 hf + 31 of W1^T and W2
         {
             const float* W1u = p.W1 + (size_t)pu * kD * kM;
             const float* W2u = p.W2 + (size_t)pu * kM * kD;
@@ -391,35 +419,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 c1[tt] = p.c1 ? p.c1[(size_t)pu * kM + h] : 0.f;
                 uint32_t w[32], pk[16];
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
+                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(W1u[(size_t)(32 * hf + i) * kM + h]);
+                tmem_st_32x32b_x32(tl + cW1 + 64 * tt + 32 * hf, w);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(W1u[(size_t)(32 * half + i) * kM + h]);
-                    tmem_st_32x32b_x32(tl + cW1 + 64 * tt + 32 * half, w);
+                for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(__uint_as_float(w[2 * k]), __uint_as_float(w[2 * k + 1]));
+                tmem_st_32x32b_x16(tl + cAW1 + 32 * tt + 16 * hf, pk);
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        pk[c] = pack_bf16x2(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
-                    tmem_st_32x32b_x16(tl + cAW1 + 32 * tt + 16 * half, pk);
-                }
+                for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(W2u[(size_t)h * kD + 32 * hf + i]);
+                tmem_st_32x32b_x32(tl + cW2 + 64 * tt + 32 * hf, w);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(W2u[(size_t)h * kD + 32 * half + i]);
-                    tmem_st_32x32b_x32(tl + cW2 + 64 * tt + 32 * half, w);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(w[8 * c + 0]), __uint_as_float(w[8 * c + 1]));
-                        v.y = pack_bf16x2(__uint_as_float(w[8 * c + 2]), __uint_as_float(w[8 * c + 3]));
-                        v.z = pack_bf16x2(__uint_as_float(w[8 * c + 4]), __uint_as_float(w[8 * c + 5]));
-                        v.w = pack_bf16x2(__uint_as_float(w[8 * c + 6]), __uint_as_float(w[8 * c + 7]));
-                        const int ch = 4 * half + c;
-                        *reinterpret_cast<uint4*>(w2s + (h >> 3) * 1024 + (h & 7) * 128 + ((ch ^ (h & 7)) << 4)) = v;
-                    }
+                for (int k = 0; k < 4; ++k) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(w[8 * k + 0]), __uint_as_float(w[8 * k + 1]));
+                    v.y = pack_bf16x2(__uint_as_float(w[8 * k + 2]), __uint_as_float(w[8 * k + 3]));
+                    v.z = pack_bf16x2(__uint_as_float(w[8 * k + 4]), __uint_as_float(w[8 * k + 5]));
+                    v.w = pack_bf16x2(__uint_as_float(w[8 * k + 6]), __uint_as_float(w[8 * k + 7]));
+                    const int ch = 4 * hf + k;
+                    *reinterpret_cast<uint4*>(w2s + (h >> 3) * 1024 + (h & 7) * 128 + ((ch ^ (h & 7)) << 4)) = v;
                 }
             }
             if (p.c2) {
-                c2f[0] = p.c2[(size_t)pu * kD + 16 * q + r];
-                c2f[1] = p.c2[(size_t)pu * kD + 16 * q + r + 8];
+                c2f[0] = p.c2[(size_t)pu * kD + 16 * qd + r];
+                c2f[1] = p.c2[(size_t)pu * kD + 16 * qd + r + 8];
             }
         }
         fence_proxy_async_smem();
@@ -438,43 +459,53 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         };
         __nv_bfloat16* Zu = p.Z + (size_t)unit * p.T * kD + j;
-        // bf16 W2 (state after batch i's update) -> buffer (i+1)&1, row h of each tile
+        // bf16 W2 (state after batch i's update) -> buffer buf: this warp's 32 columns of row h
         auto refresh_w2 = [&](int buf) {
             uint8_t* dst = w2s + 32768 * buf;
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
                 const int h = hr[tt];
+                uint32_t w[32];
+                tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * hf, w);
+                tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t w[32];
-                    tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * half, w);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(w[8 * c + 0]), __uint_as_float(w[8 * c + 1]));
-                        v.y = pack_bf16x2(__uint_as_float(w[8 * c + 2]), __uint_as_float(w[8 * c + 3]));
-                        v.z = pack_bf16x2(__uint_as_float(w[8 * c + 4]), __uint_as_float(w[8 * c + 5]));
-                        v.w = pack_bf16x2(__uint_as_float(w[8 * c + 6]), __uint_as_float(w[8 * c + 7]));
-                        const int ch = 4 * half + c;
-                        *reinterpret_cast<uint4*>(dst + (h >> 3) * 1024 + (h & 7) * 128 + ((ch ^ (h & 7)) << 4)) = v;
-                    }
+                for (int k = 0; k < 4; ++k) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(w[8 * k + 0]), __uint_as_float(w[8 * k + 1]));
+                    v.y = pack_bf16x2(__uint_as_float(w[8 * k + 2]), __uint_as_float(w[8 * k + 3]));
+                    v.z = pack_bf16x2(__uint_as_float(w[8 * k + 4]), __uint_as_float(w[8 * k + 5]));
+                    v.w = pack_bf16x2(__uint_as_float(w[8 * k + 6]), __uint_as_float(w[8 * k + 7]));
+                    const int ch = 4 * hf + k;
+                    *reinterpret_cast<uint4*>(dst + (h >> 3) * 1024 + (h & 7) * 128 + ((ch ^ (h & 7)) << 4)) = v;
                 }
             }
         };
-        float zc2 = 0.f;   // c2 of this thread's feature j before the batch's update (the Z bias;
-                           // the updates within the batch are the "+1" of tril(Hq Hk^T + 1) in S5)
-        // E5 of batch i2: Z = Z0 + c2 -> global
+        float zc2 = 0.f;   // c2 of feature j before the batch's update (the Z bias; the updates
+                           // within the batch are the "+1" of tril(Hq Hk^T + 1) in S5)
+        // E5 of batch i2: Z = Z0 + c2 -> global, this warp's 8 tokens
         auto finish_z = [&](int i2, float zc) {
             WT(d_z, i2 & 1);
             tc_fence_after();
-            uint32_t rz[16];
-            tmem_ld_x16(tl + cZ, rz);
+            uint32_t rz[8];
+            tmem_ld_32x32b_x8(tl + cZ + 8 * hf, rz);
             tmem_wait_ld();
             if (jl && !dead) {
 #pragma unroll
-                for (int t = 0; t < 16; ++t)
-                    Zu[(size_t)(i2 * kTok + t) * kD] = __float2bfloat16_rn(__uint_as_float(rz[t]) + zc);
+                for (int t = 0; t < 8; ++t)
+                    Zu[(size_t)(i2 * kTok + 8 * hf + t) * kD] = __float2bfloat16_rn(__uint_as_float(rz[t]) + zc);
+            }
+        };
+        int nx = 0;   // exchanges of partial sums so far (two alternating buffers)
+        // the other token half's partial sums of this warp's rows: a[k] += other's
+        auto exchange2 = [&](float* a, int n) {
+            float2* buf = xch + (nx & 1) * 1024;
+            ++nx;
+            for (int k = 0; k < n; k += 2) buf[(hf * 4 + qd) * 128 + (k >> 1) * 32 + lane] = make_float2(a[k], a[k + 1]);
+            named_bar_sync(2, 256);
+            for (int k = 0; k < n; k += 2) {
+                const float2 o = buf[((1 - hf) * 4 + qd) * 128 + (k >> 1) * 32 + lane];
+                a[k] += o.x;
+                a[k + 1] += o.y;
             }
         };
         for (int i = 0; i < nsteps; ++i) {
@@ -482,39 +513,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t par = (i / kStages) & 1, ip = i & 1;
             const uint8_t* st = smem + kOffStages + s * kStageBytes;
             WT(&full[s], par);
-            float et[16];
+            float et[8];   // eta of this warp's tokens
             {
                 const float* etas = reinterpret_cast<const float*>(st + kOffEta);
 #pragma unroll
-                for (int t = 0; t < 16; ++t) et[t] = p.eta ? etas[t] : p.eta_const;
+                for (int t = 0; t < 8; ++t) et[t] = p.eta ? etas[8 * hf + t] : p.eta_const;
             }
-            // E1: A -> Hk, GELU'(A); keep Aq0
+            // E1: A -> Hk, GELU'(A)
             WT(d_a, ip);
             tc_fence_after();
-            float gp[2][16];
+            float gp[2][8];
             {
-                uint32_t ra[2][32];
-                tmem_ld_32x32b_x32(tl + cA, ra[0]);
-                tmem_ld_32x32b_x32(tl + cA + 32, ra[1]);
+                uint32_t ra[2][8];
+                tmem_ld_32x32b_x8(tl + cA + 8 * hf, ra[0]);
+                tmem_ld_32x32b_x8(tl + cA + 32 + 8 * hf, ra[1]);
                 tmem_wait_ld();
                 uint8_t* hkb = hks + 8192 * ip;
 #pragma unroll
                 for (int tt = 0; tt < 2; ++tt) {
                     const int h = hr[tt];
                     uint8_t* sub = hkb + 2048 * (h >> 6);
-                    float ah[16];
+                    float ah[8];
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) {
+                    for (int t = 0; t < 8; ++t) {
                         const float a = __uint_as_float(ra[tt][t]) + c1[tt];
                         float hk;
                         gelu_and_grad_fast(a, hk, gp[tt][t]);
-                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(t, h & 63)) = __float2bfloat16_rn(hk);
+                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(8 * hf + t, h & 63)) = __float2bfloat16_rn(hk);
                         ah[t] = -et[t] * hk;
                     }
-                    uint32_t pa[8];
+                    uint32_t pa[4];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) pa[c] = pack_bf16x2(ah[2 * c], ah[2 * c + 1]);
-                    tmem_st_32x32b_x8(tl + cAHk + 8 * tt, pa);
+                    for (int k = 0; k < 4; ++k) pa[k] = pack_bf16x2(ah[2 * k], ah[2 * k + 1]);
+                    tmem_st_32x32b_x4(tl + cAHk + 8 * tt + 4 * hf, pa);
                 }
             }
             fence_proxy_async_smem();
@@ -522,79 +553,69 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             // S2 on the epilogue warps (mma.sync): E0^T = W2^T Hk^T over the 256 hidden
-            // rows, warp q rows j = 16q .. 16q + 15, accumulator layout.  Every warp's Hk
-            // rows must be in shared memory first.
-            named_bar_sync(1, 128);
-            float e0[2][4] = {};
+            // rows; this warp: features 16 qd .. 16 qd + 15, tokens of its half.  Every
+            // warp's Hk must be in shared memory first.
+            named_bar_sync(1, 256);
+            float e0[4] = {0.f, 0.f, 0.f, 0.f};
             {
                 const int mi = lane >> 3;
                 const uint32_t w2b = smem_u32(w2s + 32768 * ip), hkb = smem_u32(hks + 8192 * ip);
-                const int arow = 8 * (mi >> 1) + (lane & 7);                // h within the k-step
-                const int ach = 2 * q + (mi & 1);                           // 16-byte chunk of j
-                const int brow = 8 * (mi >> 1) + (lane & 7);                // token t
+                const int arow = 8 * (mi >> 1) + (lane & 7);   // h within the k-step
+                const int ach = 2 * qd + (mi & 1);             // 16-byte chunk of j
+                const int brow = 8 * hf + (lane & 7);          // token t (lanes 0-15 give the addresses)
 #pragma unroll 4
                 for (int ks = 0; ks < 16; ++ks) {
-                    uint32_t a[4], b[4];
+                    uint32_t a[4], b[2];
                     const int h = 16 * ks + arow;
                     ldsm_x4_tr(w2b + (h >> 3) * 1024 + (h & 7) * 128 + ((ach ^ (h & 7)) << 4), a);
-                    const int bch = 2 * (ks & 3) + (mi & 1);                // 16-byte chunk of h within its sub-tile
-                    ldsm_x4(hkb + 2048 * (ks >> 2) + brow * 128 + ((bch ^ (brow & 7)) << 4), b);
-                    mma_16816(e0[0], a, b[0], b[1]);
-                    mma_16816(e0[1], a, b[2], b[3]);
+                    const int bch = 2 * (ks & 3) + ((lane >> 3) & 1);   // 16-byte chunk of h in its sub-tile
+                    ldsm_x2(hkb + 2048 * (ks >> 2) + brow * 128 + ((bch ^ (brow & 7)) << 4), b);
+                    mma_16816(e0, a, b[0], b[1]);
                 }
             }
             // E2: E = E0 + c2 - V -> E tile [t][j], (-eta E)^T [j][t]; c2 update
             {
-                const int mi = lane >> 3;
-                const int t8 = 8 * (mi >> 1) + (lane & 7);
+                const int t8 = 8 * hf + (lane & 7);
                 const uint32_t vt = smem_u32(st + kOffV);
-                uint32_t v[4];
-                ldsm_x4_tr(vt + t8 * 128 + (((2 * q + (mi & 1)) ^ (t8 & 7)) << 4), v);
-                // eta of tokens 2c, 2c+1, 8+2c, 9+2c (read again from the stage: indexing et[]
-                // by the lane would move it to local memory)
-                float etc[4];
+                uint32_t v[2];
+                ldsm_x2_tr(vt + t8 * 128 + (((2 * qd + ((lane >> 3) & 1)) ^ (t8 & 7)) << 4), v);
+                float etc[2];
                 if (p.eta) {
-                    const float* etas = reinterpret_cast<const float*>(st + kOffEta);
-                    const float2 e0v = *reinterpret_cast<const float2*>(etas + 2 * c);
-                    const float2 e1v = *reinterpret_cast<const float2*>(etas + 8 + 2 * c);
+                    const float2 e0v = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(st + kOffEta) +
+                                                                        8 * hf + 2 * c);
                     etc[0] = e0v.x;
                     etc[1] = e0v.y;
-                    etc[2] = e1v.x;
-                    etc[3] = e1v.y;
                 } else {
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) etc[k] = p.eta_const;
+                    etc[0] = etc[1] = p.eta_const;
                 }
-                float ev[2][4], ae[2][4];
+                float ev[4], ae[4];
 #pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
+                for (int e = 0; e < 4; ++e) {
+                    ev[e] = e0[e] + c2f[e >> 1] - frag_at(v, 0, e);
+                    ae[e] = -etc[e & 1] * ev[e];
+                }
+                stsm_x2_tr(smem_u32(es) + t8 * 128 + (((2 * qd + ((lane >> 3) & 1)) ^ (t8 & 7)) << 4),
+                           pack_bf16x2(ev[0], ev[1]), pack_bf16x2(ev[2], ev[3]));
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        ev[nt][e] = e0[nt][e] + c2f[e >> 1] - frag_at(v, nt, e);
-                        ae[nt][e] = -etc[2 * nt + (e & 1)] * ev[nt][e];
-                    }
-                stsm_x4_tr(smem_u32(es) + t8 * 128 + (((2 * q + (mi & 1)) ^ (t8 & 7)) << 4),
-                           pack_bf16x2(ev[0][0], ev[0][1]), pack_bf16x2(ev[0][2], ev[0][3]),
-                           pack_bf16x2(ev[1][0], ev[1][1]), pack_bf16x2(ev[1][2], ev[1][3]));
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh)
-                        *reinterpret_cast<uint32_t*>(aes + 2048 * ip + nosw_off(16 * q + r + 8 * hh, 8 * nt + 2 * c)) =
-                            pack_bf16x2(ae[nt][2 * hh], ae[nt][2 * hh + 1]);
-                // Z bias of this batch for finish_z's thread layout (feature 16q + (lane & 15))
+                for (int hh = 0; hh < 2; ++hh)
+                    *reinterpret_cast<uint32_t*>(aes + 2048 * ip + nosw_off(16 * qd + r + 8 * hh, 8 * hf + 2 * c)) =
+                        pack_bf16x2(ae[2 * hh], ae[2 * hh + 1]);
+                // Z bias of this batch for finish_z's thread layout (feature 16 qd + (lane & 15))
                 const int l15 = lane & 15;
                 const float x0 = __shfl_sync(0xffffffffu, c2f[0], (l15 & 7) * 4);
                 const float x1 = __shfl_sync(0xffffffffu, c2f[1], (l15 & 7) * 4);
                 const float zc_now = l15 < 8 ? x0 : x1;
-                // c2 += sum over the batch's tokens of -eta e
+                // c2 += sum over the batch's 16 tokens of -eta e (this half, then the other's)
+                float cs[2];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    float cs = ae[0][2 * hh] + ae[0][2 * hh + 1] + ae[1][2 * hh] + ae[1][2 * hh + 1];
-                    cs += __shfl_xor_sync(0xffffffffu, cs, 1);
-                    cs += __shfl_xor_sync(0xffffffffu, cs, 2);
-                    c2f[hh] += cs;
+                    cs[hh] = ae[2 * hh] + ae[2 * hh + 1];
+                    cs[hh] += __shfl_xor_sync(0xffffffffu, cs[hh], 1);
+                    cs[hh] += __shfl_xor_sync(0xffffffffu, cs[hh], 2);
                 }
+                exchange2(cs, 2);
+                c2f[0] += cs[0];
+                c2f[1] += cs[1];
                 // the previous batch's outputs go out first (its bias is zc2), then keep this one's
                 if (i >= 1) finish_z(i - 1, zc2);
                 zc2 = zc_now;
@@ -609,50 +630,51 @@ __global__ void __launch_bounds__(kThreads, 1)
             // E3: D1 = G * GELU'(A) -> (-eta D1)^T; c1 update
             WT(d_g, ip);
             tc_fence_after();
-            float aqb[2][16];   // c1 before the update + sum_{s<=t} (-eta_s d1_s)
+            float c1_old[2] = {c1[0], c1[1]};
             {
-                uint32_t rg[2][16];
-                tmem_ld_x16(tl + cG, rg[0]);
-                tmem_ld_x16(tl + cG + 16, rg[1]);
+                uint32_t rg[2][8];
+                tmem_ld_32x32b_x8(tl + cG + 8 * hf, rg[0]);
+                tmem_ld_32x32b_x8(tl + cG + 16 + 8 * hf, rg[1]);
                 tmem_wait_ld();
+                float csum[2];
 #pragma unroll
                 for (int tt = 0; tt < 2; ++tt) {
-                    float ad[16], pre = c1[tt];
+                    float ad[8], sum = 0.f;
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) {
+                    for (int t = 0; t < 8; ++t) {
                         ad[t] = -et[t] * __uint_as_float(rg[tt][t]) * gp[tt][t];
-                        pre += ad[t];
-                        aqb[tt][t] = pre;
+                        sum += ad[t];
                     }
-                    c1[tt] = pre;
-                    uint32_t pa[8];
+                    csum[tt] = sum;
+                    uint32_t pa[4];
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) pa[c] = pack_bf16x2(ad[2 * c], ad[2 * c + 1]);
-                    tmem_st_32x32b_x8(tl + cAD1 + 8 * tt, pa);
+                    for (int k = 0; k < 4; ++k) pa[k] = pack_bf16x2(ad[2 * k], ad[2 * k + 1]);
+                    tmem_st_32x32b_x4(tl + cAD1 + 8 * tt + 4 * hf, pa);
                 }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(d1_rdy);
+                exchange2(csum, 2);
+                c1[0] += csum[0];
+                c1[1] += csum[1];
             }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(d1_rdy);
-            // E4: bf16 W1^T for the next S1 first, then Hq = GELU(Aq) -> Hq^T, then bf16 W2
+            // E4: bf16 W1^T for the next S1 first, then Hq = GELU(Aq + c1) -> Hq^T
+            // (Aq carries the batch's bias updates through tril(Q K^T + 1)), then bf16 W2
             WT(d_u, ip);
             tc_fence_after();
-            uint32_t rq[2][16];
-            tmem_ld_x16(tl + cA + 16, rq[0]);
-            tmem_ld_x16(tl + cA + 32 + 16, rq[1]);
+            uint32_t rq[2][8];
+            tmem_ld_32x32b_x8(tl + cA + 16 + 8 * hf, rq[0]);
+            tmem_ld_32x32b_x8(tl + cA + 32 + 16 + 8 * hf, rq[1]);
 #pragma unroll
-            for (int tt = 0; tt < 2; ++tt)
+            for (int tt = 0; tt < 2; ++tt) {
+                uint32_t w[32], pk[16];
+                tmem_ld_32x32b_x32(tl + cW1 + 64 * tt + 32 * hf, w);
+                tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t w[32], pk[16];
-                    tmem_ld_32x32b_x32(tl + cW1 + 64 * tt + 32 * half, w);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        pk[c] = pack_bf16x2(__uint_as_float(w[2 * c]), __uint_as_float(w[2 * c + 1]));
-                    tmem_st_32x32b_x16(tl + cAW1 + 32 * tt + 16 * half, pk);
-                }
+                for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(__uint_as_float(w[2 * k]), __uint_as_float(w[2 * k + 1]));
+                tmem_st_32x32b_x16(tl + cAW1 + 32 * tt + 16 * hf, pk);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -664,9 +686,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int h = hr[tt];
                     uint8_t* sub = hqb + 2048 * (h >> 6);
 #pragma unroll
-                    for (int t = 0; t < 16; ++t)
-                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(t, h & 63)) =
-                            __float2bfloat16_rn(gelu_fast(__uint_as_float(rq[tt][t]) + aqb[tt][t]));
+                    for (int t = 0; t < 8; ++t)
+                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(8 * hf + t, h & 63)) =
+                            __float2bfloat16_rn(gelu_fast(__uint_as_float(rq[tt][t]) + c1_old[tt]));
                 }
             }
             fence_proxy_async_smem();
@@ -678,30 +700,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) mbar_arrive(w2_rdy);
         }
         if (nsteps >= 1) finish_z(nsteps - 1, zc2);
-        // final state (after the last S4; W1^T / W2 accumulators in TMEM)
+        // final state (after the last S4; W1^T / W2 accumulators in TMEM): this warp's columns
         if (!dead) {
             float* W1o = p.W1_out + (size_t)unit * kD * kM;
             float* W2o = p.W2_out + (size_t)unit * kM * kD;
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
                 const int h = hr[tt];
+                uint32_t w[32];
+                tmem_ld_32x32b_x32(tl + cW1 + 64 * tt + 32 * hf, w);
+                tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t w[32];
-                    tmem_ld_32x32b_x32(tl + cW1 + 64 * tt + 32 * half, w);
-                    tmem_wait_ld();
+                for (int k = 0; k < 32; ++k) W1o[(size_t)(32 * hf + k) * kM + h] = __uint_as_float(w[k]);
+                tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * hf, w);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) W1o[(size_t)(32 * half + i) * kM + h] = __uint_as_float(w[i]);
-                    tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * half, w);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) W2o[(size_t)h * kD + 32 * half + i] = __uint_as_float(w[i]);
-                }
-                if (p.c1_out) p.c1_out[(size_t)unit * kM + h] = c1[tt];
+                for (int k = 0; k < 32; ++k) W2o[(size_t)h * kD + 32 * hf + k] = __uint_as_float(w[k]);
+                if (p.c1_out && hf == 0) p.c1_out[(size_t)unit * kM + h] = c1[tt];
             }
-            if (p.c2_out && c == 0) {
-                p.c2_out[(size_t)unit * kD + 16 * q + r] = c2f[0];
-                p.c2_out[(size_t)unit * kD + 16 * q + r + 8] = c2f[1];
+            if (p.c2_out && c == 0 && hf == 0) {
+                p.c2_out[(size_t)unit * kD + 16 * qd + r] = c2f[0];
+                p.c2_out[(size_t)unit * kD + 16 * qd + r + 8] = c2f[1];
             }
         }
     }
