@@ -563,15 +563,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int arow = 8 * (mi >> 1) + (lane & 7);   // h within the k-step
                 const int ach = 2 * qd + (mi & 1);             // 16-byte chunk of j
                 const int brow = 8 * hf + (lane & 7);          // token t (lanes 0-15 give the addresses)
-#pragma unroll 4
+                // four independent accumulators (k-steps mod 4) keep the mma.sync chains short
+                float acc[4][4] = {};
+#pragma unroll
                 for (int ks = 0; ks < 16; ++ks) {
                     uint32_t a[4], b[2];
                     const int h = 16 * ks + arow;
                     ldsm_x4_tr(w2b + (h >> 3) * 1024 + (h & 7) * 128 + ((ach ^ (h & 7)) << 4), a);
                     const int bch = 2 * (ks & 3) + ((lane >> 3) & 1);   // 16-byte chunk of h in its sub-tile
                     ldsm_x2(hkb + 2048 * (ks >> 2) + brow * 128 + ((bch ^ (brow & 7)) << 4), b);
-                    mma_16816(e0, a, b[0], b[1]);
+                    mma_16816(acc[ks & 3], a, b[0], b[1]);
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) e0[e] = (acc[0][e] + acc[1][e]) + (acc[2][e] + acc[3][e]);
             }
             // E2: E = E0 + c2 - V -> E tile [t][j], (-eta E)^T [j][t]; c2 update
             {
