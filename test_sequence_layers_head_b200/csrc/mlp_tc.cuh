@@ -12,29 +12,35 @@
 //
 // Mapping onto sm_100a (everything transposed so that the hidden dim m = 256
 // or the head dim d = 64 is the MMA's M):
-//   S1  [A^T | Aq0^T] (m x 32)  = W1^T . [K^T | Q^T]           2 tiles x 4 k-steps
-//   S2  E0^T (d x 16)           = W2^T . Hk^T                  16 k-steps (K = m)
-//   S3  G^T (m x 16)            = W2 . E^T                     2 tiles x 4 k-steps
-//   S4  W1^T += (-eta D1)^T K,  Aq^T += (-eta D1)^T tril(Q K^T)^T,
-//       W2   += (-eta Hk)^T E                                  6 MMAs
-//   S5  Z0^T (d x 16)           = W2^T . Hq^T + (-eta E)^T tril(Hq Hk^T)^T
+//   S1  [A^T | Aq0^T] (m x 32)  = W1^T . [K^T | Q^T]           tcgen05, 2 tiles x 4 k-steps
+//   S2  E0^T (d x 16)           = W2^T . Hk^T                  mma.sync on the epilogue warps
+//   S3  G^T (m x 16)            = W2 . E^T                     mma.sync on the epilogue warps
+//   S4  W1^T += (-eta D1)^T K,  Aq^T += (-eta D1)^T tril(Q K^T + 1)^T,
+//       W2   += (-eta Hk)^T E                                  tcgen05, 6 MMAs
+//   S5  Z0^T (d x 16)           = W2^T . Hq^T + (-eta E)^T tril(Hq Hk^T + 1)^T   tcgen05
 // The fp32 accumulators W1^T (m x d) and W2 (m x d) stay in tensor memory for
 // the whole sequence; bf16 W1^T is refreshed in tensor memory (A operand of
-// S1) and bf16 W2 in shared memory (A operand of S2/S5 as MN-major, of S3 as
-// K-major) once per mini-batch.  The "+1" bias terms of the causal matrices,
-// the biases and GELU are applied in fp32 registers by the epilogue; the
-// 16 x 16 products Q K^T and Hq Hk^T (below tcgen05's M range) are computed
-// by two helper warps with mma.sync.
+// S1) and bf16 W2 in shared memory (A operand of S5 as MN-major, of S2/S3 as
+// ldmatrix fragments) once per mini-batch.  S2 and S3 have N = 16 tokens, too
+// narrow for a tcgen05 round trip (issue, commit, wake-up) to pay, so the
+// epilogue warps run them on mma.sync and keep E0, G and GELU'(A) in the
+// accumulator fragment layout, which is also what tcgen05.ld.16x256b returns
+// for A: D1 = G * GELU'(A) needs no exchange.  The "+1" bias terms of the
+// causal matrices, the biases and GELU are applied in fp32 registers by the
+// epilogue; the 16 x 16 products Q K^T and Hq Hk^T are computed by two helper
+// warps with mma.sync.
 //
 // The output path of a mini-batch (Hq, S5, Z) is software-pipelined behind
 // the next mini-batch's S1/E1: bf16 W2, Hk and Hq are double-buffered so S5
 // of batch i reads the state of batch i while S2 of batch i+1 reads the next.
 //
-// One unit per CTA.  Warps 0-3: epilogue (warp q reads TMEM lanes 32q..32q+31;
-// thread owns hidden rows h = 32q + lane and 128 + 32q + lane, and for the
-// d-sized stages feature j = 16q + lane, lane < 16); warp 4 TMA producer;
-// warp 5 MMA issuer; warps 6-7 helpers.  Every wait is bounded; on expiry
-// the kernel records kStatusTimeout, drains what it issued and returns.
+// One unit per CTA, 12 warps.  Epilogue warps 0-3 and 8-11: warp w reads TMEM
+// lanes 32 (w & 3) .. + 31 (its quadrant) and covers the tokens 8 (w >> 3) .. + 7
+// of the mini-batch; in the fragment layout lane (r, c) = (lane / 4, lane % 4)
+// holds hidden rows 128 tt + 32 (w & 3) + 16 m + r (+ 8) and tokens 2c, 2c + 1
+// of that half.  Warp 4 TMA producer; warp 5 MMA issuer; warps 6-7 helpers.
+// Every wait is bounded; on expiry the kernel records kStatusTimeout, drains
+// what it issued and returns.
 #pragma once
 #include "common.cuh"
 #include "tc_common.cuh"
@@ -85,7 +91,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t cW1 = 0;     // fp32 W1^T, tile t at 64 t
 constexpr uint32_t cW2 = 128;   // fp32 W2, tile t at 128 + 64 t
 constexpr uint32_t cA = 256;    // fp32 [A | Aq], tile t at 256 + 32 t
-constexpr uint32_t cG = 320;    // fp32 G^T, tile t at 320 + 16 t
 constexpr uint32_t cE = 352;    // fp32 E0^T (M = 64)
 constexpr uint32_t cZ = 368;    // fp32 Z0^T (M = 64)
 constexpr uint32_t cAW1 = 384;  // bf16 W1^T (A of S1), tile t at 384 + 32 t
@@ -137,6 +142,15 @@ __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint32_t
     asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
                  "r"(r[2]), "r"(r[3])
                  : "memory");
+}
+__device__ __forceinline__ void tmem_ld_16x256b_x1(uint32_t taddr, uint32_t* r) {
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x1.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+}
+// packed pair (row r, col c) and (row r + 8, col c): the accumulator layout's token pairs
+__device__ __forceinline__ void tmem_st_16x128b_x1(uint32_t taddr, uint32_t r0, uint32_t r1) {
+    asm volatile("tcgen05.st.sync.aligned.16x128b.x1.b32 [%0], {%1,%2};" ::"r"(taddr), "r"(r0), "r"(r1) : "memory");
 }
 __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t* r) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
@@ -193,11 +207,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* aux1 = bars + 2 * kStages;      // [kStages] tril(Q K^T) written (helper warp 6)
     uint64_t* d_a = bars + 3 * kStages;       // S1 done
     uint64_t* d_e = d_a + 1;                  // S2 done
-    uint64_t* d_g = d_a + 2;                  // S3 done
+    // d_a + 2 unused
     uint64_t* d_u = d_a + 3;                  // S4 done
     uint64_t* d_z = d_a + 4;                  // S5 done
     uint64_t* hk_rdy = d_a + 5;               // Hk^T, (-eta Hk)^T written (4 epilogue warps)
-    uint64_t* e_rdy = d_a + 6;                // E, (-eta E)^T written
+    // d_a + 6 unused
     uint64_t* d1_rdy = d_a + 7;               // (-eta D1)^T written
     uint64_t* hq_rdy = d_a + 8;               // Hq^T written
     uint64_t* aux2 = d_a + 9;                 // tril(Hq Hk^T) written (2 helper warps)
@@ -221,7 +235,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (uint64_t* b = d_a; b <= d_z; ++b) mbar_init(b, 1);
         mbar_init(hk_rdy, 8);
-        mbar_init(e_rdy, 8);
         mbar_init(d1_rdy, 8);
         mbar_init(hq_rdy, 8);
         mbar_init(aux2, 2);
@@ -279,7 +292,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint32_t idS1 = make_idesc_bf16(128, 32, 0, 0);
             const uint32_t idS2 = make_idesc_bf16(64, 16, 1, 0);   // A = W2 as MN-major
-            const uint32_t idS3 = make_idesc_bf16(128, 16, 0, 0);
             const uint32_t idUpd = make_idesc_bf16(128, 64, 0, 1); // B MN-major (K or E tile)
             const uint32_t idAq = make_idesc_bf16(128, 16, 0, 0);
             const uint32_t idZc = make_idesc_bf16(64, 16, 0, 0);
@@ -315,7 +327,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = i % kStages;
                 const uint32_t par = (i / kStages) & 1, ip = i & 1;
                 const uint32_t st = smem_u32(smem + kOffStages + s * kStageBytes);
-                const uint32_t w2b = w2 + 32768 * ip;
                 // S1
                 if (!W(&full[s], par) || !W(aw1_rdy, ip)) break;
                 tc_fence_after();
@@ -328,16 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma_commit(d_a);
                 // the previous batch's output path runs while E1 of this batch does
                 if (i >= 1 && !issue_s5(i - 1)) break;
-                // S3 (S2, E0 = W2^T Hk^T, runs on the epilogue warps' mma.sync)
-                if (!W(e_rdy, ip)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int tt = 0; tt < 2; ++tt)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        umma_bf16(tbase + cG + 16 * tt, make_sdesc(w2b + 16384 * tt + 32 * ks, 16, 1024, kSwizzle128B),
-                                  make_sdesc(et + 32 * ks, 16, 1024, kSwizzle128B), idS3, ks > 0);
-                umma_commit(d_g);
+                // (S2 and S3 run on the epilogue warps' mma.sync)
                 // S4
                 if (!W(d1_rdy, ip) || !W(&aux1[s], par)) break;
                 tc_fence_after();
@@ -408,7 +410,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* aes = smem + kOffAE;
         float2* xch = reinterpret_cast<float2*>(smem + kOffXch);   // partial sums of the two token halves
         const int r = lane >> 2, c = lane & 3;   // accumulator layout: rows 16 qd + r (+8), tokens 8 hf + 2c (+1)
-        float c1[2], c2f[2] = {0.f, 0.f};        // c1 of rows hr; c2 of rows 16 qd + r + 8 hh
+        // hidden rows in the accumulator layout: 128 tt + 32 qd + 16 m + r + 8 hh
+        auto hrow = [&](int tt, int m, int hh) { return 128 * tt + 32 * qd + 16 * m + r + 8 * hh; };
+        float c1[2][2][2], c2f[2] = {0.f, 0.f};  // c1 of rows hrow(tt, m, hh); c2 of rows 16 qd + r + 8 hh
+        // bf16 [t][h] tile (four 128B-swizzled sub-tiles of 64 hidden rows) from the accumulator
+        // layout: x[tt][m][hh] = pair of tokens (2c, 2c+1) of row hrow(tt, m, hh)
+        auto stsm_rows = [&](uint32_t base, const uint32_t (&x)[2][2][2]) {
+            const int t = 8 * hf + (lane & 7), mi = lane >> 3;
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                // matrix mi = 2 m + hh: hidden rows 128 tt + 32 qd + 16 m + 8 hh .. + 7
+                const int h0 = 128 * tt + 32 * qd + 8 * mi;
+                const uint32_t addr = base + 2048 * (h0 >> 6) + t * 128 + ((((h0 & 63) >> 3) ^ (t & 7)) << 4);
+                stsm_x4_tr(addr, x[tt][0][0], x[tt][0][1], x[tt][1][0], x[tt][1][1]);
+            }
+        };
         // initial state: this warp writes columns 32 hf .. 32 hf + 31 of W1^T and W2
         {
             const float* W1u = p.W1 + (size_t)pu * kD * kM;
@@ -416,7 +432,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
                 const int h = hr[tt];
-                c1[tt] = p.c1 ? p.c1[(size_t)pu * kM + h] : 0.f;
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh)
+                        c1[tt][m][hh] = p.c1 ? p.c1[(size_t)pu * kM + hrow(tt, m, hh)] : 0.f;
                 uint32_t w[32], pk[16];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(W1u[(size_t)(32 * hf + i) * kM + h]);
@@ -513,45 +533,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t par = (i / kStages) & 1, ip = i & 1;
             const uint8_t* st = smem + kOffStages + s * kStageBytes;
             WT(&full[s], par);
-            float et[8];   // eta of this warp's tokens
-            {
-                const float* etas = reinterpret_cast<const float*>(st + kOffEta);
-#pragma unroll
-                for (int t = 0; t < 8; ++t) et[t] = p.eta ? etas[8 * hf + t] : p.eta_const;
+            float et2[2];   // eta of tokens 8 hf + 2c, 8 hf + 2c + 1 (the accumulator columns)
+            if (p.eta) {
+                const float2 e0v = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(st + kOffEta) +
+                                                                    8 * hf + 2 * c);
+                et2[0] = e0v.x;
+                et2[1] = e0v.y;
+            } else {
+                et2[0] = et2[1] = p.eta_const;
             }
-            // E1: A -> Hk, GELU'(A)
+            // E1: A -> Hk, GELU'(A), accumulator layout (m16 tiles (tt, m) of this quadrant,
+            // the 8 tokens of this half)
             WT(d_a, ip);
             tc_fence_after();
-            float gp[2][8];
+            float gp[2][2][4];
             {
-                uint32_t ra[2][8];
-                tmem_ld_32x32b_x8(tl + cA + 8 * hf, ra[0]);
-                tmem_ld_32x32b_x8(tl + cA + 32 + 8 * hf, ra[1]);
+                uint32_t ra[2][2][4];
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+                        tmem_ld_16x256b_x1(tbase + ((uint32_t)(32 * qd + 16 * m) << 16) + cA + 32 * tt + 8 * hf, ra[tt][m]);
                 tmem_wait_ld();
-                uint8_t* hkb = hks + 8192 * ip;
+                uint32_t hkp[2][2][2];   // [tt][m][hh]: bf16 pairs of tokens (2c, 2c+1)
 #pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
-                    const int h = hr[tt];
-                    uint8_t* sub = hkb + 2048 * (h >> 6);
-                    float ah[8];
+                for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        const float a = __uint_as_float(ra[tt][t]) + c1[tt];
-                        float hk;
-                        gelu_and_grad_fast(a, hk, gp[tt][t]);
-                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(8 * hf + t, h & 63)) = __float2bfloat16_rn(hk);
-                        ah[t] = -et[t] * hk;
+                    for (int m = 0; m < 2; ++m) {
+                        float hk[4], ah[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float a = __uint_as_float(ra[tt][m][e]) + c1[tt][m][e >> 1];
+                            gelu_and_grad_fast(a, hk[e], gp[tt][m][e]);
+                            ah[e] = -et2[e & 1] * hk[e];
+                        }
+                        hkp[tt][m][0] = pack_bf16x2(hk[0], hk[1]);
+                        hkp[tt][m][1] = pack_bf16x2(hk[2], hk[3]);
+                        tmem_st_16x128b_x1(tbase + ((uint32_t)(32 * qd + 16 * m) << 16) + cAHk + 8 * tt + 4 * hf,
+                                           pack_bf16x2(ah[0], ah[1]), pack_bf16x2(ah[2], ah[3]));
                     }
-                    uint32_t pa[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) pa[k] = pack_bf16x2(ah[2 * k], ah[2 * k + 1]);
-                    tmem_st_32x32b_x4(tl + cAHk + 8 * tt + 4 * hf, pa);
-                }
+                // Hk [t][h] in shared memory: matrices (tokens of this half, 8 hidden rows)
+                stsm_rows(smem_u32(hks + 8192 * ip), hkp);
             }
-            fence_proxy_async_smem();
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
             // S2 on the epilogue warps (mma.sync): E0^T = W2^T Hk^T over the 256 hidden
             // rows; this warp: features 16 qd .. 16 qd + 15, tokens of its half.  Every
             // warp's Hk must be in shared memory first.
@@ -583,15 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t vt = smem_u32(st + kOffV);
                 uint32_t v[2];
                 ldsm_x2_tr(vt + t8 * 128 + (((2 * qd + ((lane >> 3) & 1)) ^ (t8 & 7)) << 4), v);
-                float etc[2];
-                if (p.eta) {
-                    const float2 e0v = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(st + kOffEta) +
-                                                                        8 * hf + 2 * c);
-                    etc[0] = e0v.x;
-                    etc[1] = e0v.y;
-                } else {
-                    etc[0] = etc[1] = p.eta_const;
-                }
+                const float etc[2] = {et2[0], et2[1]};
                 float ev[4], ae[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -627,49 +642,77 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(e_rdy);
-                mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&empty[s]);
+            // S3 on the epilogue warps (mma.sync): G^T = W2 E^T (K = 64) for this warp's four
+            // m16 tiles of hidden rows and the tokens of its half; every warp's E first
+            named_bar_sync(1, 256);
+            float g[2][2][4] = {};
+            {
+                const int mi = lane >> 3;
+                const uint32_t w2b = smem_u32(w2s + 32768 * ip), eb = smem_u32(es);
+                const int t8 = 8 * hf + (lane & 7);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    uint32_t b[2];
+                    ldsm_x2(eb + t8 * 128 + (((2 * ks + ((lane >> 3) & 1)) ^ (t8 & 7)) << 4), b);
+#pragma unroll
+                    for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            uint32_t a[4];
+                            const int h = 128 * tt + 32 * qd + 16 * m + (lane & 7) + 8 * (mi & 1);
+                            const int jch = 2 * ks + (mi >> 1);
+                            ldsm_x4(w2b + (h >> 3) * 1024 + (h & 7) * 128 + ((jch ^ (h & 7)) << 4), a);
+                            mma_16816(g[tt][m], a, b[0], b[1]);
+                        }
+                }
             }
             // E3: D1 = G * GELU'(A) -> (-eta D1)^T; c1 update
-            WT(d_g, ip);
-            tc_fence_after();
-            float c1_old[2] = {c1[0], c1[1]};
+            float c1_old[2][2][2];
             {
-                uint32_t rg[2][8];
-                tmem_ld_32x32b_x8(tl + cG + 8 * hf, rg[0]);
-                tmem_ld_32x32b_x8(tl + cG + 16 + 8 * hf, rg[1]);
-                tmem_wait_ld();
-                float csum[2];
+                float csum[8];
 #pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
-                    float ad[8], sum = 0.f;
+                for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-                    for (int t = 0; t < 8; ++t) {
-                        ad[t] = -et[t] * __uint_as_float(rg[tt][t]) * gp[tt][t];
-                        sum += ad[t];
+                    for (int m = 0; m < 2; ++m) {
+                        float ad[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) ad[e] = -et2[e & 1] * g[tt][m][e] * gp[tt][m][e];
+                        tmem_st_16x128b_x1(tbase + ((uint32_t)(32 * qd + 16 * m) << 16) + cAD1 + 8 * tt + 4 * hf,
+                                           pack_bf16x2(ad[0], ad[1]), pack_bf16x2(ad[2], ad[3]));
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            float cs = ad[2 * hh] + ad[2 * hh + 1];
+                            cs += __shfl_xor_sync(0xffffffffu, cs, 1);
+                            cs += __shfl_xor_sync(0xffffffffu, cs, 2);
+                            csum[4 * tt + 2 * m + hh] = cs;
+                        }
                     }
-                    csum[tt] = sum;
-                    uint32_t pa[4];
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) pa[k] = pack_bf16x2(ad[2 * k], ad[2 * k + 1]);
-                    tmem_st_32x32b_x4(tl + cAD1 + 8 * tt + 4 * hf, pa);
-                }
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(d1_rdy);
-                exchange2(csum, 2);
-                c1[0] += csum[0];
-                c1[1] += csum[1];
+                exchange2(csum, 8);
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) {
+                            c1_old[tt][m][hh] = c1[tt][m][hh];
+                            c1[tt][m][hh] += csum[4 * tt + 2 * m + hh];
+                        }
             }
             // E4: bf16 W1^T for the next S1 first, then Hq = GELU(Aq + c1) -> Hq^T
             // (Aq carries the batch's bias updates through tril(Q K^T + 1)), then bf16 W2
             WT(d_u, ip);
             tc_fence_after();
-            uint32_t rq[2][8];
-            tmem_ld_32x32b_x8(tl + cA + 16 + 8 * hf, rq[0]);
-            tmem_ld_32x32b_x8(tl + cA + 32 + 16 + 8 * hf, rq[1]);
+            uint32_t rq[2][2][4];
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                for (int m = 0; m < 2; ++m)
+                    tmem_ld_16x256b_x1(tbase + ((uint32_t)(32 * qd + 16 * m) << 16) + cA + 32 * tt + 16 + 8 * hf, rq[tt][m]);
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
                 uint32_t w[32], pk[16];
@@ -684,16 +727,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(aw1_rdy);
             {
-                uint8_t* hqb = hqs + 8192 * ip;
+                uint32_t hqp[2][2][2];
 #pragma unroll
-                for (int tt = 0; tt < 2; ++tt) {
-                    const int h = hr[tt];
-                    uint8_t* sub = hqb + 2048 * (h >> 6);
+                for (int tt = 0; tt < 2; ++tt)
 #pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        *reinterpret_cast<__nv_bfloat16*>(sub + sw128_off(8 * hf + t, h & 63)) =
-                            __float2bfloat16_rn(gelu_fast(__uint_as_float(rq[tt][t]) + c1_old[tt]));
-                }
+                    for (int m = 0; m < 2; ++m) {
+                        float hq[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            hq[e] = gelu_fast(__uint_as_float(rq[tt][m][e]) + c1_old[tt][m][e >> 1]);
+                        hqp[tt][m][0] = pack_bf16x2(hq[0], hq[1]);
+                        hqp[tt][m][1] = pack_bf16x2(hq[2], hq[3]);
+                    }
+                stsm_rows(smem_u32(hqs + 8192 * ip), hqp);
             }
             fence_proxy_async_smem();
             __syncwarp();
@@ -720,7 +766,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < 32; ++k) W2o[(size_t)h * kD + 32 * hf + k] = __uint_as_float(w[k]);
-                if (p.c1_out && hf == 0) p.c1_out[(size_t)unit * kM + h] = c1[tt];
+            }
+            if (p.c1_out && hf == 0 && c == 0) {
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                    for (int m = 0; m < 2; ++m)
+#pragma unroll
+                        for (int hh = 0; hh < 2; ++hh) p.c1_out[(size_t)unit * kM + hrow(tt, m, hh)] = c1[tt][m][hh];
             }
             if (p.c2_out && c == 0 && hf == 0) {
                 p.c2_out[(size_t)unit * kD + 16 * qd + r] = c2f[0];
