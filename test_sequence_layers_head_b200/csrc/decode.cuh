@@ -4,16 +4,16 @@
 //
 //     u = k W,  e = u - v,  W <- W - eta k^T e,  z = q W_new = q W - eta (q.k) e
 //
-// The step is bound by one read and one write of W (d*d fp32 per unit).  One
-// CTA per unit, D/8 warps; warp w owns columns 8w..8w+7 over all D rows, lane
-// l owns the float4 column group (l & 1) of rows (l >> 1) + 16 r, so the
-// reduction over rows stays inside the warp (shuffles, no shared memory) and
-// W crosses memory exactly twice.
+// The step reads and writes W once (d*d fp32 per unit).  One CTA per unit,
+// 4 D threads.  Thread t owns the float4 column group t % (D/4) of rows
+// t / (D/4) + 16 r, so each warp-wide access covers whole rows (512
+// contiguous bytes at D = 64) and touches the fewest cache lines; the sums
+// over rows go through shuffles inside the warp, then one shared-memory
+// exchange across the D/8 warps.
 //
-// Launched with programmatic dependent launch: the launch of step n+1
-// overlaps the tail of step n, and griddepcontrol.wait (before any global
-// read) orders every read after the previous kernel's writes, so q, k, v may
-// even alias the previous step's z.
+// Plain stream order between steps: with 512 units, programmatic dependent
+// launch measured slower (the next step's early CTAs take residency from the
+// current one) at every unit count tried (64, 148, 512).
 #pragma once
 #include "common.cuh"
 
@@ -29,22 +29,22 @@ struct DecodeParams {
     void* z;
 };
 
-__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dependents_launch() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 template <int D, typename IO>
 __global__ void __launch_bounds__(D * 4) decode_kernel(DecodeParams p) {
-    constexpr int R = D / 16;        // rows per lane
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    constexpr int NT = 4 * D, NW = NT / 32;   // threads, warps
+    constexpr int CG = D / 4;                 // float4 column groups per row
+    constexpr int R = D / 16;                 // rows per thread
+    __shared__ float4 red[NW][2][CG];         // per-warp partial k W and q W
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
     const int unit = blockIdx.x;
-    const int col = 8 * w + 4 * (lane & 1);   // first of this lane's 4 columns
-    const int row0 = lane >> 1;               // rows row0 + 16 r
-    grid_dependency_wait();   // the previous kernel in the stream is complete and visible
+    const int cg = t % CG, row0 = t / CG;     // rows row0 + 16 r
     const IO* q = static_cast<const IO*>(p.q) + (size_t)unit * D;
     const IO* k = static_cast<const IO*>(p.k) + (size_t)unit * D;
     const IO* v = static_cast<const IO*>(p.v) + (size_t)unit * D;
+    float4* W = reinterpret_cast<float4*>(p.W + (size_t)unit * D * D);
+    float4 wr[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) wr[r] = W[(size_t)(row0 + 16 * r) * CG + cg];
     float kr[R], qr[R], vc[4];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -52,21 +52,13 @@ __global__ void __launch_bounds__(D * 4) decode_kernel(DecodeParams p) {
         qr[r] = IoTraits<IO>::load(q, row0 + 16 * r);
     }
 #pragma unroll
-    for (int c = 0; c < 4; ++c) vc[c] = IoTraits<IO>::load(v, col + c);
+    for (int c = 0; c < 4; ++c) vc[c] = IoTraits<IO>::load(v, 4 * cg + c);
     const float eta = p.eta ? p.eta[unit] : p.eta_const;
-    // q . k: every lane holds R (q, k) pairs of distinct rows (lane pairs repeat them)
+    // q . k, complete in every warp
     float qk = 0.f;
-#pragma unroll
-    for (int r = 0; r < R; ++r) qk += qr[r] * kr[r];
-    qk *= ((lane & 1) == 0) ? 1.f : 0.f;
+    for (int i = lane; i < D; i += 32) qk += IoTraits<IO>::load(q, i) * IoTraits<IO>::load(k, i);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
-
-    float4* W = reinterpret_cast<float4*>(p.W + (size_t)unit * D * D);
-    float4 wr[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) wr[r] = W[(size_t)(row0 + 16 * r) * (D / 4) + (col >> 2)];
-    grid_dependents_launch();
 
     float u[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
@@ -74,27 +66,39 @@ __global__ void __launch_bounds__(D * 4) decode_kernel(DecodeParams p) {
         u[0] += kr[r] * wr[r].x; u[1] += kr[r] * wr[r].y; u[2] += kr[r] * wr[r].z; u[3] += kr[r] * wr[r].w;
         pq[0] += qr[r] * wr[r].x; pq[1] += qr[r] * wr[r].y; pq[2] += qr[r] * wr[r].z; pq[3] += qr[r] * wr[r].w;
     }
-    // sum over the 16 row groups (lane bits 1..4)
+    // rows of this warp: lanes cg, cg + CG, ... share the column group
 #pragma unroll
-    for (int o = 2; o < 32; o <<= 1)
+    for (int o = CG; o < 32; o <<= 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
             u[c] += __shfl_xor_sync(0xffffffffu, u[c], o);
             pq[c] += __shfl_xor_sync(0xffffffffu, pq[c], o);
         }
-    float e[4];
+    if (lane < CG) {
+        red[w][0][lane] = make_float4(u[0], u[1], u[2], u[3]);
+        red[w][1][lane] = make_float4(pq[0], pq[1], pq[2], pq[3]);
+    }
+    __syncthreads();
+    float4 su = red[0][0][cg], sq = red[0][1][cg];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) e[c] = u[c] - vc[c];
-    if (row0 == 0) {
+    for (int x = 1; x < NW; ++x) {
+        const float4 a = red[x][0][cg], b = red[x][1][cg];
+        su.x += a.x; su.y += a.y; su.z += a.z; su.w += a.w;
+        sq.x += b.x; sq.y += b.y; sq.z += b.z; sq.w += b.w;
+    }
+    const float e[4] = {su.x - vc[0], su.y - vc[1], su.z - vc[2], su.w - vc[3]};
+    if (t < CG) {
         IO* z = static_cast<IO*>(p.z) + (size_t)unit * D;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) IoTraits<IO>::store(z, col + c, pq[c] - eta * qk * e[c]);
+        IoTraits<IO>::store(z, 4 * cg + 0, sq.x - eta * qk * e[0]);
+        IoTraits<IO>::store(z, 4 * cg + 1, sq.y - eta * qk * e[1]);
+        IoTraits<IO>::store(z, 4 * cg + 2, sq.z - eta * qk * e[2]);
+        IoTraits<IO>::store(z, 4 * cg + 3, sq.w - eta * qk * e[3]);
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
         const float a = eta * kr[r];
         wr[r].x -= a * e[0]; wr[r].y -= a * e[1]; wr[r].z -= a * e[2]; wr[r].w -= a * e[3];
-        W[(size_t)(row0 + 16 * r) * (D / 4) + (col >> 2)] = wr[r];
+        W[(size_t)(row0 + 16 * r) * CG + cg] = wr[r];
     }
 }
 

@@ -325,11 +325,6 @@ ttt_status launch_decode_t(const ttt_decode_args* a, cudaStream_t st) {
     cfg.blockDim = dim3(D * 4);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
     if (cudaLaunchKernelEx(&cfg, decode_kernel<D, IO>, p) != cudaSuccess) return launch_status();
     return launch_status();
 }
