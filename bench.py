@@ -240,7 +240,7 @@ def device_inputs(w, torch, threads):
 
 
 def time_launches(torch, fn, steps, warmup, flush=None):
-    """Per-launch CUDA-event durations (ms) plus the whole timed span (ms)."""
+    """Per-launch CUDA-event durations (ms)."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
@@ -293,6 +293,63 @@ def measure_decode(ttt, w, torch, steps=3):
             "bytes_per_step": bytes_step, "achieved_gbs": bytes_step * n / (ms / 1000.0) / 1e9,
             "note": "W (8.4 MB) stays L2-resident across steps; GB/s is against HBM peak for reference",
             "gpu_launches_per_graph": n}
+
+
+def measure_decode_variant(ttt, torch, kind, B, H, d=64, n=1024, steps=3):
+    """LN+residual or MLP decode: n single-token steps for B x H units from a
+    random state, captured in one CUDA graph (informational; parity lives in
+    the tests).  Returns per-step time and the state bytes each step moves."""
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1)
+    f32 = dict(device="cuda", dtype=torch.float32)
+    units = B * H
+    q = (torch.randn(n, B, H, d, generator=g, **f32) / 8).bfloat16()
+    k = (torch.randn(n, B, H, d, generator=g, **f32) / 8).bfloat16()
+    v = (torch.randn(n, B, H, d, generator=g, **f32) / 8).bfloat16()
+    eta = torch.sigmoid(torch.randn(n, B, H, generator=g, **f32)) / 64
+    z = torch.empty_like(q)
+    if kind == "ln":
+        W = torch.randn(B, H, d, d, generator=g, **f32) / 8
+        c = torch.zeros(B, H, d, **f32)
+        gam = 1 + torch.randn(H, d, generator=g, **f32) * 0.14
+        bet = torch.randn(H, d, generator=g, **f32) * 0.14
+
+        def step(s, st):
+            ttt.linear_decode_step(W, q[s], k[s], v[s], eta[s], z=z[s], use_ln=True, c=c, gamma=gam, beta=bet,
+                                   stream=st)
+        state_bytes = units * (2 * d * d * 4 + 2 * d * 4)
+    else:
+        m = 4 * d
+        W1 = torch.randn(B, H, d, m, generator=g, **f32) / 8
+        c1 = torch.zeros(B, H, m, **f32)
+        W2 = torch.randn(B, H, m, d, generator=g, **f32) / 16
+        c2 = torch.zeros(B, H, d, **f32)
+
+        def step(s, st):
+            ttt.mlp_decode_step(W1, c1, W2, c2, q[s], k[s], v[s], eta[s], z=z[s], stream=st)
+        state_bytes = units * (2 * 2 * d * m * 4 + 2 * (m + d) * 4)
+    st = torch.cuda.Stream()
+    st.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(st):
+        for s in range(3):
+            step(s, st)
+    torch.cuda.current_stream().wait_stream(st)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cs = torch.cuda.current_stream()
+        for s in range(n):
+            step(s, cs)
+    graph.replay()
+    torch.cuda.synchronize()
+    per = time_launches(torch, graph.replay, steps, 1)
+    ms = statistics.median(per)
+    del graph
+    bytes_step = state_bytes + units * (4 * d * 2 + 4)
+    return {"B": B, "H": H, "d": d, "steps_per_graph": n, "us_per_step": 1000.0 * ms / n,
+            "tokens_per_s": B * n / (ms / 1000.0), "bytes_per_step": bytes_step,
+            "achieved_gbs": bytes_step * n / (ms / 1000.0) / 1e9,
+            "note": "state stays L2-resident across steps; GB/s is against HBM peak for reference"}
 
 
 def measure_e2e_chunked(ttt, w, inp, torch, steps, chunks=8):
@@ -523,6 +580,8 @@ def run_ours(args):
             line["decode"] = measure_decode(ttt, w, torch)
         if not args.no_rows:
             line["rows"] = measure_rows(ttt, torch, threads)
+            line["rows"]["decode_ln_B4_H32"] = measure_decode_variant(ttt, torch, "ln", 4, 32)
+            line["rows"]["decode_mlp_B2_H32"] = measure_decode_variant(ttt, torch, "mlp", 2, 32)
         line["cpu_baseline"] = cpu_baseline(w)
     if dist is not None:
         dist.barrier()

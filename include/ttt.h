@@ -161,11 +161,15 @@ typedef struct {
 ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
 
 /*
- * ttt_linear_decode_step -- one generated token per unit, TTT-Linear without
- * LN, primal form with b = 1 (section 6.11: decode is token by token and uses
- * the primal form; section 3.1: update, then output):
- *     e = k W - v,   W <- W - eta k^T e,   z = q W   (W after the update)
- * computed as z = q W_old - eta (q . k) e so W is read and written once.
+ * ttt_linear_decode_step -- one generated token per unit, TTT-Linear plain or
+ * LN+residual, primal form with b = 1 (section 6.11: decode is token by token
+ * and uses the primal form; section 3.1: update, then output).
+ *   plain:  e = k W - v,   W <- W - eta k^T e,   z = q W   (W after the update),
+ *           computed as z = q W_old - eta (q . k) e so W is read and written once.
+ *   use_ln: f(x) = x + LN(x W + c) (section 4.4; gamma, beta fixed): the
+ *           gradient of 1/2 ||f(k) - v||^2 through LN gives delta (the
+ *           gradient at the pre-activation); W <- W - eta k^T delta,
+ *           c <- c - eta delta, z = f(q) with the updated W and c.
  *
  *   B, H, d        d in {16, 32, 64}.
  *   io_dtype       dtype of q, k, v and z.
@@ -173,6 +177,10 @@ ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
  *   q, k, v        [B, H, d].
  *   eta            [B, H] fp32, or NULL for eta_const.
  *   z              output [B, H, d] in io_dtype.
+ *   use_ln         0: plain.  1: LN+residual; then
+ *   c              [B, H, d] fp32 bias state, updated in place;
+ *   ln_gamma, ln_beta  [H, d] fp32;  ln_eps > 0 (1e-6 in the tests).
+ *   With use_ln = 0 the last five fields are ignored.
  */
 typedef struct {
     int B, H, d;
@@ -184,9 +192,49 @@ typedef struct {
     const float* eta;
     float eta_const;
     void* z;
+    int use_ln;
+    float* c;
+    const float* ln_gamma;
+    const float* ln_beta;
+    float ln_eps;
 } ttt_decode_args;
 
 ttt_status ttt_linear_decode_step(const ttt_decode_args* args, cudaStream_t stream);
+
+/*
+ * ttt_mlp_decode_step -- one generated token per unit, TTT-MLP
+ * f(x) = GELU(x W1 + c1) W2 + c2 with hidden size m = 4 d (section 4.4),
+ * primal form with b = 1 (section 6.11; section 3.1: update, then output):
+ *     a = k W1 + c1,  h = GELU(a),  e = h W2 + c2 - v,
+ *     delta1 = (e W2^T) * GELU'(a),
+ *     W1 -= eta k^T delta1,  c1 -= eta delta1,  W2 -= eta h^T e,  c2 -= eta e,
+ *     z = f(q) with the updated state.
+ * GELU is the exact erf form.
+ *
+ *   B, H, d        d in {16, 32, 64}; m = 4 d.
+ *   io_dtype       dtype of q, k, v and z.
+ *   W1 [B,H,d,m], c1 [B,H,m], W2 [B,H,m,d], c2 [B,H,d]
+ *                  fp32 state, updated in place.
+ *   q, k, v        [B, H, d].
+ *   eta            [B, H] fp32, or NULL for eta_const.
+ *   z              output [B, H, d] in io_dtype.
+ */
+typedef struct {
+    int B, H, d;
+    ttt_dtype io_dtype;
+    float* W1;
+    float* c1;
+    float* W2;
+    float* c2;
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* eta;
+    float eta_const;
+    void* z;
+} ttt_mlp_decode_args;
+
+ttt_status ttt_mlp_decode_step(const ttt_mlp_decode_args* args, cudaStream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* ttt_status_string(ttt_status s);

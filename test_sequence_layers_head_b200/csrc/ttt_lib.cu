@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "linear_frag.cuh"
+#include "mlp_decode.cuh"
 #include "mlp_tc.cuh"
 #include "simt.cuh"
 #include "tmap.h"
@@ -319,13 +320,16 @@ namespace ttt {
 namespace {
 template <int D, typename IO>
 ttt_status launch_decode_t(const ttt_decode_args* a, cudaStream_t st) {
-    DecodeParams p{a->W, a->q, a->k, a->v, a->eta, a->eta_const, a->z};
+    DecodeParams p{a->W, a->q, a->k, a->v, a->eta, a->eta_const, a->z,
+                   a->c, a->ln_gamma, a->ln_beta, a->ln_eps, a->H};
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(a->B * a->H));
     cfg.blockDim = dim3(D * 4);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
-    if (cudaLaunchKernelEx(&cfg, decode_kernel<D, IO>, p) != cudaSuccess) return launch_status();
+    const cudaError_t e = a->use_ln ? cudaLaunchKernelEx(&cfg, decode_kernel<D, IO, true>, p)
+                                    : cudaLaunchKernelEx(&cfg, decode_kernel<D, IO, false>, p);
+    if (e != cudaSuccess) return launch_status();
     return launch_status();
 }
 template <int D>
@@ -344,10 +348,46 @@ extern "C" ttt_status ttt_linear_decode_step(const ttt_decode_args* a, cudaStrea
     if ((long long)a->B * a->H == 0) return TTT_OK;
     if (!ok_ptr(a->W) || !ok_ptr(a->q) || !ok_ptr(a->k) || !ok_ptr(a->v) || !ok_ptr(a->z) || !ok_opt(a->eta))
         return TTT_ERR_INVALID_ARG;
+    if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
+    if (a->use_ln && (!ok_ptr(a->c) || !ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !(a->ln_eps > 0.f)))
+        return TTT_ERR_INVALID_ARG;
     switch (a->d) {
         case 16: return launch_decode<16>(a, stream);
         case 32: return launch_decode<32>(a, stream);
         default: return launch_decode<64>(a, stream);
+    }
+}
+
+namespace ttt {
+namespace {
+template <int D, typename IO>
+ttt_status launch_mlp_decode_t(const ttt_mlp_decode_args* a, cudaStream_t st) {
+    MlpDecodeParams p{a->W1, a->c1, a->W2, a->c2, a->q, a->k, a->v, a->eta, a->eta_const, a->z};
+    mlp_decode_kernel<D, IO><<<(unsigned)(a->B * a->H), 4 * D, 0, st>>>(p);
+    return launch_status();
+}
+template <int D>
+ttt_status launch_mlp_decode(const ttt_mlp_decode_args* a, cudaStream_t st) {
+    return a->io_dtype == TTT_F32 ? launch_mlp_decode_t<D, float>(a, st)
+                                  : launch_mlp_decode_t<D, __nv_bfloat16>(a, st);
+}
+}  // namespace
+}  // namespace ttt
+
+extern "C" ttt_status ttt_mlp_decode_step(const ttt_mlp_decode_args* a, cudaStream_t stream) {
+    if (!a) return TTT_ERR_INVALID_ARG;
+    if (a->B < 0 || a->H < 0 || a->d <= 0) return TTT_ERR_INVALID_ARG;
+    if (a->io_dtype != TTT_F32 && a->io_dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
+    if (a->d != 16 && a->d != 32 && a->d != 64) return TTT_ERR_UNSUPPORTED;
+    if ((long long)a->B * a->H > (1ll << 30)) return TTT_ERR_UNSUPPORTED;
+    if ((long long)a->B * a->H == 0) return TTT_OK;
+    if (!ok_ptr(a->W1) || !ok_ptr(a->c1) || !ok_ptr(a->W2) || !ok_ptr(a->c2) || !ok_ptr(a->q) || !ok_ptr(a->k) ||
+        !ok_ptr(a->v) || !ok_ptr(a->z) || !ok_opt(a->eta))
+        return TTT_ERR_INVALID_ARG;
+    switch (a->d) {
+        case 16: return launch_mlp_decode<16>(a, stream);
+        case 32: return launch_mlp_decode<32>(a, stream);
+        default: return launch_mlp_decode<64>(a, stream);
     }
 }
 

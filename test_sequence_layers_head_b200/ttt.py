@@ -51,7 +51,13 @@ class MlpArgs(ctypes.Structure):
 
 class DecodeArgs(ctypes.Structure):
     _fields_ = [("B", _i), ("H", _i), ("d", _i), ("io_dtype", _i), ("W", _vp), ("q", _vp), ("k", _vp),
-                ("v", _vp), ("eta", _vp), ("eta_const", _f), ("z", _vp)]
+                ("v", _vp), ("eta", _vp), ("eta_const", _f), ("z", _vp), ("use_ln", _i), ("c", _vp),
+                ("ln_gamma", _vp), ("ln_beta", _vp), ("ln_eps", _f)]
+
+
+class MlpDecodeArgs(ctypes.Structure):
+    _fields_ = [("B", _i), ("H", _i), ("d", _i), ("io_dtype", _i), ("W1", _vp), ("c1", _vp), ("W2", _vp),
+                ("c2", _vp), ("q", _vp), ("k", _vp), ("v", _vp), ("eta", _vp), ("eta_const", _f), ("z", _vp)]
 
 
 class TTTError(RuntimeError):
@@ -63,8 +69,8 @@ class TTTError(RuntimeError):
 _lib = None
 
 # Every symbol include/ttt.h declares.
-EXPORTS = ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_status_string",
-           "ttt_last_device_status", "ttt_version")
+EXPORTS = ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_mlp_decode_step",
+           "ttt_status_string", "ttt_last_device_status", "ttt_version")
 
 
 def library() -> ctypes.CDLL:
@@ -81,6 +87,8 @@ def library() -> ctypes.CDLL:
         L.ttt_mlp_forward.restype = _i
         L.ttt_linear_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
         L.ttt_linear_decode_step.restype = _i
+        L.ttt_mlp_decode_step.argtypes = [ctypes.POINTER(MlpDecodeArgs), _vp]
+        L.ttt_mlp_decode_step.restype = _i
         L.ttt_status_string.argtypes = [_i]
         L.ttt_status_string.restype = ctypes.c_char_p
         L.ttt_last_device_status.argtypes = [_vp]
@@ -171,13 +179,26 @@ def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, *, eta_const=0.0, Z=None, W1_ou
     return Z, W1_out, c1_out, W2_out, c2_out
 
 
-def linear_decode_step(W, q, k, v, eta, *, eta_const=0.0, z=None, stream=None):
-    """One decode token per unit; W [B,H,d,d] fp32 is updated in place.  Returns z."""
+def linear_decode_step(W, q, k, v, eta, *, eta_const=0.0, z=None, use_ln=False, c=None, gamma=None, beta=None,
+                       eps=1e-6, stream=None):
+    """One decode token per unit; W [B,H,d,d] fp32 (and, with use_ln, the bias
+    state c [B,H,d]) is updated in place.  Returns z."""
     B, H, d = q.shape
     z = torch.empty_like(q) if z is None else z
     a = DecodeArgs(B, H, d, _io_dtype(q), _ptr(W), _ptr(q), _ptr(k), _ptr(v), _ptr(eta), float(eta_const),
-                   _ptr(z))
+                   _ptr(z), int(bool(use_ln)), _ptr(c), _ptr(gamma), _ptr(beta), float(eps))
     _check(library().ttt_linear_decode_step(ctypes.byref(a), _stream(stream)), "ttt_linear_decode_step")
+    return z
+
+
+def mlp_decode_step(W1, c1, W2, c2, q, k, v, eta, *, eta_const=0.0, z=None, stream=None):
+    """One TTT-MLP decode token per unit; W1 [B,H,d,4d], c1 [B,H,4d], W2 [B,H,4d,d]
+    and c2 [B,H,d] (fp32) are updated in place.  Returns z."""
+    B, H, d = q.shape
+    z = torch.empty_like(q) if z is None else z
+    a = MlpDecodeArgs(B, H, d, _io_dtype(q), _ptr(W1), _ptr(c1), _ptr(W2), _ptr(c2), _ptr(q), _ptr(k), _ptr(v),
+                      _ptr(eta), float(eta_const), _ptr(z))
+    _check(library().ttt_mlp_decode_step(ctypes.byref(a), _stream(stream)), "ttt_mlp_decode_step")
     return z
 
 

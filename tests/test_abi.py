@@ -18,7 +18,7 @@ def declared_symbols():
 
 def test_header_declares_entry_points():
     syms = declared_symbols()
-    for s in ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step"):
+    for s in ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_mlp_decode_step"):
         assert s in syms
 
 
@@ -88,6 +88,7 @@ def test_null_args_struct(ttt_lib):
     assert L.ttt_linear_forward(None, None) == 1
     assert L.ttt_mlp_forward(None, None) == 1
     assert L.ttt_linear_decode_step(None, None) == 1
+    assert L.ttt_mlp_decode_step(None, None) == 1
 
 
 def test_mlp_and_decode_validation(ttt_lib):
@@ -102,6 +103,58 @@ def test_mlp_and_decode_validation(ttt_lib):
     assert L.ttt_linear_decode_step(ctypes.byref(dargs), None) == 1
     dargs.d = 24
     assert L.ttt_linear_decode_step(ctypes.byref(dargs), None) == 2
+
+
+def _decode_args(ttt, **kw):
+    a = ttt.DecodeArgs()
+    a.B, a.H, a.d, a.io_dtype = 2, 2, 64, ttt.TTT_BF16
+    fake = 1 << 20  # aligned fake device address; never dereferenced (validation fails first)
+    a.W = a.q = a.k = a.v = a.z = fake
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(use_ln=2), 1),
+    (dict(use_ln=1), 1),                                           # no c, gamma, beta
+    (dict(use_ln=1, c=1 << 20, ln_gamma=1 << 20, ln_beta=1 << 20), 1),   # eps = 0
+    (dict(use_ln=1, c=(1 << 20) + 4, ln_gamma=1 << 20, ln_beta=1 << 20, ln_eps=1e-6), 1),  # misaligned c
+    (dict(use_ln=1, c=1 << 20, ln_gamma=None, ln_beta=1 << 20, ln_eps=1e-6), 1),
+    (dict(use_ln=1, c=1 << 20, ln_gamma=1 << 20, ln_beta=1 << 20, ln_eps=1e-6, d=48), 2),
+    (dict(B=0, use_ln=1), 0),                                      # empty: no-op before pointer checks
+])
+def test_ln_decode_validation(ttt_lib, kw, code):
+    a = _decode_args(ttt_lib, **kw)
+    assert ttt_lib.library().ttt_linear_decode_step(ctypes.byref(a), None) == code
+
+
+def _mlp_decode_args(ttt, **kw):
+    a = ttt.MlpDecodeArgs()
+    a.B, a.H, a.d, a.io_dtype = 2, 2, 64, ttt.TTT_BF16
+    fake = 1 << 20
+    a.W1 = a.c1 = a.W2 = a.c2 = a.q = a.k = a.v = a.z = fake
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(W1=None), 1),
+    (dict(c1=(1 << 20) + 4), 1),
+    (dict(W2=None), 1),
+    (dict(c2=None), 1),
+    (dict(z=None), 1),
+    (dict(eta=(1 << 20) + 8), 1),
+    (dict(io_dtype=5), 1),
+    (dict(d=48), 2),
+    (dict(d=0), 1),
+    (dict(B=-1), 1),
+    (dict(B=0, W1=None), 0),
+])
+def test_mlp_decode_validation(ttt_lib, kw, code):
+    a = _mlp_decode_args(ttt_lib, **kw)
+    assert ttt_lib.library().ttt_mlp_decode_step(ctypes.byref(a), None) == code
 
 
 def test_binding_refuses_cpu_tensors(ttt_lib):

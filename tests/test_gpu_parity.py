@@ -257,6 +257,89 @@ def test_decode_steps(ttt_lib, d, io):
         assert normwise(to_host(Wd), Wo) < 1e-5
 
 
+def _f32_state(rng, shape, scale, offset=0.0):
+    """fp32 device tensor and the same values in float64 for the oracle."""
+    raw, ex = WL.store(offset + rng.standard_normal(shape) * scale, WL.F32)
+    return to_dev(raw), ex
+
+
+@pytest.mark.parametrize("d,io", [(64, WL.BF16), (32, WL.F32), (16, WL.BF16), (64, WL.F32)])
+def test_ln_decode_steps(ttt_lib, d, io):
+    """LN+residual decode (b = 1 primal step) against the oracle's forward with
+    T = b = 1 from the same state; W and c carried over six steps."""
+    B, H = 3, 5
+    w = WL.Workload("dec", "ln", B, H, 1, d, 1, io, "sigmoid", 0.0, 37)
+    rng = np.random.default_rng(100 + d)
+    Wd, Wo = _f32_state(rng, (B, H, d, d), 1 / np.sqrt(d))
+    cd, co = _f32_state(rng, (B, H, d), 0.1)
+    gd, go = _f32_state(rng, (H, d), np.sqrt(0.02), offset=1.0)
+    bd, bo = _f32_state(rng, (H, d), np.sqrt(0.02))
+    for step in range(6):
+        raw, ex = WL.make_decode_tokens(w, step)
+        q, k, v, eta = (to_dev(raw[n]) for n in ("q", "k", "v", "eta"))
+        z = ttt_lib.linear_decode_step(Wd, q, k, v, eta, use_ln=True, c=cd, gamma=gd, beta=bd, eps=1e-6)
+        Z, Wo, co = O.linear_forward(ex["q"][:, :, None], ex["k"][:, :, None], ex["v"][:, :, None],
+                                     ex["eta"][:, :, None], Wo, 1, c0=co, gamma=go, beta=bo, use_ln=True, eps=1e-6)
+        zo = Z[:, :, 0]
+        torch.cuda.synchronize()
+        if io == WL.F32:
+            assert_close("z", to_host(z), zo, io)
+        else:
+            assert normwise(to_host(z), zo) < 1e-2
+        assert normwise(to_host(Wd), Wo) < 1e-5
+        assert normwise(to_host(cd), co) < 1e-5
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+
+
+@pytest.mark.parametrize("d,io", [(64, WL.BF16), (64, WL.F32), (32, WL.F32), (16, WL.BF16)])
+def test_mlp_decode_steps(ttt_lib, d, io):
+    """TTT-MLP decode (b = 1 primal step) against the oracle's MLP forward with
+    T = b = 1 from the same per-sequence state; the four state tensors carried
+    over six steps."""
+    B, H, m = 3, 5, 4 * d
+    w = WL.Workload("dec", "mlp", B, H, 1, d, 1, io, "sigmoid", 0.0, 41)
+    rng = np.random.default_rng(200 + d)
+    W1d, W1o = _f32_state(rng, (B, H, d, m), 1 / np.sqrt(d))
+    c1d, c1o = _f32_state(rng, (B, H, m), 0.1)
+    W2d, W2o = _f32_state(rng, (B, H, m, d), 1 / np.sqrt(m))
+    c2d, c2o = _f32_state(rng, (B, H, d), 0.1)
+    for step in range(6):
+        raw, ex = WL.make_decode_tokens(w, step)
+        q, k, v, eta = (to_dev(raw[n]) for n in ("q", "k", "v", "eta"))
+        z = ttt_lib.mlp_decode_step(W1d, c1d, W2d, c2d, q, k, v, eta)
+        Z, W1o, c1o, W2o, c2o = O.mlp_forward(ex["q"][:, :, None], ex["k"][:, :, None], ex["v"][:, :, None],
+                                              ex["eta"][:, :, None], W1o, c1o, W2o, c2o, 1)
+        zo = Z[:, :, 0]
+        torch.cuda.synchronize()
+        if io == WL.F32:
+            assert_close("z", to_host(z), zo, io)
+        else:
+            assert normwise(to_host(z), zo) < 1e-2
+        for nm, g, o in (("W1", W1d, W1o), ("c1", c1d, c1o), ("W2", W2d, W2o), ("c2", c2d, c2o)):
+            assert normwise(to_host(g), o) < 1e-5, nm
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+
+
+def test_mlp_decode_eta_zero_is_a_forward(ttt_lib):
+    """eta = 0: the state is returned bit for bit and z = f(q; state)."""
+    B, H, d, m = 2, 3, 64, 256
+    rng = np.random.default_rng(7)
+    W1d, W1o = _f32_state(rng, (B, H, d, m), 1 / np.sqrt(d))
+    c1d, c1o = _f32_state(rng, (B, H, m), 0.1)
+    W2d, W2o = _f32_state(rng, (B, H, m, d), 1 / np.sqrt(m))
+    c2d, c2o = _f32_state(rng, (B, H, d), 0.1)
+    before = [t.clone() for t in (W1d, c1d, W2d, c2d)]
+    qr, qe = WL.store(rng.standard_normal((B, H, d)) / 8, WL.F32)
+    q = to_dev(qr)
+    z = ttt_lib.mlp_decode_step(W1d, c1d, W2d, c2d, q, q, q, None, eta_const=0.0)
+    torch.cuda.synchronize()
+    for a, b in zip(before, (W1d, c1d, W2d, c2d)):
+        assert torch.equal(a, b)
+    zo = O.mlp_forward(qe[:, :, None], qe[:, :, None], qe[:, :, None], np.zeros((B, H, 1)), W1o, c1o, W2o, c2o,
+                       1)[0][:, :, 0]
+    assert_close("z", to_host(z), zo, WL.F32)
+
+
 # ---------------------------------------------------------------------------
 # full-size workloads, sampled units
 # ---------------------------------------------------------------------------
