@@ -92,7 +92,7 @@ constexpr int kOffAblk = kOffH + kHring * kHslot;         // 84992 (1024-aligned
 constexpr int kAblkBytes = 16384;                         // bf16 [128 rows][64 k], K-major, no swizzle
 constexpr int kOffZs = kOffAblk + kAblkBytes;             // Z staging: [4 warps] 32 tokens x 32 j, 64B swizzle
 constexpr int kZsBytes = 2048;
-constexpr int kOffRed = kOffZs + 4 * kZsBytes;           // LN: 2 buffers x [4 warps][16 tokens] float2
+constexpr int kOffRed = kOffZs + 4 * kZsBytes;           // LN: 2 buffers x [4 warps][4 c][8] float
 constexpr int kOffBar = kOffRed + 2 * 4 * 16 * 8;
 constexpr int kNumBars = 2 * kStages + 2 * kHring + 6;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -164,47 +164,57 @@ __device__ __forceinline__ void product_store(const uint32_t (*fa)[4], const uin
         }
 }
 
-// LN: sums over the unit's 64 features of two per-token quantities.  The
-// thread's tokens are k = 2 nt + e1 -> t = 8 nt + 2 c + e1; sa, sb hold its
-// partial sums over its rows.  The unit's rows are spread over NW warps
-// (2: warps q, q ^ 1; 4: warps 0-3).  Afterwards every thread holds the
-// unit's totals for its four tokens.
+// LN: sums over the unit's 64 features of two per-token quantities sa[k],
+// sb[k] (the thread's tokens k = 2 nt + e1 -> t = 8 nt + 2 c + e1).  The eight
+// lanes of a warp that hold the same tokens (same c) reduce the eight values
+// by recursive halving: at each of three levels a lane keeps one half of its
+// list and adds the partner's copy of that half (4 + 2 + 1 shuffles), so lane
+// r = lane / 4 ends with the warp's sum of entry r.  The entries go to shared
+// memory as [warp][c][8]; after a named barrier over the unit's NW warps (2:
+// warps q, q ^ 1; 4: warps 0-3) every thread adds up the NW lists of its c.
+// (Measured: merging two of these into one reduction of more values, or the
+// forward and backward sums of a mini-batch into one, is slower.)
 template <int NW>
-__device__ __forceinline__ void tok_sum2(float* sa, float* sb, float2* red, int q, int lane) {
+__device__ __forceinline__ void tok_sum2(float* sa, float* sb, float* red, int q, int lane) {
+    const float l0[8] = {sa[0], sa[1], sa[2], sa[3], sb[0], sb[1], sb[2], sb[3]};
+    float l1[4], l2[2];
+    {
+        const bool up = (lane & 16) != 0;
 #pragma unroll
-    for (int o = 4; o < 32; o <<= 1)
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            sa[k] += __shfl_xor_sync(0xffffffffu, sa[k], o);
-            sb[k] += __shfl_xor_sync(0xffffffffu, sb[k], o);
+        for (int i = 0; i < 4; ++i) {
+            const float keep = up ? l0[4 + i] : l0[i], send = up ? l0[i] : l0[4 + i];
+            l1[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
         }
-    const int c = lane & 3;
-    if (lane < 4) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) red[q * 16 + 8 * (k >> 1) + 2 * c + (k & 1)] = make_float2(sa[k], sb[k]);
     }
-    if (NW == 2) {
+    {
+        const bool up = (lane & 8) != 0;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const float keep = up ? l1[2 + i] : l1[i], send = up ? l1[i] : l1[2 + i];
+            l2[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+        }
+    }
+    const bool up = (lane & 4) != 0;
+    const float l3 = (up ? l2[1] : l2[0]) + __shfl_xor_sync(0xffffffffu, up ? l2[0] : l2[1], 4);
+    const int c = lane & 3;
+    red[(q * 4 + c) * 8 + (lane >> 2)] = l3;
+    if (NW == 2)
         named_bar_sync(1 + (q >> 1), 64);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 o = red[(q ^ 1) * 16 + 8 * (k >> 1) + 2 * c + (k & 1)];
-            sa[k] += o.x;
-            sb[k] += o.y;
-        }
-    } else {
+    else
         named_bar_sync(1, 128);
+    float tot[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            float a = 0.f, b = 0.f;
+    for (int w = 0; w < NW; ++w) {
+        const int ww = NW == 2 ? (q & 2) + w : w;
+        const float4* src = reinterpret_cast<const float4*>(red + (ww * 4 + c) * 8);
+        const float4 x0 = src[0], x1 = src[1];
+        tot[0] += x0.x; tot[1] += x0.y; tot[2] += x0.z; tot[3] += x0.w;
+        tot[4] += x1.x; tot[5] += x1.y; tot[6] += x1.z; tot[7] += x1.w;
+    }
 #pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                const float2 o = red[w * 16 + 8 * (k >> 1) + 2 * c + (k & 1)];
-                a += o.x;
-                b += o.y;
-            }
-            sa[k] = a;
-            sb[k] = b;
-        }
+    for (int k = 0; k < 4; ++k) {
+        sa[k] = tot[k];
+        sb[k] = tot[4 + k];
     }
 }
 
@@ -417,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
         uint8_t* zs = smem + kOffZs + q * kZsBytes;   // this warp's Z staging tile
         // LN: gamma, beta and the bias state c of this thread's rows jb + 16 mt + r + 8 h
         float gam[2][2] = {}, bet[2][2] = {}, cst[2][2] = {};
-        float2* red = reinterpret_cast<float2*>(smem + kOffRed);
+        float* red = reinterpret_cast<float*>(smem + kOffRed);
         int nred = 0;   // reductions so far (two alternating buffers)
         if (LN) {
 #pragma unroll
@@ -431,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 }
         }
         auto rsum = [&](float* sa, float* sb) {
-            tok_sum2<4 / NMT>(sa, sb, red + (nred & 1) * 64, q, lane);
+            tok_sum2<4 / NMT>(sa, sb, red + (nred & 1) * 128, q, lane);
             ++nred;
         };
         // W_0^T row j = column j of W_0, in fp32 and bf16; the other unit's
@@ -523,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                     mbar_arrive(aw_ready);
                     mbar_arrive(&empty[(g - 1) % kStages]);   // MMA_W of pair g-1 was its last reader
                 }
-                store_z(g - 1);
+                if (UPC == 2) store_z(g - 1);
             }
             // 1. inputs: eta, eta * V (accumulator layout), the token products
             WT(&full[g % kStages], (g / kStages) & 1);
@@ -574,6 +584,10 @@ __global__ void __launch_bounds__(kThreads, LN ? 1 : 2)
                 ldsm_x4(a + 2 * kMat, m1);
                 ldsm_x4(a + 3 * kMat, m2);
             }
+            // one unit per CTA: the previous pair's Z goes out while these loads are in
+            // flight (measured faster there; with two units per CTA and two CTAs per SM
+            // the other CTA hides the load latency and the earlier store is better)
+            if (UPC == 1 && g >= 1) store_z(g - 1);
             // 2. P of the pair (E parts), accumulator layout
             WT(p_ready, g & 1);
             tc_fence_after();
