@@ -482,12 +482,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // bf16 W2 (state after batch i's update) -> buffer buf: this warp's 32 columns of row h
         auto refresh_w2 = [&](int buf) {
             uint8_t* dst = w2s + 32768 * buf;
+            uint32_t w2r[2][32];   // both tiles' loads in flight before one wait
+            tmem_ld_32x32b_x32(tl + cW2 + 32 * hf, w2r[0]);
+            tmem_ld_32x32b_x32(tl + cW2 + 64 + 32 * hf, w2r[1]);
+            tmem_wait_ld();
 #pragma unroll
             for (int tt = 0; tt < 2; ++tt) {
                 const int h = hr[tt];
-                uint32_t w[32];
-                tmem_ld_32x32b_x32(tl + cW2 + 64 * tt + 32 * hf, w);
-                tmem_wait_ld();
+                const uint32_t* w = w2r[tt];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     uint4 v;
@@ -713,14 +715,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int m = 0; m < 2; ++m)
                     tmem_ld_16x256b_x1(tbase + ((uint32_t)(32 * qd + 16 * m) << 16) + cA + 32 * tt + 16 + 8 * hf, rq[tt][m]);
-#pragma unroll
-            for (int tt = 0; tt < 2; ++tt) {
-                uint32_t w[32], pk[16];
-                tmem_ld_32x32b_x32(tl + cW1 + 64 * tt + 32 * hf, w);
+            {
+                // both tiles' loads in flight before one wait
+                uint32_t w[2][32];
+                tmem_ld_32x32b_x32(tl + cW1 + 32 * hf, w[0]);
+                tmem_ld_32x32b_x32(tl + cW1 + 64 + 32 * hf, w[1]);
                 tmem_wait_ld();
 #pragma unroll
-                for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(__uint_as_float(w[2 * k]), __uint_as_float(w[2 * k + 1]));
-                tmem_st_32x32b_x16(tl + cAW1 + 32 * tt + 16 * hf, pk);
+                for (int tt = 0; tt < 2; ++tt) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        pk[k] = pack_bf16x2(__uint_as_float(w[tt][2 * k]), __uint_as_float(w[tt][2 * k + 1]));
+                    tmem_st_32x32b_x16(tl + cAW1 + 32 * tt + 16 * hf, pk);
+                }
             }
             tmem_wait_st();
             tc_fence_before();
