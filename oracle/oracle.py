@@ -33,6 +33,8 @@ def lib():
         L.ttt_oracle_mlp_forward.restype = i
         L.ttt_oracle_linear_decode_step.argtypes = [i, i, i, P, P, P, P, P, P]
         L.ttt_oracle_linear_decode_step.restype = i
+        L.ttt_oracle_linear_backward.argtypes = [i, i, i, i, i, P, P, P, P, P, ll, P, P, P, P, P, P, P, i]
+        L.ttt_oracle_linear_backward.restype = i
         _lib = L
     return _lib
 
@@ -114,3 +116,22 @@ def linear_decode_step(W, q, k, v, eta):
     if rc != 0:
         raise ValueError("oracle: invalid arguments")
     return W, z
+
+
+def linear_backward(Q, K, V, eta, W0, b, dZ=None, dW_out=None, threads=None):
+    """Outer-loop gradients of the TTT-Linear forward (no LN), reverse mode
+    through the primal loop.  dZ [B,H,T,d] and dW_out [B,H,d,d] are the
+    gradients of a scalar loss with respect to the forward's outputs (None:
+    zero).  Returns (dQ, dK, dV [B,H,T,d], deta [B,H,T], dW0 [B,H,d,d]),
+    dW0 per sequence (sum over B for a shared W0)."""
+    Q, K, V, eta, W0, dZ, dW_out = map(_f64, (Q, K, V, eta, W0, dZ, dW_out))
+    B, H, T, d = Q.shape
+    W0_bstride = 0 if W0.ndim == 3 else H * d * d
+    dQ, dK, dV = np.empty((B, H, T, d)), np.empty((B, H, T, d)), np.empty((B, H, T, d))
+    deta, dW0 = np.empty((B, H, T)), np.empty((B, H, d, d))
+    rc = lib().ttt_oracle_linear_backward(B, H, T, d, b, _p(Q), _p(K), _p(V), _p(eta), _p(W0), W0_bstride,
+                                          _p(dZ), _p(dW_out), _p(dQ), _p(dK), _p(dV), _p(deta), _p(dW0),
+                                          threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: invalid arguments")
+    return dQ, dK, dV, deta, dW0

@@ -30,6 +30,10 @@
  *     value per token, scaling that token's own gradient.
  *   - Decode / generate uses the primal form one token at a time (section
  *     6.11): the b = 1 update followed by the output.
+ *   - Outer-loop gradients (section 3.3: the outer loop trains the
+ *     projections and the initial state through the inner loop's updates):
+ *     the backward of the TTT-Linear forward is reverse-mode
+ *     differentiation of the same primal loop, token by token.
  *
  * Readings of points the pages leave open (each one is listed in the design
  * notes of the repository):
@@ -313,6 +317,139 @@ int ttt_oracle_linear_decode_step(int B, int H, int d, double *W, const double *
             for (int j = 0; j < d; ++j) Wu[(size_t)i * d + j] -= eta[u] * ku[i] * e[j];
         vec_mat(d, d, qu, Wu, z + (size_t)u * d);
         free(e);
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Backward of the TTT-Linear forward (no LN): reverse-mode differentiation of
+ * the primal loop above, token by token, for the outer-loop gradients.
+ *
+ * The loss is any scalar L of the forward's outputs; the caller passes
+ * dZ = dL/dZ [B,H,T,d] and dW_out = dL/dW_out [B,H,d,d] (either may be NULL
+ * for zero).  Returned: dQ, dK, dV [B,H,T,d], deta [B,H,T] and dW0 [B,H,d,d]
+ * (one per sequence, even when W0 is shared: the caller sums over B).
+ *
+ * Forward of one mini-batch with batch-start state W_s, token by token:
+ *     e_t = k_t W_s - v_t,   W_t = W_{t-1} - eta_t k_t^T e_t,   z_t = q_t W_t.
+ * Reverse, with D the gradient with respect to the running state (starting
+ * at the gradient with respect to the state after the batch), for
+ * t = last .. first:
+ *     dq_t  = dz_t W_t^T,             D += q_t^T dz_t
+ *     deta_t = -<D, k_t^T e_t>,       de_t = -eta_t k_t D
+ *     dk_t  = -eta_t e_t D^T + de_t W_s^T,   dv_t = -de_t
+ *     dW_s += k_t^T de_t
+ * and the gradient with respect to the batch-start state is D + dW_s.
+ * The batch-start states come from a forward re-run; the running states W_t
+ * of a mini-batch are recomputed from its start.
+ * ------------------------------------------------------------------------- */
+static void linear_unit_backward(int T, int d, int b, const double *Q, const double *K, const double *V,
+                                 const double *eta, const double *W0, const double *dZ, const double *dWout,
+                                 double *dQ, double *dK, double *dV, double *deta, double *dW0) {
+    const size_t dd = (size_t)d * d;
+    const int nb = (T + b - 1) / b;
+    double *starts = malloc((size_t)(nb > 0 ? nb : 1) * dd * sizeof(double));  /* state at each batch start */
+    double *Wrun = malloc((size_t)(b + 1) * dd * sizeof(double));               /* W_{t0-1} .. W_{t1-1} */
+    double *D = malloc(dd * sizeof(double));
+    double *dWs = malloc(dd * sizeof(double));
+    double *e = malloc((size_t)b * d * sizeof(double));
+    double *de = malloc(d * sizeof(double));
+    double *Wc = malloc(dd * sizeof(double));
+    /* forward re-run: batch-start states */
+    memcpy(Wc, W0, dd * sizeof(double));
+    for (int i = 0; i < nb; ++i) {
+        const int t0 = i * b, t1 = (t0 + b < T) ? t0 + b : T;
+        memcpy(starts + (size_t)i * dd, Wc, dd * sizeof(double));
+        for (int t = t0; t < t1; ++t) {
+            double *et = e + (size_t)(t - t0) * d;
+            vec_mat(d, d, K + (size_t)t * d, starts + (size_t)i * dd, et);
+            for (int j = 0; j < d; ++j) et[j] -= V[(size_t)t * d + j];
+            for (int a = 0; a < d; ++a)
+                for (int j = 0; j < d; ++j) Wc[(size_t)a * d + j] -= eta[t] * K[(size_t)t * d + a] * et[j];
+        }
+    }
+    /* reverse sweep */
+    if (dWout) memcpy(D, dWout, dd * sizeof(double));
+    else memset(D, 0, dd * sizeof(double));
+    for (int i = nb - 1; i >= 0; --i) {
+        const int t0 = i * b, t1 = (t0 + b < T) ? t0 + b : T;
+        const double *Ws = starts + (size_t)i * dd;
+        /* running states of the batch: Wrun[0] = W_s, Wrun[t - t0 + 1] = W_t */
+        memcpy(Wrun, Ws, dd * sizeof(double));
+        for (int t = t0; t < t1; ++t) {
+            double *et = e + (size_t)(t - t0) * d;
+            vec_mat(d, d, K + (size_t)t * d, Ws, et);
+            for (int j = 0; j < d; ++j) et[j] -= V[(size_t)t * d + j];
+            const double *Wp = Wrun + (size_t)(t - t0) * dd;
+            double *Wn = Wrun + (size_t)(t - t0 + 1) * dd;
+            for (int a = 0; a < d; ++a)
+                for (int j = 0; j < d; ++j)
+                    Wn[(size_t)a * d + j] = Wp[(size_t)a * d + j] - eta[t] * K[(size_t)t * d + a] * et[j];
+        }
+        memset(dWs, 0, dd * sizeof(double));
+        for (int t = t1 - 1; t >= t0; --t) {
+            const double *q = Q + (size_t)t * d, *k = K + (size_t)t * d;
+            const double *dz = dZ ? dZ + (size_t)t * d : NULL;
+            const double *Wt = Wrun + (size_t)(t - t0 + 1) * dd;
+            const double *et = e + (size_t)(t - t0) * d;
+            /* z_t = q_t W_t */
+            for (int a = 0; a < d; ++a) {
+                double acc = 0.0;
+                if (dz)
+                    for (int j = 0; j < d; ++j) acc += dz[j] * Wt[(size_t)a * d + j];
+                dQ[(size_t)t * d + a] = acc;
+            }
+            if (dz)
+                for (int a = 0; a < d; ++a)
+                    for (int j = 0; j < d; ++j) D[(size_t)a * d + j] += q[a] * dz[j];
+            /* W_t = W_{t-1} - eta_t k_t^T e_t */
+            double ge = 0.0;
+            for (int a = 0; a < d; ++a)
+                for (int j = 0; j < d; ++j) ge += D[(size_t)a * d + j] * k[a] * et[j];
+            deta[t] = -ge;
+            for (int j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int a = 0; a < d; ++a) acc += k[a] * D[(size_t)a * d + j];
+                de[j] = -eta[t] * acc;
+            }
+            for (int a = 0; a < d; ++a) {
+                double acc1 = 0.0, acc2 = 0.0;
+                for (int j = 0; j < d; ++j) {
+                    acc1 += et[j] * D[(size_t)a * d + j];
+                    acc2 += de[j] * Ws[(size_t)a * d + j];
+                }
+                dK[(size_t)t * d + a] = -eta[t] * acc1 + acc2;
+            }
+            for (int j = 0; j < d; ++j) dV[(size_t)t * d + j] = -de[j];
+            /* e_t = k_t W_s - v_t */
+            for (int a = 0; a < d; ++a)
+                for (int j = 0; j < d; ++j) dWs[(size_t)a * d + j] += k[a] * de[j];
+        }
+        for (size_t x = 0; x < dd; ++x) D[x] += dWs[x];
+    }
+    memcpy(dW0, D, dd * sizeof(double));
+    free(starts); free(Wrun); free(D); free(dWs); free(e); free(de); free(Wc);
+}
+
+int ttt_oracle_linear_backward(int B, int H, int T, int d, int b, const double *Q, const double *K,
+                               const double *V, const double *eta, const double *W0, long long W0_bstride,
+                               const double *dZ, const double *dW_out, double *dQ, double *dK, double *dV,
+                               double *deta, double *dW0, int threads) {
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0 || !Q || !K || !V || !eta || !W0 || !dQ || !dK || !dV ||
+        !deta || !dW0)
+        return 1;
+    const long long units = (long long)B * H;
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long long u = 0; u < units; ++u) {
+        const long long n = u / H, h = u % H;
+        const size_t tok = (size_t)u * T * d;
+        linear_unit_backward(T, d, b, Q + tok, K + tok, V + tok, eta + (size_t)u * T,
+                             W0 + (size_t)n * W0_bstride + (size_t)h * d * d, dZ ? dZ + tok : NULL,
+                             dW_out ? dW_out + (size_t)u * d * d : NULL, dQ + tok, dK + tok, dV + tok,
+                             deta + (size_t)u * T, dW0 + (size_t)u * d * d);
     }
     return 0;
 }

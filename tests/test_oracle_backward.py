@@ -1,0 +1,85 @@
+"""Pins of the oracle's outer-loop backward (TTT-Linear, no LN).
+
+The backward is reverse-mode differentiation of the primal mini-batch loop
+(paper digest "论文速览 | TTT", sections 3.5-3.6: the state W is updated by
+gradient steps inside the forward, so the outer loop differentiates through
+those steps).  It is pinned against central finite differences of the
+forward oracle, which is itself pinned elsewhere, and against the closed
+form at eta = 0, where the layer reduces to Z = Q W0 and W_out = W0.
+"""
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+
+
+def _case(B, H, T, d, shared_w0, seed):
+    rng = np.random.default_rng(seed)
+    Q = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
+    K = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
+    V = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
+    eta = 0.2 + 0.3 * rng.random((B, H, T))
+    W0 = rng.standard_normal((H, d, d) if shared_w0 else (B, H, d, d)) / np.sqrt(d)
+    dZ = rng.standard_normal((B, H, T, d))
+    dW = rng.standard_normal((B, H, d, d))
+    return Q, K, V, eta, W0, dZ, dW
+
+
+def _loss(Q, K, V, eta, W0, b, dZ, dW):
+    Z, W_out, _ = O.linear_forward(Q, K, V, eta, W0, b, threads=1)
+    return float(np.sum(Z * dZ) + np.sum(W_out * dW))
+
+
+@pytest.mark.parametrize("B,H,T,d,b,shared", [
+    (1, 2, 5, 3, 2, True),     # ragged last mini-batch
+    (2, 1, 6, 2, 3, False),    # per-sequence W0
+    (1, 1, 4, 3, 1, True),     # b = 1: the sequential delta rule
+    (1, 1, 4, 2, 4, True),     # one mini-batch, b = T
+])
+def test_backward_matches_finite_differences(B, H, T, d, b, shared):
+    Q, K, V, eta, W0, dZ, dW = _case(B, H, T, d, shared, seed=10 * T + d + b)
+    dQ, dK, dV, deta, dW0 = O.linear_backward(Q, K, V, eta, W0, b, dZ=dZ, dW_out=dW, threads=1)
+    if shared:
+        dW0 = dW0.sum(axis=0)
+    grads = {"Q": dQ, "K": dK, "V": dV, "eta": deta, "W0": dW0}
+    inputs = {"Q": Q, "K": K, "V": V, "eta": eta, "W0": W0}
+    h = 1e-6
+    for name, x in inputs.items():
+        g = grads[name]
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            keep = x[idx]
+            x[idx] = keep + h
+            lp = _loss(*inputs.values(), b, dZ, dW)
+            x[idx] = keep - h
+            lm = _loss(*inputs.values(), b, dZ, dW)
+            x[idx] = keep
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.max(np.abs(fd - g)) / max(np.max(np.abs(fd)), 1e-12)
+        assert err < 1e-7, (name, err)
+
+
+def test_backward_at_zero_eta_is_the_linear_map():
+    """eta = 0: Z = Q W0 and W_out = W0, so dQ = dZ W0^T, dW0 = Q^T dZ + dW_out,
+    dK = dV = 0; deta_t = -<D_t, k_t^T e_t> with e_t = k_t W0 - v_t and D_t the
+    state gradient after token t (dW_out plus the outputs at t and later)."""
+    B, H, T, d, b = 1, 1, 6, 4, 3
+    Q, K, V, eta, W0, dZ, dW = _case(B, H, T, d, True, seed=3)
+    eta = np.zeros_like(eta)
+    dQ, dK, dV, deta, dW0 = O.linear_backward(Q, K, V, eta, W0, b, dZ=dZ, dW_out=dW, threads=1)
+    W = W0[0]
+    q, k, v, dz = Q[0, 0], K[0, 0], V[0, 0], dZ[0, 0]
+    np.testing.assert_allclose(dQ[0, 0], dz @ W.T, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dW0[0, 0], q.T @ dz + dW[0, 0], rtol=0, atol=1e-13)
+    assert np.all(dK == 0) and np.all(dV == 0)
+    e = k @ W - v
+    for t in range(T):
+        D = dW[0, 0] + q[t:].T @ dz[t:]
+        assert abs(deta[0, 0, t] + k[t] @ D @ e[t]) < 1e-12
+
+
+def test_backward_without_upstream_gradients_is_zero():
+    Q, K, V, eta, W0, _, _ = _case(1, 2, 4, 3, True, seed=5)
+    out = O.linear_backward(Q, K, V, eta, W0, 2, threads=1)
+    for g in out:
+        assert np.all(g == 0)

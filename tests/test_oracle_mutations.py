@@ -32,6 +32,18 @@ MUTATIONS = {
         "        free(e);"),
 }
 
+# mistakes in the outer-loop backward, caught by its own pins
+BACKWARD_MUTATIONS = {
+    "bwd_eta_grad_sign": ("deta[t] = -ge;", "deta[t] = ge;"),
+    "bwd_dq_from_batch_start": ("acc += dz[j] * Wt[(size_t)a * d + j];", "acc += dz[j] * Ws[(size_t)a * d + j];"),
+    "bwd_missing_residual_path": ("dK[(size_t)t * d + a] = -eta[t] * acc1 + acc2;",
+                                  "dK[(size_t)t * d + a] = -eta[t] * acc1;"),
+    "bwd_state_grad_drops_residual": ("for (size_t x = 0; x < dd; ++x) D[x] += dWs[x];", "(void)dWs;"),
+    "bwd_output_grad_dropped_from_state": (
+        "            if (dz)\n                for (int a = 0; a < d; ++a)\n                    for (int j = 0; j < d; ++j) D[(size_t)a * d + j] += q[a] * dz[j];\n",
+        ""),
+}
+
 
 def _build_mutant(name, old, new, tmp):
     src = open(SRC).read()
@@ -48,13 +60,14 @@ def _build_mutant(name, old, new, tmp):
     return so
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS))
+@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(BACKWARD_MUTATIONS))
 def test_pins_catch_planted_mistake(name):
-    old, new = MUTATIONS[name]
+    old, new = MUTATIONS[name] if name in MUTATIONS else BACKWARD_MUTATIONS[name]
+    pins = "test_oracle_backward.py" if name in BACKWARD_MUTATIONS else "test_oracle_pins.py"
     with tempfile.TemporaryDirectory() as tmp:
         so = _build_mutant(name, old, new, tmp)
         env = dict(os.environ, TTT_ORACLE_LIB_OVERRIDE=so)
         r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
-                            os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                            os.path.join(ROOT, "tests", pins)],
                            env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
         assert r.returncode != 0, f"mutation {name} survived the pins:\n{r.stdout[-2000:]}"
