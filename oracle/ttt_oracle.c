@@ -30,8 +30,9 @@
  *     value per token, scaling that token's own gradient.
  *   - Decode / generate uses the primal form one token at a time (section
  *     6.11): the b = 1 update followed by the output.
- *   - Outer-loop gradients (section 3.3: the outer loop trains the
- *     projections and the initial state through the inner loop's updates):
+ *   - Outer-loop gradients (section 3.4: the outer loop trains the
+ *     projections, the initial state and the learning-rate parameters with
+ *     gradients that pass through the inner loop's updates):
  *     the backward of the TTT-Linear forward is reverse-mode
  *     differentiation of the same primal loop, token by token.
  *

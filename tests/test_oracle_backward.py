@@ -1,9 +1,8 @@
 """Pins of the oracle's outer-loop backward (TTT-Linear, no LN).
 
 The backward is reverse-mode differentiation of the primal mini-batch loop
-(paper digest "论文速览 | TTT", sections 3.5-3.6: the state W is updated by
-gradient steps inside the forward, so the outer loop differentiates through
-those steps).  It is pinned against central finite differences of the
+(paper digest "论文速览 | TTT", section 3.4: the outer loop's gradients pass
+through the inner loop's updates of W; sections 3.5-3.6 define those updates).  It is pinned against central finite differences of the
 forward oracle, which is itself pinned elsewhere, and against the closed
 form at eta = 0, where the layer reduces to Z = Q W0 and W_out = W0.
 """
