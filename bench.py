@@ -352,6 +352,41 @@ def measure_decode_variant(ttt, torch, kind, B, H, d=64, n=1024, steps=3):
             "note": "state stays L2-resident across steps; GB/s is against HBM peak for reference"}
 
 
+def measure_backward(ttt, torch, threads, name="linear_B8_H12_T2048"):
+    """Outer-loop backward of TTT-Linear on a workload's shapes: the forward
+    that also writes the batch-start states, then the backward with random
+    upstream gradients (informational; parity lives in the tests)."""
+    w = WL.WORKLOADS[name]
+    _, dev = device_inputs(w, torch, threads)
+    B, H, T, d = w.B, w.H, w.T, w.d
+    states = torch.empty((B, H, T // w.b, d, d), device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(2)
+    dZ = torch.randn(B, H, T, d, generator=g, device="cuda").to(dev["Q"].dtype)
+    dW = torch.randn(B, H, d, d, generator=g, device="cuda")
+    outs = [torch.empty_like(dev["Q"]) for _ in range(3)]
+    deta = torch.empty((B, H, T), device="cuda")
+    dW0 = torch.empty((B, H, d, d), device="cuda")
+    flush_buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")
+
+    def fwd():
+        ttt.linear_forward(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], w.b, W_states=states)
+
+    def bwd():
+        ttt.linear_backward(dev["Q"], dev["K"], dev["V"], dev["eta"], states, w.b, dZ=dZ, dW_out=dW,
+                            dQ=outs[0], dK=outs[1], dV=outs[2], deta=deta, dW0=dW0)
+    ms_f = statistics.median(time_launches(torch, fwd, 5, 2, flush=lambda: flush_buf.zero_()))
+    ms_b = statistics.median(time_launches(torch, bwd, 5, 2, flush=lambda: flush_buf.zero_()))
+    io = dev["Q"].element_size()
+    units = B * H
+    bytes_b = units * (T * d * io * 7 + T * 8 + (T // w.b) * d * d * 4 + 3 * d * d * 4)
+    hbm, _, _ = measured_peaks()
+    return {"workload": name, "forward_with_states_ms": ms_f, "backward_ms": ms_b,
+            "tokens_per_s_backward": tokens(w) / (ms_b / 1000.0),
+            "backward_bytes": bytes_b, "backward_hbm_frac": bytes_b / (ms_b / 1000.0) / 1e9 / hbm,
+            "kernel": "simt_linear_backward_kernel (fp32 CUDA cores)"}
+
+
 def measure_e2e_chunked(ttt, w, inp, torch, steps, chunks=8):
     """The public API on pinned host buffers, streamed along the sequence:
     the T tokens go through `chunks` calls of ttt_linear_forward, each
@@ -582,6 +617,7 @@ def run_ours(args):
             line["rows"] = measure_rows(ttt, torch, threads)
             line["rows"]["decode_ln_B4_H32"] = measure_decode_variant(ttt, torch, "ln", 4, 32)
             line["rows"]["decode_mlp_B2_H32"] = measure_decode_variant(ttt, torch, "mlp", 2, 32)
+            line["rows"]["backward_linear_B8_H12_T2048"] = measure_backward(ttt, torch, threads)
         line["cpu_baseline"] = cpu_baseline(w)
     if dist is not None:
         dist.barrier()

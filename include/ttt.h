@@ -95,6 +95,11 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
  *   c_out          LN only: final bias [B, H, d] fp32, or NULL.
  *   flags          TTT_FLAG_* bits; 0 for normal use.
  *   wait_timeout_ms  limit of every device-side wait (0: 2000 ms).
+ *   W_states       optional output for the backward (gradient checkpointing
+ *                  through time, section 6.12): the state at the start of
+ *                  every mini-batch, [B, H, T/b, d, d] fp32, T/b states per
+ *                  unit.  NULL: not written.  Non-NULL requires use_ln == 0
+ *                  and runs the fp32 CUDA-core kernel.
  */
 typedef struct {
     int B, H, T, d, b;
@@ -117,9 +122,52 @@ typedef struct {
     float* c_out;
     unsigned flags;
     unsigned wait_timeout_ms;
+    float* W_states;
 } ttt_linear_args;
 
 ttt_status ttt_linear_forward(const ttt_linear_args* args, cudaStream_t stream);
+
+/*
+ * ttt_linear_backward -- outer-loop gradients of the TTT-Linear prefill
+ * (use_ln == 0): given dZ = dL/dZ and dW_out = dL/dW_out of a scalar loss L,
+ * returns dL/dQ, dL/dK, dL/dV, dL/deta and dL/dW0.  The outer loop trains
+ * the projections, the initial state and the learning rates through the
+ * inner loop's updates (section 3.4).  The mini-batches are visited last to
+ * first; each recomputes its residual E = K W - V and the causal products
+ * from its batch-start state W (section 6.12: only the kappa = T/b boundary
+ * states are kept), which ttt_linear_forward wrote to W_states.
+ *
+ *   B, H, T, d, b, io_dtype, Q, K, V, eta, eta_const
+ *                  the forward's arguments (same rules; T % b == 0,
+ *                  d in {16, 32, 64}, 1 <= b <= 64).
+ *   W_states       [B, H, T/b, d, d] fp32 from the forward with the same inputs.
+ *   dZ             [B, H, T, d] in io_dtype, or NULL for zero.
+ *   dW_out         [B, H, d, d] fp32, or NULL for zero.
+ *   dQ, dK, dV     outputs [B, H, T, d] in io_dtype.
+ *   deta           output [B, H, T] fp32, or NULL when not wanted.
+ *   dW0            output [B, H, d, d] fp32, one per sequence (a W0 shared
+ *                  over the batch receives the sum over B).
+ * Computed on the fp32 CUDA-core kernel, one CTA per (sequence, head) unit.
+ */
+typedef struct {
+    int B, H, T, d, b;
+    ttt_dtype io_dtype;
+    const void* Q;
+    const void* K;
+    const void* V;
+    const float* eta;
+    float eta_const;
+    const float* W_states;
+    const void* dZ;
+    const float* dW_out;
+    void* dQ;
+    void* dK;
+    void* dV;
+    float* deta;
+    float* dW0;
+} ttt_linear_backward_args;
+
+ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_t stream);
 
 /*
  * ttt_mlp_forward -- prefill of TTT-MLP, f(x) = GELU(x W1 + c1) W2 + c2 with

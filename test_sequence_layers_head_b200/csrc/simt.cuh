@@ -39,6 +39,7 @@ struct SimtLinearParams {
     void* Z;
     float* W_out;
     float* c_out;
+    float* W_states;   // optional [units, T/b, D, D]: the state at the start of every mini-batch
 };
 
 // Row statistics helper: LN over n features of row `row` (warp-cooperative).
@@ -88,6 +89,10 @@ __global__ void __launch_bounds__(kSimtThreads) simt_linear_kernel(SimtLinearPar
     const int warp = tid / 32, nwarps = kSimtThreads / 32;
     __syncthreads();
     for (int t0 = 0; t0 < p.T; t0 += b) {
+        if (p.W_states) {
+            float* ws = p.W_states + ((size_t)unit * (p.T / b) + t0 / b) * D * D;
+            for (int e = tid; e < D * D; e += kSimtThreads) ws[e] = W[e];
+        }
         // load the mini-batch
         for (int e = tid; e < b * D; e += kSimtThreads) {
             const size_t g = (size_t)t0 * D + e;

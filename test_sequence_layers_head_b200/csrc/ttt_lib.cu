@@ -14,6 +14,7 @@
 #include "mlp_decode.cuh"
 #include "mlp_tc.cuh"
 #include "simt.cuh"
+#include "simt_backward.cuh"
 #include "tmap.h"
 
 namespace ttt {
@@ -88,6 +89,7 @@ ttt_status launch_simt_linear(const ttt_linear_args* a, cudaStream_t st) {
     p.Z = a->Z;
     p.W_out = a->W_out;
     p.c_out = a->c_out;
+    p.W_states = a->W_states;
     const size_t smem = simt_linear_smem(D, a->b);
     auto k = simt_linear_kernel<D, LN, IO>;
     if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
@@ -199,8 +201,12 @@ extern "C" ttt_status ttt_linear_forward(const ttt_linear_args* a, cudaStream_t 
         return TTT_ERR_INVALID_ARG;
     if ((a->flags & TTT_FLAG_ONE_UNIT_PER_CTA) && (a->flags & TTT_FLAG_TWO_UNITS_PER_CTA))
         return TTT_ERR_INVALID_ARG;
+    if (a->W_states) {
+        if (!aligned16(a->W_states)) return TTT_ERR_INVALID_ARG;
+        if (a->use_ln) return TTT_ERR_UNSUPPORTED;
+    }
     const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
-                    !(a->flags & TTT_FLAG_FORCE_SIMT);
+                    !(a->flags & TTT_FLAG_FORCE_SIMT) && !a->W_states;
     if (tc) return a->use_ln ? tc_linear<true>(a, stream) : tc_linear<false>(a, stream);
     if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
     return a->use_ln ? simt_linear<true>(a, stream) : simt_linear<false>(a, stream);
@@ -388,6 +394,44 @@ extern "C" ttt_status ttt_mlp_decode_step(const ttt_mlp_decode_args* a, cudaStre
         case 16: return launch_mlp_decode<16>(a, stream);
         case 32: return launch_mlp_decode<32>(a, stream);
         default: return launch_mlp_decode<64>(a, stream);
+    }
+}
+
+namespace ttt {
+namespace {
+template <int D, typename IO>
+ttt_status launch_linear_backward_t(const ttt_linear_backward_args* a, cudaStream_t st) {
+    SimtBackwardParams p{a->H, a->T, a->b, a->Q, a->K, a->V, a->eta, a->eta_const, a->W_states,
+                         a->dZ, a->dW_out, a->dQ, a->dK, a->dV, a->deta, a->dW0};
+    const size_t smem = simt_backward_smem(D, a->b);
+    auto k = simt_linear_backward_kernel<D, IO>;
+    if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
+    k<<<a->B * a->H, kSimtThreads, smem, st>>>(p);
+    return launch_status();
+}
+template <int D>
+ttt_status launch_linear_backward(const ttt_linear_backward_args* a, cudaStream_t st) {
+    return a->io_dtype == TTT_F32 ? launch_linear_backward_t<D, float>(a, st)
+                                  : launch_linear_backward_t<D, __nv_bfloat16>(a, st);
+}
+}  // namespace
+}  // namespace ttt
+
+extern "C" ttt_status ttt_linear_backward(const ttt_linear_backward_args* a, cudaStream_t stream) {
+    if (!a) return TTT_ERR_INVALID_ARG;
+    ttt_status v = validate_common(a->B, a->H, a->T, a->d, a->b, a->io_dtype);
+    if (v != TTT_OK) return v;
+    const long long units = (long long)a->B * a->H;
+    if (units == 0) return TTT_OK;
+    if (a->T > 0 && (!ok_ptr(a->Q) || !ok_ptr(a->K) || !ok_ptr(a->V) || !ok_ptr(a->W_states) ||
+                     !ok_ptr(a->dQ) || !ok_ptr(a->dK) || !ok_ptr(a->dV)))
+        return TTT_ERR_INVALID_ARG;
+    if (!ok_ptr(a->dW0) || !ok_opt(a->eta) || !ok_opt(a->dZ) || !ok_opt(a->dW_out) || !ok_opt(a->deta))
+        return TTT_ERR_INVALID_ARG;
+    switch (a->d) {
+        case 16: return launch_linear_backward<16>(a, stream);
+        case 32: return launch_linear_backward<32>(a, stream);
+        default: return launch_linear_backward<64>(a, stream);
     }
 }
 

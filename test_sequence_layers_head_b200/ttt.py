@@ -38,7 +38,8 @@ class LinearArgs(ctypes.Structure):
                 ("Q", _vp), ("K", _vp), ("V", _vp), ("eta", _vp), ("eta_const", _f),
                 ("W0", _vp), ("W0_bstride", _ll), ("c0", _vp), ("c0_bstride", _ll),
                 ("use_ln", _i), ("ln_gamma", _vp), ("ln_beta", _vp), ("ln_eps", _f),
-                ("Z", _vp), ("W_out", _vp), ("c_out", _vp), ("flags", _u), ("wait_timeout_ms", _u)]
+                ("Z", _vp), ("W_out", _vp), ("c_out", _vp), ("flags", _u), ("wait_timeout_ms", _u),
+                ("W_states", _vp)]
 
 
 class MlpArgs(ctypes.Structure):
@@ -55,6 +56,12 @@ class DecodeArgs(ctypes.Structure):
                 ("ln_gamma", _vp), ("ln_beta", _vp), ("ln_eps", _f)]
 
 
+class BackwardArgs(ctypes.Structure):
+    _fields_ = [("B", _i), ("H", _i), ("T", _i), ("d", _i), ("b", _i), ("io_dtype", _i), ("Q", _vp), ("K", _vp),
+                ("V", _vp), ("eta", _vp), ("eta_const", _f), ("W_states", _vp), ("dZ", _vp), ("dW_out", _vp),
+                ("dQ", _vp), ("dK", _vp), ("dV", _vp), ("deta", _vp), ("dW0", _vp)]
+
+
 class MlpDecodeArgs(ctypes.Structure):
     _fields_ = [("B", _i), ("H", _i), ("d", _i), ("io_dtype", _i), ("W1", _vp), ("c1", _vp), ("W2", _vp),
                 ("c2", _vp), ("q", _vp), ("k", _vp), ("v", _vp), ("eta", _vp), ("eta_const", _f), ("z", _vp)]
@@ -69,8 +76,8 @@ class TTTError(RuntimeError):
 _lib = None
 
 # Every symbol include/ttt.h declares.
-EXPORTS = ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_mlp_decode_step",
-           "ttt_status_string", "ttt_last_device_status", "ttt_version")
+EXPORTS = ("ttt_linear_forward", "ttt_linear_backward", "ttt_mlp_forward", "ttt_linear_decode_step",
+           "ttt_mlp_decode_step", "ttt_status_string", "ttt_last_device_status", "ttt_version")
 
 
 def library() -> ctypes.CDLL:
@@ -83,6 +90,8 @@ def library() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         L.ttt_linear_forward.argtypes = [ctypes.POINTER(LinearArgs), _vp]
         L.ttt_linear_forward.restype = _i
+        L.ttt_linear_backward.argtypes = [ctypes.POINTER(BackwardArgs), _vp]
+        L.ttt_linear_backward.restype = _i
         L.ttt_mlp_forward.argtypes = [ctypes.POINTER(MlpArgs), _vp]
         L.ttt_mlp_forward.restype = _i
         L.ttt_linear_decode_step.argtypes = [ctypes.POINTER(DecodeArgs), _vp]
@@ -136,7 +145,8 @@ def _check(code: int, what: str):
 
 
 def linear_forward(Q, K, V, eta, W0, b, *, eta_const=0.0, use_ln=False, c0=None, gamma=None, beta=None,
-                   eps=1e-6, Z=None, W_out=None, c_out=None, flags=0, wait_timeout_ms=0, stream=None):
+                   eps=1e-6, Z=None, W_out=None, c_out=None, flags=0, wait_timeout_ms=0, W_states=None,
+                   stream=None):
     """TTT-Linear (optionally LN+residual) prefill; see ``ttt_linear_forward``.
 
     Q, K, V: [B,H,T,d] bf16 or fp32; eta: [B,H,T] fp32 or None (eta_const);
@@ -154,9 +164,30 @@ def linear_forward(Q, K, V, eta, W0, b, *, eta_const=0.0, use_ln=False, c0=None,
     c0_bstride = H * d if (c0 is not None and c0.dim() == 3) else 0
     a = LinearArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
                    _ptr(W0), W0_bstride, _ptr(c0), c0_bstride, int(bool(use_ln)), _ptr(gamma), _ptr(beta),
-                   float(eps), _ptr(Z), _ptr(W_out), _ptr(c_out), int(flags), int(wait_timeout_ms))
+                   float(eps), _ptr(Z), _ptr(W_out), _ptr(c_out), int(flags), int(wait_timeout_ms),
+                   _ptr(W_states))
     _check(library().ttt_linear_forward(ctypes.byref(a), _stream(stream)), "ttt_linear_forward")
     return Z, W_out, c_out
+
+
+def linear_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW_out=None, eta_const=0.0, dQ=None, dK=None,
+                    dV=None, deta=None, dW0=None, stream=None):
+    """Outer-loop gradients of the TTT-Linear prefill (no LN); see
+    ``ttt_linear_backward``.  W_states [B,H,T/b,d,d] comes from
+    ``linear_forward(..., W_states=...)`` on the same inputs.  Returns
+    (dQ, dK, dV, deta, dW0); deta is None when eta is None."""
+    B, H, T, d = Q.shape
+    dev = Q.device
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    if deta is None and eta is not None:
+        deta = torch.empty((B, H, T), device=dev, dtype=torch.float32)
+    dW0 = torch.empty((B, H, d, d), device=dev, dtype=torch.float32) if dW0 is None else dW0
+    a = BackwardArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
+                     _ptr(W_states), _ptr(dZ), _ptr(dW_out), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW0))
+    _check(library().ttt_linear_backward(ctypes.byref(a), _stream(stream)), "ttt_linear_backward")
+    return dQ, dK, dV, deta, dW0
 
 
 def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, *, eta_const=0.0, Z=None, W1_out=None, c1_out=None,

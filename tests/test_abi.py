@@ -18,7 +18,8 @@ def declared_symbols():
 
 def test_header_declares_entry_points():
     syms = declared_symbols()
-    for s in ("ttt_linear_forward", "ttt_mlp_forward", "ttt_linear_decode_step", "ttt_mlp_decode_step"):
+    for s in ("ttt_linear_forward", "ttt_linear_backward", "ttt_mlp_forward", "ttt_linear_decode_step",
+              "ttt_mlp_decode_step"):
         assert s in syms
 
 
@@ -68,6 +69,43 @@ def test_linear_forward_rejects_invalid_arguments(ttt_lib, field, value, code):
     assert ttt_lib.library().ttt_linear_forward(ctypes.byref(a), None) == code
 
 
+def test_linear_forward_w_states_rules(ttt_lib):
+    L = ttt_lib.library()
+    a = _linear_args(ttt_lib, W_states=(1 << 20) + 4)    # misaligned
+    assert L.ttt_linear_forward(ctypes.byref(a), None) == 1
+    a = _linear_args(ttt_lib, W_states=1 << 20, use_ln=1, ln_gamma=1 << 20, ln_beta=1 << 20)
+    assert L.ttt_linear_forward(ctypes.byref(a), None) == 2   # states of the LN variant: not supported
+
+
+def _backward_args(ttt, **kw):
+    a = ttt.BackwardArgs()
+    a.B, a.H, a.T, a.d, a.b, a.io_dtype = 1, 2, 32, 64, 16, ttt.TTT_BF16
+    fake = 1 << 20
+    a.Q = a.K = a.V = a.W_states = a.dQ = a.dK = a.dV = a.dW0 = fake
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=30), 1),
+    (dict(b=0), 1),
+    (dict(d=48), 2),
+    (dict(b=128, T=128), 2),
+    (dict(io_dtype=3), 1),
+    (dict(W_states=None), 1),
+    (dict(dQ=None), 1),
+    (dict(dW0=None), 1),
+    (dict(dZ=(1 << 20) + 2), 1),
+    (dict(dW_out=(1 << 20) + 8), 1),
+    (dict(deta=(1 << 20) + 4), 1),
+    (dict(B=0, Q=None), 0),
+])
+def test_linear_backward_validation(ttt_lib, kw, code):
+    a = _backward_args(ttt_lib, **kw)
+    assert ttt_lib.library().ttt_linear_backward(ctypes.byref(a), None) == code
+
+
 def test_linear_forward_large_b_unsupported(ttt_lib):
     a = _linear_args(ttt_lib, b=128, T=256)
     assert ttt_lib.library().ttt_linear_forward(ctypes.byref(a), None) == 2
@@ -89,6 +127,7 @@ def test_null_args_struct(ttt_lib):
     assert L.ttt_mlp_forward(None, None) == 1
     assert L.ttt_linear_decode_step(None, None) == 1
     assert L.ttt_mlp_decode_step(None, None) == 1
+    assert L.ttt_linear_backward(None, None) == 1
 
 
 def test_mlp_and_decode_validation(ttt_lib):

@@ -1,0 +1,111 @@
+"""Parity of the outer-loop backward of TTT-Linear (through the C ABI) with
+the float64 oracle's reverse-mode differentiation of the primal loop.
+
+The forward writes the state at every mini-batch start (W_states); those are
+checked against the oracle's forward on prefixes, then the backward's five
+gradients against the oracle's.  Tolerances are the forward's: max relative
+error <= 1e-4 for fp32 inputs, normwise <= 2e-2 with bf16 inputs and outputs.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+from test_sequence_layers_head_b200 import workloads as WL
+from tests.gpu_util import assert_close, poison_like, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+def _upstream(inp, seed, with_dz=True, with_dw=True):
+    B, H, T, d = inp.raw["Q"].shape
+    rng = np.random.default_rng(seed)
+    dz = WL.store(rng.standard_normal((B, H, T, d)), inp.w.io_dtype) if with_dz else (None, None)
+    dw = WL.store(rng.standard_normal((B, H, d, d)), WL.F32) if with_dw else (None, None)
+    return dz, dw
+
+
+def _run(ttt, inp, dz, dw, eta_none=False):
+    r, w = inp.raw, inp.w
+    Q, K, V = to_dev(r["Q"]), to_dev(r["K"]), to_dev(r["V"])
+    eta = None if eta_none else to_dev(r["eta"])
+    W0 = to_dev(r["W0"])
+    B, H, T, d = Q.shape
+    states = torch.full((B, H, T // w.b, d, d), float("nan"), device="cuda")
+    ttt.linear_forward(Q, K, V, eta, W0, w.b, eta_const=w.eta_const, W_states=states)
+    dZ = to_dev(dz[0]) if dz[0] is not None else None
+    dW = to_dev(dw[0]) if dw[0] is not None else None
+    deta = None if eta_none else torch.full((B, H, T), float("nan"), device="cuda")
+    out = ttt.linear_backward(Q, K, V, eta, states, w.b, dZ=dZ, dW_out=dW, eta_const=w.eta_const,
+                              dQ=poison_like(Q), dK=poison_like(K), dV=poison_like(V), deta=deta,
+                              dW0=torch.full((B, H, d, d), float("nan"), device="cuda"))
+    torch.cuda.synchronize()
+    assert ttt.last_device_status() == ttt.TTT_OK
+    return to_host(states), [None if g is None else to_host(g) for g in out]
+
+
+def _oracle(inp, dz, dw):
+    e, w = inp.exact, inp.w
+    return O.linear_backward(e["Q"], e["K"], e["V"], e["eta"], e["W0"], w.b, dZ=dz[1], dW_out=dw[1])
+
+
+@pytest.mark.parametrize("d,b,T,io,eta_mode,eta_const", [
+    (16, 16, 64, WL.F32, "sigmoid", 0.0),
+    (32, 8, 48, WL.F32, "const", 0.2),
+    (64, 4, 32, WL.F32, "const", 0.1),
+    (16, 1, 12, WL.F32, "sigmoid", 0.0),
+    (64, 16, 128, WL.BF16, "sigmoid", 0.0),
+    (64, 64, 128, WL.BF16, "const", 0.05),
+])
+def test_backward_matches_oracle(ttt_lib, d, b, T, io, eta_mode, eta_const):
+    inp = WL.random_case("linear", 2, 3, T, d, b, io_dtype=io, eta_mode=eta_mode, eta_const=eta_const,
+                         seed=d + b + T)
+    dz, dw = _upstream(inp, seed=d * b)
+    states, got = _run(ttt_lib, inp, dz, dw)
+    # the forward's batch-start states against the oracle's forward on prefixes
+    e = inp.exact
+    for i in range(0, T // b, max(1, (T // b) // 4)):
+        if i == 0:
+            ref = np.broadcast_to(e["W0"], states[:, :, 0].shape)
+        else:
+            t = i * b
+            ref = O.linear_forward(e["Q"][:, :, :t], e["K"][:, :, :t], e["V"][:, :, :t], e["eta"][:, :, :t],
+                                   e["W0"], b)[1]
+        assert_close(f"W_states[{i}]", states[:, :, i], np.ascontiguousarray(ref), WL.F32)
+    ref = _oracle(inp, dz, dw)
+    for name, g, o in zip(("dQ", "dK", "dV", "deta", "dW0"), got, ref):
+        assert_close(name, g, o, io if name in ("dQ", "dK", "dV") else WL.F32)
+
+
+def test_backward_partial_upstream_and_constant_eta(ttt_lib):
+    """dZ alone, dW_out alone, and eta = None (constant eta, no deta output)."""
+    inp = WL.random_case("linear", 1, 2, 64, 32, 16, io_dtype=WL.F32, eta_mode="const", eta_const=0.15, seed=9)
+    for with_dz, with_dw in ((True, False), (False, True)):
+        dz, dw = _upstream(inp, seed=11, with_dz=with_dz, with_dw=with_dw)
+        _, got = _run(ttt_lib, inp, dz, dw)
+        ref = _oracle(inp, dz, dw)
+        for name, g, o in zip(("dQ", "dK", "dV", "deta", "dW0"), got, ref):
+            if np.max(np.abs(o)) == 0:
+                assert np.all(g == 0), name
+            else:
+                assert_close(name, g, o, WL.F32)
+    dz, dw = _upstream(inp, seed=12)
+    _, got = _run(ttt_lib, inp, dz, dw, eta_none=True)
+    assert got[3] is None
+    ref = _oracle(inp, dz, dw)
+    for name, g, o in zip(("dQ", "dK", "dV", "dW0"), got[:3] + got[4:], ref[:3] + ref[4:]):
+        assert_close(name, g, o, WL.F32)
+
+
+def test_forward_with_states_equals_forward(ttt_lib):
+    """Asking for W_states moves a bf16 d = 64, b = 16 call to the fp32 kernel;
+    its Z and W_out still match the tensor-core kernel's within the bf16 bar."""
+    inp = WL.random_case("linear", 2, 3, 64, 64, 16, seed=21)
+    r = inp.raw
+    Q, K, V, eta, W0 = (to_dev(r[n]) for n in ("Q", "K", "V", "eta", "W0"))
+    Z1, W1, _ = ttt_lib.linear_forward(Q, K, V, eta, W0, 16)
+    states = torch.empty((2, 3, 4, 64, 64), device="cuda")
+    Z2, W2, _ = ttt_lib.linear_forward(Q, K, V, eta, W0, 16, W_states=states)
+    torch.cuda.synchronize()
+    assert_close("Z", to_host(Z2), to_host(Z1), WL.BF16)
+    assert_close("W_out", to_host(W2), to_host(W1), WL.BF16)
