@@ -2,9 +2,10 @@
 
 The backward is reverse-mode differentiation of the primal mini-batch loop
 (paper digest "论文速览 | TTT", section 3.4: the outer loop's gradients pass
-through the inner loop's updates of W; sections 3.5-3.6 define those updates).  It is pinned against central finite differences of the
-forward oracle, which is itself pinned elsewhere, and against the closed
-form at eta = 0, where the layer reduces to Z = Q W0 and W_out = W0.
+through the inner loop's updates of W; sections 3.5-3.6 define those
+updates).  It is pinned against central finite differences of the forward
+oracle, which is itself pinned elsewhere, and against the closed form at
+eta = 0, where the layer reduces to Z = Q W0 and W_out = W0.
 """
 import numpy as np
 import pytest
