@@ -384,7 +384,7 @@ def measure_backward(ttt, torch, threads, name="linear_B8_H12_T2048"):
     return {"workload": name, "forward_with_states_ms": ms_f, "backward_ms": ms_b,
             "tokens_per_s_backward": tokens(w) / (ms_b / 1000.0),
             "backward_bytes": bytes_b, "backward_hbm_frac": bytes_b / (ms_b / 1000.0) / 1e9 / hbm,
-            "kernel": "simt_linear_backward_kernel (fp32 CUDA cores)"}
+            "kernel": "mma_linear_backward_kernel (mma.sync, bf16 operands, fp32 accumulation)"}
 
 
 def measure_e2e_chunked(ttt, w, inp, torch, steps, chunks=8):

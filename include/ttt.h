@@ -147,7 +147,11 @@ ttt_status ttt_linear_forward(const ttt_linear_args* args, cudaStream_t stream);
  *   deta           output [B, H, T] fp32, or NULL when not wanted.
  *   dW0            output [B, H, d, d] fp32, one per sequence (a W0 shared
  *                  over the batch receives the sum over B).
- * Computed on the fp32 CUDA-core kernel, one CTA per (sequence, head) unit.
+ *   flags          0, or TTT_FLAG_FORCE_SIMT.
+ * io_dtype BF16 with d = 64 and b = 16 runs on the tensor cores (mma.sync,
+ * bf16 operands, fp32 accumulation; the state gradient is carried in fp32);
+ * every other case, or TTT_FLAG_FORCE_SIMT, on the fp32 CUDA-core kernel.
+ * One CTA per (sequence, head) unit.
  */
 typedef struct {
     int B, H, T, d, b;
@@ -165,6 +169,7 @@ typedef struct {
     void* dV;
     float* deta;
     float* dW0;
+    unsigned flags;
 } ttt_linear_backward_args;
 
 ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_t stream);

@@ -15,6 +15,7 @@
 #include "mlp_tc.cuh"
 #include "simt.cuh"
 #include "simt_backward.cuh"
+#include "mma_backward.cuh"
 #include "tmap.h"
 
 namespace ttt {
@@ -428,6 +429,13 @@ extern "C" ttt_status ttt_linear_backward(const ttt_linear_backward_args* a, cud
         return TTT_ERR_INVALID_ARG;
     if (!ok_ptr(a->dW0) || !ok_opt(a->eta) || !ok_opt(a->dZ) || !ok_opt(a->dW_out) || !ok_opt(a->deta))
         return TTT_ERR_INVALID_ARG;
+    if (a->flags & ~TTT_FLAG_FORCE_SIMT) return TTT_ERR_INVALID_ARG;
+    if (a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && !(a->flags & TTT_FLAG_FORCE_SIMT)) {
+        SimtBackwardParams p{a->H, a->T, a->b, a->Q, a->K, a->V, a->eta, a->eta_const, a->W_states,
+                             a->dZ, a->dW_out, a->dQ, a->dK, a->dV, a->deta, a->dW0};
+        mbk::mma_linear_backward_kernel<<<(unsigned)units, mbk::kThreads, mbk::kSmemBytes, stream>>>(p);
+        return launch_status();
+    }
     switch (a->d) {
         case 16: return launch_linear_backward<16>(a, stream);
         case 32: return launch_linear_backward<32>(a, stream);

@@ -59,7 +59,7 @@ class DecodeArgs(ctypes.Structure):
 class BackwardArgs(ctypes.Structure):
     _fields_ = [("B", _i), ("H", _i), ("T", _i), ("d", _i), ("b", _i), ("io_dtype", _i), ("Q", _vp), ("K", _vp),
                 ("V", _vp), ("eta", _vp), ("eta_const", _f), ("W_states", _vp), ("dZ", _vp), ("dW_out", _vp),
-                ("dQ", _vp), ("dK", _vp), ("dV", _vp), ("deta", _vp), ("dW0", _vp)]
+                ("dQ", _vp), ("dK", _vp), ("dV", _vp), ("deta", _vp), ("dW0", _vp), ("flags", _u)]
 
 
 class MlpDecodeArgs(ctypes.Structure):
@@ -171,7 +171,7 @@ def linear_forward(Q, K, V, eta, W0, b, *, eta_const=0.0, use_ln=False, c0=None,
 
 
 def linear_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW_out=None, eta_const=0.0, dQ=None, dK=None,
-                    dV=None, deta=None, dW0=None, stream=None):
+                    dV=None, deta=None, dW0=None, flags=0, stream=None):
     """Outer-loop gradients of the TTT-Linear prefill (no LN); see
     ``ttt_linear_backward``.  W_states [B,H,T/b,d,d] comes from
     ``linear_forward(..., W_states=...)`` on the same inputs.  Returns
@@ -185,7 +185,8 @@ def linear_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW_out=None, eta_cons
         deta = torch.empty((B, H, T), device=dev, dtype=torch.float32)
     dW0 = torch.empty((B, H, d, d), device=dev, dtype=torch.float32) if dW0 is None else dW0
     a = BackwardArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
-                     _ptr(W_states), _ptr(dZ), _ptr(dW_out), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW0))
+                     _ptr(W_states), _ptr(dZ), _ptr(dW_out), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW0),
+                     int(flags))
     _check(library().ttt_linear_backward(ctypes.byref(a), _stream(stream)), "ttt_linear_backward")
     return dQ, dK, dV, deta, dW0
 

@@ -100,6 +100,7 @@ def _backward_args(ttt, **kw):
     (dict(dW_out=(1 << 20) + 8), 1),
     (dict(deta=(1 << 20) + 4), 1),
     (dict(B=0, Q=None), 0),
+    (dict(flags=0x2), 1),
 ])
 def test_linear_backward_validation(ttt_lib, kw, code):
     a = _backward_args(ttt_lib, **kw)

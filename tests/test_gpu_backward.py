@@ -73,8 +73,9 @@ def test_backward_matches_oracle(ttt_lib, d, b, T, io, eta_mode, eta_const):
                                    e["W0"], b)[1]
         assert_close(f"W_states[{i}]", states[:, :, i], np.ascontiguousarray(ref), WL.F32)
     ref = _oracle(inp, dz, dw)
+    # bf16 inputs with d = 64, b = 16 run on the tensor cores (bf16 operands): the bf16 bar for all five
     for name, g, o in zip(("dQ", "dK", "dV", "deta", "dW0"), got, ref):
-        assert_close(name, g, o, io if name in ("dQ", "dK", "dV") else WL.F32)
+        assert_close(name, g, o, io)
 
 
 def test_backward_partial_upstream_and_constant_eta(ttt_lib):
@@ -95,6 +96,45 @@ def test_backward_partial_upstream_and_constant_eta(ttt_lib):
     ref = _oracle(inp, dz, dw)
     for name, g, o in zip(("dQ", "dK", "dV", "dW0"), got[:3] + got[4:], ref[:3] + ref[4:]):
         assert_close(name, g, o, WL.F32)
+
+
+@pytest.mark.parametrize("B,H,T,eta_mode,eta_const", [
+    (2, 4, 512, "sigmoid", 0.0),    # 32 mini-batches on the tensor-core kernel
+    (1, 3, 256, "const", 0.1),      # larger steps: the bf16 operands over 16 mini-batches
+    (3, 1, 16, "sigmoid", 0.0),     # one mini-batch
+])
+def test_tensor_core_backward_matches_oracle(ttt_lib, B, H, T, eta_mode, eta_const):
+    """bf16, d = 64, b = 16 runs on mma.sync; checked against the oracle and
+    against the fp32 CUDA-core backward on the same states."""
+    inp = WL.random_case("linear", B, H, T, 64, 16, io_dtype=WL.BF16, eta_mode=eta_mode, eta_const=eta_const,
+                         seed=T + H)
+    dz, dw = _upstream(inp, seed=T)
+    _, got = _run(ttt_lib, inp, dz, dw)
+    ref = _oracle(inp, dz, dw)
+    for name, g, o in zip(("dQ", "dK", "dV", "deta", "dW0"), got, ref):
+        assert_close(name, g, o, WL.BF16)
+    # the same backward on the fp32 kernel
+    r = inp.raw
+    Q, K, V, eta, W0 = (to_dev(r[n]) for n in ("Q", "K", "V", "eta", "W0"))
+    states = torch.empty((B, H, T // 16, 64, 64), device="cuda")
+    ttt_lib.linear_forward(Q, K, V, eta, W0, 16, W_states=states)
+    dZ, dW = to_dev(dz[0]), to_dev(dw[0])
+    tc = ttt_lib.linear_backward(Q, K, V, eta, states, 16, dZ=dZ, dW_out=dW)
+    ft = ttt_lib.linear_backward(Q, K, V, eta, states, 16, dZ=dZ, dW_out=dW, flags=ttt_lib.FLAG_FORCE_SIMT)
+    torch.cuda.synchronize()
+    for name, x, y in zip(("dQ", "dK", "dV", "deta", "dW0"), tc, ft):
+        assert_close(name, to_host(x), to_host(y), WL.BF16)
+
+
+def test_backward_empty_sequence_passes_dw_out_through(ttt_lib):
+    """T = 0: no mini-batch, dW0 = dW_out."""
+    Q = torch.empty((2, 2, 0, 64), device="cuda", dtype=torch.bfloat16)
+    states = torch.empty((2, 2, 0, 64, 64), device="cuda")
+    dW = torch.randn(2, 2, 64, 64, device="cuda")
+    for flags in (0, ttt_lib.FLAG_FORCE_SIMT):
+        out = ttt_lib.linear_backward(Q, Q, Q, None, states, 16, dW_out=dW, eta_const=0.1, flags=flags)
+        torch.cuda.synchronize()
+        assert torch.equal(out[4], dW)
 
 
 def test_forward_with_states_equals_forward(ttt_lib):
