@@ -98,8 +98,10 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
  *   W_states       optional output for the backward (gradient checkpointing
  *                  through time, section 6.12): the state at the start of
  *                  every mini-batch, [B, H, T/b, d, d] fp32, T/b states per
- *                  unit.  NULL: not written.  Non-NULL requires use_ln == 0
- *                  and runs the fp32 CUDA-core kernel.
+ *                  unit.  NULL: not written.  Non-NULL requires use_ln == 0;
+ *                  with io_dtype BF16, d = 64, b = 16 it runs the mma.sync
+ *                  forward (bf16 operands, fp32 state), otherwise the fp32
+ *                  CUDA-core kernel.
  */
 typedef struct {
     int B, H, T, d, b;

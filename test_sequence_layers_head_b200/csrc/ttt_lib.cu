@@ -16,6 +16,7 @@
 #include "simt.cuh"
 #include "simt_backward.cuh"
 #include "mma_backward.cuh"
+#include "mma_forward.cuh"
 #include "tmap.h"
 
 namespace ttt {
@@ -207,7 +208,15 @@ extern "C" ttt_status ttt_linear_forward(const ttt_linear_args* a, cudaStream_t 
         if (a->use_ln) return TTT_ERR_UNSUPPORTED;
     }
     const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
-                    !(a->flags & TTT_FLAG_FORCE_SIMT) && !a->W_states;
+                    !(a->flags & TTT_FLAG_FORCE_SIMT);
+    if (tc && a->W_states) {
+        // training: the mma.sync forward that also writes the batch-start states
+        if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
+        mbk::FwdStatesParams p{a->H, a->T, a->Q, a->K, a->V, a->eta, a->eta_const, a->W0, a->W0_bstride,
+                               a->Z, a->W_out, a->W_states};
+        mbk::mma_linear_forward_states_kernel<<<(unsigned)units, mbk::kThreads, mbk::kFSmemBytes, stream>>>(p);
+        return launch_status();
+    }
     if (tc) return a->use_ln ? tc_linear<true>(a, stream) : tc_linear<false>(a, stream);
     if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
     return a->use_ln ? simt_linear<true>(a, stream) : simt_linear<false>(a, stream);

@@ -71,7 +71,7 @@ def test_backward_matches_oracle(ttt_lib, d, b, T, io, eta_mode, eta_const):
             t = i * b
             ref = O.linear_forward(e["Q"][:, :, :t], e["K"][:, :, :t], e["V"][:, :, :t], e["eta"][:, :, :t],
                                    e["W0"], b)[1]
-        assert_close(f"W_states[{i}]", states[:, :, i], np.ascontiguousarray(ref), WL.F32)
+        assert_close(f"W_states[{i}]", states[:, :, i], np.ascontiguousarray(ref), io)
     ref = _oracle(inp, dz, dw)
     # bf16 inputs with d = 64, b = 16 run on the tensor cores (bf16 operands): the bf16 bar for all five
     for name, g, o in zip(("dQ", "dK", "dV", "deta", "dW0"), got, ref):
@@ -96,6 +96,28 @@ def test_backward_partial_upstream_and_constant_eta(ttt_lib):
     ref = _oracle(inp, dz, dw)
     for name, g, o in zip(("dQ", "dK", "dV", "dW0"), got[:3] + got[4:], ref[:3] + ref[4:]):
         assert_close(name, g, o, WL.F32)
+
+
+@pytest.mark.parametrize("B,H,T,eta_mode,eta_const", [(2, 4, 512, "sigmoid", 0.0), (1, 2, 256, "const", 0.1)])
+def test_forward_with_states_matches_oracle(ttt_lib, B, H, T, eta_mode, eta_const):
+    """The mma.sync forward (bf16, d = 64, b = 16, with W_states): Z, W_out and
+    sampled batch-start states against the oracle."""
+    inp = WL.random_case("linear", B, H, T, 64, 16, io_dtype=WL.BF16, eta_mode=eta_mode, eta_const=eta_const,
+                         seed=7 * T + H)
+    r, e = inp.raw, inp.exact
+    Q, K, V, eta, W0 = (to_dev(r[n]) for n in ("Q", "K", "V", "eta", "W0"))
+    states = torch.full((B, H, T // 16, 64, 64), float("nan"), device="cuda")
+    Z, Wout, _ = ttt_lib.linear_forward(Q, K, V, eta, W0, 16, Z=poison_like(Q), W_states=states)
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    Zo, Wo, _ = O.linear_forward(e["Q"], e["K"], e["V"], e["eta"], e["W0"], 16)
+    assert_close("Z", to_host(Z), Zo, WL.BF16)
+    assert_close("W_out", to_host(Wout), Wo, WL.BF16)
+    for i in (1, T // 32, T // 16 - 1):
+        t = 16 * i
+        ref = O.linear_forward(e["Q"][:, :, :t], e["K"][:, :, :t], e["V"][:, :, :t], e["eta"][:, :, :t], e["W0"],
+                               16)[1]
+        assert_close(f"W_states[{i}]", to_host(states[:, :, i]), ref, WL.BF16)
 
 
 @pytest.mark.parametrize("B,H,T,eta_mode,eta_const", [
@@ -138,8 +160,8 @@ def test_backward_empty_sequence_passes_dw_out_through(ttt_lib):
 
 
 def test_forward_with_states_equals_forward(ttt_lib):
-    """Asking for W_states moves a bf16 d = 64, b = 16 call to the fp32 kernel;
-    its Z and W_out still match the tensor-core kernel's within the bf16 bar."""
+    """Asking for W_states moves a bf16 d = 64, b = 16 call to the mma.sync
+    forward; its Z and W_out match the tcgen05 kernel's within the bf16 bar."""
     inp = WL.random_case("linear", 2, 3, 64, 64, 16, seed=21)
     r = inp.raw
     Q, K, V, eta, W0 = (to_dev(r[n]) for n in ("Q", "K", "V", "eta", "W0"))
