@@ -109,15 +109,37 @@ __global__ void __launch_bounds__(kThreads) mma_linear_backward_kernel(SimtBackw
             g[nt][e] = p.dW_out ? p.dW_out[(size_t)unit * kD * kD + (size_t)(f0 + r + 8 * (e >> 1)) * kD +
                                            8 * nt + 2 * c + (e & 1)]
                                 : 0.f;
+    // the next mini-batch's operands are loaded into registers while the current one computes
+    float4 pw[8];
+    uint4 pkq[3];
+    uint32_t pv[2][2];
+    float pe = 0.f;
+    auto prefetch = [&](int i) {
+        const float4* Ws = reinterpret_cast<const float4*>(p.W_states + ((size_t)unit * nb + i) * kD * kD);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) pw[q] = Ws[tid + kThreads * q];
+        const int t0 = i * kB, row = tid >> 3, ch = tid & 7;
+        const size_t gi = (size_t)(t0 + row) * kD + 8 * ch;
+        pkq[0] = *reinterpret_cast<const uint4*>(K + gi);
+        pkq[1] = *reinterpret_cast<const uint4*>(Q + gi);
+        pkq[2] = dZ ? *reinterpret_cast<const uint4*>(dZ + gi) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                pv[nt][h] = *reinterpret_cast<const uint32_t*>(V + (size_t)(t0 + r + 8 * h) * kD + f0 + 8 * nt + 2 * c);
+        if (tid < kB) pe = p.eta ? p.eta[(size_t)unit * p.T + t0 + tid] : p.eta_const;
+    };
+    if (nb > 0) prefetch(nb - 1);
     for (int i = nb - 1; i >= 0; --i) {
         const int t0 = i * kB;
-        // ---- loads: batch-start state (bf16), G (bf16), K, Q, dZ tiles, eta
+        // ---- this mini-batch's operands to shared memory: batch-start state (bf16), G (bf16), K, Q, dZ, eta
+        uint32_t vcur[2][2];
         {
-            const float4* Ws = reinterpret_cast<const float4*>(p.W_states + ((size_t)unit * nb + i) * kD * kD);
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
                 const int idx = tid + kThreads * q;   // float4 index: row idx / 16, columns 4 (idx % 16) ..
-                const float4 v = Ws[idx];
+                const float4 v = pw[q];
                 const int row = idx >> 4, c4 = idx & 15;
                 *reinterpret_cast<uint2*>(smem + kOffW + toff(row, c4 >> 1) + 8 * (c4 & 1)) =
                     make_uint2(pk(v.x, v.y), pk(v.z, v.w));
@@ -129,13 +151,16 @@ __global__ void __launch_bounds__(kThreads) mma_linear_backward_kernel(SimtBackw
                     *reinterpret_cast<uint32_t*>(smem + kOffG + toff(f0 + r + 8 * h, nt) + 4 * c) =
                         pk(g[nt][2 * h], g[nt][2 * h + 1]);
             const int row = tid >> 3, ch = tid & 7;
-            const size_t gi = (size_t)(t0 + row) * kD + 8 * ch;
-            *reinterpret_cast<uint4*>(smem + kOffK + toff(row, ch)) = *reinterpret_cast<const uint4*>(K + gi);
-            *reinterpret_cast<uint4*>(smem + kOffQ + toff(row, ch)) = *reinterpret_cast<const uint4*>(Q + gi);
-            *reinterpret_cast<uint4*>(smem + kOffDZ + toff(row, ch)) =
-                dZ ? *reinterpret_cast<const uint4*>(dZ + gi) : make_uint4(0u, 0u, 0u, 0u);
-            if (tid < kB) s_eta[tid] = p.eta ? p.eta[(size_t)unit * p.T + t0 + tid] : p.eta_const;
+            *reinterpret_cast<uint4*>(smem + kOffK + toff(row, ch)) = pkq[0];
+            *reinterpret_cast<uint4*>(smem + kOffQ + toff(row, ch)) = pkq[1];
+            *reinterpret_cast<uint4*>(smem + kOffDZ + toff(row, ch)) = pkq[2];
+            if (tid < kB) s_eta[tid] = pe;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) vcur[nt][h] = pv[nt][h];
         }
+        if (i > 0) prefetch(i - 1);
         __syncthreads();
         const float eta_r[2] = {s_eta[r], s_eta[r + 8]};
         // ---- E = K W - V on features f0..f0+15 (rows t = r, r + 8)
@@ -144,8 +169,7 @@ __global__ void __launch_bounds__(kThreads) mma_linear_backward_kernel(SimtBackw
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const __nv_bfloat162 v2 =
-                    *reinterpret_cast<const __nv_bfloat162*>(V + (size_t)(t0 + r + 8 * h) * kD + f0 + 8 * nt + 2 * c);
+                const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&vcur[nt][h]);
                 e[nt][2 * h] = -__bfloat162float(v2.x);
                 e[nt][2 * h + 1] = -__bfloat162float(v2.y);
             }

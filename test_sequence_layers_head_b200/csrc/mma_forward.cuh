@@ -65,6 +65,23 @@ __global__ void __launch_bounds__(kThreads) mma_linear_forward_states_kernel(Fwd
                 wr[nt][2 * h + 1] = v.y;
             }
     }
+    // the next mini-batch's tiles are loaded into registers while the current one computes
+    uint4 pkq[2];
+    uint32_t pv[2][2];
+    float pe = 0.f;
+    auto prefetch = [&](int i) {
+        const int t0 = i * kB, row = tid >> 3, ch = tid & 7;
+        const size_t gi = (size_t)(t0 + row) * kD + 8 * ch;
+        pkq[0] = *reinterpret_cast<const uint4*>(K + gi);
+        pkq[1] = *reinterpret_cast<const uint4*>(Q + gi);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                pv[nt][h] = *reinterpret_cast<const uint32_t*>(V + (size_t)(t0 + r + 8 * h) * kD + f0 + 8 * nt + 2 * c);
+        if (tid < kB) pe = p.eta ? p.eta[(size_t)unit * p.T + t0 + tid] : p.eta_const;
+    };
+    if (nb > 0) prefetch(0);
     for (int i = 0; i < nb; ++i) {
         const int t0 = i * kB;
         // ---- batch-start state: fp32 to the checkpoints, bf16 to shared memory; the tiles
@@ -79,13 +96,18 @@ __global__ void __launch_bounds__(kThreads) mma_linear_forward_states_kernel(Fwd
                 *reinterpret_cast<uint32_t*>(smem + kFOffW + toff(row, nt) + 4 * c) =
                     pk(wr[nt][2 * h], wr[nt][2 * h + 1]);
             }
+        uint32_t vcur[2][2];
         {
             const int row = tid >> 3, ch = tid & 7;
-            const size_t gi = (size_t)(t0 + row) * kD + 8 * ch;
-            *reinterpret_cast<uint4*>(smem + kFOffK + toff(row, ch)) = *reinterpret_cast<const uint4*>(K + gi);
-            *reinterpret_cast<uint4*>(smem + kFOffQ + toff(row, ch)) = *reinterpret_cast<const uint4*>(Q + gi);
-            if (tid < kB) s_eta[tid] = p.eta ? p.eta[(size_t)unit * p.T + t0 + tid] : p.eta_const;
+            *reinterpret_cast<uint4*>(smem + kFOffK + toff(row, ch)) = pkq[0];
+            *reinterpret_cast<uint4*>(smem + kFOffQ + toff(row, ch)) = pkq[1];
+            if (tid < kB) s_eta[tid] = pe;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) vcur[nt][h] = pv[nt][h];
         }
+        if (i + 1 < nb) prefetch(i + 1);
         __syncthreads();
         const float eta_r[2] = {s_eta[r], s_eta[r + 8]};
         // ---- E = K W - V on this warp's features; A = diag(eta) E -> shared
@@ -94,8 +116,7 @@ __global__ void __launch_bounds__(kThreads) mma_linear_forward_states_kernel(Fwd
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const __nv_bfloat162 v2 =
-                    *reinterpret_cast<const __nv_bfloat162*>(V + (size_t)(t0 + r + 8 * h) * kD + f0 + 8 * nt + 2 * c);
+                const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162*>(&vcur[nt][h]);
                 e[nt][2 * h] = -__bfloat162float(v2.x);
                 e[nt][2 * h + 1] = -__bfloat162float(v2.y);
             }
