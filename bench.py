@@ -668,6 +668,45 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_b_sweep(args):
+    """Mini-batch size study (paper digest "论文速览 | TTT", section 5.3): forward
+    time split into computing the state and computing the outputs, per b, on
+    the fp32 CUDA-core kernel (every b <= 64; the state-only call passes
+    Z = NULL), plus the tensor-core kernel at b = 16.  Prints one JSON line."""
+    import torch
+    from test_sequence_layers_head_b200 import ttt
+    w = WL.WORKLOADS[args.workload if args.workload != DEFAULT_WORKLOAD else "linear_B8_H12_T2048"]
+    if args.T:
+        w = WL.scaled(w, T=args.T)
+    threads = len(os.sched_getaffinity(0))
+    _, dev = device_inputs(w, torch, threads)
+    B, H, T, d = w.B, w.H, w.T, w.d
+    Z = torch.empty_like(dev["Q"])
+    W_out = torch.empty((B, H, d, d), device="cuda")
+    flush_buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")
+    eta = dev.get("eta")
+
+    def fwd(b, outputs, flags):
+        ttt.linear_forward(dev["Q"], dev["K"], dev["V"], eta, dev["W0"], b, eta_const=w.eta_const, Z=Z, W_out=W_out,
+                           outputs=outputs, flags=flags)
+    rows = []
+    for b in (1, 2, 4, 8, 16, 32, 64):
+        if T % b:
+            continue
+        full = statistics.median(time_launches(torch, lambda: fwd(b, True, ttt.FLAG_FORCE_SIMT), 3, 1,
+                                               flush=lambda: flush_buf.zero_()))
+        state = statistics.median(time_launches(torch, lambda: fwd(b, False, ttt.FLAG_FORCE_SIMT), 3, 1,
+                                                flush=lambda: flush_buf.zero_()))
+        rows.append({"b": b, "forward_ms": full, "state_only_ms": state, "outputs_ms": full - state,
+                     "tokens_per_s": tokens(w) / (full / 1000.0)})
+    tc = statistics.median(time_launches(torch, lambda: fwd(16, True, 0), 5, 2, flush=lambda: flush_buf.zero_()))
+    assert ttt.last_device_status() == ttt.TTT_OK
+    print(json.dumps({"b_sweep": rows, "workload": w.name, "dtype": "bf16" if w.io_dtype == WL.BF16 else "f32",
+                      "kernel": "fp32 CUDA-core forward (state only: Z = NULL)",
+                      "tensor_core_b16_ms": tc, "tensor_core_b16_tokens_per_s": tokens(w) / (tc / 1000.0)}),
+          flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -681,8 +720,12 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch from an ncu capture of the current kernel build")
+    ap.add_argument("--b-sweep", action="store_true",
+                    help="mini-batch size study (state vs outputs time per b) instead of the benchmark line")
     args = ap.parse_args()
-    if args.impl == "reference":
+    if args.b_sweep:
+        run_b_sweep(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

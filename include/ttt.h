@@ -90,7 +90,10 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
  *   c0             LN only: initial bias [H, d] with the same batch-stride
  *                  rule (c0_bstride), or NULL for zeros.
  *   ln_gamma, ln_beta  LN only: [H, d] fp32.
- *   Z              output [B, H, T, d] in io_dtype.
+ *   Z              output [B, H, T, d] in io_dtype, or NULL: only the final
+ *                  state is computed, on the fp32 CUDA-core kernel (the
+ *                  "computing W" part of the mini-batch size study, section
+ *                  5.3).
  *   W_out          output final state [B, H, d, d] fp32.
  *   c_out          LN only: final bias [B, H, d] fp32, or NULL.
  *   flags          TTT_FLAG_* bits; 0 for normal use.

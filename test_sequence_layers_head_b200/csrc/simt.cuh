@@ -36,7 +36,7 @@ struct SimtLinearParams {
     const float* gamma;
     const float* beta;
     float eps;
-    void* Z;
+    void* Z;           // null: only the state is computed (no outputs)
     float* W_out;
     float* c_out;
     float* W_states;   // optional [units, T/b, D, D]: the state at the start of every mini-batch
@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_linear_kernel(SimtLinearPar
             Yt[e] = LN ? acc + c[j] : acc;
         }
         // S = tril(Q K^T (+1)) * eta_s
-        for (int e = tid; e < b * b; e += kSimtThreads) {
+        for (int e = tid; p.Z && e < b * b; e += kSimtThreads) {
             const int t = e / b, s = e % b;
             float acc = 0.f;
             if (s <= t) {
@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_linear_kernel(SimtLinearPar
         }
         __syncthreads();
         // Zpre = Q W0 (+ c) - S Delta
-        for (int e = tid; e < b * D; e += kSimtThreads) {
+        for (int e = tid; p.Z && e < b * D; e += kSimtThreads) {
             const int t = e / D, j = e % D;
             float acc = 0.f;
 #pragma unroll 8
@@ -165,7 +165,8 @@ __global__ void __launch_bounds__(kSimtThreads) simt_linear_kernel(SimtLinearPar
             Yt[e] = (LN ? acc + c[j] : acc) - corr;
         }
         __syncthreads();
-        if (!LN) {
+        if (!p.Z) {
+        } else if (!LN) {
             for (int e = tid; e < b * D; e += kSimtThreads) IoTraits<IO>::store(Z, (size_t)t0 * D + e, Yt[e]);
         } else {
             for (int t = warp; t < b; t += nwarps) {

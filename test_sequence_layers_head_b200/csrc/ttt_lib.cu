@@ -188,7 +188,7 @@ extern "C" ttt_status ttt_linear_forward(const ttt_linear_args* a, cudaStream_t 
     if (v != TTT_OK) return v;
     const long long units = (long long)a->B * a->H;
     if (units == 0) return TTT_OK;
-    if (a->T > 0 && (!ok_ptr(a->Q) || !ok_ptr(a->K) || !ok_ptr(a->V) || !ok_ptr(a->Z)))
+    if (a->T > 0 && (!ok_ptr(a->Q) || !ok_ptr(a->K) || !ok_ptr(a->V) || !ok_opt(a->Z)))
         return TTT_ERR_INVALID_ARG;
     if (!ok_ptr(a->W0) || !ok_ptr(a->W_out) || !ok_opt(a->eta)) return TTT_ERR_INVALID_ARG;
     if (a->W0_bstride < 0 || a->c0_bstride < 0) return TTT_ERR_INVALID_ARG;
@@ -207,7 +207,7 @@ extern "C" ttt_status ttt_linear_forward(const ttt_linear_args* a, cudaStream_t 
         if (!aligned16(a->W_states)) return TTT_ERR_INVALID_ARG;
         if (a->use_ln) return TTT_ERR_UNSUPPORTED;
     }
-    const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
+    const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 && a->Z &&
                     !(a->flags & TTT_FLAG_FORCE_SIMT);
     if (tc && a->W_states) {
         // training: the mma.sync forward that also writes the batch-start states

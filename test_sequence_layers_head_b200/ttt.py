@@ -146,15 +146,20 @@ def _check(code: int, what: str):
 
 def linear_forward(Q, K, V, eta, W0, b, *, eta_const=0.0, use_ln=False, c0=None, gamma=None, beta=None,
                    eps=1e-6, Z=None, W_out=None, c_out=None, flags=0, wait_timeout_ms=0, W_states=None,
-                   stream=None):
+                   outputs=True, stream=None):
     """TTT-Linear (optionally LN+residual) prefill; see ``ttt_linear_forward``.
 
     Q, K, V: [B,H,T,d] bf16 or fp32; eta: [B,H,T] fp32 or None (eta_const);
     W0: [H,d,d] (shared) or [B,H,d,d] fp32.  Returns (Z, W_out, c_out).
+    W_states: optional [B,H,T/b,d,d] fp32 output, the state at every mini-batch
+    start (for ``linear_backward``).  outputs=False: Z is not computed (None is
+    returned), only the state.
     """
     B, H, T, d = Q.shape
     dev = Q.device
-    if Z is None:
+    if not outputs:
+        Z = None   # state only: the library skips the outputs
+    elif Z is None:
         Z = torch.empty_like(Q)
     if W_out is None:
         W_out = torch.empty((B, H, d, d), device=dev, dtype=torch.float32)

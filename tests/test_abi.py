@@ -56,6 +56,7 @@ def _linear_args(ttt, **kw):
     ("b", 128, 1),         # T = 32 is not a multiple of 128
     ("io_dtype", 7, 1),
     ("Q", None, 1),        # null pointer
+    ("Z", (1 << 20) + 4, 1),  # misaligned (NULL is allowed: state only)
     ("K", (1 << 20) + 4, 1),  # misaligned
     ("W_out", None, 1),
     ("eta", (1 << 20) + 8, 1),

@@ -148,6 +148,32 @@ def test_tensor_core_backward_matches_oracle(ttt_lib, B, H, T, eta_mode, eta_con
         assert_close(name, to_host(x), to_host(y), WL.BF16)
 
 
+def test_training_kernels_per_sequence_state_and_constant_eta(ttt_lib):
+    """The mma.sync forward with states and backward with a per-sequence W0
+    [B,H,d,d] and eta = None (eta_const)."""
+    B, H, T = 2, 2, 64
+    inp = WL.random_case("linear", B, H, T, 64, 16, io_dtype=WL.BF16, eta_mode="const", eta_const=0.08, seed=77)
+    rng = np.random.default_rng(78)
+    W0r, W0e = WL.store(rng.standard_normal((B, H, 64, 64)) / 8, WL.F32)
+    r, e = inp.raw, inp.exact
+    Q, K, V = (to_dev(r[n]) for n in ("Q", "K", "V"))
+    W0 = to_dev(W0r)
+    states = torch.full((B, H, T // 16, 64, 64), float("nan"), device="cuda")
+    Z, Wout, _ = ttt_lib.linear_forward(Q, K, V, None, W0, 16, eta_const=0.08, W_states=states)
+    dz, dw = _upstream(inp, seed=79)
+    out = ttt_lib.linear_backward(Q, K, V, None, states, 16, eta_const=0.08, dZ=to_dev(dz[0]), dW_out=to_dev(dw[0]))
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    eta = np.full((B, H, T), 0.08)
+    Zo, Wo, _ = O.linear_forward(e["Q"], e["K"], e["V"], eta, W0e, 16)
+    assert_close("Z", to_host(Z), Zo, WL.BF16)
+    assert_close("W_out", to_host(Wout), Wo, WL.BF16)
+    ref = O.linear_backward(e["Q"], e["K"], e["V"], eta, W0e, 16, dZ=dz[1], dW_out=dw[1])
+    assert out[3] is None
+    for name, g, o in zip(("dQ", "dK", "dV", "dW0"), out[:3] + out[4:], ref[:3] + ref[4:]):
+        assert_close(name, to_host(g), o, WL.BF16)
+
+
 def test_backward_empty_sequence_passes_dw_out_through(ttt_lib):
     """T = 0: no mini-batch, dW0 = dW_out."""
     Q = torch.empty((2, 2, 0, 64), device="cuda", dtype=torch.bfloat16)

@@ -160,6 +160,27 @@ def test_linear_tc_chunked_calls(ttt_lib, use_ln):
 # TTT-Linear, fp32 CUDA-core kernel
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("d,b,io,use_ln", [(64, 16, WL.BF16, False), (32, 4, WL.F32, False),
+                                         (16, 1, WL.F32, False), (64, 8, WL.BF16, True)])
+def test_state_only_forward(ttt_lib, d, b, io, use_ln):
+    """Z = NULL (the state-only half of the mini-batch size study): W_out (and
+    c_out) equal those of the same fp32 kernel with outputs, bit for bit, and
+    the oracle's within the tolerance."""
+    inp = WL.random_case("ln" if use_ln else "linear", 2, 3, 64, d, b, io_dtype=io, seed=d + b)
+    r, w = inp.raw, inp.w
+    Q, K, V, eta, W0 = (to_dev(r[n]) for n in ("Q", "K", "V", "eta", "W0"))
+    kw = dict(c0=to_dev(r["c0"]), gamma=to_dev(r["gamma"]), beta=to_dev(r["beta"]), eps=w.ln_eps) if use_ln else {}
+    _, Wa, ca = ttt_lib.linear_forward(Q, K, V, eta, W0, b, use_ln=use_ln, flags=ttt_lib.FLAG_FORCE_SIMT, **kw)
+    Zb, Wb, cb = ttt_lib.linear_forward(Q, K, V, eta, W0, b, use_ln=use_ln, outputs=False, **kw)
+    torch.cuda.synchronize()
+    assert Zb is None
+    assert torch.equal(Wa, Wb)
+    if use_ln:
+        assert torch.equal(ca, cb)
+    _, Wo, co = oracle_linear(inp, use_ln)
+    assert_close("W_out", to_host(Wb), Wo, io)
+
+
 def test_linear_d16_f32_workload(ttt_lib):
     """The fp32 workload (d = 16, T = 256, eta = 0.1): max relative error <= 1e-4."""
     w = WL.WORKLOADS["linear_d16_T256_f32"]
