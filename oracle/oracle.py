@@ -31,6 +31,9 @@ def lib():
         L.ttt_oracle_linear_forward.restype = i
         L.ttt_oracle_mlp_forward.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, ll, P, P, P, P, P, i]
         L.ttt_oracle_mlp_forward.restype = i
+        L.ttt_oracle_mlp_ln_forward.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, ll, i, P, P, dbl,
+                                                P, P, P, P, P, i]
+        L.ttt_oracle_mlp_ln_forward.restype = i
         L.ttt_oracle_linear_decode_step.argtypes = [i, i, i, P, P, P, P, P, P]
         L.ttt_oracle_linear_decode_step.restype = i
         L.ttt_oracle_linear_backward.argtypes = [i, i, i, i, i, P, P, P, P, P, ll, P, P, P, P, P, P, P, i]
@@ -82,22 +85,24 @@ def linear_forward(Q, K, V, eta, W0, b, c0=None, gamma=None, beta=None, use_ln=F
     return Z, W_out, c_out
 
 
-def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, threads=None):
-    """Primal mini-batch TTT-MLP forward, f(x) = GELU(x W1 + c1) W2 + c2.
+def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, threads=None, use_ln=False, gamma=None, beta=None, eps=1e-6):
+    """Primal mini-batch TTT-MLP forward, f(x) = GELU(x W1 + c1) W2 + c2, or
+    with use_ln f(x) = x + gamma LN(GELU(x W1 + c1) W2 + c2) + beta.
 
-    Parameters are [H,...] (shared over the batch) or [B,H,...].
+    Parameters are [H,...] (shared over the batch) or [B,H,...]; gamma, beta [H,d].
     Returns (Z, W1_out [B,H,d,m], c1_out [B,H,m], W2_out [B,H,m,d], c2_out [B,H,d]).
     """
     Q, K, V, eta, W1, c1, W2, c2 = map(_f64, (Q, K, V, eta, W1, c1, W2, c2))
+    gamma, beta = map(_f64, (gamma, beta))
     B, H, T, d = Q.shape
     m = W1.shape[-1]
     per_seq = 1 if W1.ndim == 4 else 0
     Z = np.empty((B, H, T, d))
     W1o, c1o = np.empty((B, H, d, m)), np.empty((B, H, m))
     W2o, c2o = np.empty((B, H, m, d)), np.empty((B, H, d))
-    rc = lib().ttt_oracle_mlp_forward(B, H, T, d, m, b, _p(Q), _p(K), _p(V), _p(eta), _p(W1), _p(c1),
-                                      _p(W2), _p(c2), per_seq, _p(Z), _p(W1o), _p(c1o), _p(W2o), _p(c2o),
-                                      threads or default_threads())
+    rc = lib().ttt_oracle_mlp_ln_forward(B, H, T, d, m, b, _p(Q), _p(K), _p(V), _p(eta), _p(W1), _p(c1),
+                                         _p(W2), _p(c2), per_seq, int(bool(use_ln)), _p(gamma), _p(beta), eps,
+                                         _p(Z), _p(W1o), _p(c1o), _p(W2o), _p(c2o), threads or default_threads())
     if rc != 0:
         raise ValueError("oracle: invalid arguments")
     return Z, W1o, c1o, W2o, c2o

@@ -25,7 +25,8 @@
  *     GPU's route, not the oracle's.
  *   - Inner models (section 4.4): linear f(x) = x W; LN+residual
  *     f(x) = x + LN(x W + c); two-layer MLP f(x) = GELU(x W1 + c1) W2 + c2
- *     with hidden size 4d.
+ *     with hidden size 4d, optionally with LN+residual on its output layer,
+ *     f(x) = x + LN(GELU(x W1 + c1) W2 + c2).
  *   - Learnable per-token learning rate (section 4.6): eta_t is an input, one
  *     value per token, scaling that token's own gradient.
  *   - Decode / generate uses the primal form one token at a time (section
@@ -112,6 +113,28 @@ static void linear_model_forward(int d, const double *x, const double *W, const 
 }
 
 /*
+ * LN+residual output f = x + gamma * LN(y) + beta over d features: the
+ * gradient of 1/2 || f - v ||^2 with respect to y (x is the model's input).
+ */
+static void ln_residual_delta(int d, const double *x, const double *v, const double *y, const double *gamma,
+                              const double *beta, double eps, double *delta, double *xh) {
+    const double r = layer_norm(d, y, eps, xh);
+    /* e = f(k) - v ; g = dL/dxhat = gamma * e */
+    double mean_g = 0.0, mean_gx = 0.0;
+    for (int j = 0; j < d; ++j) {
+        const double e = x[j] + gamma[j] * xh[j] + beta[j] - v[j];
+        const double g = gamma[j] * e;
+        delta[j] = g; /* keep g for now */
+        mean_g += g;
+        mean_gx += g * xh[j];
+    }
+    mean_g /= d;
+    mean_gx /= d;
+    /* backward through xhat = (y - mu) r */
+    for (int j = 0; j < d; ++j) delta[j] = r * (delta[j] - mean_g - xh[j] * mean_gx);
+}
+
+/*
  * Gradient of 1/2 || f(k; W, c) - v ||^2 with respect to the pre-activation
  * y = k W (+ c).  grad_W = k^T delta, grad_c = delta.
  */
@@ -124,20 +147,7 @@ static void linear_model_delta(int d, const double *k, const double *v, const do
         return;
     }
     for (int j = 0; j < d; ++j) y[j] += c[j];
-    const double r = layer_norm(d, y, eps, xh);
-    /* e = f(k) - v ; g = dL/dxhat = gamma * e */
-    double mean_g = 0.0, mean_gx = 0.0;
-    for (int j = 0; j < d; ++j) {
-        const double e = k[j] + gamma[j] * xh[j] + beta[j] - v[j];
-        const double g = gamma[j] * e;
-        delta[j] = g; /* keep g for now */
-        mean_g += g;
-        mean_gx += g * xh[j];
-    }
-    mean_g /= d;
-    mean_gx /= d;
-    /* backward through xhat = (y - mu) r */
-    for (int j = 0; j < d; ++j) delta[j] = r * (delta[j] - mean_g - xh[j] * mean_gx);
+    ln_residual_delta(d, k, v, y, gamma, beta, eps, delta, xh);
 }
 
 static void linear_unit(int T, int d, int b, const double *Q, const double *K, const double *V,
@@ -211,8 +221,8 @@ int ttt_oracle_linear_forward(int B, int H, int T, int d, int b, const double *Q
  * ------------------------------------------------------------------------- */
 static void mlp_unit(int T, int d, int m, int b, const double *Q, const double *K, const double *V,
                      const double *eta, const double *W1_0, const double *c1_0, const double *W2_0,
-                     const double *c2_0, double *Z, double *W1_out, double *c1_out, double *W2_out,
-                     double *c2_out) {
+                     const double *c2_0, int use_ln, const double *gamma, const double *beta, double eps,
+                     double *Z, double *W1_out, double *c1_out, double *W2_out, double *c2_out) {
     const size_t n1 = (size_t)d * m, n2 = (size_t)m * d;
     double *W1s = malloc(n1 * sizeof(double)), *W1c = malloc(n1 * sizeof(double));
     double *W2s = malloc(n2 * sizeof(double)), *W2c = malloc(n2 * sizeof(double));
@@ -220,6 +230,7 @@ static void mlp_unit(int T, int d, int m, int b, const double *Q, const double *
     double *c2s = malloc(d * sizeof(double)), *c2c = malloc(d * sizeof(double));
     double *a = malloc(m * sizeof(double)), *hh = malloc(m * sizeof(double));
     double *d1 = malloc(m * sizeof(double)), *e = malloc(d * sizeof(double));
+    double *y = malloc(d * sizeof(double)), *xh = malloc(d * sizeof(double));
     memcpy(W1c, W1_0, n1 * sizeof(double));
     memcpy(W2c, W2_0, n2 * sizeof(double));
     if (c1_0) memcpy(c1c, c1_0, m * sizeof(double)); else memset(c1c, 0, m * sizeof(double));
@@ -236,8 +247,15 @@ static void mlp_unit(int T, int d, int m, int b, const double *Q, const double *
             /* forward at the batch-start parameters */
             vec_mat(d, m, k, W1s, a);
             for (int p = 0; p < m; ++p) { a[p] += c1s[p]; hh[p] = gelu(a[p]); }
-            vec_mat(m, d, hh, W2s, e);
-            for (int j = 0; j < d; ++j) e[j] += c2s[j] - v[j];
+            if (!use_ln) {
+                vec_mat(m, d, hh, W2s, e);
+                for (int j = 0; j < d; ++j) e[j] += c2s[j] - v[j];
+            } else {
+                /* f = k + LN(h W2 + c2): e becomes the gradient with respect to y = h W2 + c2 */
+                vec_mat(m, d, hh, W2s, y);
+                for (int j = 0; j < d; ++j) y[j] += c2s[j];
+                ln_residual_delta(d, k, v, y, gamma, beta, eps, e, xh);
+            }
             /* backward: d1 = (e W2^T) * GELU'(a) */
             for (int p = 0; p < m; ++p) {
                 double s = 0.0;
@@ -265,6 +283,10 @@ static void mlp_unit(int T, int d, int m, int b, const double *Q, const double *
             double *z = Z + (size_t)t * d;
             vec_mat(m, d, hh, W2c, z);
             for (int j = 0; j < d; ++j) z[j] += c2c[j];
+            if (use_ln) {
+                layer_norm(d, z, eps, xh);
+                for (int j = 0; j < d; ++j) z[j] = q[j] + gamma[j] * xh[j] + beta[j];
+            }
         }
     }
     memcpy(W1_out, W1c, n1 * sizeof(double));
@@ -272,16 +294,21 @@ static void mlp_unit(int T, int d, int m, int b, const double *Q, const double *
     if (c1_out) memcpy(c1_out, c1c, m * sizeof(double));
     if (c2_out) memcpy(c2_out, c2c, d * sizeof(double));
     free(W1s); free(W1c); free(W2s); free(W2c); free(c1s); free(c1c); free(c2s); free(c2c);
-    free(a); free(hh); free(d1); free(e);
+    free(a); free(hh); free(d1); free(e); free(y); free(xh);
 }
 
-int ttt_oracle_mlp_forward(int B, int H, int T, int d, int m, int b, const double *Q, const double *K,
-                           const double *V, const double *eta, const double *W1, const double *c1,
-                           const double *W2, const double *c2, long long p_bstride_scale, double *Z,
-                           double *W1_out, double *c1_out, double *W2_out, double *c2_out, int nthreads) {
+/* TTT-MLP, optionally with LN+residual on the output layer,
+ *     f(x) = x + gamma LN(GELU(x W1 + c1) W2 + c2) + beta   (use_ln = 1),
+ * the form the pages give for TTT-MLP in practice (section 4.4). */
+int ttt_oracle_mlp_ln_forward(int B, int H, int T, int d, int m, int b, const double *Q, const double *K,
+                              const double *V, const double *eta, const double *W1, const double *c1,
+                              const double *W2, const double *c2, long long p_bstride_scale, int use_ln,
+                              const double *gamma, const double *beta, double eps, double *Z, double *W1_out,
+                              double *c1_out, double *W2_out, double *c2_out, int nthreads) {
     /* p_bstride_scale = 0: parameters are [H, ...] shared over the batch;
-       1: parameters are [B, H, ...] (one set per sequence). */
+       1: parameters are [B, H, ...] (one set per sequence).  gamma, beta: [H, d]. */
     if (B < 0 || H < 0 || T < 0 || d <= 0 || m <= 0 || b <= 0) return 1;
+    if (use_ln && (!gamma || !beta || !(eps > 0.0))) return 1;
     if (!W1 || !W2 || !W1_out || !W2_out || (T > 0 && (!Q || !K || !V || !eta || !Z))) return 1;
     const long long units = (long long)B * H;
 #ifdef _OPENMP
@@ -291,13 +318,23 @@ int ttt_oracle_mlp_forward(int B, int H, int T, int d, int m, int b, const doubl
     for (long long u = 0; u < units; ++u) {
         const long long pu = p_bstride_scale ? u : (u % H);
         const size_t tok = (size_t)u * T * d;
+        const long long hd = u % H;
         mlp_unit(T, d, m, b, Q + tok, K + tok, V + tok, eta + (size_t)u * T, W1 + (size_t)pu * d * m,
                  c1 ? c1 + (size_t)pu * m : NULL, W2 + (size_t)pu * m * d, c2 ? c2 + (size_t)pu * d : NULL,
+                 use_ln, use_ln ? gamma + (size_t)hd * d : NULL, use_ln ? beta + (size_t)hd * d : NULL, eps,
                  Z + tok, W1_out + (size_t)u * d * m, c1_out ? c1_out + (size_t)u * m : NULL,
                  W2_out + (size_t)u * m * d, c2_out ? c2_out + (size_t)u * d : NULL);
     }
     (void)nthreads;
     return 0;
+}
+
+int ttt_oracle_mlp_forward(int B, int H, int T, int d, int m, int b, const double *Q, const double *K,
+                           const double *V, const double *eta, const double *W1, const double *c1,
+                           const double *W2, const double *c2, long long p_bstride_scale, double *Z,
+                           double *W1_out, double *c1_out, double *W2_out, double *c2_out, int nthreads) {
+    return ttt_oracle_mlp_ln_forward(B, H, T, d, m, b, Q, K, V, eta, W1, c1, W2, c2, p_bstride_scale, 0, NULL,
+                                     NULL, 1e-6, Z, W1_out, c1_out, W2_out, c2_out, nthreads);
 }
 
 /* ---------------------------------------------------------------------------

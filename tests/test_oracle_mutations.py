@@ -60,10 +60,24 @@ def _build_mutant(name, old, new, tmp):
     return so
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS) + sorted(BACKWARD_MUTATIONS))
+# mistakes in the MLP with LN+residual, caught by its own pins
+MLP_LN_MUTATIONS = {
+    "mlp_ln_residual_from_wrong_input": ("ln_residual_delta(d, k, v, y, gamma, beta, eps, e, xh);",
+                                         "ln_residual_delta(d, v, v, y, gamma, beta, eps, e, xh);"),
+    "mlp_ln_output_without_residual": ("z[j] = q[j] + gamma[j] * xh[j] + beta[j];",
+                                       "z[j] = gamma[j] * xh[j] + beta[j];"),
+}
+
+PIN_FILES = {**{n: "test_oracle_pins.py" for n in MUTATIONS},
+             **{n: "test_oracle_backward.py" for n in BACKWARD_MUTATIONS},
+             **{n: "test_oracle_mlp_ln.py" for n in MLP_LN_MUTATIONS}}
+ALL_MUTATIONS = {**MUTATIONS, **BACKWARD_MUTATIONS, **MLP_LN_MUTATIONS}
+
+
+@pytest.mark.parametrize("name", sorted(ALL_MUTATIONS))
 def test_pins_catch_planted_mistake(name):
-    old, new = MUTATIONS[name] if name in MUTATIONS else BACKWARD_MUTATIONS[name]
-    pins = "test_oracle_backward.py" if name in BACKWARD_MUTATIONS else "test_oracle_pins.py"
+    old, new = ALL_MUTATIONS[name]
+    pins = PIN_FILES[name]
     with tempfile.TemporaryDirectory() as tmp:
         so = _build_mutant(name, old, new, tmp)
         env = dict(os.environ, TTT_ORACLE_LIB_OVERRIDE=so)
