@@ -193,6 +193,11 @@ ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_
  *                  be NULL (zeros).
  *   W1_out [B,H,d,m], c1_out [B,H,m], W2_out [B,H,m,d], c2_out [B,H,d]
  *                  final parameters (fp32); c1_out / c2_out may be NULL.
+ *   use_ln         1: LN+residual on the output layer (section 4.4: the form
+ *                  TTT-MLP takes in practice),
+ *                  f(x) = x + ln_gamma * LN(GELU(x W1 + c1) W2 + c2) + ln_beta,
+ *                  LN as in ttt_linear_forward (ln_gamma, ln_beta [H, d] fp32,
+ *                  ln_eps > 0).  Runs on the fp32 CUDA-core kernel.  0: plain.
  */
 typedef struct {
     int B, H, T, d, b;
@@ -214,6 +219,10 @@ typedef struct {
     float* c2_out;
     unsigned flags;
     unsigned wait_timeout_ms;
+    int use_ln;
+    const float* ln_gamma;
+    const float* ln_beta;
+    float ln_eps;
 } ttt_mlp_args;
 
 ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);

@@ -223,9 +223,15 @@ struct SimtMlpParams {
     float* c1_out;
     float* W2_out;
     float* c2_out;
+    const float* gamma;   // LN+residual on the output layer: [H, D]
+    const float* beta;
+    float eps;
 };
 
-template <int D, typename IO>
+// LN = true: f(x) = x + gamma LN(GELU(x W1 + c1) W2 + c2) + beta; the residual E of
+// layer 2 is replaced by the LN+residual backward Delta2 (as in the linear model),
+// and the outputs pass through the same LN and residual.
+template <int D, typename IO, bool LN>
 __global__ void __launch_bounds__(kSimtThreads) simt_mlp_kernel(SimtMlpParams p) {
     constexpr int M = 4 * D;
     extern __shared__ __align__(16) float sm[];
@@ -242,9 +248,13 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_kernel(SimtMlpParams p)
     float* Hq = Hk + b * M;      // b*M  (Aq, then Hq)
     float* S = Hq + b * M;       // b*b
     float* et = S + b * b;       // b
+    float* Yt = et + b;          // b*D  (LN: pre-activation of the output layer)
     const int tid = threadIdx.x;
+    const int warp = tid / 32, nwarps = kSimtThreads / 32;
     const int unit = blockIdx.x;
     const int pu = p.per_seq ? unit : unit % p.H;
+    const float* gam = LN ? p.gamma + (size_t)(unit % p.H) * D : nullptr;
+    const float* bet = LN ? p.beta + (size_t)(unit % p.H) * D : nullptr;
     const IO* Q = static_cast<const IO*>(p.Q) + (size_t)unit * p.T * D;
     const IO* K = static_cast<const IO*>(p.K) + (size_t)unit * p.T * D;
     const IO* V = static_cast<const IO*>(p.V) + (size_t)unit * p.T * D;
@@ -284,14 +294,42 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_kernel(SimtMlpParams p)
             S[e] = acc;
         }
         __syncthreads();
-        // E = Hk W2 + c2 - V
+        // E = Hk W2 + c2 - V   (LN: Delta2 = LN+residual backward at Y = Hk W2 + c2)
         for (int e = tid; e < b * D; e += kSimtThreads) {
             const int t = e / D, j = e % D;
             float acc = c2[j];
             for (int q = 0; q < M; ++q) acc += Hk[t * M + q] * W2[q * D + j];
-            Et[e] = acc - Et[e];
+            if (LN)
+                Yt[e] = acc;
+            else
+                Et[e] = acc - Et[e];
         }
         __syncthreads();
+        if (LN) {
+            for (int t = warp; t < b; t += nwarps) {
+                float mu, r;
+                warp_ln_stats(Yt + t * D, D, p.eps, mu, r);
+                float s1 = 0.f, s2 = 0.f;
+                for (int j = tid % 32; j < D; j += 32) {
+                    const float xh = (Yt[t * D + j] - mu) * r;
+                    const float g = gam[j] * (Kt[t * D + j] + gam[j] * xh + bet[j] - Et[t * D + j]);
+                    s1 += g;
+                    s2 += g * xh;
+                }
+                for (int o = 16; o > 0; o >>= 1) {
+                    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+                    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+                }
+                s1 /= D;
+                s2 /= D;
+                for (int j = tid % 32; j < D; j += 32) {
+                    const float xh = (Yt[t * D + j] - mu) * r;
+                    const float g = gam[j] * (Kt[t * D + j] + gam[j] * xh + bet[j] - Et[t * D + j]);
+                    Et[t * D + j] = r * (g - s1 - xh * s2);   // Delta2 in place of V
+                }
+            }
+            __syncthreads();
+        }
         // D1 = (E W2^T) * GELU'(A)   (in place of A)
         for (int e = tid; e < b * M; e += kSimtThreads) {
             const int t = e / M, q = e % M;
@@ -320,15 +358,27 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_kernel(SimtMlpParams p)
             S[e] = acc;
         }
         __syncthreads();
-        // Z = Hq W2 + c2 - S2 E
+        // Z = Hq W2 + c2 - S2 E   (LN: Z = Q + gamma LN(that) + beta)
         for (int e = tid; e < b * D; e += kSimtThreads) {
             const int t = e / D, j = e % D;
             float acc = c2[j];
             for (int q = 0; q < M; ++q) acc += Hq[t * M + q] * W2[q * D + j];
             for (int s = 0; s <= t; ++s) acc -= S[t * b + s] * Et[s * D + j];
-            IoTraits<IO>::store(Z, (size_t)t0 * D + e, acc);
+            if (LN)
+                Yt[e] = acc;
+            else
+                IoTraits<IO>::store(Z, (size_t)t0 * D + e, acc);
         }
         __syncthreads();
+        if (LN) {
+            for (int t = warp; t < b; t += nwarps) {
+                float mu, r;
+                warp_ln_stats(Yt + t * D, D, p.eps, mu, r);
+                for (int j = tid % 32; j < D; j += 32)
+                    IoTraits<IO>::store(Z, (size_t)(t0 + t) * D + j,
+                                        Qt[t * D + j] + gam[j] * (Yt[t * D + j] - mu) * r + bet[j]);
+            }
+        }
         // state update
         for (int e = tid; e < D * M; e += kSimtThreads) {
             const int i = e / M, q = e % M;
@@ -364,9 +414,9 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_kernel(SimtMlpParams p)
         for (int e = tid; e < D; e += kSimtThreads) p.c2_out[(size_t)unit * D + e] = c2[e];
 }
 
-inline size_t simt_mlp_smem(int D, int b) {
+inline size_t simt_mlp_smem(int D, int b, bool ln) {
     const size_t M = 4 * (size_t)D;
-    return sizeof(float) * (2 * D * M + M + D + 3 * (size_t)b * D + 3 * (size_t)b * M + (size_t)b * b + b);
+    return sizeof(float) * (2 * D * M + M + D + (ln ? 4 : 3) * (size_t)b * D + 3 * (size_t)b * M + (size_t)b * b + b);
 }
 
 }  // namespace ttt

@@ -249,8 +249,11 @@ ttt_status launch_simt_mlp(const ttt_mlp_args* a, cudaStream_t st) {
     p.c1_out = a->c1_out;
     p.W2_out = a->W2_out;
     p.c2_out = a->c2_out;
-    const size_t smem = simt_mlp_smem(D, a->b);
-    auto k = simt_mlp_kernel<D, IO>;
+    p.gamma = a->ln_gamma;
+    p.beta = a->ln_beta;
+    p.eps = a->ln_eps;
+    const size_t smem = simt_mlp_smem(D, a->b, a->use_ln != 0);
+    auto k = a->use_ln ? simt_mlp_kernel<D, IO, true> : simt_mlp_kernel<D, IO, false>;
     if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
     k<<<a->B * a->H, kSimtThreads, smem, st>>>(p);
     return launch_status();
@@ -317,7 +320,9 @@ extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream
         return TTT_ERR_INVALID_ARG;
     if (a->params_per_sequence != 0 && a->params_per_sequence != 1) return TTT_ERR_INVALID_ARG;
     if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL)) return TTT_ERR_INVALID_ARG;
-    const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
+    if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
+    if (a->use_ln && (!ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !(a->ln_eps > 0.f))) return TTT_ERR_INVALID_ARG;
+    const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 && !a->use_ln &&
                     !(a->flags & TTT_FLAG_FORCE_SIMT);
     if (tc) return tc_mlp(a, stream);
     if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;

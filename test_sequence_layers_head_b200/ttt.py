@@ -47,7 +47,8 @@ class MlpArgs(ctypes.Structure):
                 ("Q", _vp), ("K", _vp), ("V", _vp), ("eta", _vp), ("eta_const", _f),
                 ("W1", _vp), ("c1", _vp), ("W2", _vp), ("c2", _vp), ("params_per_sequence", _i),
                 ("Z", _vp), ("W1_out", _vp), ("c1_out", _vp), ("W2_out", _vp), ("c2_out", _vp),
-                ("flags", _u), ("wait_timeout_ms", _u)]
+                ("flags", _u), ("wait_timeout_ms", _u), ("use_ln", _i), ("ln_gamma", _vp), ("ln_beta", _vp),
+                ("ln_eps", _f)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -197,8 +198,10 @@ def linear_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW_out=None, eta_cons
 
 
 def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, *, eta_const=0.0, Z=None, W1_out=None, c1_out=None,
-                W2_out=None, c2_out=None, flags=0, wait_timeout_ms=0, stream=None):
-    """TTT-MLP prefill; see ``ttt_mlp_forward``.  Returns (Z, W1, c1, W2, c2)."""
+                W2_out=None, c2_out=None, flags=0, wait_timeout_ms=0, use_ln=False, gamma=None, beta=None,
+                eps=1e-6, stream=None):
+    """TTT-MLP prefill; see ``ttt_mlp_forward``.  Returns (Z, W1, c1, W2, c2).
+    use_ln: LN+residual on the output layer with gamma, beta [H,d]."""
     B, H, T, d = Q.shape
     m = W1.shape[-1]
     dev = Q.device
@@ -211,7 +214,8 @@ def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, *, eta_const=0.0, Z=None, W1_ou
     per_seq = 1 if W1.dim() == 4 else 0
     a = MlpArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
                 _ptr(W1), _ptr(c1), _ptr(W2), _ptr(c2), per_seq, _ptr(Z), _ptr(W1_out), _ptr(c1_out),
-                _ptr(W2_out), _ptr(c2_out), int(flags), int(wait_timeout_ms))
+                _ptr(W2_out), _ptr(c2_out), int(flags), int(wait_timeout_ms), int(bool(use_ln)), _ptr(gamma),
+                _ptr(beta), float(eps))
     _check(library().ttt_mlp_forward(ctypes.byref(a), _stream(stream)), "ttt_mlp_forward")
     return Z, W1_out, c1_out, W2_out, c2_out
 

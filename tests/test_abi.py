@@ -198,6 +198,23 @@ def test_mlp_decode_validation(ttt_lib, kw, code):
     assert ttt_lib.library().ttt_mlp_decode_step(ctypes.byref(a), None) == code
 
 
+def test_mlp_ln_validation(ttt_lib):
+    L = ttt_lib.library()
+    fake = 1 << 20
+    m = ttt_lib.MlpArgs()
+    m.B, m.H, m.T, m.d, m.b, m.io_dtype = 1, 1, 32, 64, 16, ttt_lib.TTT_BF16
+    m.Q = m.K = m.V = m.Z = m.W1 = m.W2 = m.W1_out = m.W2_out = fake
+    m.use_ln = 2
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
+    m.use_ln = 1                     # no gamma / beta
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
+    m.ln_gamma = m.ln_beta = fake    # eps = 0
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
+    m.ln_eps = 1e-6
+    m.ln_beta = fake + 4             # misaligned
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
+
+
 def test_binding_refuses_cpu_tensors(ttt_lib):
     import torch
     x = torch.zeros(1, 1, 16, 64, dtype=torch.bfloat16)

@@ -235,6 +235,26 @@ def test_mlp_d64_bf16(ttt_lib, B, H, T):
     check_mlp(ttt_lib, inp)
 
 
+@pytest.mark.parametrize("d,b,T,io", [(16, 16, 64, WL.F32), (32, 4, 48, WL.F32), (64, 16, 64, WL.BF16),
+                                      (16, 1, 12, WL.F32)])
+def test_mlp_ln_matches_oracle(ttt_lib, d, b, T, io):
+    """TTT-MLP with LN+residual on the output layer (fp32 CUDA-core kernel)."""
+    inp = WL.random_case("mlp", 2, 3, T, d, b, io_dtype=io, eta_mode="sigmoid", seed=d + b + T)
+    rng = np.random.default_rng(d + 3 * b)
+    gr, ge = WL.store(1 + rng.standard_normal((3, d)) * 0.14, WL.F32)
+    br, be = WL.store(rng.standard_normal((3, d)) * 0.14, WL.F32)
+    r, e = inp.raw, inp.exact
+    dev = {k: to_dev(r[k]) for k in ("Q", "K", "V", "eta", "W1", "c1", "W2", "c2")}
+    out = ttt_lib.mlp_forward(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W1"], dev["c1"], dev["W2"], dev["c2"],
+                              b, Z=poison_like(dev["Q"]), use_ln=True, gamma=to_dev(gr), beta=to_dev(br))
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    ref = O.mlp_forward(e["Q"], e["K"], e["V"], e["eta"], e["W1"], e["c1"], e["W2"], e["c2"], b, use_ln=True,
+                        gamma=ge, beta=be)
+    for name, g, o in zip(("Z", "W1", "c1", "W2", "c2"), out, ref):
+        assert_close(name, to_host(g), o, io)
+
+
 def test_mlp_tc_matches_simt(ttt_lib):
     """The tensor-core and the fp32 CUDA-core MLP kernels agree on the same inputs."""
     inp = WL.random_case("mlp", 1, 3, 96, 64, 16, io_dtype=WL.BF16, eta_mode="const", eta_const=1 / 64, seed=41)
