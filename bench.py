@@ -387,6 +387,27 @@ def measure_backward(ttt, torch, threads, name="linear_B8_H12_T2048"):
             "kernel": "mma_linear_backward_kernel (mma.sync, bf16 operands, fp32 accumulation)"}
 
 
+def measure_mlp_ln(ttt, torch, threads, T=2048):
+    """TTT-MLP with LN+residual on the output layer (fp32 CUDA-core kernel) on
+    the MLP workload's shapes at a shorter T (informational)."""
+    w = WL.scaled(WL.WORKLOADS["mlp_B2_H32_T8192"], T=T)
+    _, dev = device_inputs(w, torch, threads)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(3)
+    gam = 1 + 0.14 * torch.randn(w.H, w.d, generator=g, device="cuda")
+    bet = 0.14 * torch.randn(w.H, w.d, generator=g, device="cuda")
+    flush_buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")
+
+    def fn():
+        ttt.mlp_forward(dev["Q"], dev["K"], dev["V"], dev.get("eta"), dev["W1"], dev["c1"], dev["W2"], dev["c2"],
+                        w.b, eta_const=w.eta_const, use_ln=True, gamma=gam, beta=bet)
+    ms = statistics.median(time_launches(torch, fn, 3, 1, flush=lambda: flush_buf.zero_()))
+    _, tflops, _ = measured_peaks()
+    return {"ms": ms, "tokens_per_s": tokens(w) / (ms / 1000.0),
+            "tensor_frac": algorithmic_flops(w) / (ms / 1000.0) / 1e12 / tflops,
+            "kernel": "simt_mlp_kernel<64, bf16, LN> (fp32 CUDA cores)"}
+
+
 def measure_e2e_chunked(ttt, w, inp, torch, steps, chunks=8):
     """The public API on pinned host buffers, streamed along the sequence:
     the T tokens go through `chunks` calls of ttt_linear_forward, each
@@ -618,6 +639,7 @@ def run_ours(args):
             line["rows"]["decode_ln_B4_H32"] = measure_decode_variant(ttt, torch, "ln", 4, 32)
             line["rows"]["decode_mlp_B2_H32"] = measure_decode_variant(ttt, torch, "mlp", 2, 32)
             line["rows"]["backward_linear_B8_H12_T2048"] = measure_backward(ttt, torch, threads)
+            line["rows"]["mlp_ln_B2_H32_T2048"] = measure_mlp_ln(ttt, torch, threads)
         line["cpu_baseline"] = cpu_baseline(w)
     if dist is not None:
         dist.barrier()
@@ -653,9 +675,28 @@ def run_reference(args):
     w = WL.WORKLOADS[args.workload]
     if args.T:
         w = WL.scaled(w, T=args.T)
+    # the sample (generated once): sequence 0, one head per host core (its first heads are the
+    # workload's own), so every step keeps all cores busy and takes a fraction of a second
+    from oracle import oracle as O
+    cores = O.default_threads()
+    heads = max(1, min(w.H, cores))
+    sample = WL.scaled(w, B=1, H=heads)
+    e = WL.make_inputs(sample, threads=cores).exact
+    eta = e["eta"] if w.eta_mode == "sigmoid" else np.full(e["eta"].shape, w.eta_const)
+
+    def step():
+        t0 = time.perf_counter()
+        if w.kind == "mlp":
+            O.mlp_forward(e["Q"], e["K"], e["V"], eta, e["W1"], e["c1"], e["W2"], e["c2"], w.b, threads=cores)
+        else:
+            ln = w.kind == "ln"
+            kw = dict(c0=e["c0"], gamma=e["gamma"], beta=e["beta"], eps=w.ln_eps) if ln else {}
+            O.linear_forward(e["Q"], e["K"], e["V"], eta, e["W0"], w.b, use_ln=ln, threads=cores, **kw)
+        dt = time.perf_counter() - t0
+        return {"value": w.T * heads / w.H / dt, "seconds": dt, "cores": cores}
     for _ in range(args.warmup):
-        cpu_baseline(w, sample_sequences=1)
-    vals = [cpu_baseline(w, sample_sequences=1) for _ in range(args.steps)]
+        step()
+    vals = [step() for _ in range(args.steps)]
     value = statistics.mean(v["value"] for v in vals)
     secs = sum(v["seconds"] for v in vals)
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
@@ -663,7 +704,8 @@ def run_reference(args):
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "kind": w.kind, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "b": w.b},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": vals[0]["cores"], "kind": "oracle",
-                             "sample": f"each step: 1 of {w.B} sequences x {w.H} heads x T={w.T}"},
+                             "sample": f"each step: 1 of {w.B} sequences x {heads} of {w.H} heads x T={w.T} "
+                                       f"(tokens/s scaled by {w.H}/{heads} heads)"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -710,8 +752,9 @@ def run_b_sweep(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=3)
+    # about 0.5 s of timed work on the default workload, so that the 100 ms clock samples cover it
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WL.WORKLOAD_ORDER)
     ap.add_argument("--T", type=int, default=0, help="override T (profiling a smaller case)")
