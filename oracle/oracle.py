@@ -38,6 +38,9 @@ def lib():
         L.ttt_oracle_linear_decode_step.restype = i
         L.ttt_oracle_linear_backward.argtypes = [i, i, i, i, i, P, P, P, P, P, ll, P, P, P, P, P, P, P, i]
         L.ttt_oracle_linear_backward.restype = i
+        L.ttt_oracle_linear_ln_backward.argtypes = [i, i, i, i, i, P, P, P, P, P, ll, P, ll, P, P, dbl, P, P, P,
+                                                    P, P, P, P, P, P, P, P, i]
+        L.ttt_oracle_linear_ln_backward.restype = i
         _lib = L
     return _lib
 
@@ -140,3 +143,26 @@ def linear_backward(Q, K, V, eta, W0, b, dZ=None, dW_out=None, threads=None):
     if rc != 0:
         raise ValueError("oracle: invalid arguments")
     return dQ, dK, dV, deta, dW0
+
+
+def linear_ln_backward(Q, K, V, eta, W0, b, c0, gamma, beta, eps=1e-6, dZ=None, dW_out=None, dc_out=None,
+                       threads=None):
+    """Outer-loop gradients of the LN+residual TTT-Linear forward, reverse mode
+    through the primal loop.  Returns (dQ, dK, dV, deta, dW0, dc0, dgamma,
+    dbeta); dW0, dc0, dgamma and dbeta are per unit [B,H,...] (sum over what
+    is shared)."""
+    Q, K, V, eta, W0, c0, gamma, beta = map(_f64, (Q, K, V, eta, W0, c0, gamma, beta))
+    dZ, dW_out, dc_out = map(_f64, (dZ, dW_out, dc_out))
+    B, H, T, d = Q.shape
+    W0_bstride = 0 if W0.ndim == 3 else H * d * d
+    c0_bstride = 0 if (c0 is None or c0.ndim == 2) else H * d
+    dQ, dK, dV = np.empty((B, H, T, d)), np.empty((B, H, T, d)), np.empty((B, H, T, d))
+    deta, dW0, dc0 = np.empty((B, H, T)), np.empty((B, H, d, d)), np.empty((B, H, d))
+    dgamma, dbeta = np.empty((B, H, d)), np.empty((B, H, d))
+    rc = lib().ttt_oracle_linear_ln_backward(B, H, T, d, b, _p(Q), _p(K), _p(V), _p(eta), _p(W0), W0_bstride,
+                                             _p(c0), c0_bstride, _p(gamma), _p(beta), eps, _p(dZ), _p(dW_out),
+                                             _p(dc_out), _p(dQ), _p(dK), _p(dV), _p(deta), _p(dW0), _p(dc0),
+                                             _p(dgamma), _p(dbeta), threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: invalid arguments")
+    return dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta

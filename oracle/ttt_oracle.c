@@ -34,7 +34,8 @@
  *   - Outer-loop gradients (section 3.4: the outer loop trains the
  *     projections, the initial state and the learning-rate parameters with
  *     gradients that pass through the inner loop's updates):
- *     the backward of the TTT-Linear forward is reverse-mode
+ *     the backward of the TTT-Linear forward, plain and LN+residual (there
+ *     also the initial bias and the LN parameters), is reverse-mode
  *     differentiation of the same primal loop, token by token.
  *
  * Readings of points the pages leave open (each one is listed in the design
@@ -488,6 +489,233 @@ int ttt_oracle_linear_backward(int B, int H, int T, int d, int b, const double *
                              W0 + (size_t)n * W0_bstride + (size_t)h * d * d, dZ ? dZ + tok : NULL,
                              dW_out ? dW_out + (size_t)u * d * d : NULL, dQ + tok, dK + tok, dV + tok,
                              deta + (size_t)u * T, dW0 + (size_t)u * d * d);
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Backward of the LN+residual TTT-Linear forward, f(x) = x + gamma LN(x W + c)
+ * + beta: reverse-mode differentiation of the primal loop, token by token.
+ * Besides the linear model's gradients it returns dc0 (the initial bias) and
+ * dgamma, dbeta (the LN parameters, outer-loop parameters fixed inside the
+ * inner loop), each per unit; the caller sums over what it shares.
+ *
+ * Forward of token t with batch-start state (W_s, c_s) and running (W, c):
+ *   y = k W_s + c_s,  xh = (y - mean y) r,  r = 1/sqrt(var y + eps)
+ *   e = k + gamma xh + beta - v,  g = gamma e
+ *   u = g - mean(g) - xh mean(g xh),  delta = r u
+ *   W_t = W_{t-1} - eta k^T delta,  c_t = c_{t-1} - eta delta
+ *   p = q W_t + c_t,  xo = LN(p) (with r_o),  z = q + gamma xo + beta
+ * Each step below is the adjoint of one of these lines, last to first.
+ * ------------------------------------------------------------------------- */
+
+/* adjoint of xh = LN(y) (mean and variance over d, r = 1/sqrt(var + eps)):
+   dy = r (dxh - mean(dxh) - xh mean(dxh xh)) */
+static void ln_adjoint(int d, const double *xh, double r, const double *dxh, double *dy) {
+    double m1 = 0.0, m2 = 0.0;
+    for (int j = 0; j < d; ++j) { m1 += dxh[j]; m2 += dxh[j] * xh[j]; }
+    m1 /= d;
+    m2 /= d;
+    for (int j = 0; j < d; ++j) dy[j] = r * (dxh[j] - m1 - xh[j] * m2);
+}
+
+static void linear_ln_unit_backward(int T, int d, int b, const double *Q, const double *K, const double *V,
+                                    const double *eta, const double *W0, const double *c0, const double *gamma,
+                                    const double *beta, double eps, const double *dZ, const double *dWout,
+                                    const double *dcout, double *dQ, double *dK, double *dV, double *deta,
+                                    double *dW0, double *dc0, double *dgamma, double *dbeta) {
+    const size_t dd = (size_t)d * d;
+    const int nb = (T + b - 1) / b;
+    double *Wst = malloc((size_t)(nb > 0 ? nb : 1) * dd * sizeof(double));   /* batch-start W */
+    double *cst = malloc((size_t)(nb > 0 ? nb : 1) * d * sizeof(double));    /* batch-start c */
+    double *Wrun = malloc((size_t)(b + 1) * dd * sizeof(double));
+    double *crun = malloc((size_t)(b + 1) * d * sizeof(double));
+    double *DW = malloc(dd * sizeof(double)), *Dc = malloc(d * sizeof(double));
+    double *DWs = malloc(dd * sizeof(double)), *Dcs = malloc(d * sizeof(double));
+    /* per token of a batch: xh, r, e, g, u, delta */
+    double *xh = malloc((size_t)b * d * sizeof(double)), *rr = malloc((size_t)b * sizeof(double));
+    double *ee = malloc((size_t)b * d * sizeof(double)), *gg = malloc((size_t)b * d * sizeof(double));
+    double *uu = malloc((size_t)b * d * sizeof(double)), *dl = malloc((size_t)b * d * sizeof(double));
+    double *mgx = malloc((size_t)b * sizeof(double));
+    double *y = malloc(d * sizeof(double)), *p = malloc(d * sizeof(double)), *xo = malloc(d * sizeof(double));
+    double *t1 = malloc(d * sizeof(double)), *t2 = malloc(d * sizeof(double)), *t3 = malloc(d * sizeof(double));
+    double *dxh = malloc(d * sizeof(double)), *dy = malloc(d * sizeof(double));
+    double *Wc = malloc(dd * sizeof(double)), *cc = malloc(d * sizeof(double));
+
+    /* token forward at the batch start: fills xh, r, e, g, u, delta of row i */
+    #define TOKEN_FWD(t, i, Ws, cs)                                                                    \
+        do {                                                                                           \
+            const double *k_ = K + (size_t)(t) * d, *v_ = V + (size_t)(t) * d;                         \
+            vec_mat(d, d, k_, (Ws), y);                                                                \
+            for (int j = 0; j < d; ++j) y[j] += (cs)[j];                                               \
+            rr[i] = layer_norm(d, y, eps, xh + (size_t)(i) * d);                                       \
+            double mg = 0.0, mgx_ = 0.0;                                                               \
+            for (int j = 0; j < d; ++j) {                                                              \
+                const double x_ = xh[(size_t)(i) * d + j];                                             \
+                ee[(size_t)(i) * d + j] = k_[j] + gamma[j] * x_ + beta[j] - v_[j];                     \
+                gg[(size_t)(i) * d + j] = gamma[j] * ee[(size_t)(i) * d + j];                          \
+                mg += gg[(size_t)(i) * d + j];                                                         \
+                mgx_ += gg[(size_t)(i) * d + j] * x_;                                                  \
+            }                                                                                          \
+            mg /= d;                                                                                   \
+            mgx_ /= d;                                                                                 \
+            mgx[i] = mgx_;                                                                             \
+            for (int j = 0; j < d; ++j) {                                                              \
+                const double x_ = xh[(size_t)(i) * d + j];                                             \
+                uu[(size_t)(i) * d + j] = gg[(size_t)(i) * d + j] - mg - x_ * mgx_;                    \
+                dl[(size_t)(i) * d + j] = rr[i] * uu[(size_t)(i) * d + j];                             \
+            }                                                                                          \
+        } while (0)
+
+    /* forward re-run: batch-start states */
+    memcpy(Wc, W0, dd * sizeof(double));
+    if (c0) memcpy(cc, c0, d * sizeof(double)); else memset(cc, 0, d * sizeof(double));
+    for (int i = 0; i < nb; ++i) {
+        const int t0 = i * b, t1_ = (t0 + b < T) ? t0 + b : T;
+        memcpy(Wst + (size_t)i * dd, Wc, dd * sizeof(double));
+        memcpy(cst + (size_t)i * d, cc, d * sizeof(double));
+        for (int t = t0; t < t1_; ++t) {
+            TOKEN_FWD(t, t - t0, Wst + (size_t)i * dd, cst + (size_t)i * d);
+            const double *k = K + (size_t)t * d;
+            for (int a = 0; a < d; ++a)
+                for (int j = 0; j < d; ++j) Wc[(size_t)a * d + j] -= eta[t] * k[a] * dl[(size_t)(t - t0) * d + j];
+            for (int j = 0; j < d; ++j) cc[j] -= eta[t] * dl[(size_t)(t - t0) * d + j];
+        }
+    }
+    /* reverse sweep */
+    if (dWout) memcpy(DW, dWout, dd * sizeof(double)); else memset(DW, 0, dd * sizeof(double));
+    if (dcout) memcpy(Dc, dcout, d * sizeof(double)); else memset(Dc, 0, d * sizeof(double));
+    memset(dgamma, 0, d * sizeof(double));
+    memset(dbeta, 0, d * sizeof(double));
+    for (int i = nb - 1; i >= 0; --i) {
+        const int t0 = i * b, t1_ = (t0 + b < T) ? t0 + b : T;
+        const double *Ws = Wst + (size_t)i * dd, *cs = cst + (size_t)i * d;
+        /* recompute the batch: per-token quantities and running states */
+        memcpy(Wrun, Ws, dd * sizeof(double));
+        memcpy(crun, cs, d * sizeof(double));
+        for (int t = t0; t < t1_; ++t) {
+            const int li = t - t0;
+            TOKEN_FWD(t, li, Ws, cs);
+            const double *k = K + (size_t)t * d;
+            const double *Wp = Wrun + (size_t)li * dd, *cp = crun + (size_t)li * d;
+            double *Wn = Wrun + (size_t)(li + 1) * dd, *cn = crun + (size_t)(li + 1) * d;
+            for (int a = 0; a < d; ++a)
+                for (int j = 0; j < d; ++j)
+                    Wn[(size_t)a * d + j] = Wp[(size_t)a * d + j] - eta[t] * k[a] * dl[(size_t)li * d + j];
+            for (int j = 0; j < d; ++j) cn[j] = cp[j] - eta[t] * dl[(size_t)li * d + j];
+        }
+        memset(DWs, 0, dd * sizeof(double));
+        memset(Dcs, 0, d * sizeof(double));
+        for (int t = t1_ - 1; t >= t0; --t) {
+            const int li = t - t0;
+            const double *q = Q + (size_t)t * d, *k = K + (size_t)t * d;
+            const double *Wt = Wrun + (size_t)(li + 1) * dd, *ct = crun + (size_t)(li + 1) * d;
+            const double *xt = xh + (size_t)li * d, *et = ee + (size_t)li * d, *gt = gg + (size_t)li * d;
+            const double *ut = uu + (size_t)li * d, *dt = dl + (size_t)li * d;
+            double *dq = dQ + (size_t)t * d, *dk = dK + (size_t)t * d, *dv = dV + (size_t)t * d;
+            for (int j = 0; j < d; ++j) { dq[j] = 0.0; dk[j] = 0.0; }
+            /* z = q + gamma xo + beta, xo = LN(p), p = q W_t + c_t */
+            if (dZ) {
+                const double *dz = dZ + (size_t)t * d;
+                vec_mat(d, d, q, Wt, p);
+                for (int j = 0; j < d; ++j) p[j] += ct[j];
+                const double ro = layer_norm(d, p, eps, xo);
+                for (int j = 0; j < d; ++j) {
+                    dq[j] += dz[j];
+                    dgamma[j] += dz[j] * xo[j];
+                    dbeta[j] += dz[j];
+                    t1[j] = gamma[j] * dz[j];
+                }
+                ln_adjoint(d, xo, ro, t1, t2);   /* t2 = dp */
+                for (int a = 0; a < d; ++a) {
+                    double acc = 0.0;
+                    for (int j = 0; j < d; ++j) acc += t2[j] * Wt[(size_t)a * d + j];
+                    dq[a] += acc;
+                }
+                for (int a = 0; a < d; ++a)
+                    for (int j = 0; j < d; ++j) DW[(size_t)a * d + j] += q[a] * t2[j];
+                for (int j = 0; j < d; ++j) Dc[j] += t2[j];
+            }
+            /* W_t = W_{t-1} - eta k^T delta,  c_t = c_{t-1} - eta delta */
+            double ge = 0.0;
+            for (int j = 0; j < d; ++j) {
+                double acc = Dc[j];
+                for (int a = 0; a < d; ++a) acc += k[a] * DW[(size_t)a * d + j];
+                t3[j] = -eta[t] * acc;   /* t3 = ddelta */
+                ge += acc * dt[j];
+            }
+            deta[t] = -ge;
+            for (int a = 0; a < d; ++a) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += dt[j] * DW[(size_t)a * d + j];
+                dk[a] += -eta[t] * acc;
+            }
+            /* delta = r u, u = g - mean(g) - xh mean(g xh) */
+            double dr = 0.0;
+            for (int j = 0; j < d; ++j) { dr += t3[j] * ut[j]; t1[j] = rr[li] * t3[j]; }   /* t1 = du */
+            double mdu = 0.0, mdux = 0.0;
+            for (int j = 0; j < d; ++j) { mdu += t1[j]; mdux += t1[j] * xt[j]; }
+            mdu /= d;
+            mdux /= d;
+            for (int j = 0; j < d; ++j) {
+                const double dg = t1[j] - mdu - xt[j] * mdux;
+                dxh[j] = -t1[j] * mgx[li] - gt[j] * mdux;   /* through the xh of u */
+                /* g = gamma e, e = k + gamma xh + beta - v */
+                const double de = gamma[j] * dg;
+                dgamma[j] += et[j] * dg + xt[j] * de;
+                dbeta[j] += de;
+                dk[j] += de;
+                dv[j] = -de;
+                dxh[j] += gamma[j] * de;
+            }
+            /* xh = LN(y), and r = 1/sqrt(var + eps) in delta = r u: dr/dy_j = -r^2 xh_j / d */
+            ln_adjoint(d, xt, rr[li], dxh, dy);
+            for (int j = 0; j < d; ++j) dy[j] += dr * (-rr[li] * rr[li] * xt[j] / d);
+            /* y = k W_s + c_s */
+            for (int a = 0; a < d; ++a) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += dy[j] * Ws[(size_t)a * d + j];
+                dk[a] += acc;
+            }
+            for (int a = 0; a < d; ++a)
+                for (int j = 0; j < d; ++j) DWs[(size_t)a * d + j] += k[a] * dy[j];
+            for (int j = 0; j < d; ++j) Dcs[j] += dy[j];
+        }
+        for (size_t x = 0; x < dd; ++x) DW[x] += DWs[x];
+        for (int j = 0; j < d; ++j) Dc[j] += Dcs[j];
+    }
+    #undef TOKEN_FWD
+    memcpy(dW0, DW, dd * sizeof(double));
+    memcpy(dc0, Dc, d * sizeof(double));
+    free(Wst); free(cst); free(Wrun); free(crun); free(DW); free(Dc); free(DWs); free(Dcs);
+    free(xh); free(rr); free(ee); free(gg); free(uu); free(dl); free(mgx);
+    free(y); free(p); free(xo); free(t1); free(t2); free(t3); free(dxh); free(dy); free(Wc); free(cc);
+}
+
+int ttt_oracle_linear_ln_backward(int B, int H, int T, int d, int b, const double *Q, const double *K,
+                                  const double *V, const double *eta, const double *W0, long long W0_bstride,
+                                  const double *c0, long long c0_bstride, const double *gamma, const double *beta,
+                                  double eps, const double *dZ, const double *dW_out, const double *dc_out,
+                                  double *dQ, double *dK, double *dV, double *deta, double *dW0, double *dc0,
+                                  double *dgamma, double *dbeta, int threads) {
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || b <= 0 || !Q || !K || !V || !eta || !W0 || !gamma || !beta ||
+        !(eps > 0.0) || !dQ || !dK || !dV || !deta || !dW0 || !dc0 || !dgamma || !dbeta)
+        return 1;
+    const long long units = (long long)B * H;
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long long u = 0; u < units; ++u) {
+        const long long n = u / H, h = u % H;
+        const size_t tok = (size_t)u * T * d;
+        linear_ln_unit_backward(T, d, b, Q + tok, K + tok, V + tok, eta + (size_t)u * T,
+                                W0 + (size_t)n * W0_bstride + (size_t)h * d * d,
+                                c0 ? c0 + (size_t)n * c0_bstride + (size_t)h * d : NULL, gamma + (size_t)h * d,
+                                beta + (size_t)h * d, eps, dZ ? dZ + tok : NULL,
+                                dW_out ? dW_out + (size_t)u * d * d : NULL, dc_out ? dc_out + (size_t)u * d : NULL,
+                                dQ + tok, dK + tok, dV + tok, deta + (size_t)u * T, dW0 + (size_t)u * d * d,
+                                dc0 + (size_t)u * d, dgamma + (size_t)u * d, dbeta + (size_t)u * d);
     }
     return 0;
 }

@@ -83,3 +83,56 @@ def test_backward_without_upstream_gradients_is_zero():
     out = O.linear_backward(Q, K, V, eta, W0, 2, threads=1)
     for g in out:
         assert np.all(g == 0)
+
+
+# ---------------------------------------------------------------------------
+# LN+residual: f(x) = x + gamma LN(x W + c) + beta (section 4.4); the outer
+# loop also trains the LN parameters and the initial bias
+# ---------------------------------------------------------------------------
+
+def _ln_case(B, H, T, d, shared, seed):
+    Q, K, V, eta, W0, dZ, dW = _case(B, H, T, d, shared, seed)
+    rng = np.random.default_rng(seed + 1)
+    c0 = rng.standard_normal((H, d) if shared else (B, H, d)) * 0.2
+    gamma = 1 + rng.standard_normal((H, d)) * 0.3
+    beta = rng.standard_normal((H, d)) * 0.3
+    dc = rng.standard_normal((B, H, d))
+    return Q, K, V, eta, W0, c0, gamma, beta, dZ, dW, dc
+
+
+def _ln_loss(Q, K, V, eta, W0, c0, gamma, beta, b, dZ, dW, dc):
+    Z, W_out, c_out = O.linear_forward(Q, K, V, eta, W0, b, c0=c0, gamma=gamma, beta=beta, use_ln=True, threads=1)
+    return float(np.sum(Z * dZ) + np.sum(W_out * dW) + np.sum(c_out * dc))
+
+
+@pytest.mark.parametrize("B,H,T,d,b,shared", [
+    (1, 2, 5, 3, 2, True),     # ragged last mini-batch
+    (2, 1, 6, 3, 3, False),    # per-sequence W0 and c0
+    (1, 1, 4, 3, 1, True),     # b = 1
+    (1, 1, 4, 4, 4, True),     # one mini-batch
+])
+def test_ln_backward_matches_finite_differences(B, H, T, d, b, shared):
+    Q, K, V, eta, W0, c0, gamma, beta, dZ, dW, dc = _ln_case(B, H, T, d, shared, seed=100 + 10 * T + d + b)
+    g = O.linear_ln_backward(Q, K, V, eta, W0, b, c0, gamma, beta, dZ=dZ, dW_out=dW, dc_out=dc, threads=1)
+    dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta = g
+    if shared:
+        dW0, dc0 = dW0.sum(axis=0), dc0.sum(axis=0)
+    grads = {"Q": dQ, "K": dK, "V": dV, "eta": deta, "W0": dW0, "c0": dc0, "gamma": dgamma.sum(axis=0),
+             "beta": dbeta.sum(axis=0)}
+    inputs = {"Q": Q, "K": K, "V": V, "eta": eta, "W0": W0, "c0": c0, "gamma": gamma, "beta": beta}
+    # the LN makes the loss strongly curved in some directions (the central difference's error
+    # falls as h^2 there), so a smaller step than for the linear model
+    h = 1e-7
+    for name, x in inputs.items():
+        gr = grads[name]
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            keep = x[idx]
+            x[idx] = keep + h
+            lp = _ln_loss(*inputs.values(), b, dZ, dW, dc)
+            x[idx] = keep - h
+            lm = _ln_loss(*inputs.values(), b, dZ, dW, dc)
+            x[idx] = keep
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.max(np.abs(fd - gr)) / max(np.max(np.abs(fd)), 1e-12)
+        assert err < 1e-6, (name, err)

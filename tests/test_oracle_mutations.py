@@ -39,6 +39,9 @@ BACKWARD_MUTATIONS = {
     "bwd_missing_residual_path": ("dK[(size_t)t * d + a] = -eta[t] * acc1 + acc2;",
                                   "dK[(size_t)t * d + a] = -eta[t] * acc1;"),
     "bwd_state_grad_drops_residual": ("for (size_t x = 0; x < dd; ++x) D[x] += dWs[x];", "(void)dWs;"),
+    "bwd_ln_explicit_r_term_dropped": ("for (int j = 0; j < d; ++j) dy[j] += dr * (-rr[li] * rr[li] * xt[j] / d);",
+                                       "(void)dr;"),
+    "bwd_ln_xhat_path_through_u_dropped": ("dxh[j] = -t1[j] * mgx[li] - gt[j] * mdux;", "dxh[j] = 0.0;"),
     "bwd_output_grad_dropped_from_state": (
         "            if (dz)\n                for (int a = 0; a < d; ++a)\n                    for (int j = 0; j < d; ++j) D[(size_t)a * d + j] += q[a] * dz[j];\n",
         ""),
