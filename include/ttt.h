@@ -101,10 +101,11 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
  *   W_states       optional output for the backward (gradient checkpointing
  *                  through time, section 6.12): the state at the start of
  *                  every mini-batch, [B, H, T/b, d, d] fp32, T/b states per
- *                  unit.  NULL: not written.  Non-NULL requires use_ln == 0;
- *                  with io_dtype BF16, d = 64, b = 16 it runs the mma.sync
- *                  forward (bf16 operands, fp32 state), otherwise the fp32
- *                  CUDA-core kernel.
+ *                  unit.  NULL: not written.  With use_ln == 0, io_dtype
+ *                  BF16, d = 64, b = 16 it runs the mma.sync forward (bf16
+ *                  operands, fp32 state), otherwise the fp32 CUDA-core kernel.
+ *   c_states       with use_ln and W_states: the bias at the start of every
+ *                  mini-batch, [B, H, T/b, d] fp32 (required then).
  */
 typedef struct {
     int B, H, T, d, b;
@@ -128,6 +129,7 @@ typedef struct {
     unsigned flags;
     unsigned wait_timeout_ms;
     float* W_states;
+    float* c_states;
 } ttt_linear_args;
 
 ttt_status ttt_linear_forward(const ttt_linear_args* args, cudaStream_t stream);
@@ -153,10 +155,18 @@ ttt_status ttt_linear_forward(const ttt_linear_args* args, cudaStream_t stream);
  *   dW0            output [B, H, d, d] fp32, one per sequence (a W0 shared
  *                  over the batch receives the sum over B).
  *   flags          0, or TTT_FLAG_FORCE_SIMT.
- * io_dtype BF16 with d = 64 and b = 16 runs on the tensor cores (mma.sync,
- * bf16 operands, fp32 accumulation; the state gradient is carried in fp32);
- * every other case, or TTT_FLAG_FORCE_SIMT, on the fp32 CUDA-core kernel.
- * One CTA per (sequence, head) unit.
+ *   use_ln         1: the LN+residual model (ttt_linear_forward's use_ln);
+ *                  then also
+ *     c_states       [B, H, T/b, d] fp32 from the forward,
+ *     ln_gamma, ln_beta, ln_eps   the forward's LN parameters,
+ *     dc_out         [B, H, d] fp32 dL/dc_out, or NULL for zero,
+ *     dc0, dgamma, dbeta   outputs [B, H, d] fp32: dL/dc0, dL/dgamma and
+ *                  dL/dbeta per (sequence, head) unit (sum what is shared).
+ * Plain: io_dtype BF16 with d = 64 and b = 16 runs on the tensor cores
+ * (mma.sync, bf16 operands, fp32 accumulation; the state gradient is carried
+ * in fp32); every other case, TTT_FLAG_FORCE_SIMT, or use_ln, on the fp32
+ * CUDA-core kernels (LN: b <= 32 at d = 64).  One CTA per (sequence, head)
+ * unit.
  */
 typedef struct {
     int B, H, T, d, b;
@@ -175,6 +185,15 @@ typedef struct {
     float* deta;
     float* dW0;
     unsigned flags;
+    int use_ln;
+    const float* c_states;
+    const float* ln_gamma;
+    const float* ln_beta;
+    float ln_eps;
+    const float* dc_out;
+    float* dc0;
+    float* dgamma;
+    float* dbeta;
 } ttt_linear_backward_args;
 
 ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_t stream);

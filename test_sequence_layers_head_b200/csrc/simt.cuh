@@ -40,6 +40,7 @@ struct SimtLinearParams {
     float* W_out;
     float* c_out;
     float* W_states;   // optional [units, T/b, D, D]: the state at the start of every mini-batch
+    float* c_states;   // LN, with W_states: [units, T/b, D], the bias at the start of every mini-batch
 };
 
 // Row statistics helper: LN over n features of row `row` (warp-cooperative).
@@ -92,6 +93,10 @@ __global__ void __launch_bounds__(kSimtThreads) simt_linear_kernel(SimtLinearPar
         if (p.W_states) {
             float* ws = p.W_states + ((size_t)unit * (p.T / b) + t0 / b) * D * D;
             for (int e = tid; e < D * D; e += kSimtThreads) ws[e] = W[e];
+            if (LN) {
+                float* cs = p.c_states + ((size_t)unit * (p.T / b) + t0 / b) * D;
+                for (int j = tid; j < D; j += kSimtThreads) cs[j] = c[j];
+            }
         }
         // load the mini-batch
         for (int e = tid; e < b * D; e += kSimtThreads) {

@@ -15,6 +15,7 @@
 #include "mlp_tc.cuh"
 #include "simt.cuh"
 #include "simt_backward.cuh"
+#include "simt_backward_ln.cuh"
 #include "mma_backward.cuh"
 #include "mma_forward.cuh"
 #include "tmap.h"
@@ -92,6 +93,7 @@ ttt_status launch_simt_linear(const ttt_linear_args* a, cudaStream_t st) {
     p.W_out = a->W_out;
     p.c_out = a->c_out;
     p.W_states = a->W_states;
+    p.c_states = a->c_states;
     const size_t smem = simt_linear_smem(D, a->b);
     auto k = simt_linear_kernel<D, LN, IO>;
     if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
@@ -205,10 +207,11 @@ extern "C" ttt_status ttt_linear_forward(const ttt_linear_args* a, cudaStream_t 
         return TTT_ERR_INVALID_ARG;
     if (a->W_states) {
         if (!aligned16(a->W_states)) return TTT_ERR_INVALID_ARG;
-        if (a->use_ln) return TTT_ERR_UNSUPPORTED;
+        if (a->use_ln && !ok_ptr(a->c_states)) return TTT_ERR_INVALID_ARG;
     }
+    const bool states_on_simt = a->W_states && a->use_ln;   // the LN states come from the fp32 kernel
     const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 && a->Z &&
-                    !(a->flags & TTT_FLAG_FORCE_SIMT);
+                    !(a->flags & TTT_FLAG_FORCE_SIMT) && !states_on_simt;
     if (tc && a->W_states) {
         // training: the mma.sync forward that also writes the batch-start states
         if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
@@ -415,6 +418,22 @@ extern "C" ttt_status ttt_mlp_decode_step(const ttt_mlp_decode_args* a, cudaStre
 namespace ttt {
 namespace {
 template <int D, typename IO>
+ttt_status launch_ln_backward_t(const ttt_linear_backward_args* a, cudaStream_t st) {
+    SimtLnBackwardParams p{a->H, a->T, a->b, a->Q, a->K, a->V, a->eta, a->eta_const, a->W_states, a->c_states,
+                           a->ln_gamma, a->ln_beta, a->ln_eps, a->dZ, a->dW_out, a->dc_out, a->dQ, a->dK, a->dV,
+                           a->deta, a->dW0, a->dc0, a->dgamma, a->dbeta};
+    const size_t smem = simt_ln_backward_smem(D, a->b);
+    auto k = simt_ln_backward_kernel<D, IO>;
+    if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
+    k<<<a->B * a->H, kSimtThreads, smem, st>>>(p);
+    return launch_status();
+}
+template <int D>
+ttt_status launch_ln_backward(const ttt_linear_backward_args* a, cudaStream_t st) {
+    return a->io_dtype == TTT_F32 ? launch_ln_backward_t<D, float>(a, st)
+                                  : launch_ln_backward_t<D, __nv_bfloat16>(a, st);
+}
+template <int D, typename IO>
 ttt_status launch_linear_backward_t(const ttt_linear_backward_args* a, cudaStream_t st) {
     SimtBackwardParams p{a->H, a->T, a->b, a->Q, a->K, a->V, a->eta, a->eta_const, a->W_states,
                          a->dZ, a->dW_out, a->dQ, a->dK, a->dV, a->deta, a->dW0};
@@ -444,6 +463,17 @@ extern "C" ttt_status ttt_linear_backward(const ttt_linear_backward_args* a, cud
     if (!ok_ptr(a->dW0) || !ok_opt(a->eta) || !ok_opt(a->dZ) || !ok_opt(a->dW_out) || !ok_opt(a->deta))
         return TTT_ERR_INVALID_ARG;
     if (a->flags & ~TTT_FLAG_FORCE_SIMT) return TTT_ERR_INVALID_ARG;
+    if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
+    if (a->use_ln) {
+        if ((a->T > 0 && !ok_ptr(a->c_states)) || !ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) ||
+            !(a->ln_eps > 0.f) || !ok_opt(a->dc_out) || !ok_ptr(a->dc0) || !ok_ptr(a->dgamma) || !ok_ptr(a->dbeta))
+            return TTT_ERR_INVALID_ARG;
+        switch (a->d) {
+            case 16: return launch_ln_backward<16>(a, stream);
+            case 32: return launch_ln_backward<32>(a, stream);
+            default: return launch_ln_backward<64>(a, stream);
+        }
+    }
     if (a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && !(a->flags & TTT_FLAG_FORCE_SIMT)) {
         SimtBackwardParams p{a->H, a->T, a->b, a->Q, a->K, a->V, a->eta, a->eta_const, a->W_states,
                              a->dZ, a->dW_out, a->dQ, a->dK, a->dV, a->deta, a->dW0};

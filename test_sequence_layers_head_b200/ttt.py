@@ -39,7 +39,7 @@ class LinearArgs(ctypes.Structure):
                 ("W0", _vp), ("W0_bstride", _ll), ("c0", _vp), ("c0_bstride", _ll),
                 ("use_ln", _i), ("ln_gamma", _vp), ("ln_beta", _vp), ("ln_eps", _f),
                 ("Z", _vp), ("W_out", _vp), ("c_out", _vp), ("flags", _u), ("wait_timeout_ms", _u),
-                ("W_states", _vp)]
+                ("W_states", _vp), ("c_states", _vp)]
 
 
 class MlpArgs(ctypes.Structure):
@@ -60,7 +60,9 @@ class DecodeArgs(ctypes.Structure):
 class BackwardArgs(ctypes.Structure):
     _fields_ = [("B", _i), ("H", _i), ("T", _i), ("d", _i), ("b", _i), ("io_dtype", _i), ("Q", _vp), ("K", _vp),
                 ("V", _vp), ("eta", _vp), ("eta_const", _f), ("W_states", _vp), ("dZ", _vp), ("dW_out", _vp),
-                ("dQ", _vp), ("dK", _vp), ("dV", _vp), ("deta", _vp), ("dW0", _vp), ("flags", _u)]
+                ("dQ", _vp), ("dK", _vp), ("dV", _vp), ("deta", _vp), ("dW0", _vp), ("flags", _u),
+                ("use_ln", _i), ("c_states", _vp), ("ln_gamma", _vp), ("ln_beta", _vp), ("ln_eps", _f),
+                ("dc_out", _vp), ("dc0", _vp), ("dgamma", _vp), ("dbeta", _vp)]
 
 
 class MlpDecodeArgs(ctypes.Structure):
@@ -147,14 +149,14 @@ def _check(code: int, what: str):
 
 def linear_forward(Q, K, V, eta, W0, b, *, eta_const=0.0, use_ln=False, c0=None, gamma=None, beta=None,
                    eps=1e-6, Z=None, W_out=None, c_out=None, flags=0, wait_timeout_ms=0, W_states=None,
-                   outputs=True, stream=None):
+                   c_states=None, outputs=True, stream=None):
     """TTT-Linear (optionally LN+residual) prefill; see ``ttt_linear_forward``.
 
     Q, K, V: [B,H,T,d] bf16 or fp32; eta: [B,H,T] fp32 or None (eta_const);
     W0: [H,d,d] (shared) or [B,H,d,d] fp32.  Returns (Z, W_out, c_out).
     W_states: optional [B,H,T/b,d,d] fp32 output, the state at every mini-batch
-    start (for ``linear_backward``).  outputs=False: Z is not computed (None is
-    returned), only the state.
+    start (for ``linear_backward``); with use_ln also c_states [B,H,T/b,d].
+    outputs=False: Z is not computed (None is returned), only the state.
     """
     B, H, T, d = Q.shape
     dev = Q.device
@@ -171,17 +173,21 @@ def linear_forward(Q, K, V, eta, W0, b, *, eta_const=0.0, use_ln=False, c0=None,
     a = LinearArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
                    _ptr(W0), W0_bstride, _ptr(c0), c0_bstride, int(bool(use_ln)), _ptr(gamma), _ptr(beta),
                    float(eps), _ptr(Z), _ptr(W_out), _ptr(c_out), int(flags), int(wait_timeout_ms),
-                   _ptr(W_states))
+                   _ptr(W_states), _ptr(c_states))
     _check(library().ttt_linear_forward(ctypes.byref(a), _stream(stream)), "ttt_linear_forward")
     return Z, W_out, c_out
 
 
 def linear_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW_out=None, eta_const=0.0, dQ=None, dK=None,
-                    dV=None, deta=None, dW0=None, flags=0, stream=None):
+                    dV=None, deta=None, dW0=None, flags=0, use_ln=False, c_states=None, gamma=None, beta=None,
+                    eps=1e-6, dc_out=None, stream=None):
     """Outer-loop gradients of the TTT-Linear prefill (no LN); see
     ``ttt_linear_backward``.  W_states [B,H,T/b,d,d] comes from
     ``linear_forward(..., W_states=...)`` on the same inputs.  Returns
-    (dQ, dK, dV, deta, dW0); deta is None when eta is None."""
+    (dQ, dK, dV, deta, dW0); deta is None when eta is None.  use_ln: the
+    LN+residual model (c_states from the forward, gamma, beta, eps, optional
+    dc_out); then returns (dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta), the last
+    three per unit [B,H,d]."""
     B, H, T, d = Q.shape
     dev = Q.device
     dQ = torch.empty_like(Q) if dQ is None else dQ
@@ -190,10 +196,17 @@ def linear_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW_out=None, eta_cons
     if deta is None and eta is not None:
         deta = torch.empty((B, H, T), device=dev, dtype=torch.float32)
     dW0 = torch.empty((B, H, d, d), device=dev, dtype=torch.float32) if dW0 is None else dW0
+    f32 = dict(device=dev, dtype=torch.float32)
+    dc0 = torch.empty((B, H, d), **f32) if use_ln else None
+    dgamma = torch.empty((B, H, d), **f32) if use_ln else None
+    dbeta = torch.empty((B, H, d), **f32) if use_ln else None
     a = BackwardArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
                      _ptr(W_states), _ptr(dZ), _ptr(dW_out), _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW0),
-                     int(flags))
+                     int(flags), int(bool(use_ln)), _ptr(c_states), _ptr(gamma), _ptr(beta), float(eps),
+                     _ptr(dc_out), _ptr(dc0), _ptr(dgamma), _ptr(dbeta))
     _check(library().ttt_linear_backward(ctypes.byref(a), _stream(stream)), "ttt_linear_backward")
+    if use_ln:
+        return dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta
     return dQ, dK, dV, deta, dW0
 
 

@@ -75,7 +75,7 @@ def test_linear_forward_w_states_rules(ttt_lib):
     a = _linear_args(ttt_lib, W_states=(1 << 20) + 4)    # misaligned
     assert L.ttt_linear_forward(ctypes.byref(a), None) == 1
     a = _linear_args(ttt_lib, W_states=1 << 20, use_ln=1, ln_gamma=1 << 20, ln_beta=1 << 20)
-    assert L.ttt_linear_forward(ctypes.byref(a), None) == 2   # states of the LN variant: not supported
+    assert L.ttt_linear_forward(ctypes.byref(a), None) == 1   # the LN variant needs c_states too
 
 
 def _backward_args(ttt, **kw):
@@ -102,6 +102,12 @@ def _backward_args(ttt, **kw):
     (dict(deta=(1 << 20) + 4), 1),
     (dict(B=0, Q=None), 0),
     (dict(flags=0x2), 1),
+    (dict(use_ln=2), 1),
+    (dict(use_ln=1), 1),                                       # no c_states / gamma / beta / outputs
+    (dict(use_ln=1, c_states=1 << 20, ln_gamma=1 << 20, ln_beta=1 << 20, ln_eps=1e-6, dc0=1 << 20,
+          dgamma=1 << 20, dbeta=(1 << 20) + 4), 1),            # misaligned dbeta
+    (dict(use_ln=1, c_states=1 << 20, ln_gamma=1 << 20, ln_beta=1 << 20, dc0=1 << 20, dgamma=1 << 20,
+          dbeta=1 << 20), 1),                                  # eps = 0
 ])
 def test_linear_backward_validation(ttt_lib, kw, code):
     a = _backward_args(ttt_lib, **kw)

@@ -197,3 +197,38 @@ def test_forward_with_states_equals_forward(ttt_lib):
     torch.cuda.synchronize()
     assert_close("Z", to_host(Z2), to_host(Z1), WL.BF16)
     assert_close("W_out", to_host(W2), to_host(W1), WL.BF16)
+
+
+@pytest.mark.parametrize("d,b,T,io", [(16, 16, 64, WL.F32), (32, 4, 32, WL.F32), (64, 16, 64, WL.BF16),
+                                      (16, 1, 8, WL.F32), (64, 32, 64, WL.F32)])
+def test_ln_backward_matches_oracle(ttt_lib, d, b, T, io):
+    """The LN+residual model: the fp32 forward writes W_states and c_states, the
+    backward returns dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta; all against the
+    oracle's reverse-mode gradients."""
+    B, H = 2, 3
+    inp = WL.random_case("ln", B, H, T, d, b, io_dtype=io, seed=3 * d + b + T)
+    r, e, w = inp.raw, inp.exact, inp.w
+    Q, K, V, eta, W0, c0, gam, bet = (to_dev(r[n]) for n in ("Q", "K", "V", "eta", "W0", "c0", "gamma", "beta"))
+    states = torch.full((B, H, T // b, d, d), float("nan"), device="cuda")
+    cst = torch.full((B, H, T // b, d), float("nan"), device="cuda")
+    ttt_lib.linear_forward(Q, K, V, eta, W0, b, use_ln=True, c0=c0, gamma=gam, beta=bet, eps=w.ln_eps,
+                           W_states=states, c_states=cst)
+    rng = np.random.default_rng(d + b)
+    dz = WL.store(rng.standard_normal((B, H, T, d)), io)
+    dw = WL.store(rng.standard_normal((B, H, d, d)), WL.F32)
+    dc = WL.store(rng.standard_normal((B, H, d)), WL.F32)
+    out = ttt_lib.linear_backward(Q, K, V, eta, states, b, dZ=to_dev(dz[0]), dW_out=to_dev(dw[0]), use_ln=True,
+                                  c_states=cst, gamma=gam, beta=bet, eps=w.ln_eps, dc_out=to_dev(dc[0]))
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    if T // b > 1:
+        t = b
+        _, Wo, co = O.linear_forward(e["Q"][:, :, :t], e["K"][:, :, :t], e["V"][:, :, :t], e["eta"][:, :, :t],
+                                     e["W0"], b, c0=e["c0"], gamma=e["gamma"], beta=e["beta"], use_ln=True,
+                                     eps=w.ln_eps)
+        assert_close("W_states[1]", to_host(states[:, :, 1]), Wo, WL.F32)
+        assert_close("c_states[1]", to_host(cst[:, :, 1]), co, WL.F32)
+    ref = O.linear_ln_backward(e["Q"], e["K"], e["V"], e["eta"], e["W0"], b, e["c0"], e["gamma"], e["beta"],
+                               eps=w.ln_eps, dZ=dz[1], dW_out=dw[1], dc_out=dc[1])
+    for name, g, o in zip(("dQ", "dK", "dV", "deta", "dW0", "dc0", "dgamma", "dbeta"), out, ref):
+        assert_close(name, to_host(g), o, io)
