@@ -387,6 +387,37 @@ def measure_backward(ttt, torch, threads, name="linear_B8_H12_T2048"):
             "kernel": "mma_linear_backward_kernel (mma.sync, bf16 operands, fp32 accumulation)"}
 
 
+def measure_ln_backward(ttt, torch, threads, T=2048):
+    """Outer-loop backward of the LN+residual TTT-Linear (fp32 CUDA-core kernels:
+    the forward writing W_states and c_states, then the backward) on the LN
+    workload's shapes at a shorter T (informational)."""
+    w = WL.scaled(WL.WORKLOADS["ln_B4_H32_T8192"], T=T)
+    _, dev = device_inputs(w, torch, threads)
+    B, H, d = w.B, w.H, w.d
+    nb = T // w.b
+    states = torch.empty((B, H, nb, d, d), device="cuda")
+    cst = torch.empty((B, H, nb, d), device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(4)
+    dZ = torch.randn(B, H, T, d, generator=g, device="cuda").to(dev["Q"].dtype)
+    dW = torch.randn(B, H, d, d, generator=g, device="cuda")
+    flush_buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")
+    ln = dict(use_ln=True, gamma=dev["gamma"], beta=dev["beta"], eps=w.ln_eps)
+
+    def fwd():
+        ttt.linear_forward(dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W0"], w.b, c0=dev["c0"], W_states=states,
+                           c_states=cst, **ln)
+
+    def bwd():
+        ttt.linear_backward(dev["Q"], dev["K"], dev["V"], dev["eta"], states, w.b, dZ=dZ, dW_out=dW, c_states=cst,
+                            **ln)
+    ms_f = statistics.median(time_launches(torch, fwd, 3, 1, flush=lambda: flush_buf.zero_()))
+    ms_b = statistics.median(time_launches(torch, bwd, 3, 1, flush=lambda: flush_buf.zero_()))
+    return {"workload": w.name + f" (T={T})", "forward_with_states_ms": ms_f, "backward_ms": ms_b,
+            "tokens_per_s_backward": tokens(w) / (ms_b / 1000.0),
+            "kernel": "simt_ln_backward_kernel (fp32 CUDA cores)"}
+
+
 def measure_mlp_ln(ttt, torch, threads, T=2048):
     """TTT-MLP with LN+residual on the output layer (fp32 CUDA-core kernel) on
     the MLP workload's shapes at a shorter T (informational)."""
@@ -640,6 +671,7 @@ def run_ours(args):
             line["rows"]["decode_mlp_B2_H32"] = measure_decode_variant(ttt, torch, "mlp", 2, 32)
             line["rows"]["backward_linear_B8_H12_T2048"] = measure_backward(ttt, torch, threads)
             line["rows"]["mlp_ln_B2_H32_T2048"] = measure_mlp_ln(ttt, torch, threads)
+            line["rows"]["backward_ln_B4_H32_T2048"] = measure_ln_backward(ttt, torch, threads)
         line["cpu_baseline"] = cpu_baseline(w)
     if dist is not None:
         dist.barrier()
