@@ -784,8 +784,8 @@ def run_b_sweep(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    # about 0.5 s of timed work on the default workload, so that the 100 ms clock samples cover it
-    ap.add_argument("--steps", type=int, default=300)
+    # about 0.2 s of timed work on the default workload, so that the 100 ms clock samples see the load
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WL.WORKLOAD_ORDER)
