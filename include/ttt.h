@@ -216,7 +216,8 @@ ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_
  *                  TTT-MLP takes in practice),
  *                  f(x) = x + ln_gamma * LN(GELU(x W1 + c1) W2 + c2) + ln_beta,
  *                  LN as in ttt_linear_forward (ln_gamma, ln_beta [H, d] fp32,
- *                  ln_eps > 0).  Runs on the fp32 CUDA-core kernel.  0: plain.
+ *                  ln_eps > 0).  Same kernel choice as the plain model.
+ *                  0: plain.
  */
 typedef struct {
     int B, H, T, d, b;

@@ -113,6 +113,10 @@ struct Params {
     int* status;
     unsigned long long wait_ns;
     unsigned flags;
+    // LN+residual on the output layer (template LN): gamma, beta [H, 64]
+    const float* gamma;
+    const float* beta;
+    float eps;
 };
 
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b_x16(taddr, r); }
@@ -193,6 +197,7 @@ __device__ __forceinline__ void tril_product(uint32_t xbase, uint32_t ybase, int
     }
 }
 
+template <bool LN>
 __global__ void __launch_bounds__(kThreads, 1)
     mlp_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, Params p) {
@@ -413,6 +418,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         // hidden rows in the accumulator layout: 128 tt + 32 qd + 16 m + r + 8 hh
         auto hrow = [&](int tt, int m, int hh) { return 128 * tt + 32 * qd + 16 * m + r + 8 * hh; };
         float c1[2][2][2], c2f[2] = {0.f, 0.f};  // c1 of rows hrow(tt, m, hh); c2 of rows 16 qd + r + 8 hh
+        // LN: gamma, beta of rows 16 qd + r + 8 hh (accumulator layout) and of feature j (output
+        // layout); the Q values of the finished mini-batch's output tokens 8 hf .. + 7 at feature j
+        float lg[2] = {0.f, 0.f}, lb[2] = {0.f, 0.f}, lgz = 0.f, lbz = 0.f;
+        uint32_t qz[4] = {0u, 0u, 0u, 0u};
+        if (LN) {
+            const int hd = unit % p.H;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                lg[hh] = p.gamma[(size_t)hd * kD + 16 * qd + r + 8 * hh];
+                lb[hh] = p.beta[(size_t)hd * kD + 16 * qd + r + 8 * hh];
+            }
+            lgz = p.gamma[(size_t)hd * kD + j];
+            lbz = p.beta[(size_t)hd * kD + j];
+        }
         // bf16 [t][h] tile (four 128B-swizzled sub-tiles of 64 hidden rows) from the accumulator
         // layout: x[tt][m][hh] = pair of tokens (2c, 2c+1) of row hrow(tt, m, hh)
         auto stsm_rows = [&](uint32_t base, const uint32_t (&x)[2][2][2]) {
@@ -502,21 +521,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         };
-        float zc2 = 0.f;   // c2 of feature j before the batch's update (the Z bias; the updates
-                           // within the batch are the "+1" of tril(Hq Hk^T + 1) in S5)
-        // E5 of batch i2: Z = Z0 + c2 -> global, this warp's 8 tokens
-        auto finish_z = [&](int i2, float zc) {
-            WT(d_z, i2 & 1);
-            tc_fence_after();
-            uint32_t rz[8];
-            tmem_ld_32x32b_x8(tl + cZ + 8 * hf, rz);
-            tmem_wait_ld();
-            if (jl && !dead) {
-#pragma unroll
-                for (int t = 0; t < 8; ++t)
-                    Zu[(size_t)(i2 * kTok + 8 * hf + t) * kD] = __float2bfloat16_rn(__uint_as_float(rz[t]) + zc);
-            }
-        };
         int nx = 0;   // exchanges of partial sums so far (two alternating buffers)
         // the other token half's partial sums of this warp's rows: a[k] += other's
         auto exchange2 = [&](float* a, int n) {
@@ -528,6 +532,92 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float2 o = buf[((1 - hf) * 4 + qd) * 128 + (k >> 1) * 32 + lane];
                 a[k] += o.x;
                 a[k + 1] += o.y;
+            }
+        };
+        // LN: per-token sums over the 64 features (the four quadrant warps of this token half);
+        // same buffers and barrier as exchange2, so every epilogue warp calls it at the same points.
+        // Accumulator layout: v[tok][q] for the thread's tokens 2c, 2c+1 and two quantities.
+        auto ln_sum_acc = [&](float (&v)[2][2]) {
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1)
+#pragma unroll
+                for (int a = 0; a < 2; ++a)
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) v[a][b] += __shfl_xor_sync(0xffffffffu, v[a][b], o);
+            float* buf = reinterpret_cast<float*>(xch + (nx & 1) * 1024);
+            ++nx;
+            if (lane < 4)
+                *reinterpret_cast<float4*>(buf + ((hf * 4 + qd) * 4 + c) * 4) = make_float4(v[0][0], v[0][1], v[1][0], v[1][1]);
+            named_bar_sync(2, 256);
+            float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4) {
+                const float4 x = *reinterpret_cast<const float4*>(buf + ((hf * 4 + w4) * 4 + c) * 4);
+                t4.x += x.x; t4.y += x.y; t4.z += x.z; t4.w += x.w;
+            }
+            v[0][0] = t4.x; v[0][1] = t4.y; v[1][0] = t4.z; v[1][1] = t4.w;
+        };
+        // output layout (lane = feature j for lane < 16, tokens 8 hf + t): v[t][q], 16 values
+        auto ln_sum_out = [&](float (&v)[8][2]) {
+#pragma unroll
+            for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+#pragma unroll
+                    for (int b = 0; b < 2; ++b) v[t][b] += __shfl_xor_sync(0xffffffffu, v[t][b], o);
+            float* buf = reinterpret_cast<float*>(xch + (nx & 1) * 1024);
+            ++nx;
+            if (lane == 0) {
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    *reinterpret_cast<float2*>(buf + (hf * 4 + qd) * 16 + 2 * t) = make_float2(v[t][0], v[t][1]);
+            }
+            named_bar_sync(2, 256);
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                float a = 0.f, b = 0.f;
+#pragma unroll
+                for (int w4 = 0; w4 < 4; ++w4) {
+                    const float2 x = *reinterpret_cast<const float2*>(buf + (hf * 4 + w4) * 16 + 2 * t);
+                    a += x.x;
+                    b += x.y;
+                }
+                v[t][0] = a;
+                v[t][1] = b;
+            }
+        };
+        float zc2 = 0.f;   // c2 of feature j before the batch's update (the Z bias; the updates
+                           // within the batch are the "+1" of tril(Hq Hk^T + 1) in S5)
+        // E5 of batch i2: Z = Z0 + c2 -> global, this warp's 8 tokens
+        auto finish_z = [&](int i2, float zc) {
+            WT(d_z, i2 & 1);
+            tc_fence_after();
+            uint32_t rz[8];
+            tmem_ld_32x32b_x8(tl + cZ + 8 * hf, rz);
+            tmem_wait_ld();
+            float zv[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) zv[t] = __uint_as_float(rz[t]) + zc;
+            if (LN) {
+                // Z = Q + gamma LN(pre) + beta over the 64 features of each token
+                float sm2[8][2];
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    sm2[t][0] = jl ? zv[t] : 0.f;
+                    sm2[t][1] = jl ? zv[t] * zv[t] : 0.f;
+                }
+                ln_sum_out(sm2);
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    const float mu = sm2[t][0] * (1.f / kD);
+                    const float rs = rsqrtf(fmaxf(sm2[t][1] * (1.f / kD) - mu * mu, 0.f) + p.eps);
+                    const float q = (t & 1) ? bf16_hi(qz[t >> 1]) : bf16_lo(qz[t >> 1]);
+                    zv[t] = q + lgz * (zv[t] - mu) * rs + lbz;
+                }
+            }
+            if (jl && !dead) {
+#pragma unroll
+                for (int t = 0; t < 8; ++t) Zu[(size_t)(i2 * kTok + 8 * hf + t) * kD] = __float2bfloat16_rn(zv[t]);
             }
         };
         for (int i = 0; i < nsteps; ++i) {
@@ -610,11 +700,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ldsm_x2_tr(vt + t8 * 128 + (((2 * qd + ((lane >> 3) & 1)) ^ (t8 & 7)) << 4), v);
                 const float etc[2] = {et2[0], et2[1]};
                 float ev[4], ae[4];
+                if (!LN) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    ev[e] = e0[e] + c2f[e >> 1] - frag_at(v, 0, e);
-                    ae[e] = -etc[e & 1] * ev[e];
+                    for (int e = 0; e < 4; ++e) ev[e] = e0[e] + c2f[e >> 1] - frag_at(v, 0, e);
+                } else {
+                    // y = E0 + c2; f = k + gamma LN(y) + beta; ev becomes the LN+residual backward
+                    uint32_t kv[2];
+                    ldsm_x2_tr(smem_u32(st + kOffK) + t8 * 128 + (((2 * qd + ((lane >> 3) & 1)) ^ (t8 & 7)) << 4), kv);
+                    float y[4], s1[2][2];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) y[e] = e0[e] + c2f[e >> 1];
+#pragma unroll
+                    for (int tk = 0; tk < 2; ++tk) {
+                        s1[tk][0] = y[tk] + y[tk + 2];
+                        s1[tk][1] = y[tk] * y[tk] + y[tk + 2] * y[tk + 2];
+                    }
+                    ln_sum_acc(s1);
+                    float mu[2], rs[2], xh[4], g[4], s2[2][2];
+#pragma unroll
+                    for (int tk = 0; tk < 2; ++tk) {
+                        mu[tk] = s1[tk][0] * (1.f / kD);
+                        rs[tk] = rsqrtf(fmaxf(s1[tk][1] * (1.f / kD) - mu[tk] * mu[tk], 0.f) + p.eps);
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int tk = e & 1, hh = e >> 1;
+                        xh[e] = (y[e] - mu[tk]) * rs[tk];
+                        g[e] = lg[hh] * (frag_at(kv, 0, e) + lg[hh] * xh[e] + lb[hh] - frag_at(v, 0, e));
+                    }
+#pragma unroll
+                    for (int tk = 0; tk < 2; ++tk) {
+                        s2[tk][0] = g[tk] + g[tk + 2];
+                        s2[tk][1] = g[tk] * xh[tk] + g[tk + 2] * xh[tk + 2];
+                    }
+                    ln_sum_acc(s2);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int tk = e & 1;
+                        ev[e] = rs[tk] * (g[e] - s2[tk][0] * (1.f / kD) - xh[e] * s2[tk][1] * (1.f / kD));
+                    }
                 }
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ae[e] = -etc[e & 1] * ev[e];
                 stsm_x2_tr(smem_u32(es) + t8 * 128 + (((2 * qd + ((lane >> 3) & 1)) ^ (t8 & 7)) << 4),
                            pack_bf16x2(ev[0], ev[1]), pack_bf16x2(ev[2], ev[3]));
 #pragma unroll
@@ -640,6 +767,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // the previous batch's outputs go out first (its bias is zc2), then keep this one's
                 if (i >= 1) finish_z(i - 1, zc2);
                 zc2 = zc_now;
+                if (LN) {
+                    // Q of this mini-batch at feature j, tokens 8 hf .. + 7 (for its output LN)
+#pragma unroll
+                    for (int t = 0; t < 8; t += 2) {
+                        const float q0 = ld_bf16(st + kOffQ, sw128_off(8 * hf + t, j));
+                        const float q1 = ld_bf16(st + kOffQ, sw128_off(8 * hf + t + 1, j));
+                        qz[t >> 1] = pack_bf16x2(q0, q1);
+                    }
+                }
             }
             fence_proxy_async_smem();
             tc_fence_before();

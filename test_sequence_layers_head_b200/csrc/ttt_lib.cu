@@ -301,9 +301,13 @@ ttt_status tc_mlp(const ttt_mlp_args* a, cudaStream_t st) {
     p.status = status_ptr();
     p.wait_ns = wait_ns(a->wait_timeout_ms);
     p.flags = a->flags;
+    p.gamma = a->ln_gamma;
+    p.beta = a->ln_beta;
+    p.eps = a->ln_eps;
     if (!p.status) return TTT_ERR_CUDA;
-    if (!set_smem(mlp_tc_kernel, kSmemBytes)) return TTT_ERR_CUDA;
-    mlp_tc_kernel<<<(int)U, kThreads, kSmemBytes, st>>>(mQ, mK, mV, p);
+    auto k = a->use_ln ? mlp_tc_kernel<true> : mlp_tc_kernel<false>;
+    if (!set_smem(k, kSmemBytes)) return TTT_ERR_CUDA;
+    k<<<(int)U, kThreads, kSmemBytes, st>>>(mQ, mK, mV, p);
     return launch_status();
 }
 }  // namespace
@@ -325,7 +329,7 @@ extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream
     if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL)) return TTT_ERR_INVALID_ARG;
     if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
     if (a->use_ln && (!ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !(a->ln_eps > 0.f))) return TTT_ERR_INVALID_ARG;
-    const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 && !a->use_ln &&
+    const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
                     !(a->flags & TTT_FLAG_FORCE_SIMT);
     if (tc) return tc_mlp(a, stream);
     if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;

@@ -255,6 +255,30 @@ def test_mlp_ln_matches_oracle(ttt_lib, d, b, T, io):
         assert_close(name, to_host(g), o, io)
 
 
+@pytest.mark.parametrize("B,H,T,eta_mode", [(2, 4, 256, "sigmoid"), (1, 3, 48, "const"), (3, 1, 16, "sigmoid")])
+def test_mlp_ln_tensor_core(ttt_lib, B, H, T, eta_mode):
+    """bf16, d = 64, b = 16 with LN+residual runs on the tensor-core MLP kernel:
+    against the oracle, and against the fp32 CUDA-core kernel on the same inputs."""
+    d, b = 64, 16
+    inp = WL.random_case("mlp", B, H, T, d, b, io_dtype=WL.BF16, eta_mode=eta_mode, eta_const=1 / 64,
+                         seed=5 * T + H)
+    rng = np.random.default_rng(T + B)
+    gr, ge = WL.store(1 + rng.standard_normal((H, d)) * 0.14, WL.F32)
+    br, be = WL.store(rng.standard_normal((H, d)) * 0.14, WL.F32)
+    r, e = inp.raw, inp.exact
+    dev = {k: to_dev(r[k]) for k in ("Q", "K", "V", "eta", "W1", "c1", "W2", "c2")}
+    args = (dev["Q"], dev["K"], dev["V"], dev["eta"], dev["W1"], dev["c1"], dev["W2"], dev["c2"], b)
+    tc = ttt_lib.mlp_forward(*args, Z=poison_like(dev["Q"]), use_ln=True, gamma=to_dev(gr), beta=to_dev(br))
+    ft = ttt_lib.mlp_forward(*args, use_ln=True, gamma=to_dev(gr), beta=to_dev(br), flags=ttt_lib.FLAG_FORCE_SIMT)
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    ref = O.mlp_forward(e["Q"], e["K"], e["V"], e["eta"], e["W1"], e["c1"], e["W2"], e["c2"], b, use_ln=True,
+                        gamma=ge, beta=be)
+    for name, g, f, o in zip(("Z", "W1", "c1", "W2", "c2"), tc, ft, ref):
+        assert_close(name, to_host(g), o, WL.BF16)
+        assert normwise(to_host(g), to_host(f)) < 1e-2, name
+
+
 def test_mlp_tc_matches_simt(ttt_lib):
     """The tensor-core and the fp32 CUDA-core MLP kernels agree on the same inputs."""
     inp = WL.random_case("mlp", 1, 3, 96, 64, 16, io_dtype=WL.BF16, eta_mode="const", eta_const=1 / 64, seed=41)
