@@ -16,17 +16,22 @@ from tests.gpu_util import assert_close, to_dev, to_host
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("kind", ["linear", "ln", "mlp"])
+@pytest.mark.parametrize("kind", ["linear", "ln", "mlp", "mlp_ln"])
 def test_stalled_wait_reports_timeout_and_context_survives(ttt_lib, kind):
-    inp = WL.random_case(kind, 1, 3, 128, 64, 16, eta_mode="const" if kind == "mlp" else "sigmoid",
+    mlp = kind.startswith("mlp")
+    inp = WL.random_case("mlp" if mlp else kind, 1, 3, 128, 64, 16, eta_mode="const" if mlp else "sigmoid",
                          eta_const=1 / 64, seed=71)
     d = {k: to_dev(v) for k, v in inp.raw.items()}
+    rng = np.random.default_rng(72)
+    gr, ge = WL.store(1 + rng.standard_normal((3, 64)) * 0.14, WL.F32)
+    br, be = WL.store(rng.standard_normal((3, 64)) * 0.14, WL.F32)
+    mln = dict(use_ln=True, gamma=to_dev(gr), beta=to_dev(br)) if kind == "mlp_ln" else {}
     assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
 
     def run(flags):
-        if kind == "mlp":
+        if mlp:
             return ttt_lib.mlp_forward(d["Q"], d["K"], d["V"], d["eta"], d["W1"], d["c1"], d["W2"], d["c2"], 16,
-                                       flags=flags, wait_timeout_ms=300)
+                                       flags=flags, wait_timeout_ms=300, **mln)
         ln = kind == "ln"
         kw = dict(c0=d["c0"], gamma=d["gamma"], beta=d["beta"]) if ln else {}
         return ttt_lib.linear_forward(d["Q"], d["K"], d["V"], d["eta"], d["W0"], 16, use_ln=ln, flags=flags,
@@ -39,8 +44,9 @@ def test_stalled_wait_reports_timeout_and_context_survives(ttt_lib, kind):
     torch.cuda.synchronize()
     assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
     e = inp.exact
-    if kind == "mlp":
-        ref = O.mlp_forward(e["Q"], e["K"], e["V"], e["eta"], e["W1"], e["c1"], e["W2"], e["c2"], 16)
+    if mlp:
+        kw = dict(use_ln=True, gamma=ge, beta=be) if kind == "mlp_ln" else {}
+        ref = O.mlp_forward(e["Q"], e["K"], e["V"], e["eta"], e["W1"], e["c1"], e["W2"], e["c2"], 16, **kw)
     else:
         ln = kind == "ln"
         kw = dict(c0=e["c0"], gamma=e["gamma"], beta=e["beta"]) if ln else {}
