@@ -41,6 +41,9 @@ def lib():
         L.ttt_oracle_linear_ln_backward.argtypes = [i, i, i, i, i, P, P, P, P, P, ll, P, ll, P, P, dbl, P, P, P,
                                                     P, P, P, P, P, P, P, P, i]
         L.ttt_oracle_linear_ln_backward.restype = i
+        L.ttt_oracle_mlp_backward.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, ll, P, P, P, P, P,
+                                              P, P, P, P, P, P, P, P, i]
+        L.ttt_oracle_mlp_backward.restype = i
         _lib = L
     return _lib
 
@@ -166,3 +169,27 @@ def linear_ln_backward(Q, K, V, eta, W0, b, c0, gamma, beta, eps=1e-6, dZ=None, 
     if rc != 0:
         raise ValueError("oracle: invalid arguments")
     return dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta
+
+
+def mlp_backward(Q, K, V, eta, W1, c1, W2, c2, b, dZ=None, dW1_out=None, dc1_out=None, dW2_out=None,
+                 dc2_out=None, threads=None):
+    """Outer-loop gradients of the TTT-MLP forward (no LN), reverse mode through
+    the primal loop.  Parameters [H,...] (shared) or [B,H,...].  Returns
+    (dQ, dK, dV, deta, dW1, dc1, dW2, dc2), the parameter gradients per unit
+    [B,H,...] (sum over B for shared parameters)."""
+    Q, K, V, eta, W1, c1, W2, c2 = map(_f64, (Q, K, V, eta, W1, c1, W2, c2))
+    dZ, dW1_out, dc1_out, dW2_out, dc2_out = map(_f64, (dZ, dW1_out, dc1_out, dW2_out, dc2_out))
+    B, H, T, d = Q.shape
+    m = W1.shape[-1]
+    per_seq = 1 if W1.ndim == 4 else 0
+    dQ, dK, dV = np.empty((B, H, T, d)), np.empty((B, H, T, d)), np.empty((B, H, T, d))
+    deta = np.empty((B, H, T))
+    dW1, dc1 = np.empty((B, H, d, m)), np.empty((B, H, m))
+    dW2, dc2 = np.empty((B, H, m, d)), np.empty((B, H, d))
+    rc = lib().ttt_oracle_mlp_backward(B, H, T, d, m, b, _p(Q), _p(K), _p(V), _p(eta), _p(W1), _p(c1), _p(W2),
+                                       _p(c2), per_seq, _p(dZ), _p(dW1_out), _p(dc1_out), _p(dW2_out),
+                                       _p(dc2_out), _p(dQ), _p(dK), _p(dV), _p(deta), _p(dW1), _p(dc1), _p(dW2),
+                                       _p(dc2), threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: invalid arguments")
+    return dQ, dK, dV, deta, dW1, dc1, dW2, dc2

@@ -35,8 +35,9 @@
  *     projections, the initial state and the learning-rate parameters with
  *     gradients that pass through the inner loop's updates):
  *     the backward of the TTT-Linear forward, plain and LN+residual (there
- *     also the initial bias and the LN parameters), is reverse-mode
- *     differentiation of the same primal loop, token by token.
+ *     also the initial bias and the LN parameters), and of the TTT-MLP
+ *     forward, is reverse-mode differentiation of the same primal loop,
+ *     token by token.
  *
  * Readings of points the pages leave open (each one is listed in the design
  * notes of the repository):
@@ -717,5 +718,228 @@ int ttt_oracle_linear_ln_backward(int B, int H, int T, int d, int b, const doubl
                                 dQ + tok, dK + tok, dV + tok, deta + (size_t)u * T, dW0 + (size_t)u * d * d,
                                 dc0 + (size_t)u * d, dgamma + (size_t)u * d, dbeta + (size_t)u * d);
     }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Backward of the TTT-MLP forward (no LN): reverse-mode differentiation of
+ * the primal loop, token by token.  Returns dQ, dK, dV, deta and the
+ * gradients of the initial parameters dW1, dc1, dW2, dc2 (per unit).
+ *
+ * Forward of token t with batch-start (W1s, c1s, W2s, c2s) and running state:
+ *   a = k W1s + c1s,  h = GELU(a),  e = h W2s + c2s - v
+ *   m = e W2s^T,  d1 = m * GELU'(a)
+ *   W1 -= eta k^T d1,  c1 -= eta d1,  W2 -= eta h^T e,  c2 -= eta e
+ *   aq = q W1_t + c1_t,  hq = GELU(aq),  z = hq W2_t + c2_t
+ * GELU''(x) = phi(x) (2 - x^2), the derivative of Phi(x) + x phi(x).
+ * ------------------------------------------------------------------------- */
+static double gelu_grad2(double x) { return exp(-0.5 * x * x) / sqrt(2.0 * M_PI) * (2.0 - x * x); }
+
+static void mlp_unit_backward(int T, int d, int m, int b, const double *Q, const double *K, const double *V,
+                              const double *eta, const double *W1_0, const double *c1_0, const double *W2_0,
+                              const double *c2_0, const double *dZ, const double *dW1o, const double *dc1o,
+                              const double *dW2o, const double *dc2o, double *dQ, double *dK, double *dV,
+                              double *deta, double *dW1, double *dc1, double *dW2, double *dc2) {
+    const size_t n1 = (size_t)d * m;
+    const int nb = (T + b - 1) / b;
+    const size_t sz = n1 + m + n1 + d;   /* one state: W1, c1, W2, c2 */
+    double *starts = malloc((size_t)(nb > 0 ? nb : 1) * sz * sizeof(double));
+    double *run = malloc((size_t)(b + 1) * sz * sizeof(double));   /* running states of a batch */
+    double *cur = malloc(sz * sizeof(double));
+    double *D = malloc(sz * sizeof(double)), *Ds = malloc(sz * sizeof(double));   /* adjoints */
+    double *A = malloc((size_t)b * m * sizeof(double)), *Hh = malloc((size_t)b * m * sizeof(double));
+    double *E = malloc((size_t)b * d * sizeof(double)), *Mm = malloc((size_t)b * m * sizeof(double));
+    double *D1 = malloc((size_t)b * m * sizeof(double));
+    double *aq = malloc(m * sizeof(double)), *hq = malloc(m * sizeof(double)), *dhq = malloc(m * sizeof(double));
+    double *dd1 = malloc(m * sizeof(double)), *dmv = malloc(m * sizeof(double)), *dh = malloc(m * sizeof(double));
+    double *da = malloc(m * sizeof(double)), *de = malloc(d * sizeof(double));
+    #define W1P(x) (x)
+    #define C1P(x) ((x) + n1)
+    #define W2P(x) ((x) + n1 + m)
+    #define C2P(x) ((x) + n1 + m + n1)
+
+    /* batch quantities at the batch-start state S, row i = token t */
+    #define BATCH_FWD(t, i, S)                                                                         \
+        do {                                                                                           \
+            const double *k_ = K + (size_t)(t) * d, *v_ = V + (size_t)(t) * d;                         \
+            double *a_ = A + (size_t)(i) * m, *h_ = Hh + (size_t)(i) * m, *e_ = E + (size_t)(i) * d;   \
+            vec_mat(d, m, k_, W1P(S), a_);                                                             \
+            for (int p = 0; p < m; ++p) { a_[p] += C1P(S)[p]; h_[p] = gelu(a_[p]); }                   \
+            vec_mat(m, d, h_, W2P(S), e_);                                                             \
+            for (int j = 0; j < d; ++j) e_[j] += C2P(S)[j] - v_[j];                                    \
+            for (int p = 0; p < m; ++p) {                                                              \
+                double acc = 0.0;                                                                      \
+                for (int j = 0; j < d; ++j) acc += W2P(S)[(size_t)p * d + j] * e_[j];                  \
+                Mm[(size_t)(i) * m + p] = acc;                                                         \
+                D1[(size_t)(i) * m + p] = acc * gelu_grad(a_[p]);                                      \
+            }                                                                                          \
+        } while (0)
+    /* one token's update applied to state X (in place) */
+    #define TOKEN_UPD(t, i, X)                                                                         \
+        do {                                                                                           \
+            const double *k_ = K + (size_t)(t) * d, et_ = eta[t];                                      \
+            const double *d1_ = D1 + (size_t)(i) * m, *h_ = Hh + (size_t)(i) * m, *e_ = E + (size_t)(i) * d; \
+            for (int a2 = 0; a2 < d; ++a2)                                                             \
+                for (int p = 0; p < m; ++p) W1P(X)[(size_t)a2 * m + p] -= et_ * k_[a2] * d1_[p];       \
+            for (int p = 0; p < m; ++p) C1P(X)[p] -= et_ * d1_[p];                                     \
+            for (int p = 0; p < m; ++p)                                                                \
+                for (int j = 0; j < d; ++j) W2P(X)[(size_t)p * d + j] -= et_ * h_[p] * e_[j];          \
+            for (int j = 0; j < d; ++j) C2P(X)[j] -= et_ * e_[j];                                      \
+        } while (0)
+
+    memcpy(W1P(cur), W1_0, n1 * sizeof(double));
+    if (c1_0) memcpy(C1P(cur), c1_0, m * sizeof(double)); else memset(C1P(cur), 0, m * sizeof(double));
+    memcpy(W2P(cur), W2_0, n1 * sizeof(double));
+    if (c2_0) memcpy(C2P(cur), c2_0, d * sizeof(double)); else memset(C2P(cur), 0, d * sizeof(double));
+    for (int i = 0; i < nb; ++i) {
+        const int t0 = i * b, t1_ = (t0 + b < T) ? t0 + b : T;
+        memcpy(starts + (size_t)i * sz, cur, sz * sizeof(double));
+        for (int t = t0; t < t1_; ++t) BATCH_FWD(t, t - t0, starts + (size_t)i * sz);
+        for (int t = t0; t < t1_; ++t) TOKEN_UPD(t, t - t0, cur);
+    }
+    /* adjoint of the final state */
+    memset(D, 0, sz * sizeof(double));
+    if (dW1o) memcpy(W1P(D), dW1o, n1 * sizeof(double));
+    if (dc1o) memcpy(C1P(D), dc1o, m * sizeof(double));
+    if (dW2o) memcpy(W2P(D), dW2o, n1 * sizeof(double));
+    if (dc2o) memcpy(C2P(D), dc2o, d * sizeof(double));
+    for (int i = nb - 1; i >= 0; --i) {
+        const int t0 = i * b, t1_ = (t0 + b < T) ? t0 + b : T;
+        const double *S = starts + (size_t)i * sz;
+        for (int t = t0; t < t1_; ++t) BATCH_FWD(t, t - t0, S);
+        memcpy(run, S, sz * sizeof(double));
+        for (int t = t0; t < t1_; ++t) {
+            memcpy(run + (size_t)(t - t0 + 1) * sz, run + (size_t)(t - t0) * sz, sz * sizeof(double));
+            TOKEN_UPD(t, t - t0, run + (size_t)(t - t0 + 1) * sz);
+        }
+        memset(Ds, 0, sz * sizeof(double));
+        for (int t = t1_ - 1; t >= t0; --t) {
+            const int li = t - t0;
+            const double *q = Q + (size_t)t * d, *k = K + (size_t)t * d;
+            const double *Rt = run + (size_t)(li + 1) * sz;   /* state after token t */
+            const double *a = A + (size_t)li * m, *h = Hh + (size_t)li * m, *e = E + (size_t)li * d;
+            const double *mm = Mm + (size_t)li * m, *d1 = D1 + (size_t)li * m;
+            double *dq = dQ + (size_t)t * d, *dk = dK + (size_t)t * d, *dv = dV + (size_t)t * d;
+            for (int j = 0; j < d; ++j) { dq[j] = 0.0; dk[j] = 0.0; }
+            /* z = GELU(q W1_t + c1_t) W2_t + c2_t */
+            if (dZ) {
+                const double *dz = dZ + (size_t)t * d;
+                vec_mat(d, m, q, W1P(Rt), aq);
+                for (int p = 0; p < m; ++p) { aq[p] += C1P(Rt)[p]; hq[p] = gelu(aq[p]); }
+                for (int p = 0; p < m; ++p) {
+                    double acc = 0.0;
+                    for (int j = 0; j < d; ++j) acc += dz[j] * W2P(Rt)[(size_t)p * d + j];
+                    dhq[p] = acc * gelu_grad(aq[p]);   /* d(aq) */
+                }
+                for (int p = 0; p < m; ++p)
+                    for (int j = 0; j < d; ++j) W2P(D)[(size_t)p * d + j] += hq[p] * dz[j];
+                for (int j = 0; j < d; ++j) C2P(D)[j] += dz[j];
+                for (int a2 = 0; a2 < d; ++a2) {
+                    double acc = 0.0;
+                    for (int p = 0; p < m; ++p) acc += dhq[p] * W1P(Rt)[(size_t)a2 * m + p];
+                    dq[a2] += acc;
+                }
+                for (int a2 = 0; a2 < d; ++a2)
+                    for (int p = 0; p < m; ++p) W1P(D)[(size_t)a2 * m + p] += q[a2] * dhq[p];
+                for (int p = 0; p < m; ++p) C1P(D)[p] += dhq[p];
+            }
+            /* the token's update: W1 -= eta k^T d1, c1 -= eta d1, W2 -= eta h^T e, c2 -= eta e */
+            double g = 0.0;
+            for (int p = 0; p < m; ++p) {
+                double acc = C1P(D)[p];
+                for (int a2 = 0; a2 < d; ++a2) acc += k[a2] * W1P(D)[(size_t)a2 * m + p];
+                dd1[p] = -eta[t] * acc;
+                g += acc * d1[p];
+            }
+            for (int j = 0; j < d; ++j) {
+                double acc = C2P(D)[j];
+                for (int p = 0; p < m; ++p) acc += h[p] * W2P(D)[(size_t)p * d + j];
+                de[j] = -eta[t] * acc;
+                g += acc * e[j];
+            }
+            deta[t] = -g;
+            for (int a2 = 0; a2 < d; ++a2) {
+                double acc = 0.0;
+                for (int p = 0; p < m; ++p) acc += d1[p] * W1P(D)[(size_t)a2 * m + p];
+                dk[a2] += -eta[t] * acc;
+            }
+            for (int p = 0; p < m; ++p) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += e[j] * W2P(D)[(size_t)p * d + j];
+                dh[p] = -eta[t] * acc;
+            }
+            /* d1 = m * GELU'(a), m = e W2s^T */
+            for (int p = 0; p < m; ++p) {
+                dmv[p] = dd1[p] * gelu_grad(a[p]);
+                da[p] = dd1[p] * mm[p] * gelu_grad2(a[p]);
+            }
+            for (int j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int p = 0; p < m; ++p) acc += dmv[p] * W2P(S)[(size_t)p * d + j];
+                de[j] += acc;
+            }
+            for (int p = 0; p < m; ++p)
+                for (int j = 0; j < d; ++j) W2P(Ds)[(size_t)p * d + j] += dmv[p] * e[j];
+            /* e = h W2s + c2s - v */
+            for (int p = 0; p < m; ++p) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += de[j] * W2P(S)[(size_t)p * d + j];
+                dh[p] += acc;
+            }
+            for (int p = 0; p < m; ++p)
+                for (int j = 0; j < d; ++j) W2P(Ds)[(size_t)p * d + j] += h[p] * de[j];
+            for (int j = 0; j < d; ++j) { C2P(Ds)[j] += de[j]; dv[j] = -de[j]; }
+            /* h = GELU(a), a = k W1s + c1s */
+            for (int p = 0; p < m; ++p) da[p] += dh[p] * gelu_grad(a[p]);
+            for (int a2 = 0; a2 < d; ++a2) {
+                double acc = 0.0;
+                for (int p = 0; p < m; ++p) acc += da[p] * W1P(S)[(size_t)a2 * m + p];
+                dk[a2] += acc;
+            }
+            for (int a2 = 0; a2 < d; ++a2)
+                for (int p = 0; p < m; ++p) W1P(Ds)[(size_t)a2 * m + p] += k[a2] * da[p];
+            for (int p = 0; p < m; ++p) C1P(Ds)[p] += da[p];
+        }
+        for (size_t x = 0; x < sz; ++x) D[x] += Ds[x];
+    }
+    #undef BATCH_FWD
+    #undef TOKEN_UPD
+    memcpy(dW1, W1P(D), n1 * sizeof(double));
+    memcpy(dc1, C1P(D), m * sizeof(double));
+    memcpy(dW2, W2P(D), n1 * sizeof(double));
+    memcpy(dc2, C2P(D), d * sizeof(double));
+    #undef W1P
+    #undef C1P
+    #undef W2P
+    #undef C2P
+    free(starts); free(run); free(cur); free(D); free(Ds); free(A); free(Hh); free(E); free(Mm); free(D1);
+    free(aq); free(hq); free(dhq); free(dd1); free(dmv); free(dh); free(da); free(de);
+}
+
+int ttt_oracle_mlp_backward(int B, int H, int T, int d, int m, int b, const double *Q, const double *K,
+                            const double *V, const double *eta, const double *W1, const double *c1,
+                            const double *W2, const double *c2, long long p_bstride_scale, const double *dZ,
+                            const double *dW1o, const double *dc1o, const double *dW2o, const double *dc2o,
+                            double *dQ, double *dK, double *dV, double *deta, double *dW1, double *dc1,
+                            double *dW2, double *dc2, int nthreads) {
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || m <= 0 || b <= 0 || !Q || !K || !V || !eta || !W1 || !W2 ||
+        !dQ || !dK || !dV || !deta || !dW1 || !dc1 || !dW2 || !dc2)
+        return 1;
+    const long long units = (long long)B * H;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long long u = 0; u < units; ++u) {
+        const long long pu = p_bstride_scale ? u : (u % H);
+        const size_t tok = (size_t)u * T * d;
+        mlp_unit_backward(T, d, m, b, Q + tok, K + tok, V + tok, eta + (size_t)u * T, W1 + (size_t)pu * d * m,
+                          c1 ? c1 + (size_t)pu * m : NULL, W2 + (size_t)pu * m * d, c2 ? c2 + (size_t)pu * d : NULL,
+                          dZ ? dZ + tok : NULL, dW1o ? dW1o + (size_t)u * d * m : NULL,
+                          dc1o ? dc1o + (size_t)u * m : NULL, dW2o ? dW2o + (size_t)u * m * d : NULL,
+                          dc2o ? dc2o + (size_t)u * d : NULL, dQ + tok, dK + tok, dV + tok, deta + (size_t)u * T,
+                          dW1 + (size_t)u * d * m, dc1 + (size_t)u * m, dW2 + (size_t)u * m * d, dc2 + (size_t)u * d);
+    }
+    (void)nthreads;
     return 0;
 }

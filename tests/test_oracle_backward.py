@@ -136,3 +136,68 @@ def test_ln_backward_matches_finite_differences(B, H, T, d, b, shared):
             fd[idx] = (lp - lm) / (2 * h)
         err = np.max(np.abs(fd - gr)) / max(np.max(np.abs(fd)), 1e-12)
         assert err < 1e-6, (name, err)
+
+
+# ---------------------------------------------------------------------------
+# TTT-MLP, f(x) = GELU(x W1 + c1) W2 + c2 (section 4.4): the outer loop also
+# trains the initial parameters of both layers
+# ---------------------------------------------------------------------------
+
+def _mlp_case(B, H, T, d, m, shared, seed):
+    rng = np.random.default_rng(seed)
+    Q, K, V = (rng.standard_normal((B, H, T, d)) / np.sqrt(d) for _ in range(3))
+    eta = 0.2 + 0.3 * rng.random((B, H, T))
+    pre = (H,) if shared else (B, H)
+    W1 = rng.standard_normal(pre + (d, m)) / np.sqrt(d)
+    c1 = rng.standard_normal(pre + (m,)) * 0.2
+    W2 = rng.standard_normal(pre + (m, d)) / np.sqrt(m)
+    c2 = rng.standard_normal(pre + (d,)) * 0.2
+    up = [rng.standard_normal((B, H, T, d)), rng.standard_normal((B, H, d, m)), rng.standard_normal((B, H, m)),
+          rng.standard_normal((B, H, m, d)), rng.standard_normal((B, H, d))]
+    return Q, K, V, eta, W1, c1, W2, c2, up
+
+
+def _mlp_loss(Q, K, V, eta, W1, c1, W2, c2, b, up):
+    out = O.mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, threads=1)
+    return float(sum(np.sum(o * u) for o, u in zip(out, up)))
+
+
+@pytest.mark.parametrize("B,H,T,d,m,b,shared", [
+    (1, 2, 5, 2, 6, 2, True),     # ragged last mini-batch
+    (2, 1, 4, 3, 5, 2, False),    # per-sequence parameters
+    (1, 1, 4, 2, 4, 1, True),     # b = 1
+    (1, 1, 3, 3, 4, 3, True),     # one mini-batch
+])
+def test_mlp_backward_matches_finite_differences(B, H, T, d, m, b, shared):
+    Q, K, V, eta, W1, c1, W2, c2, up = _mlp_case(B, H, T, d, m, shared, seed=200 + 10 * T + d + m + b)
+    g = O.mlp_backward(Q, K, V, eta, W1, c1, W2, c2, b, *up, threads=1)
+    dQ, dK, dV, deta, dW1, dc1, dW2, dc2 = g
+    if shared:
+        dW1, dc1, dW2, dc2 = (x.sum(axis=0) for x in (dW1, dc1, dW2, dc2))
+    grads = {"Q": dQ, "K": dK, "V": dV, "eta": deta, "W1": dW1, "c1": dc1, "W2": dW2, "c2": dc2}
+    inputs = {"Q": Q, "K": K, "V": V, "eta": eta, "W1": W1, "c1": c1, "W2": W2, "c2": c2}
+    h = 1e-6
+    for name, x in inputs.items():
+        gr = grads[name]
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            keep = x[idx]
+            x[idx] = keep + h
+            lp = _mlp_loss(*inputs.values(), b, up)
+            x[idx] = keep - h
+            lm = _mlp_loss(*inputs.values(), b, up)
+            x[idx] = keep
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.max(np.abs(fd - gr)) / max(np.max(np.abs(fd)), 1e-12)
+        assert err < 1e-6, (name, err)
+
+
+def test_gelu_second_derivative():
+    """GELU'' used by the MLP backward, against central differences of GELU'."""
+    from scipy.special import erf
+    x = np.linspace(-4, 4, 81)
+    g1 = lambda t: 0.5 * (1 + erf(t / np.sqrt(2))) + t * np.exp(-0.5 * t * t) / np.sqrt(2 * np.pi)
+    h = 1e-5
+    fd = (g1(x + h) - g1(x - h)) / (2 * h)
+    g2 = np.exp(-0.5 * x * x) / np.sqrt(2 * np.pi) * (2 - x * x)
+    assert np.max(np.abs(fd - g2)) < 1e-8

@@ -42,6 +42,9 @@ BACKWARD_MUTATIONS = {
     "bwd_ln_explicit_r_term_dropped": ("for (int j = 0; j < d; ++j) dy[j] += dr * (-rr[li] * rr[li] * xt[j] / d);",
                                        "(void)dr;"),
     "bwd_ln_xhat_path_through_u_dropped": ("dxh[j] = -t1[j] * mgx[li] - gt[j] * mdux;", "dxh[j] = 0.0;"),
+    "bwd_mlp_gelu_second_derivative_dropped": ("da[p] = dd1[p] * mm[p] * gelu_grad2(a[p]);", "da[p] = 0.0;"),
+    "bwd_mlp_path_through_e_w2t_dropped": ("for (int p = 0; p < m; ++p) acc += dmv[p] * W2P(S)[(size_t)p * d + j];",
+                                           "(void)dmv;"),
     "bwd_output_grad_dropped_from_state": (
         "            if (dz)\n                for (int a = 0; a < d; ++a)\n                    for (int j = 0; j < d; ++j) D[(size_t)a * d + j] += q[a] * dz[j];\n",
         ""),
