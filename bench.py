@@ -781,6 +781,35 @@ def run_b_sweep(args):
           flush=True)
 
 
+def run_train(args):
+    """One training step of TTT-Linear (no LN) per timed step: the forward that
+    writes the batch-start states, then the outer-loop backward with random
+    upstream gradients.  Prints one JSON line (not the benchmark line)."""
+    import torch
+    from test_sequence_layers_head_b200 import ttt
+    w = WL.WORKLOADS[args.workload if args.workload != DEFAULT_WORKLOAD else "linear_B8_H12_T2048"]
+    if args.T:
+        w = WL.scaled(w, T=args.T)
+    _, dev = device_inputs(w, torch, len(os.sched_getaffinity(0)))
+    B, H, T, d = w.B, w.H, w.T, w.d
+    states = torch.empty((B, H, T // w.b, d, d), device="cuda")
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    dZ = torch.randn(B, H, T, d, generator=g, device="cuda").to(dev["Q"].dtype)
+    dW = torch.randn(B, H, d, d, generator=g, device="cuda")
+    eta = dev.get("eta")
+
+    def step():
+        ttt.linear_forward(dev["Q"], dev["K"], dev["V"], eta, dev["W0"], w.b, eta_const=w.eta_const, W_states=states)
+        ttt.linear_backward(dev["Q"], dev["K"], dev["V"], eta, states, w.b, eta_const=w.eta_const, dZ=dZ, dW_out=dW)
+    per = time_launches(torch, step, args.steps, args.warmup)
+    assert ttt.last_device_status() == ttt.TTT_OK
+    ms = statistics.mean(per)
+    print(json.dumps({"train_step_ms": ms, "tokens_per_s": tokens(w) / (ms / 1000.0), "workload": w.name,
+                      "steps": args.steps, "warmup": args.warmup,
+                      "kernels": "forward with states, then the backward"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -797,8 +826,12 @@ def main():
                     help="DRAM bytes per launch from an ncu capture of the current kernel build")
     ap.add_argument("--b-sweep", action="store_true",
                     help="mini-batch size study (state vs outputs time per b) instead of the benchmark line")
+    ap.add_argument("--train", action="store_true",
+                    help="TTT-Linear training step (forward with states + backward) instead of the benchmark line")
     args = ap.parse_args()
-    if args.b_sweep:
+    if args.train:
+        run_train(args)
+    elif args.b_sweep:
         run_b_sweep(args)
     elif args.impl == "reference":
         run_reference(args)
