@@ -18,10 +18,15 @@ Prints ONE JSON line:
               buffers (H2D of Q/K/V/eta, D2H of Z and the final state inside
               the timed region)
   decode      the 1024-step decode phase of the same workload (CUDA graph)
-  rows        the other workloads measured the same way (informational)
+  rows        the other workloads measured the same way, the LN+residual and
+              MLP decode steps, the TTT-MLP with LN+residual and the
+              backward passes (informational)
 
 --impl reference times the float64 oracle (the reference arm) on a bounded
-sample of the same workload.
+sample of the same workload.  --b-sweep prints the mini-batch size study
+(state and outputs time per b) and --train one TTT-Linear training step
+(forward writing the batch-start states, then the backward) instead of the
+benchmark line.
 """
 from __future__ import annotations
 
