@@ -44,6 +44,8 @@ def lib():
         L.ttt_oracle_mlp_backward.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, ll, P, P, P, P, P,
                                               P, P, P, P, P, P, P, P, i]
         L.ttt_oracle_mlp_backward.restype = i
+        L.ttt_oracle_qkv_prologue.argtypes = [i, i, i, i, i, P, P, P, P, P, dbl, P, P, P, P, i]
+        L.ttt_oracle_qkv_prologue.restype = i
         _lib = L
     return _lib
 
@@ -193,3 +195,24 @@ def mlp_backward(Q, K, V, eta, W1, c1, W2, c2, b, dZ=None, dW1_out=None, dc1_out
     if rc != 0:
         raise ValueError("oracle: invalid arguments")
     return dQ, dK, dV, deta, dW1, dc1, dW2, dc2
+
+
+def qkv_prologue(x, theta_q, theta_k, theta_v, theta_lr, eta_base, d, threads=None):
+    """The views and the learning-rate gate from the layer input x [B, T, Dm]:
+    theta_q/k/v [H*d, Dm] (head h owns rows h*d .. h*d+d-1), theta_lr [H, Dm].
+    Returns (Q, K, V) [B, H, T, d] and eta [B, H, T]."""
+    x, theta_q, theta_k, theta_v, theta_lr = map(_f64, (x, theta_q, theta_k, theta_v, theta_lr))
+    B, T, Dm = x.shape
+    H = theta_lr.shape[0]
+    if theta_q.shape != (H * d, Dm) or theta_k.shape != (H * d, Dm) or theta_v.shape != (H * d, Dm):
+        raise ValueError("oracle: view matrices must be [H*d, Dm]")
+    if theta_lr.shape != (H, Dm):
+        raise ValueError("oracle: theta_lr must be [H, Dm]")
+    Q, K, V = np.empty((B, H, T, d)), np.empty((B, H, T, d)), np.empty((B, H, T, d))
+    eta = np.empty((B, H, T))
+    rc = lib().ttt_oracle_qkv_prologue(B, T, Dm, H, d, _p(x), _p(theta_q), _p(theta_k), _p(theta_v),
+                                       _p(theta_lr), float(eta_base), _p(Q), _p(K), _p(V), _p(eta),
+                                       threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: invalid arguments")
+    return Q, K, V, eta

@@ -14,8 +14,12 @@
  *   - Multi-view reconstruction loss and output rule (section 3.3):
  *         l(W; x_t) = || f(theta_K x_t; W) - theta_V x_t ||^2,
  *         z_t = f(theta_Q x_t; W_t)
- *     The projections are outside this path: the oracle receives k_t, v_t,
- *     q_t directly.
+ *     The inner-loop routines receive q_t, k_t, v_t directly; the views
+ *     themselves, with the learning-rate gate below, are computed from the
+ *     layer input x by ttt_oracle_qkv_prologue (the fused prologue).
+ *   - Learnable inner learning rate (section 4.6):
+ *         eta(x) = eta_base * sigmoid(theta_lr^T x),
+ *     one theta_lr vector per head.
  *   - Mini-batch gradient descent (section 3.5): inside a mini-batch of b
  *     tokens every gradient is taken at the state W_{t'} of the batch start,
  *     and the updates are applied cumulatively token by token:
@@ -939,6 +943,65 @@ int ttt_oracle_mlp_backward(int B, int H, int T, int d, int m, int b, const doub
                           dc1o ? dc1o + (size_t)u * m : NULL, dW2o ? dW2o + (size_t)u * m * d : NULL,
                           dc2o ? dc2o + (size_t)u * d : NULL, dQ + tok, dK + tok, dV + tok, deta + (size_t)u * T,
                           dW1 + (size_t)u * d * m, dc1 + (size_t)u * m, dW2 + (size_t)u * m * d, dc2 + (size_t)u * d);
+    }
+    (void)nthreads;
+    return 0;
+}
+
+/*
+ * Prologue: the three views and the learning-rate gate of every token and
+ * head, from the layer input (sections 3.3 and 4.6).
+ *
+ *   x        : [B, T, Dm]    the layer input, one row per token
+ *   theta_q, theta_k, theta_v : [H * d, Dm]   the pages' column form: the
+ *              view of token t is theta x_t, and head h owns the rows
+ *              h d .. h d + d - 1
+ *   theta_lr : [H, Dm]       one gate vector per head
+ *   Q, K, V  : [B, H, T, d]  Q[n, h, t, j] = sum_k theta_q[h d + j, k] x[n, t, k]
+ *   eta      : [B, H, T]     eta[n, h, t] = eta_base * sigmoid(theta_lr[h] . x[n, t])
+ *
+ * eta_base is taken as given: the caller states it in the half-loss
+ * convention of the inner-loop routines (twice the pages' value).
+ */
+static double sigmoid(double u) { return 1.0 / (1.0 + exp(-u)); }
+
+/* one view of one token: out[h T d + j] = sum_k theta[(h d + j) Dm + k] x[k] */
+static void project_view(int H, int d, int Dm, const double *theta, const double *x, double *out,
+                         size_t head_stride) {
+    for (int h = 0; h < H; ++h)
+        for (int j = 0; j < d; ++j) {
+            const double *row = theta + (size_t)(h * d + j) * Dm;
+            double acc = 0.0;
+            for (int k = 0; k < Dm; ++k) acc += row[k] * x[k];
+            out[(size_t)h * head_stride + j] = acc;
+        }
+}
+
+int ttt_oracle_qkv_prologue(int B, int T, int Dm, int H, int d, const double *x, const double *theta_q,
+                            const double *theta_k, const double *theta_v, const double *theta_lr,
+                            double eta_base, double *Q, double *K, double *V, double *eta, int nthreads) {
+    if (B < 0 || T < 0 || Dm <= 0 || H < 0 || d <= 0 || !x || !theta_q || !theta_k || !theta_v || !theta_lr ||
+        !Q || !K || !V || !eta)
+        return 1;
+    const long long rows = (long long)B * T;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(static)
+#endif
+    for (long long r = 0; r < rows; ++r) {
+        const long long n = r / T, t = r % T;
+        const double *xt = x + (size_t)r * Dm;
+        const size_t o = ((size_t)n * H * T + (size_t)t) * d;   /* (n, h = 0, t, 0) */
+        const size_t hs = (size_t)T * d;                         /* one head further */
+        project_view(H, d, Dm, theta_q, xt, Q + o, hs);
+        project_view(H, d, Dm, theta_k, xt, K + o, hs);
+        project_view(H, d, Dm, theta_v, xt, V + o, hs);
+        for (int h = 0; h < H; ++h) {
+            const double *g = theta_lr + (size_t)h * Dm;
+            double u = 0.0;
+            for (int k = 0; k < Dm; ++k) u += g[k] * xt[k];
+            eta[((size_t)n * H + h) * T + t] = eta_base * sigmoid(u);
+        }
     }
     (void)nthreads;
     return 0;

@@ -74,10 +74,22 @@ MLP_LN_MUTATIONS = {
                                        "z[j] = gamma[j] * xh[j] + beta[j];"),
 }
 
+# mistakes in the prologue (views and learning-rate gate), caught by its own pins
+PROLOGUE_MUTATIONS = {
+    "prologue_transposed_view": ("acc += row[k] * x[k];", "acc += theta[(size_t)k * H * d + h * d + j] * x[k];"),
+    "prologue_head_stride": ("const size_t hs = (size_t)T * d;", "const size_t hs = (size_t)d;"),
+    "prologue_k_from_q_view": ("project_view(H, d, Dm, theta_k, xt, K + o, hs);",
+                               "project_view(H, d, Dm, theta_q, xt, K + o, hs);"),
+    "prologue_gate_sign": ("eta_base * sigmoid(u);", "eta_base * sigmoid(-u);"),
+    "prologue_gate_base_dropped": ("eta_base * sigmoid(u);", "sigmoid(u);"),
+    "prologue_gate_head_row": ("const double *g = theta_lr + (size_t)h * Dm;", "const double *g = theta_lr;"),
+}
+
 PIN_FILES = {**{n: "test_oracle_pins.py" for n in MUTATIONS},
              **{n: "test_oracle_backward.py" for n in BACKWARD_MUTATIONS},
-             **{n: "test_oracle_mlp_ln.py" for n in MLP_LN_MUTATIONS}}
-ALL_MUTATIONS = {**MUTATIONS, **BACKWARD_MUTATIONS, **MLP_LN_MUTATIONS}
+             **{n: "test_oracle_mlp_ln.py" for n in MLP_LN_MUTATIONS},
+             **{n: "test_oracle_prologue.py" for n in PROLOGUE_MUTATIONS}}
+ALL_MUTATIONS = {**MUTATIONS, **BACKWARD_MUTATIONS, **MLP_LN_MUTATIONS, **PROLOGUE_MUTATIONS}
 
 
 @pytest.mark.parametrize("name", sorted(ALL_MUTATIONS))
