@@ -323,6 +323,55 @@ typedef struct {
 
 ttt_status ttt_mlp_decode_step(const ttt_mlp_decode_args* args, cudaStream_t stream);
 
+/*
+ * ttt_qkv_prologue -- the inputs of the inner loop from the layer input: the
+ * three views of every token (section 3.3, multi-view reconstruction: the
+ * training view theta_K x_t, the label view theta_V x_t and the test view
+ * theta_Q x_t) and the learnable per-token learning rate (section 4.6):
+ *     Q[n,h,t,j] = sum_k theta_q[h d + j, k] x[n,t,k]      (K, V alike)
+ *     eta[n,h,t] = eta_base * sigmoid(sum_k theta_lr[h,k] x[n,t,k])
+ * One dense contraction on the tensor cores (bf16 operands, fp32
+ * accumulation); the epilogue writes each view in the [B, H, T, d] layout
+ * that the inner-loop entry points read, rounded once to bf16, and applies
+ * the gate in fp32.
+ *
+ *   B, T           sequences and tokens per sequence (any T >= 0).
+ *   Dm             width of the layer input; Dm % 8 == 0 (16-byte rows).
+ *   H, d           heads and head dim; d in {16, 32, 64}, 1 <= H <= 256.
+ *   io_dtype       BF16 (x, the theta matrices and Q, K, V); F32 is
+ *                  TTT_ERR_UNSUPPORTED.
+ *   x              [B, T, Dm].
+ *   theta_q, theta_k, theta_v
+ *                  [H*d, Dm] each, the pages' column form: head h owns rows
+ *                  h*d .. h*d+d-1.
+ *   theta_lr       [H, Dm], or NULL for no gate (then eta must be NULL too).
+ *   eta_base       scale of the gate, in the half-loss convention of the
+ *                  inner-loop entry points (twice the pages' value).
+ *   Q, K, V        outputs [B, H, T, d] in io_dtype.
+ *   eta            output [B, H, T] fp32, or NULL with theta_lr NULL.
+ *   flags          TTT_FLAG_TEST_STALL; any other bit is TTT_ERR_INVALID_ARG.
+ *   wait_timeout_ms  limit of one device-side wait (0: 2000 ms).
+ * Outputs must not overlap the inputs.
+ */
+typedef struct {
+    int B, T, Dm, H, d;
+    ttt_dtype io_dtype;
+    const void* x;
+    const void* theta_q;
+    const void* theta_k;
+    const void* theta_v;
+    const void* theta_lr;
+    float eta_base;
+    void* Q;
+    void* K;
+    void* V;
+    float* eta;
+    unsigned flags;
+    unsigned wait_timeout_ms;
+} ttt_qkv_prologue_args;
+
+ttt_status ttt_qkv_prologue(const ttt_qkv_prologue_args* args, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* ttt_status_string(ttt_status s);
 

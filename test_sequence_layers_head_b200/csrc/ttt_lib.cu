@@ -18,6 +18,7 @@
 #include "simt_backward_ln.cuh"
 #include "mma_backward.cuh"
 #include "mma_forward.cuh"
+#include "prologue.cuh"
 #include "tmap.h"
 
 namespace ttt {
@@ -489,6 +490,76 @@ extern "C" ttt_status ttt_linear_backward(const ttt_linear_backward_args* a, cud
         case 32: return launch_linear_backward<32>(a, stream);
         default: return launch_linear_backward<64>(a, stream);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Prologue: views and learning-rate gate from the layer input
+// ---------------------------------------------------------------------------
+extern "C" ttt_status ttt_qkv_prologue(const ttt_qkv_prologue_args* a, cudaStream_t stream) {
+    if (!a) return TTT_ERR_INVALID_ARG;
+    if (a->B < 0 || a->T < 0 || a->Dm <= 0 || a->H <= 0 || a->d <= 0) return TTT_ERR_INVALID_ARG;
+    if (a->io_dtype != TTT_F32 && a->io_dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
+    if ((a->theta_lr == nullptr) != (a->eta == nullptr)) return TTT_ERR_INVALID_ARG;
+    if (a->flags & ~TTT_FLAG_TEST_STALL) return TTT_ERR_INVALID_ARG;
+    if (a->io_dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
+    if (a->d != 16 && a->d != 32 && a->d != 64) return TTT_ERR_UNSUPPORTED;
+    if (a->H > 256 || a->Dm % 8 != 0) return TTT_ERR_UNSUPPORTED;
+    const long long rows = (long long)a->B * a->T;
+    if (rows >= (1ll << 31)) return TTT_ERR_UNSUPPORTED;
+    if (rows == 0) return TTT_OK;
+    if (!ok_ptr(a->x) || !ok_ptr(a->theta_q) || !ok_ptr(a->theta_k) || !ok_ptr(a->theta_v) || !ok_ptr(a->Q) ||
+        !ok_ptr(a->K) || !ok_ptr(a->V) || !ok_opt(a->theta_lr) || !ok_opt(a->eta))
+        return TTT_ERR_INVALID_ARG;
+
+    using namespace pro;
+    const int Hd = a->H * a->d;
+    PrologueParams p;
+    p.rows = (int)rows;
+    p.T = a->T;
+    p.H = a->H;
+    p.d = a->d;
+    p.Hd = Hd;
+    p.nk = (a->Dm + kBK - 1) / kBK;
+    p.nvt = (Hd + kBN - 1) / kBN;
+    p.ntn = 3 * p.nvt + (a->theta_lr ? 1 : 0);
+    p.tiles = ((rows + kBM - 1) / kBM) * p.ntn;
+    p.brows = Hd < kBN ? Hd : kBN;
+    p.ng = (a->H + 15) / 16 * 16;
+    p.Q = static_cast<__nv_bfloat16*>(a->Q);
+    p.K = static_cast<__nv_bfloat16*>(a->K);
+    p.V = static_cast<__nv_bfloat16*>(a->V);
+    p.eta = a->eta;
+    p.eta_base = a->eta_base;
+    p.status = status_ptr();
+    p.wait_ns = wait_ns(a->wait_timeout_ms);
+    p.flags = a->flags;
+    if (!p.status) return TTT_ERR_CUDA;
+
+    // x [rows, Dm] and theta [Hd or H, Dm], K-major tiles of 64 model-width
+    // elements (128 bytes, 128-byte swizzle); without the gate its map is a
+    // copy of x's and is never read
+    const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+    const uint64_t pitch = (uint64_t)a->Dm * 2;
+    CUtensorMap mX, mTq, mTk, mTv, mTl;
+    if (!encode_2d(&mX, a->x, bf, a->Dm, rows, pitch, kBK, kBM, sw) ||
+        !encode_2d(&mTq, a->theta_q, bf, a->Dm, Hd, pitch, kBK, p.brows, sw) ||
+        !encode_2d(&mTk, a->theta_k, bf, a->Dm, Hd, pitch, kBK, p.brows, sw) ||
+        !encode_2d(&mTv, a->theta_v, bf, a->Dm, Hd, pitch, kBK, p.brows, sw))
+        return TTT_ERR_CUDA;
+    if (a->theta_lr) {
+        if (!encode_2d(&mTl, a->theta_lr, bf, a->Dm, a->H, pitch, kBK, p.ng, sw)) return TTT_ERR_CUDA;
+    } else {
+        mTl = mX;
+    }
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        return TTT_ERR_CUDA;
+    const int grid = (int)(p.tiles < sms ? p.tiles : sms);
+    if (!set_smem(prologue_kernel, kSmemBytes)) return TTT_ERR_CUDA;
+    prologue_kernel<<<grid, kThreads, kSmemBytes, stream>>>(mX, mTq, mTk, mTv, mTl, p);
+    return launch_status();
 }
 
 extern "C" const char* ttt_status_string(ttt_status s) {

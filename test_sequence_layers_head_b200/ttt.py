@@ -70,6 +70,12 @@ class MlpDecodeArgs(ctypes.Structure):
                 ("c2", _vp), ("q", _vp), ("k", _vp), ("v", _vp), ("eta", _vp), ("eta_const", _f), ("z", _vp)]
 
 
+class QkvPrologueArgs(ctypes.Structure):
+    _fields_ = [("B", _i), ("T", _i), ("Dm", _i), ("H", _i), ("d", _i), ("io_dtype", _i), ("x", _vp),
+                ("theta_q", _vp), ("theta_k", _vp), ("theta_v", _vp), ("theta_lr", _vp), ("eta_base", _f),
+                ("Q", _vp), ("K", _vp), ("V", _vp), ("eta", _vp), ("flags", _u), ("wait_timeout_ms", _u)]
+
+
 class TTTError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: {status_string(code)}")
@@ -80,7 +86,8 @@ _lib = None
 
 # Every symbol include/ttt.h declares.
 EXPORTS = ("ttt_linear_forward", "ttt_linear_backward", "ttt_mlp_forward", "ttt_linear_decode_step",
-           "ttt_mlp_decode_step", "ttt_status_string", "ttt_last_device_status", "ttt_version")
+           "ttt_mlp_decode_step", "ttt_qkv_prologue", "ttt_status_string", "ttt_last_device_status",
+           "ttt_version")
 
 
 def library() -> ctypes.CDLL:
@@ -101,6 +108,8 @@ def library() -> ctypes.CDLL:
         L.ttt_linear_decode_step.restype = _i
         L.ttt_mlp_decode_step.argtypes = [ctypes.POINTER(MlpDecodeArgs), _vp]
         L.ttt_mlp_decode_step.restype = _i
+        L.ttt_qkv_prologue.argtypes = [ctypes.POINTER(QkvPrologueArgs), _vp]
+        L.ttt_qkv_prologue.restype = _i
         L.ttt_status_string.argtypes = [_i]
         L.ttt_status_string.restype = ctypes.c_char_p
         L.ttt_last_device_status.argtypes = [_vp]
@@ -254,6 +263,27 @@ def mlp_decode_step(W1, c1, W2, c2, q, k, v, eta, *, eta_const=0.0, z=None, stre
                       _ptr(eta), float(eta_const), _ptr(z))
     _check(library().ttt_mlp_decode_step(ctypes.byref(a), _stream(stream)), "ttt_mlp_decode_step")
     return z
+
+
+def qkv_prologue(x, theta_q, theta_k, theta_v, theta_lr, eta_base, d, *, Q=None, K=None, V=None, eta=None,
+                 flags=0, wait_timeout_ms=0, stream=None):
+    """The views and the learning-rate gate from the layer input; see
+    ``ttt_qkv_prologue``.  x [B,T,Dm] bf16; theta_q/k/v [H*d, Dm]; theta_lr
+    [H, Dm] or None (no gate).  Returns (Q, K, V) [B,H,T,d] and eta [B,H,T]
+    (None without the gate)."""
+    B, T, Dm = x.shape
+    H = theta_q.shape[0] // d
+    dev = x.device
+    Q = torch.empty((B, H, T, d), device=dev, dtype=x.dtype) if Q is None else Q
+    K = torch.empty((B, H, T, d), device=dev, dtype=x.dtype) if K is None else K
+    V = torch.empty((B, H, T, d), device=dev, dtype=x.dtype) if V is None else V
+    if theta_lr is not None and eta is None:
+        eta = torch.empty((B, H, T), device=dev, dtype=torch.float32)
+    a = QkvPrologueArgs(B, T, Dm, H, d, _io_dtype(x), _ptr(x), _ptr(theta_q), _ptr(theta_k), _ptr(theta_v),
+                        _ptr(theta_lr), float(eta_base), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), int(flags),
+                        int(wait_timeout_ms))
+    _check(library().ttt_qkv_prologue(ctypes.byref(a), _stream(stream)), "ttt_qkv_prologue")
+    return Q, K, V, eta
 
 
 def last_device_status(stream=None) -> int:

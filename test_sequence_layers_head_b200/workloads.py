@@ -255,3 +255,94 @@ def random_case(kind: str, B: int, H: int, T: int, d: int, b: int, io_dtype: str
     """A small ad-hoc case with the same distributions (parity tests)."""
     w = Workload(f"{kind}_case", kind, B, H, T, d, b, io_dtype, eta_mode, eta_const, seed)
     return make_inputs(w, threads=1)
+
+
+# ----------------------------------------------------------------------------
+# the fused prologue: layer input and the view / gate weights
+# ----------------------------------------------------------------------------
+# Recipe: x ~ N(0, 1) per element (a normalised layer input); theta_q, theta_k,
+# theta_v ~ N(0, 1/(Dm d)), so each view element has variance 1/d like the
+# inner-loop workloads' Q, K, V; theta_lr ~ N(0, 1/Dm), so the gate's logits
+# are ~ N(0, 1) like their u_t and eta_base = 1/64 reproduces their
+# eta_t = (1/64) sigmoid(u_t).  All values are rounded once to bf16.  x is
+# drawn in blocks of 128 tokens, one stream per (sequence, block), so any
+# block can be regenerated alone.
+
+_S_PRO_X, _S_PRO_THETA = 4, 5
+PRO_BLOCK = 128
+
+
+@dataclasses.dataclass(frozen=True)
+class PrologueWorkload:
+    name: str
+    B: int
+    T: int
+    Dm: int
+    H: int
+    d: int
+    gate: bool
+    eta_base: float
+    seed: int
+
+    @property
+    def tokens(self) -> int:
+        return self.B * self.T
+
+
+# the two model widths of the inner-loop workloads: 12 heads of 64 (width 768)
+# and 32 heads of 64 (width 2048), at their batch and sequence sizes
+PROLOGUE_WORKLOADS = {
+    w.name: w
+    for w in [
+        PrologueWorkload("prologue_B8_T2048_Dm768_H12", 8, 2048, 768, 12, 64, True, 1.0 / 64.0, 20260011),
+        PrologueWorkload("prologue_B16_T32768_Dm2048_H32", 16, 32768, 2048, 32, 64, True, 1.0 / 64.0, 20260014),
+    ]
+}
+
+
+def prologue_x_block(w: PrologueWorkload, n: int, blk: int) -> np.ndarray:
+    """Rows PRO_BLOCK*blk .. of sequence n of the layer input, float64 draws."""
+    rows = min(PRO_BLOCK, w.T - PRO_BLOCK * blk)
+    return _rng(w.seed, _S_PRO_X, n * 1_000_003 + blk).standard_normal((rows, w.Dm))
+
+
+def prologue_theta(w: PrologueWorkload) -> dict:
+    """theta_q, theta_k, theta_v [H*d, Dm] and theta_lr [H, Dm], float64 draws."""
+    g = _rng(w.seed, _S_PRO_THETA, 0)
+    sd = np.sqrt(1.0 / (w.Dm * w.d))
+    out = {nm: g.standard_normal((w.H * w.d, w.Dm)) * sd for nm in ("theta_q", "theta_k", "theta_v")}
+    out["theta_lr"] = g.standard_normal((w.H, w.Dm)) * np.sqrt(1.0 / w.Dm)
+    return out
+
+
+def make_prologue_inputs(w: PrologueWorkload, want_exact: bool = True, threads: int = 8) -> dict:
+    """{"raw": ..., "exact": ...}: x [B, T, Dm] and the theta matrices as bf16
+    bits (raw) and their exact float64 values (exact; skipped for x when
+    want_exact is False)."""
+    nblk = (w.T + PRO_BLOCK - 1) // PRO_BLOCK
+    raw = {"x": np.empty((w.B, w.T, w.Dm), np.uint16)}
+    exact = {"x": np.empty((w.B, w.T, w.Dm))} if want_exact else {}
+
+    def fill(jobs):
+        for n, blk in jobs:
+            r, e = store(prologue_x_block(w, n, blk), BF16)
+            s = slice(PRO_BLOCK * blk, PRO_BLOCK * blk + r.shape[0])
+            raw["x"][n, s] = r
+            if want_exact:
+                exact["x"][n, s] = e
+
+    jobs = [(n, blk) for n in range(w.B) for blk in range(nblk)]
+    parts = [jobs[i::threads] for i in range(min(threads, len(jobs)))]
+    if parts:
+        with ThreadPoolExecutor(max_workers=len(parts)) as ex:
+            list(ex.map(fill, parts))
+    for nm, x in prologue_theta(w).items():
+        raw[nm], exact[nm] = store(x, BF16)
+    return {"raw": raw, "exact": exact}
+
+
+def prologue_case(B: int, T: int, Dm: int, H: int, d: int, gate: bool = True, eta_base: float = 1.0 / 64.0,
+                  seed: int = 11) -> tuple:
+    """A small ad-hoc prologue case with the same distributions (parity tests)."""
+    w = PrologueWorkload(f"prologue_case_B{B}_T{T}_Dm{Dm}_H{H}_d{d}", B, T, Dm, H, d, gate, eta_base, seed)
+    return w, make_prologue_inputs(w, threads=1)

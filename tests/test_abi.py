@@ -19,7 +19,7 @@ def declared_symbols():
 def test_header_declares_entry_points():
     syms = declared_symbols()
     for s in ("ttt_linear_forward", "ttt_linear_backward", "ttt_mlp_forward", "ttt_linear_decode_step",
-              "ttt_mlp_decode_step"):
+              "ttt_mlp_decode_step", "ttt_qkv_prologue"):
         assert s in syms
 
 
@@ -136,6 +136,7 @@ def test_null_args_struct(ttt_lib):
     assert L.ttt_linear_decode_step(None, None) == 1
     assert L.ttt_mlp_decode_step(None, None) == 1
     assert L.ttt_linear_backward(None, None) == 1
+    assert L.ttt_qkv_prologue(None, None) == 1
 
 
 def test_mlp_and_decode_validation(ttt_lib):
@@ -219,6 +220,44 @@ def test_mlp_ln_validation(ttt_lib):
     m.ln_eps = 1e-6
     m.ln_beta = fake + 4             # misaligned
     assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
+
+
+def _prologue_args(ttt, **kw):
+    a = ttt.QkvPrologueArgs()
+    a.B, a.T, a.Dm, a.H, a.d, a.io_dtype = 2, 64, 768, 12, 64, ttt.TTT_BF16
+    fake = 1 << 20
+    a.x = a.theta_q = a.theta_k = a.theta_v = a.theta_lr = a.Q = a.K = a.V = a.eta = fake
+    a.eta_base = 1.0
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), 1),
+    (dict(T=-1), 1),
+    (dict(Dm=0), 1),
+    (dict(H=0), 1),
+    (dict(d=0), 1),
+    (dict(io_dtype=4), 1),
+    (dict(io_dtype=0), 2),                       # fp32 input: no kernel
+    (dict(d=48), 2),
+    (dict(H=257), 2),                            # the gate tile holds at most 256 heads
+    (dict(Dm=772), 2),                           # rows of x must be 16-byte multiples
+    (dict(theta_lr=None), 1),                    # gate pointers come in pairs
+    (dict(eta=None), 1),
+    (dict(flags=0x1), 1),                        # only the stall hook is a valid flag
+    (dict(x=None), 1),
+    (dict(theta_v=(1 << 20) + 2), 1),
+    (dict(Q=None), 1),
+    (dict(K=(1 << 20) + 8), 1),
+    (dict(eta=(1 << 20) + 4), 1),
+    (dict(B=0, x=None, Q=None), 0),              # nothing to do
+    (dict(T=0, x=None, Q=None), 0),
+])
+def test_qkv_prologue_validation(ttt_lib, kw, code):
+    a = _prologue_args(ttt_lib, **kw)
+    assert ttt_lib.library().ttt_qkv_prologue(ctypes.byref(a), None) == code
 
 
 def test_binding_refuses_cpu_tensors(ttt_lib):
