@@ -24,9 +24,10 @@ Prints ONE JSON line:
 
 --impl reference times the float64 oracle (the reference arm) on a bounded
 sample of the same workload.  --b-sweep prints the mini-batch size study
-(state and outputs time per b) and --train one TTT-Linear training step
-(forward writing the batch-start states, then the backward) instead of the
-benchmark line.
+(state and outputs time per b), --train one TTT-Linear training step
+(forward writing the batch-start states, then the backward) and --prologue
+the fused prologue (the views and the learning-rate gate from the layer
+input, alone and followed by the forward) instead of the benchmark line.
 """
 from __future__ import annotations
 
@@ -815,6 +816,71 @@ def run_train(args):
                       "kernels": "forward with states, then the backward"}), flush=True)
 
 
+def prologue_flops(w) -> int:
+    """Algorithmic flops of one prologue launch: 2 Dm per output column per
+    token, over the 3 H d view columns and the H gate columns."""
+    return 2 * w.tokens * w.Dm * (3 * w.H * w.d + (w.H if w.gate else 0))
+
+
+def prologue_bytes(w) -> int:
+    """Algorithmic HBM bytes of one launch: x and the theta matrices read once
+    (bf16), Q, K, V written once (bf16), eta written once (fp32)."""
+    cols = 3 * w.H * w.d + (w.H if w.gate else 0)
+    return 2 * w.tokens * w.Dm + 2 * cols * w.Dm + 2 * 3 * w.tokens * w.H * w.d + (4 * w.tokens * w.H if w.gate else 0)
+
+
+def run_prologue(args):
+    """The fused prologue (views and learning-rate gate from the layer input,
+    ttt_qkv_prologue) on the two model widths, then the prologue followed by
+    the TTT-Linear forward on the 32-head width.  Tensor-bound: the roofline
+    is the dense bf16 peak.  Prints one JSON line (not the benchmark line)."""
+    import torch
+    from test_sequence_layers_head_b200 import ttt
+    hbm, tflops, src = measured_peaks()
+    threads = len(os.sched_getaffinity(0))
+    flush_buf = torch.empty(256 * 1024 * 1024 // 4, device="cuda")
+    rows = []
+    for name, w in WL.PROLOGUE_WORKLOADS.items():
+        inp = WL.make_prologue_inputs(w, want_exact=False, threads=threads)
+        dev = {k: to_dev(v, torch) for k, v in inp["raw"].items()}
+        B, H, T, d = w.B, w.H, w.T, w.d
+        Q, K, V = (torch.empty((B, H, T, d), device="cuda", dtype=torch.bfloat16) for _ in range(3))
+        eta = torch.empty((B, H, T), device="cuda")
+
+        def pro():
+            ttt.qkv_prologue(dev["x"], dev["theta_q"], dev["theta_k"], dev["theta_v"], dev["theta_lr"], w.eta_base,
+                             d, Q=Q, K=K, V=V, eta=eta)
+        with ClockSampler(torch.cuda.current_device()) as clk:
+            per = time_launches(torch, pro, args.steps, args.warmup, flush=lambda: flush_buf.zero_())
+        assert ttt.last_device_status() == ttt.TTT_OK
+        ms = statistics.mean(per)
+        ach = prologue_flops(w) / (ms / 1000.0) / 1e12
+        row = {"workload": name, "ms": ms, "tokens_per_s": w.tokens / (ms / 1000.0),
+               "roofline": {"bound": "tensor", "achieved": ach, "peak": tflops, "unit": "TFLOP/s",
+                            "frac": ach / tflops, "peak_source": src},
+               "hbm_gbs": prologue_bytes(w) / (ms / 1000.0) / 1e9, "clocks": clk.summary()}
+        if H == 32:
+            # the TTT-Linear forward on the views just computed (W0 per head)
+            g = torch.Generator(device="cuda")
+            g.manual_seed(3)
+            W0 = torch.randn(H, d, d, generator=g, device="cuda") / d ** 0.5
+            Z = torch.empty_like(Q)
+            W_out = torch.empty((B, H, d, d), device="cuda")
+
+            def layer():
+                pro()
+                ttt.linear_forward(Q, K, V, eta, W0, 16, Z=Z, W_out=W_out)
+            per2 = time_launches(torch, layer, max(3, args.steps // 4), args.warmup, flush=lambda: flush_buf.zero_())
+            assert ttt.last_device_status() == ttt.TTT_OK
+            ms2 = statistics.mean(per2)
+            row["with_linear_forward"] = {"ms": ms2, "tokens_per_s": w.tokens / (ms2 / 1000.0)}
+        rows.append(row)
+        del dev, Q, K, V, eta
+        torch.cuda.empty_cache()
+    print(json.dumps({"prologue": rows, "dtype": "bf16", "data": "synthetic",
+                      "flush": "256 MiB L2 flush before every timed launch"}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -833,8 +899,13 @@ def main():
                     help="mini-batch size study (state vs outputs time per b) instead of the benchmark line")
     ap.add_argument("--train", action="store_true",
                     help="TTT-Linear training step (forward with states + backward) instead of the benchmark line")
+    ap.add_argument("--prologue", action="store_true",
+                    help="the fused prologue (views and learning-rate gate from the layer input) instead of the "
+                         "benchmark line")
     args = ap.parse_args()
-    if args.train:
+    if args.prologue:
+        run_prologue(args)
+    elif args.train:
         run_train(args)
     elif args.b_sweep:
         run_b_sweep(args)
