@@ -218,6 +218,11 @@ ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_
  *                  LN as in ttt_linear_forward (ln_gamma, ln_beta [H, d] fp32,
  *                  ln_eps > 0).  Same kernel choice as the plain model.
  *                  0: plain.
+ *   W_states       NULL, or [B, H, T/b, 2dm + m + d] fp32: the state at the
+ *                  start of every mini-batch, each one W1 [d][m], c1 [m],
+ *                  W2 [m][d], c2 [d] (the checkpoints ttt_mlp_backward reads;
+ *                  section 6.12).  Served by the fp32 CUDA-core kernel for
+ *                  every dtype and d; not with use_ln (TTT_ERR_UNSUPPORTED).
  */
 typedef struct {
     int B, H, T, d, b;
@@ -243,9 +248,62 @@ typedef struct {
     const float* ln_gamma;
     const float* ln_beta;
     float ln_eps;
+    float* W_states;
 } ttt_mlp_args;
 
 ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
+
+/*
+ * ttt_mlp_backward -- outer-loop gradients of the TTT-MLP prefill (no LN):
+ * reverse-mode differentiation of ttt_mlp_forward through the inner loop's
+ * updates (section 3.4), one mini-batch at a time in reverse order from the
+ * batch-start states ttt_mlp_forward wrote to W_states (section 6.12).
+ *
+ *   B, H, T, d, b, io_dtype, Q, K, V, eta, eta_const
+ *                  exactly as given to the forward that wrote W_states.
+ *                  Served by an fp32 CUDA-core kernel: d in {16, 32, 64},
+ *                  b up to the shared-memory limit (16 at d = 64).
+ *   W_states       [B, H, T/b, 2dm + m + d] fp32, from ttt_mlp_forward.
+ *   dZ             [B, H, T, d] io_dtype, or NULL (zero).
+ *   dW1_out [B,H,d,m], dc1_out [B,H,m], dW2_out [B,H,m,d], dc2_out [B,H,d]
+ *                  gradients with respect to the final state, each or NULL
+ *                  (zero).
+ * Outputs
+ *   dQ, dK, dV     [B, H, T, d] io_dtype.
+ *   deta           [B, H, T] fp32, or NULL (not computed).
+ *   dW1 [B,H,d,m], dc1 [B,H,m], dW2 [B,H,m,d], dc2 [B,H,d]
+ *                  gradients with respect to each unit's initial state (for
+ *                  parameters shared over sequences, the caller sums over B).
+ *                  They also serve as the kernel's running adjoint, so they
+ *                  must not overlap any input.
+ *   flags          must be 0.
+ */
+typedef struct {
+    int B, H, T, d, b;
+    ttt_dtype io_dtype;
+    const void* Q;
+    const void* K;
+    const void* V;
+    const float* eta;
+    float eta_const;
+    const float* W_states;
+    const void* dZ;
+    const float* dW1_out;
+    const float* dc1_out;
+    const float* dW2_out;
+    const float* dc2_out;
+    void* dQ;
+    void* dK;
+    void* dV;
+    float* deta;
+    float* dW1;
+    float* dc1;
+    float* dW2;
+    float* dc2;
+    unsigned flags;
+} ttt_mlp_backward_args;
+
+ttt_status ttt_mlp_backward(const ttt_mlp_backward_args* args, cudaStream_t stream);
 
 /*
  * ttt_linear_decode_step -- one generated token per unit, TTT-Linear plain or

@@ -39,6 +39,12 @@ __device__ __forceinline__ float gelu_grad_f(float x) {
     return Phi + x * phi;
 }
 
+// GELU'' = phi(x) (2 - x^2), the derivative of Phi + x phi (phi' = -x phi), for the
+// backward of the MLP's GELU' term
+__device__ __forceinline__ float gelu_grad2_f(float x) {
+    return 0.39894228040143268f * expf(-0.5f * x * x) * (2.0f - x * x);
+}
+
 // GELU and GELU' together for the tensor-core MLP kernel: erf by the rational
 // approximation of Abramowitz & Stegun, Handbook of Mathematical Functions,
 // formula 7.1.26 (|error| <= 1.5e-7 for every argument), on z = |x| / sqrt(2);

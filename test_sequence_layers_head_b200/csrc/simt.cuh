@@ -231,6 +231,7 @@ struct SimtMlpParams {
     const float* gamma;   // LN+residual on the output layer: [H, D]
     const float* beta;
     float eps;
+    float* W_states;      // [units, T / b, 2 D M + M + D] batch-start states (W1, c1, W2, c2), or null
 };
 
 // LN = true: f(x) = x + gamma LN(GELU(x W1 + c1) W2 + c2) + beta; the residual E of
@@ -272,6 +273,16 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_kernel(SimtMlpParams p)
     for (int e = tid; e < D; e += kSimtThreads) c2[e] = p.c2 ? p.c2[(size_t)pu * D + e] : 0.f;
     __syncthreads();
     for (int t0 = 0; t0 < p.T; t0 += b) {
+        if (p.W_states) {
+            // the state at the start of this mini-batch: W1 [D][M], c1 [M], W2 [M][D], c2 [D]
+            float* st = p.W_states + ((size_t)unit * (p.T / b) + t0 / b) * (2 * (size_t)D * M + M + D);
+            for (int e = tid; e < D * M; e += kSimtThreads) {
+                st[e] = W1[e];
+                st[(size_t)D * M + M + e] = W2[e];
+            }
+            for (int e = tid; e < M; e += kSimtThreads) st[(size_t)D * M + e] = c1[e];
+            for (int e = tid; e < D; e += kSimtThreads) st[2 * (size_t)D * M + M + e] = c2[e];
+        }
         for (int e = tid; e < b * D; e += kSimtThreads) {
             const size_t g = (size_t)t0 * D + e;
             Kt[e] = IoTraits<IO>::load(K, g);

@@ -16,6 +16,7 @@
 #include "simt.cuh"
 #include "simt_backward.cuh"
 #include "simt_backward_ln.cuh"
+#include "simt_mlp_backward.cuh"
 #include "mma_backward.cuh"
 #include "mma_forward.cuh"
 #include "prologue.cuh"
@@ -256,6 +257,7 @@ ttt_status launch_simt_mlp(const ttt_mlp_args* a, cudaStream_t st) {
     p.gamma = a->ln_gamma;
     p.beta = a->ln_beta;
     p.eps = a->ln_eps;
+    p.W_states = a->W_states;
     const size_t smem = simt_mlp_smem(D, a->b, a->use_ln != 0);
     auto k = a->use_ln ? simt_mlp_kernel<D, IO, true> : simt_mlp_kernel<D, IO, false>;
     if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
@@ -330,8 +332,10 @@ extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream
     if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL)) return TTT_ERR_INVALID_ARG;
     if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
     if (a->use_ln && (!ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !(a->ln_eps > 0.f))) return TTT_ERR_INVALID_ARG;
+    if (!ok_opt(a->W_states)) return TTT_ERR_INVALID_ARG;
+    if (a->W_states && a->use_ln) return TTT_ERR_UNSUPPORTED;
     const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
-                    !(a->flags & TTT_FLAG_FORCE_SIMT);
+                    !(a->flags & TTT_FLAG_FORCE_SIMT) && !a->W_states;
     if (tc) return tc_mlp(a, stream);
     if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
     switch (a->d) {
@@ -489,6 +493,50 @@ extern "C" ttt_status ttt_linear_backward(const ttt_linear_backward_args* a, cud
         case 16: return launch_linear_backward<16>(a, stream);
         case 32: return launch_linear_backward<32>(a, stream);
         default: return launch_linear_backward<64>(a, stream);
+    }
+}
+
+namespace ttt {
+namespace {
+template <int D, typename IO>
+ttt_status launch_mlp_backward_t(const ttt_mlp_backward_args* a, cudaStream_t st) {
+    SimtMlpBackwardParams p{a->H,       a->T,       a->b,       a->Q,       a->K,       a->V,
+                            a->eta,     a->eta_const, a->W_states, a->dZ,   a->dW1_out, a->dc1_out,
+                            a->dW2_out, a->dc2_out, a->dQ,      a->dK,      a->dV,      a->deta,
+                            a->dW1,     a->dc1,     a->dW2,     a->dc2};
+    const size_t smem = simt_mlp_backward_smem(D, a->b);
+    auto k = simt_mlp_backward_kernel<D, IO>;
+    if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
+    k<<<(unsigned)(a->B * a->H), kSimtThreads, smem, st>>>(p);
+    return launch_status();
+}
+template <int D>
+ttt_status launch_mlp_backward(const ttt_mlp_backward_args* a, cudaStream_t st) {
+    return a->io_dtype == TTT_F32 ? launch_mlp_backward_t<D, float>(a, st)
+                                  : launch_mlp_backward_t<D, __nv_bfloat16>(a, st);
+}
+}  // namespace
+}  // namespace ttt
+
+extern "C" ttt_status ttt_mlp_backward(const ttt_mlp_backward_args* a, cudaStream_t stream) {
+    if (!a) return TTT_ERR_INVALID_ARG;
+    ttt_status v = validate_common(a->B, a->H, a->T, a->d, a->b, a->io_dtype);
+    if (v != TTT_OK) return v;
+    const long long units = (long long)a->B * a->H;
+    if (units == 0) return TTT_OK;
+    if (a->T > 0 && (!ok_ptr(a->Q) || !ok_ptr(a->K) || !ok_ptr(a->V) || !ok_ptr(a->W_states) ||
+                     !ok_ptr(a->dQ) || !ok_ptr(a->dK) || !ok_ptr(a->dV)))
+        return TTT_ERR_INVALID_ARG;
+    if (!ok_ptr(a->dW1) || !ok_ptr(a->dc1) || !ok_ptr(a->dW2) || !ok_ptr(a->dc2)) return TTT_ERR_INVALID_ARG;
+    if (!ok_opt(a->eta) || !ok_opt(a->dZ) || !ok_opt(a->deta) || !ok_opt(a->dW1_out) || !ok_opt(a->dc1_out) ||
+        !ok_opt(a->dW2_out) || !ok_opt(a->dc2_out))
+        return TTT_ERR_INVALID_ARG;
+    if (a->flags != 0) return TTT_ERR_INVALID_ARG;
+    if (simt_mlp_backward_smem(a->d, a->b) > 227 * 1024) return TTT_ERR_UNSUPPORTED;
+    switch (a->d) {
+        case 16: return launch_mlp_backward<16>(a, stream);
+        case 32: return launch_mlp_backward<32>(a, stream);
+        default: return launch_mlp_backward<64>(a, stream);
     }
 }
 

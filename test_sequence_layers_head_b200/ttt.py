@@ -48,7 +48,14 @@ class MlpArgs(ctypes.Structure):
                 ("W1", _vp), ("c1", _vp), ("W2", _vp), ("c2", _vp), ("params_per_sequence", _i),
                 ("Z", _vp), ("W1_out", _vp), ("c1_out", _vp), ("W2_out", _vp), ("c2_out", _vp),
                 ("flags", _u), ("wait_timeout_ms", _u), ("use_ln", _i), ("ln_gamma", _vp), ("ln_beta", _vp),
-                ("ln_eps", _f)]
+                ("ln_eps", _f), ("W_states", _vp)]
+
+
+class MlpBackwardArgs(ctypes.Structure):
+    _fields_ = [("B", _i), ("H", _i), ("T", _i), ("d", _i), ("b", _i), ("io_dtype", _i), ("Q", _vp), ("K", _vp),
+                ("V", _vp), ("eta", _vp), ("eta_const", _f), ("W_states", _vp), ("dZ", _vp), ("dW1_out", _vp),
+                ("dc1_out", _vp), ("dW2_out", _vp), ("dc2_out", _vp), ("dQ", _vp), ("dK", _vp), ("dV", _vp),
+                ("deta", _vp), ("dW1", _vp), ("dc1", _vp), ("dW2", _vp), ("dc2", _vp), ("flags", _u)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -86,8 +93,8 @@ _lib = None
 
 # Every symbol include/ttt.h declares.
 EXPORTS = ("ttt_linear_forward", "ttt_linear_backward", "ttt_mlp_forward", "ttt_linear_decode_step",
-           "ttt_mlp_decode_step", "ttt_qkv_prologue", "ttt_status_string", "ttt_last_device_status",
-           "ttt_version")
+           "ttt_mlp_decode_step", "ttt_mlp_backward", "ttt_qkv_prologue", "ttt_status_string",
+           "ttt_last_device_status", "ttt_version")
 
 
 def library() -> ctypes.CDLL:
@@ -108,6 +115,8 @@ def library() -> ctypes.CDLL:
         L.ttt_linear_decode_step.restype = _i
         L.ttt_mlp_decode_step.argtypes = [ctypes.POINTER(MlpDecodeArgs), _vp]
         L.ttt_mlp_decode_step.restype = _i
+        L.ttt_mlp_backward.argtypes = [ctypes.POINTER(MlpBackwardArgs), _vp]
+        L.ttt_mlp_backward.restype = _i
         L.ttt_qkv_prologue.argtypes = [ctypes.POINTER(QkvPrologueArgs), _vp]
         L.ttt_qkv_prologue.restype = _i
         L.ttt_status_string.argtypes = [_i]
@@ -221,9 +230,11 @@ def linear_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW_out=None, eta_cons
 
 def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, *, eta_const=0.0, Z=None, W1_out=None, c1_out=None,
                 W2_out=None, c2_out=None, flags=0, wait_timeout_ms=0, use_ln=False, gamma=None, beta=None,
-                eps=1e-6, stream=None):
+                eps=1e-6, W_states=None, stream=None):
     """TTT-MLP prefill; see ``ttt_mlp_forward``.  Returns (Z, W1, c1, W2, c2).
-    use_ln: LN+residual on the output layer with gamma, beta [H,d]."""
+    use_ln: LN+residual on the output layer with gamma, beta [H,d].
+    W_states: [B,H,T/b,2dm+m+d] fp32 to receive the batch-start states (the
+    checkpoints of ``mlp_backward``)."""
     B, H, T, d = Q.shape
     m = W1.shape[-1]
     dev = Q.device
@@ -237,7 +248,7 @@ def mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, *, eta_const=0.0, Z=None, W1_ou
     a = MlpArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
                 _ptr(W1), _ptr(c1), _ptr(W2), _ptr(c2), per_seq, _ptr(Z), _ptr(W1_out), _ptr(c1_out),
                 _ptr(W2_out), _ptr(c2_out), int(flags), int(wait_timeout_ms), int(bool(use_ln)), _ptr(gamma),
-                _ptr(beta), float(eps))
+                _ptr(beta), float(eps), _ptr(W_states))
     _check(library().ttt_mlp_forward(ctypes.byref(a), _stream(stream)), "ttt_mlp_forward")
     return Z, W1_out, c1_out, W2_out, c2_out
 
@@ -263,6 +274,31 @@ def mlp_decode_step(W1, c1, W2, c2, q, k, v, eta, *, eta_const=0.0, z=None, stre
                       _ptr(eta), float(eta_const), _ptr(z))
     _check(library().ttt_mlp_decode_step(ctypes.byref(a), _stream(stream)), "ttt_mlp_decode_step")
     return z
+
+
+def mlp_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW1_out=None, dc1_out=None, dW2_out=None, dc2_out=None,
+                 eta_const=0.0, dQ=None, dK=None, dV=None, deta=None, want_deta=True, dW1=None, dc1=None, dW2=None,
+                 dc2=None, stream=None):
+    """Outer-loop gradients of the TTT-MLP prefill; see ``ttt_mlp_backward``.
+    Returns (dQ, dK, dV, deta, dW1, dc1, dW2, dc2); deta is None when
+    ``want_deta`` is False."""
+    B, H, T, d = Q.shape
+    m = 4 * d
+    dev, f32 = Q.device, torch.float32
+    dQ = torch.empty_like(Q) if dQ is None else dQ
+    dK = torch.empty_like(Q) if dK is None else dK
+    dV = torch.empty_like(Q) if dV is None else dV
+    if want_deta and deta is None:
+        deta = torch.empty((B, H, T), device=dev, dtype=f32)
+    dW1 = torch.empty((B, H, d, m), device=dev, dtype=f32) if dW1 is None else dW1
+    dc1 = torch.empty((B, H, m), device=dev, dtype=f32) if dc1 is None else dc1
+    dW2 = torch.empty((B, H, m, d), device=dev, dtype=f32) if dW2 is None else dW2
+    dc2 = torch.empty((B, H, d), device=dev, dtype=f32) if dc2 is None else dc2
+    a = MlpBackwardArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
+                        _ptr(W_states), _ptr(dZ), _ptr(dW1_out), _ptr(dc1_out), _ptr(dW2_out), _ptr(dc2_out),
+                        _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW1), _ptr(dc1), _ptr(dW2), _ptr(dc2), 0)
+    _check(library().ttt_mlp_backward(ctypes.byref(a), _stream(stream)), "ttt_mlp_backward")
+    return dQ, dK, dV, deta, dW1, dc1, dW2, dc2
 
 
 def qkv_prologue(x, theta_q, theta_k, theta_v, theta_lr, eta_base, d, *, Q=None, K=None, V=None, eta=None,

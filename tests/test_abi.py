@@ -137,6 +137,7 @@ def test_null_args_struct(ttt_lib):
     assert L.ttt_mlp_decode_step(None, None) == 1
     assert L.ttt_linear_backward(None, None) == 1
     assert L.ttt_qkv_prologue(None, None) == 1
+    assert L.ttt_mlp_backward(None, None) == 1
 
 
 def test_mlp_and_decode_validation(ttt_lib):
@@ -220,6 +221,50 @@ def test_mlp_ln_validation(ttt_lib):
     m.ln_eps = 1e-6
     m.ln_beta = fake + 4             # misaligned
     assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
+
+
+def _mlp_backward_args(ttt, **kw):
+    a = ttt.MlpBackwardArgs()
+    a.B, a.H, a.T, a.d, a.b, a.io_dtype = 1, 2, 32, 64, 16, ttt.TTT_BF16
+    fake = 1 << 20
+    a.Q = a.K = a.V = a.W_states = a.dQ = a.dK = a.dV = a.dW1 = a.dc1 = a.dW2 = a.dc2 = fake
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(T=30), 1),
+    (dict(b=0), 1),
+    (dict(d=48), 2),
+    (dict(b=32, T=64), 2),                       # the b x 4d intermediates exceed shared memory at d = 64
+    (dict(io_dtype=3), 1),
+    (dict(W_states=None), 1),
+    (dict(dQ=None), 1),
+    (dict(dW1=None), 1),
+    (dict(dc2=(1 << 20) + 4), 1),
+    (dict(dZ=(1 << 20) + 2), 1),
+    (dict(dW2_out=(1 << 20) + 8), 1),
+    (dict(deta=(1 << 20) + 4), 1),
+    (dict(flags=0x1), 1),
+    (dict(B=0, Q=None, dW1=None), 0),
+])
+def test_mlp_backward_validation(ttt_lib, kw, code):
+    a = _mlp_backward_args(ttt_lib, **kw)
+    assert ttt_lib.library().ttt_mlp_backward(ctypes.byref(a), None) == code
+
+
+def test_mlp_forward_states_rules(ttt_lib):
+    L = ttt_lib.library()
+    fake = 1 << 20
+    m = ttt_lib.MlpArgs()
+    m.B, m.H, m.T, m.d, m.b, m.io_dtype = 1, 1, 32, 64, 16, ttt_lib.TTT_BF16
+    m.Q = m.K = m.V = m.Z = m.W1 = m.W2 = m.W1_out = m.W2_out = fake
+    m.W_states = fake + 4                        # misaligned
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
+    m.W_states = fake
+    m.use_ln, m.ln_gamma, m.ln_beta, m.ln_eps = 1, fake, fake, 1e-6
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 2   # no backward of the LN variant
 
 
 def _prologue_args(ttt, **kw):

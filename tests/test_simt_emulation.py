@@ -1,0 +1,120 @@
+"""The fp32 CUDA-core kernels' own source, run on the CPU under a host
+emulation of the CUDA execution model (tests/emulation/simt_emu.cpp: one
+std::thread per CUDA thread, __syncthreads as a barrier, shuffles through a
+per-warp exchange), against the float64 oracle.
+
+This checks the source's index arithmetic, phase order and barrier placement
+where no GPU is present.  It is not the GPU parity: the tests marked gpu run
+the same kernels on the B200 through the C ABI, and the library itself has no
+CPU path.
+
+Covered: the TTT-MLP forward writing its batch-start states and the
+outer-loop backward that reads them (paper digest "论文速览 | TTT",
+sections 3.4, 3.7, 6.12).
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import oracle as O
+from test_sequence_layers_head_b200 import workloads as WL
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "tests", "emulation", "simt_emu.cpp")
+
+
+@pytest.fixture(scope="module")
+def emu(tmp_path_factory):
+    so = str(tmp_path_factory.mktemp("emu") / "simt_emu.so")
+    subprocess.run(["g++", "-std=c++20", "-O1", "-fPIC", "-shared", "-I/usr/local/cuda/include", "-o", so, SRC,
+                    "-lpthread"], check=True)
+    return ctypes.CDLL(so)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def maxrel(x, y):
+    return float(np.max(np.abs(x - y)) / max(np.max(np.abs(y)), 1e-300)) if y.size else 0.0
+
+
+def normwise(x, y):
+    return float(np.linalg.norm((x - y).ravel()) / max(np.linalg.norm(y.ravel()), 1e-300)) if y.size else 0.0
+
+
+CASES = [
+    # B, H, T, d, b, io dtype, eta per token, upstream state gradients
+    (1, 2, 32, 16, 16, WL.F32, True, True),
+    (1, 1, 24, 16, 8, WL.F32, False, False),
+    (2, 1, 20, 16, 4, WL.F32, True, True),
+    (1, 1, 32, 32, 16, WL.F32, True, False),
+    (1, 1, 32, 64, 16, WL.F32, True, True),
+    (1, 1, 32, 64, 16, WL.BF16, True, True),
+    (1, 1, 16, 16, 1, WL.F32, True, True),
+    (1, 1, 0, 16, 16, WL.F32, True, True),
+]
+
+
+@pytest.mark.parametrize("B,H,T,d,b,io,per_token,upstream", CASES)
+def test_mlp_forward_states_and_backward(emu, B, H, T, d, b, io, per_token, upstream):
+    m = 4 * d
+    inp = WL.random_case("mlp", B, H, T, d, b, io_dtype=io, eta_mode="sigmoid", seed=31 + T + d + b)
+    raw, ex = inp.raw, inp.exact
+    rng = np.random.default_rng(7 + d)
+    # non-zero biases (the workloads start them at zero)
+    c1 = (rng.standard_normal((H, m)) * 0.1).astype(np.float32)
+    c2 = (rng.standard_normal((H, d)) * 0.1).astype(np.float32)
+    W1, W2 = raw["W1"], raw["W2"]
+    eta = raw["eta"] if per_token else None
+    eta_const = np.float32(0.02)
+    dZd = rng.standard_normal((B, H, T, d))
+    dZr, dZe = WL.store(dZd, io)
+    ups = ([rng.standard_normal(s).astype(np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+           if upstream else [None] * 4)
+    nb = T // b
+    iot = np.uint16 if io == WL.BF16 else np.float32
+    Z = np.zeros((B, H, T, d), iot)
+    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    dQ, dK, dV = (np.zeros((B, H, T, d), iot) for _ in range(3))
+    deta = np.zeros((B, H, T), np.float32)
+    grads = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    emu.emu_mlp_train.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + \
+        [ctypes.c_void_p] * 23
+    rc = emu.emu_mlp_train(1 if io == WL.BF16 else 0, B, H, T, d, b, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]),
+                           _p(eta), eta_const, _p(W1), _p(c1), _p(W2), _p(c2), _p(dZr), *[_p(u) for u in ups],
+                           _p(Z), *[_p(o) for o in outs], _p(states), _p(dQ), _p(dK), _p(dV), _p(deta),
+                           *[_p(g) for g in grads])
+    assert rc == 0
+
+    f64 = lambda a: a.astype(np.float64)
+    h = WL.bf16_bits_to_f64 if io == WL.BF16 else f64
+    eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(eta_const))
+    params = (f64(W1), f64(c1), f64(W2), f64(c2))
+    ref_f = O.mlp_forward(ex["Q"], ex["K"], ex["V"], eta_e, *params, b)
+    ref_b = O.mlp_backward(ex["Q"], ex["K"], ex["V"], eta_e, *params, b, dZ=dZe,
+                           **{k: (None if u is None else f64(u))
+                              for k, u in zip(("dW1_out", "dc1_out", "dW2_out", "dc2_out"), ups)})
+    # the checkpoints: state i is the oracle's final state after the first i mini-batches
+    for i in sorted({0, nb // 2, nb - 1} if nb else set()):
+        t = i * b
+        st = O.mlp_forward(ex["Q"][:, :, :t], ex["K"][:, :, :t], ex["V"][:, :, :t], eta_e[:, :, :t], *params, b)[1:]
+        got = states[:, :, i]
+        parts = np.split(got, [d * m, d * m + m, 2 * d * m + m], axis=-1)
+        for g, r in zip(parts, st):
+            assert maxrel(f64(g).reshape(r.shape), r) < 1e-4
+
+    names = ["dQ", "dK", "dV", "deta", "dW1", "dc1", "dW2", "dc2"]
+    gots = [h(dQ), h(dK), h(dV), f64(deta)] + [f64(g) for g in grads]
+    for nm, got, ref in zip(names, gots, ref_b):
+        if nm == "deta" and not per_token:
+            continue
+        if io == WL.BF16 and nm in ("dQ", "dK", "dV"):
+            assert normwise(got, ref) < 2e-2, nm      # bf16 outputs: normwise bar
+        else:
+            assert maxrel(got, ref) < 1e-4, (nm, maxrel(got, ref))
+    assert (normwise(h(Z), ref_f[0]) < 2e-2) if io == WL.BF16 else (maxrel(h(Z), ref_f[0]) < 1e-4)
