@@ -788,9 +788,10 @@ def run_b_sweep(args):
 
 
 def run_train(args):
-    """One training step of TTT-Linear (no LN) per timed step: the forward that
-    writes the batch-start states, then the outer-loop backward with random
-    upstream gradients.  Prints one JSON line (not the benchmark line)."""
+    """One training step per timed step, TTT-Linear (no LN) or, with the MLP
+    workload, TTT-MLP: the forward that writes the batch-start states, then
+    the outer-loop backward with random upstream gradients.  Prints one JSON
+    line (not the benchmark line)."""
     import torch
     from test_sequence_layers_head_b200 import ttt
     w = WL.WORKLOADS[args.workload if args.workload != DEFAULT_WORKLOAD else "linear_B8_H12_T2048"]
@@ -798,16 +799,28 @@ def run_train(args):
         w = WL.scaled(w, T=args.T)
     _, dev = device_inputs(w, torch, len(os.sched_getaffinity(0)))
     B, H, T, d = w.B, w.H, w.T, w.d
-    states = torch.empty((B, H, T // w.b, d, d), device="cuda")
     g = torch.Generator(device="cuda")
     g.manual_seed(5)
     dZ = torch.randn(B, H, T, d, generator=g, device="cuda").to(dev["Q"].dtype)
-    dW = torch.randn(B, H, d, d, generator=g, device="cuda")
     eta = dev.get("eta")
+    if w.kind == "mlp":
+        m = w.hidden
+        states = torch.empty((B, H, T // w.b, 2 * d * m + m + d), device="cuda")
 
-    def step():
-        ttt.linear_forward(dev["Q"], dev["K"], dev["V"], eta, dev["W0"], w.b, eta_const=w.eta_const, W_states=states)
-        ttt.linear_backward(dev["Q"], dev["K"], dev["V"], eta, states, w.b, eta_const=w.eta_const, dZ=dZ, dW_out=dW)
+        def step():
+            ttt.mlp_forward(dev["Q"], dev["K"], dev["V"], eta, dev["W1"], dev["c1"], dev["W2"], dev["c2"], w.b,
+                            eta_const=w.eta_const, W_states=states)
+            ttt.mlp_backward(dev["Q"], dev["K"], dev["V"], eta, states, w.b, eta_const=w.eta_const, dZ=dZ,
+                             want_deta=eta is not None)
+    else:
+        states = torch.empty((B, H, T // w.b, d, d), device="cuda")
+        dW = torch.randn(B, H, d, d, generator=g, device="cuda")
+
+        def step():
+            ttt.linear_forward(dev["Q"], dev["K"], dev["V"], eta, dev["W0"], w.b, eta_const=w.eta_const,
+                               W_states=states)
+            ttt.linear_backward(dev["Q"], dev["K"], dev["V"], eta, states, w.b, eta_const=w.eta_const, dZ=dZ,
+                                dW_out=dW)
     per = time_launches(torch, step, args.steps, args.warmup)
     assert ttt.last_device_status() == ttt.TTT_OK
     ms = statistics.mean(per)
@@ -898,7 +911,8 @@ def main():
     ap.add_argument("--b-sweep", action="store_true",
                     help="mini-batch size study (state vs outputs time per b) instead of the benchmark line")
     ap.add_argument("--train", action="store_true",
-                    help="TTT-Linear training step (forward with states + backward) instead of the benchmark line")
+                    help="training step (forward with states + backward; TTT-Linear, or TTT-MLP with the MLP "
+                         "workload) instead of the benchmark line")
     ap.add_argument("--prologue", action="store_true",
                     help="the fused prologue (views and learning-rate gate from the layer input) instead of the "
                          "benchmark line")
