@@ -34,6 +34,11 @@ constexpr int kSmemBytes = kOffDP + 256;
 
 __device__ __forceinline__ uint32_t toff(int row, int chunk) { return row * 128 + ((chunk ^ (row & 7)) << 4); }
 
+// The three warp-collective operations (ldmatrix x4, its transposing form, and
+// the m16n8k16 bf16 MMA).  The CPU test suite's host emulation of these
+// kernels supplies its own definitions, written from the same documented
+// fragment layouts, and defines TTT_HOST_EMULATION.
+#ifndef TTT_HOST_EMULATION
 __device__ __forceinline__ void ldsm4(uint32_t addr, uint32_t* r) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
@@ -50,6 +55,7 @@ __device__ __forceinline__ void mma(float* d, const uint32_t* a, uint32_t b0, ui
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+#endif
 __device__ __forceinline__ uint32_t pk(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&v);

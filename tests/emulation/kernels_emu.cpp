@@ -1,76 +1,22 @@
-// Host emulation of the CUDA execution model for the fp32 CUDA-core (SIMT)
-// kernels' source, used by tests/test_simt_emulation.py.  TEST
-// INFRASTRUCTURE: the library has no CPU path; this file only lets the CPU
-// test suite run the kernels' own source (index arithmetic, phase order,
-// barrier placement) against the float64 oracle where no GPU is present.
-//
-// One CTA at a time: 256 std::threads run the kernel function; __syncthreads
-// is a std::barrier over them, a warp shuffle goes through a per-warp
-// exchange array between two barriers of that warp, and the kernels'
-// dynamic shared array is one static buffer.
-#include <cuda_runtime.h>
-#include <cuda_bf16.h>
+// Entry points of the CPU tests' host emulation of the library's kernels
+// (emu_core.h has the execution model): TEST INFRASTRUCTURE; the library has
+// no CPU path.  Each entry point runs a kernel pair on host arrays exactly as
+// the library launches it on a GPU (one CTA per unit).
+#include "emu_core.h"
 
-#include <barrier>
-#include <cmath>
-#include <thread>
-#include <vector>
-
-namespace emu {
-constexpr int NT = 256;
-thread_local uint3 tid3, bid3;
-std::barrier<>* block_bar = nullptr;
-std::barrier<>* warp_bar[NT / 32];
-float xch[NT / 32][32];
-}  // namespace emu
-
-#undef threadIdx
-#undef blockIdx
-#define threadIdx emu::tid3
-#define blockIdx emu::bid3
-inline void __syncthreads() { emu::block_bar->arrive_and_wait(); }
-inline float __shfl_xor_sync(unsigned, float v, int o) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    emu::xch[w][lane] = v;
-    emu::warp_bar[w]->arrive_and_wait();
-    const float r = emu::xch[w][lane ^ o];
-    emu::warp_bar[w]->arrive_and_wait();
-    return r;
-}
-inline float rsqrtf(float x) { return 1.0f / std::sqrt(x); }
-inline float __expf(float x) { return std::exp(x); }
-inline float __fdividef(float a, float b) { return a / b; }
-#define __launch_bounds__(...)
-#undef __shared__
-#define __shared__
-
-// the kernels declare `extern __shared__ float sm[]` inside namespace ttt
+// the kernels' dynamic shared arrays
 namespace ttt {
-alignas(16) float sm[65536];
+alignas(1024) float sm[65536];
+namespace mbk {
+alignas(1024) uint8_t smem[65536];
 }
+}  // namespace ttt
 
 #include "../../test_sequence_layers_head_b200/csrc/simt.cuh"
 #include "../../test_sequence_layers_head_b200/csrc/simt_mlp_backward.cuh"
+#include "../../test_sequence_layers_head_b200/csrc/mma_forward.cuh"
 
 namespace {
-
-template <typename F>
-void run_grid(int blocks, F f) {
-    for (int bx = 0; bx < blocks; ++bx) {
-        std::barrier<> bb(emu::NT);
-        for (int w = 0; w < emu::NT / 32; ++w) emu::warp_bar[w] = new std::barrier<>(32);
-        emu::block_bar = &bb;
-        std::vector<std::thread> th;
-        for (int t = 0; t < emu::NT; ++t)
-            th.emplace_back([&, t, bx] {
-                emu::tid3 = make_uint3(t, 0, 0);
-                emu::bid3 = make_uint3(bx, 0, 0);
-                f();
-            });
-        for (auto& x : th) x.join();
-        for (int w = 0; w < emu::NT / 32; ++w) delete emu::warp_bar[w];
-    }
-}
 
 // TTT-MLP forward writing the batch-start states, then the backward from them
 template <int D, typename IO>
@@ -101,10 +47,10 @@ int train(int B, int H, int T, int b, const IO* Q, const IO* K, const IO* V, con
     p.W2_out = W2_out;
     p.c2_out = c2_out;
     p.W_states = W_states;
-    run_grid(B * H, [&] { ttt::simt_mlp_kernel<D, IO, false>(p); });
+    emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { ttt::simt_mlp_kernel<D, IO, false>(p); });
     ttt::SimtMlpBackwardParams q{H,  T,  b,  Q,     K,     V,     eta,  eta_const, W_states, dZ,  dW1o,
                                  dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1, dc1, dW2, dc2};
-    run_grid(B * H, [&] { ttt::simt_mlp_backward_kernel<D, IO>(q); });
+    emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { ttt::simt_mlp_backward_kernel<D, IO>(q); });
     return 0;
 }
 
@@ -139,4 +85,19 @@ extern "C" int emu_mlp_train(int io, int B, int H, int T, int d, int b, const vo
         }
     }
     return 1;
+}
+
+// TTT-Linear training on the tensor-core (mma.sync) kernels, bf16, d = 64, b = 16:
+// the forward writing the batch-start states, then the backward
+extern "C" int emu_linear_train_mma(int B, int H, int T, const void* Q, const void* K, const void* V,
+                                    const float* eta, float eta_const, const float* W0, long long W0_bstride,
+                                    void* Z, float* W_out, float* W_states, const void* dZ, const float* dW_out,
+                                    void* dQ, void* dK, void* dV, float* deta, float* dW0) {
+    using namespace ttt::mbk;
+    if (kFSmemBytes > (int)sizeof(smem) || kSmemBytes > (int)sizeof(smem)) return 2;
+    FwdStatesParams f{H, T, Q, K, V, eta, eta_const, W0, W0_bstride, Z, W_out, W_states};
+    emu::run_grid(B * H, kThreads, smem, [&] { mma_linear_forward_states_kernel(f); });
+    ttt::SimtBackwardParams p{H, T, 16, Q, K, V, eta, eta_const, W_states, dZ, dW_out, dQ, dK, dV, deta, dW0};
+    emu::run_grid(B * H, kThreads, smem, [&] { mma_linear_backward_kernel(p); });
+    return 0;
 }

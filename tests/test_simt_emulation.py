@@ -1,7 +1,8 @@
-"""The fp32 CUDA-core kernels' own source, run on the CPU under a host
-emulation of the CUDA execution model (tests/emulation/simt_emu.cpp: one
-std::thread per CUDA thread, __syncthreads as a barrier, shuffles through a
-per-warp exchange), against the float64 oracle.
+"""The library's CUDA-core and mma.sync kernels' own source, run on the CPU
+under a host emulation of the CUDA execution model (tests/emulation: one
+std::thread per CUDA thread, __syncthreads as a barrier, shuffles, ldmatrix
+and mma through a per-warp exchange with the PTX ISA's documented fragment
+layouts), against the float64 oracle.
 
 This checks the source's index arithmetic, phase order and barrier placement
 where no GPU is present.  It is not the GPU parity: the tests marked gpu run
@@ -9,8 +10,10 @@ the same kernels on the B200 through the C ABI, and the library itself has no
 CPU path.
 
 Covered: the TTT-MLP forward writing its batch-start states and the
-outer-loop backward that reads them (paper digest "论文速览 | TTT",
-sections 3.4, 3.7, 6.12).
+outer-loop backward that reads them (fp32 CUDA cores), and the TTT-Linear
+pair on mma.sync (bf16, d = 64, b = 16) -- already verified on the B200,
+which pins the emulated ldmatrix / mma semantics (paper digest
+"论文速览 | TTT", sections 3.4, 3.6, 3.7, 6.12).
 """
 import ctypes
 import os
@@ -23,12 +26,12 @@ from oracle import oracle as O
 from test_sequence_layers_head_b200 import workloads as WL
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-SRC = os.path.join(ROOT, "tests", "emulation", "simt_emu.cpp")
+SRC = os.path.join(ROOT, "tests", "emulation", "kernels_emu.cpp")
 
 
 @pytest.fixture(scope="module")
 def emu(tmp_path_factory):
-    so = str(tmp_path_factory.mktemp("emu") / "simt_emu.so")
+    so = str(tmp_path_factory.mktemp("emu") / "kernels_emu.so")
     subprocess.run(["g++", "-std=c++20", "-O1", "-fPIC", "-shared", "-I/usr/local/cuda/include", "-o", so, SRC,
                     "-lpthread"], check=True)
     return ctypes.CDLL(so)
@@ -118,3 +121,46 @@ def test_mlp_forward_states_and_backward(emu, B, H, T, d, b, io, per_token, upst
         else:
             assert maxrel(got, ref) < 1e-4, (nm, maxrel(got, ref))
     assert (normwise(h(Z), ref_f[0]) < 2e-2) if io == WL.BF16 else (maxrel(h(Z), ref_f[0]) < 1e-4)
+
+
+@pytest.mark.parametrize("B,H,T,per_token,upstream", [(1, 2, 64, True, True), (2, 1, 48, False, False),
+                                                     (1, 1, 16, True, True)])
+def test_linear_training_on_mma_sync(emu, B, H, T, per_token, upstream):
+    d, b = 64, 16
+    inp = WL.random_case("linear", B, H, T, d, b, io_dtype=WL.BF16, eta_mode="sigmoid" if per_token else "const",
+                         eta_const=0.0 if per_token else 0.05, seed=T + B)
+    raw, ex = inp.raw, inp.exact
+    rng = np.random.default_rng(T)
+    dZr, dZe = WL.store(rng.standard_normal((B, H, T, d)), WL.BF16)
+    dW = rng.standard_normal((B, H, d, d)).astype(np.float32) if upstream else None
+    nb = T // b
+    Z = np.zeros((B, H, T, d), np.uint16)
+    W_out = np.zeros((B, H, d, d), np.float32)
+    states = np.zeros((B, H, nb, d, d), np.float32)
+    dQ, dK, dV = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
+    deta = np.zeros((B, H, T), np.float32)
+    dW0 = np.zeros((B, H, d, d), np.float32)
+    eta = raw["eta"] if per_token else None
+    f = emu.emu_linear_train_mma
+    f.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_longlong] + \
+        [ctypes.c_void_p] * 10
+    assert f(B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const),
+             _p(raw["W0"]), 0, _p(Z), _p(W_out), _p(states), _p(dZr), _p(dW), _p(dQ), _p(dK), _p(dV), _p(deta),
+             _p(dW0)) == 0
+    eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(inp.w.eta_const)))
+    Zr, Wr, _ = O.linear_forward(ex["Q"], ex["K"], ex["V"], eta_e, ex["W0"], b)
+    assert normwise(WL.bf16_bits_to_f64(Z), Zr) < 2e-2
+    assert normwise(W_out.astype(np.float64), Wr) < 2e-2
+    for i in range(nb):
+        t = i * b
+        Wi = O.linear_forward(ex["Q"][:, :, :t], ex["K"][:, :, :t], ex["V"][:, :, :t], eta_e[:, :, :t], ex["W0"],
+                              b)[1]
+        assert normwise(states[:, :, i].astype(np.float64), Wi) < 2e-2
+    ref = O.linear_backward(ex["Q"], ex["K"], ex["V"], eta_e, ex["W0"], b, dZ=dZe,
+                            dW_out=None if dW is None else dW.astype(np.float64))
+    gots = [WL.bf16_bits_to_f64(dQ), WL.bf16_bits_to_f64(dK), WL.bf16_bits_to_f64(dV), deta.astype(np.float64),
+            dW0.astype(np.float64)]
+    for nm, got, want in zip(("dQ", "dK", "dV", "deta", "dW0"), gots, ref):
+        if nm == "deta" and not per_token:
+            continue
+        assert normwise(got, want) < 2e-2, (nm, normwise(got, want))
