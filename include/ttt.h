@@ -58,6 +58,9 @@ typedef enum { TTT_F32 = 0, TTT_BF16 = 1 } ttt_dtype;
 #define TTT_FLAG_FORCE_SIMT 0x1u   /* use the fp32 CUDA-core kernel even where the tensor-core one applies */
 #define TTT_FLAG_ONE_UNIT_PER_CTA 0x2u  /* tensor-core linear kernel: one (sequence, head) unit per CTA */
 #define TTT_FLAG_TWO_UNITS_PER_CTA 0x4u /* tensor-core linear kernel: two units per CTA */
+#define TTT_FLAG_LN_MMA_TRAINING 0x8u /* LN+residual training (ttt_linear_forward with W_states, ttt_linear_backward)
+                                        on the mma.sync tensor-core kernels (BF16, d = 64, b = 16); without it those
+                                        calls run on the fp32 CUDA-core kernels */
 #define TTT_FLAG_TEST_STALL 0x100u /* test hook: one device wait is made to expire (see ttt_last_device_status) */
 /* Without either UNITS_PER_CTA flag the library takes one unit per CTA when
  * B*H <= 148 (the SM count: the work is a serial chain per unit, and one unit

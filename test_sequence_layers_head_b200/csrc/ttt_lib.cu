@@ -19,6 +19,7 @@
 #include "simt_mlp_backward.cuh"
 #include "mma_backward.cuh"
 #include "mma_forward.cuh"
+#include "mma_ln.cuh"
 #include "prologue.cuh"
 #include "tmap.h"
 
@@ -203,13 +204,24 @@ extern "C" ttt_status ttt_linear_forward(const ttt_linear_args* a, cudaStream_t 
         if (!(a->ln_eps > 0.f)) return TTT_ERR_INVALID_ARG;
     }
     if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_TEST_STALL | TTT_FLAG_ONE_UNIT_PER_CTA |
-                     TTT_FLAG_TWO_UNITS_PER_CTA))
+                     TTT_FLAG_TWO_UNITS_PER_CTA | TTT_FLAG_LN_MMA_TRAINING))
         return TTT_ERR_INVALID_ARG;
     if ((a->flags & TTT_FLAG_ONE_UNIT_PER_CTA) && (a->flags & TTT_FLAG_TWO_UNITS_PER_CTA))
         return TTT_ERR_INVALID_ARG;
     if (a->W_states) {
         if (!aligned16(a->W_states)) return TTT_ERR_INVALID_ARG;
         if (a->use_ln && !ok_ptr(a->c_states)) return TTT_ERR_INVALID_ARG;
+    }
+    if (a->W_states && a->use_ln && (a->flags & TTT_FLAG_LN_MMA_TRAINING) && a->io_dtype == TTT_BF16 &&
+        a->d == 64 && a->b == 16 && a->T > 0 && !(a->flags & TTT_FLAG_FORCE_SIMT)) {
+        // LN+residual training on mma.sync: the forward that writes (W, c) at every mini-batch start
+        if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
+        mbk::FwdLnStatesParams p{a->H,      a->T,          a->Q,    a->K,          a->V,        a->eta,
+                                 a->eta_const, a->W0,      a->W0_bstride, a->c0,   a->c0_bstride, a->ln_gamma,
+                                 a->ln_beta, a->ln_eps,    a->Z,    a->W_out,      a->c_out,    a->W_states,
+                                 a->c_states};
+        mbk::mma_ln_forward_states_kernel<<<(unsigned)units, mbk::kThreads, mbk::kLFSmemBytes, stream>>>(p);
+        return launch_status();
     }
     const bool states_on_simt = a->W_states && a->use_ln;   // the LN states come from the fp32 kernel
     const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 && a->Z &&
@@ -471,12 +483,21 @@ extern "C" ttt_status ttt_linear_backward(const ttt_linear_backward_args* a, cud
         return TTT_ERR_INVALID_ARG;
     if (!ok_ptr(a->dW0) || !ok_opt(a->eta) || !ok_opt(a->dZ) || !ok_opt(a->dW_out) || !ok_opt(a->deta))
         return TTT_ERR_INVALID_ARG;
-    if (a->flags & ~TTT_FLAG_FORCE_SIMT) return TTT_ERR_INVALID_ARG;
+    if (a->flags & ~(TTT_FLAG_FORCE_SIMT | TTT_FLAG_LN_MMA_TRAINING)) return TTT_ERR_INVALID_ARG;
     if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
     if (a->use_ln) {
         if ((a->T > 0 && !ok_ptr(a->c_states)) || !ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) ||
             !(a->ln_eps > 0.f) || !ok_opt(a->dc_out) || !ok_ptr(a->dc0) || !ok_ptr(a->dgamma) || !ok_ptr(a->dbeta))
             return TTT_ERR_INVALID_ARG;
+        if ((a->flags & TTT_FLAG_LN_MMA_TRAINING) && !(a->flags & TTT_FLAG_FORCE_SIMT) && a->io_dtype == TTT_BF16 &&
+            a->d == 64 && a->b == 16) {
+            SimtLnBackwardParams p{a->H,      a->T,      a->b,     a->Q,      a->K,      a->V,
+                                   a->eta,    a->eta_const, a->W_states, a->c_states, a->ln_gamma, a->ln_beta,
+                                   a->ln_eps, a->dZ,     a->dW_out, a->dc_out, a->dQ,     a->dK,
+                                   a->dV,     a->deta,   a->dW0,   a->dc0,    a->dgamma, a->dbeta};
+            mbk::mma_ln_backward_kernel<<<(unsigned)units, mbk::kThreads, mbk::kLBSmemBytes, stream>>>(p);
+            return launch_status();
+        }
         switch (a->d) {
             case 16: return launch_ln_backward<16>(a, stream);
             case 32: return launch_ln_backward<32>(a, stream);

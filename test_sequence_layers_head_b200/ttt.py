@@ -24,6 +24,7 @@ TTT_F32, TTT_BF16 = 0, 1
 FLAG_FORCE_SIMT = 0x1
 FLAG_ONE_UNIT_PER_CTA = 0x2
 FLAG_TWO_UNITS_PER_CTA = 0x4
+FLAG_LN_MMA_TRAINING = 0x8
 FLAG_TEST_STALL = 0x100
 
 _vp = ctypes.c_void_p

@@ -15,6 +15,7 @@ alignas(1024) uint8_t smem[65536];
 #include "../../test_sequence_layers_head_b200/csrc/simt.cuh"
 #include "../../test_sequence_layers_head_b200/csrc/simt_mlp_backward.cuh"
 #include "../../test_sequence_layers_head_b200/csrc/mma_forward.cuh"
+#include "../../test_sequence_layers_head_b200/csrc/mma_ln.cuh"
 
 namespace {
 
@@ -99,5 +100,38 @@ extern "C" int emu_linear_train_mma(int B, int H, int T, const void* Q, const vo
     emu::run_grid(B * H, kThreads, smem, [&] { mma_linear_forward_states_kernel(f); });
     ttt::SimtBackwardParams p{H, T, 16, Q, K, V, eta, eta_const, W_states, dZ, dW_out, dQ, dK, dV, deta, dW0};
     emu::run_grid(B * H, kThreads, smem, [&] { mma_linear_backward_kernel(p); });
+    return 0;
+}
+
+// TTT-Linear with LN+residual on the tensor-core (mma.sync) kernels, bf16, d = 64, b = 16: the forward
+// writing the batch-start states (W, c)
+extern "C" int emu_ln_forward_mma(int B, int H, int T, const void* Q, const void* K, const void* V, const float* eta,
+                                  float eta_const, const float* W0, const float* c0, const float* gamma,
+                                  const float* beta, float eps, void* Z, float* W_out, float* c_out, float* W_states,
+                                  float* c_states) {
+    using namespace ttt::mbk;
+    if (kLFSmemBytes > (int)sizeof(smem)) return 2;
+    FwdLnStatesParams f{H, T, Q, K, V, eta, eta_const, W0, 0, c0, 0, gamma, beta, eps, Z, W_out, c_out,
+                        W_states, c_states};
+    emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_forward_states_kernel(f); });
+    return 0;
+}
+
+// TTT-Linear with LN+residual on the tensor-core (mma.sync) kernels: the forward writing the batch-start
+// states, then the backward from them
+extern "C" int emu_ln_train_mma(int B, int H, int T, const void* Q, const void* K, const void* V, const float* eta,
+                                float eta_const, const float* W0, const float* c0, const float* gamma,
+                                const float* beta, float eps, float* W_out, float* c_out, float* W_states,
+                                float* c_states, const void* dZ, const float* dW_out, const float* dc_out, void* dQ,
+                                void* dK, void* dV, float* deta, float* dW0, float* dc0, float* dgamma,
+                                float* dbeta) {
+    using namespace ttt::mbk;
+    if (kLFSmemBytes > (int)sizeof(smem) || kLBSmemBytes > (int)sizeof(smem)) return 2;
+    FwdLnStatesParams f{H, T, Q, K, V, eta, eta_const, W0, 0, c0, 0, gamma, beta, eps, nullptr, W_out, c_out,
+                        W_states, c_states};
+    emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_forward_states_kernel(f); });
+    ttt::SimtLnBackwardParams q{H,  T,  16, Q,  K,      V,      eta,    eta_const, W_states, c_states, gamma, beta,
+                                eps, dZ, dW_out, dc_out, dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta};
+    emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_backward_kernel(q); });
     return 0;
 }

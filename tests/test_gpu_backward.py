@@ -232,3 +232,51 @@ def test_ln_backward_matches_oracle(ttt_lib, d, b, T, io):
                                eps=w.ln_eps, dZ=dz[1], dW_out=dw[1], dc_out=dc[1])
     for name, g, o in zip(("dQ", "dK", "dV", "deta", "dW0", "dc0", "dgamma", "dbeta"), out, ref):
         assert_close(name, to_host(g), o, io)
+
+
+@pytest.mark.skip(reason="mma.sync LN+residual training kernels: first supervised B200 run pending")
+@pytest.mark.parametrize("B,H,T,per_token", [(2, 3, 64, True), (1, 2, 48, False), (2, 2, 256, True)])
+def test_ln_training_on_mma_sync(ttt_lib, B, H, T, per_token):
+    """TTT_FLAG_LN_MMA_TRAINING: the LN+residual forward with states and the
+    backward on the mma.sync kernels (bf16, d = 64, b = 16) against the oracle,
+    with a non-zero initial bias and every upstream gradient."""
+    d, b = 64, 16
+    inp = WL.random_case("ln", B, H, T, d, b, io_dtype=WL.BF16, eta_mode="sigmoid" if per_token else "const",
+                         eta_const=0.0 if per_token else 0.05, seed=T + H)
+    r, e, w = inp.raw, inp.exact, inp.w
+    rng = np.random.default_rng(T)
+    c0r, c0e = WL.store(rng.standard_normal((H, d)) * 0.1, WL.F32)
+    Q, K, V, W0, gam, bet = (to_dev(r[n]) for n in ("Q", "K", "V", "W0", "gamma", "beta"))
+    eta = to_dev(r["eta"]) if per_token else None
+    c0 = to_dev(c0r)
+    flags = ttt_lib.FLAG_LN_MMA_TRAINING
+    states = torch.full((B, H, T // b, d, d), float("nan"), device="cuda")
+    cst = torch.full((B, H, T // b, d), float("nan"), device="cuda")
+    Z, Wout, cout = ttt_lib.linear_forward(Q, K, V, eta, W0, b, eta_const=w.eta_const, use_ln=True, c0=c0, gamma=gam,
+                                           beta=bet, eps=w.ln_eps, W_states=states, c_states=cst, flags=flags)
+    dz = WL.store(rng.standard_normal((B, H, T, d)), WL.BF16)
+    dw = WL.store(rng.standard_normal((B, H, d, d)), WL.F32)
+    dc = WL.store(rng.standard_normal((B, H, d)), WL.F32)
+    out = ttt_lib.linear_backward(Q, K, V, eta, states, b, eta_const=w.eta_const, dZ=to_dev(dz[0]),
+                                  dW_out=to_dev(dw[0]), use_ln=True, c_states=cst, gamma=gam, beta=bet,
+                                  eps=w.ln_eps, dc_out=to_dev(dc[0]), flags=flags)
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    eta_e = e["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(w.eta_const)))
+    Zo, Wo, co = O.linear_forward(e["Q"], e["K"], e["V"], eta_e, e["W0"], b, c0=c0e, gamma=e["gamma"],
+                                  beta=e["beta"], use_ln=True, eps=w.ln_eps)
+    assert_close("Z", to_host(Z), Zo, WL.BF16)
+    assert_close("W_out", to_host(Wout), Wo, WL.BF16)
+    assert_close("c_out", to_host(cout), co, WL.BF16)
+    for i in (1, T // b - 1):
+        t = i * b
+        _, Wi, ci = O.linear_forward(e["Q"][:, :, :t], e["K"][:, :, :t], e["V"][:, :, :t], eta_e[:, :, :t], e["W0"],
+                                     b, c0=c0e, gamma=e["gamma"], beta=e["beta"], use_ln=True, eps=w.ln_eps)
+        assert_close("W_states", to_host(states[:, :, i]), Wi, WL.BF16)
+        assert_close("c_states", to_host(cst[:, :, i]), ci, WL.BF16)
+    ref = O.linear_ln_backward(e["Q"], e["K"], e["V"], eta_e, e["W0"], b, c0e, e["gamma"], e["beta"],
+                               eps=w.ln_eps, dZ=dz[1], dW_out=dw[1], dc_out=dc[1])
+    for name, g, o in zip(("dQ", "dK", "dV", "deta", "dW0", "dc0", "dgamma", "dbeta"), out, ref):
+        if g is None:
+            continue
+        assert_close(name, to_host(g), o, WL.BF16)

@@ -10,10 +10,10 @@ the same kernels on the B200 through the C ABI, and the library itself has no
 CPU path.
 
 Covered: the TTT-MLP forward writing its batch-start states and the
-outer-loop backward that reads them (fp32 CUDA cores), and the TTT-Linear
-pair on mma.sync (bf16, d = 64, b = 16) -- already verified on the B200,
-which pins the emulated ldmatrix / mma semantics (paper digest
-"论文速览 | TTT", sections 3.4, 3.6, 3.7, 6.12).
+outer-loop backward that reads them (fp32 CUDA cores); the TTT-Linear pair
+on mma.sync (bf16, d = 64, b = 16) -- already verified on the B200, which
+pins the emulated ldmatrix / mma semantics; and the LN+residual pair on
+mma.sync (paper digest "论文速览 | TTT", sections 3.4, 3.6, 3.7, 4.4, 6.12).
 """
 import ctypes
 import os
@@ -161,6 +161,56 @@ def test_linear_training_on_mma_sync(emu, B, H, T, per_token, upstream):
     gots = [WL.bf16_bits_to_f64(dQ), WL.bf16_bits_to_f64(dK), WL.bf16_bits_to_f64(dV), deta.astype(np.float64),
             dW0.astype(np.float64)]
     for nm, got, want in zip(("dQ", "dK", "dV", "deta", "dW0"), gots, ref):
+        if nm == "deta" and not per_token:
+            continue
+        assert normwise(got, want) < 2e-2, (nm, normwise(got, want))
+
+
+@pytest.mark.parametrize("B,H,T,per_token,upstream", [(1, 2, 64, True, True), (2, 1, 48, False, False),
+                                                     (1, 1, 16, True, True)])
+def test_ln_training_on_mma_sync(emu, B, H, T, per_token, upstream):
+    d, b = 64, 16
+    inp = WL.random_case("ln", B, H, T, d, b, io_dtype=WL.BF16, eta_mode="sigmoid" if per_token else "const",
+                         eta_const=0.0 if per_token else 0.05, seed=5 + T)
+    raw, ex = inp.raw, inp.exact
+    rng = np.random.default_rng(1 + T)
+    c0 = (rng.standard_normal((H, d)) * 0.1).astype(np.float32)
+    dZr, dZe = WL.store(rng.standard_normal((B, H, T, d)), WL.BF16)
+    dWo = rng.standard_normal((B, H, d, d)).astype(np.float32) if upstream else None
+    dco = rng.standard_normal((B, H, d)).astype(np.float32) if upstream else None
+    nb = T // b
+    W_out, c_out = np.zeros((B, H, d, d), np.float32), np.zeros((B, H, d), np.float32)
+    Ws, cs = np.zeros((B, H, nb, d, d), np.float32), np.zeros((B, H, nb, d), np.float32)
+    dQ, dK, dV = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
+    deta = np.zeros((B, H, T), np.float32)
+    dW0 = np.zeros((B, H, d, d), np.float32)
+    dc0, dgam, dbet = (np.zeros((B, H, d), np.float32) for _ in range(3))
+    f = emu.emu_ln_train_mma
+    f.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 4 + \
+        [ctypes.c_float] + [ctypes.c_void_p] * 15
+    eta = raw["eta"] if per_token else None
+    assert f(B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const),
+             _p(raw["W0"]), _p(c0), _p(raw["gamma"]), _p(raw["beta"]), np.float32(inp.w.ln_eps), _p(W_out),
+             _p(c_out), _p(Ws), _p(cs), _p(dZr), _p(dWo), _p(dco), _p(dQ), _p(dK), _p(dV), _p(deta), _p(dW0),
+             _p(dc0), _p(dgam), _p(dbet)) == 0
+    eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(inp.w.eta_const)))
+    c0e = c0.astype(np.float64)
+    _, Wr, cr = O.linear_forward(ex["Q"], ex["K"], ex["V"], eta_e, ex["W0"], b, c0=c0e, gamma=ex["gamma"],
+                                 beta=ex["beta"], use_ln=True, eps=inp.w.ln_eps)
+    assert normwise(W_out.astype(np.float64), Wr) < 2e-2 and normwise(c_out.astype(np.float64), cr) < 2e-2
+    for i in range(1, nb):
+        t = i * b
+        _, Wi, ci = O.linear_forward(ex["Q"][:, :, :t], ex["K"][:, :, :t], ex["V"][:, :, :t], eta_e[:, :, :t],
+                                     ex["W0"], b, c0=c0e, gamma=ex["gamma"], beta=ex["beta"], use_ln=True,
+                                     eps=inp.w.ln_eps)
+        assert normwise(Ws[:, :, i].astype(np.float64), Wi) < 2e-2
+        assert normwise(cs[:, :, i].astype(np.float64), ci) < 2e-2
+    ref = O.linear_ln_backward(ex["Q"], ex["K"], ex["V"], eta_e, ex["W0"], b, c0e, ex["gamma"], ex["beta"],
+                               inp.w.ln_eps, dZ=dZe, dW_out=None if dWo is None else dWo.astype(np.float64),
+                               dc_out=None if dco is None else dco.astype(np.float64))
+    h = WL.bf16_bits_to_f64
+    gots = [h(dQ), h(dK), h(dV), deta.astype(np.float64)] + [x.astype(np.float64) for x in (dW0, dc0, dgam, dbet)]
+    for nm, got, want in zip(("dQ", "dK", "dV", "deta", "dW0", "dc0", "dgamma", "dbeta"), gots, ref):
         if nm == "deta" and not per_token:
             continue
         assert normwise(got, want) < 2e-2, (nm, normwise(got, want))
