@@ -788,10 +788,10 @@ def run_b_sweep(args):
 
 
 def run_train(args):
-    """One training step per timed step, TTT-Linear (no LN) or, with the MLP
-    workload, TTT-MLP: the forward that writes the batch-start states, then
-    the outer-loop backward with random upstream gradients.  Prints one JSON
-    line (not the benchmark line)."""
+    """One training step per timed step: TTT-Linear (no LN), or, on the LN and
+    MLP workloads, TTT-Linear with LN+residual and TTT-MLP: the forward that
+    writes the batch-start states, then the outer-loop backward with random
+    upstream gradients.  Prints one JSON line (not the benchmark line)."""
     import torch
     from test_sequence_layers_head_b200 import ttt
     w = WL.WORKLOADS[args.workload if args.workload != DEFAULT_WORKLOAD else "linear_B8_H12_T2048"]
@@ -812,6 +812,19 @@ def run_train(args):
                             eta_const=w.eta_const, W_states=states)
             ttt.mlp_backward(dev["Q"], dev["K"], dev["V"], eta, states, w.b, eta_const=w.eta_const, dZ=dZ,
                              want_deta=eta is not None)
+    elif w.kind == "ln":
+        states = torch.empty((B, H, T // w.b, d, d), device="cuda")
+        cst = torch.empty((B, H, T // w.b, d), device="cuda")
+        dW = torch.randn(B, H, d, d, generator=g, device="cuda")
+        dc = torch.randn(B, H, d, generator=g, device="cuda")
+        flags = ttt.FLAG_LN_MMA_TRAINING if args.ln_mma else 0
+        ln = dict(use_ln=True, gamma=dev["gamma"], beta=dev["beta"], eps=w.ln_eps, flags=flags)
+
+        def step():
+            ttt.linear_forward(dev["Q"], dev["K"], dev["V"], eta, dev["W0"], w.b, eta_const=w.eta_const, c0=dev["c0"],
+                               W_states=states, c_states=cst, **ln)
+            ttt.linear_backward(dev["Q"], dev["K"], dev["V"], eta, states, w.b, eta_const=w.eta_const, dZ=dZ,
+                                dW_out=dW, c_states=cst, dc_out=dc, **ln)
     else:
         states = torch.empty((B, H, T // w.b, d, d), device="cuda")
         dW = torch.randn(B, H, d, d, generator=g, device="cuda")
@@ -824,9 +837,11 @@ def run_train(args):
     per = time_launches(torch, step, args.steps, args.warmup)
     assert ttt.last_device_status() == ttt.TTT_OK
     ms = statistics.mean(per)
+    kernels = "forward with states, then the backward"
+    if w.kind == "ln":
+        kernels += " (mma.sync LN kernels)" if args.ln_mma else " (fp32 CUDA-core LN kernels)"
     print(json.dumps({"train_step_ms": ms, "tokens_per_s": tokens(w) / (ms / 1000.0), "workload": w.name,
-                      "steps": args.steps, "warmup": args.warmup,
-                      "kernels": "forward with states, then the backward"}), flush=True)
+                      "steps": args.steps, "warmup": args.warmup, "kernels": kernels}), flush=True)
 
 
 def prologue_flops(w) -> int:
@@ -913,6 +928,8 @@ def main():
     ap.add_argument("--train", action="store_true",
                     help="training step (forward with states + backward; TTT-Linear, or TTT-MLP with the MLP "
                          "workload) instead of the benchmark line")
+    ap.add_argument("--ln-mma", action="store_true",
+                    help="with --train on the LN workload: the mma.sync LN training kernels")
     ap.add_argument("--prologue", action="store_true",
                     help="the fused prologue (views and learning-rate gate from the layer input) instead of the "
                          "benchmark line")
