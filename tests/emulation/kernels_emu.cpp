@@ -135,3 +135,72 @@ extern "C" int emu_ln_train_mma(int B, int H, int T, const void* Q, const void* 
     emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_backward_kernel(q); });
     return 0;
 }
+
+// The same kernels one launch at a time (the tests' dry runs call them as the library would)
+extern "C" int emu_mlp_forward(int io, int B, int H, int T, int d, int b, const void* Q, const void* K, const void* V,
+                               const float* eta, float eta_const, const float* W1, const float* c1, const float* W2,
+                               const float* c2, void* Z, float* W1_out, float* c1_out, float* W2_out, float* c2_out,
+                               float* W_states) {
+    ttt::SimtMlpParams p{};
+    p.H = H;
+    p.T = T;
+    p.b = b;
+    p.Q = Q;
+    p.K = K;
+    p.V = V;
+    p.eta = eta;
+    p.eta_const = eta_const;
+    p.W1 = W1;
+    p.c1 = c1;
+    p.W2 = W2;
+    p.c2 = c2;
+    p.Z = Z;
+    p.W1_out = W1_out;
+    p.c1_out = c1_out;
+    p.W2_out = W2_out;
+    p.c2_out = c2_out;
+    p.W_states = W_states;
+    if (ttt::simt_mlp_smem(d, b, false) > sizeof(ttt::sm)) return 2;
+    auto run = [&](auto kernel) { emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { kernel(p); }); };
+    if (io == 0) {
+        if (d == 16) run(ttt::simt_mlp_kernel<16, float, false>);
+        else if (d == 32) run(ttt::simt_mlp_kernel<32, float, false>);
+        else run(ttt::simt_mlp_kernel<64, float, false>);
+    } else {
+        if (d == 16) run(ttt::simt_mlp_kernel<16, __nv_bfloat16, false>);
+        else if (d == 32) run(ttt::simt_mlp_kernel<32, __nv_bfloat16, false>);
+        else run(ttt::simt_mlp_kernel<64, __nv_bfloat16, false>);
+    }
+    return 0;
+}
+extern "C" int emu_mlp_backward(int io, int B, int H, int T, int d, int b, const void* Q, const void* K,
+                                const void* V, const float* eta, float eta_const, const float* W_states,
+                                const void* dZ, const float* dW1o, const float* dc1o, const float* dW2o,
+                                const float* dc2o, void* dQ, void* dK, void* dV, float* deta, float* dW1, float* dc1,
+                                float* dW2, float* dc2) {
+    ttt::SimtMlpBackwardParams q{H,    T,    b,  Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
+                                 dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2};
+    if (ttt::simt_mlp_backward_smem(d, b) > sizeof(ttt::sm)) return 2;
+    auto run = [&](auto kernel) { emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { kernel(q); }); };
+    if (io == 0) {
+        if (d == 16) run(ttt::simt_mlp_backward_kernel<16, float>);
+        else if (d == 32) run(ttt::simt_mlp_backward_kernel<32, float>);
+        else run(ttt::simt_mlp_backward_kernel<64, float>);
+    } else {
+        if (d == 16) run(ttt::simt_mlp_backward_kernel<16, __nv_bfloat16>);
+        else if (d == 32) run(ttt::simt_mlp_backward_kernel<32, __nv_bfloat16>);
+        else run(ttt::simt_mlp_backward_kernel<64, __nv_bfloat16>);
+    }
+    return 0;
+}
+extern "C" int emu_ln_backward_mma(int B, int H, int T, const void* Q, const void* K, const void* V, const float* eta,
+                                   float eta_const, const float* W_states, const float* c_states, const float* gamma,
+                                   const float* beta, float eps, const void* dZ, const float* dW_out,
+                                   const float* dc_out, void* dQ, void* dK, void* dV, float* deta, float* dW0,
+                                   float* dc0, float* dgamma, float* dbeta) {
+    using namespace ttt::mbk;
+    ttt::SimtLnBackwardParams q{H,  T,  16, Q,  K,      V,      eta,    eta_const, W_states, c_states, gamma, beta,
+                                eps, dZ, dW_out, dc_out, dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta};
+    emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_backward_kernel(q); });
+    return 0;
+}
