@@ -391,16 +391,16 @@ ttt_status ttt_mlp_decode_step(const ttt_mlp_decode_args* args, cudaStream_t str
  * theta_Q x_t) and the learnable per-token learning rate (section 4.6):
  *     Q[n,h,t,j] = sum_k theta_q[h d + j, k] x[n,t,k]      (K, V alike)
  *     eta[n,h,t] = eta_base * sigmoid(sum_k theta_lr[h,k] x[n,t,k])
- * One dense contraction on the tensor cores (bf16 operands, fp32
- * accumulation); the epilogue writes each view in the [B, H, T, d] layout
- * that the inner-loop entry points read, rounded once to bf16, and applies
- * the gate in fp32.
+ * For BF16 input, one dense contraction on the tensor cores (bf16 operands,
+ * fp32 accumulation); the epilogue writes each view in the [B, H, T, d]
+ * layout that the inner-loop entry points read, rounded once to bf16, and
+ * applies the gate in fp32.  F32 input (and BF16 with TTT_FLAG_FORCE_SIMT)
+ * runs on fp32 CUDA cores.
  *
  *   B, T           sequences and tokens per sequence (any T >= 0).
  *   Dm             width of the layer input; Dm % 8 == 0 (16-byte rows).
  *   H, d           heads and head dim; d in {16, 32, 64}, 1 <= H <= 256.
- *   io_dtype       BF16 (x, the theta matrices and Q, K, V); F32 is
- *                  TTT_ERR_UNSUPPORTED.
+ *   io_dtype       BF16 or F32: x, the theta matrices and Q, K, V.
  *   x              [B, T, Dm].
  *   theta_q, theta_k, theta_v
  *                  [H*d, Dm] each, the pages' column form: head h owns rows
@@ -410,7 +410,8 @@ ttt_status ttt_mlp_decode_step(const ttt_mlp_decode_args* args, cudaStream_t str
  *                  inner-loop entry points (twice the pages' value).
  *   Q, K, V        outputs [B, H, T, d] in io_dtype.
  *   eta            output [B, H, T] fp32, or NULL with theta_lr NULL.
- *   flags          TTT_FLAG_TEST_STALL; any other bit is TTT_ERR_INVALID_ARG.
+ *   flags          TTT_FLAG_FORCE_SIMT, TTT_FLAG_TEST_STALL (tensor-core
+ *                  kernel only); any other bit is TTT_ERR_INVALID_ARG.
  *   wait_timeout_ms  limit of one device-side wait (0: 2000 ms).
  * Outputs must not overlap the inputs.
  */

@@ -21,6 +21,7 @@
 #include "mma_forward.cuh"
 #include "mma_ln.cuh"
 #include "prologue.cuh"
+#include "simt_prologue.cuh"
 #include "tmap.h"
 
 namespace ttt {
@@ -569,8 +570,7 @@ extern "C" ttt_status ttt_qkv_prologue(const ttt_qkv_prologue_args* a, cudaStrea
     if (a->B < 0 || a->T < 0 || a->Dm <= 0 || a->H <= 0 || a->d <= 0) return TTT_ERR_INVALID_ARG;
     if (a->io_dtype != TTT_F32 && a->io_dtype != TTT_BF16) return TTT_ERR_INVALID_ARG;
     if ((a->theta_lr == nullptr) != (a->eta == nullptr)) return TTT_ERR_INVALID_ARG;
-    if (a->flags & ~TTT_FLAG_TEST_STALL) return TTT_ERR_INVALID_ARG;
-    if (a->io_dtype != TTT_BF16) return TTT_ERR_UNSUPPORTED;
+    if (a->flags & ~(TTT_FLAG_TEST_STALL | TTT_FLAG_FORCE_SIMT)) return TTT_ERR_INVALID_ARG;
     if (a->d != 16 && a->d != 32 && a->d != 64) return TTT_ERR_UNSUPPORTED;
     if (a->H > 256 || a->Dm % 8 != 0) return TTT_ERR_UNSUPPORTED;
     const long long rows = (long long)a->B * a->T;
@@ -580,6 +580,19 @@ extern "C" ttt_status ttt_qkv_prologue(const ttt_qkv_prologue_args* a, cudaStrea
         !ok_ptr(a->K) || !ok_ptr(a->V) || !ok_opt(a->theta_lr) || !ok_opt(a->eta))
         return TTT_ERR_INVALID_ARG;
 
+    if (a->io_dtype == TTT_F32 || (a->flags & TTT_FLAG_FORCE_SIMT)) {
+        // fp32 CUDA cores (every dtype); no device-side waits, so no stall hook
+        if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
+        SimtPrologueParams q{(int)rows, a->T,       a->Dm, a->H, a->d, a->x, a->theta_q, a->theta_k,
+                             a->theta_v, a->theta_lr, a->eta_base, a->Q, a->K, a->V, a->eta};
+        const long long ncol = 3LL * a->H * a->d + (a->theta_lr ? a->H : 0);
+        const dim3 grid((unsigned)((rows + kProTok - 1) / kProTok), (unsigned)((ncol + kProCols - 1) / kProCols));
+        if (a->io_dtype == TTT_F32)
+            simt_prologue_kernel<float><<<grid, kSimtThreads, kProSmemBytes, stream>>>(q);
+        else
+            simt_prologue_kernel<__nv_bfloat16><<<grid, kSimtThreads, kProSmemBytes, stream>>>(q);
+        return launch_status();
+    }
     using namespace pro;
     const int Hd = a->H * a->d;
     PrologueParams p;

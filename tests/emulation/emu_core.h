@@ -100,6 +100,8 @@ inline float __shfl_xor_sync(unsigned, float v, int o) {
     return r;
 }
 inline float rsqrtf(float x) { return 1.0f / std::sqrt(x); }
+inline int min(int a, int b) { return a < b ? a : b; }
+inline int max(int a, int b) { return a > b ? a : b; }
 inline float __expf(float x) { return std::exp(x); }
 inline float __fdividef(float a, float b) { return a / b; }
 #define __launch_bounds__(...)

@@ -16,6 +16,7 @@ alignas(1024) uint8_t smem[65536];
 #include "../../test_sequence_layers_head_b200/csrc/simt_mlp_backward.cuh"
 #include "../../test_sequence_layers_head_b200/csrc/mma_forward.cuh"
 #include "../../test_sequence_layers_head_b200/csrc/mma_ln.cuh"
+#include "../../test_sequence_layers_head_b200/csrc/simt_prologue.cuh"
 
 namespace {
 
@@ -202,5 +203,25 @@ extern "C" int emu_ln_backward_mma(int B, int H, int T, const void* Q, const voi
     ttt::SimtLnBackwardParams q{H,  T,  16, Q,  K,      V,      eta,    eta_const, W_states, c_states, gamma, beta,
                                 eps, dZ, dW_out, dc_out, dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta};
     emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_backward_kernel(q); });
+    return 0;
+}
+
+// the fused prologue on fp32 CUDA cores (grid: token blocks x column blocks, run as one flat loop of CTAs)
+extern "C" int emu_prologue_simt(int io, int B, int T, int Dm, int H, int d, const void* x, const void* tq,
+                                 const void* tk, const void* tv, const void* tl, float eta_base, void* Q, void* K,
+                                 void* V, float* eta) {
+    const int rows = B * T;
+    if (rows == 0) return 0;
+    ttt::SimtPrologueParams q{rows, T, Dm, H, d, x, tq, tk, tv, tl, eta_base, Q, K, V, eta};
+    const long long ncol = 3LL * H * d + (tl ? H : 0);
+    const int gx = (rows + ttt::kProTok - 1) / ttt::kProTok, gy = (int)((ncol + ttt::kProCols - 1) / ttt::kProCols);
+    emu::run_grid(gx * gy, ttt::kSimtThreads, ttt::sm, [&] {
+        const unsigned flat = emu::bid3.x;
+        emu::bid3 = make_uint3(flat % gx, flat / gx, 0);
+        if (io == 0)
+            ttt::simt_prologue_kernel<float>(q);
+        else
+            ttt::simt_prologue_kernel<__nv_bfloat16>(q);
+    });
     return 0;
 }

@@ -285,13 +285,13 @@ def _prologue_args(ttt, **kw):
     (dict(H=0), 1),
     (dict(d=0), 1),
     (dict(io_dtype=4), 1),
-    (dict(io_dtype=0), 2),                       # fp32 input: no kernel
+    (dict(io_dtype=0, flags=0x100), 2),          # the fp32 kernel has no stall hook
     (dict(d=48), 2),
     (dict(H=257), 2),                            # the gate tile holds at most 256 heads
     (dict(Dm=772), 2),                           # rows of x must be 16-byte multiples
     (dict(theta_lr=None), 1),                    # gate pointers come in pairs
     (dict(eta=None), 1),
-    (dict(flags=0x1), 1),                        # only the stall hook is a valid flag
+    (dict(flags=0x2), 1),                        # only FORCE_SIMT and the stall hook are valid flags
     (dict(x=None), 1),
     (dict(theta_v=(1 << 20) + 2), 1),
     (dict(Q=None), 1),

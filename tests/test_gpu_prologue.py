@@ -17,7 +17,7 @@ import torch
 
 from oracle import oracle as O
 from test_sequence_layers_head_b200 import workloads as WL
-from tests.gpu_util import TOL_BF16_NORMWISE, normwise, to_dev, to_host
+from tests.gpu_util import TOL_BF16_NORMWISE, maxrel, normwise, to_dev, to_host
 
 pytestmark = [pytest.mark.gpu,
               pytest.mark.skip(reason="prologue kernel: first supervised B200 run pending")]
@@ -144,3 +144,38 @@ def test_prologue_stall_reports_timeout(ttt_lib):
     ref = O.qkv_prologue(e["x"], e["theta_q"], e["theta_k"], e["theta_v"], e["theta_lr"], w.eta_base, w.d)
     check_views(to_host(Q), ref[0], view_bounds(e["x"], e["theta_q"], w.H, w.d))
     assert ttt_lib.last_device_status() == 0
+
+
+@pytest.mark.parametrize("B,T,Dm,H,d,gate", [(2, 20, 40, 3, 16, True), (1, 33, 264, 2, 64, True),
+                                             (1, 256, 768, 12, 64, True)])
+def test_prologue_fp32_on_cuda_cores(ttt_lib, B, T, Dm, H, d, gate):
+    """fp32 input runs on the CUDA-core kernel: max relative error <= 1e-4."""
+    from test_sequence_layers_head_b200 import ttt
+    w, inp = WL.prologue_case(B, T, Dm, H, d, gate=gate, eta_base=0.5)
+    e = inp["exact"]
+    dev = {k: torch.from_numpy(v.astype(np.float32)).cuda() for k, v in e.items()}
+    Q, K, V, eta = ttt.qkv_prologue(dev["x"], dev["theta_q"], dev["theta_k"], dev["theta_v"],
+                                    dev["theta_lr"] if gate else None, 0.5, d)
+    torch.cuda.synchronize()
+    ref = O.qkv_prologue(e["x"], e["theta_q"], e["theta_k"], e["theta_v"], e["theta_lr"], 0.5, d)
+    for got, want in zip((Q, K, V), ref[:3]):
+        assert maxrel(to_host(got), want) <= 1e-4
+    if gate:
+        assert maxrel(to_host(eta), ref[3]) <= 1e-4
+
+
+def test_prologue_tensor_cores_match_cuda_cores_at_full_width(ttt_lib):
+    """bf16 at the 32-head width (Dm = 2048): the tcgen05 kernel against the
+    CUDA-core kernel (TTT_FLAG_FORCE_SIMT) on every output, within two bf16
+    roundings."""
+    from test_sequence_layers_head_b200 import ttt
+    w, inp = WL.prologue_case(2, 512, 2048, 32, 64, gate=True)
+    dev = {k: to_dev(v) for k, v in inp["raw"].items()}
+    a = ttt.qkv_prologue(dev["x"], dev["theta_q"], dev["theta_k"], dev["theta_v"], dev["theta_lr"], w.eta_base, 64)
+    b = ttt.qkv_prologue(dev["x"], dev["theta_q"], dev["theta_k"], dev["theta_v"], dev["theta_lr"], w.eta_base, 64,
+                         flags=ttt.FLAG_FORCE_SIMT)
+    torch.cuda.synchronize()
+    for x, y in zip(a[:3], b[:3]):
+        x, y = to_host(x), to_host(y)
+        assert np.all(np.abs(x - y) <= 2.0 ** -7 * np.abs(y) + 1e-3)
+    assert maxrel(to_host(a[3]), to_host(b[3])) <= 1e-3

@@ -13,7 +13,8 @@ Covered: the TTT-MLP forward writing its batch-start states and the
 outer-loop backward that reads them (fp32 CUDA cores); the TTT-Linear pair
 on mma.sync (bf16, d = 64, b = 16) -- already verified on the B200, which
 pins the emulated ldmatrix / mma semantics; and the LN+residual pair on
-mma.sync (paper digest "论文速览 | TTT", sections 3.4, 3.6, 3.7, 4.4, 6.12).
+mma.sync; and the fused prologue on fp32 CUDA cores (paper digest
+"论文速览 | TTT", sections 3.3, 3.4, 3.6, 3.7, 4.4, 4.6, 6.12).
 """
 import ctypes
 import os
@@ -214,3 +215,33 @@ def test_ln_training_on_mma_sync(emu, B, H, T, per_token, upstream):
         if nm == "deta" and not per_token:
             continue
         assert normwise(got, want) < 2e-2, (nm, normwise(got, want))
+
+
+@pytest.mark.parametrize("B,T,Dm,H,d,gate,io", [(2, 20, 40, 3, 16, True, WL.F32), (1, 33, 264, 2, 64, True, WL.F32),
+                                                (1, 17, 64, 7, 64, False, WL.F32), (2, 9, 24, 5, 32, True, WL.BF16)])
+def test_prologue_on_cuda_cores(emu, B, T, Dm, H, d, gate, io):
+    """The CUDA-core prologue (fp32 input, and bf16 with TTT_FLAG_FORCE_SIMT)
+    against the oracle: two column blocks when 3 H d + H > 1024, ragged token
+    blocks, no gate."""
+    w, inp = WL.prologue_case(B, T, Dm, H, d, gate=gate, eta_base=0.5)
+    e = inp["exact"]
+    if io == WL.F32:
+        raw = {k: v.astype(np.float32) for k, v in e.items()}
+        iot = np.float32
+    else:
+        raw, iot = inp["raw"], np.uint16
+    Q, K, V = (np.zeros((B, H, T, d), iot) for _ in range(3))
+    eta = np.zeros((B, H, T), np.float32) if gate else None
+    f = emu.emu_prologue_simt
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 4
+    assert f(0 if io == WL.F32 else 1, B, T, Dm, H, d, _p(raw["x"]), _p(raw["theta_q"]), _p(raw["theta_k"]),
+             _p(raw["theta_v"]), _p(raw["theta_lr"]) if gate else None, 0.5, _p(Q), _p(K), _p(V), _p(eta)) == 0
+    ref = O.qkv_prologue(e["x"], e["theta_q"], e["theta_k"], e["theta_v"], e["theta_lr"], 0.5, d)
+    h = (lambda a: a.astype(np.float64)) if io == WL.F32 else WL.bf16_bits_to_f64
+    for got, want in zip((Q, K, V), ref[:3]):
+        if io == WL.F32:
+            assert maxrel(h(got), want) < 1e-4
+        else:
+            assert normwise(h(got), want) < 2e-2
+    if gate:
+        assert maxrel(eta.astype(np.float64), ref[3]) < 1e-4
