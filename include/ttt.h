@@ -264,8 +264,10 @@ ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
  *
  *   B, H, T, d, b, io_dtype, Q, K, V, eta, eta_const
  *                  exactly as given to the forward that wrote W_states.
- *                  Served by an fp32 CUDA-core kernel: d in {16, 32, 64},
- *                  b up to the shared-memory limit (16 at d = 64).
+ *                  BF16 with d = 64, b = 16 runs on the tensor cores
+ *                  (mma.sync); every other case (and TTT_FLAG_FORCE_SIMT) on
+ *                  fp32 CUDA cores: d in {16, 32, 64}, b up to the
+ *                  shared-memory limit (16 at d = 64).
  *   W_states       [B, H, T/b, 2dm + m + d] fp32, from ttt_mlp_forward.
  *   dZ             [B, H, T, d] io_dtype, or NULL (zero).
  *   dW1_out [B,H,d,m], dc1_out [B,H,m], dW2_out [B,H,m,d], dc2_out [B,H,d]
@@ -279,7 +281,7 @@ ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
  *                  parameters shared over sequences, the caller sums over B).
  *                  They also serve as the kernel's running adjoint, so they
  *                  must not overlap any input.
- *   flags          must be 0.
+ *   flags          TTT_FLAG_FORCE_SIMT; any other bit is TTT_ERR_INVALID_ARG.
  */
 typedef struct {
     int B, H, T, d, b;

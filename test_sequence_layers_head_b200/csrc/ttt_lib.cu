@@ -20,6 +20,7 @@
 #include "mma_backward.cuh"
 #include "mma_forward.cuh"
 #include "mma_ln.cuh"
+#include "mma_mlp_backward.cuh"
 #include "prologue.cuh"
 #include "simt_prologue.cuh"
 #include "tmap.h"
@@ -553,7 +554,16 @@ extern "C" ttt_status ttt_mlp_backward(const ttt_mlp_backward_args* a, cudaStrea
     if (!ok_opt(a->eta) || !ok_opt(a->dZ) || !ok_opt(a->deta) || !ok_opt(a->dW1_out) || !ok_opt(a->dc1_out) ||
         !ok_opt(a->dW2_out) || !ok_opt(a->dc2_out))
         return TTT_ERR_INVALID_ARG;
-    if (a->flags != 0) return TTT_ERR_INVALID_ARG;
+    if (a->flags & ~TTT_FLAG_FORCE_SIMT) return TTT_ERR_INVALID_ARG;
+    if (a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 && !(a->flags & TTT_FLAG_FORCE_SIMT)) {
+        SimtMlpBackwardParams p{a->H,       a->T,       a->b,       a->Q,       a->K,       a->V,
+                                a->eta,     a->eta_const, a->W_states, a->dZ,   a->dW1_out, a->dc1_out,
+                                a->dW2_out, a->dc2_out, a->dQ,      a->dK,      a->dV,      a->deta,
+                                a->dW1,     a->dc1,     a->dW2,     a->dc2};
+        if (!set_smem(mmb::mma_mlp_backward_kernel, mmb::kSmemBytes)) return TTT_ERR_CUDA;
+        mmb::mma_mlp_backward_kernel<<<(unsigned)units, mmb::kThreads, mmb::kSmemBytes, stream>>>(p);
+        return launch_status();
+    }
     if (simt_mlp_backward_smem(a->d, a->b) > 227 * 1024) return TTT_ERR_UNSUPPORTED;
     switch (a->d) {
         case 16: return launch_mlp_backward<16>(a, stream);

@@ -279,7 +279,7 @@ def mlp_decode_step(W1, c1, W2, c2, q, k, v, eta, *, eta_const=0.0, z=None, stre
 
 def mlp_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW1_out=None, dc1_out=None, dW2_out=None, dc2_out=None,
                  eta_const=0.0, dQ=None, dK=None, dV=None, deta=None, want_deta=True, dW1=None, dc1=None, dW2=None,
-                 dc2=None, stream=None):
+                 dc2=None, flags=0, stream=None):
     """Outer-loop gradients of the TTT-MLP prefill; see ``ttt_mlp_backward``.
     Returns (dQ, dK, dV, deta, dW1, dc1, dW2, dc2); deta is None when
     ``want_deta`` is False."""
@@ -297,7 +297,8 @@ def mlp_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW1_out=None, dc1_out=No
     dc2 = torch.empty((B, H, d), device=dev, dtype=f32) if dc2 is None else dc2
     a = MlpBackwardArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
                         _ptr(W_states), _ptr(dZ), _ptr(dW1_out), _ptr(dc1_out), _ptr(dW2_out), _ptr(dc2_out),
-                        _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW1), _ptr(dc1), _ptr(dW2), _ptr(dc2), 0)
+                        _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW1), _ptr(dc1), _ptr(dW2), _ptr(dc2),
+                        int(flags))
     _check(library().ttt_mlp_backward(ctypes.byref(a), _stream(stream)), "ttt_mlp_backward")
     return dQ, dK, dV, deta, dW1, dc1, dW2, dc2
 

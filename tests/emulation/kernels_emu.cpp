@@ -10,6 +10,9 @@ alignas(1024) float sm[65536];
 namespace mbk {
 alignas(1024) uint8_t smem[65536];
 }
+namespace mmb {
+alignas(1024) uint8_t smem[4 * 65536];
+}
 }  // namespace ttt
 
 #include "../../test_sequence_layers_head_b200/csrc/simt.cuh"
@@ -17,6 +20,7 @@ alignas(1024) uint8_t smem[65536];
 #include "../../test_sequence_layers_head_b200/csrc/mma_forward.cuh"
 #include "../../test_sequence_layers_head_b200/csrc/mma_ln.cuh"
 #include "../../test_sequence_layers_head_b200/csrc/simt_prologue.cuh"
+#include "../../test_sequence_layers_head_b200/csrc/mma_mlp_backward.cuh"
 
 namespace {
 
@@ -223,5 +227,18 @@ extern "C" int emu_prologue_simt(int io, int B, int T, int Dm, int H, int d, con
         else
             ttt::simt_prologue_kernel<__nv_bfloat16>(q);
     });
+    return 0;
+}
+
+// the TTT-MLP backward on mma.sync (bf16, d = 64, b = 16), from states written by the CUDA-core forward
+extern "C" int emu_mlp_backward_mma(int B, int H, int T, const void* Q, const void* K, const void* V,
+                                    const float* eta, float eta_const, const float* W_states, const void* dZ,
+                                    const float* dW1o, const float* dc1o, const float* dW2o, const float* dc2o,
+                                    void* dQ, void* dK, void* dV, float* deta, float* dW1, float* dc1, float* dW2,
+                                    float* dc2) {
+    static_assert(ttt::mmb::kSmemBytes <= (int)sizeof(ttt::mmb::smem), "emulated shared memory");
+    ttt::SimtMlpBackwardParams q{H,    T,    16, Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
+                                 dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2};
+    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_backward_kernel(q); });
     return 0;
 }

@@ -246,7 +246,7 @@ def _mlp_backward_args(ttt, **kw):
     (dict(dZ=(1 << 20) + 2), 1),
     (dict(dW2_out=(1 << 20) + 8), 1),
     (dict(deta=(1 << 20) + 4), 1),
-    (dict(flags=0x1), 1),
+    (dict(flags=0x2), 1),
     (dict(B=0, Q=None, dW1=None), 0),
 ])
 def test_mlp_backward_validation(ttt_lib, kw, code):

@@ -147,3 +147,23 @@ def test_mlp_backward_full_size_sampled(ttt_lib):
         for nm, k in (("dW1", 4), ("dc1", 5), ("dW2", 6), ("dc2", 7)):
             got = out[k][n:n + 1, h:h + 1].cpu().numpy().astype(np.float64)
             assert normwise(got, ref[k]) <= 2e-2, nm
+
+
+def test_mlp_backward_tensor_cores_match_cuda_cores(ttt_lib):
+    """bf16, d = 64, b = 16 runs on mma.sync; TTT_FLAG_FORCE_SIMT runs the same
+    call on the fp32 CUDA-core kernel: both against the oracle, and each other."""
+    inp, c1, c2, dz, ups = _case(2, 2, 64, 64, 16, WL.BF16, True, True, seed=17)
+    r, w = inp.raw, inp.w
+    Q, K, V, eta = (to_dev(r[n]) for n in ("Q", "K", "V", "eta"))
+    B, H, T, d = Q.shape
+    m = 4 * d
+    states = torch.empty((B, H, T // 16, 2 * d * m + m + d), device="cuda")
+    ttt_lib.mlp_forward(Q, K, V, eta, to_dev(r["W1"]), to_dev(c1), to_dev(r["W2"]), to_dev(c2), 16, W_states=states)
+    kw = dict(dZ=to_dev(dz[0]), **{k: to_dev(u) for k, u in zip(("dW1_out", "dc1_out", "dW2_out", "dc2_out"), ups)})
+    tc = ttt_lib.mlp_backward(Q, K, V, eta, states, 16, **kw)
+    simt = ttt_lib.mlp_backward(Q, K, V, eta, states, 16, flags=ttt_lib.FLAG_FORCE_SIMT, **kw)
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    for a, b_ in zip(tc, simt):
+        assert normwise(to_host(a), to_host(b_)) <= 2e-2
+    _check(inp, c1, c2, dz, ups, True, to_host(states), [to_host(g) for g in tc])

@@ -13,7 +13,8 @@ Covered: the TTT-MLP forward writing its batch-start states and the
 outer-loop backward that reads them (fp32 CUDA cores); the TTT-Linear pair
 on mma.sync (bf16, d = 64, b = 16) -- already verified on the B200, which
 pins the emulated ldmatrix / mma semantics; and the LN+residual pair on
-mma.sync; and the fused prologue on fp32 CUDA cores (paper digest
+mma.sync; the TTT-MLP backward on mma.sync; and the fused prologue on fp32
+CUDA cores (paper digest
 "论文速览 | TTT", sections 3.3, 3.4, 3.6, 3.7, 4.4, 4.6, 6.12).
 """
 import ctypes
@@ -245,3 +246,46 @@ def test_prologue_on_cuda_cores(emu, B, T, Dm, H, d, gate, io):
             assert normwise(h(got), want) < 2e-2
     if gate:
         assert maxrel(eta.astype(np.float64), ref[3]) < 1e-4
+
+
+@pytest.mark.parametrize("B,H,T,per_token,upstream", [(1, 2, 32, True, True), (1, 1, 48, False, False)])
+def test_mlp_backward_on_mma_sync(emu, B, H, T, per_token, upstream):
+    """The TTT-MLP backward on mma.sync (bf16, d = 64, b = 16) from the states
+    the CUDA-core forward writes, against the oracle (bf16 bar)."""
+    d, b, m = 64, 16, 256
+    inp = WL.random_case("mlp", B, H, T, d, b, io_dtype=WL.BF16, eta_mode="sigmoid" if per_token else "const",
+                         eta_const=0.0 if per_token else 0.02, seed=41 + T)
+    raw, ex = inp.raw, inp.exact
+    rng = np.random.default_rng(100 + T)
+    c1 = (rng.standard_normal((H, m)) * 0.1).astype(np.float32)
+    c2 = (rng.standard_normal((H, d)) * 0.1).astype(np.float32)
+    dZr, dZe = WL.store(rng.standard_normal((B, H, T, d)), WL.BF16)
+    ups = ([rng.standard_normal(s).astype(np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+           if upstream else [None] * 4)
+    nb = T // b
+    Z = np.zeros((B, H, T, d), np.uint16)
+    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    eta = raw["eta"] if per_token else None
+    f = emu.emu_mlp_forward
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 10
+    assert f(1, B, H, T, d, b, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const),
+             _p(raw["W1"]), _p(c1), _p(raw["W2"]), _p(c2), _p(Z), *[_p(o) for o in outs], _p(states)) == 0
+    dQ, dK, dV = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
+    deta = np.zeros((B, H, T), np.float32)
+    grads = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    g = emu.emu_mlp_backward_mma
+    g.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 14
+    assert g(B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const), _p(states),
+             _p(dZr), *[_p(u) for u in ups], _p(dQ), _p(dK), _p(dV), _p(deta), *[_p(x) for x in grads]) == 0
+    eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(inp.w.eta_const)))
+    ref = O.mlp_backward(ex["Q"], ex["K"], ex["V"], eta_e, ex["W1"], c1.astype(np.float64), ex["W2"],
+                         c2.astype(np.float64), b, dZ=dZe,
+                         **{k: (None if u is None else u.astype(np.float64))
+                            for k, u in zip(("dW1_out", "dc1_out", "dW2_out", "dc2_out"), ups)})
+    h = WL.bf16_bits_to_f64
+    gots = [h(dQ), h(dK), h(dV), deta.astype(np.float64)] + [x.astype(np.float64) for x in grads]
+    for nm, got, want in zip(("dQ", "dK", "dV", "deta", "dW1", "dc1", "dW2", "dc2"), gots, ref):
+        if nm == "deta" and not per_token:
+            continue
+        assert normwise(got, want) < 2e-2, (nm, normwise(got, want))
