@@ -224,8 +224,10 @@ ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_
  *   W_states       NULL, or [B, H, T/b, 2dm + m + d] fp32: the state at the
  *                  start of every mini-batch, each one W1 [d][m], c1 [m],
  *                  W2 [m][d], c2 [d] (the checkpoints ttt_mlp_backward reads;
- *                  section 6.12).  Served by the fp32 CUDA-core kernel for
- *                  every dtype and d; not with use_ln (TTT_ERR_UNSUPPORTED).
+ *                  section 6.12).  BF16 with d = 64, b = 16 runs on an
+ *                  mma.sync tensor-core kernel, every other case (and
+ *                  TTT_FLAG_FORCE_SIMT) on the fp32 CUDA-core kernel; not with
+ *                  use_ln (TTT_ERR_UNSUPPORTED).
  */
 typedef struct {
     int B, H, T, d, b;

@@ -83,6 +83,138 @@ __device__ __forceinline__ void frag_from_f32(const float* S, bool transpose, co
     a[3] = pk(el(g + 8, 2 * c + 8), el(g + 8, 2 * c + 9));
 }
 
+// A lane's place in the kernels' layout (warp w, lane l = 4 r + c; hidden units p0 .. p0 + 31; features
+// j0 .. j0 + 7 = half jh of the 16-column window jn0) and the products and exchanges built on it
+struct Ops {
+    uint8_t* smem;
+    float* part;
+    float* rowp;
+    int tid, w, l, r, c, p0, jn0, jh, j0;
+
+    // the per-lane columns of a 16 x 256 product: hidden unit p0 + 8 nt + 2 c + k
+    __device__ __forceinline__ int hid(int nt, int k) const { return p0 + 8 * nt + 2 * c + k; }
+    // store a warp's 16 x 32 block (four n-tiles) of a 16 x 256 intermediate as bf16
+    __device__ __forceinline__ void store_mm(int off, const float (&x)[4][4]) const {
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                *reinterpret_cast<uint32_t*>(smem + off + mm_off(kTileBD, r + 8 * h, hid(nt, 0))) =
+                    pk(x[nt][2 * h], x[nt][2 * h + 1]);
+    }
+    // store a warp's 16 x 8 block of a 16 x 64 product as bf16
+    __device__ __forceinline__ void store_bd(int off, const float (&x)[4]) const {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+            *reinterpret_cast<uint32_t*>(smem + off + toff(r + 8 * h, j0 >> 3) + 4 * c) = pk(x[2 * h], x[2 * h + 1]);
+    }
+    // 16 x 32 block (this warp's hidden units) of A (16 x K, [m][k] tile at ta, K = 16 kst) times
+    // B[k][p] stored [k][n] in 64-column tiles of `btile` bytes at tb (rows k)
+    __device__ __forceinline__ void mm_AB_kn(float (&x)[4][4], uint32_t ta, int a_is_mm, int kst, uint32_t tb, int btile) const {
+#pragma unroll 1
+        for (int ks = 0; ks < kst; ++ks) {
+            uint32_t a[4];
+            if (a_is_mm)
+                ldsm4(a_addr(ta + (ks >> 2) * kTileBD, 0, ks & 3, l), a);
+            else
+                ldsm4(a_addr(ta, 0, ks, l), a);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t b[4];
+                const int n0 = p0 + 16 * np;
+                ldsm4t(bt_addr(tb + (n0 >> 6) * btile, n0 & 63, ks, l), b);
+                mma(x[2 * np], a, b[0], b[1]);
+                mma(x[2 * np + 1], a, b[2], b[3]);
+            }
+        }
+    }
+    // 16 x 32 block of A (16 x 64 token tile at ta) times B[k=j][n=p] = X[p][j], X stored [256 p][64 j] at tb
+    __device__ __forceinline__ void mm_A_Xt(float (&x)[4][4], uint32_t ta, uint32_t tb) const {
+#pragma unroll 1
+        for (int ks = 0; ks < 4; ++ks) {
+            uint32_t a[4];
+            ldsm4(a_addr(ta, 0, ks, l), a);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t b[4];
+                ldsm4(b_addr(tb, p0 + 16 * np, ks, l), b);
+                mma(x[2 * np], a, b[0], b[1]);
+                mma(x[2 * np + 1], a, b[2], b[3]);
+            }
+        }
+    }
+    // 16 x 8 block (this warp's features) of A (16 x 256 intermediate at ta) times
+    // B[k=p][n=j] = X[p][j], X stored [256 p][64 j] at tb
+    __device__ __forceinline__ void bd_A_X(float (&y)[4], uint32_t ta, uint32_t tb) const {
+#pragma unroll 2
+        for (int ks = 0; ks < 16; ++ks) {
+            uint32_t a[4], b[4];
+            ldsm4(a_addr(ta + (ks >> 2) * kTileBD, 0, ks & 3, l), a);
+            ldsm4t(bt_addr(tb, jn0, ks, l), b);
+            mma(y, a, jh ? b[2] : b[0], jh ? b[3] : b[1]);
+        }
+    }
+    // 16 x 8 block of A (16 x 256 intermediate at ta) times B[k=p][n=a] = X[a][p], X stored [64 a][256 p]
+    __device__ __forceinline__ void bd_A_Yt(float (&y)[4], uint32_t ta, uint32_t tb) const {
+#pragma unroll 2
+        for (int ks = 0; ks < 16; ++ks) {
+            uint32_t a[4], b[4];
+            ldsm4(a_addr(ta + (ks >> 2) * kTileBD, 0, ks & 3, l), a);
+            ldsm4(b_addr(tb + (ks >> 2) * 8192, jn0, ks & 3, l), b);
+            mma(y, a, jh ? b[2] : b[0], jh ? b[3] : b[1]);
+        }
+    }
+    // per-row sums over the CTA of the lane's partials v[h] (rows r + 8 h): quad shuffle, per-warp
+    // partials in shared memory, one barrier
+    __device__ __forceinline__ void row_total(float (&v)[2]) const {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            v[h] += __shfl_xor_sync(0xffffffffu, v[h], 1);
+            v[h] += __shfl_xor_sync(0xffffffffu, v[h], 2);
+        }
+        if (c == 0) {
+            rowp[w * kB + r] = v[0];
+            rowp[w * kB + r + 8] = v[1];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float s = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < 8; ++ww) s += rowp[ww * kB + r + 8 * h];
+            v[h] = s;
+        }
+    }
+    // split-K 16 x 16 product over the hidden units: sum over warps of A[:, p0..] B[:, p0..]^T into dst,
+    // masked to s <= t and with `add` on the kept entries, scaled by `scale`
+    __device__ __forceinline__ void tt_split(uint32_t ta, uint32_t tb, float* dst, float add, float scale) const {
+        float x[2][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+            const int ks = 2 * w + kk;   // 16-unit step of this warp's 32 hidden units
+            uint32_t a[4], b[4];
+            ldsm4(a_addr(ta + (ks >> 2) * kTileBD, 0, ks & 3, l), a);
+            ldsm4(b_addr(tb + (ks >> 2) * kTileBD, 0, ks & 3, l), b);
+            mma(x[0], a, b[0], b[1]);
+            mma(x[1], a, b[2], b[3]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) part[w * 256 + (r + 8 * (q >> 1)) * 16 + 8 * nt + 2 * c + (q & 1)] = x[nt][q];
+        __syncthreads();
+        {
+            const int t = tid >> 4, s = tid & 15;
+            float v = 0.f;
+#pragma unroll
+            for (int ww = 0; ww < 8; ++ww) v += part[ww * 256 + tid];
+            dst[tid] = s <= t ? scale * (v + add) : 0.f;
+        }
+        __syncthreads();
+    }
+
+};
+
 __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBackwardParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t s0 = smem_u32(smem);
@@ -116,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
     const int jn0 = 16 * (w >> 1), jh = w & 1;   // its features: half jh of the 16-column window jn0
     const int j0 = jn0 + 8 * jh;
     constexpr size_t SZ = 2 * (size_t)kD * kM + kM + kD;
+    const Ops ops{smem, part, rowp, tid, w, l, r, c, p0, jn0, jh, j0};
 
     // the adjoint of the final state: the upstream gradients, or zero
     for (int e = tid; e < kD * kM; e += kThreads) {
@@ -125,128 +258,6 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
     for (int e = tid; e < kM; e += kThreads) gc1[e] = p.dc1_out ? p.dc1_out[(size_t)unit * kM + e] : 0.f;
     for (int e = tid; e < kD; e += kThreads) gc2[e] = p.dc2_out ? p.dc2_out[(size_t)unit * kD + e] : 0.f;
     __syncthreads();
-
-    // the per-lane columns of a 16 x 256 product: hidden unit p0 + 8 nt + 2 c + k
-    auto hid = [&](int nt, int k) { return p0 + 8 * nt + 2 * c + k; };
-    // store a warp's 16 x 32 block (four n-tiles) of a 16 x 256 intermediate as bf16
-    auto store_mm = [&](int off, const float (&x)[4][4]) {
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-                *reinterpret_cast<uint32_t*>(smem + off + mm_off(kTileBD, r + 8 * h, hid(nt, 0))) =
-                    pk(x[nt][2 * h], x[nt][2 * h + 1]);
-    };
-    // store a warp's 16 x 8 block of a 16 x 64 product as bf16
-    auto store_bd = [&](int off, const float (&x)[4]) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-            *reinterpret_cast<uint32_t*>(smem + off + toff(r + 8 * h, j0 >> 3) + 4 * c) = pk(x[2 * h], x[2 * h + 1]);
-    };
-    // 16 x 32 block (this warp's hidden units) of A (16 x K, [m][k] tile at ta, K = 16 kst) times
-    // B[k][p] stored [k][n] in 64-column tiles of `btile` bytes at tb (rows k)
-    auto mm_AB_kn = [&](float (&x)[4][4], uint32_t ta, int a_is_mm, int kst, uint32_t tb, int btile) {
-#pragma unroll 1
-        for (int ks = 0; ks < kst; ++ks) {
-            uint32_t a[4];
-            if (a_is_mm)
-                ldsm4(a_addr(ta + (ks >> 2) * kTileBD, 0, ks & 3, l), a);
-            else
-                ldsm4(a_addr(ta, 0, ks, l), a);
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                uint32_t b[4];
-                const int n0 = p0 + 16 * np;
-                ldsm4t(bt_addr(tb + (n0 >> 6) * btile, n0 & 63, ks, l), b);
-                mma(x[2 * np], a, b[0], b[1]);
-                mma(x[2 * np + 1], a, b[2], b[3]);
-            }
-        }
-    };
-    // 16 x 32 block of A (16 x 64 token tile at ta) times B[k=j][n=p] = X[p][j], X stored [256 p][64 j] at tb
-    auto mm_A_Xt = [&](float (&x)[4][4], uint32_t ta, uint32_t tb) {
-#pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks) {
-            uint32_t a[4];
-            ldsm4(a_addr(ta, 0, ks, l), a);
-#pragma unroll
-            for (int np = 0; np < 2; ++np) {
-                uint32_t b[4];
-                ldsm4(b_addr(tb, p0 + 16 * np, ks, l), b);
-                mma(x[2 * np], a, b[0], b[1]);
-                mma(x[2 * np + 1], a, b[2], b[3]);
-            }
-        }
-    };
-    // 16 x 8 block (this warp's features) of A (16 x 256 intermediate at ta) times
-    // B[k=p][n=j] = X[p][j], X stored [256 p][64 j] at tb
-    auto bd_A_X = [&](float (&y)[4], uint32_t ta, uint32_t tb) {
-#pragma unroll 2
-        for (int ks = 0; ks < 16; ++ks) {
-            uint32_t a[4], b[4];
-            ldsm4(a_addr(ta + (ks >> 2) * kTileBD, 0, ks & 3, l), a);
-            ldsm4t(bt_addr(tb, jn0, ks, l), b);
-            mma(y, a, jh ? b[2] : b[0], jh ? b[3] : b[1]);
-        }
-    };
-    // 16 x 8 block of A (16 x 256 intermediate at ta) times B[k=p][n=a] = X[a][p], X stored [64 a][256 p]
-    auto bd_A_Yt = [&](float (&y)[4], uint32_t ta, uint32_t tb) {
-#pragma unroll 2
-        for (int ks = 0; ks < 16; ++ks) {
-            uint32_t a[4], b[4];
-            ldsm4(a_addr(ta + (ks >> 2) * kTileBD, 0, ks & 3, l), a);
-            ldsm4(b_addr(tb + (ks >> 2) * 8192, jn0, ks & 3, l), b);
-            mma(y, a, jh ? b[2] : b[0], jh ? b[3] : b[1]);
-        }
-    };
-    // per-row sums over the CTA of the lane's partials v[h] (rows r + 8 h): quad shuffle, per-warp
-    // partials in shared memory, one barrier
-    auto row_total = [&](float (&v)[2]) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            v[h] += __shfl_xor_sync(0xffffffffu, v[h], 1);
-            v[h] += __shfl_xor_sync(0xffffffffu, v[h], 2);
-        }
-        if (c == 0) {
-            rowp[w * kB + r] = v[0];
-            rowp[w * kB + r + 8] = v[1];
-        }
-        __syncthreads();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            float s = 0.f;
-#pragma unroll
-            for (int ww = 0; ww < 8; ++ww) s += rowp[ww * kB + r + 8 * h];
-            v[h] = s;
-        }
-    };
-    // split-K 16 x 16 product over the hidden units: sum over warps of A[:, p0..] B[:, p0..]^T into dst,
-    // masked to s <= t and with `add` on the kept entries, scaled by `scale`
-    auto tt_split = [&](uint32_t ta, uint32_t tb, float* dst, float add, float scale) {
-        float x[2][4] = {};
-#pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-            const int ks = 2 * w + kk;   // 16-unit step of this warp's 32 hidden units
-            uint32_t a[4], b[4];
-            ldsm4(a_addr(ta + (ks >> 2) * kTileBD, 0, ks & 3, l), a);
-            ldsm4(b_addr(tb + (ks >> 2) * kTileBD, 0, ks & 3, l), b);
-            mma(x[0], a, b[0], b[1]);
-            mma(x[1], a, b[2], b[3]);
-        }
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) part[w * 256 + (r + 8 * (q >> 1)) * 16 + 8 * nt + 2 * c + (q & 1)] = x[nt][q];
-        __syncthreads();
-        {
-            const int t = tid >> 4, s = tid & 15;
-            float v = 0.f;
-#pragma unroll
-            for (int ww = 0; ww < 8; ++ww) v += part[ww * 256 + tid];
-            dst[tid] = s <= t ? scale * (v + add) : 0.f;
-        }
-        __syncthreads();
-    };
 
     for (int i = nb - 1; i >= 0; --i) {
         const int t0 = i * kB;
@@ -286,16 +297,16 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) A_[nt][q] = Aq[nt][q] = c1s[hid(nt, q & 1)];
-        mm_AB_kn(A_, sK, 0, 4, sW1, 8192);
-        mm_AB_kn(Aq, sQ, 0, 4, sW1, 8192);
+            for (int q = 0; q < 4; ++q) A_[nt][q] = Aq[nt][q] = c1s[ops.hid(nt, q & 1)];
+        ops.mm_AB_kn(A_, sK, 0, 4, sW1, 8192);
+        ops.mm_AB_kn(Aq, sQ, 0, 4, sW1, 8192);
         {
             float hk[4][4];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) hk[nt][q] = gelu_f(A_[nt][q]);
-            store_mm(kOffHk, hk);
+            ops.store_mm(kOffHk, hk);
         }
         // P1 = tril(Q K^T + 1) (warp 0)
         if (w == 0) {
@@ -323,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             const float2 cc = *reinterpret_cast<const float2*>(c2s + j0 + 2 * c);
             E_[0] = E_[2] = cc.x;
             E_[1] = E_[3] = cc.y;
-            bd_A_X(E_, sHk, sW2);
+            ops.bd_A_X(E_, sHk, sW2);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const __nv_bfloat162 v2 =
@@ -331,19 +342,19 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
                 E_[2 * h] -= __bfloat162float(v2.x);
                 E_[2 * h + 1] -= __bfloat162float(v2.y);
             }
-            store_bd(kOffE, E_);
+            ops.store_bd(kOffE, E_);
         }
         __syncthreads();   // E
         // M = E W2^T, D1 = M GELU'(A) on this warp's hidden units
         float M_[4][4] = {};
-        mm_A_Xt(M_, sE, sW2);
+        ops.mm_A_Xt(M_, sE, sW2);
         {
             float d1[4][4];
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) d1[nt][q] = M_[nt][q] * gelu_grad_f(A_[nt][q]);
-            store_mm(kOffD1, d1);
+            ops.store_mm(kOffD1, d1);
         }
         __syncthreads();   // D1
         // Aq = Aq0 - L1 D1 with L1 = P1 diag(eta); Hq = GELU(Aq)
@@ -365,11 +376,11 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) hq[nt][q] = gelu_f(Aq[nt][q]);
-            store_mm(kOffHq, hq);
+            ops.store_mm(kOffHq, hq);
         }
         __syncthreads();   // Hq
         // P2 = tril(Hq Hk^T + 1)
-        tt_split(sHq, sHk, P2, 1.f, 1.f);
+        ops.tt_split(sHq, sHk, P2, 1.f, 1.f);
         // ---- backward.  Products with the end-state adjoint (GW1, GW2 copies), dHq = dZ W2^T,
         // dL2 = tril(-dZ E^T)
         float G2[4], dKx[4];
@@ -377,10 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             const float2 gg = *reinterpret_cast<const float2*>(gc2 + j0 + 2 * c);
             G2[0] = G2[2] = gg.x;
             G2[1] = G2[3] = gg.y;
-            bd_A_X(G2, sHk, sG2);   // dc2' + Hk dW2'
+            ops.bd_A_X(G2, sHk, sG2);   // dc2' + Hk dW2'
             float x[4] = {};
             // D1 dW1'^T: B[k=p][n=a] = GW1[a][p]
-            bd_A_Yt(x, sD1, sG1);
+            ops.bd_A_Yt(x, sD1, sG1);
 #pragma unroll
             for (int q = 0; q < 4; ++q) dKx[q] = -eta_r[q >> 1] * x[q];
         }
@@ -390,16 +401,16 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    G1[nt][q] = gc1[hid(nt, q & 1)];
+                    G1[nt][q] = gc1[ops.hid(nt, q & 1)];
                     dHk[nt][q] = 0.f;
                 }
-            mm_AB_kn(G1, sK, 0, 4, sG1, 8192);   // dc1' + K dW1'
-            mm_A_Xt(dHk, sE, sG2);              // E dW2'^T
+            ops.mm_AB_kn(G1, sK, 0, 4, sG1, 8192);   // dc1' + K dW1'
+            ops.mm_A_Xt(dHk, sE, sG2);              // E dW2'^T
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) dHk[nt][q] *= -eta_r[q >> 1];
-            mm_A_Xt(dHq, sDZ, sW2);             // dZ W2^T
+            ops.mm_A_Xt(dHq, sDZ, sW2);             // dZ W2^T
         }
         if (w == 1) {
             float x[2][4] = {};
@@ -430,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
                     v[q >> 1] -= G1[nt][q] * M_[nt][q] * gelu_grad_f(A_[nt][q]);
-            row_total(v);   // (barrier: L2 complete too)
+            ops.row_total(v);   // (barrier: L2 complete too)
             det[0] = v[0];
             det[1] = v[1];
         }
@@ -478,13 +489,13 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) dHq[nt][q] *= gelu_grad_f(Aq[nt][q]);   // dAq
-            store_mm(kOffDAq, dHq);
+            ops.store_mm(kOffDAq, dHq);
         }
         __syncthreads();   // dAq
         // dQ = dAq W1^T (this warp's features); dL1 = tril(-dAq D1^T); dD1 = -eta G1 - L1^T dAq
         float dQx[4] = {};
-        bd_A_Yt(dQx, sDAq, sW1);
-        tt_split(sDAq, sD1, L1, 0.f, -1.f);
+        ops.bd_A_Yt(dQx, sDAq, sW1);
+        ops.tt_split(sDAq, sD1, L1, 0.f, -1.f);
         {
             uint32_t a[4];
             frag_from_f32(P1, true, nullptr, l, a);   // P1^T; L1^T = (P1 diag(eta))^T = diag(eta) P1^T
@@ -520,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
                     dm[nt][q] = G1[nt][q] * gelu_grad_f(A_[nt][q]);
                     M_[nt][q] = G1[nt][q] * M_[nt][q] * gelu_grad2_f(A_[nt][q]);
                 }
-            store_mm(kOffDM, dm);
+            ops.store_mm(kOffDM, dm);
         }
         __syncthreads();   // dM
         // with dP1 = dL1 diag(eta): dQ += dP1 K;  dK += dP1^T Q;  dE += dM W2
@@ -535,8 +546,8 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             mma(y, at, jh ? b[2] : b[0], jh ? b[3] : b[1]);
 #pragma unroll
             for (int q = 0; q < 4; ++q) dKx[q] += eta_r[q >> 1] * y[q];
-            bd_A_X(G2, sDM, sW2);   // dE += dM W2
-            store_bd(kOffDE, G2);
+            ops.bd_A_X(G2, sDM, sW2);   // dE += dM W2
+            ops.store_bd(kOffDE, G2);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 *reinterpret_cast<__nv_bfloat162*>(dV + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c) =
@@ -548,16 +559,16 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
         __syncthreads();   // dE
         // dHk += dE W2^T;  dA = dD1 M GELU''(A) + dHk GELU'(A) -> shared
         {
-            mm_A_Xt(dHk, sDE, sW2);
+            ops.mm_A_Xt(dHk, sDE, sW2);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q) M_[nt][q] += dHk[nt][q] * gelu_grad_f(A_[nt][q]);
-            store_mm(kOffDA, M_);
+            ops.store_mm(kOffDA, M_);
         }
         __syncthreads();   // dA
         // dK += dA W1^T (this warp's features)
-        bd_A_Yt(dKx, sDA, sW1);
+        ops.bd_A_Yt(dKx, sDA, sW1);
 #pragma unroll
         for (int h = 0; h < 2; ++h)
             *reinterpret_cast<__nv_bfloat162*>(dK + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c) =
@@ -575,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    x[nt][q] = gW1[(size_t)(16 * mt + r + 8 * (q >> 1)) * kM + hid(nt, q & 1)];
+                    x[nt][q] = gW1[(size_t)(16 * mt + r + 8 * (q >> 1)) * kM + ops.hid(nt, q & 1)];
             uint32_t aq[4], ak[4];
             ldsm4t(at_addr(sQ, 16 * mt, l), aq);
             ldsm4t(at_addr(sK, 16 * mt, l), ak);
@@ -594,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
-                    *reinterpret_cast<float2*>(gW1 + (size_t)(16 * mt + r + 8 * h) * kM + hid(nt, 0)) =
+                    *reinterpret_cast<float2*>(gW1 + (size_t)(16 * mt + r + 8 * h) * kM + ops.hid(nt, 0)) =
                         make_float2(x[nt][2 * h], x[nt][2 * h + 1]);
         }
         // GW2[p][j] += (Hq^T dZ + dM^T E + Hk^T dE)[p][j] on this warp's hidden units (two 16-row blocks)
@@ -648,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
 #pragma unroll
                 for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-                    for (int k = 0; k < 2; ++k) gc1[hid(nt, k)] += s1[nt][k];
+                    for (int k = 0; k < 2; ++k) gc1[ops.hid(nt, k)] += s1[nt][k];
             float s2[2];
             const float2 z0 = tile_pair_bf16(smem, kOffDZ, r, j0 + 2 * c);
             const float2 z1 = tile_pair_bf16(smem, kOffDZ, r + 8, j0 + 2 * c);
@@ -666,6 +677,305 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             }
         }
         __syncthreads();   // every read of this mini-batch's shared data and of the adjoint is done
+    }
+}
+
+// The TTT-MLP forward that writes the batch-start states, on mma.sync (bf16, d = 64, b = 16): the dual
+// form of section 3.7 per mini-batch, in the layout of the backward above.  The state is not kept in
+// registers: mini-batch i reads S_i from its checkpoint W_states[i] (S_0 = the initial state, copied
+// there first) and each warp writes its block of S_{i+1} = S_i + (update) to W_states[i + 1], or to the
+// final-state outputs after the last mini-batch.
+struct MlpFwdStatesParams {
+    int H, T;
+    const void* Q;
+    const void* K;
+    const void* V;
+    const float* eta;
+    float eta_const;
+    const float* W1;   // initial state, [H, ...] or [B, H, ...] (per_seq)
+    const float* c1;   // or null
+    const float* W2;
+    const float* c2;   // or null
+    int per_seq;
+    void* Z;           // or null (state only)
+    float* W1_out;
+    float* c1_out;     // or null
+    float* W2_out;
+    float* c2_out;     // or null
+    float* W_states;   // [units, T/16, 2 d m + m + d]
+};
+
+__global__ void __launch_bounds__(kThreads, 1) mma_mlp_forward_states_kernel(MlpFwdStatesParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const uint32_t s0 = smem_u32(smem);
+    const uint32_t sW1 = s0 + kOffW1, sW2 = s0 + kOffW2;
+    const uint32_t sHk = s0 + kOffHk, sD1 = s0 + kOffD1, sHq = s0 + kOffHq;
+    const uint32_t sK = s0 + kOffK, sQ = s0 + kOffQ, sE = s0 + kOffE, sEE = s0 + kOffDE;
+    float* P1 = reinterpret_cast<float*>(smem + kOffP1);
+    float* P2 = reinterpret_cast<float*>(smem + kOffP2);
+    float* part = reinterpret_cast<float*>(smem + kOffPart);
+    float* rowp = reinterpret_cast<float*>(smem + kOffRow);
+    float* s_eta = reinterpret_cast<float*>(smem + kOffEta);
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31, r = l >> 2, c = l & 3;
+    const int unit = blockIdx.x;
+    const int T = p.T, nb = T / kB;
+    const int pu = p.per_seq ? unit : unit % p.H;
+    const size_t tok = (size_t)unit * T * kD;
+    const __nv_bfloat16* Q = static_cast<const __nv_bfloat16*>(p.Q) + tok;
+    const __nv_bfloat16* K = static_cast<const __nv_bfloat16*>(p.K) + tok;
+    const __nv_bfloat16* V = static_cast<const __nv_bfloat16*>(p.V) + tok;
+    __nv_bfloat16* Z = p.Z ? static_cast<__nv_bfloat16*>(p.Z) + tok : nullptr;
+    const int p0 = 32 * w;
+    const int jn0 = 16 * (w >> 1), jh = w & 1;
+    const int j0 = jn0 + 8 * jh;
+    constexpr size_t SZ = 2 * (size_t)kD * kM + kM + kD;
+    const Ops ops{smem, part, rowp, tid, w, l, r, c, p0, jn0, jh, j0};
+    float* states = p.W_states + (size_t)unit * nb * SZ;
+
+    // S_0: the initial state, to the first checkpoint
+    if (nb > 0) {
+        for (int e = tid; e < kD * kM; e += kThreads) {
+            states[e] = p.W1[(size_t)pu * kD * kM + e];
+            states[kD * kM + kM + e] = p.W2[(size_t)pu * kM * kD + e];
+        }
+        for (int e = tid; e < kM; e += kThreads) states[kD * kM + e] = p.c1 ? p.c1[(size_t)pu * kM + e] : 0.f;
+        for (int e = tid; e < kD; e += kThreads) states[2 * kD * kM + kM + e] = p.c2 ? p.c2[(size_t)pu * kD + e] : 0.f;
+    }
+    __syncthreads();
+    for (int i = 0; i < nb; ++i) {
+        const int t0 = i * kB;
+        const float* S = states + (size_t)i * SZ;
+        const float* W1s = S;
+        const float* c1s = S + kD * kM;
+        const float* W2s = c1s + kM;
+        const float* c2s = W2s + kM * kD;
+        const bool last = i + 1 == nb;
+        float* N = last ? nullptr : states + (size_t)(i + 1) * SZ;
+        // where S_{i+1} goes: the next checkpoint, or the final-state outputs (c1_out, c2_out may be null)
+        float* nW1 = last ? p.W1_out + (size_t)unit * kD * kM : N;
+        float* nW2 = last ? p.W2_out + (size_t)unit * kM * kD : N + kD * kM + kM;
+        float* nc1 = !last ? N + kD * kM : p.c1_out ? p.c1_out + (size_t)unit * kM : nullptr;
+        float* nc2 = !last ? N + 2 * kD * kM + kM : p.c2_out ? p.c2_out + (size_t)unit * kD : nullptr;
+        // ---- bf16 copies of the state, token tiles, eta
+        for (int e = tid; e < kD * kM / 4; e += kThreads) {
+            const int a = (4 * e) / kM, pp = (4 * e) % kM;
+            const float4 v = reinterpret_cast<const float4*>(W1s)[e];
+            *reinterpret_cast<uint2*>(smem + kOffW1 + mm_off(8192, a, pp)) = make_uint2(pk(v.x, v.y), pk(v.z, v.w));
+            const int q = (4 * e) / kD, j = (4 * e) % kD;
+            const float4 v2 = reinterpret_cast<const float4*>(W2s)[e];
+            *reinterpret_cast<uint2*>(smem + kOffW2 + toff(q, j >> 3) + 2 * (j & 7)) =
+                make_uint2(pk(v2.x, v2.y), pk(v2.z, v2.w));
+        }
+        if (tid < 128) {
+            const int row = tid >> 3, ch = tid & 7;
+            const size_t gi = (size_t)(t0 + row) * kD + 8 * ch;
+            *reinterpret_cast<uint4*>(smem + kOffK + toff(row, ch)) = *reinterpret_cast<const uint4*>(K + gi);
+            *reinterpret_cast<uint4*>(smem + kOffQ + toff(row, ch)) = *reinterpret_cast<const uint4*>(Q + gi);
+        }
+        if (tid < kB) s_eta[tid] = p.eta ? p.eta[(size_t)unit * T + t0 + tid] : p.eta_const;
+        __syncthreads();
+        const float eta_r[2] = {s_eta[r], s_eta[r + 8]};
+        // ---- A = K W1 + c1, Aq0 = Q W1 + c1 on this warp's hidden units; Hk = GELU(A); P1 (warp 0)
+        float A_[4][4], Aq[4][4];
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) A_[nt][q] = Aq[nt][q] = c1s[ops.hid(nt, q & 1)];
+        ops.mm_AB_kn(A_, sK, 0, 4, sW1, 8192);
+        ops.mm_AB_kn(Aq, sQ, 0, 4, sW1, 8192);
+        {
+            float hk[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) hk[nt][q] = gelu_f(A_[nt][q]);
+            ops.store_mm(kOffHk, hk);
+        }
+        if (w == 0) {
+            float x[2][4] = {};
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                uint32_t a[4], b[4];
+                ldsm4(a_addr(sQ, 0, ks, l), a);
+                ldsm4(b_addr(sK, 0, ks, l), b);
+                mma(x[0], a, b[0], b[1]);
+                mma(x[1], a, b[2], b[3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int t = r + 8 * (q >> 1), s_ = 8 * nt + 2 * c + (q & 1);
+                    P1[t * 16 + s_] = s_ <= t ? x[nt][q] + 1.f : 0.f;
+                }
+        }
+        __syncthreads();   // Hk, P1
+        // ---- E = Hk W2 + c2 - V on this warp's features -> E and diag(eta) E (bf16); c2 update
+        float E_[4];
+        {
+            const float2 cc = *reinterpret_cast<const float2*>(c2s + j0 + 2 * c);
+            E_[0] = E_[2] = cc.x;
+            E_[1] = E_[3] = cc.y;
+            ops.bd_A_X(E_, sHk, sW2);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const __nv_bfloat162 v2 =
+                    *reinterpret_cast<const __nv_bfloat162*>(V + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c);
+                E_[2 * h] -= __bfloat162float(v2.x);
+                E_[2 * h + 1] -= __bfloat162float(v2.y);
+            }
+            ops.store_bd(kOffE, E_);
+            float ee[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) ee[q] = eta_r[q >> 1] * E_[q];
+            ops.store_bd(kOffDE, ee);
+            float s2[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                s2[k] = ee[k] + ee[2 + k];
+                s2[k] += __shfl_xor_sync(0xffffffffu, s2[k], 4);
+                s2[k] += __shfl_xor_sync(0xffffffffu, s2[k], 8);
+                s2[k] += __shfl_xor_sync(0xffffffffu, s2[k], 16);
+            }
+            if (r == 0 && nc2) {
+                nc2[j0 + 2 * c] = c2s[j0 + 2 * c] - s2[0];
+                nc2[j0 + 2 * c + 1] = c2s[j0 + 2 * c + 1] - s2[1];
+            }
+        }
+        __syncthreads();   // E, diag(eta) E
+        // ---- M = E W2^T, D1 = M GELU'(A) -> diag(eta) D1 (bf16); c1 update
+        {
+            float M_[4][4] = {};
+            ops.mm_A_Xt(M_, sE, sW2);
+            float s1[4][2];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) M_[nt][q] = eta_r[q >> 1] * M_[nt][q] * gelu_grad_f(A_[nt][q]);
+            ops.store_mm(kOffD1, M_);
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    s1[nt][k] = M_[nt][k] + M_[nt][2 + k];
+                    s1[nt][k] += __shfl_xor_sync(0xffffffffu, s1[nt][k], 4);
+                    s1[nt][k] += __shfl_xor_sync(0xffffffffu, s1[nt][k], 8);
+                    s1[nt][k] += __shfl_xor_sync(0xffffffffu, s1[nt][k], 16);
+                }
+            if (r == 0 && nc1)
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) nc1[ops.hid(nt, k)] = c1s[ops.hid(nt, k)] - s1[nt][k];
+        }
+        __syncthreads();   // diag(eta) D1
+        // ---- Aq = Aq0 - P1 (diag(eta) D1); Hq = GELU(Aq)
+        {
+            uint32_t a[4];
+            frag_from_f32(P1, false, nullptr, l, a);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a[q] ^= 0x80008000u;
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t b[4];
+                const int n0 = p0 + 16 * np;
+                ldsm4t(bt_addr(sD1 + (n0 >> 6) * kTileBD, n0 & 63, 0, l), b);
+                mma(Aq[2 * np], a, b[0], b[1]);
+                mma(Aq[2 * np + 1], a, b[2], b[3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) Aq[nt][q] = gelu_f(Aq[nt][q]);
+            ops.store_mm(kOffHq, Aq);
+        }
+        __syncthreads();   // Hq
+        // ---- P2 = tril(Hq Hk^T + 1);  Z = Hq W2 + c2 - P2 (diag(eta) E) on this warp's features
+        ops.tt_split(sHq, sHk, P2, 1.f, 1.f);
+        if (Z) {
+            float z[4];
+            const float2 cc = *reinterpret_cast<const float2*>(c2s + j0 + 2 * c);
+            z[0] = z[2] = cc.x;
+            z[1] = z[3] = cc.y;
+            ops.bd_A_X(z, sHq, sW2);
+            uint32_t a[4], b[4];
+            frag_from_f32(P2, false, nullptr, l, a);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a[q] ^= 0x80008000u;
+            ldsm4t(bt_addr(sEE, jn0, 0, l), b);
+            mma(z, a, jh ? b[2] : b[0], jh ? b[3] : b[1]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+                *reinterpret_cast<__nv_bfloat162*>(Z + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c) =
+                    __floats2bfloat162_rn(z[2 * h], z[2 * h + 1]);
+        }
+        // ---- S_{i+1}: W1 - K^T diag(eta) D1 and W2 - Hk^T diag(eta) E, this warp's blocks
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt) {
+            float x[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    x[nt][q] = W1s[(size_t)(16 * mt + r + 8 * (q >> 1)) * kM + ops.hid(nt, q & 1)];
+            uint32_t ak[4];
+            ldsm4t(at_addr(sK, 16 * mt, l), ak);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) ak[q] ^= 0x80008000u;
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+                uint32_t b[4];
+                const int n0 = p0 + 16 * np;
+                ldsm4t(bt_addr(sD1 + (n0 >> 6) * kTileBD, n0 & 63, 0, l), b);
+                mma(x[2 * np], ak, b[0], b[1]);
+                mma(x[2 * np + 1], ak, b[2], b[3]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    *reinterpret_cast<float2*>(nW1 + (size_t)(16 * mt + r + 8 * h) * kM + ops.hid(nt, 0)) =
+                        make_float2(x[nt][2 * h], x[nt][2 * h + 1]);
+        }
+#pragma unroll 1
+        for (int mt = 0; mt < 2; ++mt) {
+            const int pr = p0 + 16 * mt;
+            uint32_t ak[4];
+            ldsm4t(at_addr(sHk + (pr >> 6) * kTileBD, pr & 63, l), ak);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) ak[q] ^= 0x80008000u;
+#pragma unroll 1
+            for (int np = 0; np < 4; ++np) {
+                float x[2][4];
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        x[nt][q] = W2s[(size_t)(pr + r + 8 * (q >> 1)) * kD + 16 * np + 8 * nt + 2 * c + (q & 1)];
+                uint32_t b[4];
+                ldsm4t(bt_addr(sEE, 16 * np, 0, l), b);
+                mma(x[0], ak, b[0], b[1]);
+                mma(x[1], ak, b[2], b[3]);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        *reinterpret_cast<float2*>(nW2 + (size_t)(pr + r + 8 * h) * kD + 16 * np + 8 * nt + 2 * c) =
+                            make_float2(x[nt][2 * h], x[nt][2 * h + 1]);
+            }
+        }
+        __syncthreads();   // S_{i+1} written; every read of this mini-batch's shared data is done
+    }
+    if (nb == 0) {
+        // no mini-batch: the final state is the initial one
+        for (int e = tid; e < kD * kM; e += kThreads) {
+            p.W1_out[(size_t)unit * kD * kM + e] = p.W1[(size_t)pu * kD * kM + e];
+            p.W2_out[(size_t)unit * kM * kD + e] = p.W2[(size_t)pu * kM * kD + e];
+        }
+        if (p.c1_out)
+            for (int e = tid; e < kM; e += kThreads) p.c1_out[(size_t)unit * kM + e] = p.c1 ? p.c1[(size_t)pu * kM + e] : 0.f;
+        if (p.c2_out)
+            for (int e = tid; e < kD; e += kThreads) p.c2_out[(size_t)unit * kD + e] = p.c2 ? p.c2[(size_t)pu * kD + e] : 0.f;
     }
 }
 

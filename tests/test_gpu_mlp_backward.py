@@ -68,7 +68,10 @@ def _check(inp, c1, c2, dz, ups, per_token, states, grads):
         st = O.mlp_forward(e["Q"][:, :, :t], e["K"][:, :, :t], e["V"][:, :, :t], eta[:, :, :t], *params, w.b)[1:]
         parts = np.split(states[:, :, i], [d * m, d * m + m, 2 * d * m + m], axis=-1)
         for g, r in zip(parts, st):
-            assert maxrel(g.reshape(r.shape), r) <= 1e-4
+            if w.io_dtype == WL.BF16:
+                assert normwise(g.reshape(r.shape), r) <= 2e-2
+            else:
+                assert maxrel(g.reshape(r.shape), r) <= 1e-4
     for nm, got, want in zip(["dQ", "dK", "dV", "deta", "dW1", "dc1", "dW2", "dc2"], grads, ref):
         if got is None:
             continue
