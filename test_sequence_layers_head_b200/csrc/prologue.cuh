@@ -69,6 +69,22 @@ struct PrologueParams {
     unsigned flags;
 };
 
+// The tile plan of one call (host side): everything in PrologueParams but the pointers.
+inline void prologue_plan(PrologueParams& p, long long rows, int T, int H, int d, int Dm, bool gate) {
+    const int Hd = H * d;
+    p.rows = (int)rows;
+    p.T = T;
+    p.H = H;
+    p.d = d;
+    p.Hd = Hd;
+    p.nk = (Dm + kBK - 1) / kBK;
+    p.nvt = (Hd + kBN - 1) / kBN;
+    p.ntn = 3 * p.nvt + (gate ? 1 : 0);
+    p.tiles = ((rows + kBM - 1) / kBM) * p.ntn;
+    p.brows = Hd < kBN ? Hd : kBN;
+    p.ng = (H + 15) / 16 * 16;
+}
+
 struct Tile {
     int m0;     // first token
     int view;   // 0, 1, 2: Q, K, V; 3: the gate

@@ -617,17 +617,7 @@ extern "C" ttt_status ttt_qkv_prologue(const ttt_qkv_prologue_args* a, cudaStrea
     using namespace pro;
     const int Hd = a->H * a->d;
     PrologueParams p;
-    p.rows = (int)rows;
-    p.T = a->T;
-    p.H = a->H;
-    p.d = a->d;
-    p.Hd = Hd;
-    p.nk = (a->Dm + kBK - 1) / kBK;
-    p.nvt = (Hd + kBN - 1) / kBN;
-    p.ntn = 3 * p.nvt + (a->theta_lr ? 1 : 0);
-    p.tiles = ((rows + kBM - 1) / kBM) * p.ntn;
-    p.brows = Hd < kBN ? Hd : kBN;
-    p.ng = (a->H + 15) / 16 * 16;
+    prologue_plan(p, rows, a->T, a->H, a->d, a->Dm, a->theta_lr != nullptr);
     p.Q = static_cast<__nv_bfloat16*>(a->Q);
     p.K = static_cast<__nv_bfloat16*>(a->K);
     p.V = static_cast<__nv_bfloat16*>(a->V);

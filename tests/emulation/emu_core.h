@@ -34,6 +34,7 @@
 namespace emu {
 constexpr int kMaxThreads = 1024;
 inline thread_local uint3 tid3, bid3;
+inline uint3 grid3;
 inline std::barrier<>* block_bar = nullptr;
 inline std::barrier<>* warp_bar[kMaxThreads / 32];
 inline const uint8_t* shared_base = nullptr;
@@ -50,6 +51,7 @@ inline void warp_sync() { warp_bar[tid3.x >> 5]->arrive_and_wait(); }
 template <typename F>
 void run_grid(int blocks, int threads, const void* shared, F f) {
     shared_base = static_cast<const uint8_t*>(shared);
+    grid3 = make_uint3(blocks, 1, 1);
     for (int bx = 0; bx < blocks; ++bx) {
         std::barrier<> bb(threads);
         for (int w = 0; w < threads / 32; ++w) warp_bar[w] = new std::barrier<>(32);
@@ -88,8 +90,10 @@ inline uint16_t ld16(uint32_t saddr) {
 
 #undef threadIdx
 #undef blockIdx
+#undef gridDim
 #define threadIdx emu::tid3
 #define blockIdx emu::bid3
+#define gridDim emu::grid3
 inline void __syncthreads() { emu::block_bar->arrive_and_wait(); }
 inline float __shfl_xor_sync(unsigned, float v, int o) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;

@@ -1,0 +1,195 @@
+// Host emulation of the sm_100a asynchronous operations used by the tensor-core
+// prologue kernel, on top of emu_core.h: TEST INFRASTRUCTURE, never part of the
+// library.
+//
+// Semantics (from the PTX ISA's descriptions):
+//   mbarrier: an expected arrival count and a transaction count per phase; the
+//     phase completes when both reach zero, then the next phase starts with the
+//     initial arrival count.  try_wait.parity(P) succeeds once the phase with
+//     parity P has completed, i.e. when the current phase's parity differs from P.
+//   cp.async.bulk.tensor (2-D tile, 128-byte swizzle): the box is copied to
+//     shared memory with the 16-byte chunk c of row r stored at chunk c ^ (r % 8);
+//     elements outside the tensor are zero; the whole box's bytes count toward
+//     the mbarrier's transaction count.
+//   tcgen05.mma kind::f16 (bf16 x bf16 -> f32), K = 16, both operands K-major
+//     with the 128-byte swizzle: element (row, k) of an operand is at byte
+//     start + (row / 8) * SBO + (row % 8) * 128 + 2 k, with address bits 4-6
+//     XORed with bits 7-9.  D (M x N) is at TMEM lanes 0 .. M-1, columns
+//     col .. col + N - 1.
+//   tcgen05.ld .32x32b.xN: lane t of the warp reads TMEM lane (base + t),
+//     columns col .. col + N - 1; a warp may access the 32 lanes of its
+//     quadrant (warp % 4) only.
+//   tcgen05.commit: arrives once on the mbarrier when the MMAs issued before it
+//     have completed.
+// Asynchronous operations complete when they are issued: one of the schedules
+// the hardware may produce, which a correct kernel must handle.
+#pragma once
+#include <atomic>
+#include <chrono>
+#include <cuda.h>
+#include <map>
+#include <mutex>
+#include <thread>
+
+#include "emu_core.h"
+
+namespace emu {
+struct Bar {
+    int count = 0, pending = 0;
+    long long tx = 0;
+    unsigned phase = 0;
+};
+inline std::mutex bar_mu;
+inline std::map<const void*, Bar> bars;
+inline uint32_t tmem[128][512];
+inline std::atomic<int> errors{0};   // emulated-hardware rule violations (quadrant, layout)
+
+// what the harness puts in a CUtensorMap
+struct FakeMap {
+    const void* base;
+    unsigned long long cols, rows, pitch;   // elements, elements, bytes
+    unsigned box_cols, box_rows, elem;      // elements, elements, bytes per element
+    int swizzle128;
+};
+static_assert(sizeof(FakeMap) <= sizeof(CUtensorMap), "tensor map space");
+inline void make_map(CUtensorMap* m, const void* base, unsigned long long cols, unsigned long long rows,
+                     unsigned long long pitch, unsigned box_cols, unsigned box_rows, unsigned elem) {
+    std::memset(m, 0, sizeof(*m));
+    FakeMap f{base, cols, rows, pitch, box_cols, box_rows, elem, 1};
+    std::memcpy(m, &f, sizeof(f));
+}
+
+inline void complete_if_done(Bar& b) {
+    if (b.pending == 0 && b.tx == 0) {
+        ++b.phase;
+        b.pending = b.count;
+    }
+}
+inline void bar_arrive(const void* bar, long long tx_add) {
+    std::lock_guard<std::mutex> lk(bar_mu);
+    Bar& b = bars[bar];
+    b.tx += tx_add;
+    --b.pending;
+    complete_if_done(b);
+}
+inline void bar_complete_tx(const void* bar, long long bytes) {
+    std::lock_guard<std::mutex> lk(bar_mu);
+    Bar& b = bars[bar];
+    b.tx -= bytes;
+    complete_if_done(b);
+}
+inline uint32_t tmem_lane(uint32_t a) { return a >> 16; }
+inline uint32_t tmem_col(uint32_t a) { return a & 0xFFFFu; }
+}  // namespace emu
+
+#undef __grid_constant__
+#define __grid_constant__
+inline float __uint_as_float(uint32_t v) {
+    float f;
+    std::memcpy(&f, &v, 4);
+    return f;
+}
+inline int atomicOr(int* p, int v) { return __atomic_fetch_or(p, v, __ATOMIC_SEQ_CST); }
+inline void __syncwarp(unsigned = 0xffffffffu) { emu::warp_sync(); }
+
+namespace ttt {
+inline void mbar_init(uint64_t* bar, uint32_t count) {
+    std::lock_guard<std::mutex> lk(emu::bar_mu);
+    emu::Bar& b = emu::bars[bar];
+    b.count = b.pending = (int)count;
+    b.tx = 0;
+    b.phase = 0;
+}
+inline void fence_mbar_init() {}
+inline void mbar_arrive(uint64_t* bar) { emu::bar_arrive(bar, 0); }
+inline void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) { emu::bar_arrive(bar, bytes); }
+inline bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    std::lock_guard<std::mutex> lk(emu::bar_mu);
+    return (emu::bars[bar].phase & 1u) != (parity & 1u);
+}
+inline uint64_t globaltimer_ns() {
+    return (uint64_t)std::chrono::duration_cast<std::chrono::nanoseconds>(
+               std::chrono::steady_clock::now().time_since_epoch())
+        .count();
+}
+inline bool wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns, volatile int* abort) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (abort && *abort) return false;
+        if (globaltimer_ns() - t0 > limit_ns) return false;
+        std::this_thread::yield();
+    }
+}
+inline void fence_proxy_async_smem() {}
+inline void prefetch_tmap(const CUtensorMap*) {}
+// 2-D tiled load, 128-byte swizzle, out-of-range elements zero
+inline void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+    emu::FakeMap f;
+    std::memcpy(&f, map, sizeof(f));
+    uint8_t* d = static_cast<uint8_t*>(dst);
+    const unsigned rowb = f.box_cols * f.elem;
+    if (((uintptr_t)(d - emu::shared_base)) % 1024 != 0 || rowb != 128 || (x * f.elem) % 16 != 0) ++emu::errors;
+    for (unsigned r = 0; r < f.box_rows; ++r)
+        for (unsigned cb = 0; cb < rowb; ++cb) {
+            const long long gx = (long long)x + cb / f.elem, gy = (long long)y + r;
+            uint8_t v = 0;
+            if (gx >= 0 && gy >= 0 && (unsigned long long)gx < f.cols && (unsigned long long)gy < f.rows)
+                v = static_cast<const uint8_t*>(f.base)[gy * f.pitch + gx * f.elem + cb % f.elem];
+            const unsigned chunk = (cb >> 4) ^ (r & 7);
+            d[r * 128 + chunk * 16 + (cb & 15)] = v;
+        }
+    emu::bar_complete_tx(bar, (long long)rowb * f.box_rows);
+}
+inline void tmem_alloc(uint32_t* dst, uint32_t) { *dst = 0; }
+inline void tmem_relinquish() {}
+inline void tmem_dealloc(uint32_t, uint32_t) {}
+inline void tc_fence_before() {}
+inline void tc_fence_after() {}
+inline void tmem_wait_ld() {}
+inline void tmem_wait_st() {}
+template <int N>
+inline void tmem_ld_32x32b(uint32_t taddr, uint32_t* r) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const uint32_t l0 = emu::tmem_lane(taddr), c0 = emu::tmem_col(taddr);
+    if (l0 / 32 != (uint32_t)(w % 4) || l0 % 32 != 0 || c0 + N > 512) ++emu::errors;
+    for (int i = 0; i < N; ++i) r[i] = emu::tmem[(l0 + lane) & 127][(c0 + i) & 511];
+    emu::warp_sync();
+}
+inline void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b<16>(taddr, r); }
+inline void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b<32>(taddr, r); }
+
+// The descriptors are the library's own encoding (make_sdesc, make_idesc_bf16 in ptx.cuh); layout
+// code 2 is the 128-byte swizzle.
+// element (row, k) of a K-major, 128-byte-swizzled bf16 operand
+inline float sw128_elem(uint64_t desc, int row, int k) {
+    const uint32_t start = (uint32_t)(desc & 0x3FFFu) << 4;
+    const uint32_t sbo = (uint32_t)((desc >> 32) & 0x3FFFu) << 4;
+    const uint32_t lin = start + (row / 8) * sbo + (row % 8) * 128 + 2 * k;
+    const uint32_t phys = lin ^ (((lin >> 7) & 7u) << 4);
+    const uint16_t h = emu::ld16(phys);
+    uint32_t b = (uint32_t)h << 16;
+    float f;
+    std::memcpy(&f, &b, 4);
+    return f;
+}
+inline void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+    const int M = (int)((idesc >> 24) & 0x1Fu) << 4, N = (int)((idesc >> 17) & 0x3Fu) << 3;
+    const bool a_mn = (idesc >> 15) & 1u, b_mn = (idesc >> 16) & 1u;
+    if (a_mn || b_mn || (adesc >> 61) != 2u || (bdesc >> 61) != 2u || M != 128 ||
+        N % 16 != 0 || N < 16 || N > 256 || ((adesc & 0x3FFFu) << 4) % 16 != 0)
+        ++emu::errors;
+    const uint32_t l0 = emu::tmem_lane(d_tmem), c0 = emu::tmem_col(d_tmem);
+    for (int row = 0; row < M; ++row)
+        for (int col = 0; col < N; ++col) {
+            float acc = 0.f;
+            for (int k = 0; k < 16; ++k) acc += sw128_elem(adesc, row, k) * sw128_elem(bdesc, col, k);
+            uint32_t& cell = emu::tmem[(l0 + row) & 127][(c0 + col) & 511];
+            float prev;
+            std::memcpy(&prev, &cell, 4);
+            const float v = (accumulate ? prev : 0.f) + acc;
+            std::memcpy(&cell, &v, 4);
+        }
+}
+inline void umma_commit(uint64_t* bar) { emu::bar_arrive(bar, 0); }
+}  // namespace ttt

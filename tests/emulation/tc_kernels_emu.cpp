@@ -1,0 +1,47 @@
+// Entry points of the CPU tests' host emulation of the tensor-core (tcgen05)
+// kernels (tc_emu.h and emu_core.h have the execution model): TEST
+// INFRASTRUCTURE; the library has no CPU path.
+#include "tc_emu.h"
+
+namespace ttt {
+namespace pro {
+alignas(1024) uint8_t smem[4 * 65536];
+}
+}  // namespace ttt
+
+#include "../../test_sequence_layers_head_b200/csrc/prologue.cuh"
+
+// the fused prologue on tcgen05 with the library's tile plan and tensor maps, on `grid` persistent CTAs;
+// returns the number of emulated-hardware rule violations (0 when none), or -1 for a bad request
+extern "C" int emu_prologue_tc(int B, int T, int Dm, int H, int d, const void* x, const void* tq, const void* tk,
+                               const void* tv, const void* tl, float eta_base, void* Q, void* K, void* V,
+                               float* eta, int grid, int* status) {
+    using namespace ttt::pro;
+    const long long rows = (long long)B * T;
+    if (rows == 0 || Dm % 8 || H > 256) return -1;
+    PrologueParams p{};
+    prologue_plan(p, rows, T, H, d, Dm, tl != nullptr);
+    p.Q = static_cast<__nv_bfloat16*>(Q);
+    p.K = static_cast<__nv_bfloat16*>(K);
+    p.V = static_cast<__nv_bfloat16*>(V);
+    p.eta = eta;
+    p.eta_base = eta_base;
+    p.status = status;
+    p.wait_ns = 120ull * 1000000000ull;   // generous: the emulated threads share few host cores
+    p.flags = 0;
+    const unsigned long long pitch = (unsigned long long)Dm * 2;
+    CUtensorMap mX, mTq, mTk, mTv, mTl;
+    emu::make_map(&mX, x, Dm, rows, pitch, kBK, kBM, 2);
+    emu::make_map(&mTq, tq, Dm, p.Hd, pitch, kBK, p.brows, 2);
+    emu::make_map(&mTk, tk, Dm, p.Hd, pitch, kBK, p.brows, 2);
+    emu::make_map(&mTv, tv, Dm, p.Hd, pitch, kBK, p.brows, 2);
+    if (tl)
+        emu::make_map(&mTl, tl, Dm, H, pitch, kBK, p.ng, 2);
+    else
+        mTl = mX;
+    const int g = (int)(p.tiles < grid ? p.tiles : grid);
+    emu::errors = 0;
+    // a persistent CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...: gridDim must be the grid
+    emu::run_grid(g, kThreads, smem, [&] { prologue_kernel(mX, mTq, mTk, mTv, mTl, p); });
+    return emu::errors.load();
+}

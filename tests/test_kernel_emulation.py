@@ -1,8 +1,9 @@
-"""The library's CUDA-core and mma.sync kernels' own source, run on the CPU
-under a host emulation of the CUDA execution model (tests/emulation: one
-std::thread per CUDA thread, __syncthreads as a barrier, shuffles, ldmatrix
-and mma through a per-warp exchange with the PTX ISA's documented fragment
-layouts), against the float64 oracle.
+"""The library's kernels' own source, run on the CPU under a host emulation of
+the CUDA execution model (tests/emulation: one std::thread per CUDA thread,
+__syncthreads as a barrier, shuffles, ldmatrix and mma through a per-warp
+exchange with the PTX ISA's documented fragment layouts; for the tcgen05
+prologue also mbarriers, 2-D TMA loads, tensor memory and tcgen05.mma, with
+asynchronous operations completing at issue), against the float64 oracle.
 
 This checks the source's index arithmetic, phase order and barrier placement
 where no GPU is present.  It is not the GPU parity: the tests marked gpu run
@@ -13,8 +14,8 @@ Covered: the TTT-MLP forward writing its batch-start states and the
 outer-loop backward that reads them (fp32 CUDA cores); the TTT-Linear pair
 on mma.sync (bf16, d = 64, b = 16) -- already verified on the B200, which
 pins the emulated ldmatrix / mma semantics; and the LN+residual pair on
-mma.sync; the TTT-MLP backward on mma.sync; and the fused prologue on fp32
-CUDA cores (paper digest
+mma.sync; the TTT-MLP training pair on mma.sync; and the fused prologue on
+fp32 CUDA cores and on tcgen05 (paper digest
 "论文速览 | TTT", sections 3.3, 3.4, 3.6, 3.7, 4.4, 4.6, 6.12).
 """
 import ctypes
@@ -324,3 +325,46 @@ def test_mlp_forward_states_on_mma_sync(emu, B, H, T, per_token):
         parts = np.split(states[:, :, i], [d * m, d * m + m, 2 * d * m + m], axis=-1)
         for g, r in zip(parts, st):
             assert normwise(g.astype(np.float64).reshape(r.shape), r) < 2e-2
+
+
+@pytest.fixture(scope="module")
+def tc_emu(tmp_path_factory):
+    so = str(tmp_path_factory.mktemp("tcemu") / "tc_kernels_emu.so")
+    subprocess.run(["g++", "-std=c++20", "-O1", "-fPIC", "-shared", "-I/usr/local/cuda/include", "-o", so,
+                    os.path.join(ROOT, "tests", "emulation", "tc_kernels_emu.cpp"), "-lpthread"], check=True)
+    return ctypes.CDLL(so)
+
+
+@pytest.mark.parametrize("B,T,Dm,H,d,gate,grid", [
+    (1, 8, 64, 1, 16, True, 1),        # one tile of each kind
+    (2, 200, 136, 5, 64, True, 3),     # ragged tokens and width, a partial column tile, persistent CTAs
+    (3, 100, 72, 17, 16, True, 2),     # H not a multiple of 16 in the gate tile
+    (2, 77, 64, 12, 64, False, 4),     # no gate
+    (4, 33, 16, 7, 32, True, 1),       # width below one chunk
+    (2, 64, 768, 12, 64, True, 7),     # the 12-head width
+])
+def test_prologue_on_tcgen05(tc_emu, B, T, Dm, H, d, gate, grid):
+    """The tcgen05 prologue kernel with the library's tile plan and tensor maps: every output written, the
+    views within one bf16 rounding plus the fp32 accumulation bound, the gate within its bound, no
+    emulated-hardware rule broken (TMA alignment, TMEM lane quadrant, MMA shape), no expired wait."""
+    w, inp = WL.prologue_case(B, T, Dm, H, d, gate=gate, eta_base=0.5)
+    r, e = inp["raw"], inp["exact"]
+    Q, K, V = (np.full((B, H, T, d), 0x7FC0, np.uint16) for _ in range(3))   # NaN until written
+    eta = np.full((B, H, T), np.nan, np.float32) if gate else None
+    status = np.zeros(1, np.int32)
+    f = tc_emu.emu_prologue_tc
+    f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 4 + \
+        [ctypes.c_int, ctypes.c_void_p]
+    rc = f(B, T, Dm, H, d, _p(r["x"]), _p(r["theta_q"]), _p(r["theta_k"]), _p(r["theta_v"]),
+           _p(r["theta_lr"]) if gate else None, 0.5, _p(Q), _p(K), _p(V), _p(eta), grid, _p(status))
+    assert rc == 0 and status[0] == 0
+    ref = O.qkv_prologue(e["x"], e["theta_q"], e["theta_k"], e["theta_v"], e["theta_lr"], 0.5, d)
+    for got, want, nm in zip((Q, K, V), ref[:3], ("theta_q", "theta_k", "theta_v")):
+        g = WL.bf16_bits_to_f64(got)
+        S = (np.abs(e["x"]) @ np.abs(e[nm]).T).reshape(B, T, H, d).transpose(0, 2, 1, 3)
+        assert np.all(np.isfinite(g))
+        assert np.all(np.abs(g - want) <= 2.0 ** -8 * np.abs(want) + 2.0 ** -12 * S)
+    if gate:
+        S_lr = (np.abs(e["x"]) @ np.abs(e["theta_lr"]).T).transpose(0, 2, 1)
+        assert np.all(np.isfinite(eta))
+        assert np.all(np.abs(eta - ref[3]) <= 0.5 * (2.0 ** -12 * S_lr / 4 + 1e-6))
