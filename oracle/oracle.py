@@ -44,6 +44,9 @@ def lib():
         L.ttt_oracle_mlp_backward.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, ll, P, P, P, P, P,
                                               P, P, P, P, P, P, P, P, i]
         L.ttt_oracle_mlp_backward.restype = i
+        L.ttt_oracle_mlp_ln_backward.argtypes = [i, i, i, i, i, i, P, P, P, P, P, P, P, P, ll, P, P, dbl, P, P, P,
+                                                 P, P, P, P, P, P, P, P, P, P, P, P, i]
+        L.ttt_oracle_mlp_ln_backward.restype = i
         L.ttt_oracle_qkv_prologue.argtypes = [i, i, i, i, i, P, P, P, P, P, dbl, P, P, P, P, i]
         L.ttt_oracle_qkv_prologue.restype = i
         _lib = L
@@ -216,3 +219,30 @@ def qkv_prologue(x, theta_q, theta_k, theta_v, theta_lr, eta_base, d, threads=No
     if rc != 0:
         raise ValueError("oracle: invalid arguments")
     return Q, K, V, eta
+
+
+def mlp_ln_backward(Q, K, V, eta, W1, c1, W2, c2, b, gamma, beta, eps=1e-6, dZ=None, dW1_out=None, dc1_out=None,
+                    dW2_out=None, dc2_out=None, threads=None):
+    """Outer-loop gradients of TTT-MLP with LN+residual on the output layer,
+    reverse mode through the primal loop.  Parameters [H,...] (shared) or
+    [B,H,...]; gamma, beta [H,d].  Returns (dQ, dK, dV, deta, dW1, dc1, dW2,
+    dc2, dgamma, dbeta), the parameter gradients per unit [B,H,...] (sum over
+    what is shared)."""
+    Q, K, V, eta, W1, c1, W2, c2, gamma, beta = map(_f64, (Q, K, V, eta, W1, c1, W2, c2, gamma, beta))
+    dZ, dW1_out, dc1_out, dW2_out, dc2_out = map(_f64, (dZ, dW1_out, dc1_out, dW2_out, dc2_out))
+    B, H, T, d = Q.shape
+    m = W1.shape[-1]
+    per_seq = 1 if W1.ndim == 4 else 0
+    dQ, dK, dV = np.empty((B, H, T, d)), np.empty((B, H, T, d)), np.empty((B, H, T, d))
+    deta = np.empty((B, H, T))
+    dW1, dc1 = np.empty((B, H, d, m)), np.empty((B, H, m))
+    dW2, dc2 = np.empty((B, H, m, d)), np.empty((B, H, d))
+    dgamma, dbeta = np.empty((B, H, d)), np.empty((B, H, d))
+    rc = lib().ttt_oracle_mlp_ln_backward(B, H, T, d, m, b, _p(Q), _p(K), _p(V), _p(eta), _p(W1), _p(c1), _p(W2),
+                                          _p(c2), per_seq, _p(gamma), _p(beta), float(eps), _p(dZ), _p(dW1_out),
+                                          _p(dc1_out), _p(dW2_out), _p(dc2_out), _p(dQ), _p(dK), _p(dV), _p(deta),
+                                          _p(dW1), _p(dc1), _p(dW2), _p(dc2), _p(dgamma), _p(dbeta),
+                                          threads or default_threads())
+    if rc != 0:
+        raise ValueError("oracle: invalid arguments")
+    return dQ, dK, dV, deta, dW1, dc1, dW2, dc2, dgamma, dbeta

@@ -1006,3 +1006,284 @@ int ttt_oracle_qkv_prologue(int B, int T, int Dm, int H, int d, const double *x,
     (void)nthreads;
     return 0;
 }
+
+/*
+ * Outer-loop gradients of TTT-MLP with LN+residual on the output layer,
+ * f(x) = x + gamma LN(GELU(x W1 + c1) W2 + c2) + beta (section 4.4; section 3.4
+ * for the outer loop): reverse-mode differentiation of the primal loop of
+ * mlp_unit (use_ln = 1), token by token.  Per token, at the batch-start state
+ * S: a = k W1 + c1, h = GELU(a), y = h W2 + c2, Delta2 = the LN+residual
+ * backward at y (as in ln_residual_delta), m = Delta2 W2^T, d1 = m GELU'(a);
+ * the updates use d1 and Delta2; the output is z = q + gamma LN(p) + beta with
+ * p = GELU(q W1_t + c1_t) W2_t + c2_t at the state after the token.
+ */
+static void mlp_ln_unit_backward(int T, int d, int m, int b, const double *Q, const double *K, const double *V,
+                                 const double *eta, const double *W1_0, const double *c1_0, const double *W2_0,
+                                 const double *c2_0, const double *gamma, const double *beta, double eps,
+                                 const double *dZ, const double *dW1o, const double *dc1o, const double *dW2o,
+                                 const double *dc2o, double *dQ, double *dK, double *dV, double *deta, double *dW1,
+                                 double *dc1, double *dW2, double *dc2, double *dgamma, double *dbeta) {
+    const size_t n1 = (size_t)d * m;
+    const int nb = (T + b - 1) / b;
+    const size_t sz = n1 + m + n1 + d;   /* one state: W1, c1, W2, c2 */
+    double *starts = malloc((size_t)(nb > 0 ? nb : 1) * sz * sizeof(double));
+    double *run = malloc((size_t)(b + 1) * sz * sizeof(double));
+    double *cur = malloc(sz * sizeof(double));
+    double *D = malloc(sz * sizeof(double)), *Ds = malloc(sz * sizeof(double));
+    /* per token of a batch */
+    double *A = malloc((size_t)b * m * sizeof(double)), *Hh = malloc((size_t)b * m * sizeof(double));
+    double *Mm = malloc((size_t)b * m * sizeof(double)), *D1 = malloc((size_t)b * m * sizeof(double));
+    double *XH = malloc((size_t)b * d * sizeof(double)), *EE = malloc((size_t)b * d * sizeof(double));
+    double *UU = malloc((size_t)b * d * sizeof(double)), *D2 = malloc((size_t)b * d * sizeof(double));
+    double *RR = malloc((size_t)b * sizeof(double)), *MGX = malloc((size_t)b * sizeof(double));
+    double *y = malloc(d * sizeof(double)), *pp = malloc(d * sizeof(double)), *xo = malloc(d * sizeof(double));
+    double *t1 = malloc(d * sizeof(double)), *dp = malloc(d * sizeof(double)), *dd2 = malloc(d * sizeof(double));
+    double *du = malloc(d * sizeof(double)), *dxh = malloc(d * sizeof(double)), *dy = malloc(d * sizeof(double));
+    double *aq = malloc(m * sizeof(double)), *hq = malloc(m * sizeof(double)), *daq = malloc(m * sizeof(double));
+    double *dd1 = malloc(m * sizeof(double)), *dm = malloc(m * sizeof(double)), *dh = malloc(m * sizeof(double));
+    double *da = malloc(m * sizeof(double));
+    #define W1P(x) (x)
+    #define C1P(x) ((x) + n1)
+    #define W2P(x) ((x) + n1 + m)
+    #define C2P(x) ((x) + n1 + m + n1)
+
+    /* token i of the batch at the batch-start state S: a, h, the LN quantities, Delta2, m, d1 */
+    #define BATCH_FWD(t, i, S)                                                                         \
+        do {                                                                                           \
+            const double *k_ = K + (size_t)(t) * d, *v_ = V + (size_t)(t) * d;                         \
+            double *a_ = A + (size_t)(i) * m, *h_ = Hh + (size_t)(i) * m;                              \
+            double *x_ = XH + (size_t)(i) * d, *e_ = EE + (size_t)(i) * d;                             \
+            double *u_ = UU + (size_t)(i) * d, *d2_ = D2 + (size_t)(i) * d;                            \
+            vec_mat(d, m, k_, W1P(S), a_);                                                             \
+            for (int p = 0; p < m; ++p) { a_[p] += C1P(S)[p]; h_[p] = gelu(a_[p]); }                   \
+            vec_mat(m, d, h_, W2P(S), y);                                                              \
+            for (int j = 0; j < d; ++j) y[j] += C2P(S)[j];                                             \
+            RR[i] = layer_norm(d, y, eps, x_);                                                         \
+            double mg = 0.0, mgx_ = 0.0;                                                               \
+            for (int j = 0; j < d; ++j) {                                                              \
+                e_[j] = k_[j] + gamma[j] * x_[j] + beta[j] - v_[j];                                    \
+                mg += gamma[j] * e_[j];                                                                \
+                mgx_ += gamma[j] * e_[j] * x_[j];                                                      \
+            }                                                                                          \
+            mg /= d;                                                                                   \
+            mgx_ /= d;                                                                                 \
+            MGX[i] = mgx_;                                                                             \
+            for (int j = 0; j < d; ++j) {                                                              \
+                u_[j] = gamma[j] * e_[j] - mg - x_[j] * mgx_;                                          \
+                d2_[j] = RR[i] * u_[j];                                                                \
+            }                                                                                          \
+            for (int p = 0; p < m; ++p) {                                                              \
+                double acc = 0.0;                                                                      \
+                for (int j = 0; j < d; ++j) acc += W2P(S)[(size_t)p * d + j] * d2_[j];                 \
+                Mm[(size_t)(i) * m + p] = acc;                                                         \
+                D1[(size_t)(i) * m + p] = acc * gelu_grad(a_[p]);                                      \
+            }                                                                                          \
+        } while (0)
+    /* one token's update applied to state X (in place) */
+    #define TOKEN_UPD(t, i, X)                                                                         \
+        do {                                                                                           \
+            const double *k_ = K + (size_t)(t) * d, et_ = eta[t];                                      \
+            const double *d1_ = D1 + (size_t)(i) * m, *h_ = Hh + (size_t)(i) * m;                      \
+            const double *d2_ = D2 + (size_t)(i) * d;                                                  \
+            for (int a2 = 0; a2 < d; ++a2)                                                             \
+                for (int p = 0; p < m; ++p) W1P(X)[(size_t)a2 * m + p] -= et_ * k_[a2] * d1_[p];       \
+            for (int p = 0; p < m; ++p) C1P(X)[p] -= et_ * d1_[p];                                     \
+            for (int p = 0; p < m; ++p)                                                                \
+                for (int j = 0; j < d; ++j) W2P(X)[(size_t)p * d + j] -= et_ * h_[p] * d2_[j];         \
+            for (int j = 0; j < d; ++j) C2P(X)[j] -= et_ * d2_[j];                                     \
+        } while (0)
+
+    memcpy(W1P(cur), W1_0, n1 * sizeof(double));
+    if (c1_0) memcpy(C1P(cur), c1_0, m * sizeof(double)); else memset(C1P(cur), 0, m * sizeof(double));
+    memcpy(W2P(cur), W2_0, n1 * sizeof(double));
+    if (c2_0) memcpy(C2P(cur), c2_0, d * sizeof(double)); else memset(C2P(cur), 0, d * sizeof(double));
+    for (int i = 0; i < nb; ++i) {
+        const int t0 = i * b, t1_ = (t0 + b < T) ? t0 + b : T;
+        memcpy(starts + (size_t)i * sz, cur, sz * sizeof(double));
+        for (int t = t0; t < t1_; ++t) BATCH_FWD(t, t - t0, starts + (size_t)i * sz);
+        for (int t = t0; t < t1_; ++t) TOKEN_UPD(t, t - t0, cur);
+    }
+    memset(D, 0, sz * sizeof(double));
+    if (dW1o) memcpy(W1P(D), dW1o, n1 * sizeof(double));
+    if (dc1o) memcpy(C1P(D), dc1o, m * sizeof(double));
+    if (dW2o) memcpy(W2P(D), dW2o, n1 * sizeof(double));
+    if (dc2o) memcpy(C2P(D), dc2o, d * sizeof(double));
+    memset(dgamma, 0, d * sizeof(double));
+    memset(dbeta, 0, d * sizeof(double));
+    for (int i = nb - 1; i >= 0; --i) {
+        const int t0 = i * b, t1_ = (t0 + b < T) ? t0 + b : T;
+        const double *S = starts + (size_t)i * sz;
+        for (int t = t0; t < t1_; ++t) BATCH_FWD(t, t - t0, S);
+        memcpy(run, S, sz * sizeof(double));
+        for (int t = t0; t < t1_; ++t) {
+            memcpy(run + (size_t)(t - t0 + 1) * sz, run + (size_t)(t - t0) * sz, sz * sizeof(double));
+            TOKEN_UPD(t, t - t0, run + (size_t)(t - t0 + 1) * sz);
+        }
+        memset(Ds, 0, sz * sizeof(double));
+        for (int t = t1_ - 1; t >= t0; --t) {
+            const int li = t - t0;
+            const double *q = Q + (size_t)t * d, *k = K + (size_t)t * d;
+            const double *Rt = run + (size_t)(li + 1) * sz;   /* state after token t */
+            const double *a = A + (size_t)li * m, *h = Hh + (size_t)li * m, *mm = Mm + (size_t)li * m;
+            const double *d1 = D1 + (size_t)li * m;
+            const double *xh = XH + (size_t)li * d, *e = EE + (size_t)li * d, *u = UU + (size_t)li * d;
+            const double *d2 = D2 + (size_t)li * d;
+            double *dq = dQ + (size_t)t * d, *dk = dK + (size_t)t * d, *dv = dV + (size_t)t * d;
+            for (int j = 0; j < d; ++j) { dq[j] = 0.0; dk[j] = 0.0; }
+            /* z = q + gamma LN(p) + beta, p = GELU(q W1_t + c1_t) W2_t + c2_t */
+            if (dZ) {
+                const double *dz = dZ + (size_t)t * d;
+                vec_mat(d, m, q, W1P(Rt), aq);
+                for (int p = 0; p < m; ++p) { aq[p] += C1P(Rt)[p]; hq[p] = gelu(aq[p]); }
+                vec_mat(m, d, hq, W2P(Rt), pp);
+                for (int j = 0; j < d; ++j) pp[j] += C2P(Rt)[j];
+                const double ro = layer_norm(d, pp, eps, xo);
+                for (int j = 0; j < d; ++j) {
+                    dq[j] += dz[j];
+                    dgamma[j] += dz[j] * xo[j];
+                    dbeta[j] += dz[j];
+                    t1[j] = gamma[j] * dz[j];
+                }
+                ln_adjoint(d, xo, ro, t1, dp);
+                for (int p = 0; p < m; ++p) {
+                    double acc = 0.0;
+                    for (int j = 0; j < d; ++j) acc += dp[j] * W2P(Rt)[(size_t)p * d + j];
+                    daq[p] = acc * gelu_grad(aq[p]);
+                }
+                for (int p = 0; p < m; ++p)
+                    for (int j = 0; j < d; ++j) W2P(D)[(size_t)p * d + j] += hq[p] * dp[j];
+                for (int j = 0; j < d; ++j) C2P(D)[j] += dp[j];
+                for (int a2 = 0; a2 < d; ++a2) {
+                    double acc = 0.0;
+                    for (int p = 0; p < m; ++p) acc += daq[p] * W1P(Rt)[(size_t)a2 * m + p];
+                    dq[a2] += acc;
+                }
+                for (int a2 = 0; a2 < d; ++a2)
+                    for (int p = 0; p < m; ++p) W1P(D)[(size_t)a2 * m + p] += q[a2] * daq[p];
+                for (int p = 0; p < m; ++p) C1P(D)[p] += daq[p];
+            }
+            /* the token's update: W1 -= eta k^T d1, c1 -= eta d1, W2 -= eta h^T Delta2, c2 -= eta Delta2 */
+            double g = 0.0;
+            for (int p = 0; p < m; ++p) {
+                double acc = C1P(D)[p];
+                for (int a2 = 0; a2 < d; ++a2) acc += k[a2] * W1P(D)[(size_t)a2 * m + p];
+                dd1[p] = -eta[t] * acc;
+                g += acc * d1[p];
+            }
+            for (int j = 0; j < d; ++j) {
+                double acc = C2P(D)[j];
+                for (int p = 0; p < m; ++p) acc += h[p] * W2P(D)[(size_t)p * d + j];
+                dd2[j] = -eta[t] * acc;
+                g += acc * d2[j];
+            }
+            deta[t] = -g;
+            for (int a2 = 0; a2 < d; ++a2) {
+                double acc = 0.0;
+                for (int p = 0; p < m; ++p) acc += d1[p] * W1P(D)[(size_t)a2 * m + p];
+                dk[a2] += -eta[t] * acc;
+            }
+            for (int p = 0; p < m; ++p) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += d2[j] * W2P(D)[(size_t)p * d + j];
+                dh[p] = -eta[t] * acc;
+            }
+            /* d1 = m GELU'(a), m = Delta2 W2s^T */
+            for (int p = 0; p < m; ++p) {
+                dm[p] = dd1[p] * gelu_grad(a[p]);
+                da[p] = dd1[p] * mm[p] * gelu_grad2(a[p]);
+            }
+            for (int j = 0; j < d; ++j) {
+                double acc = 0.0;
+                for (int p = 0; p < m; ++p) acc += dm[p] * W2P(S)[(size_t)p * d + j];
+                dd2[j] += acc;
+            }
+            for (int p = 0; p < m; ++p)
+                for (int j = 0; j < d; ++j) W2P(Ds)[(size_t)p * d + j] += dm[p] * d2[j];
+            /* Delta2 = r u, u = g - mean(g) - xh mean(g xh), g = gamma e, e = k + gamma xh + beta - v */
+            double dr = 0.0;
+            for (int j = 0; j < d; ++j) { dr += dd2[j] * u[j]; du[j] = RR[li] * dd2[j]; }
+            double mdu = 0.0, mdux = 0.0;
+            for (int j = 0; j < d; ++j) { mdu += du[j]; mdux += du[j] * xh[j]; }
+            mdu /= d;
+            mdux /= d;
+            for (int j = 0; j < d; ++j) {
+                const double dg = du[j] - mdu - xh[j] * mdux;
+                const double de = gamma[j] * dg;
+                dxh[j] = -du[j] * MGX[li] - gamma[j] * e[j] * mdux + gamma[j] * de;
+                dgamma[j] += e[j] * dg + xh[j] * de;
+                dbeta[j] += de;
+                dk[j] += de;
+                dv[j] = -de;
+            }
+            /* xh = LN(y) and the r of Delta2 = r u */
+            ln_adjoint(d, xh, RR[li], dxh, dy);
+            for (int j = 0; j < d; ++j) dy[j] += dr * (-RR[li] * RR[li] * xh[j] / d);
+            /* y = h W2s + c2s */
+            for (int p = 0; p < m; ++p) {
+                double acc = 0.0;
+                for (int j = 0; j < d; ++j) acc += dy[j] * W2P(S)[(size_t)p * d + j];
+                dh[p] += acc;
+            }
+            for (int p = 0; p < m; ++p)
+                for (int j = 0; j < d; ++j) W2P(Ds)[(size_t)p * d + j] += h[p] * dy[j];
+            for (int j = 0; j < d; ++j) C2P(Ds)[j] += dy[j];
+            /* h = GELU(a), a = k W1s + c1s */
+            for (int p = 0; p < m; ++p) da[p] += dh[p] * gelu_grad(a[p]);
+            for (int a2 = 0; a2 < d; ++a2) {
+                double acc = 0.0;
+                for (int p = 0; p < m; ++p) acc += da[p] * W1P(S)[(size_t)a2 * m + p];
+                dk[a2] += acc;
+            }
+            for (int a2 = 0; a2 < d; ++a2)
+                for (int p = 0; p < m; ++p) W1P(Ds)[(size_t)a2 * m + p] += k[a2] * da[p];
+            for (int p = 0; p < m; ++p) C1P(Ds)[p] += da[p];
+        }
+        for (size_t x = 0; x < sz; ++x) D[x] += Ds[x];
+    }
+    #undef BATCH_FWD
+    #undef TOKEN_UPD
+    memcpy(dW1, W1P(D), n1 * sizeof(double));
+    memcpy(dc1, C1P(D), m * sizeof(double));
+    memcpy(dW2, W2P(D), n1 * sizeof(double));
+    memcpy(dc2, C2P(D), d * sizeof(double));
+    #undef W1P
+    #undef C1P
+    #undef W2P
+    #undef C2P
+    free(starts); free(run); free(cur); free(D); free(Ds); free(A); free(Hh); free(Mm); free(D1);
+    free(XH); free(EE); free(UU); free(D2); free(RR); free(MGX); free(y); free(pp); free(xo); free(t1); free(dp);
+    free(dd2); free(du); free(dxh); free(dy); free(aq); free(hq); free(daq); free(dd1); free(dm); free(dh); free(da);
+}
+
+int ttt_oracle_mlp_ln_backward(int B, int H, int T, int d, int m, int b, const double *Q, const double *K,
+                               const double *V, const double *eta, const double *W1, const double *c1,
+                               const double *W2, const double *c2, long long p_bstride_scale, const double *gamma,
+                               const double *beta, double eps, const double *dZ, const double *dW1o,
+                               const double *dc1o, const double *dW2o, const double *dc2o, double *dQ, double *dK,
+                               double *dV, double *deta, double *dW1, double *dc1, double *dW2, double *dc2,
+                               double *dgamma, double *dbeta, int nthreads) {
+    if (B < 0 || H < 0 || T < 0 || d <= 0 || m <= 0 || b <= 0 || !Q || !K || !V || !eta || !W1 || !W2 ||
+        !gamma || !beta || !(eps > 0.0) || !dQ || !dK || !dV || !deta || !dW1 || !dc1 || !dW2 || !dc2 ||
+        !dgamma || !dbeta)
+        return 1;
+    const long long units = (long long)B * H;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (long long u = 0; u < units; ++u) {
+        const long long pu = p_bstride_scale ? u : (u % H);
+        const long long hd = u % H;
+        const size_t tok = (size_t)u * T * d;
+        mlp_ln_unit_backward(T, d, m, b, Q + tok, K + tok, V + tok, eta + (size_t)u * T, W1 + (size_t)pu * d * m,
+                             c1 ? c1 + (size_t)pu * m : NULL, W2 + (size_t)pu * m * d,
+                             c2 ? c2 + (size_t)pu * d : NULL, gamma + (size_t)hd * d, beta + (size_t)hd * d, eps,
+                             dZ ? dZ + tok : NULL, dW1o ? dW1o + (size_t)u * d * m : NULL,
+                             dc1o ? dc1o + (size_t)u * m : NULL, dW2o ? dW2o + (size_t)u * m * d : NULL,
+                             dc2o ? dc2o + (size_t)u * d : NULL, dQ + tok, dK + tok, dV + tok, deta + (size_t)u * T,
+                             dW1 + (size_t)u * d * m, dc1 + (size_t)u * m, dW2 + (size_t)u * m * d,
+                             dc2 + (size_t)u * d, dgamma + (size_t)u * d, dbeta + (size_t)u * d);
+    }
+    (void)nthreads;
+    return 0;
+}

@@ -201,3 +201,65 @@ def test_gelu_second_derivative():
     fd = (g1(x + h) - g1(x - h)) / (2 * h)
     g2 = np.exp(-0.5 * x * x) / np.sqrt(2 * np.pi) * (2 - x * x)
     assert np.max(np.abs(fd - g2)) < 1e-8
+
+
+# ---------------------------------------------------------------------------
+# TTT-MLP with LN+residual on the output layer, f(x) = x + gamma LN(GELU(x W1 +
+# c1) W2 + c2) + beta (section 4.4): the outer loop also trains gamma and beta
+# ---------------------------------------------------------------------------
+
+def _mlp_ln_loss(Q, K, V, eta, W1, c1, W2, c2, gamma, beta, b, up):
+    out = O.mlp_forward(Q, K, V, eta, W1, c1, W2, c2, b, threads=1, use_ln=True, gamma=gamma, beta=beta)
+    return float(sum(np.sum(o * u) for o, u in zip(out, up)))
+
+
+@pytest.mark.parametrize("B,H,T,d,m,b,shared", [
+    (1, 2, 5, 3, 6, 2, True),     # ragged last mini-batch
+    (2, 1, 4, 3, 5, 2, False),    # per-sequence parameters
+    (1, 1, 4, 3, 4, 1, True),     # b = 1
+    (1, 1, 3, 4, 4, 3, True),     # one mini-batch
+])
+def test_mlp_ln_backward_matches_finite_differences(B, H, T, d, m, b, shared):
+    Q, K, V, eta, W1, c1, W2, c2, up = _mlp_case(B, H, T, d, m, shared, seed=300 + 10 * T + d + m + b)
+    rng = np.random.default_rng(T + d)
+    gamma = 1 + rng.standard_normal((H, d)) * 0.3
+    beta = rng.standard_normal((H, d)) * 0.3
+    g = O.mlp_ln_backward(Q, K, V, eta, W1, c1, W2, c2, b, gamma, beta, dZ=up[0], dW1_out=up[1], dc1_out=up[2],
+                          dW2_out=up[3], dc2_out=up[4], threads=1)
+    dQ, dK, dV, deta, dW1, dc1, dW2, dc2, dgamma, dbeta = g
+    if shared:
+        dW1, dc1, dW2, dc2 = (x.sum(axis=0) for x in (dW1, dc1, dW2, dc2))
+    grads = {"Q": dQ, "K": dK, "V": dV, "eta": deta, "W1": dW1, "c1": dc1, "W2": dW2, "c2": dc2,
+             "gamma": dgamma.sum(axis=0), "beta": dbeta.sum(axis=0)}
+    inputs = {"Q": Q, "K": K, "V": V, "eta": eta, "W1": W1, "c1": c1, "W2": W2, "c2": c2, "gamma": gamma,
+              "beta": beta}
+    h = 1e-7   # the LN's curvature, as for the linear model with LN
+    for name, x in inputs.items():
+        gr = grads[name]
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            keep = x[idx]
+            x[idx] = keep + h
+            lp = _mlp_ln_loss(*inputs.values(), b, up)
+            x[idx] = keep - h
+            lm = _mlp_ln_loss(*inputs.values(), b, up)
+            x[idx] = keep
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.max(np.abs(fd - gr)) / max(np.max(np.abs(fd)), 1e-12)
+        assert err < 1e-6, (name, err)
+
+
+def test_mlp_ln_backward_at_zero_eta():
+    """eta = 0: the state never moves, so dZ reaches only the outputs of the initial state and the
+    final-state gradients pass straight through to the initial state (plus the outputs' terms)."""
+    Q, K, V, eta, W1, c1, W2, c2, up = _mlp_case(1, 1, 4, 3, 5, True, seed=7)
+    eta[:] = 0.0
+    rng = np.random.default_rng(8)
+    gamma = 1 + rng.standard_normal((1, 3)) * 0.3
+    beta = rng.standard_normal((1, 3)) * 0.3
+    g = O.mlp_ln_backward(Q, K, V, eta, W1, c1, W2, c2, 2, gamma, beta, dZ=None, dW1_out=up[1], dc1_out=up[2],
+                          dW2_out=up[3], dc2_out=up[4], threads=1)
+    for got, u in zip(g[4:8], up[1:]):
+        assert np.array_equal(got, u)
+    for x in (g[0], g[1], g[2]):
+        assert not np.any(x)

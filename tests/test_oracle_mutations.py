@@ -74,6 +74,16 @@ MLP_LN_MUTATIONS = {
                                        "z[j] = gamma[j] * xh[j] + beta[j];"),
 }
 
+# mistakes in the backward of TTT-MLP with LN+residual, caught by the backward pins
+MLP_LN_BACKWARD_MUTATIONS = {
+    "bwd_mlp_ln_delta2_path_through_w2_dropped": ("dd2[j] += acc;", "(void)acc;"),
+    "bwd_mlp_ln_xhat_path_through_e_dropped": (
+        "dxh[j] = -du[j] * MGX[li] - gamma[j] * e[j] * mdux + gamma[j] * de;",
+        "dxh[j] = -du[j] * MGX[li] - gamma[j] * e[j] * mdux;"),
+    "bwd_mlp_ln_explicit_r_term_dropped": (
+        "for (int j = 0; j < d; ++j) dy[j] += dr * (-RR[li] * RR[li] * xh[j] / d);", "(void)dr;"),
+}
+
 # mistakes in the prologue (views and learning-rate gate), caught by its own pins
 PROLOGUE_MUTATIONS = {
     "prologue_transposed_view": ("acc += row[k] * x[k];", "acc += theta[(size_t)k * H * d + h * d + j] * x[k];"),
@@ -88,8 +98,10 @@ PROLOGUE_MUTATIONS = {
 PIN_FILES = {**{n: "test_oracle_pins.py" for n in MUTATIONS},
              **{n: "test_oracle_backward.py" for n in BACKWARD_MUTATIONS},
              **{n: "test_oracle_mlp_ln.py" for n in MLP_LN_MUTATIONS},
-             **{n: "test_oracle_prologue.py" for n in PROLOGUE_MUTATIONS}}
-ALL_MUTATIONS = {**MUTATIONS, **BACKWARD_MUTATIONS, **MLP_LN_MUTATIONS, **PROLOGUE_MUTATIONS}
+             **{n: "test_oracle_prologue.py" for n in PROLOGUE_MUTATIONS},
+             **{n: "test_oracle_backward.py" for n in MLP_LN_BACKWARD_MUTATIONS}}
+ALL_MUTATIONS = {**MUTATIONS, **BACKWARD_MUTATIONS, **MLP_LN_MUTATIONS, **PROLOGUE_MUTATIONS,
+                 **MLP_LN_BACKWARD_MUTATIONS}
 
 
 @pytest.mark.parametrize("name", sorted(ALL_MUTATIONS))
