@@ -224,10 +224,9 @@ ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_
  *   W_states       NULL, or [B, H, T/b, 2dm + m + d] fp32: the state at the
  *                  start of every mini-batch, each one W1 [d][m], c1 [m],
  *                  W2 [m][d], c2 [d] (the checkpoints ttt_mlp_backward reads;
- *                  section 6.12).  BF16 with d = 64, b = 16 runs on an
- *                  mma.sync tensor-core kernel, every other case (and
- *                  TTT_FLAG_FORCE_SIMT) on the fp32 CUDA-core kernel; not with
- *                  use_ln (TTT_ERR_UNSUPPORTED).
+ *                  section 6.12).  BF16 with d = 64, b = 16 and no LN runs on
+ *                  an mma.sync tensor-core kernel, every other case (and
+ *                  TTT_FLAG_FORCE_SIMT) on the fp32 CUDA-core kernel.
  */
 typedef struct {
     int B, H, T, d, b;
@@ -259,7 +258,8 @@ typedef struct {
 ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
 
 /*
- * ttt_mlp_backward -- outer-loop gradients of the TTT-MLP prefill (no LN):
+ * ttt_mlp_backward -- outer-loop gradients of the TTT-MLP prefill, plain or
+ * with LN+residual on the output layer (use_ln):
  * reverse-mode differentiation of ttt_mlp_forward through the inner loop's
  * updates (section 3.4), one mini-batch at a time in reverse order from the
  * batch-start states ttt_mlp_forward wrote to W_states (section 6.12).
@@ -284,6 +284,11 @@ ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
  *                  They also serve as the kernel's running adjoint, so they
  *                  must not overlap any input.
  *   flags          TTT_FLAG_FORCE_SIMT; any other bit is TTT_ERR_INVALID_ARG.
+ *   use_ln         1: the model of ttt_mlp_forward with use_ln (ln_gamma,
+ *                  ln_beta [H, d], ln_eps as given to it); the outputs dgamma,
+ *                  dbeta [B, H, d] receive the per-unit gradients of gamma and
+ *                  beta.  Runs on the fp32 CUDA-core kernel (b up to 16 at
+ *                  d = 64 for shared memory).  0: plain.
  */
 typedef struct {
     int B, H, T, d, b;
@@ -308,6 +313,12 @@ typedef struct {
     float* dW2;
     float* dc2;
     unsigned flags;
+    int use_ln;
+    const float* ln_gamma;
+    const float* ln_beta;
+    float ln_eps;
+    float* dgamma;
+    float* dbeta;
 } ttt_mlp_backward_args;
 
 ttt_status ttt_mlp_backward(const ttt_mlp_backward_args* args, cudaStream_t stream);

@@ -49,14 +49,27 @@ struct SimtMlpBackwardParams {
     float* dc1;
     float* dW2;
     float* dc2;
+    // LN+residual on the output layer (the LN template instance only): gamma, beta [H, D], eps; the
+    // per-unit gradients dgamma, dbeta [units, D]
+    const float* gamma;
+    const float* beta;
+    float eps;
+    float* dgamma;
+    float* dbeta;
 };
 
-inline size_t simt_mlp_backward_smem(int D, int b) {
+inline size_t simt_mlp_backward_smem(int D, int b, bool ln = false) {
     const size_t M = 4 * (size_t)D;
-    return sizeof(float) * (7 * (size_t)b * D + 9 * (size_t)b * M + 4 * (size_t)b * b + 2 * (size_t)b);
+    return sizeof(float) * ((ln ? 13 : 7) * (size_t)b * D + 9 * (size_t)b * M + 4 * (size_t)b * b +
+                            (ln ? 5 : 2) * (size_t)b + (ln ? 4 * (size_t)D : 0));
 }
 
-template <int D, typename IO>
+// LN = true: f(x) = x + gamma LN(GELU(x W1 + c1) W2 + c2) + beta.  Delta2, the LN+residual backward at
+// Y = Hk W2 + c2, takes E's place in every product (the dual form's updates use it); the outputs pass
+// through the LN, so dP (the LN adjoint of gamma dZ at the recomputed P) takes dZ's place; and the
+// complete adjoint of Delta2 goes through the LN+residual backward of each row to dY (for Hk, W2, c2)
+// and de (for K, V, gamma, beta), as in the linear model with LN.
+template <int D, typename IO, bool LN = false>
 __global__ void __launch_bounds__(kSimtThreads) simt_mlp_backward_kernel(SimtMlpBackwardParams p) {
     constexpr int M = 4 * D;
     constexpr int NT = kSimtThreads;
@@ -86,6 +99,21 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_backward_kernel(SimtMlp
     float* dL1 = dL2 + bb;    // b x b   tril(-dAq D1^T)
     float* et = dL1 + bb;     // b
     float* det = et + b;      // b
+    // LN only: Xh (LN(Y), then the output's LN(P)), Ev (E = K + gamma Xh + beta - V), dZr (dZ as given),
+    // dYt, deT (b x D); per row r, mean(G), mean(G Xh); gamma, beta, dgamma, dbeta (D)
+    float* Xh = det + b;
+    float* Ev = Xh + (LN ? bD : 0);
+    float* Xo = Ev + (LN ? bD : 0);
+    float* dZr = Xo + (LN ? bD : 0);
+    float* dYt = dZr + (LN ? bD : 0);
+    float* deT = dYt + (LN ? bD : 0);
+    float* rr = deT + (LN ? bD : 0);
+    float* mgv = rr + (LN ? b : 0);
+    float* mgx = mgv + (LN ? b : 0);
+    float* gam = mgx + (LN ? b : 0);
+    float* bet = gam + (LN ? D : 0);
+    float* dgam = bet + (LN ? D : 0);
+    float* dbet = dgam + (LN ? D : 0);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = NT / 32;
     const int unit = blockIdx.x;
     const int T = p.T, nb = T / b;
@@ -109,6 +137,13 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_backward_kernel(SimtMlp
     }
     for (int e = tid; e < M; e += NT) gc1[e] = p.dc1_out ? p.dc1_out[(size_t)unit * M + e] : 0.f;
     for (int e = tid; e < D; e += NT) gc2[e] = p.dc2_out ? p.dc2_out[(size_t)unit * D + e] : 0.f;
+    if (LN)
+        for (int j = tid; j < D; j += NT) {
+            gam[j] = p.gamma[(size_t)(unit % p.H) * D + j];
+            bet[j] = p.beta[(size_t)(unit % p.H) * D + j];
+            dgam[j] = 0.f;
+            dbet[j] = 0.f;
+        }
     __syncthreads();
 
     for (int i = nb - 1; i >= 0; --i) {
@@ -148,14 +183,47 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_backward_kernel(SimtMlp
             P1[e] = acc;
         }
         __syncthreads();
-        // E = Hk W2 + c2 - V (in place of V)
+        // E = Hk W2 + c2 - V (in place of V); LN: Y = Hk W2 + c2 (into Xh), then per row the LN+residual
+        // backward Delta2 (in place of V), with E, Xh, r, mean(G), mean(G Xh) kept
         for (int e = tid; e < bD; e += NT) {
             const int s = e / D, j = e % D;
             float acc = c2s[j];
             for (int q = 0; q < M; ++q) acc += Hk[s * M + q] * W2s[q * D + j];
-            Et[e] = acc - Et[e];
+            if (LN)
+                Xh[e] = acc;
+            else
+                Et[e] = acc - Et[e];
         }
         __syncthreads();
+        if (LN) {
+            for (int s = warp; s < b; s += nwarps) {
+                float mu, r;
+                warp_ln_stats(Xh + s * D, D, p.eps, mu, r);
+                float mg = 0.f, mgx_ = 0.f;
+                for (int j = lane; j < D; j += 32) {
+                    const float x = (Xh[s * D + j] - mu) * r;
+                    Xh[s * D + j] = x;
+                    const float ev = Kt[s * D + j] + gam[j] * x + bet[j] - Et[s * D + j];
+                    Ev[s * D + j] = ev;
+                    mg += gam[j] * ev;
+                    mgx_ += gam[j] * ev * x;
+                }
+                for (int o = 16; o > 0; o >>= 1) {
+                    mg += __shfl_xor_sync(0xffffffffu, mg, o);
+                    mgx_ += __shfl_xor_sync(0xffffffffu, mgx_, o);
+                }
+                mg /= D;
+                mgx_ /= D;
+                for (int j = lane; j < D; j += 32)
+                    Et[s * D + j] = r * (gam[j] * Ev[s * D + j] - mg - Xh[s * D + j] * mgx_);   // Delta2
+                if (lane == 0) {
+                    rr[s] = r;
+                    mgv[s] = mg;
+                    mgx[s] = mgx_;
+                }
+            }
+            __syncthreads();
+        }
         // M = E W2^T, D1 = M GELU'(A)
         for (int e = tid; e < bM; e += NT) {
             const int s = e / M, q = e % M;
@@ -175,8 +243,55 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_backward_kernel(SimtMlp
             Hq[e] = gelu_f(acc);
         }
         __syncthreads();
+        if (LN) {
+            // the outputs' pre-LN P = Hq W2 + c2 - L2 Delta2 (L2 = tril(Hq Hk^T + 1) diag(eta)), its LN, and
+            // dP = the LN adjoint of gamma dZ, which takes dZ's place below (dZ kept in dZr)
+            for (int e = tid; e < bb; e += NT) {
+                const int t = e / b, s = e % b;
+                float acc = 0.f;
+                if (s <= t) {
+                    for (int q = 0; q < M; ++q) acc += Hq[t * M + q] * Hk[s * M + q];
+                    acc += 1.f;
+                }
+                P2[e] = acc;
+            }
+            __syncthreads();
+            for (int e = tid; e < bD; e += NT) {
+                const int t = e / D, j = e % D;
+                float acc = c2s[j];
+                for (int q = 0; q < M; ++q) acc += Hq[t * M + q] * W2s[q * D + j];
+                for (int s = 0; s <= t; ++s) acc -= P2[t * b + s] * et[s] * Et[s * D + j];
+                Xo[e] = acc;
+                dZr[e] = dZt[e];
+            }
+            __syncthreads();
+            for (int t = warp; t < b; t += nwarps) {
+                float mu, r;
+                warp_ln_stats(Xo + t * D, D, p.eps, mu, r);
+                float m1 = 0.f, m2 = 0.f;
+                for (int j = lane; j < D; j += 32) {
+                    const float x = (Xo[t * D + j] - mu) * r;
+                    Xo[t * D + j] = x;
+                    const float g = gam[j] * dZr[t * D + j];
+                    m1 += g;
+                    m2 += g * x;
+                }
+                for (int o = 16; o > 0; o >>= 1) {
+                    m1 += __shfl_xor_sync(0xffffffffu, m1, o);
+                    m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+                }
+                m1 /= D;
+                m2 /= D;
+                for (int j = lane; j < D; j += 32) {
+                    const float x = Xo[t * D + j];
+                    dZt[t * D + j] = r * (gam[j] * dZr[t * D + j] - m1 - x * m2);   // dP
+                }
+            }
+            __syncthreads();
+        }
         // ---- backward.  First every product with the end-state adjoint (read before
         // this mini-batch adds to it), P2, dHq = dZ W2^T and dL2 = tril(-dZ E^T)
+        // (LN: dP in dZ's place and Delta2 in E's)
         for (int e = tid; e < bb; e += NT) {
             const int t = e / b, s = e % b;
             float acc = 0.f, acc2 = 0.f;
@@ -288,22 +403,72 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_backward_kernel(SimtMlp
             dE[e] += ae;
         }
         __syncthreads();
+        if (LN) {
+            // dE holds the adjoint of Delta2 = r U: per row, the LN+residual backward to de (E's adjoint,
+            // for K, V, gamma, beta) and dY (Y = Hk W2 + c2); the dgamma terms of the row go to Ev
+            for (int s = warp; s < b; s += nwarps) {
+                const float r = rr[s];
+                float dr = 0.f, mdu = 0.f, mdux = 0.f;
+                for (int j = lane; j < D; j += 32) {
+                    const float x = Xh[s * D + j];
+                    const float u = gam[j] * Ev[s * D + j] - mgv[s] - x * mgx[s];
+                    const float dd = dE[s * D + j];
+                    dr += dd * u;
+                    mdu += r * dd;
+                    mdux += r * dd * x;
+                }
+                for (int o = 16; o > 0; o >>= 1) {
+                    dr += __shfl_xor_sync(0xffffffffu, dr, o);
+                    mdu += __shfl_xor_sync(0xffffffffu, mdu, o);
+                    mdux += __shfl_xor_sync(0xffffffffu, mdux, o);
+                }
+                mdu /= D;
+                mdux /= D;
+                float m1 = 0.f, m2 = 0.f;
+                for (int j = lane; j < D; j += 32) {
+                    const float x = Xh[s * D + j];
+                    const float du = r * dE[s * D + j];
+                    const float dg = du - mdu - x * mdux;
+                    const float de = gam[j] * dg;
+                    const float dx = -du * mgx[s] - gam[j] * Ev[s * D + j] * mdux + gam[j] * de;
+                    Ev[s * D + j] = Ev[s * D + j] * dg + x * de;   // the row's dgamma terms
+                    deT[s * D + j] = de;
+                    dYt[s * D + j] = dx;   // dXh for now
+                    m1 += dx;
+                    m2 += dx * x;
+                }
+                for (int o = 16; o > 0; o >>= 1) {
+                    m1 += __shfl_xor_sync(0xffffffffu, m1, o);
+                    m2 += __shfl_xor_sync(0xffffffffu, m2, o);
+                }
+                m1 /= D;
+                m2 /= D;
+                for (int j = lane; j < D; j += 32) {
+                    const float x = Xh[s * D + j];
+                    dYt[s * D + j] = r * (dYt[s * D + j] - m1 - x * m2) - dr * r * r * x / D;
+                }
+            }
+            __syncthreads();
+        }
+        // the adjoint that reaches Hk, W2 and c2 (E's, or with LN Y's) and the one that reaches K and V
+        const float* dYu = LN ? dYt : dE;
+        const float* dEv = LN ? deT : dE;
         // dHk += dE W2^T;  dA = dD1 M GELU''(A) + dHk GELU'(A) (in Mv);  dV = -dE;  dQ out
         for (int e = tid; e < bM; e += NT) {
             const int s = e / M, q = e % M;
             float acc = dHk[e];
-            for (int j = 0; j < D; ++j) acc += dE[s * D + j] * W2s[q * D + j];
+            for (int j = 0; j < D; ++j) acc += dYu[s * D + j] * W2s[q * D + j];
             Mv[e] += acc * gelu_grad_f(A[e]);
         }
         for (int e = tid; e < bD; e += NT) {
-            IoTraits<IO>::store(dV, (size_t)t0 * D + e, -dE[e]);
-            IoTraits<IO>::store(dQ, (size_t)t0 * D + e, dQt[e]);
+            IoTraits<IO>::store(dV, (size_t)t0 * D + e, -dEv[e]);
+            IoTraits<IO>::store(dQ, (size_t)t0 * D + e, dQt[e] + (LN ? dZr[e] : 0.f));
         }
         __syncthreads();
         // dK += dA W1^T;  this mini-batch's terms of the start-state adjoint
         for (int e = tid; e < bD; e += NT) {
             const int s = e / D, a = e % D;
-            float acc = dKt[e];
+            float acc = dKt[e] + (LN ? deT[e] : 0.f);
             for (int q = 0; q < M; ++q) acc += Mv[s * M + q] * W1s[a * M + q];
             IoTraits<IO>::store(dK, (size_t)t0 * D + e, acc);
         }
@@ -317,7 +482,7 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_backward_kernel(SimtMlp
             const int q = e / D, j = e % D;
             float acc = 0.f;
             for (int t = 0; t < b; ++t)
-                acc += Hq[t * M + q] * dZt[t * D + j] + dD1[t * M + q] * Et[t * D + j] + Hk[t * M + q] * dE[t * D + j];
+                acc += Hq[t * M + q] * dZt[t * D + j] + dD1[t * M + q] * Et[t * D + j] + Hk[t * M + q] * dYu[t * D + j];
             gW2[e] += acc;
         }
         for (int q = tid; q < M; q += NT) {
@@ -327,13 +492,27 @@ __global__ void __launch_bounds__(kSimtThreads) simt_mlp_backward_kernel(SimtMlp
         }
         for (int j = tid; j < D; j += NT) {
             float acc = 0.f;
-            for (int t = 0; t < b; ++t) acc += dZt[t * D + j] + dE[t * D + j];
+            for (int t = 0; t < b; ++t) acc += dZt[t * D + j] + dYu[t * D + j];
             gc2[j] += acc;
+            if (LN) {
+                float g = 0.f, bb_ = 0.f;
+                for (int t = 0; t < b; ++t) {
+                    g += dZr[t * D + j] * Xo[t * D + j] + Ev[t * D + j];
+                    bb_ += dZr[t * D + j] + deT[t * D + j];
+                }
+                dgam[j] += g;
+                dbet[j] += bb_;
+            }
         }
         if (p.deta)
             for (int t = tid; t < b; t += NT) p.deta[(size_t)unit * T + t0 + t] = det[t];
         __syncthreads();
     }
+    if (LN)
+        for (int j = tid; j < D; j += NT) {
+            p.dgamma[(size_t)unit * D + j] = dgam[j];
+            p.dbeta[(size_t)unit * D + j] = dbet[j];
+        }
 }
 
 }  // namespace ttt

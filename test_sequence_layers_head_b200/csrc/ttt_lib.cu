@@ -347,8 +347,7 @@ extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream
     if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
     if (a->use_ln && (!ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !(a->ln_eps > 0.f))) return TTT_ERR_INVALID_ARG;
     if (!ok_opt(a->W_states)) return TTT_ERR_INVALID_ARG;
-    if (a->W_states && a->use_ln) return TTT_ERR_UNSUPPORTED;
-    if (a->W_states && a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
+    if (a->W_states && !a->use_ln && a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
         !(a->flags & TTT_FLAG_FORCE_SIMT)) {
         // training: the mma.sync forward that writes the batch-start states
         if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
@@ -537,9 +536,10 @@ ttt_status launch_mlp_backward_t(const ttt_mlp_backward_args* a, cudaStream_t st
     SimtMlpBackwardParams p{a->H,       a->T,       a->b,       a->Q,       a->K,       a->V,
                             a->eta,     a->eta_const, a->W_states, a->dZ,   a->dW1_out, a->dc1_out,
                             a->dW2_out, a->dc2_out, a->dQ,      a->dK,      a->dV,      a->deta,
-                            a->dW1,     a->dc1,     a->dW2,     a->dc2};
-    const size_t smem = simt_mlp_backward_smem(D, a->b);
-    auto k = simt_mlp_backward_kernel<D, IO>;
+                            a->dW1,     a->dc1,     a->dW2,     a->dc2,     a->ln_gamma, a->ln_beta,
+                            a->ln_eps,  a->dgamma,  a->dbeta};
+    const size_t smem = simt_mlp_backward_smem(D, a->b, a->use_ln != 0);
+    auto k = a->use_ln ? simt_mlp_backward_kernel<D, IO, true> : simt_mlp_backward_kernel<D, IO, false>;
     if (!set_smem(k, smem)) return TTT_ERR_UNSUPPORTED;
     k<<<(unsigned)(a->B * a->H), kSimtThreads, smem, st>>>(p);
     return launch_status();
@@ -566,16 +566,22 @@ extern "C" ttt_status ttt_mlp_backward(const ttt_mlp_backward_args* a, cudaStrea
         !ok_opt(a->dW2_out) || !ok_opt(a->dc2_out))
         return TTT_ERR_INVALID_ARG;
     if (a->flags & ~TTT_FLAG_FORCE_SIMT) return TTT_ERR_INVALID_ARG;
-    if (a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 && !(a->flags & TTT_FLAG_FORCE_SIMT)) {
+    if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
+    if (a->use_ln && (!ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !(a->ln_eps > 0.f) || !ok_ptr(a->dgamma) ||
+                      !ok_ptr(a->dbeta)))
+        return TTT_ERR_INVALID_ARG;
+    if (!a->use_ln && a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
+        !(a->flags & TTT_FLAG_FORCE_SIMT)) {
         SimtMlpBackwardParams p{a->H,       a->T,       a->b,       a->Q,       a->K,       a->V,
                                 a->eta,     a->eta_const, a->W_states, a->dZ,   a->dW1_out, a->dc1_out,
                                 a->dW2_out, a->dc2_out, a->dQ,      a->dK,      a->dV,      a->deta,
-                                a->dW1,     a->dc1,     a->dW2,     a->dc2};
+                                a->dW1,     a->dc1,     a->dW2,     a->dc2,     nullptr,    nullptr,
+                                0.f,        nullptr,    nullptr};
         if (!set_smem(mmb::mma_mlp_backward_kernel, mmb::kSmemBytes)) return TTT_ERR_CUDA;
         mmb::mma_mlp_backward_kernel<<<(unsigned)units, mmb::kThreads, mmb::kSmemBytes, stream>>>(p);
         return launch_status();
     }
-    if (simt_mlp_backward_smem(a->d, a->b) > 227 * 1024) return TTT_ERR_UNSUPPORTED;
+    if (simt_mlp_backward_smem(a->d, a->b, a->use_ln != 0) > 227 * 1024) return TTT_ERR_UNSUPPORTED;
     switch (a->d) {
         case 16: return launch_mlp_backward<16>(a, stream);
         case 32: return launch_mlp_backward<32>(a, stream);

@@ -56,7 +56,9 @@ class MlpBackwardArgs(ctypes.Structure):
     _fields_ = [("B", _i), ("H", _i), ("T", _i), ("d", _i), ("b", _i), ("io_dtype", _i), ("Q", _vp), ("K", _vp),
                 ("V", _vp), ("eta", _vp), ("eta_const", _f), ("W_states", _vp), ("dZ", _vp), ("dW1_out", _vp),
                 ("dc1_out", _vp), ("dW2_out", _vp), ("dc2_out", _vp), ("dQ", _vp), ("dK", _vp), ("dV", _vp),
-                ("deta", _vp), ("dW1", _vp), ("dc1", _vp), ("dW2", _vp), ("dc2", _vp), ("flags", _u)]
+                ("deta", _vp), ("dW1", _vp), ("dc1", _vp), ("dW2", _vp), ("dc2", _vp), ("flags", _u),
+                ("use_ln", _i), ("ln_gamma", _vp), ("ln_beta", _vp), ("ln_eps", _f), ("dgamma", _vp),
+                ("dbeta", _vp)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -279,10 +281,10 @@ def mlp_decode_step(W1, c1, W2, c2, q, k, v, eta, *, eta_const=0.0, z=None, stre
 
 def mlp_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW1_out=None, dc1_out=None, dW2_out=None, dc2_out=None,
                  eta_const=0.0, dQ=None, dK=None, dV=None, deta=None, want_deta=True, dW1=None, dc1=None, dW2=None,
-                 dc2=None, flags=0, stream=None):
+                 dc2=None, flags=0, use_ln=False, gamma=None, beta=None, eps=1e-6, stream=None):
     """Outer-loop gradients of the TTT-MLP prefill; see ``ttt_mlp_backward``.
-    Returns (dQ, dK, dV, deta, dW1, dc1, dW2, dc2); deta is None when
-    ``want_deta`` is False."""
+    Returns (dQ, dK, dV, deta, dW1, dc1, dW2, dc2), with use_ln also (dgamma,
+    dbeta) [B,H,d]; deta is None when ``want_deta`` is False."""
     B, H, T, d = Q.shape
     m = 4 * d
     dev, f32 = Q.device, torch.float32
@@ -295,11 +297,16 @@ def mlp_backward(Q, K, V, eta, W_states, b, *, dZ=None, dW1_out=None, dc1_out=No
     dc1 = torch.empty((B, H, m), device=dev, dtype=f32) if dc1 is None else dc1
     dW2 = torch.empty((B, H, m, d), device=dev, dtype=f32) if dW2 is None else dW2
     dc2 = torch.empty((B, H, d), device=dev, dtype=f32) if dc2 is None else dc2
+    dgamma = torch.empty((B, H, d), device=dev, dtype=f32) if use_ln else None
+    dbeta = torch.empty((B, H, d), device=dev, dtype=f32) if use_ln else None
     a = MlpBackwardArgs(B, H, T, d, b, _io_dtype(Q), _ptr(Q), _ptr(K), _ptr(V), _ptr(eta), float(eta_const),
                         _ptr(W_states), _ptr(dZ), _ptr(dW1_out), _ptr(dc1_out), _ptr(dW2_out), _ptr(dc2_out),
                         _ptr(dQ), _ptr(dK), _ptr(dV), _ptr(deta), _ptr(dW1), _ptr(dc1), _ptr(dW2), _ptr(dc2),
-                        int(flags))
+                        int(flags), int(bool(use_ln)), _ptr(gamma), _ptr(beta), float(eps), _ptr(dgamma),
+                        _ptr(dbeta))
     _check(library().ttt_mlp_backward(ctypes.byref(a), _stream(stream)), "ttt_mlp_backward")
+    if use_ln:
+        return dQ, dK, dV, deta, dW1, dc1, dW2, dc2, dgamma, dbeta
     return dQ, dK, dV, deta, dW1, dc1, dW2, dc2
 
 

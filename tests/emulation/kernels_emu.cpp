@@ -253,3 +253,57 @@ extern "C" int emu_mlp_forward_mma(int B, int H, int T, const void* Q, const voi
     emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_forward_states_kernel(f); });
     return 0;
 }
+
+// TTT-MLP with LN+residual on fp32 CUDA cores: the forward writing the batch-start states, then the backward
+extern "C" int emu_mlp_ln_train(int io, int B, int H, int T, int d, int b, const void* Q, const void* K,
+                                const void* V, const float* eta, float eta_const, const float* W1, const float* c1,
+                                const float* W2, const float* c2, const float* gamma, const float* beta, float eps,
+                                const void* dZ, const float* dW1o, const float* dc1o, const float* dW2o,
+                                const float* dc2o, float* W_states, void* dQ, void* dK, void* dV, float* deta,
+                                float* dW1, float* dc1, float* dW2, float* dc2, float* dgamma, float* dbeta) {
+    std::vector<uint8_t> Z((size_t)B * H * T * d * (io ? 2 : 4) + 16);
+    std::vector<float> W1o((size_t)B * H * d * 4 * d), c1o((size_t)B * H * 4 * d), W2o((size_t)B * H * 4 * d * d),
+        c2o((size_t)B * H * d);
+    ttt::SimtMlpParams f{};
+    f.H = H;
+    f.T = T;
+    f.b = b;
+    f.Q = Q;
+    f.K = K;
+    f.V = V;
+    f.eta = eta;
+    f.eta_const = eta_const;
+    f.W1 = W1;
+    f.c1 = c1;
+    f.W2 = W2;
+    f.c2 = c2;
+    f.Z = Z.data();
+    f.W1_out = W1o.data();
+    f.c1_out = c1o.data();
+    f.W2_out = W2o.data();
+    f.c2_out = c2o.data();
+    f.gamma = gamma;
+    f.beta = beta;
+    f.eps = eps;
+    f.W_states = W_states;
+    ttt::SimtMlpBackwardParams q{H,    T,    b,  Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
+                                 dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2,
+                                 gamma, beta, eps, dgamma, dbeta};
+    if (ttt::simt_mlp_smem(d, b, true) > sizeof(ttt::sm) || ttt::simt_mlp_backward_smem(d, b, true) > sizeof(ttt::sm))
+        return 2;
+    auto go = [&](auto fwd, auto bwd) {
+        emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { fwd(f); });
+        emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { bwd(q); });
+    };
+    if (io == 0) {
+        if (d == 16) go(ttt::simt_mlp_kernel<16, float, true>, ttt::simt_mlp_backward_kernel<16, float, true>);
+        else if (d == 32) go(ttt::simt_mlp_kernel<32, float, true>, ttt::simt_mlp_backward_kernel<32, float, true>);
+        else go(ttt::simt_mlp_kernel<64, float, true>, ttt::simt_mlp_backward_kernel<64, float, true>);
+    } else {
+        if (d == 16)
+            go(ttt::simt_mlp_kernel<16, __nv_bfloat16, true>, ttt::simt_mlp_backward_kernel<16, __nv_bfloat16, true>);
+        else
+            go(ttt::simt_mlp_kernel<64, __nv_bfloat16, true>, ttt::simt_mlp_backward_kernel<64, __nv_bfloat16, true>);
+    }
+    return 0;
+}

@@ -248,6 +248,13 @@ def _mlp_backward_args(ttt, **kw):
     (dict(deta=(1 << 20) + 4), 1),
     (dict(flags=0x2), 1),
     (dict(B=0, Q=None, dW1=None), 0),
+    (dict(use_ln=2), 1),
+    (dict(use_ln=1), 1),                                       # no gamma / beta / eps / dgamma / dbeta
+    (dict(use_ln=1, ln_gamma=1 << 20, ln_beta=1 << 20, ln_eps=1e-6, dgamma=1 << 20,
+          dbeta=(1 << 20) + 4), 1),                            # misaligned dbeta
+    (dict(use_ln=1, ln_gamma=1 << 20, ln_beta=1 << 20, dgamma=1 << 20, dbeta=1 << 20), 1),   # eps = 0
+    (dict(use_ln=1, ln_gamma=1 << 20, ln_beta=1 << 20, ln_eps=1e-6, dgamma=1 << 20, dbeta=1 << 20, b=32,
+          T=64), 2),                                           # the LN variant's shared memory at d = 64
 ])
 def test_mlp_backward_validation(ttt_lib, kw, code):
     a = _mlp_backward_args(ttt_lib, **kw)
@@ -263,8 +270,8 @@ def test_mlp_forward_states_rules(ttt_lib):
     m.W_states = fake + 4                        # misaligned
     assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1
     m.W_states = fake
-    m.use_ln, m.ln_gamma, m.ln_beta, m.ln_eps = 1, fake, fake, 1e-6
-    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 2   # no backward of the LN variant
+    m.use_ln, m.ln_gamma, m.ln_beta, m.ln_eps = 1, fake, fake, 0.0
+    assert L.ttt_mlp_forward(ctypes.byref(m), None) == 1   # the LN variant still needs eps > 0
 
 
 def _prologue_args(ttt, **kw):

@@ -172,3 +172,35 @@ def test_mlp_backward_tensor_cores_match_cuda_cores(ttt_lib):
     for a, b_ in zip(tc, simt):
         assert normwise(to_host(a), to_host(b_)) <= 2e-2
     _check(inp, c1, c2, dz, ups, True, to_host(states), [to_host(g) for g in tc])
+
+
+@pytest.mark.parametrize("B,H,T,d,b,io", [(1, 2, 64, 16, 16, WL.F32), (2, 2, 64, 64, 16, WL.BF16),
+                                          (1, 1, 32, 32, 4, WL.F32)])
+def test_mlp_ln_training_matches_oracle(ttt_lib, B, H, T, d, b, io):
+    """TTT-MLP with LN+residual on the output layer: the forward writes its states (fp32 CUDA cores),
+    the backward returns the eight gradients plus dgamma, dbeta; all against the oracle's reverse mode."""
+    m = 4 * d
+    inp, c1, c2, dz, ups = _case(B, H, T, d, b, io, True, True, seed=50 + T + d)
+    r, e, w = inp.raw, inp.exact, inp.w
+    rng = np.random.default_rng(T + d)
+    gam = (1 + rng.standard_normal((H, d)) * 0.2).astype(np.float32)
+    bet = (rng.standard_normal((H, d)) * 0.2).astype(np.float32)
+    Q, K, V, eta = (to_dev(r[n]) for n in ("Q", "K", "V", "eta"))
+    states = torch.full((B, H, T // b, 2 * d * m + m + d), float("nan"), device="cuda")
+    ttt_lib.mlp_forward(Q, K, V, eta, to_dev(r["W1"]), to_dev(c1), to_dev(r["W2"]), to_dev(c2), b, use_ln=True,
+                        gamma=to_dev(gam), beta=to_dev(bet), W_states=states)
+    out = ttt_lib.mlp_backward(Q, K, V, eta, states, b, dZ=to_dev(dz[0]), use_ln=True, gamma=to_dev(gam),
+                               beta=to_dev(bet), **{k: to_dev(u) for k, u in
+                                                    zip(("dW1_out", "dc1_out", "dW2_out", "dc2_out"), ups)})
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    f64 = lambda a: a.astype(np.float64)
+    ref = O.mlp_ln_backward(e["Q"], e["K"], e["V"], e["eta"], e["W1"], f64(c1), e["W2"], f64(c2), b, f64(gam),
+                            f64(bet), dZ=dz[1], **{k: f64(u) for k, u in
+                                                   zip(("dW1_out", "dc1_out", "dW2_out", "dc2_out"), ups)})
+    for nm, got, want in zip(("dQ", "dK", "dV", "deta", "dW1", "dc1", "dW2", "dc2", "dgamma", "dbeta"), out, ref):
+        g = to_host(got)
+        if io == WL.BF16:
+            assert normwise(g, want) <= 2e-2, nm
+        else:
+            assert maxrel(g, want) <= 1e-4, (nm, maxrel(g, want))
