@@ -307,3 +307,65 @@ extern "C" int emu_mlp_ln_train(int io, int B, int H, int T, int d, int b, const
     }
     return 0;
 }
+
+// the two launches of emu_mlp_ln_train one at a time (the tests' dry runs call them as the library would)
+extern "C" int emu_mlp_ln_forward(int io, int B, int H, int T, int d, int b, const void* Q, const void* K,
+                                  const void* V, const float* eta, float eta_const, const float* W1, const float* c1,
+                                  const float* W2, const float* c2, const float* gamma, const float* beta, float eps,
+                                  void* Z, float* W1_out, float* c1_out, float* W2_out, float* c2_out,
+                                  float* W_states) {
+    ttt::SimtMlpParams f{};
+    f.H = H;
+    f.T = T;
+    f.b = b;
+    f.Q = Q;
+    f.K = K;
+    f.V = V;
+    f.eta = eta;
+    f.eta_const = eta_const;
+    f.W1 = W1;
+    f.c1 = c1;
+    f.W2 = W2;
+    f.c2 = c2;
+    f.Z = Z;
+    f.W1_out = W1_out;
+    f.c1_out = c1_out;
+    f.W2_out = W2_out;
+    f.c2_out = c2_out;
+    f.gamma = gamma;
+    f.beta = beta;
+    f.eps = eps;
+    f.W_states = W_states;
+    auto run = [&](auto kernel) { emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { kernel(f); }); };
+    if (io == 0) {
+        if (d == 16) run(ttt::simt_mlp_kernel<16, float, true>);
+        else if (d == 32) run(ttt::simt_mlp_kernel<32, float, true>);
+        else run(ttt::simt_mlp_kernel<64, float, true>);
+    } else {
+        if (d == 16) run(ttt::simt_mlp_kernel<16, __nv_bfloat16, true>);
+        else if (d == 32) run(ttt::simt_mlp_kernel<32, __nv_bfloat16, true>);
+        else run(ttt::simt_mlp_kernel<64, __nv_bfloat16, true>);
+    }
+    return 0;
+}
+extern "C" int emu_mlp_ln_backward(int io, int B, int H, int T, int d, int b, const void* Q, const void* K,
+                                   const void* V, const float* eta, float eta_const, const float* W_states,
+                                   const void* dZ, const float* dW1o, const float* dc1o, const float* dW2o,
+                                   const float* dc2o, const float* gamma, const float* beta, float eps, void* dQ,
+                                   void* dK, void* dV, float* deta, float* dW1, float* dc1, float* dW2, float* dc2,
+                                   float* dgamma, float* dbeta) {
+    ttt::SimtMlpBackwardParams q{H,    T,    b,  Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
+                                 dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2,
+                                 gamma, beta, eps, dgamma, dbeta};
+    auto run = [&](auto kernel) { emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { kernel(q); }); };
+    if (io == 0) {
+        if (d == 16) run(ttt::simt_mlp_backward_kernel<16, float, true>);
+        else if (d == 32) run(ttt::simt_mlp_backward_kernel<32, float, true>);
+        else run(ttt::simt_mlp_backward_kernel<64, float, true>);
+    } else {
+        if (d == 16) run(ttt::simt_mlp_backward_kernel<16, __nv_bfloat16, true>);
+        else if (d == 32) run(ttt::simt_mlp_backward_kernel<32, __nv_bfloat16, true>);
+        else run(ttt::simt_mlp_backward_kernel<64, __nv_bfloat16, true>);
+    }
+    return 0;
+}
