@@ -806,12 +806,19 @@ def run_train(args):
     if w.kind == "mlp":
         m = w.hidden
         states = torch.empty((B, H, T // w.b, 2 * d * m + m + d), device="cuda")
+        ln = {}
+        if args.mlp_ln:
+            # LN+residual on the output layer, gamma ~ 1 + N(0, .02), beta ~ N(0, .02) as for the LN workload
+            g2 = torch.Generator(device="cuda")
+            g2.manual_seed(6)
+            ln = dict(use_ln=True, gamma=1 + 0.02 ** 0.5 * torch.randn(H, d, generator=g2, device="cuda"),
+                      beta=0.02 ** 0.5 * torch.randn(H, d, generator=g2, device="cuda"))
 
         def step():
             ttt.mlp_forward(dev["Q"], dev["K"], dev["V"], eta, dev["W1"], dev["c1"], dev["W2"], dev["c2"], w.b,
-                            eta_const=w.eta_const, W_states=states)
+                            eta_const=w.eta_const, W_states=states, **ln)
             ttt.mlp_backward(dev["Q"], dev["K"], dev["V"], eta, states, w.b, eta_const=w.eta_const, dZ=dZ,
-                             want_deta=eta is not None)
+                             want_deta=eta is not None, **ln)
     elif w.kind == "ln":
         states = torch.empty((B, H, T // w.b, d, d), device="cuda")
         cst = torch.empty((B, H, T // w.b, d), device="cuda")
@@ -840,6 +847,8 @@ def run_train(args):
     kernels = "forward with states, then the backward"
     if w.kind == "ln":
         kernels += " (mma.sync LN kernels)" if args.ln_mma else " (fp32 CUDA-core LN kernels)"
+    if w.kind == "mlp":
+        kernels += " (LN+residual on the output layer, fp32 CUDA cores)" if args.mlp_ln else " (mma.sync)"
     print(json.dumps({"train_step_ms": ms, "tokens_per_s": tokens(w) / (ms / 1000.0), "workload": w.name,
                       "steps": args.steps, "warmup": args.warmup, "kernels": kernels}), flush=True)
 
@@ -930,6 +939,8 @@ def main():
                          "workload) instead of the benchmark line")
     ap.add_argument("--ln-mma", action="store_true",
                     help="with --train on the LN workload: the mma.sync LN training kernels")
+    ap.add_argument("--mlp-ln", action="store_true",
+                    help="with --train on the MLP workload: TTT-MLP with LN+residual on the output layer")
     ap.add_argument("--prologue", action="store_true",
                     help="the fused prologue (views and learning-rate gate from the layer input) instead of the "
                          "benchmark line")
