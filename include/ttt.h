@@ -287,8 +287,10 @@ ttt_status ttt_mlp_forward(const ttt_mlp_args* args, cudaStream_t stream);
  *   use_ln         1: the model of ttt_mlp_forward with use_ln (ln_gamma,
  *                  ln_beta [H, d], ln_eps as given to it); the outputs dgamma,
  *                  dbeta [B, H, d] receive the per-unit gradients of gamma and
- *                  beta.  Runs on the fp32 CUDA-core kernel (b up to 16 at
- *                  d = 64 for shared memory).  0: plain.
+ *                  beta.  BF16 with d = 64, b = 16 runs on the mma.sync
+ *                  kernel as for the plain model; every other case on the
+ *                  fp32 CUDA-core kernel (b up to 16 at d = 64 for shared
+ *                  memory).  0: plain.
  */
 typedef struct {
     int B, H, T, d, b;

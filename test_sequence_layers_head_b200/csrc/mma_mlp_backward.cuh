@@ -56,7 +56,8 @@ constexpr int kOffL1 = kOffL2 + 1024;            // tril(-dAq D1^T)
 constexpr int kOffPart = kOffL1 + 1024;          // split-K partials: 8 warps x 16 x 16 fp32
 constexpr int kOffRow = kOffPart + 8 * 1024;     // per-warp row partials: 8 x 16 fp32
 constexpr int kOffEta = kOffRow + 512;
-constexpr int kSmemBytes = kOffEta + 64;
+constexpr int kOffX = kOffEta + 64;              // LN row sums: two areas of 8 warps x 16 rows x 4 fp32
+constexpr int kSmemBytes = kOffX + 2 * 2048;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
 // element (row, col) of a [rows][256] bf16 matrix stored as four [rows][64] tiles of `tile` bytes
@@ -187,6 +188,33 @@ struct Ops {
     }
     // split-K 16 x 16 product over the hidden units: sum over warps of A[:, p0..] B[:, p0..]^T into dst,
     // masked to s <= t and with `add` on the kept entries, scaled by `scale`
+    // sums over the CTA's 64 features of rows r and r + 8 for NQ quantities v[k][h], through exchange area
+    // `xa` (two areas used in turn, so consecutive calls never overwrite values still being read)
+    template <int NQ>
+    __device__ __forceinline__ void rows(float (&v)[NQ][2], float* xa) const {
+#pragma unroll
+        for (int k = 0; k < NQ; ++k)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                v[k][h] += __shfl_xor_sync(0xffffffffu, v[k][h], 1);
+                v[k][h] += __shfl_xor_sync(0xffffffffu, v[k][h], 2);
+            }
+        if (c == 0)
+#pragma unroll
+            for (int k = 0; k < NQ; ++k)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) xa[(w * kB + r + 8 * h) * 4 + k] = v[k][h];
+        __syncthreads();
+#pragma unroll
+        for (int k = 0; k < NQ; ++k)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float sum = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < 8; ++ww) sum += xa[(ww * kB + r + 8 * h) * 4 + k];
+                v[k][h] = sum;
+            }
+    }
     __device__ __forceinline__ void tt_split(uint32_t ta, uint32_t tb, float* dst, float add, float scale) const {
         float x[2][4] = {};
 #pragma unroll
@@ -215,6 +243,10 @@ struct Ops {
 
 };
 
+// LN = true: LN+residual on the output layer (the steps of simt_mlp_backward_kernel<D, IO, true>): Delta2
+// takes E's place, dP takes dZ's (the dZ tile is overwritten by dP), and the complete adjoint of Delta2
+// goes through each row's LN+residual backward to dY (written to the dE tile) and de.
+template <bool LN = false>
 __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBackwardParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t s0 = smem_u32(smem);
@@ -249,6 +281,17 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
     const int j0 = jn0 + 8 * jh;
     constexpr size_t SZ = 2 * (size_t)kD * kM + kM + kD;
     const Ops ops{smem, part, rowp, tid, w, l, r, c, p0, jn0, jh, j0};
+    float* xa0 = reinterpret_cast<float*>(smem + kOffX);
+    float* xa1 = xa0 + 512;
+    const float inv_d = 1.f / kD;
+    // LN: gamma, beta of this lane's two features j0 + 2c + k, and the lane's partial dgamma, dbeta
+    float gm[2] = {0.f, 0.f}, bt[2] = {0.f, 0.f}, dgp[2] = {0.f, 0.f}, dbp[2] = {0.f, 0.f};
+    if (LN)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            gm[k] = p.gamma[(size_t)(unit % p.H) * kD + j0 + 2 * c + k];
+            bt[k] = p.beta[(size_t)(unit % p.H) * kD + j0 + 2 * c + k];
+        }
 
     // the adjoint of the final state: the upstream gradients, or zero
     for (int e = tid; e < kD * kM; e += kThreads) {
@@ -335,16 +378,60 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             E_[0] = E_[2] = cc.x;
             E_[1] = E_[3] = cc.y;
             ops.bd_A_X(E_, sHk, sW2);
+            if (!LN) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const __nv_bfloat162 v2 =
+                        *reinterpret_cast<const __nv_bfloat162*>(V + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c);
+                    E_[2 * h] -= __bfloat162float(v2.x);
+                    E_[2 * h + 1] -= __bfloat162float(v2.y);
+                }
+            }
+        }
+        // LN: E_ holds Y = Hk W2 + c2; per row, Xh = LN(Y) (r), E = K + gamma Xh + beta - V,
+        // Delta2 = r (G - mean(G) - Xh mean(G Xh)) with G = gamma E, which takes E's place
+        float xh[4] = {}, rY[2] = {}, mg[2] = {}, mgx[2] = {};
+        auto e_of = [&](int q) {   // E at (row r + 8 (q >> 1), feature j0 + 2c + (q & 1))
+            const int row = r + 8 * (q >> 1), j = j0 + 2 * c + (q & 1);
+            const float kv = __bfloat162float(
+                *reinterpret_cast<const __nv_bfloat16*>(smem + kOffK + toff(row, j >> 3) + 2 * (j & 7)));
+            const float vv = __bfloat162float(V[(size_t)(t0 + row) * kD + j]);
+            return kv + gm[q & 1] * xh[q] + bt[q & 1] - vv;
+        };
+        if (LN) {
+            float sy[2][2] = {};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                sy[0][q >> 1] += E_[q];
+                sy[1][q >> 1] += E_[q] * E_[q];
+            }
+            ops.rows<2>(sy, xa0);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const __nv_bfloat162 v2 =
-                    *reinterpret_cast<const __nv_bfloat162*>(V + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c);
-                E_[2 * h] -= __bfloat162float(v2.x);
-                E_[2 * h + 1] -= __bfloat162float(v2.y);
+                const float mu = sy[0][h] * inv_d;
+                rY[h] = rsqrtf(fmaxf(sy[1][h] * inv_d - mu * mu, 0.f) + p.eps);
+                xh[2 * h] = (E_[2 * h] - mu) * rY[h];
+                xh[2 * h + 1] = (E_[2 * h + 1] - mu) * rY[h];
             }
-            ops.store_bd(kOffE, E_);
+            float sg[2][2] = {};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float g = gm[q & 1] * e_of(q);
+                sg[0][q >> 1] += g;
+                sg[1][q >> 1] += g * xh[q];
+            }
+            ops.rows<2>(sg, xa1);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                mg[h] = sg[0][h] * inv_d;
+                mgx[h] = sg[1][h] * inv_d;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                E_[q] = rY[q >> 1] * (gm[q & 1] * e_of(q) - mg[q >> 1] - xh[q] * mgx[q >> 1]);
         }
-        __syncthreads();   // E
+        ops.store_bd(kOffE, E_);
+        __syncthreads();   // E (LN: Delta2)
         // M = E W2^T, D1 = M GELU'(A) on this warp's hidden units
         float M_[4][4] = {};
         ops.mm_A_Xt(M_, sE, sW2);
@@ -381,6 +468,55 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
         __syncthreads();   // Hq
         // P2 = tril(Hq Hk^T + 1)
         ops.tt_split(sHq, sHk, P2, 1.f, 1.f);
+        if (LN) {
+            // the outputs' pre-LN P = Hq W2 + c2 - P2 diag(eta) Delta2 on this warp's features, its LN, and
+            // dP = the LN adjoint of gamma dZ, written over the dZ tile (dZ itself is read again from global
+            // memory for dQ); the outputs' dgamma, dbeta terms
+            float pz[4];
+            const float2 cc = *reinterpret_cast<const float2*>(c2s + j0 + 2 * c);
+            pz[0] = pz[2] = cc.x;
+            pz[1] = pz[3] = cc.y;
+            ops.bd_A_X(pz, sHq, sW2);
+            uint32_t a[4], b[4];
+            frag_from_f32(P2, false, s_eta, l, a);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) a[q] ^= 0x80008000u;
+            ldsm4t(bt_addr(sE, jn0, 0, l), b);
+            mma(pz, a, jh ? b[2] : b[0], jh ? b[3] : b[1]);
+            float sp[2][2] = {};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                sp[0][q >> 1] += pz[q];
+                sp[1][q >> 1] += pz[q] * pz[q];
+            }
+            ops.rows<2>(sp, xa0);
+            float ro[2], dz[4], sd[2][2] = {};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float mu = sp[0][h] * inv_d;
+                ro[h] = rsqrtf(fmaxf(sp[1][h] * inv_d - mu * mu, 0.f) + p.eps);
+                const float2 zz = tile_pair_bf16(smem, kOffDZ, r + 8 * h, j0 + 2 * c);
+                dz[2 * h] = zz.x;
+                dz[2 * h + 1] = zz.y;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int q = 2 * h + k;
+                    pz[q] = (pz[q] - mu) * ro[h];   // Xo
+                    const float gd = gm[k] * dz[q];
+                    sd[0][h] += gd;
+                    sd[1][h] += gd * pz[q];
+                    dgp[k] += dz[q] * pz[q];
+                    dbp[k] += dz[q];
+                }
+            }
+            ops.rows<2>(sd, xa1);
+            float dpv[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                dpv[q] = ro[q >> 1] * (gm[q & 1] * dz[q] - sd[0][q >> 1] * inv_d - pz[q] * sd[1][q >> 1] * inv_d);
+            ops.store_bd(kOffDZ, dpv);
+            __syncthreads();   // dP over the dZ tile
+        }
         // ---- backward.  Products with the end-state adjoint (GW1, GW2 copies), dHq = dZ W2^T,
         // dL2 = tril(-dZ E^T)
         float G2[4], dKx[4];
@@ -547,11 +683,57 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
 #pragma unroll
             for (int q = 0; q < 4; ++q) dKx[q] += eta_r[q >> 1] * y[q];
             ops.bd_A_X(G2, sDM, sW2);   // dE += dM W2
+            float dev_[4];               // the adjoint that reaches K and V (de with LN)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dev_[q] = G2[q];
+            if (LN) {
+                // G2 holds dDelta2: each row's LN+residual backward to de and dY (dY into G2)
+                float s3[3][2] = {};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int h = q >> 1;
+                    const float u = gm[q & 1] * e_of(q) - mg[h] - xh[q] * mgx[h];
+                    const float du = rY[h] * G2[q];
+                    s3[0][h] += G2[q] * u;
+                    s3[1][h] += du;
+                    s3[2][h] += du * xh[q];
+                }
+                ops.rows<3>(s3, xa0);
+                float s2[2][2] = {}, dx[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int h = q >> 1, k = q & 1;
+                    const float ev = e_of(q);
+                    const float du = rY[h] * G2[q];
+                    const float dg = du - s3[1][h] * inv_d - xh[q] * s3[2][h] * inv_d;
+                    const float de = gm[k] * dg;
+                    dx[q] = -du * mgx[h] - gm[k] * ev * s3[2][h] * inv_d + gm[k] * de;
+                    dgp[k] += ev * dg + xh[q] * de;
+                    dbp[k] += de;
+                    dev_[q] = de;
+                    s2[0][h] += dx[q];
+                    s2[1][h] += dx[q] * xh[q];
+                }
+                ops.rows<2>(s2, xa1);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int h = q >> 1;
+                    G2[q] = rY[h] * (dx[q] - s2[0][h] * inv_d - xh[q] * s2[1][h] * inv_d) -
+                            s3[0][h] * rY[h] * rY[h] * xh[q] * inv_d;   // dY
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    dKx[q] += dev_[q];
+                    // dQ also has the output residual's dZ (read again from global memory)
+                    dQx[q] += dZ ? __bfloat162float(dZ[(size_t)(t0 + r + 8 * (q >> 1)) * kD + j0 + 2 * c + (q & 1)])
+                                 : 0.f;
+                }
+            }
             ops.store_bd(kOffDE, G2);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 *reinterpret_cast<__nv_bfloat162*>(dV + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c) =
-                    __floats2bfloat162_rn(-G2[2 * h], -G2[2 * h + 1]);
+                    __floats2bfloat162_rn(-dev_[2 * h], -dev_[2 * h + 1]);
                 *reinterpret_cast<__nv_bfloat162*>(dQ + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c) =
                     __floats2bfloat162_rn(dQx[2 * h], dQx[2 * h + 1]);
             }
@@ -677,6 +859,23 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_backward_kernel(SimtMlpBa
             }
         }
         __syncthreads();   // every read of this mini-batch's shared data and of the adjoint is done
+    }
+    if (LN) {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            dgp[k] += __shfl_xor_sync(0xffffffffu, dgp[k], 4);
+            dgp[k] += __shfl_xor_sync(0xffffffffu, dgp[k], 8);
+            dgp[k] += __shfl_xor_sync(0xffffffffu, dgp[k], 16);
+            dbp[k] += __shfl_xor_sync(0xffffffffu, dbp[k], 4);
+            dbp[k] += __shfl_xor_sync(0xffffffffu, dbp[k], 8);
+            dbp[k] += __shfl_xor_sync(0xffffffffu, dbp[k], 16);
+        }
+        if (r == 0)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                p.dgamma[(size_t)unit * kD + j0 + 2 * c + k] = dgp[k];
+                p.dbeta[(size_t)unit * kD + j0 + 2 * c + k] = dbp[k];
+            }
     }
 }
 

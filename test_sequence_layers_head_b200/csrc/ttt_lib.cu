@@ -570,15 +570,15 @@ extern "C" ttt_status ttt_mlp_backward(const ttt_mlp_backward_args* a, cudaStrea
     if (a->use_ln && (!ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !(a->ln_eps > 0.f) || !ok_ptr(a->dgamma) ||
                       !ok_ptr(a->dbeta)))
         return TTT_ERR_INVALID_ARG;
-    if (!a->use_ln && a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
-        !(a->flags & TTT_FLAG_FORCE_SIMT)) {
+    if (a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 && !(a->flags & TTT_FLAG_FORCE_SIMT)) {
         SimtMlpBackwardParams p{a->H,       a->T,       a->b,       a->Q,       a->K,       a->V,
                                 a->eta,     a->eta_const, a->W_states, a->dZ,   a->dW1_out, a->dc1_out,
                                 a->dW2_out, a->dc2_out, a->dQ,      a->dK,      a->dV,      a->deta,
-                                a->dW1,     a->dc1,     a->dW2,     a->dc2,     nullptr,    nullptr,
-                                0.f,        nullptr,    nullptr};
-        if (!set_smem(mmb::mma_mlp_backward_kernel, mmb::kSmemBytes)) return TTT_ERR_CUDA;
-        mmb::mma_mlp_backward_kernel<<<(unsigned)units, mmb::kThreads, mmb::kSmemBytes, stream>>>(p);
+                                a->dW1,     a->dc1,     a->dW2,     a->dc2,     a->ln_gamma, a->ln_beta,
+                                a->ln_eps,  a->dgamma,  a->dbeta};
+        auto k = a->use_ln ? mmb::mma_mlp_backward_kernel<true> : mmb::mma_mlp_backward_kernel<false>;
+        if (!set_smem(k, mmb::kSmemBytes)) return TTT_ERR_CUDA;
+        k<<<(unsigned)units, mmb::kThreads, mmb::kSmemBytes, stream>>>(p);
         return launch_status();
     }
     if (simt_mlp_backward_smem(a->d, a->b, a->use_ln != 0) > 227 * 1024) return TTT_ERR_UNSUPPORTED;

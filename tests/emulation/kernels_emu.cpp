@@ -239,7 +239,7 @@ extern "C" int emu_mlp_backward_mma(int B, int H, int T, const void* Q, const vo
     static_assert(ttt::mmb::kSmemBytes <= (int)sizeof(ttt::mmb::smem), "emulated shared memory");
     ttt::SimtMlpBackwardParams q{H,    T,    16, Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
                                  dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2};
-    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_backward_kernel(q); });
+    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_backward_kernel<false>(q); });
     return 0;
 }
 
@@ -367,5 +367,19 @@ extern "C" int emu_mlp_ln_backward(int io, int B, int H, int T, int d, int b, co
         else if (d == 32) run(ttt::simt_mlp_backward_kernel<32, __nv_bfloat16, true>);
         else run(ttt::simt_mlp_backward_kernel<64, __nv_bfloat16, true>);
     }
+    return 0;
+}
+
+// the TTT-MLP with LN+residual backward on mma.sync (bf16, d = 64, b = 16), from the CUDA-core LN forward's states
+extern "C" int emu_mlp_ln_backward_mma(int B, int H, int T, const void* Q, const void* K, const void* V,
+                                       const float* eta, float eta_const, const float* W_states, const void* dZ,
+                                       const float* dW1o, const float* dc1o, const float* dW2o, const float* dc2o,
+                                       const float* gamma, const float* beta, float eps, void* dQ, void* dK,
+                                       void* dV, float* deta, float* dW1, float* dc1, float* dW2, float* dc2,
+                                       float* dgamma, float* dbeta) {
+    ttt::SimtMlpBackwardParams q{H,    T,    16, Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
+                                 dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2,
+                                 gamma, beta, eps, dgamma, dbeta};
+    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_backward_kernel<true>(q); });
     return 0;
 }

@@ -204,3 +204,26 @@ def test_mlp_ln_training_matches_oracle(ttt_lib, B, H, T, d, b, io):
             assert normwise(g, want) <= 2e-2, nm
         else:
             assert maxrel(g, want) <= 1e-4, (nm, maxrel(g, want))
+
+
+def test_mlp_ln_backward_tensor_cores_match_cuda_cores(ttt_lib):
+    """With LN+residual, bf16 d = 64 b = 16 runs the backward on mma.sync and TTT_FLAG_FORCE_SIMT on fp32
+    CUDA cores: the two agree within the bf16 bar on every gradient, dgamma and dbeta included."""
+    d, b, m = 64, 16, 256
+    inp, c1, c2, dz, ups = _case(2, 2, 64, d, b, WL.BF16, True, True, seed=71)
+    r = inp.raw
+    rng = np.random.default_rng(72)
+    gam = to_dev((1 + rng.standard_normal((2, d)) * 0.2).astype(np.float32))
+    bet = to_dev((rng.standard_normal((2, d)) * 0.2).astype(np.float32))
+    Q, K, V, eta = (to_dev(r[n]) for n in ("Q", "K", "V", "eta"))
+    states = torch.empty((2, 2, 64 // b, 2 * d * m + m + d), device="cuda")
+    ttt_lib.mlp_forward(Q, K, V, eta, to_dev(r["W1"]), to_dev(c1), to_dev(r["W2"]), to_dev(c2), b, use_ln=True,
+                        gamma=gam, beta=bet, W_states=states)
+    kw = dict(dZ=to_dev(dz[0]), use_ln=True, gamma=gam, beta=bet,
+              **{k: to_dev(u) for k, u in zip(("dW1_out", "dc1_out", "dW2_out", "dc2_out"), ups)})
+    tc = ttt_lib.mlp_backward(Q, K, V, eta, states, b, **kw)
+    simt = ttt_lib.mlp_backward(Q, K, V, eta, states, b, flags=ttt_lib.FLAG_FORCE_SIMT, **kw)
+    torch.cuda.synchronize()
+    assert ttt_lib.last_device_status() == ttt_lib.TTT_OK
+    for a, b_ in zip(tc, simt):
+        assert normwise(to_host(a), to_host(b_)) <= 2e-2

@@ -420,3 +420,53 @@ def test_mlp_ln_forward_states_and_backward(emu, B, H, T, d, b, io, per_token, u
             assert normwise(got, want) < 2e-2, nm
         else:
             assert maxrel(got, want) < 1e-4, (nm, maxrel(got, want))
+
+
+@pytest.mark.parametrize("B,H,T,per_token,upstream", [(1, 2, 32, True, True), (1, 1, 48, False, False)])
+def test_mlp_ln_backward_on_mma_sync(emu, B, H, T, per_token, upstream):
+    """The TTT-MLP with LN+residual backward on mma.sync (bf16, d = 64, b = 16), from the states the
+    CUDA-core LN forward writes, against the oracle (bf16 bar), dgamma and dbeta included."""
+    d, b, m = 64, 16, 256
+    inp = WL.random_case("mlp", B, H, T, d, b, io_dtype=WL.BF16, eta_mode="sigmoid", seed=5 + T)
+    raw, ex = inp.raw, inp.exact
+    rng = np.random.default_rng(3 + T)
+    c1 = (rng.standard_normal((H, m)) * 0.1).astype(np.float32)
+    c2 = (rng.standard_normal((H, d)) * 0.1).astype(np.float32)
+    gam = (1 + rng.standard_normal((H, d)) * 0.2).astype(np.float32)
+    bet = (rng.standard_normal((H, d)) * 0.2).astype(np.float32)
+    dZr, dZe = WL.store(rng.standard_normal((B, H, T, d)), WL.BF16)
+    ups = ([rng.standard_normal(s).astype(np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+           if upstream else [None] * 4)
+    nb = T // b
+    Z = np.zeros((B, H, T, d), np.uint16)
+    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    eta = raw["eta"] if per_token else None
+    f = emu.emu_mlp_ln_forward
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
+        [ctypes.c_float] + [ctypes.c_void_p] * 6
+    assert f(1, B, H, T, d, b, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(0.02), _p(raw["W1"]),
+             _p(c1), _p(raw["W2"]), _p(c2), _p(gam), _p(bet), np.float32(1e-6), _p(Z), *[_p(o) for o in outs],
+             _p(states)) == 0
+    dQ, dK, dV = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
+    deta = np.zeros((B, H, T), np.float32)
+    g = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d), (B, H, d), (B, H, d))]
+    bw = emu.emu_mlp_ln_backward_mma
+    bw.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 8 + \
+        [ctypes.c_float] + [ctypes.c_void_p] * 10
+    assert bw(B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(0.02), _p(states), _p(dZr),
+              *[_p(u) for u in ups], _p(gam), _p(bet), np.float32(1e-6), _p(dQ), _p(dK), _p(dV), _p(deta),
+              *[_p(x) for x in g]) == 0
+    eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(0.02)))
+    f64 = lambda a: a.astype(np.float64)
+    ref = O.mlp_ln_backward(ex["Q"], ex["K"], ex["V"], eta_e, ex["W1"], f64(c1), ex["W2"], f64(c2), b, f64(gam),
+                            f64(bet), 1e-6, dZ=dZe,
+                            **{k: (None if u is None else f64(u))
+                               for k, u in zip(("dW1_out", "dc1_out", "dW2_out", "dc2_out"), ups)})
+    h = WL.bf16_bits_to_f64
+    gots = [h(dQ), h(dK), h(dV), f64(deta)] + [f64(x) for x in g]
+    names = ("dQ", "dK", "dV", "deta", "dW1", "dc1", "dW2", "dc2", "dgamma", "dbeta")
+    for nm, got, want in zip(names, gots, ref):
+        if nm == "deta" and not per_token:
+            continue
+        assert normwise(got, want) < 2e-2, (nm, normwise(got, want))
