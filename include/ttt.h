@@ -224,9 +224,9 @@ ttt_status ttt_linear_backward(const ttt_linear_backward_args* args, cudaStream_
  *   W_states       NULL, or [B, H, T/b, 2dm + m + d] fp32: the state at the
  *                  start of every mini-batch, each one W1 [d][m], c1 [m],
  *                  W2 [m][d], c2 [d] (the checkpoints ttt_mlp_backward reads;
- *                  section 6.12).  BF16 with d = 64, b = 16 and no LN runs on
- *                  an mma.sync tensor-core kernel, every other case (and
- *                  TTT_FLAG_FORCE_SIMT) on the fp32 CUDA-core kernel.
+ *                  section 6.12).  BF16 with d = 64, b = 16 runs on an
+ *                  mma.sync tensor-core kernel (plain or use_ln), every other
+ *                  case (and TTT_FLAG_FORCE_SIMT) on the fp32 CUDA-core kernel.
  */
 typedef struct {
     int B, H, T, d, b;

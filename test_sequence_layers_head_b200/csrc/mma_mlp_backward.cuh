@@ -902,8 +902,14 @@ struct MlpFwdStatesParams {
     float* W2_out;
     float* c2_out;     // or null
     float* W_states;   // [units, T/16, 2 d m + m + d]
+    const float* gamma;   // LN+residual on the output layer (the LN instance): [H, 64]
+    const float* beta;
+    float eps;
 };
 
+// LN = true: f(x) = x + gamma LN(GELU(x W1 + c1) W2 + c2) + beta: Delta2 (the LN+residual backward at
+// Y = Hk W2 + c2) takes E's place, and Z = Q + gamma LN(P) + beta with P the plain model's output.
+template <bool LN = false>
 __global__ void __launch_bounds__(kThreads, 1) mma_mlp_forward_states_kernel(MlpFwdStatesParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     const uint32_t s0 = smem_u32(smem);
@@ -930,6 +936,16 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_forward_states_kernel(Mlp
     constexpr size_t SZ = 2 * (size_t)kD * kM + kM + kD;
     const Ops ops{smem, part, rowp, tid, w, l, r, c, p0, jn0, jh, j0};
     float* states = p.W_states + (size_t)unit * nb * SZ;
+    float* xa0 = reinterpret_cast<float*>(smem + kOffX);
+    float* xa1 = xa0 + 512;
+    const float inv_d = 1.f / kD;
+    float gm[2] = {0.f, 0.f}, bt[2] = {0.f, 0.f};
+    if (LN)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            gm[k] = p.gamma[(size_t)(unit % p.H) * kD + j0 + 2 * c + k];
+            bt[k] = p.beta[(size_t)(unit % p.H) * kD + j0 + 2 * c + k];
+        }
 
     // S_0: the initial state, to the first checkpoint
     if (nb > 0) {
@@ -1016,12 +1032,50 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_forward_states_kernel(Mlp
             E_[0] = E_[2] = cc.x;
             E_[1] = E_[3] = cc.y;
             ops.bd_A_X(E_, sHk, sW2);
+            float vv[4], kk[4];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const __nv_bfloat162 v2 =
                     *reinterpret_cast<const __nv_bfloat162*>(V + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c);
-                E_[2 * h] -= __bfloat162float(v2.x);
-                E_[2 * h + 1] -= __bfloat162float(v2.y);
+                vv[2 * h] = __bfloat162float(v2.x);
+                vv[2 * h + 1] = __bfloat162float(v2.y);
+                const float2 k2 = tile_pair_bf16(smem, kOffK, r + 8 * h, j0 + 2 * c);
+                kk[2 * h] = k2.x;
+                kk[2 * h + 1] = k2.y;
+            }
+            if (!LN) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) E_[q] -= vv[q];
+            } else {
+                // E_ holds Y: per row Xh = LN(Y), E = K + gamma Xh + beta - V, Delta2 = r (G - mean(G) - Xh
+                // mean(G Xh)), G = gamma E, which takes E's place
+                float sy[2][2] = {};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    sy[0][q >> 1] += E_[q];
+                    sy[1][q >> 1] += E_[q] * E_[q];
+                }
+                ops.rows<2>(sy, xa0);
+                float rY[2], xh[4], g[4], sg[2][2] = {};
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float mu = sy[0][h] * inv_d;
+                    rY[h] = rsqrtf(fmaxf(sy[1][h] * inv_d - mu * mu, 0.f) + p.eps);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int h = q >> 1;
+                    xh[q] = (E_[q] - sy[0][h] * inv_d) * rY[h];
+                    g[q] = gm[q & 1] * (kk[q] + gm[q & 1] * xh[q] + bt[q & 1] - vv[q]);
+                    sg[0][h] += g[q];
+                    sg[1][h] += g[q] * xh[q];
+                }
+                ops.rows<2>(sg, xa1);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int h = q >> 1;
+                    E_[q] = rY[h] * (g[q] - sg[0][h] * inv_d - xh[q] * sg[1][h] * inv_d);
+                }
             }
             ops.store_bd(kOffE, E_);
             float ee[4];
@@ -1103,6 +1157,24 @@ __global__ void __launch_bounds__(kThreads, 1) mma_mlp_forward_states_kernel(Mlp
             for (int q = 0; q < 4; ++q) a[q] ^= 0x80008000u;
             ldsm4t(bt_addr(sEE, jn0, 0, l), b);
             mma(z, a, jh ? b[2] : b[0], jh ? b[3] : b[1]);
+            if (LN) {
+                // Z = Q + gamma LN(P) + beta
+                float sz[2][2] = {};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    sz[0][q >> 1] += z[q];
+                    sz[1][q >> 1] += z[q] * z[q];
+                }
+                ops.rows<2>(sz, xa0);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float mu = sz[0][h] * inv_d;
+                    const float ro = rsqrtf(fmaxf(sz[1][h] * inv_d - mu * mu, 0.f) + p.eps);
+                    const float2 qv = tile_pair_bf16(smem, kOffQ, r + 8 * h, j0 + 2 * c);
+                    z[2 * h] = qv.x + gm[0] * (z[2 * h] - mu) * ro + bt[0];
+                    z[2 * h + 1] = qv.y + gm[1] * (z[2 * h + 1] - mu) * ro + bt[1];
+                }
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h)
                 *reinterpret_cast<__nv_bfloat162*>(Z + (size_t)(t0 + r + 8 * h) * kD + j0 + 2 * c) =

@@ -347,15 +347,17 @@ extern "C" ttt_status ttt_mlp_forward(const ttt_mlp_args* a, cudaStream_t stream
     if (a->use_ln != 0 && a->use_ln != 1) return TTT_ERR_INVALID_ARG;
     if (a->use_ln && (!ok_ptr(a->ln_gamma) || !ok_ptr(a->ln_beta) || !(a->ln_eps > 0.f))) return TTT_ERR_INVALID_ARG;
     if (!ok_opt(a->W_states)) return TTT_ERR_INVALID_ARG;
-    if (a->W_states && !a->use_ln && a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
+    if (a->W_states && a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&
         !(a->flags & TTT_FLAG_FORCE_SIMT)) {
         // training: the mma.sync forward that writes the batch-start states
         if (a->flags & TTT_FLAG_TEST_STALL) return TTT_ERR_UNSUPPORTED;
         mmb::MlpFwdStatesParams p{a->H,      a->T,     a->Q,     a->K,      a->V,     a->eta,
                                   a->eta_const, a->W1, a->c1,    a->W2,     a->c2,    a->params_per_sequence,
-                                  a->Z,      a->W1_out, a->c1_out, a->W2_out, a->c2_out, a->W_states};
-        if (!set_smem(mmb::mma_mlp_forward_states_kernel, mmb::kSmemBytes)) return TTT_ERR_CUDA;
-        mmb::mma_mlp_forward_states_kernel<<<(unsigned)units, mmb::kThreads, mmb::kSmemBytes, stream>>>(p);
+                                  a->Z,      a->W1_out, a->c1_out, a->W2_out, a->c2_out, a->W_states,
+                                  a->ln_gamma, a->ln_beta, a->ln_eps};
+        auto k = a->use_ln ? mmb::mma_mlp_forward_states_kernel<true> : mmb::mma_mlp_forward_states_kernel<false>;
+        if (!set_smem(k, mmb::kSmemBytes)) return TTT_ERR_CUDA;
+        k<<<(unsigned)units, mmb::kThreads, mmb::kSmemBytes, stream>>>(p);
         return launch_status();
     }
     const bool tc = a->io_dtype == TTT_BF16 && a->d == 64 && a->b == 16 && a->T > 0 &&

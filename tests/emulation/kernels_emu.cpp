@@ -250,7 +250,7 @@ extern "C" int emu_mlp_forward_mma(int B, int H, int T, const void* Q, const voi
                                    float* c2_out, float* W_states) {
     ttt::mmb::MlpFwdStatesParams f{H,  T,      Q,      K,      V,      eta,    eta_const, W1,      c1,
                                    W2, c2,     0,      Z,      W1_out, c1_out, W2_out,    c2_out, W_states};
-    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_forward_states_kernel(f); });
+    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_forward_states_kernel<false>(f); });
     return 0;
 }
 
@@ -381,5 +381,18 @@ extern "C" int emu_mlp_ln_backward_mma(int B, int H, int T, const void* Q, const
                                  dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2,
                                  gamma, beta, eps, dgamma, dbeta};
     emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_backward_kernel<true>(q); });
+    return 0;
+}
+
+// the TTT-MLP with LN+residual forward writing the batch-start states on mma.sync (bf16, d = 64, b = 16)
+extern "C" int emu_mlp_ln_forward_mma(int B, int H, int T, const void* Q, const void* K, const void* V,
+                                      const float* eta, float eta_const, const float* W1, const float* c1,
+                                      const float* W2, const float* c2, const float* gamma, const float* beta,
+                                      float eps, void* Z, float* W1_out, float* c1_out, float* W2_out, float* c2_out,
+                                      float* W_states) {
+    ttt::mmb::MlpFwdStatesParams f{H,  T,      Q,      K,      V,      eta,    eta_const, W1,      c1,
+                                   W2, c2,     0,      Z,      W1_out, c1_out, W2_out,    c2_out, W_states,
+                                   gamma, beta, eps};
+    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_forward_states_kernel<true>(f); });
     return 0;
 }

@@ -470,3 +470,44 @@ def test_mlp_ln_backward_on_mma_sync(emu, B, H, T, per_token, upstream):
         if nm == "deta" and not per_token:
             continue
         assert normwise(got, want) < 2e-2, (nm, normwise(got, want))
+
+
+@pytest.mark.parametrize("B,H,T,per_token", [(1, 2, 48, True), (2, 1, 32, False)])
+def test_mlp_ln_forward_states_on_mma_sync(emu, B, H, T, per_token):
+    """TTT-MLP with LN+residual, the forward writing its batch-start states on mma.sync (bf16, d = 64,
+    b = 16): Z, the final state and every checkpoint against the oracle (bf16 bar)."""
+    d, b, m = 64, 16, 256
+    inp = WL.random_case("mlp", B, H, T, d, b, io_dtype=WL.BF16, eta_mode="sigmoid" if per_token else "const",
+                         eta_const=0.0 if per_token else 0.02, seed=81 + T)
+    raw, ex = inp.raw, inp.exact
+    rng = np.random.default_rng(300 + T)
+    c1 = (rng.standard_normal((H, m)) * 0.1).astype(np.float32)
+    c2 = (rng.standard_normal((H, d)) * 0.1).astype(np.float32)
+    gam = (1 + rng.standard_normal((H, d)) * 0.2).astype(np.float32)
+    bet = (rng.standard_normal((H, d)) * 0.2).astype(np.float32)
+    nb = T // b
+    Z = np.zeros((B, H, T, d), np.uint16)
+    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    eta = raw["eta"] if per_token else None
+    f = emu.emu_mlp_ln_forward_mma
+    f.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
+        [ctypes.c_float] + [ctypes.c_void_p] * 6
+    assert f(B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const), _p(raw["W1"]),
+             _p(c1), _p(raw["W2"]), _p(c2), _p(gam), _p(bet), np.float32(1e-6), _p(Z), *[_p(o) for o in outs],
+             _p(states)) == 0
+    eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(inp.w.eta_const)))
+    f64 = lambda a: a.astype(np.float64)
+    params = (ex["W1"], f64(c1), ex["W2"], f64(c2))
+    ln = dict(use_ln=True, gamma=f64(gam), beta=f64(bet))
+    ref = O.mlp_forward(ex["Q"], ex["K"], ex["V"], eta_e, *params, b, **ln)
+    assert normwise(WL.bf16_bits_to_f64(Z), ref[0]) < 2e-2
+    for got, want in zip(outs, ref[1:]):
+        assert normwise(f64(got), want) < 2e-2
+    for i in range(nb):
+        t = i * b
+        st = O.mlp_forward(ex["Q"][:, :, :t], ex["K"][:, :, :t], ex["V"][:, :, :t], eta_e[:, :, :t], *params, b,
+                           **ln)[1:]
+        parts = np.split(states[:, :, i], [d * m, d * m + m, 2 * d * m + m], axis=-1)
+        for g, r in zip(parts, st):
+            assert normwise(f64(g).reshape(r.shape), r) < 2e-2
