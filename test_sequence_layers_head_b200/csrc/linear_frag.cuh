@@ -112,6 +112,7 @@ __device__ __forceinline__ uint32_t ablk_off(int m, int k) {
     return (m >> 3) * 1024 + (k >> 3) * 128 + (m & 7) * 16 + (k & 7) * 2;
 }
 
+#ifndef TTT_HOST_EMULATION   // the host emulation supplies these four
 __device__ __forceinline__ void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t* r) {
     asm volatile("tcgen05.ld.sync.aligned.16x256b.x2.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
@@ -137,6 +138,7 @@ __device__ __forceinline__ void mma16816(float* d, const uint32_t* a, uint32_t b
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
+#endif
 
 // Helper: the 16 x 16 product X Y^T + add of two 16 x 64 tiles (fragments
 // given), masked to s <= t if `causal`, stored in bf16 at `dst` (layout of

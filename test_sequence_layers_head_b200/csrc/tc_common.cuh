@@ -43,6 +43,7 @@ __device__ __forceinline__ float ld_bf16(const uint8_t* base, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
 }
 
+#ifndef TTT_HOST_EMULATION   // the host emulation supplies these two
 // ldmatrix x4 (four 8x8 b16 matrices)
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -57,6 +58,7 @@ __device__ __forceinline__ void mma_16816(float* d, const uint32_t* a, uint32_t 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+#endif
 // A fragments (4 k-steps) of a 16 x 64 bf16 tile stored with the 128B swizzle
 __device__ __forceinline__ void load_a_frags(uint32_t tile, int lane, uint32_t (*f)[4]) {
     const int row = (lane & 7) + 8 * ((lane >> 3) & 1);
@@ -76,6 +78,7 @@ __device__ __forceinline__ void load_b_frags(uint32_t tile, int lane, uint32_t (
         ldsm_x4(tile + row * 128 + ((ch ^ (row & 7)) << 4), f[ks]);
     }
 }
+#ifndef TTT_HOST_EMULATION   // the host emulation supplies these
 __device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t* r) {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), TTT_W8(r, 0)
                  : "memory");
@@ -98,6 +101,7 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
         "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+#endif
 
 }  // namespace tcc
 }  // namespace ttt

@@ -159,37 +159,66 @@ inline void tmem_ld_32x32b(uint32_t taddr, uint32_t* r) {
 inline void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b<16>(taddr, r); }
 inline void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b<32>(taddr, r); }
 
-// The descriptors are the library's own encoding (make_sdesc, make_idesc_bf16 in ptx.cuh); layout
-// code 2 is the 128-byte swizzle.
-// element (row, k) of a K-major, 128-byte-swizzled bf16 operand
-inline float sw128_elem(uint64_t desc, int row, int k) {
+// The descriptors are the library's own encoding (make_sdesc, make_idesc_bf16 in ptx.cuh): start address,
+// leading (LBO) and stride (SBO) byte offsets, and the layout code (2: 128-byte swizzle, 0: none).
+// Element (mn, k) of a bf16 operand, mn the M or N index:
+//   K-major, 128-byte swizzle:  start + (mn / 8) SBO + (mn % 8) 128 + 2 k, address bits 4-6 ^= bits 7-9
+//   MN-major, 128-byte swizzle: start + (k / 8) SBO + (mn / 64) LBO + (k % 8) 128 + 2 (mn % 64), same XOR
+//   K-major, no swizzle (8 x 16-byte core matrices): start + (mn / 8) SBO + (k / 8) LBO + (mn % 8) 16 + 2 (k % 8)
+inline float operand_elem(uint64_t desc, bool mn_major, int mn, int k) {
     const uint32_t start = (uint32_t)(desc & 0x3FFFu) << 4;
+    const uint32_t lbo = (uint32_t)((desc >> 16) & 0x3FFFu) << 4;
     const uint32_t sbo = (uint32_t)((desc >> 32) & 0x3FFFu) << 4;
-    const uint32_t lin = start + (row / 8) * sbo + (row % 8) * 128 + 2 * k;
-    const uint32_t phys = lin ^ (((lin >> 7) & 7u) << 4);
+    const uint32_t layout = (uint32_t)(desc >> 61);
+    uint32_t phys = 0;
+    if (layout == 2u) {
+        const uint32_t lin = mn_major ? start + (k / 8) * sbo + (mn / 64) * lbo + (k % 8) * 128 + 2 * (mn % 64)
+                                      : start + (mn / 8) * sbo + (mn % 8) * 128 + 2 * k;
+        phys = lin ^ (((lin >> 7) & 7u) << 4);
+    } else if (layout == 0u && !mn_major) {
+        phys = start + (mn / 8) * sbo + (k / 8) * lbo + (mn % 8) * 16 + 2 * (k % 8);
+    } else {
+        ++emu::errors;
+    }
     const uint16_t h = emu::ld16(phys);
     uint32_t b = (uint32_t)h << 16;
     float f;
     std::memcpy(&f, &b, 4);
     return f;
 }
-inline void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+// D (M x N, fp32, TMEM lanes = rows) (+)= A B^T over K = 16; a(row, k) and b(col, k) give the operands
+template <typename FA, typename FB>
+inline void umma_apply(uint32_t d_tmem, uint32_t idesc, uint32_t accumulate, FA a, FB b) {
     const int M = (int)((idesc >> 24) & 0x1Fu) << 4, N = (int)((idesc >> 17) & 0x3Fu) << 3;
-    const bool a_mn = (idesc >> 15) & 1u, b_mn = (idesc >> 16) & 1u;
-    if (a_mn || b_mn || (adesc >> 61) != 2u || (bdesc >> 61) != 2u || M != 128 ||
-        N % 16 != 0 || N < 16 || N > 256 || ((adesc & 0x3FFFu) << 4) % 16 != 0)
-        ++emu::errors;
+    if (M != 128 || N % 16 != 0 || N < 16 || N > 256) ++emu::errors;
     const uint32_t l0 = emu::tmem_lane(d_tmem), c0 = emu::tmem_col(d_tmem);
+    float av[128][16];
     for (int row = 0; row < M; ++row)
-        for (int col = 0; col < N; ++col) {
+        for (int k = 0; k < 16; ++k) av[row][k] = a(row, k);
+    for (int col = 0; col < N; ++col) {
+        float bv[16];
+        for (int k = 0; k < 16; ++k) bv[k] = b(col, k);
+        for (int row = 0; row < M; ++row) {
             float acc = 0.f;
-            for (int k = 0; k < 16; ++k) acc += sw128_elem(adesc, row, k) * sw128_elem(bdesc, col, k);
+            for (int k = 0; k < 16; ++k) acc += av[row][k] * bv[k];
             uint32_t& cell = emu::tmem[(l0 + row) & 127][(c0 + col) & 511];
             float prev;
             std::memcpy(&prev, &cell, 4);
             const float v = (accumulate ? prev : 0.f) + acc;
             std::memcpy(&cell, &v, 4);
         }
+    }
+}
+inline void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+    const bool a_mn = (idesc >> 15) & 1u, b_mn = (idesc >> 16) & 1u;
+    umma_apply(
+        d_tmem, idesc, accumulate, [&](int row, int k) { return operand_elem(adesc, a_mn, row, k); },
+        [&](int col, int k) { return operand_elem(bdesc, b_mn, col, k); });
+}
+// A in tensor memory: element (row, k) at lane (lane + row), column (col + k / 2), the low half for even k
+inline float tmem_bf16(uint32_t a_tmem, int row, int k) {
+    const uint32_t v = emu::tmem[(emu::tmem_lane(a_tmem) + row) & 127][(emu::tmem_col(a_tmem) + k / 2) & 511];
+    return (k & 1) ? emu::bf16_hi(v) : emu::bf16_lo(v);
 }
 inline void umma_commit(uint64_t* bar) { emu::bar_arrive(bar, 0); }
 }  // namespace ttt
