@@ -1,6 +1,6 @@
 // Host emulation of the sm_100a asynchronous operations used by the tensor-core
-// prologue kernel, on top of emu_core.h: TEST INFRASTRUCTURE, never part of the
-// library.
+// kernels (tc_emu_lfr.h adds the rest of what the TTT-Linear kernel uses), on
+// top of emu_core.h: TEST INFRASTRUCTURE, never part of the library.
 //
 // Semantics (from the PTX ISA's descriptions):
 //   mbarrier: an expected arrival count and a transaction count per phase; the
@@ -11,11 +11,10 @@
 //     shared memory with the 16-byte chunk c of row r stored at chunk c ^ (r % 8);
 //     elements outside the tensor are zero; the whole box's bytes count toward
 //     the mbarrier's transaction count.
-//   tcgen05.mma kind::f16 (bf16 x bf16 -> f32), K = 16, both operands K-major
-//     with the 128-byte swizzle: element (row, k) of an operand is at byte
-//     start + (row / 8) * SBO + (row % 8) * 128 + 2 k, with address bits 4-6
-//     XORed with bits 7-9.  D (M x N) is at TMEM lanes 0 .. M-1, columns
-//     col .. col + N - 1.
+//   tcgen05.mma kind::f16 (bf16 x bf16 -> f32), K = 16, operands in shared
+//     memory (K-major or MN-major with the 128-byte swizzle, K-major without
+//     swizzle: the addressing is given at operand_elem below) or A in tensor
+//     memory.  D (M x N) is at TMEM lanes 0 .. M-1, columns col .. col + N - 1.
 //   tcgen05.ld .32x32b.xN: lane t of the warp reads TMEM lane (base + t),
 //     columns col .. col + N - 1; a warp may access the 32 lanes of its
 //     quadrant (warp % 4) only.

@@ -2,8 +2,9 @@
 the CUDA execution model (tests/emulation: one std::thread per CUDA thread,
 __syncthreads as a barrier, shuffles, ldmatrix and mma through a per-warp
 exchange with the PTX ISA's documented fragment layouts; for the tcgen05
-prologue also mbarriers, 2-D TMA loads, tensor memory and tcgen05.mma, with
-asynchronous operations completing at issue), against the float64 oracle.
+kernels also mbarriers, 2-D TMA loads and stores, tensor memory and
+tcgen05.mma, with asynchronous operations completing at issue), against the
+float64 oracle.
 
 This checks the source's index arithmetic, phase order and barrier placement
 where no GPU is present.  It is not the GPU parity: the tests marked gpu run
@@ -14,8 +15,9 @@ Covered: the TTT-MLP forward writing its batch-start states and the
 outer-loop backward that reads them (fp32 CUDA cores); the TTT-Linear pair
 on mma.sync (bf16, d = 64, b = 16) -- already verified on the B200, which
 pins the emulated ldmatrix / mma semantics; and the LN+residual pair on
-mma.sync; the TTT-MLP training pair on mma.sync; and the fused prologue on
-fp32 CUDA cores and on tcgen05 (paper digest
+mma.sync; the TTT-MLP training pair on mma.sync; the fused prologue on fp32
+CUDA cores and on tcgen05; and the TTT-Linear tensor-core prefill (tcgen05,
+already verified on the B200, which pins the emulated tcgen05 semantics) (paper digest
 "论文速览 | TTT", sections 3.3, 3.4, 3.6, 3.7, 4.4, 4.6, 6.12).
 """
 import ctypes
@@ -511,3 +513,58 @@ def test_mlp_ln_forward_states_on_mma_sync(emu, B, H, T, per_token):
         parts = np.split(states[:, :, i], [d * m, d * m + m, 2 * d * m + m], axis=-1)
         for g, r in zip(parts, st):
             assert normwise(f64(g).reshape(r.shape), r) < 2e-2
+
+
+@pytest.fixture(scope="module")
+def lfr_emu(tmp_path_factory):
+    so = str(tmp_path_factory.mktemp("lfr") / "tc_linear_emu.so")
+    subprocess.run(["g++", "-std=c++20", "-O1", "-fPIC", "-shared", "-I/usr/local/cuda/include", "-o", so,
+                    os.path.join(ROOT, "tests", "emulation", "tc_linear_emu.cpp"), "-lpthread"], check=True)
+    return ctypes.CDLL(so)
+
+
+@pytest.mark.parametrize("ln,upc,B,H,T,per_token", [
+    (False, 2, 1, 2, 64, True), (False, 1, 1, 1, 48, False), (False, 2, 1, 3, 80, True),
+    (True, 2, 1, 2, 64, True), (True, 1, 2, 1, 48, False), (True, 2, 1, 3, 48, True)])
+def test_linear_prefill_on_tcgen05(lfr_emu, ln, upc, B, H, T, per_token):
+    """The TTT-Linear tensor-core prefill (B200-verified) under the emulated
+    tcgen05 operations.  Its agreement with the oracle pins the emulation of
+    the MMA operand descriptors (K-major and MN-major 128-byte swizzle, K-major
+    without swizzle, A in tensor memory), the 32x32b TMEM loads and stores, the
+    accumulator layout of the 16x256b load, stmatrix.trans and the 32- and
+    64-byte swizzled TMA stores.  The state update W_T - W_0 is compared on its
+    own: the full state is dominated by W_0."""
+    d, b = 64, 16
+    inp = WL.random_case("ln" if ln else "linear", B, H, T, d, b, io_dtype=WL.BF16,
+                         eta_mode="sigmoid" if per_token else "const", eta_const=0.0 if per_token else 0.05,
+                         seed=3 + T)
+    raw, ex = inp.raw, inp.exact
+    rng = np.random.default_rng(2 + T)
+    c0 = (rng.standard_normal((H, d)) * 0.1).astype(np.float32) if ln else None
+    Z = np.zeros((B, H, T, d), np.uint16)
+    W_out = np.zeros((B, H, d, d), np.float32)
+    c_out = np.zeros((B, H, d), np.float32) if ln else None
+    status = np.zeros(1, np.int32)
+    eta = raw["eta"] if per_token else None
+    f = lfr_emu.emu_linear_tc
+    f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_longlong,
+                                                                ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p,
+                                                                ctypes.c_void_p, ctypes.c_float] + \
+        [ctypes.c_void_p] * 4
+    rc = f(int(ln), upc, B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const),
+           _p(raw["W0"]), 0, _p(c0), 0, _p(raw["gamma"]) if ln else None, _p(raw["beta"]) if ln else None,
+           np.float32(inp.w.ln_eps if ln else 0.0), _p(Z), _p(W_out), _p(c_out), _p(status))
+    assert rc == 0 and status[0] == 0
+    eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(inp.w.eta_const)))
+    if ln:
+        c0e = c0.astype(np.float64)
+        Zr, Wr, cr = O.linear_forward(ex["Q"], ex["K"], ex["V"], eta_e, ex["W0"], b, c0=c0e, gamma=ex["gamma"],
+                                      beta=ex["beta"], use_ln=True, eps=inp.w.ln_eps)
+        c0b = np.broadcast_to(c0e, cr.shape)
+        assert normwise(c_out.astype(np.float64) - c0b, cr - c0b) < 2e-2
+    else:
+        Zr, Wr, _ = O.linear_forward(ex["Q"], ex["K"], ex["V"], eta_e, ex["W0"], b)
+    W0b = np.broadcast_to(ex["W0"], Wr.shape)
+    assert normwise(WL.bf16_bits_to_f64(Z), Zr) < 2e-2
+    assert normwise(W_out.astype(np.float64), Wr) < 2e-2
+    assert normwise(W_out.astype(np.float64) - W0b, Wr - W0b) < 2e-2
