@@ -121,6 +121,7 @@ struct Params {
 
 __device__ __forceinline__ void tmem_ld_x16(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b_x16(taddr, r); }
 
+#ifndef TTT_HOST_EMULATION   // the host emulation supplies these nine
 // ldmatrix / stmatrix x4 with transpose
 __device__ __forceinline__ void ldsm_x4_tr(uint32_t addr, uint32_t* r) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
@@ -161,6 +162,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t* r) {
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
                  : "r"(taddr));
 }
+#endif
 // element e (accumulator order) of an ldmatrix.trans fragment set: n-tile nt,
 // rows r (e < 2) or r + 8, tokens 2c + (e & 1)
 __device__ __forceinline__ float frag_at(const uint32_t* f, int nt, int e) {

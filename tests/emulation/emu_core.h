@@ -103,6 +103,14 @@ inline float __shfl_xor_sync(unsigned, float v, int o) {
     emu::warp_sync();
     return r;
 }
+inline float __shfl_sync(unsigned, float v, int src) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    emu::xch[w].f[lane] = v;
+    emu::warp_sync();
+    const float r = emu::xch[w].f[src & 31];
+    emu::warp_sync();
+    return r;
+}
 inline float rsqrtf(float x) { return 1.0f / std::sqrt(x); }
 inline int min(int a, int b) { return a < b ? a : b; }
 inline int max(int a, int b) { return a > b ? a : b; }

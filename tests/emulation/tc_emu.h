@@ -185,11 +185,14 @@ inline float operand_elem(uint64_t desc, bool mn_major, int mn, int k) {
     std::memcpy(&f, &b, 4);
     return f;
 }
-// D (M x N, fp32, TMEM lanes = rows) (+)= A B^T over K = 16; a(row, k) and b(col, k) give the operands
+// D (M x N, fp32) (+)= A B^T over K = 16; a(row, k) and b(col, k) give the operands.  M = 128: row i of D
+// at TMEM lane (lane + i); M = 64: rows 16 q .. 16 q + 15 at lanes 32 q + (lane + 0 .. 15) of quadrant q
 template <typename FA, typename FB>
 inline void umma_apply(uint32_t d_tmem, uint32_t idesc, uint32_t accumulate, FA a, FB b) {
     const int M = (int)((idesc >> 24) & 0x1Fu) << 4, N = (int)((idesc >> 17) & 0x3Fu) << 3;
-    if (M != 128 || N % 16 != 0 || N < 16 || N > 256) ++emu::errors;
+    if (M == 128 ? (N % 16 != 0 || N < 16 || N > 256) : M == 64 ? (N % 8 != 0 || N < 8 || N > 256) : true)
+        ++emu::errors;
+    if (M == 64 && emu::tmem_lane(d_tmem) % 32 + 16 > 32) ++emu::errors;
     const uint32_t l0 = emu::tmem_lane(d_tmem), c0 = emu::tmem_col(d_tmem);
     float av[128][16];
     for (int row = 0; row < M; ++row)
@@ -200,7 +203,8 @@ inline void umma_apply(uint32_t d_tmem, uint32_t idesc, uint32_t accumulate, FA 
         for (int row = 0; row < M; ++row) {
             float acc = 0.f;
             for (int k = 0; k < 16; ++k) acc += av[row][k] * bv[k];
-            uint32_t& cell = emu::tmem[(l0 + row) & 127][(c0 + col) & 511];
+            const uint32_t dl = M == 64 ? l0 + 32 * (row / 16) + row % 16 : l0 + row;
+            uint32_t& cell = emu::tmem[dl & 127][(c0 + col) & 511];
             float prev;
             std::memcpy(&prev, &cell, 4);
             const float v = (accumulate ? prev : 0.f) + acc;

@@ -1,0 +1,62 @@
+// Entry point of the CPU tests' host emulation of the TTT-MLP tensor-core
+// kernel (tcgen05, M = 128 and M = 64 accumulators, TMEM-resident state):
+// TEST INFRASTRUCTURE; the library has no CPU path.  The kernel is the one
+// already verified on the B200, so this run pins the emulated M = 64
+// accumulator layout, MN-major A operands, the 16x128b TMEM store and the
+// x2 ldmatrix / stmatrix forms to hardware behaviour.
+#include "tc_emu_mtc.h"
+
+namespace ttt {
+namespace mtc {
+alignas(1024) uint8_t smem[160 * 1024];
+}
+}  // namespace ttt
+
+#include "../../test_sequence_layers_head_b200/csrc/mlp_tc.cuh"
+
+// The TTT-MLP prefill (plain or LN+residual on the output layer) with the
+// library's tensor maps, parameters and grid (one unit per CTA).  Returns the
+// number of emulated-hardware rule violations (0 when none), or -1 for a bad
+// request.
+extern "C" int emu_mlp_tc(int ln, int B, int H, int T, int per_seq, const void* Q, const void* K, const void* V,
+                          const float* eta, float eta_const, const float* W1, const float* c1, const float* W2,
+                          const float* c2, const float* gamma, const float* beta, float eps, void* Z, float* W1_out,
+                          float* c1_out, float* W2_out, float* c2_out, int* status) {
+    using namespace ttt::mtc;
+    if (T < kTok || T % kTok || static_cast<int>(sizeof(smem)) < kSmemBytes) return -1;
+    const long long U = (long long)B * H, rows = U * T;
+    CUtensorMap mQ, mK, mV;
+    emu::make_map(&mQ, Q, kD, rows, kD * 2, kD, kTok, 2);
+    emu::make_map(&mK, K, kD, rows, kD * 2, kD, kTok, 2);
+    emu::make_map(&mV, V, kD, rows, kD * 2, kD, kTok, 2);
+    Params p{};
+    p.H = H;
+    p.T = T;
+    p.nsteps = T / kTok;
+    p.per_seq = per_seq;
+    p.eta = eta;
+    p.eta_const = eta_const;
+    p.W1 = W1;
+    p.c1 = c1;
+    p.W2 = W2;
+    p.c2 = c2;
+    p.Z = static_cast<__nv_bfloat16*>(Z);
+    p.W1_out = W1_out;
+    p.c1_out = c1_out;
+    p.W2_out = W2_out;
+    p.c2_out = c2_out;
+    p.status = status;
+    p.wait_ns = 240ull * 1000000000ull;   // generous: the emulated threads share few host cores
+    p.flags = 0;
+    p.gamma = gamma;
+    p.beta = beta;
+    p.eps = eps;
+    emu::errors = 0;
+    emu::reset_named();
+    if (ln)
+        emu::run_grid((int)U, kThreads, smem, [&] { mlp_tc_kernel<true>(mQ, mK, mV, p); });
+    else
+        emu::run_grid((int)U, kThreads, smem, [&] { mlp_tc_kernel<false>(mQ, mK, mV, p); });
+    emu::reset_named();
+    return emu::errors.load();
+}

@@ -16,8 +16,9 @@ outer-loop backward that reads them (fp32 CUDA cores); the TTT-Linear pair
 on mma.sync (bf16, d = 64, b = 16) -- already verified on the B200, which
 pins the emulated ldmatrix / mma semantics; and the LN+residual pair on
 mma.sync; the TTT-MLP training pair on mma.sync; the fused prologue on fp32
-CUDA cores and on tcgen05; and the TTT-Linear tensor-core prefill (tcgen05,
-already verified on the B200, which pins the emulated tcgen05 semantics) (paper digest
+CUDA cores and on tcgen05; and the TTT-Linear and TTT-MLP tensor-core
+prefills (tcgen05, already verified on the B200, which pin the emulated
+tcgen05 semantics) (paper digest
 "论文速览 | TTT", sections 3.3, 3.4, 3.6, 3.7, 4.4, 4.6, 6.12).
 """
 import ctypes
@@ -568,3 +569,59 @@ def test_linear_prefill_on_tcgen05(lfr_emu, ln, upc, B, H, T, per_token):
     assert normwise(WL.bf16_bits_to_f64(Z), Zr) < 2e-2
     assert normwise(W_out.astype(np.float64), Wr) < 2e-2
     assert normwise(W_out.astype(np.float64) - W0b, Wr - W0b) < 2e-2
+
+
+@pytest.fixture(scope="module")
+def mtc_emu(tmp_path_factory):
+    so = str(tmp_path_factory.mktemp("mtc") / "tc_mlp_emu.so")
+    subprocess.run(["g++", "-std=c++20", "-O1", "-fPIC", "-shared", "-I/usr/local/cuda/include", "-o", so,
+                    os.path.join(ROOT, "tests", "emulation", "tc_mlp_emu.cpp"), "-lpthread"], check=True)
+    return ctypes.CDLL(so)
+
+
+@pytest.mark.parametrize("ln,B,H,T,per_token,biases,per_seq", [
+    (False, 1, 1, 32, True, True, False), (True, 1, 1, 32, True, True, False), (False, 2, 1, 48, False, True, False),
+    (True, 1, 2, 48, True, False, False), (False, 1, 1, 16, True, True, False), (False, 2, 1, 32, True, True, True)])
+def test_mlp_prefill_on_tcgen05(mtc_emu, ln, B, H, T, per_token, biases, per_seq):
+    """The TTT-MLP tensor-core prefill (B200-verified) under the emulated
+    tcgen05 operations.  Its agreement with the oracle pins the emulation of
+    the M = 64 accumulator layout (rows in lanes 0-15 of each quadrant), the
+    MN-major A operand, the 16x128b TMEM store, the 16x256b x1 load and the x2
+    ldmatrix / stmatrix forms.  Each parameter's update (final minus initial)
+    is compared on its own."""
+    d, b, m = 64, 16, 256
+    inp = WL.random_case("mlp", B, H, T, d, b, io_dtype=WL.BF16, eta_mode="sigmoid" if per_token else "const",
+                         eta_const=0.0 if per_token else 0.05, seed=11 + T + B)
+    raw, ex = inp.raw, inp.exact
+    rng = np.random.default_rng(5 + T)
+    lead = (B, H) if per_seq else (H,)
+    if per_seq:
+        W1 = (raw["W1"][None] + 0.01 * rng.standard_normal((B,) + raw["W1"].shape)).astype(np.float32)
+        W2 = (raw["W2"][None] + 0.01 * rng.standard_normal((B,) + raw["W2"].shape)).astype(np.float32)
+    else:
+        W1, W2 = raw["W1"], raw["W2"]
+    c1 = (rng.standard_normal(lead + (m,)) * 0.1).astype(np.float32) if biases else np.zeros(lead + (m,), np.float32)
+    c2 = (rng.standard_normal(lead + (d,)) * 0.1).astype(np.float32) if biases else np.zeros(lead + (d,), np.float32)
+    gam = (1 + 0.1 * rng.standard_normal((H, d))).astype(np.float32)
+    bet = (0.1 * rng.standard_normal((H, d))).astype(np.float32)
+    Z = np.zeros((B, H, T, d), np.uint16)
+    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    status = np.zeros(1, np.int32)
+    eta = raw["eta"] if per_token else None
+    f = mtc_emu.emu_mlp_tc
+    f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
+        [ctypes.c_float] + [ctypes.c_void_p] * 6
+    rc = f(int(ln), B, H, T, int(per_seq), _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta),
+           np.float32(inp.w.eta_const), _p(W1), _p(c1), _p(W2), _p(c2), _p(gam) if ln else None,
+           _p(bet) if ln else None, np.float32(1e-6), _p(Z), *[_p(o) for o in outs], _p(status))
+    assert rc == 0 and status[0] == 0
+    eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(inp.w.eta_const)))
+    f64 = lambda a: a.astype(np.float64)
+    ref = O.mlp_forward(ex["Q"], ex["K"], ex["V"], eta_e, f64(W1), f64(c1), f64(W2), f64(c2), b, use_ln=ln,
+                        gamma=f64(gam), beta=f64(bet), eps=1e-6)
+    assert normwise(WL.bf16_bits_to_f64(Z), ref[0]) < 2e-2
+    for nm, got, want, init in zip(("W1", "c1", "W2", "c2"), outs, ref[1:], (W1, c1, W2, c2)):
+        i0 = np.broadcast_to(f64(init), want.shape)
+        assert normwise(f64(got), want) < 2e-2, nm
+        if biases or nm[0] == "W":
+            assert normwise(f64(got) - i0, want - i0) < 2e-2, (nm, normwise(f64(got) - i0, want - i0))
