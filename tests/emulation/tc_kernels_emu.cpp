@@ -11,6 +11,15 @@ alignas(1024) uint8_t smem[4 * 65536];
 
 #include "../../test_sequence_layers_head_b200/csrc/prologue.cuh"
 
+// test knobs: launch flags and the wait limit of the next run (the stall hook
+// TTT_FLAG_TEST_STALL makes the MMA issuer wait on a barrier nothing arrives on)
+static unsigned g_flags = 0;
+static unsigned long long g_wait_ns = 120ull * 1000000000ull;   // generous: the emulated threads share few host cores
+extern "C" void emu_prologue_tc_knobs(unsigned flags, unsigned long long wait_ns) {
+    g_flags = flags;
+    g_wait_ns = wait_ns;
+}
+
 // the fused prologue on tcgen05 with the library's tile plan and tensor maps, on `grid` persistent CTAs;
 // returns the number of emulated-hardware rule violations (0 when none), or -1 for a bad request
 extern "C" int emu_prologue_tc(int B, int T, int Dm, int H, int d, const void* x, const void* tq, const void* tk,
@@ -27,8 +36,8 @@ extern "C" int emu_prologue_tc(int B, int T, int Dm, int H, int d, const void* x
     p.eta = eta;
     p.eta_base = eta_base;
     p.status = status;
-    p.wait_ns = 120ull * 1000000000ull;   // generous: the emulated threads share few host cores
-    p.flags = 0;
+    p.wait_ns = g_wait_ns;
+    p.flags = g_flags;
     const unsigned long long pitch = (unsigned long long)Dm * 2;
     CUtensorMap mX, mTq, mTk, mTv, mTl;
     emu::make_map(&mX, x, Dm, rows, pitch, kBK, kBM, 2);

@@ -14,6 +14,15 @@ alignas(1024) uint8_t smem[128 * 1024];
 
 #include "../../test_sequence_layers_head_b200/csrc/linear_frag.cuh"
 
+// test knobs: launch flags and the wait limit of the next run (the stall hook
+// TTT_FLAG_TEST_STALL makes the MMA issuer wait on a barrier nothing arrives on)
+static unsigned g_flags = 0;
+static unsigned long long g_wait_ns = 120ull * 1000000000ull;   // generous: the emulated threads share few host cores
+extern "C" void emu_linear_tc_knobs(unsigned flags, unsigned long long wait_ns) {
+    g_flags = flags;
+    g_wait_ns = wait_ns;
+}
+
 // The TTT-Linear prefill (plain or LN+residual) with the library's tensor maps,
 // parameters and grid; upc = units per CTA (1 or 2).  Returns the number of
 // emulated-hardware rule violations (0 when none), or -1 for a bad request.
@@ -49,8 +58,8 @@ extern "C" int emu_linear_tc(int ln, int upc, int B, int H, int T, const void* Q
     p.W_out = W_out;
     p.c_out = c_out;
     p.status = status;
-    p.wait_ns = 120ull * 1000000000ull;   // generous: the emulated threads share few host cores
-    p.flags = 0;
+    p.wait_ns = g_wait_ns;
+    p.flags = g_flags;
     emu::errors = 0;
     emu::reset_named();
     const int grid = upc == 1 ? (int)U : (int)((U + 1) / 2);

@@ -14,6 +14,15 @@ alignas(1024) uint8_t smem[160 * 1024];
 
 #include "../../test_sequence_layers_head_b200/csrc/mlp_tc.cuh"
 
+// test knobs: launch flags and the wait limit of the next run (the stall hook
+// TTT_FLAG_TEST_STALL makes the MMA issuer wait on a barrier nothing arrives on)
+static unsigned g_flags = 0;
+static unsigned long long g_wait_ns = 120ull * 1000000000ull;   // generous: the emulated threads share few host cores
+extern "C" void emu_mlp_tc_knobs(unsigned flags, unsigned long long wait_ns) {
+    g_flags = flags;
+    g_wait_ns = wait_ns;
+}
+
 // The TTT-MLP prefill (plain or LN+residual on the output layer) with the
 // library's tensor maps, parameters and grid (one unit per CTA).  Returns the
 // number of emulated-hardware rule violations (0 when none), or -1 for a bad
@@ -46,8 +55,8 @@ extern "C" int emu_mlp_tc(int ln, int B, int H, int T, int per_seq, const void* 
     p.W2_out = W2_out;
     p.c2_out = c2_out;
     p.status = status;
-    p.wait_ns = 240ull * 1000000000ull;   // generous: the emulated threads share few host cores
-    p.flags = 0;
+    p.wait_ns = g_wait_ns;
+    p.flags = g_flags;
     p.gamma = gamma;
     p.beta = beta;
     p.eps = eps;

@@ -625,3 +625,70 @@ def test_mlp_prefill_on_tcgen05(mtc_emu, ln, B, H, T, per_token, biases, per_seq
         assert normwise(f64(got), want) < 2e-2, nm
         if biases or nm[0] == "W":
             assert normwise(f64(got) - i0, want - i0) < 2e-2, (nm, normwise(f64(got) - i0, want - i0))
+
+
+@pytest.mark.parametrize("kind", ["prologue", "linear", "linear_one_unit", "mlp", "mlp_ln"])
+def test_tcgen05_stall_hook_times_out_and_every_thread_exits(tc_emu, lfr_emu, mtc_emu, kind):
+    """The stall hook (the MMA issuer waits on a barrier nothing arrives on)
+    with a 20 ms wait limit: the run returns, with kStatusTimeout recorded and
+    no emulated-hardware rule broken, so every wait of the kernel's other
+    roles ends once the abort flag is up and every thread reaches the end
+    (a wait that never ended would hang this test).  The same path runs on the
+    B200 in the tests marked gpu."""
+    stall, limit = 0x100, 20_000_000
+    status = np.zeros(1, np.int32)
+    if kind == "prologue":
+        B, T, Dm, H, d = 2, 200, 136, 5, 64
+        w, inp = WL.prologue_case(B, T, Dm, H, d, gate=True, eta_base=0.5)
+        r = inp["raw"]
+        Q, K, V = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
+        eta = np.zeros((B, H, T), np.float32)
+        tc_emu.emu_prologue_tc_knobs.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
+        tc_emu.emu_prologue_tc_knobs(stall, limit)
+        f = tc_emu.emu_prologue_tc
+        f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 4 + \
+            [ctypes.c_int, ctypes.c_void_p]
+        try:
+            rc = f(B, T, Dm, H, d, _p(r["x"]), _p(r["theta_q"]), _p(r["theta_k"]), _p(r["theta_v"]),
+                   _p(r["theta_lr"]), 0.5, _p(Q), _p(K), _p(V), _p(eta), 3, _p(status))
+        finally:
+            tc_emu.emu_prologue_tc_knobs(0, 120_000_000_000)
+    elif kind.startswith("linear"):
+        B, H, T, d = 1, 3, 64, 64
+        inp = WL.random_case("linear", B, H, T, d, 16, io_dtype=WL.BF16, eta_mode="sigmoid", seed=9)
+        raw = inp.raw
+        Z = np.zeros((B, H, T, d), np.uint16)
+        W_out = np.zeros((B, H, d, d), np.float32)
+        lfr_emu.emu_linear_tc_knobs.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
+        lfr_emu.emu_linear_tc_knobs(stall, limit)
+        f = lfr_emu.emu_linear_tc
+        f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + \
+            [ctypes.c_float, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p,
+             ctypes.c_void_p, ctypes.c_float] + [ctypes.c_void_p] * 4
+        try:
+            rc = f(0, 1 if kind.endswith("one_unit") else 2, B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]),
+                   _p(raw["eta"]), 0.0, _p(raw["W0"]), 0, None, 0, None, None, 0.0, _p(Z), _p(W_out), None,
+                   _p(status))
+        finally:
+            lfr_emu.emu_linear_tc_knobs(0, 120_000_000_000)
+    else:
+        B, H, T, d, m = 1, 2, 48, 64, 256
+        inp = WL.random_case("mlp", B, H, T, d, 16, io_dtype=WL.BF16, eta_mode="sigmoid", seed=9)
+        raw = inp.raw
+        gam, bet = np.ones((H, d), np.float32), np.zeros((H, d), np.float32)
+        Z = np.zeros((B, H, T, d), np.uint16)
+        outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+        mtc_emu.emu_mlp_tc_knobs.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
+        mtc_emu.emu_mlp_tc_knobs(stall, limit)
+        f = mtc_emu.emu_mlp_tc
+        f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
+            [ctypes.c_float] + [ctypes.c_void_p] * 6
+        ln = kind == "mlp_ln"
+        try:
+            rc = f(int(ln), B, H, T, 0, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(raw["eta"]), 0.0,
+                   _p(raw["W1"]), _p(raw["c1"]), _p(raw["W2"]), _p(raw["c2"]), _p(gam) if ln else None,
+                   _p(bet) if ln else None, np.float32(1e-6), _p(Z), *[_p(o) for o in outs], _p(status))
+        finally:
+            mtc_emu.emu_mlp_tc_knobs(0, 120_000_000_000)
+    assert rc == 0
+    assert status[0] & 1
