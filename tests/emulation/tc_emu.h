@@ -20,12 +20,16 @@
 //     quadrant (warp % 4) only.
 //   tcgen05.commit: arrives once on the mbarrier when the MMAs issued before it
 //     have completed.
-// Asynchronous operations complete when they are issued: one of the schedules
-// the hardware may produce, which a correct kernel must handle.
+// Asynchronous operations complete when they are issued (one of the schedules
+// the hardware may produce, which a correct kernel must handle), or, in the
+// deferred mode (emu::deferred), later, on an engine thread (see Engine).
 #pragma once
 #include <atomic>
 #include <chrono>
+#include <condition_variable>
 #include <cuda.h>
+#include <deque>
+#include <functional>
 #include <map>
 #include <mutex>
 #include <thread>
@@ -79,6 +83,82 @@ inline void bar_complete_tx(const void* bar, long long bytes) {
 }
 inline uint32_t tmem_lane(uint32_t a) { return a >> 16; }
 inline uint32_t tmem_col(uint32_t a) { return a & 0xFFFFu; }
+
+// Deferred completion (off by default): TMA and bulk loads, MMAs and commits
+// go to two FIFOs that one engine thread works through, each job after a
+// pause: loads first (they may overtake MMAs: the copy engine and the tensor
+// core are separate units), MMAs and commits in issue order, as tcgen05
+// guarantees for one issuing thread, so a commit arrives once the MMAs before
+// it have run.  A kernel that touches a buffer before the wait that orders
+// it, or reuses one too early, then sees stale or overwritten data.
+// pending_stores counts each thread's TMA stores not yet done.
+struct Engine {
+    std::mutex mu;
+    std::condition_variable cv;
+    std::deque<std::function<void()>> q[2];   // 0: loads, 1: MMAs and commits
+    std::thread th;
+    bool started = false, quit = false;
+    std::atomic<long> inflight{0};
+    void run() {
+        for (;;) {
+            std::function<void()> job;
+            {
+                std::unique_lock<std::mutex> lk(mu);
+                cv.wait(lk, [&] { return !q[0].empty() || !q[1].empty() || quit; });
+                if (q[0].empty() && q[1].empty()) return;
+                auto& src = q[0].empty() ? q[1] : q[0];
+                job = std::move(src.front());
+                src.pop_front();
+            }
+            std::this_thread::sleep_for(std::chrono::microseconds(30));
+            job();
+            --inflight;
+        }
+    }
+    void push(std::function<void()> job, int kind) {
+        std::lock_guard<std::mutex> lk(mu);
+        if (!started) {
+            quit = false;
+            th = std::thread([this] { run(); });
+            started = true;
+        }
+        ++inflight;
+        q[kind].push_back(std::move(job));
+        cv.notify_one();
+    }
+    // wait for the queues to empty, then end the engine thread (a harness call's last step, so that no
+    // thread waits on the condition variable when the library is unloaded)
+    void finish() {
+        while (inflight.load() != 0) std::this_thread::yield();
+        {
+            std::lock_guard<std::mutex> lk(mu);
+            if (!started) return;
+            quit = true;
+        }
+        cv.notify_all();
+        th.join();
+        started = false;
+    }
+};
+inline Engine engine;
+inline std::atomic<bool> deferred{false};
+inline std::atomic<int> pending_stores[kMaxThreads];
+// In the deferred mode a TMA store is held until its thread waits for it
+// (cp.async.bulk.wait_group), the latest point at which it may read shared
+// memory; a store never waited for is done when the run ends, after later
+// CTAs have reused the shared memory.
+inline std::vector<std::function<void()>> held_stores[kMaxThreads];
+inline void flush_stores(int tid) {
+    for (auto& job : held_stores[tid]) job();
+    held_stores[tid].clear();
+}
+enum { kLoad = 0, kMma = 1 };
+inline void async_do(std::function<void()> job, int kind) {
+    if (deferred.load())
+        engine.push(std::move(job), kind);
+    else
+        job();
+}
 }  // namespace emu
 
 #undef __grid_constant__
@@ -129,16 +209,18 @@ inline void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_
     uint8_t* d = static_cast<uint8_t*>(dst);
     const unsigned rowb = f.box_cols * f.elem;
     if (((uintptr_t)(d - emu::shared_base)) % 1024 != 0 || rowb != 128 || (x * f.elem) % 16 != 0) ++emu::errors;
-    for (unsigned r = 0; r < f.box_rows; ++r)
-        for (unsigned cb = 0; cb < rowb; ++cb) {
-            const long long gx = (long long)x + cb / f.elem, gy = (long long)y + r;
-            uint8_t v = 0;
-            if (gx >= 0 && gy >= 0 && (unsigned long long)gx < f.cols && (unsigned long long)gy < f.rows)
-                v = static_cast<const uint8_t*>(f.base)[gy * f.pitch + gx * f.elem + cb % f.elem];
-            const unsigned chunk = (cb >> 4) ^ (r & 7);
-            d[r * 128 + chunk * 16 + (cb & 15)] = v;
-        }
-    emu::bar_complete_tx(bar, (long long)rowb * f.box_rows);
+    emu::async_do([=] {
+        for (unsigned r = 0; r < f.box_rows; ++r)
+            for (unsigned cb = 0; cb < rowb; ++cb) {
+                const long long gx = (long long)x + cb / f.elem, gy = (long long)y + r;
+                uint8_t v = 0;
+                if (gx >= 0 && gy >= 0 && (unsigned long long)gx < f.cols && (unsigned long long)gy < f.rows)
+                    v = static_cast<const uint8_t*>(f.base)[gy * f.pitch + gx * f.elem + cb % f.elem];
+                const unsigned chunk = (cb >> 4) ^ (r & 7);
+                d[r * 128 + chunk * 16 + (cb & 15)] = v;
+            }
+        emu::bar_complete_tx(bar, (long long)rowb * f.box_rows);
+    }, emu::kLoad);
 }
 inline void tmem_alloc(uint32_t* dst, uint32_t) { *dst = 0; }
 inline void tmem_relinquish() {}
@@ -213,15 +295,19 @@ inline void umma_apply(uint32_t d_tmem, uint32_t idesc, uint32_t accumulate, FA 
     }
 }
 inline void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
-    const bool a_mn = (idesc >> 15) & 1u, b_mn = (idesc >> 16) & 1u;
-    umma_apply(
-        d_tmem, idesc, accumulate, [&](int row, int k) { return operand_elem(adesc, a_mn, row, k); },
-        [&](int col, int k) { return operand_elem(bdesc, b_mn, col, k); });
+    emu::async_do([=] {
+        const bool a_mn = (idesc >> 15) & 1u, b_mn = (idesc >> 16) & 1u;
+        umma_apply(
+            d_tmem, idesc, accumulate, [&](int row, int k) { return operand_elem(adesc, a_mn, row, k); },
+            [&](int col, int k) { return operand_elem(bdesc, b_mn, col, k); });
+    }, emu::kMma);
 }
 // A in tensor memory: element (row, k) at lane (lane + row), column (col + k / 2), the low half for even k
 inline float tmem_bf16(uint32_t a_tmem, int row, int k) {
     const uint32_t v = emu::tmem[(emu::tmem_lane(a_tmem) + row) & 127][(emu::tmem_col(a_tmem) + k / 2) & 511];
     return (k & 1) ? emu::bf16_hi(v) : emu::bf16_lo(v);
 }
-inline void umma_commit(uint64_t* bar) { emu::bar_arrive(bar, 0); }
+inline void umma_commit(uint64_t* bar) {
+    emu::async_do([=] { emu::bar_arrive(bar, 0); }, emu::kMma);
+}
 }  // namespace ttt

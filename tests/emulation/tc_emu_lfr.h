@@ -18,7 +18,8 @@
 //     shared byte lin = r * rowbytes + b of the box is read at
 //     lin ^ (((lin >> 7) & mask) << 4) (mask 1, 3, 7); rows outside the tensor
 //     are not written.
-// As in tc_emu.h, asynchronous operations complete when they are issued.
+// As in tc_emu.h, asynchronous operations complete when they are issued, or,
+// in the deferred mode, later on the engine thread.
 #pragma once
 #include "tc_emu.h"
 
@@ -80,14 +81,23 @@ inline void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
     if ((emu::shared_base && ((static_cast<uint8_t*>(dst) - emu::shared_base) % 16)) || bytes % 16 ||
         (reinterpret_cast<uintptr_t>(src) % 16))
         ++emu::errors;
-    std::memcpy(dst, src, bytes);
-    emu::bar_complete_tx(bar, bytes);
+    emu::async_do([=] {
+        std::memcpy(dst, src, bytes);
+        emu::bar_complete_tx(bar, bytes);
+    }, emu::kLoad);
 }
 inline void bulk_commit() {}
+// every store of this thread issued so far (one store per group in these kernels, so N = 0 only)
 template <int N>
-inline void bulk_wait_read() {}
+inline void bulk_wait_read() {
+    static_assert(N == 0, "one store per group");
+    emu::flush_stores(threadIdx.x);
+    while (emu::pending_stores[threadIdx.x].load() != 0) std::this_thread::yield();
+}
 template <int N>
-inline void bulk_wait() {}
+inline void bulk_wait() {
+    bulk_wait_read<N>();
+}
 inline void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
     emu::FakeMap f;
     std::memcpy(&f, map, sizeof(f));
@@ -98,14 +108,23 @@ inline void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) 
     if ((unsigned)span != rowb || ((s - emu::shared_base) % (8 * span)) != 0 || x < 0 || y < 0 ||
         (x * f.elem) % 16 != 0)
         ++emu::errors;
-    for (unsigned r = 0; r < f.box_rows; ++r)
-        for (unsigned b = 0; b < rowb; ++b) {
-            const unsigned long long gx = (unsigned long long)x + b / f.elem, gy = (unsigned long long)y + r;
-            if (gx >= f.cols || gy >= f.rows) continue;
-            const uint32_t lin = r * rowb + b;
-            const uint32_t phys = lin ^ (((lin >> 7) & mask) << 4);
-            static_cast<uint8_t*>(const_cast<void*>(f.base))[gy * f.pitch + gx * f.elem + b % f.elem] = s[phys];
-        }
+    std::atomic<int>* pend = &emu::pending_stores[threadIdx.x];
+    ++*pend;
+    auto job = [=] {
+        for (unsigned r = 0; r < f.box_rows; ++r)
+            for (unsigned b = 0; b < rowb; ++b) {
+                const unsigned long long gx = (unsigned long long)x + b / f.elem, gy = (unsigned long long)y + r;
+                if (gx >= f.cols || gy >= f.rows) continue;
+                const uint32_t lin = r * rowb + b;
+                const uint32_t phys = lin ^ (((lin >> 7) & mask) << 4);
+                static_cast<uint8_t*>(const_cast<void*>(f.base))[gy * f.pitch + gx * f.elem + b % f.elem] = s[phys];
+            }
+        --*pend;
+    };
+    if (emu::deferred.load())
+        emu::held_stores[threadIdx.x].push_back(job);
+    else
+        job();
 }
 
 namespace tcc {
@@ -116,9 +135,11 @@ inline void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t* r) { emu::tmem_st
 inline void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
     const bool b_mn = (idesc >> 16) & 1u;
     if ((idesc >> 15) & 1u) ++emu::errors;   // an A in tensor memory is K-major
-    umma_apply(
-        d_tmem, idesc, accumulate, [&](int row, int k) { return tmem_bf16(a_tmem, row, k); },
-        [&](int col, int k) { return operand_elem(bdesc, b_mn, col, k); });
+    emu::async_do([=] {
+        umma_apply(
+            d_tmem, idesc, accumulate, [&](int row, int k) { return tmem_bf16(a_tmem, row, k); },
+            [&](int col, int k) { return operand_elem(bdesc, b_mn, col, k); });
+    }, emu::kMma);
 }
 }  // namespace tcc
 

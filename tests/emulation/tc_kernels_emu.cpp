@@ -19,6 +19,8 @@ extern "C" void emu_prologue_tc_knobs(unsigned flags, unsigned long long wait_ns
     g_flags = flags;
     g_wait_ns = wait_ns;
 }
+// deferred completion of the asynchronous operations (tc_emu.h, Engine) for the next runs
+extern "C" void emu_deferred(int on) { emu::deferred = on != 0; }
 
 // the fused prologue on tcgen05 with the library's tile plan and tensor maps, on `grid` persistent CTAs;
 // returns the number of emulated-hardware rule violations (0 when none), or -1 for a bad request
@@ -52,5 +54,7 @@ extern "C" int emu_prologue_tc(int B, int T, int Dm, int H, int d, const void* x
     emu::errors = 0;
     // a persistent CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...: gridDim must be the grid
     emu::run_grid(g, kThreads, smem, [&] { prologue_kernel(mX, mTq, mTk, mTv, mTl, p); });
+    emu::engine.finish();
+    for (int t = 0; t < emu::kMaxThreads; ++t) emu::flush_stores(t);
     return emu::errors.load();
 }

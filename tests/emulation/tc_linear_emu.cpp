@@ -22,6 +22,8 @@ extern "C" void emu_linear_tc_knobs(unsigned flags, unsigned long long wait_ns) 
     g_flags = flags;
     g_wait_ns = wait_ns;
 }
+// deferred completion of the asynchronous operations (tc_emu.h, Engine) for the next runs
+extern "C" void emu_deferred(int on) { emu::deferred = on != 0; }
 
 // The TTT-Linear prefill (plain or LN+residual) with the library's tensor maps,
 // parameters and grid; upc = units per CTA (1 or 2).  Returns the number of
@@ -75,5 +77,7 @@ extern "C" int emu_linear_tc(int ln, int upc, int B, int H, int T, const void* Q
             emu::run_grid(grid, kThreads, smem, [&] { linear_frag_kernel<false, 2>(mQ, mK, mV, mZ, mZ1, p); });
     }
     emu::reset_named();
+    emu::engine.finish();
+    for (int t = 0; t < emu::kMaxThreads; ++t) emu::flush_stores(t);
     return emu::errors.load();
 }

@@ -22,6 +22,8 @@ extern "C" void emu_mlp_tc_knobs(unsigned flags, unsigned long long wait_ns) {
     g_flags = flags;
     g_wait_ns = wait_ns;
 }
+// deferred completion of the asynchronous operations (tc_emu.h, Engine) for the next runs
+extern "C" void emu_deferred(int on) { emu::deferred = on != 0; }
 
 // The TTT-MLP prefill (plain or LN+residual on the output layer) with the
 // library's tensor maps, parameters and grid (one unit per CTA).  Returns the
@@ -67,5 +69,7 @@ extern "C" int emu_mlp_tc(int ln, int B, int H, int T, int per_seq, const void* 
     else
         emu::run_grid((int)U, kThreads, smem, [&] { mlp_tc_kernel<false>(mQ, mK, mV, p); });
     emu::reset_named();
+    emu::engine.finish();
+    for (int t = 0; t < emu::kMaxThreads; ++t) emu::flush_stores(t);
     return emu::errors.load();
 }

@@ -346,10 +346,13 @@ def tc_emu(tmp_path_factory):
     (4, 33, 16, 7, 32, True, 1),       # width below one chunk
     (2, 64, 768, 12, 64, True, 7),     # the 12-head width
 ])
-def test_prologue_on_tcgen05(tc_emu, B, T, Dm, H, d, gate, grid):
+@pytest.mark.parametrize("deferred", [False, True])
+def test_prologue_on_tcgen05(tc_emu, B, T, Dm, H, d, gate, grid, deferred):
     """The tcgen05 prologue kernel with the library's tile plan and tensor maps: every output written, the
     views within one bf16 rounding plus the fp32 accumulation bound, the gate within its bound, no
-    emulated-hardware rule broken (TMA alignment, TMEM lane quadrant, MMA shape), no expired wait."""
+    emulated-hardware rule broken (TMA alignment, TMEM lane quadrant, MMA shape), no expired wait.  With
+    `deferred`, the asynchronous operations complete late (loads overtaking MMAs, stores held until
+    waited for): a missing or misplaced wait then shows as wrong data."""
     w, inp = WL.prologue_case(B, T, Dm, H, d, gate=gate, eta_base=0.5)
     r, e = inp["raw"], inp["exact"]
     Q, K, V = (np.full((B, H, T, d), 0x7FC0, np.uint16) for _ in range(3))   # NaN until written
@@ -358,8 +361,12 @@ def test_prologue_on_tcgen05(tc_emu, B, T, Dm, H, d, gate, grid):
     f = tc_emu.emu_prologue_tc
     f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 4 + \
         [ctypes.c_int, ctypes.c_void_p]
-    rc = f(B, T, Dm, H, d, _p(r["x"]), _p(r["theta_q"]), _p(r["theta_k"]), _p(r["theta_v"]),
-           _p(r["theta_lr"]) if gate else None, 0.5, _p(Q), _p(K), _p(V), _p(eta), grid, _p(status))
+    tc_emu.emu_deferred(int(deferred))
+    try:
+        rc = f(B, T, Dm, H, d, _p(r["x"]), _p(r["theta_q"]), _p(r["theta_k"]), _p(r["theta_v"]),
+               _p(r["theta_lr"]) if gate else None, 0.5, _p(Q), _p(K), _p(V), _p(eta), grid, _p(status))
+    finally:
+        tc_emu.emu_deferred(0)
     assert rc == 0 and status[0] == 0
     ref = O.qkv_prologue(e["x"], e["theta_q"], e["theta_k"], e["theta_v"], e["theta_lr"], 0.5, d)
     for got, want, nm in zip((Q, K, V), ref[:3], ("theta_q", "theta_k", "theta_v")):
@@ -527,14 +534,15 @@ def lfr_emu(tmp_path_factory):
 @pytest.mark.parametrize("ln,upc,B,H,T,per_token", [
     (False, 2, 1, 2, 64, True), (False, 1, 1, 1, 48, False), (False, 2, 1, 3, 80, True),
     (True, 2, 1, 2, 64, True), (True, 1, 2, 1, 48, False), (True, 2, 1, 3, 48, True)])
-def test_linear_prefill_on_tcgen05(lfr_emu, ln, upc, B, H, T, per_token):
+@pytest.mark.parametrize("deferred", [False, True])
+def test_linear_prefill_on_tcgen05(lfr_emu, ln, upc, B, H, T, per_token, deferred):
     """The TTT-Linear tensor-core prefill (B200-verified) under the emulated
     tcgen05 operations.  Its agreement with the oracle pins the emulation of
     the MMA operand descriptors (K-major and MN-major 128-byte swizzle, K-major
     without swizzle, A in tensor memory), the 32x32b TMEM loads and stores, the
     accumulator layout of the 16x256b load, stmatrix.trans and the 32- and
     64-byte swizzled TMA stores.  The state update W_T - W_0 is compared on its
-    own: the full state is dominated by W_0."""
+    own: the full state is dominated by W_0.  `deferred` as in the prologue's test."""
     d, b = 64, 16
     inp = WL.random_case("ln" if ln else "linear", B, H, T, d, b, io_dtype=WL.BF16,
                          eta_mode="sigmoid" if per_token else "const", eta_const=0.0 if per_token else 0.05,
@@ -552,9 +560,14 @@ def test_linear_prefill_on_tcgen05(lfr_emu, ln, upc, B, H, T, per_token):
                                                                 ctypes.c_void_p, ctypes.c_longlong, ctypes.c_void_p,
                                                                 ctypes.c_void_p, ctypes.c_float] + \
         [ctypes.c_void_p] * 4
-    rc = f(int(ln), upc, B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const),
-           _p(raw["W0"]), 0, _p(c0), 0, _p(raw["gamma"]) if ln else None, _p(raw["beta"]) if ln else None,
-           np.float32(inp.w.ln_eps if ln else 0.0), _p(Z), _p(W_out), _p(c_out), _p(status))
+    lfr_emu.emu_deferred(int(deferred))
+    try:
+        rc = f(int(ln), upc, B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta),
+               np.float32(inp.w.eta_const), _p(raw["W0"]), 0, _p(c0), 0, _p(raw["gamma"]) if ln else None,
+               _p(raw["beta"]) if ln else None, np.float32(inp.w.ln_eps if ln else 0.0), _p(Z), _p(W_out), _p(c_out),
+               _p(status))
+    finally:
+        lfr_emu.emu_deferred(0)
     assert rc == 0 and status[0] == 0
     eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(inp.w.eta_const)))
     if ln:
@@ -582,13 +595,14 @@ def mtc_emu(tmp_path_factory):
 @pytest.mark.parametrize("ln,B,H,T,per_token,biases,per_seq", [
     (False, 1, 1, 32, True, True, False), (True, 1, 1, 32, True, True, False), (False, 2, 1, 48, False, True, False),
     (True, 1, 2, 48, True, False, False), (False, 1, 1, 16, True, True, False), (False, 2, 1, 32, True, True, True)])
-def test_mlp_prefill_on_tcgen05(mtc_emu, ln, B, H, T, per_token, biases, per_seq):
+@pytest.mark.parametrize("deferred", [False, True])
+def test_mlp_prefill_on_tcgen05(mtc_emu, ln, B, H, T, per_token, biases, per_seq, deferred):
     """The TTT-MLP tensor-core prefill (B200-verified) under the emulated
     tcgen05 operations.  Its agreement with the oracle pins the emulation of
     the M = 64 accumulator layout (rows in lanes 0-15 of each quadrant), the
     MN-major A operand, the 16x128b TMEM store, the 16x256b x1 load and the x2
     ldmatrix / stmatrix forms.  Each parameter's update (final minus initial)
-    is compared on its own."""
+    is compared on its own.  `deferred` as in the prologue's test."""
     d, b, m = 64, 16, 256
     inp = WL.random_case("mlp", B, H, T, d, b, io_dtype=WL.BF16, eta_mode="sigmoid" if per_token else "const",
                          eta_const=0.0 if per_token else 0.05, seed=11 + T + B)
@@ -611,9 +625,13 @@ def test_mlp_prefill_on_tcgen05(mtc_emu, ln, B, H, T, per_token, biases, per_seq
     f = mtc_emu.emu_mlp_tc
     f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
         [ctypes.c_float] + [ctypes.c_void_p] * 6
-    rc = f(int(ln), B, H, T, int(per_seq), _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta),
-           np.float32(inp.w.eta_const), _p(W1), _p(c1), _p(W2), _p(c2), _p(gam) if ln else None,
-           _p(bet) if ln else None, np.float32(1e-6), _p(Z), *[_p(o) for o in outs], _p(status))
+    mtc_emu.emu_deferred(int(deferred))
+    try:
+        rc = f(int(ln), B, H, T, int(per_seq), _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta),
+               np.float32(inp.w.eta_const), _p(W1), _p(c1), _p(W2), _p(c2), _p(gam) if ln else None,
+               _p(bet) if ln else None, np.float32(1e-6), _p(Z), *[_p(o) for o in outs], _p(status))
+    finally:
+        mtc_emu.emu_deferred(0)
     assert rc == 0 and status[0] == 0
     eta_e = ex["eta"] if per_token else np.full((B, H, T), np.float64(np.float32(inp.w.eta_const)))
     f64 = lambda a: a.astype(np.float64)
