@@ -31,6 +31,7 @@
 #include <deque>
 #include <functional>
 #include <map>
+#include <vector>
 #include <mutex>
 #include <thread>
 
@@ -152,6 +153,33 @@ inline void flush_stores(int tid) {
     for (auto& job : held_stores[tid]) job();
     held_stores[tid].clear();
 }
+// Deferred tensor-memory loads and stores: a tcgen05.ld reads tensor memory
+// at issue, but its registers hold NaN until the thread's tcgen05.wait::ld; a
+// tcgen05.st reaches tensor memory at the thread's tcgen05.wait::st (a store
+// never waited for is lost).
+struct TmemLd {
+    uint32_t* dst;
+    std::vector<uint32_t> vals;
+};
+struct TmemSt {
+    uint32_t lane, col, val;
+};
+inline thread_local std::vector<TmemLd> pend_ld;
+inline thread_local std::vector<TmemSt> pend_st;
+inline void deliver(uint32_t* r, const uint32_t* vals, int n) {
+    if (deferred.load()) {
+        pend_ld.push_back({r, std::vector<uint32_t>(vals, vals + n)});
+        for (int i = 0; i < n; ++i) r[i] = 0x7FC00000u;
+    } else {
+        for (int i = 0; i < n; ++i) r[i] = vals[i];
+    }
+}
+inline void tmem_put(uint32_t lane, uint32_t col, uint32_t val) {
+    if (deferred.load())
+        pend_st.push_back({lane & 127, col & 511, val});
+    else
+        tmem[lane & 127][col & 511] = val;
+}
 enum { kLoad = 0, kMma = 1 };
 inline void async_do(std::function<void()> job, int kind) {
     if (deferred.load())
@@ -227,14 +255,22 @@ inline void tmem_relinquish() {}
 inline void tmem_dealloc(uint32_t, uint32_t) {}
 inline void tc_fence_before() {}
 inline void tc_fence_after() {}
-inline void tmem_wait_ld() {}
-inline void tmem_wait_st() {}
+inline void tmem_wait_ld() {
+    for (auto& l : emu::pend_ld) std::memcpy(l.dst, l.vals.data(), l.vals.size() * 4);
+    emu::pend_ld.clear();
+}
+inline void tmem_wait_st() {
+    for (auto& t : emu::pend_st) emu::tmem[t.lane][t.col] = t.val;
+    emu::pend_st.clear();
+}
 template <int N>
 inline void tmem_ld_32x32b(uint32_t taddr, uint32_t* r) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const uint32_t l0 = emu::tmem_lane(taddr), c0 = emu::tmem_col(taddr);
     if (l0 / 32 != (uint32_t)(w % 4) || l0 % 32 != 0 || c0 + N > 512) ++emu::errors;
-    for (int i = 0; i < N; ++i) r[i] = emu::tmem[(l0 + lane) & 127][(c0 + i) & 511];
+    uint32_t vals[N];
+    for (int i = 0; i < N; ++i) vals[i] = emu::tmem[(l0 + lane) & 127][(c0 + i) & 511];
+    emu::deliver(r, vals, N);
     emu::warp_sync();
 }
 inline void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t* r) { tmem_ld_32x32b<16>(taddr, r); }

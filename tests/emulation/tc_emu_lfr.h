@@ -19,7 +19,8 @@
 //     lin ^ (((lin >> 7) & mask) << 4) (mask 1, 3, 7); rows outside the tensor
 //     are not written.
 // As in tc_emu.h, asynchronous operations complete when they are issued, or,
-// in the deferred mode, later on the engine thread.
+// in the deferred mode, later (on the engine thread, or, for tensor-memory
+// loads and stores, at the thread's tcgen05.wait).
 #pragma once
 #include "tc_emu.h"
 
@@ -48,7 +49,7 @@ inline void tmem_st_32x32b(uint32_t taddr, const uint32_t* r) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const uint32_t l0 = tmem_lane(taddr), c0 = tmem_col(taddr);
     if (l0 / 32 != (uint32_t)(w % 4) || l0 % 32 != 0 || c0 + N > 512) ++errors;
-    for (int i = 0; i < N; ++i) tmem[(l0 + lane) & 127][(c0 + i) & 511] = r[i];
+    for (int i = 0; i < N; ++i) tmem_put(l0 + lane, c0 + i, r[i]);
     warp_sync();
 }
 }  // namespace emu
@@ -149,9 +150,11 @@ inline void tmem_ld_16x256b_x2(uint32_t taddr, uint32_t* r) {
     const uint32_t l0 = emu::tmem_lane(taddr), c0 = emu::tmem_col(taddr);
     if (l0 / 32 != (uint32_t)(w % 4) || l0 % 16 != 0 || c0 + 16 > 512) ++emu::errors;
     const int g = lane / 4, c = lane % 4;
+    uint32_t vals[8];
     for (int rep = 0; rep < 2; ++rep)
         for (int e = 0; e < 4; ++e)
-            r[4 * rep + e] = emu::tmem[(l0 + g + 8 * (e >> 1)) & 127][(c0 + 8 * rep + 2 * c + (e & 1)) & 511];
+            vals[4 * rep + e] = emu::tmem[(l0 + g + 8 * (e >> 1)) & 127][(c0 + 8 * rep + 2 * c + (e & 1)) & 511];
+    emu::deliver(r, vals, 8);
     emu::warp_sync();
 }
 inline void stsm_x4_t(uint32_t addr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {

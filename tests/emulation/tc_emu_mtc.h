@@ -69,7 +69,9 @@ inline void tmem_ld_16x256b_x1(uint32_t taddr, uint32_t* r) {
     const uint32_t l0 = emu::tmem_lane(taddr), c0 = emu::tmem_col(taddr);
     if (l0 / 32 != (uint32_t)(w % 4) || l0 % 16 != 0 || c0 + 8 > 512) ++emu::errors;
     const int g = lane / 4, c = lane % 4;
-    for (int e = 0; e < 4; ++e) r[e] = emu::tmem[(l0 + g + 8 * (e >> 1)) & 127][(c0 + 2 * c + (e & 1)) & 511];
+    uint32_t vals[4];
+    for (int e = 0; e < 4; ++e) vals[e] = emu::tmem[(l0 + g + 8 * (e >> 1)) & 127][(c0 + 2 * c + (e & 1)) & 511];
+    emu::deliver(r, vals, 4);
     emu::warp_sync();
 }
 inline void tmem_st_16x128b_x1(uint32_t taddr, uint32_t r0, uint32_t r1) {
@@ -77,8 +79,8 @@ inline void tmem_st_16x128b_x1(uint32_t taddr, uint32_t r0, uint32_t r1) {
     const uint32_t l0 = emu::tmem_lane(taddr), c0 = emu::tmem_col(taddr);
     if (l0 / 32 != (uint32_t)(w % 4) || l0 % 16 != 0 || c0 + 4 > 512) ++emu::errors;
     const int g = lane / 4, c = lane % 4;
-    emu::tmem[(l0 + g) & 127][(c0 + c) & 511] = r0;
-    emu::tmem[(l0 + g + 8) & 127][(c0 + c) & 511] = r1;
+    emu::tmem_put(l0 + g, c0 + c, r0);
+    emu::tmem_put(l0 + g + 8, c0 + c, r1);
     emu::warp_sync();
 }
 }  // namespace mtc

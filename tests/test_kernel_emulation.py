@@ -533,7 +533,8 @@ def lfr_emu(tmp_path_factory):
 
 @pytest.mark.parametrize("ln,upc,B,H,T,per_token", [
     (False, 2, 1, 2, 64, True), (False, 1, 1, 1, 48, False), (False, 2, 1, 3, 80, True),
-    (True, 2, 1, 2, 64, True), (True, 1, 2, 1, 48, False), (True, 2, 1, 3, 48, True)])
+    (True, 2, 1, 2, 64, True), (True, 1, 2, 1, 48, False), (True, 2, 1, 3, 48, True),
+    (False, 2, 1, 2, 256, False)])   # long enough that a stale state shows above the bar
 @pytest.mark.parametrize("deferred", [False, True])
 def test_linear_prefill_on_tcgen05(lfr_emu, ln, upc, B, H, T, per_token, deferred):
     """The TTT-Linear tensor-core prefill (B200-verified) under the emulated
