@@ -2,7 +2,8 @@
 // INFRASTRUCTURE, never part of the library (which has no CPU path).
 //
 // One CTA at a time.  Each CUDA thread of the CTA is a std::thread running
-// the kernel function; __syncthreads is a std::barrier over the CTA; a
+// the kernel function; __syncthreads is a barrier over the CTA (EBar: all
+// threads concurrent, or one at a time under the serial scheduler); a
 // warp-collective operation (shuffle, ldmatrix, mma) has every lane write its
 // operands to the warp's exchange area, waits on the warp's barrier, computes
 // its own result from all lanes' operands, and waits again before the area is
@@ -24,8 +25,11 @@
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
+#include <atomic>
 #include <barrier>
 #include <cmath>
+#include <condition_variable>
+#include <mutex>
 #include <cstdint>
 #include <cstring>
 #include <thread>
@@ -35,8 +39,104 @@ namespace emu {
 constexpr int kMaxThreads = 1024;
 inline thread_local uint3 tid3, bid3;
 inline uint3 grid3;
-inline std::barrier<>* block_bar = nullptr;
-inline std::barrier<>* warp_bar[kMaxThreads / 32];
+
+// Serial mode (off by default; 1: lowest thread first, 2: highest first).
+// One thread of the CTA runs at a time and hands the CPU on only where it
+// blocks (a barrier not yet complete, a warp collective) or spins (a wait on
+// an mbarrier or a store).  At a block the next thread is the ready one of
+// lowest (1) or highest (2) index, so the first warp runs as far as it can,
+// to its next block-wide barrier, before the others move; a spinning thread
+// hands on round-robin.  A read of data another thread writes without a
+// barrier between them, or a write into data others still read, then shows
+// as wrong data in one of the two orders.
+inline std::atomic<int> serial{0};
+struct Sched {
+    std::mutex m;
+    std::condition_variable cv[kMaxThreads];   // one per thread: a hand-off wakes only the new owner
+    int n = 0, owner = -1;
+    bool ready[kMaxThreads];
+    bool stuck = false;   // every live thread blocked on a barrier: the kernel would hang
+};
+inline Sched sched;
+// the ready thread of lowest (1) or highest (2) index, or -1 (lock held)
+inline int sched_next(int) {
+    const int n = sched.n;
+    for (int i = 0; i < n; ++i) {
+        const int t = serial.load() == 1 ? i : n - 1 - i;
+        if (sched.ready[t]) return t;
+    }
+    return -1;
+}
+// the next ready thread after `from`, round-robin (itself last), or -1 (lock held)
+inline int sched_next_rr(int from) {
+    const int n = sched.n;
+    for (int i = 1; i <= n; ++i) {
+        const int t = (from + i) % n;
+        if (sched.ready[t]) return t;
+    }
+    return -1;
+}
+// hand the CPU on (lock held) and wait until it comes back
+inline void sched_wake() {
+    if (sched.stuck)
+        for (int t = 0; t < sched.n; ++t) sched.cv[t].notify_all();
+    else if (sched.owner >= 0)
+        sched.cv[sched.owner].notify_all();
+}
+inline void sched_handoff(std::unique_lock<std::mutex>& lk, int tid, bool rr = false) {
+    sched.owner = rr ? sched_next_rr(tid) : sched_next(tid);
+    if (sched.owner < 0) sched.stuck = true;
+    if (sched.owner != tid) {
+        sched_wake();
+        sched.cv[tid].wait(lk, [&] { return sched.owner == tid || sched.stuck; });
+    }
+}
+// a spin-wait iteration: stay ready, let the others run first
+inline void spin_yield() {
+    if (!serial.load()) {
+        std::this_thread::yield();
+        return;
+    }
+    const int tid = (int)tid3.x;
+    std::unique_lock<std::mutex> lk(sched.m);
+    sched.ready[tid] = true;
+    sched_handoff(lk, tid, true);
+}
+
+// A barrier over `count` threads: std::barrier, or in the serial mode the
+// scheduler's own.
+struct EBar {
+    std::barrier<> b;
+    int count, arrived = 0;
+    long gen = 0;
+    explicit EBar(int c) : b(c), count(c) {}
+    void wait() {
+        if (!serial.load()) {
+            b.arrive_and_wait();
+            return;
+        }
+        const int tid = (int)tid3.x;
+        std::unique_lock<std::mutex> lk(sched.m);
+        if (++arrived == count) {
+            arrived = 0;
+            ++gen;
+            for (int t = 0; t < sched.n; ++t)
+                if (waiting_on[t] == this) {
+                    waiting_on[t] = nullptr;
+                    sched.ready[t] = true;
+                }
+            sched.ready[tid] = true;   // the last arriver waits its turn like the others
+            sched_handoff(lk, tid);
+            return;
+        }
+        waiting_on[tid] = this;
+        sched.ready[tid] = false;
+        sched_handoff(lk, tid);
+    }
+    static inline EBar* waiting_on[kMaxThreads];
+};
+inline EBar* block_bar = nullptr;
+inline EBar* warp_bar[kMaxThreads / 32];
 inline const uint8_t* shared_base = nullptr;
 struct WarpXch {
     float f[32];
@@ -45,26 +145,53 @@ struct WarpXch {
     float c[32][4];
 };
 inline WarpXch xch[kMaxThreads / 32];
+inline std::atomic<int> sched_errors{0};   // serial runs that found every thread blocked
 
-inline void warp_sync() { warp_bar[tid3.x >> 5]->arrive_and_wait(); }
+inline void warp_sync() { warp_bar[tid3.x >> 5]->wait(); }
 
 template <typename F>
 void run_grid(int blocks, int threads, const void* shared, F f) {
     shared_base = static_cast<const uint8_t*>(shared);
     grid3 = make_uint3(blocks, 1, 1);
     for (int bx = 0; bx < blocks; ++bx) {
-        std::barrier<> bb(threads);
-        for (int w = 0; w < threads / 32; ++w) warp_bar[w] = new std::barrier<>(32);
+        EBar bb(threads);
+        for (int w = 0; w < threads / 32; ++w) warp_bar[w] = new EBar(32);
         block_bar = &bb;
+        {
+            std::lock_guard<std::mutex> lk(sched.m);
+            sched.n = threads;
+            sched.stuck = false;
+            for (int t = 0; t < threads; ++t) {
+                sched.ready[t] = true;
+                EBar::waiting_on[t] = nullptr;
+            }
+            sched.owner = serial.load() == 2 ? threads - 1 : 0;
+        }
         std::vector<std::thread> th;
         th.reserve(threads);
         for (int t = 0; t < threads; ++t)
             th.emplace_back([&, t, bx] {
                 tid3 = make_uint3(t, 0, 0);
                 bid3 = make_uint3(bx, 0, 0);
-                f();
+                if (serial.load()) {
+                    std::unique_lock<std::mutex> lk(sched.m);
+                    sched.cv[t].wait(lk, [&] { return sched.owner == t || sched.stuck; });
+                }
+                if (!sched.stuck) f();
+                if (serial.load()) {
+                    std::unique_lock<std::mutex> lk(sched.m);
+                    sched.ready[t] = false;
+                    if (sched.owner == t) {
+                        sched.owner = sched_next(t);
+                        bool live = false;
+                        for (int u = 0; u < sched.n; ++u) live = live || EBar::waiting_on[u] != nullptr;
+                        if (sched.owner < 0 && live) sched.stuck = true;
+                        sched_wake();
+                    }
+                }
             });
         for (auto& x : th) x.join();
+        if (sched.stuck) ++sched_errors;
         for (int w = 0; w < threads / 32; ++w) delete warp_bar[w];
     }
 }
@@ -94,7 +221,7 @@ inline uint16_t ld16(uint32_t saddr) {
 #define threadIdx emu::tid3
 #define blockIdx emu::bid3
 #define gridDim emu::grid3
-inline void __syncthreads() { emu::block_bar->arrive_and_wait(); }
+inline void __syncthreads() { emu::block_bar->wait(); }
 inline float __shfl_xor_sync(unsigned, float v, int o) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     emu::xch[w].f[lane] = v;

@@ -396,3 +396,8 @@ extern "C" int emu_mlp_ln_forward_mma(int B, int H, int T, const void* Q, const 
     emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_forward_states_kernel<true>(f); });
     return 0;
 }
+
+// serial scheduling of the next runs (emu_core.h: 0 off, 1 ascending, 2 descending thread order), and the
+// number of runs since the last call in which every live thread was blocked (a hang on the GPU)
+extern "C" void emu_serial(int mode) { emu::serial = mode; }
+extern "C" int emu_sched_errors() { return emu::sched_errors.exchange(0); }

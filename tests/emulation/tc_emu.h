@@ -225,7 +225,7 @@ inline bool wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns, vola
         if (mbar_try_wait(bar, parity)) return true;
         if (abort && *abort) return false;
         if (globaltimer_ns() - t0 > limit_ns) return false;
-        std::this_thread::yield();
+        emu::spin_yield();
     }
 }
 inline void fence_proxy_async_smem() {}

@@ -12,7 +12,7 @@
 //   stmatrix .m8n8.x4.trans .b16: lanes 8i .. 8i+7 give the row addresses of
 //     matrix i; register i of lane L holds fragment elements (L/4, 2(L%4)) and
 //     (L/4, 2(L%4)+1), which land at (2(L%4), L/4) and (2(L%4)+1, L/4).
-//   bar.sync id, n: a barrier over n threads, one per id.
+//   bar.sync id, n: a barrier over n threads, one per id (emu_core.h's EBar).
 //   cp.async.bulk (global -> shared): the bytes count toward the mbarrier.
 //   cp.async.bulk.tensor store, 2-D tile with a 32-, 64- or 128-byte swizzle:
 //     shared byte lin = r * rowbytes + b of the box is read at
@@ -26,7 +26,7 @@
 
 namespace emu {
 inline std::mutex named_mu;
-inline std::barrier<>* named[16];
+inline EBar* named[16];
 inline int named_count[16];
 inline void reset_named() {
     for (int i = 0; i < 16; ++i) {
@@ -63,7 +63,7 @@ inline uint32_t __float_as_uint(float f) {
 namespace ttt {
 inline void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t* r) { emu::tmem_st_32x32b<16>(taddr, r); }
 inline void named_bar_sync(int id, int nthreads) {
-    std::barrier<>* b;
+    emu::EBar* b;
     {
         std::lock_guard<std::mutex> lk(emu::named_mu);
         if (id < 0 || id >= 16 || (emu::named[id] && emu::named_count[id] != nthreads)) {
@@ -71,12 +71,12 @@ inline void named_bar_sync(int id, int nthreads) {
             return;
         }
         if (!emu::named[id]) {
-            emu::named[id] = new std::barrier<>(nthreads);
+            emu::named[id] = new emu::EBar(nthreads);
             emu::named_count[id] = nthreads;
         }
         b = emu::named[id];
     }
-    b->arrive_and_wait();
+    b->wait();
 }
 inline void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     if ((emu::shared_base && ((static_cast<uint8_t*>(dst) - emu::shared_base) % 16)) || bytes % 16 ||
@@ -93,7 +93,7 @@ template <int N>
 inline void bulk_wait_read() {
     static_assert(N == 0, "one store per group");
     emu::flush_stores(threadIdx.x);
-    while (emu::pending_stores[threadIdx.x].load() != 0) std::this_thread::yield();
+    while (emu::pending_stores[threadIdx.x].load() != 0) emu::spin_yield();
 }
 template <int N>
 inline void bulk_wait() {

@@ -81,3 +81,8 @@ extern "C" int emu_linear_tc(int ln, int upc, int B, int H, int T, const void* Q
     for (int t = 0; t < emu::kMaxThreads; ++t) emu::flush_stores(t);
     return emu::errors.load();
 }
+
+// serial scheduling of the next runs (emu_core.h: 0 off, 1 ascending, 2 descending thread order), and the
+// number of runs since the last call in which every live thread was blocked (a hang on the GPU)
+extern "C" void emu_serial(int mode) { emu::serial = mode; }
+extern "C" int emu_sched_errors() { return emu::sched_errors.exchange(0); }

@@ -711,3 +711,42 @@ def test_tcgen05_stall_hook_times_out_and_every_thread_exits(tc_emu, lfr_emu, mt
             mtc_emu.emu_mlp_tc_knobs(0, 120_000_000_000)
     assert rc == 0
     assert status[0] & 1
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("name,args", [
+    ("test_mlp_backward_on_mma_sync", (1, 1, 32, True, True)),
+    ("test_mlp_ln_backward_on_mma_sync", (1, 1, 32, True, True)),
+    ("test_mlp_forward_states_on_mma_sync", (1, 1, 32, True)),
+    ("test_mlp_ln_forward_states_on_mma_sync", (1, 1, 32, True)),
+    ("test_ln_training_on_mma_sync", (1, 1, 32, True, True)),
+    ("test_mlp_forward_states_and_backward", (1, 1, 32, 16, 16, WL.F32, True, True)),
+    ("test_prologue_on_cuda_cores", (2, 20, 40, 3, 16, True, WL.F32)),
+])
+def test_serial_schedules(emu, name, args, mode):
+    """The kernels not yet run on the B200 under the serial scheduler
+    (emu_core.h): one thread at a time, handing on only at a barrier, a warp
+    collective or a spin, the lowest (1) or highest (2) ready thread first, so
+    that one warp runs to its next block-wide barrier before the others move.
+    A missing __syncthreads (a read before the write it needs, or a write into
+    a tile others still read) then gives wrong data deterministically; no run
+    may end with every thread blocked."""
+    emu.emu_serial(mode)
+    try:
+        globals()[name](emu, *args)
+    finally:
+        emu.emu_serial(0)
+    assert emu.emu_sched_errors() == 0
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_serial_schedules_tcgen05_prologue(tc_emu, mode):
+    """The tcgen05 prologue (not yet run on the B200) under the serial
+    scheduler, as above, both with completion at issue and deferred."""
+    for deferred in (False, True):
+        tc_emu.emu_serial(mode)
+        try:
+            test_prologue_on_tcgen05(tc_emu, 2, 40, 136, 5, 64, True, 2, deferred)
+        finally:
+            tc_emu.emu_serial(0)
+        assert tc_emu.emu_sched_errors() == 0
