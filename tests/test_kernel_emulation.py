@@ -721,6 +721,7 @@ def test_tcgen05_stall_hook_times_out_and_every_thread_exits(tc_emu, lfr_emu, mt
     ("test_mlp_ln_forward_states_on_mma_sync", (1, 1, 32, True)),
     ("test_ln_training_on_mma_sync", (1, 1, 32, True, True)),
     ("test_mlp_forward_states_and_backward", (1, 1, 32, 16, 16, WL.F32, True, True)),
+    ("test_mlp_ln_forward_states_and_backward", (1, 1, 32, 16, 16, WL.F32, True, True)),
     ("test_prologue_on_cuda_cores", (2, 20, 40, 3, 16, True, WL.F32)),
 ])
 def test_serial_schedules(emu, name, args, mode):
