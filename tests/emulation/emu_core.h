@@ -149,6 +149,14 @@ inline std::atomic<int> sched_errors{0};   // serial runs that found every threa
 
 inline void warp_sync() { warp_bar[tid3.x >> 5]->wait(); }
 
+// Shared-memory guard: with run_grid_bounded, the buffer beyond the launch's
+// dynamic size is filled with a pattern before each CTA and checked after
+// it; a changed byte counts as an overrun (on the GPU, an access outside the
+// CTA's allocation).
+inline std::atomic<int> smem_overruns{0};
+inline size_t guard_bytes = 0, guard_cap = 0;
+constexpr uint8_t kGuard = 0xA5;
+
 template <typename F>
 void run_grid(int blocks, int threads, const void* shared, F f) {
     shared_base = static_cast<const uint8_t*>(shared);
@@ -167,6 +175,8 @@ void run_grid(int blocks, int threads, const void* shared, F f) {
             }
             sched.owner = serial.load() == 2 ? threads - 1 : 0;
         }
+        uint8_t* guard = const_cast<uint8_t*>(shared_base) + guard_bytes;
+        if (guard_cap > guard_bytes) std::memset(guard, kGuard, guard_cap - guard_bytes);
         std::vector<std::thread> th;
         th.reserve(threads);
         for (int t = 0; t < threads; ++t)
@@ -192,8 +202,26 @@ void run_grid(int blocks, int threads, const void* shared, F f) {
             });
         for (auto& x : th) x.join();
         if (sched.stuck) ++sched_errors;
+        for (size_t i = 0; guard_cap > guard_bytes && i < guard_cap - guard_bytes; ++i)
+            if (guard[i] != kGuard) {
+                ++smem_overruns;
+                break;
+            }
         for (int w = 0; w < threads / 32; ++w) delete warp_bar[w];
     }
+}
+
+// run_grid with the shared-memory guard: `bytes` is the launch's dynamic size, `cap` the buffer's
+template <typename F>
+void run_grid_bounded(int blocks, int threads, void* shared, size_t bytes, size_t cap, F f) {
+    if (bytes > cap) {
+        ++smem_overruns;
+        return;
+    }
+    guard_bytes = bytes;
+    guard_cap = cap;
+    run_grid(blocks, threads, shared, f);
+    guard_bytes = guard_cap = 0;
 }
 
 inline float bf16_lo(uint32_t v) {

@@ -102,9 +102,9 @@ extern "C" int emu_linear_train_mma(int B, int H, int T, const void* Q, const vo
     using namespace ttt::mbk;
     if (kFSmemBytes > (int)sizeof(smem) || kSmemBytes > (int)sizeof(smem)) return 2;
     FwdStatesParams f{H, T, Q, K, V, eta, eta_const, W0, W0_bstride, Z, W_out, W_states};
-    emu::run_grid(B * H, kThreads, smem, [&] { mma_linear_forward_states_kernel(f); });
+    emu::run_grid_bounded(B * H, kThreads, smem, kFSmemBytes, sizeof(smem), [&] { mma_linear_forward_states_kernel(f); });
     ttt::SimtBackwardParams p{H, T, 16, Q, K, V, eta, eta_const, W_states, dZ, dW_out, dQ, dK, dV, deta, dW0};
-    emu::run_grid(B * H, kThreads, smem, [&] { mma_linear_backward_kernel(p); });
+    emu::run_grid_bounded(B * H, kThreads, smem, kSmemBytes, sizeof(smem), [&] { mma_linear_backward_kernel(p); });
     return 0;
 }
 
@@ -118,7 +118,7 @@ extern "C" int emu_ln_forward_mma(int B, int H, int T, const void* Q, const void
     if (kLFSmemBytes > (int)sizeof(smem)) return 2;
     FwdLnStatesParams f{H, T, Q, K, V, eta, eta_const, W0, 0, c0, 0, gamma, beta, eps, Z, W_out, c_out,
                         W_states, c_states};
-    emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_forward_states_kernel(f); });
+    emu::run_grid_bounded(B * H, kThreads, smem, kLFSmemBytes, sizeof(smem), [&] { mma_ln_forward_states_kernel(f); });
     return 0;
 }
 
@@ -134,10 +134,10 @@ extern "C" int emu_ln_train_mma(int B, int H, int T, const void* Q, const void* 
     if (kLFSmemBytes > (int)sizeof(smem) || kLBSmemBytes > (int)sizeof(smem)) return 2;
     FwdLnStatesParams f{H, T, Q, K, V, eta, eta_const, W0, 0, c0, 0, gamma, beta, eps, nullptr, W_out, c_out,
                         W_states, c_states};
-    emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_forward_states_kernel(f); });
+    emu::run_grid_bounded(B * H, kThreads, smem, kLFSmemBytes, sizeof(smem), [&] { mma_ln_forward_states_kernel(f); });
     ttt::SimtLnBackwardParams q{H,  T,  16, Q,  K,      V,      eta,    eta_const, W_states, c_states, gamma, beta,
                                 eps, dZ, dW_out, dc_out, dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta};
-    emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_backward_kernel(q); });
+    emu::run_grid_bounded(B * H, kThreads, smem, kLBSmemBytes, sizeof(smem), [&] { mma_ln_backward_kernel(q); });
     return 0;
 }
 
@@ -206,7 +206,7 @@ extern "C" int emu_ln_backward_mma(int B, int H, int T, const void* Q, const voi
     using namespace ttt::mbk;
     ttt::SimtLnBackwardParams q{H,  T,  16, Q,  K,      V,      eta,    eta_const, W_states, c_states, gamma, beta,
                                 eps, dZ, dW_out, dc_out, dQ, dK, dV, deta, dW0, dc0, dgamma, dbeta};
-    emu::run_grid(B * H, kThreads, smem, [&] { mma_ln_backward_kernel(q); });
+    emu::run_grid_bounded(B * H, kThreads, smem, kLBSmemBytes, sizeof(smem), [&] { mma_ln_backward_kernel(q); });
     return 0;
 }
 
@@ -239,7 +239,7 @@ extern "C" int emu_mlp_backward_mma(int B, int H, int T, const void* Q, const vo
     static_assert(ttt::mmb::kSmemBytes <= (int)sizeof(ttt::mmb::smem), "emulated shared memory");
     ttt::SimtMlpBackwardParams q{H,    T,    16, Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
                                  dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2};
-    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_backward_kernel<false>(q); });
+    emu::run_grid_bounded(B * H, ttt::mmb::kThreads, ttt::mmb::smem, ttt::mmb::kSmemBytes, sizeof(ttt::mmb::smem), [&] { ttt::mmb::mma_mlp_backward_kernel<false>(q); });
     return 0;
 }
 
@@ -250,7 +250,7 @@ extern "C" int emu_mlp_forward_mma(int B, int H, int T, const void* Q, const voi
                                    float* c2_out, float* W_states) {
     ttt::mmb::MlpFwdStatesParams f{H,  T,      Q,      K,      V,      eta,    eta_const, W1,      c1,
                                    W2, c2,     0,      Z,      W1_out, c1_out, W2_out,    c2_out, W_states};
-    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_forward_states_kernel<false>(f); });
+    emu::run_grid_bounded(B * H, ttt::mmb::kThreads, ttt::mmb::smem, ttt::mmb::kSmemBytes, sizeof(ttt::mmb::smem), [&] { ttt::mmb::mma_mlp_forward_states_kernel<false>(f); });
     return 0;
 }
 
@@ -380,7 +380,7 @@ extern "C" int emu_mlp_ln_backward_mma(int B, int H, int T, const void* Q, const
     ttt::SimtMlpBackwardParams q{H,    T,    16, Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
                                  dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2,
                                  gamma, beta, eps, dgamma, dbeta};
-    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_backward_kernel<true>(q); });
+    emu::run_grid_bounded(B * H, ttt::mmb::kThreads, ttt::mmb::smem, ttt::mmb::kSmemBytes, sizeof(ttt::mmb::smem), [&] { ttt::mmb::mma_mlp_backward_kernel<true>(q); });
     return 0;
 }
 
@@ -393,7 +393,7 @@ extern "C" int emu_mlp_ln_forward_mma(int B, int H, int T, const void* Q, const 
     ttt::mmb::MlpFwdStatesParams f{H,  T,      Q,      K,      V,      eta,    eta_const, W1,      c1,
                                    W2, c2,     0,      Z,      W1_out, c1_out, W2_out,    c2_out, W_states,
                                    gamma, beta, eps};
-    emu::run_grid(B * H, ttt::mmb::kThreads, ttt::mmb::smem, [&] { ttt::mmb::mma_mlp_forward_states_kernel<true>(f); });
+    emu::run_grid_bounded(B * H, ttt::mmb::kThreads, ttt::mmb::smem, ttt::mmb::kSmemBytes, sizeof(ttt::mmb::smem), [&] { ttt::mmb::mma_mlp_forward_states_kernel<true>(f); });
     return 0;
 }
 
@@ -401,3 +401,6 @@ extern "C" int emu_mlp_ln_forward_mma(int B, int H, int T, const void* Q, const 
 // number of runs since the last call in which every live thread was blocked (a hang on the GPU)
 extern "C" void emu_serial(int mode) { emu::serial = mode; }
 extern "C" int emu_sched_errors() { return emu::sched_errors.exchange(0); }
+
+// shared-memory overruns (accesses beyond the launch's dynamic size) since the last call
+extern "C" int emu_smem_overruns() { return emu::smem_overruns.exchange(0); }

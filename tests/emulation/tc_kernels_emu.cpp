@@ -53,7 +53,7 @@ extern "C" int emu_prologue_tc(int B, int T, int Dm, int H, int d, const void* x
     const int g = (int)(p.tiles < grid ? p.tiles : grid);
     emu::errors = 0;
     // a persistent CTA walks tiles blockIdx.x, blockIdx.x + gridDim.x, ...: gridDim must be the grid
-    emu::run_grid(g, kThreads, smem, [&] { prologue_kernel(mX, mTq, mTk, mTv, mTl, p); });
+    emu::run_grid_bounded(g, kThreads, smem, kSmemBytes, sizeof(smem), [&] { prologue_kernel(mX, mTq, mTk, mTv, mTl, p); });
     emu::engine.finish();
     for (int t = 0; t < emu::kMaxThreads; ++t) emu::flush_stores(t);
     return emu::errors.load();
@@ -63,3 +63,6 @@ extern "C" int emu_prologue_tc(int B, int T, int Dm, int H, int d, const void* x
 // number of runs since the last call in which every live thread was blocked (a hang on the GPU)
 extern "C" void emu_serial(int mode) { emu::serial = mode; }
 extern "C" int emu_sched_errors() { return emu::sched_errors.exchange(0); }
+
+// shared-memory overruns (accesses beyond the launch's dynamic size) since the last call
+extern "C" int emu_smem_overruns() { return emu::smem_overruns.exchange(0); }

@@ -67,14 +67,14 @@ extern "C" int emu_linear_tc(int ln, int upc, int B, int H, int T, const void* Q
     const int grid = upc == 1 ? (int)U : (int)((U + 1) / 2);
     if (ln) {
         if (upc == 1)
-            emu::run_grid(grid, kThreads, smem, [&] { linear_frag_kernel<true, 1>(mQ, mK, mV, mZ, mZ1, p); });
+            emu::run_grid_bounded(grid, kThreads, smem, kSmemBytes, sizeof(smem), [&] { linear_frag_kernel<true, 1>(mQ, mK, mV, mZ, mZ1, p); });
         else
-            emu::run_grid(grid, kThreads, smem, [&] { linear_frag_kernel<true, 2>(mQ, mK, mV, mZ, mZ1, p); });
+            emu::run_grid_bounded(grid, kThreads, smem, kSmemBytes, sizeof(smem), [&] { linear_frag_kernel<true, 2>(mQ, mK, mV, mZ, mZ1, p); });
     } else {
         if (upc == 1)
-            emu::run_grid(grid, kThreads, smem, [&] { linear_frag_kernel<false, 1>(mQ, mK, mV, mZ, mZ1, p); });
+            emu::run_grid_bounded(grid, kThreads, smem, kSmemBytes, sizeof(smem), [&] { linear_frag_kernel<false, 1>(mQ, mK, mV, mZ, mZ1, p); });
         else
-            emu::run_grid(grid, kThreads, smem, [&] { linear_frag_kernel<false, 2>(mQ, mK, mV, mZ, mZ1, p); });
+            emu::run_grid_bounded(grid, kThreads, smem, kSmemBytes, sizeof(smem), [&] { linear_frag_kernel<false, 2>(mQ, mK, mV, mZ, mZ1, p); });
     }
     emu::reset_named();
     emu::engine.finish();
@@ -86,3 +86,6 @@ extern "C" int emu_linear_tc(int ln, int upc, int B, int H, int T, const void* Q
 // number of runs since the last call in which every live thread was blocked (a hang on the GPU)
 extern "C" void emu_serial(int mode) { emu::serial = mode; }
 extern "C" int emu_sched_errors() { return emu::sched_errors.exchange(0); }
+
+// shared-memory overruns (accesses beyond the launch's dynamic size) since the last call
+extern "C" int emu_smem_overruns() { return emu::smem_overruns.exchange(0); }

@@ -65,9 +65,9 @@ extern "C" int emu_mlp_tc(int ln, int B, int H, int T, int per_seq, const void* 
     emu::errors = 0;
     emu::reset_named();
     if (ln)
-        emu::run_grid((int)U, kThreads, smem, [&] { mlp_tc_kernel<true>(mQ, mK, mV, p); });
+        emu::run_grid_bounded((int)U, kThreads, smem, kSmemBytes, sizeof(smem), [&] { mlp_tc_kernel<true>(mQ, mK, mV, p); });
     else
-        emu::run_grid((int)U, kThreads, smem, [&] { mlp_tc_kernel<false>(mQ, mK, mV, p); });
+        emu::run_grid_bounded((int)U, kThreads, smem, kSmemBytes, sizeof(smem), [&] { mlp_tc_kernel<false>(mQ, mK, mV, p); });
     emu::reset_named();
     emu::engine.finish();
     for (int t = 0; t < emu::kMaxThreads; ++t) emu::flush_stores(t);
@@ -78,3 +78,6 @@ extern "C" int emu_mlp_tc(int ln, int B, int H, int T, int per_seq, const void* 
 // number of runs since the last call in which every live thread was blocked (a hang on the GPU)
 extern "C" void emu_serial(int mode) { emu::serial = mode; }
 extern "C" int emu_sched_errors() { return emu::sched_errors.exchange(0); }
+
+// shared-memory overruns (accesses beyond the launch's dynamic size) since the last call
+extern "C" int emu_smem_overruns() { return emu::smem_overruns.exchange(0); }

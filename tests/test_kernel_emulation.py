@@ -43,6 +43,17 @@ def emu(tmp_path_factory):
     return ctypes.CDLL(so)
 
 
+@pytest.fixture(autouse=True)
+def no_shared_memory_overrun(request):
+    """After each test: no kernel run touched its shared-memory buffer beyond
+    the dynamic size the library launches it with (on the GPU, an access
+    outside the CTA's allocation)."""
+    yield
+    for name in ("emu", "tc_emu", "lfr_emu", "mtc_emu"):
+        if name in request.fixturenames:
+            assert request.getfixturevalue(name).emu_smem_overruns() == 0, name
+
+
 def _p(a):
     return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
 
