@@ -53,10 +53,12 @@ int train(int B, int H, int T, int b, const IO* Q, const IO* K, const IO* V, con
     p.W2_out = W2_out;
     p.c2_out = c2_out;
     p.W_states = W_states;
-    emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { ttt::simt_mlp_kernel<D, IO, false>(p); });
+    emu::run_grid_bounded(B * H, ttt::kSimtThreads, ttt::sm, ttt::simt_mlp_smem(D, b, false), sizeof(ttt::sm),
+                          [&] { ttt::simt_mlp_kernel<D, IO, false>(p); });
     ttt::SimtMlpBackwardParams q{H,  T,  b,  Q,     K,     V,     eta,  eta_const, W_states, dZ,  dW1o,
                                  dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1, dc1, dW2, dc2};
-    emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { ttt::simt_mlp_backward_kernel<D, IO>(q); });
+    emu::run_grid_bounded(B * H, ttt::kSimtThreads, ttt::sm, ttt::simt_mlp_backward_smem(D, b), sizeof(ttt::sm),
+                          [&] { ttt::simt_mlp_backward_kernel<D, IO>(q); });
     return 0;
 }
 
@@ -166,7 +168,10 @@ extern "C" int emu_mlp_forward(int io, int B, int H, int T, int d, int b, const 
     p.c2_out = c2_out;
     p.W_states = W_states;
     if (ttt::simt_mlp_smem(d, b, false) > sizeof(ttt::sm)) return 2;
-    auto run = [&](auto kernel) { emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { kernel(p); }); };
+    auto run = [&](auto kernel) {
+        emu::run_grid_bounded(B * H, ttt::kSimtThreads, ttt::sm, ttt::simt_mlp_smem(d, b, false), sizeof(ttt::sm),
+                              [&] { kernel(p); });
+    };
     if (io == 0) {
         if (d == 16) run(ttt::simt_mlp_kernel<16, float, false>);
         else if (d == 32) run(ttt::simt_mlp_kernel<32, float, false>);
@@ -186,7 +191,10 @@ extern "C" int emu_mlp_backward(int io, int B, int H, int T, int d, int b, const
     ttt::SimtMlpBackwardParams q{H,    T,    b,  Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
                                  dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2};
     if (ttt::simt_mlp_backward_smem(d, b) > sizeof(ttt::sm)) return 2;
-    auto run = [&](auto kernel) { emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { kernel(q); }); };
+    auto run = [&](auto kernel) {
+        emu::run_grid_bounded(B * H, ttt::kSimtThreads, ttt::sm, ttt::simt_mlp_backward_smem(d, b), sizeof(ttt::sm),
+                              [&] { kernel(q); });
+    };
     if (io == 0) {
         if (d == 16) run(ttt::simt_mlp_backward_kernel<16, float>);
         else if (d == 32) run(ttt::simt_mlp_backward_kernel<32, float>);
@@ -219,7 +227,7 @@ extern "C" int emu_prologue_simt(int io, int B, int T, int Dm, int H, int d, con
     ttt::SimtPrologueParams q{rows, T, Dm, H, d, x, tq, tk, tv, tl, eta_base, Q, K, V, eta};
     const long long ncol = 3LL * H * d + (tl ? H : 0);
     const int gx = (rows + ttt::kProTok - 1) / ttt::kProTok, gy = (int)((ncol + ttt::kProCols - 1) / ttt::kProCols);
-    emu::run_grid(gx * gy, ttt::kSimtThreads, ttt::sm, [&] {
+    emu::run_grid_bounded(gx * gy, ttt::kSimtThreads, ttt::sm, ttt::kProSmemBytes, sizeof(ttt::sm), [&] {
         const unsigned flat = emu::bid3.x;
         emu::bid3 = make_uint3(flat % gx, flat / gx, 0);
         if (io == 0)
@@ -292,8 +300,10 @@ extern "C" int emu_mlp_ln_train(int io, int B, int H, int T, int d, int b, const
     if (ttt::simt_mlp_smem(d, b, true) > sizeof(ttt::sm) || ttt::simt_mlp_backward_smem(d, b, true) > sizeof(ttt::sm))
         return 2;
     auto go = [&](auto fwd, auto bwd) {
-        emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { fwd(f); });
-        emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { bwd(q); });
+        emu::run_grid_bounded(B * H, ttt::kSimtThreads, ttt::sm, ttt::simt_mlp_smem(d, b, true), sizeof(ttt::sm),
+                              [&] { fwd(f); });
+        emu::run_grid_bounded(B * H, ttt::kSimtThreads, ttt::sm, ttt::simt_mlp_backward_smem(d, b, true),
+                              sizeof(ttt::sm), [&] { bwd(q); });
     };
     if (io == 0) {
         if (d == 16) go(ttt::simt_mlp_kernel<16, float, true>, ttt::simt_mlp_backward_kernel<16, float, true>);
@@ -336,7 +346,10 @@ extern "C" int emu_mlp_ln_forward(int io, int B, int H, int T, int d, int b, con
     f.beta = beta;
     f.eps = eps;
     f.W_states = W_states;
-    auto run = [&](auto kernel) { emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { kernel(f); }); };
+    auto run = [&](auto kernel) {
+        emu::run_grid_bounded(B * H, ttt::kSimtThreads, ttt::sm, ttt::simt_mlp_smem(d, b, true), sizeof(ttt::sm),
+                              [&] { kernel(f); });
+    };
     if (io == 0) {
         if (d == 16) run(ttt::simt_mlp_kernel<16, float, true>);
         else if (d == 32) run(ttt::simt_mlp_kernel<32, float, true>);
@@ -357,7 +370,10 @@ extern "C" int emu_mlp_ln_backward(int io, int B, int H, int T, int d, int b, co
     ttt::SimtMlpBackwardParams q{H,    T,    b,  Q,  K,  V,    eta, eta_const, W_states, dZ,  dW1o,
                                  dc1o, dW2o, dc2o, dQ, dK, dV, deta, dW1,      dc1,      dW2, dc2,
                                  gamma, beta, eps, dgamma, dbeta};
-    auto run = [&](auto kernel) { emu::run_grid(B * H, ttt::kSimtThreads, ttt::sm, [&] { kernel(q); }); };
+    auto run = [&](auto kernel) {
+        emu::run_grid_bounded(B * H, ttt::kSimtThreads, ttt::sm, ttt::simt_mlp_backward_smem(d, b, true),
+                              sizeof(ttt::sm), [&] { kernel(q); });
+    };
     if (io == 0) {
         if (d == 16) run(ttt::simt_mlp_backward_kernel<16, float, true>);
         else if (d == 32) run(ttt::simt_mlp_backward_kernel<32, float, true>);
