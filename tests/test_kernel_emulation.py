@@ -43,6 +43,44 @@ def emu(tmp_path_factory):
     return ctypes.CDLL(so)
 
 
+# Arrays handed to the kernels come with 4 KB guard bands on both sides, filled
+# with a pattern; every test checks afterwards that no kernel wrote into them
+# (on the GPU, a write outside the caller's buffer).
+_GUARD_BYTES = 4096
+_guards = []
+
+
+def _guarded(shape, dtype, fill):
+    dtype = np.dtype(dtype)
+    n = int(np.prod(shape))
+    pad = _GUARD_BYTES // dtype.itemsize
+    raw = np.empty(n + 2 * pad, dtype)
+    raw.view(np.uint8)[:] = 0xA5
+    raw[pad:pad + n] = fill
+    _guards.append((raw, pad, n))
+    return raw[pad:pad + n].reshape(shape)
+
+
+def gzeros(shape, dtype=np.float64):
+    return _guarded(shape, dtype, 0)
+
+
+def gfull(shape, value, dtype):
+    return _guarded(shape, dtype, value)
+
+
+@pytest.fixture(autouse=True)
+def no_out_of_bounds_write():
+    """After each test: every guard band is intact."""
+    _guards.clear()
+    yield
+    for raw, pad, n in _guards:
+        b = raw.view(np.uint8)
+        k = pad * raw.itemsize
+        assert np.all(b[:k] == 0xA5) and np.all(b[k + n * raw.itemsize:] == 0xA5), "write outside the buffer"
+    _guards.clear()
+
+
 @pytest.fixture(autouse=True)
 def no_shared_memory_overrun(request):
     """After each test: no kernel run touched its shared-memory buffer beyond
@@ -97,12 +135,12 @@ def test_mlp_forward_states_and_backward(emu, B, H, T, d, b, io, per_token, upst
            if upstream else [None] * 4)
     nb = T // b
     iot = np.uint16 if io == WL.BF16 else np.float32
-    Z = np.zeros((B, H, T, d), iot)
-    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
-    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
-    dQ, dK, dV = (np.zeros((B, H, T, d), iot) for _ in range(3))
-    deta = np.zeros((B, H, T), np.float32)
-    grads = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    Z = gzeros((B, H, T, d), iot)
+    outs = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = gzeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    dQ, dK, dV = (gzeros((B, H, T, d), iot) for _ in range(3))
+    deta = gzeros((B, H, T), np.float32)
+    grads = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
     emu.emu_mlp_train.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + \
         [ctypes.c_void_p] * 23
     rc = emu.emu_mlp_train(1 if io == WL.BF16 else 0, B, H, T, d, b, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]),
@@ -151,12 +189,12 @@ def test_linear_training_on_mma_sync(emu, B, H, T, per_token, upstream):
     dZr, dZe = WL.store(rng.standard_normal((B, H, T, d)), WL.BF16)
     dW = rng.standard_normal((B, H, d, d)).astype(np.float32) if upstream else None
     nb = T // b
-    Z = np.zeros((B, H, T, d), np.uint16)
-    W_out = np.zeros((B, H, d, d), np.float32)
-    states = np.zeros((B, H, nb, d, d), np.float32)
-    dQ, dK, dV = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
-    deta = np.zeros((B, H, T), np.float32)
-    dW0 = np.zeros((B, H, d, d), np.float32)
+    Z = gzeros((B, H, T, d), np.uint16)
+    W_out = gzeros((B, H, d, d), np.float32)
+    states = gzeros((B, H, nb, d, d), np.float32)
+    dQ, dK, dV = (gzeros((B, H, T, d), np.uint16) for _ in range(3))
+    deta = gzeros((B, H, T), np.float32)
+    dW0 = gzeros((B, H, d, d), np.float32)
     eta = raw["eta"] if per_token else None
     f = emu.emu_linear_train_mma
     f.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_longlong] + \
@@ -196,12 +234,12 @@ def test_ln_training_on_mma_sync(emu, B, H, T, per_token, upstream):
     dWo = rng.standard_normal((B, H, d, d)).astype(np.float32) if upstream else None
     dco = rng.standard_normal((B, H, d)).astype(np.float32) if upstream else None
     nb = T // b
-    W_out, c_out = np.zeros((B, H, d, d), np.float32), np.zeros((B, H, d), np.float32)
-    Ws, cs = np.zeros((B, H, nb, d, d), np.float32), np.zeros((B, H, nb, d), np.float32)
-    dQ, dK, dV = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
-    deta = np.zeros((B, H, T), np.float32)
-    dW0 = np.zeros((B, H, d, d), np.float32)
-    dc0, dgam, dbet = (np.zeros((B, H, d), np.float32) for _ in range(3))
+    W_out, c_out = gzeros((B, H, d, d), np.float32), gzeros((B, H, d), np.float32)
+    Ws, cs = gzeros((B, H, nb, d, d), np.float32), gzeros((B, H, nb, d), np.float32)
+    dQ, dK, dV = (gzeros((B, H, T, d), np.uint16) for _ in range(3))
+    deta = gzeros((B, H, T), np.float32)
+    dW0 = gzeros((B, H, d, d), np.float32)
+    dc0, dgam, dbet = (gzeros((B, H, d), np.float32) for _ in range(3))
     f = emu.emu_ln_train_mma
     f.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 4 + \
         [ctypes.c_float] + [ctypes.c_void_p] * 15
@@ -246,8 +284,8 @@ def test_prologue_on_cuda_cores(emu, B, T, Dm, H, d, gate, io):
         iot = np.float32
     else:
         raw, iot = inp["raw"], np.uint16
-    Q, K, V = (np.zeros((B, H, T, d), iot) for _ in range(3))
-    eta = np.zeros((B, H, T), np.float32) if gate else None
+    Q, K, V = (gzeros((B, H, T, d), iot) for _ in range(3))
+    eta = gzeros((B, H, T), np.float32) if gate else None
     f = emu.emu_prologue_simt
     f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 4
     assert f(0 if io == WL.F32 else 1, B, T, Dm, H, d, _p(raw["x"]), _p(raw["theta_q"]), _p(raw["theta_k"]),
@@ -278,17 +316,17 @@ def test_mlp_backward_on_mma_sync(emu, B, H, T, per_token, upstream):
     ups = ([rng.standard_normal(s).astype(np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
            if upstream else [None] * 4)
     nb = T // b
-    Z = np.zeros((B, H, T, d), np.uint16)
-    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
-    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    Z = gzeros((B, H, T, d), np.uint16)
+    outs = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = gzeros((B, H, nb, 2 * d * m + m + d), np.float32)
     eta = raw["eta"] if per_token else None
     f = emu.emu_mlp_forward
     f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 10
     assert f(1, B, H, T, d, b, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const),
              _p(raw["W1"]), _p(c1), _p(raw["W2"]), _p(c2), _p(Z), *[_p(o) for o in outs], _p(states)) == 0
-    dQ, dK, dV = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
-    deta = np.zeros((B, H, T), np.float32)
-    grads = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    dQ, dK, dV = (gzeros((B, H, T, d), np.uint16) for _ in range(3))
+    deta = gzeros((B, H, T), np.float32)
+    grads = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
     g = emu.emu_mlp_backward_mma
     g.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 14
     assert g(B, H, T, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(inp.w.eta_const), _p(states),
@@ -318,9 +356,9 @@ def test_mlp_forward_states_on_mma_sync(emu, B, H, T, per_token):
     c1 = (rng.standard_normal((H, m)) * 0.1).astype(np.float32)
     c2 = (rng.standard_normal((H, d)) * 0.1).astype(np.float32)
     nb = T // b
-    Z = np.zeros((B, H, T, d), np.uint16)
-    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
-    states = np.zeros((B, H, max(nb, 1), 2 * d * m + m + d), np.float32)
+    Z = gzeros((B, H, T, d), np.uint16)
+    outs = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = gzeros((B, H, max(nb, 1), 2 * d * m + m + d), np.float32)
     eta = raw["eta"] if per_token else None
     f = emu.emu_mlp_forward_mma
     f.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 10
@@ -366,9 +404,9 @@ def test_prologue_on_tcgen05(tc_emu, B, T, Dm, H, d, gate, grid, deferred):
     waited for): a missing or misplaced wait then shows as wrong data."""
     w, inp = WL.prologue_case(B, T, Dm, H, d, gate=gate, eta_base=0.5)
     r, e = inp["raw"], inp["exact"]
-    Q, K, V = (np.full((B, H, T, d), 0x7FC0, np.uint16) for _ in range(3))   # NaN until written
-    eta = np.full((B, H, T), np.nan, np.float32) if gate else None
-    status = np.zeros(1, np.int32)
+    Q, K, V = (gfull((B, H, T, d), 0x7FC0, np.uint16) for _ in range(3))   # NaN until written
+    eta = gfull((B, H, T), np.nan, np.float32) if gate else None
+    status = gzeros(1, np.int32)
     f = tc_emu.emu_prologue_tc
     f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 5 + [ctypes.c_float] + [ctypes.c_void_p] * 4 + \
         [ctypes.c_int, ctypes.c_void_p]
@@ -414,10 +452,10 @@ def test_mlp_ln_forward_states_and_backward(emu, B, H, T, d, b, io, per_token, u
            if upstream else [None] * 4)
     nb = T // b
     iot = np.uint16 if io == WL.BF16 else np.float32
-    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
-    dQ, dK, dV = (np.zeros((B, H, T, d), iot) for _ in range(3))
-    deta = np.zeros((B, H, T), np.float32)
-    g = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d), (B, H, d), (B, H, d))]
+    states = gzeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    dQ, dK, dV = (gzeros((B, H, T, d), iot) for _ in range(3))
+    deta = gzeros((B, H, T), np.float32)
+    g = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d), (B, H, d), (B, H, d))]
     eta = raw["eta"] if per_token else None
     f = emu.emu_mlp_ln_train
     f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
@@ -459,9 +497,9 @@ def test_mlp_ln_backward_on_mma_sync(emu, B, H, T, per_token, upstream):
     ups = ([rng.standard_normal(s).astype(np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
            if upstream else [None] * 4)
     nb = T // b
-    Z = np.zeros((B, H, T, d), np.uint16)
-    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
-    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    Z = gzeros((B, H, T, d), np.uint16)
+    outs = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = gzeros((B, H, nb, 2 * d * m + m + d), np.float32)
     eta = raw["eta"] if per_token else None
     f = emu.emu_mlp_ln_forward
     f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
@@ -469,9 +507,9 @@ def test_mlp_ln_backward_on_mma_sync(emu, B, H, T, per_token, upstream):
     assert f(1, B, H, T, d, b, _p(raw["Q"]), _p(raw["K"]), _p(raw["V"]), _p(eta), np.float32(0.02), _p(raw["W1"]),
              _p(c1), _p(raw["W2"]), _p(c2), _p(gam), _p(bet), np.float32(1e-6), _p(Z), *[_p(o) for o in outs],
              _p(states)) == 0
-    dQ, dK, dV = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
-    deta = np.zeros((B, H, T), np.float32)
-    g = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d), (B, H, d), (B, H, d))]
+    dQ, dK, dV = (gzeros((B, H, T, d), np.uint16) for _ in range(3))
+    deta = gzeros((B, H, T), np.float32)
+    g = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d), (B, H, d), (B, H, d))]
     bw = emu.emu_mlp_ln_backward_mma
     bw.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 8 + \
         [ctypes.c_float] + [ctypes.c_void_p] * 10
@@ -507,9 +545,9 @@ def test_mlp_ln_forward_states_on_mma_sync(emu, B, H, T, per_token):
     gam = (1 + rng.standard_normal((H, d)) * 0.2).astype(np.float32)
     bet = (rng.standard_normal((H, d)) * 0.2).astype(np.float32)
     nb = T // b
-    Z = np.zeros((B, H, T, d), np.uint16)
-    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
-    states = np.zeros((B, H, nb, 2 * d * m + m + d), np.float32)
+    Z = gzeros((B, H, T, d), np.uint16)
+    outs = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    states = gzeros((B, H, nb, 2 * d * m + m + d), np.float32)
     eta = raw["eta"] if per_token else None
     f = emu.emu_mlp_ln_forward_mma
     f.argtypes = [ctypes.c_int] * 3 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
@@ -562,10 +600,10 @@ def test_linear_prefill_on_tcgen05(lfr_emu, ln, upc, B, H, T, per_token, deferre
     raw, ex = inp.raw, inp.exact
     rng = np.random.default_rng(2 + T)
     c0 = (rng.standard_normal((H, d)) * 0.1).astype(np.float32) if ln else None
-    Z = np.zeros((B, H, T, d), np.uint16)
-    W_out = np.zeros((B, H, d, d), np.float32)
-    c_out = np.zeros((B, H, d), np.float32) if ln else None
-    status = np.zeros(1, np.int32)
+    Z = gzeros((B, H, T, d), np.uint16)
+    W_out = gzeros((B, H, d, d), np.float32)
+    c_out = gzeros((B, H, d), np.float32) if ln else None
+    status = gzeros(1, np.int32)
     eta = raw["eta"] if per_token else None
     f = lfr_emu.emu_linear_tc
     f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + [ctypes.c_float, ctypes.c_void_p, ctypes.c_longlong,
@@ -626,13 +664,13 @@ def test_mlp_prefill_on_tcgen05(mtc_emu, ln, B, H, T, per_token, biases, per_seq
         W2 = (raw["W2"][None] + 0.01 * rng.standard_normal((B,) + raw["W2"].shape)).astype(np.float32)
     else:
         W1, W2 = raw["W1"], raw["W2"]
-    c1 = (rng.standard_normal(lead + (m,)) * 0.1).astype(np.float32) if biases else np.zeros(lead + (m,), np.float32)
-    c2 = (rng.standard_normal(lead + (d,)) * 0.1).astype(np.float32) if biases else np.zeros(lead + (d,), np.float32)
+    c1 = (rng.standard_normal(lead + (m,)) * 0.1).astype(np.float32) if biases else gzeros(lead + (m,), np.float32)
+    c2 = (rng.standard_normal(lead + (d,)) * 0.1).astype(np.float32) if biases else gzeros(lead + (d,), np.float32)
     gam = (1 + 0.1 * rng.standard_normal((H, d))).astype(np.float32)
     bet = (0.1 * rng.standard_normal((H, d))).astype(np.float32)
-    Z = np.zeros((B, H, T, d), np.uint16)
-    outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
-    status = np.zeros(1, np.int32)
+    Z = gzeros((B, H, T, d), np.uint16)
+    outs = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+    status = gzeros(1, np.int32)
     eta = raw["eta"] if per_token else None
     f = mtc_emu.emu_mlp_tc
     f.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p] * 4 + [ctypes.c_float] + [ctypes.c_void_p] * 6 + \
@@ -666,13 +704,13 @@ def test_tcgen05_stall_hook_times_out_and_every_thread_exits(tc_emu, lfr_emu, mt
     (a wait that never ended would hang this test).  The same path runs on the
     B200 in the tests marked gpu."""
     stall, limit = 0x100, 20_000_000
-    status = np.zeros(1, np.int32)
+    status = gzeros(1, np.int32)
     if kind == "prologue":
         B, T, Dm, H, d = 2, 200, 136, 5, 64
         w, inp = WL.prologue_case(B, T, Dm, H, d, gate=True, eta_base=0.5)
         r = inp["raw"]
-        Q, K, V = (np.zeros((B, H, T, d), np.uint16) for _ in range(3))
-        eta = np.zeros((B, H, T), np.float32)
+        Q, K, V = (gzeros((B, H, T, d), np.uint16) for _ in range(3))
+        eta = gzeros((B, H, T), np.float32)
         tc_emu.emu_prologue_tc_knobs.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
         tc_emu.emu_prologue_tc_knobs(stall, limit)
         f = tc_emu.emu_prologue_tc
@@ -687,8 +725,8 @@ def test_tcgen05_stall_hook_times_out_and_every_thread_exits(tc_emu, lfr_emu, mt
         B, H, T, d = 1, 3, 64, 64
         inp = WL.random_case("linear", B, H, T, d, 16, io_dtype=WL.BF16, eta_mode="sigmoid", seed=9)
         raw = inp.raw
-        Z = np.zeros((B, H, T, d), np.uint16)
-        W_out = np.zeros((B, H, d, d), np.float32)
+        Z = gzeros((B, H, T, d), np.uint16)
+        W_out = gzeros((B, H, d, d), np.float32)
         lfr_emu.emu_linear_tc_knobs.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
         lfr_emu.emu_linear_tc_knobs(stall, limit)
         f = lfr_emu.emu_linear_tc
@@ -705,9 +743,9 @@ def test_tcgen05_stall_hook_times_out_and_every_thread_exits(tc_emu, lfr_emu, mt
         B, H, T, d, m = 1, 2, 48, 64, 256
         inp = WL.random_case("mlp", B, H, T, d, 16, io_dtype=WL.BF16, eta_mode="sigmoid", seed=9)
         raw = inp.raw
-        gam, bet = np.ones((H, d), np.float32), np.zeros((H, d), np.float32)
-        Z = np.zeros((B, H, T, d), np.uint16)
-        outs = [np.zeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
+        gam, bet = np.ones((H, d), np.float32), gzeros((H, d), np.float32)
+        Z = gzeros((B, H, T, d), np.uint16)
+        outs = [gzeros(s, np.float32) for s in ((B, H, d, m), (B, H, m), (B, H, m, d), (B, H, d))]
         mtc_emu.emu_mlp_tc_knobs.argtypes = [ctypes.c_uint, ctypes.c_ulonglong]
         mtc_emu.emu_mlp_tc_knobs(stall, limit)
         f = mtc_emu.emu_mlp_tc
