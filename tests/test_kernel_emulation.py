@@ -7,7 +7,11 @@ tcgen05.mma, with asynchronous operations completing at issue), against the
 float64 oracle.
 
 This checks the source's index arithmetic, phase order and barrier placement
-where no GPU is present.  It is not the GPU parity: the tests marked gpu run
+where no GPU is present.  Beyond parity: a deferred-completion mode (late
+asynchronous copies, MMAs and TMEM accesses) and a serial scheduler (one
+thread at a time, in index order) turn a missing wait or barrier into wrong
+data; guards around every shared buffer and every array catch accesses
+outside them; the stall hook checks that every wait ends.  It is not the GPU parity: the tests marked gpu run
 the same kernels on the B200 through the C ABI, and the library itself has no
 CPU path.
 
