@@ -46,7 +46,8 @@ inline uint3 grid3;
 // an mbarrier or a store).  At a block the next thread is the ready one of
 // lowest (1) or highest (2) index, so the first warp runs as far as it can,
 // to its next block-wide barrier, before the others move; a spinning thread
-// hands on round-robin.  A read of data another thread writes without a
+// hands on round-robin and runs again only when no thread that is not
+// spinning is ready.  A read of data another thread writes without a
 // barrier between them, or a write into data others still read, then shows
 // as wrong data in one of the two orders.
 inline std::atomic<int> serial{0};
@@ -55,18 +56,10 @@ struct Sched {
     std::condition_variable cv[kMaxThreads];   // one per thread: a hand-off wakes only the new owner
     int n = 0, owner = -1;
     bool ready[kMaxThreads];
+    bool spinning[kMaxThreads];   // last handed on from a spin-wait: runs only when no other thread is ready
     bool stuck = false;   // every live thread blocked on a barrier: the kernel would hang
 };
 inline Sched sched;
-// the ready thread of lowest (1) or highest (2) index, or -1 (lock held)
-inline int sched_next(int) {
-    const int n = sched.n;
-    for (int i = 0; i < n; ++i) {
-        const int t = serial.load() == 1 ? i : n - 1 - i;
-        if (sched.ready[t]) return t;
-    }
-    return -1;
-}
 // the next ready thread after `from`, round-robin (itself last), or -1 (lock held)
 inline int sched_next_rr(int from) {
     const int n = sched.n;
@@ -75,6 +68,16 @@ inline int sched_next_rr(int from) {
         if (sched.ready[t]) return t;
     }
     return -1;
+}
+// the ready thread of lowest (1) or highest (2) index that is not spinning, else the next spinner
+// round-robin, or -1 (lock held)
+inline int sched_next(int from) {
+    const int n = sched.n;
+    for (int i = 0; i < n; ++i) {
+        const int t = serial.load() == 1 ? i : n - 1 - i;
+        if (sched.ready[t] && !sched.spinning[t]) return t;
+    }
+    return sched_next_rr(from);
 }
 // hand the CPU on (lock held) and wait until it comes back
 inline void sched_wake() {
@@ -100,6 +103,7 @@ inline void spin_yield() {
     const int tid = (int)tid3.x;
     std::unique_lock<std::mutex> lk(sched.m);
     sched.ready[tid] = true;
+    sched.spinning[tid] = true;
     sched_handoff(lk, tid, true);
 }
 
@@ -117,6 +121,7 @@ struct EBar {
         }
         const int tid = (int)tid3.x;
         std::unique_lock<std::mutex> lk(sched.m);
+        sched.spinning[tid] = false;
         if (++arrived == count) {
             arrived = 0;
             ++gen;
@@ -171,6 +176,7 @@ void run_grid(int blocks, int threads, const void* shared, F f) {
             sched.stuck = false;
             for (int t = 0; t < threads; ++t) {
                 sched.ready[t] = true;
+                sched.spinning[t] = false;
                 EBar::waiting_on[t] = nullptr;
             }
             sched.owner = serial.load() == 2 ? threads - 1 : 0;

@@ -804,3 +804,19 @@ def test_serial_schedules_tcgen05_prologue(tc_emu, mode):
         finally:
             tc_emu.emu_serial(0)
         assert tc_emu.emu_sched_errors() == 0
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+def test_serial_schedules_tcgen05_verified(lfr_emu, mtc_emu, mode):
+    """The two B200-verified tensor-core prefills under the serial scheduler
+    with deferred completion: a check of the checker (no false alarm on
+    kernels known to be right)."""
+    for lib, run in ((lfr_emu, lambda: test_linear_prefill_on_tcgen05(lfr_emu, True, 2, 1, 2, 32, True, True)),
+                     (mtc_emu, lambda: test_mlp_prefill_on_tcgen05(mtc_emu, False, 1, 1, 32, True, True, False,
+                                                                   True))):
+        lib.emu_serial(mode)
+        try:
+            run()
+        finally:
+            lib.emu_serial(0)
+        assert lib.emu_sched_errors() == 0
