@@ -269,7 +269,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (long long tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++ai) {
             const Tile tl = decode_tile(p, tile);
             const int a = ai & 1;
-            if (!wait_bounded(&acc_full[a], (uint32_t)(ai >> 1) & 1u, lim, s_abort)) {
+            // the warp leaves together: a lane that saw the wait expire takes the others with it, so the
+            // warp-wide tcgen05.ld below never runs with part of the warp
+            const bool got = wait_bounded(&acc_full[a], (uint32_t)(ai >> 1) & 1u, lim, s_abort);
+            if (__any_sync(0xffffffffu, !got)) {
                 if (lane == 0) fail();
                 break;
             }

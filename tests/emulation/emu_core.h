@@ -272,6 +272,15 @@ inline float __shfl_sync(unsigned, float v, int src) {
     emu::warp_sync();
     return r;
 }
+inline int __any_sync(unsigned, int pred) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    emu::xch[w].f[lane] = pred ? 1.f : 0.f;
+    emu::warp_sync();
+    int any = 0;
+    for (int i = 0; i < 32; ++i) any |= emu::xch[w].f[i] != 0.f;
+    emu::warp_sync();
+    return any;
+}
 inline float rsqrtf(float x) { return 1.0f / std::sqrt(x); }
 inline int min(int a, int b) { return a < b ? a : b; }
 inline int max(int a, int b) { return a > b ? a : b; }
